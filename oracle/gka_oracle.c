@@ -1,0 +1,303 @@
+/*
+ * Gated KalmaNet (GKA) layer: plain float64 CPU oracle.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or
+ * load this file: only the tests, the package smoke check and the benchmark's
+ * CPU-baseline leg use it.  It shares no code, header, table or helper with
+ * the CUDA library; the two are independent restatements of the same method.
+ *
+ * Source: "Gated KalmaNet: A Fading Memory Layer Through Test-Time Ridge
+ * Regression" (arXiv 2511.21016), as summarised on the ai.info page
+ * (Key Contributions 2-3, Main Findings, Methodology in Plain English) and
+ * the appendix fragments on the pith.science page (Lemma 3 / Lemma 4 on the
+ * Chebyshev weight schedule, and the rate table for kappa = 51).
+ *
+ * What it computes, per (batch, head), token by token (no chunking, no
+ * blocking, no fusion):
+ *   H_t = beta_t H_{t-1} + k_t k_t^T          (gated fading Gram state)
+ *   M_t = beta_t M_{t-1} + v_t k_t^T          (value state; the pages' U_t)
+ *   n_t = ||H_t||_F,  lambda_t = a n_t        (adaptive ridge)
+ *   x_t = r-step Chebyshev iterate for (H_t + lambda_t I) x = q_t on the
+ *         spectral interval [a n_t, (1+a) n_t], started at x = 0
+ *   o_t = M_t x_t
+ * The decay beta_t multiplies the old state (the pages' gate gamma_t of the
+ * weighted ridge objective, Eq. 3, with eta_{t,i} = prod_{j=i+1..t} gamma_j).
+ *
+ * All arithmetic is float64.  Matrices are dense row-major.
+ */
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/*
+ * Chebyshev weight schedule (pith.science appendix, Lemma 3 "weight
+ * schedule"): omega_0 = 2 and omega_i = 1 / (1 - rho^2 omega_{i-1} / 4),
+ * where rho = (L - mu) / (L + mu).  omega_i is used by the i-th update that
+ * follows the first step x_1 = q / d.  Fills omega[0..n-1].
+ */
+void gka_oracle_omegas(double rho, int n, double *omega)
+{
+    if (n <= 0) return;
+    omega[0] = 2.0;
+    for (int i = 1; i < n; ++i)
+        omega[i] = 1.0 / (1.0 - rho * rho * omega[i - 1] / 4.0);
+}
+
+/*
+ * r-step Chebyshev iteration for A x = q, where A (D x D, symmetric) has its
+ * spectrum in [mu, L] (ai.info, Key Contributions 2 and Methodology: the
+ * iteration needs only matrix-vector products).  Three-term form with
+ * d = (L + mu)/2:
+ *   x_0 = 0,  x_1 = q / d,
+ *   x_{i+1} = x_{i-1} + omega_i * ( (q - A x_i) / d + x_i - x_{i-1} ),
+ *   i = 1 .. r-1,  result x_r  (r - 1 matrix-vector products).
+ * r must be >= 1.  work must hold 3*D doubles.
+ */
+void gka_oracle_cheb_solve(const double *A, const double *q, int D,
+                           double mu, double L, int r, double *x, double *work)
+{
+    double d = 0.5 * (L + mu);
+    double rho = (L - mu) / (L + mu);
+    double *xprev = work, *xnew = work + D, *y = work + 2 * D;
+    double *omega = (double *)malloc(sizeof(double) * (size_t)(r > 1 ? r : 1));
+    gka_oracle_omegas(rho, r, omega);
+
+    for (int i = 0; i < D; ++i) {
+        xprev[i] = 0.0;
+        x[i] = q[i] / d;
+    }
+    for (int it = 1; it < r; ++it) {
+        for (int i = 0; i < D; ++i) {
+            double s = 0.0;
+            for (int j = 0; j < D; ++j) s += A[(size_t)i * D + j] * x[j];
+            y[i] = s;
+        }
+        double w = omega[it];
+        for (int i = 0; i < D; ++i)
+            xnew[i] = xprev[i] + w * ((q[i] - y[i]) / d + x[i] - xprev[i]);
+        for (int i = 0; i < D; ++i) {
+            xprev[i] = x[i];
+            x[i] = xnew[i];
+        }
+    }
+    free(omega);
+}
+
+/*
+ * One token of the recurrence on one head, in place on (H, M).
+ * Writes the token's output o (D) and returns n_t = ||H_t||_F.
+ * If solve == 0 only the state update and the norm are done.
+ * work: D*D + 4*D doubles.
+ */
+static double gka_token(double *H, double *M, const double *q, const double *k,
+                        const double *v, double beta, int D, double a, int r,
+                        int solve, double *o, double *work)
+{
+    /* state update (ai.info, Methodology: running weighted covariances
+     * with a decay factor) */
+    for (int i = 0; i < D; ++i)
+        for (int j = 0; j < D; ++j) {
+            H[(size_t)i * D + j] = beta * H[(size_t)i * D + j] + k[i] * k[j];
+            M[(size_t)i * D + j] = beta * M[(size_t)i * D + j] + v[i] * k[j];
+        }
+    /* Frobenius norm and adaptive ridge (ai.info, Key Contributions 2) */
+    double n2 = 0.0;
+    for (size_t e = 0; e < (size_t)D * D; ++e) n2 += H[e] * H[e];
+    double n = sqrt(n2);
+    if (!solve) return n;
+
+    double *A = work, *x = work + (size_t)D * D, *cw = x + D;
+    if (n == 0.0) {
+        /* zero state: the regularised system degenerates; the output is 0 */
+        for (int i = 0; i < D; ++i) o[i] = 0.0;
+        return n;
+    }
+    double lam = a * n;
+    memcpy(A, H, sizeof(double) * (size_t)D * D);
+    for (int i = 0; i < D; ++i) A[(size_t)i * D + i] += lam;
+    gka_oracle_cheb_solve(A, q, D, lam, (1.0 + a) * n, r, x, cw);
+    /* readout o_t = M_t x_t (ai.info, Methodology: "then multiplying by U_t") */
+    for (int i = 0; i < D; ++i) {
+        double s = 0.0;
+        for (int j = 0; j < D; ++j) s += M[(size_t)i * D + j] * x[j];
+        o[i] = s;
+    }
+    return n;
+}
+
+/*
+ * Token-by-token forward over [B, Hh, T, D] inputs (row-major, D fastest).
+ *   init_state  nullable, [B, Hh, 2, D, D]: H then M at t = -1 (zero if NULL)
+ *   solve_from  tokens t < solve_from only advance the state (o not written)
+ *   o           [B, Hh, T, D]
+ *   norms       nullable, [B, Hh, T]: ||H_t||_F
+ *   final_state nullable, [B, Hh, 2, D, D]
+ *   chunk, chunk_states  nullable pair: when chunk > 0 and chunk_states is
+ *               given, the state in force before token n*chunk is stored at
+ *               chunk_states[B, Hh, T/chunk, 2, D, D]
+ *   nthreads    OpenMP threads over (b, h); <= 0 means the runtime default
+ * Returns 0, or -1 on bad arguments.
+ */
+int gka_oracle_forward(const double *q, const double *k, const double *v,
+                       const double *beta, int B, int Hh, int T, int D,
+                       double a, int r, const double *init_state,
+                       int solve_from, double *o, double *norms,
+                       double *final_state, int chunk, double *chunk_states,
+                       int nthreads)
+{
+    if (B < 0 || Hh < 0 || T < 0 || D <= 0 || r < 1 || !(a > 0.0)) return -1;
+    long nh = (long)B * Hh;
+    size_t DD = (size_t)D * D;
+    int nchunks = (chunk > 0) ? T / chunk : 0;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (long h = 0; h < nh; ++h) {
+        double *H = (double *)calloc(2 * DD, sizeof(double));
+        double *M = H + DD;
+        double *work = (double *)malloc(sizeof(double) * (DD + 4 * (size_t)D));
+        if (init_state) memcpy(H, init_state + (size_t)h * 2 * DD, sizeof(double) * 2 * DD);
+        for (int t = 0; t < T; ++t) {
+            if (chunk_states && chunk > 0 && t % chunk == 0 && t / chunk < nchunks)
+                memcpy(chunk_states + ((size_t)h * nchunks + t / chunk) * 2 * DD, H,
+                       sizeof(double) * 2 * DD);
+            size_t row = ((size_t)h * T + t) * D;
+            double n = gka_token(H, M, q + row, k + row, v + row, beta[(size_t)h * T + t],
+                                 D, a, r, t >= solve_from, o + row, work);
+            if (norms) norms[(size_t)h * T + t] = n;
+        }
+        if (final_state) memcpy(final_state + (size_t)h * 2 * DD, H, sizeof(double) * 2 * DD);
+        free(work);
+        free(H);
+    }
+    return 0;
+}
+
+/*
+ * One recurrent decode step for [B, Hh] heads: the same token update as the
+ * forward, applied in place to state [B, Hh, 2, D, D] (H then M).
+ * q, k, v, o: [B, Hh, D];  beta: [B, Hh].
+ */
+int gka_oracle_decode_step(double *state, const double *q, const double *k,
+                           const double *v, const double *beta, int B, int Hh,
+                           int D, double a, int r, double *o, int nthreads)
+{
+    if (B < 0 || Hh < 0 || D <= 0 || r < 1 || !(a > 0.0)) return -1;
+    long nh = (long)B * Hh;
+    size_t DD = (size_t)D * D;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (long h = 0; h < nh; ++h) {
+        double *work = (double *)malloc(sizeof(double) * (DD + 4 * (size_t)D));
+        double *H = state + (size_t)h * 2 * DD;
+        gka_token(H, H + DD, q + (size_t)h * D, k + (size_t)h * D, v + (size_t)h * D,
+                  beta[h], D, a, r, 1, o + (size_t)h * D, work);
+        free(work);
+    }
+    return 0;
+}
+
+/*
+ * Chunk-wise ||H_t||_F (ai.info, Key Contributions 3 and Methodology: a
+ * closed-form chunk-wise expression through the Gram matrix of the keys;
+ * only the chunk-start state is carried from chunk to chunk).
+ * Within a chunk with start state H_s and positions j = 0..C-1:
+ *   b_j    = prod_{m <= j} beta_m               (decay of H_s to token j)
+ *   w_{ji} = prod_{i < m <= j} beta_m, i <= j   (decay of token i to token j)
+ *   H_j    = b_j H_s + sum_{i<=j} w_{ji} k_i k_i^T
+ *   ||H_j||_F^2 = b_j^2 ||H_s||_F^2 + 2 b_j sum_{i<=j} w_{ji} k_i^T H_s k_i
+ *               + sum_{i,l<=j} w_{ji} w_{jl} (k_i^T k_l)^2
+ * and the next chunk starts from H_s' = b_{C-1} H_s + sum_i w_{C-1,i} k_i k_i^T.
+ * The products are formed directly (no logarithms).  T must be a multiple
+ * of C.  norms: [B, Hh, T].
+ */
+int gka_oracle_chunked_norms(const double *k, const double *beta, int B, int Hh,
+                             int T, int D, int C, double *norms, int nthreads)
+{
+    if (B < 0 || Hh < 0 || T < 0 || D <= 0 || C <= 0 || T % C != 0) return -1;
+    long nh = (long)B * Hh;
+    size_t DD = (size_t)D * D;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (long h = 0; h < nh; ++h) {
+        double *Hs = (double *)calloc(DD, sizeof(double));
+        double *Hn = (double *)malloc(sizeof(double) * DD);
+        double *u = (double *)malloc(sizeof(double) * C);
+        double *G = (double *)malloc(sizeof(double) * (size_t)C * C);
+        double *w = (double *)malloc(sizeof(double) * (size_t)C * C);
+        double *b = (double *)malloc(sizeof(double) * C);
+        for (int c0 = 0; c0 < T; c0 += C) {
+            const double *K = k + ((size_t)h * T + c0) * D;
+            const double *bt = beta + (size_t)h * T + c0;
+            /* decays */
+            for (int j = 0; j < C; ++j) {
+                double p = 1.0;
+                for (int m = 0; m <= j; ++m) p *= bt[m];
+                b[j] = p;
+                for (int i = 0; i < C; ++i) {
+                    double wji = 0.0;
+                    if (i <= j) {
+                        wji = 1.0;
+                        for (int m = i + 1; m <= j; ++m) wji *= bt[m];
+                    }
+                    w[(size_t)j * C + i] = wji;
+                }
+            }
+            /* ||H_s||^2, u_i = k_i^T H_s k_i, G = K K^T */
+            double hs2 = 0.0;
+            for (size_t e = 0; e < DD; ++e) hs2 += Hs[e] * Hs[e];
+            for (int i = 0; i < C; ++i) {
+                double s = 0.0;
+                for (int p = 0; p < D; ++p)
+                    for (int qd = 0; qd < D; ++qd)
+                        s += K[(size_t)i * D + p] * Hs[(size_t)p * D + qd] * K[(size_t)i * D + qd];
+                u[i] = s;
+                for (int l = 0; l < C; ++l) {
+                    double g = 0.0;
+                    for (int p = 0; p < D; ++p) g += K[(size_t)i * D + p] * K[(size_t)l * D + p];
+                    G[(size_t)i * C + l] = g;
+                }
+            }
+            for (int j = 0; j < C; ++j) {
+                double cross = 0.0, intra = 0.0;
+                for (int i = 0; i <= j; ++i) cross += w[(size_t)j * C + i] * u[i];
+                for (int i = 0; i <= j; ++i)
+                    for (int l = 0; l <= j; ++l) {
+                        double g = G[(size_t)i * C + l];
+                        intra += w[(size_t)j * C + i] * w[(size_t)j * C + l] * g * g;
+                    }
+                double n2 = b[j] * b[j] * hs2 + 2.0 * b[j] * cross + intra;
+                norms[(size_t)h * T + c0 + j] = sqrt(n2 > 0.0 ? n2 : 0.0);
+            }
+            /* chunk-start state for the next chunk */
+            for (int p = 0; p < D; ++p)
+                for (int qd = 0; qd < D; ++qd) {
+                    double s = b[C - 1] * Hs[(size_t)p * D + qd];
+                    for (int i = 0; i < C; ++i)
+                        s += w[(size_t)(C - 1) * C + i] * K[(size_t)i * D + p] * K[(size_t)i * D + qd];
+                    Hn[(size_t)p * D + qd] = s;
+                }
+            memcpy(Hs, Hn, sizeof(double) * DD);
+        }
+        free(Hs); free(Hn); free(u); free(G); free(w); free(b);
+    }
+    return 0;
+}
+
+/* Threads OpenMP would use for the calls above (1 without OpenMP). */
+int gka_oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

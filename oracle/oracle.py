@@ -1,0 +1,160 @@
+"""ctypes front end of the float64 oracle in ``gka_oracle.c``.
+
+TEST INFRASTRUCTURE ONLY (tests, smoke check, CPU baseline).  Arrays are numpy
+float64, C-contiguous.  Inputs of lower precision (bf16, fp32) are upcast
+exactly by the caller before they reach these functions.
+
+Source: "Gated KalmaNet: A Fading Memory Layer Through Test-Time Ridge
+Regression" (arXiv 2511.21016); see the C file for the passages each routine
+follows.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from pathlib import Path
+
+import numpy as np
+
+_HERE = Path(__file__).resolve().parent
+_SRC = _HERE / "gka_oracle.c"
+_LIB = _HERE / "libgka_oracle.so"
+_lib = None
+
+_dp = ctypes.POINTER(ctypes.c_double)
+
+
+def build(force: bool = False) -> Path:
+    """Compile the oracle with gcc (-O2, OpenMP, strict IEEE float64)."""
+    if force or not _LIB.exists() or _LIB.stat().st_mtime < _SRC.stat().st_mtime:
+        tmp = _LIB.with_suffix(f".so.{os.getpid()}.tmp")
+        subprocess.check_call(
+            ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+             "-fno-fast-math", "-ffp-contract=off",
+             str(_SRC), "-o", str(tmp), "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(str(_LIB))
+        i, d = ctypes.c_int, ctypes.c_double
+        lib.gka_oracle_omegas.argtypes = [d, i, _dp]
+        lib.gka_oracle_omegas.restype = None
+        lib.gka_oracle_cheb_solve.argtypes = [_dp, _dp, i, d, d, i, _dp, _dp]
+        lib.gka_oracle_cheb_solve.restype = None
+        lib.gka_oracle_forward.argtypes = [_dp, _dp, _dp, _dp, i, i, i, i, d, i,
+                                           _dp, i, _dp, _dp, _dp, i, _dp, i]
+        lib.gka_oracle_forward.restype = i
+        lib.gka_oracle_decode_step.argtypes = [_dp, _dp, _dp, _dp, _dp, i, i, i,
+                                               d, i, _dp, i]
+        lib.gka_oracle_decode_step.restype = i
+        lib.gka_oracle_chunked_norms.argtypes = [_dp, _dp, i, i, i, i, i, _dp, i]
+        lib.gka_oracle_chunked_norms.restype = i
+        lib.gka_oracle_max_threads.argtypes = []
+        lib.gka_oracle_max_threads.restype = i
+        _lib = lib
+    return _lib
+
+
+def _f64(x) -> np.ndarray:
+    if hasattr(x, "detach"):  # torch tensor: exact upcast on the host
+        x = x.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(_dp)
+
+
+def max_threads() -> int:
+    return int(_load().gka_oracle_max_threads())
+
+
+def omegas(rho: float, n: int) -> np.ndarray:
+    """Chebyshev weights omega_0..omega_{n-1} (omega_0 = 2)."""
+    out = np.zeros(max(n, 1), dtype=np.float64)
+    _load().gka_oracle_omegas(float(rho), int(n), _ptr(out))
+    return out[:n]
+
+
+def cheb_solve(A, q, mu: float, L: float, r: int) -> np.ndarray:
+    """r-step Chebyshev iterate for A x = q, spectrum of A in [mu, L], x_0 = 0."""
+    A = _f64(A)
+    q = _f64(q)
+    D = q.shape[0]
+    assert A.shape == (D, D)
+    x = np.zeros(D)
+    work = np.zeros(3 * D)
+    _load().gka_oracle_cheb_solve(_ptr(A), _ptr(q), D, float(mu), float(L), int(r),
+                                  _ptr(x), _ptr(work))
+    return x
+
+
+def forward(q, k, v, beta, a: float, r: int, *, init_state=None, solve_from: int = 0,
+            want_norms: bool = False, want_final_state: bool = False,
+            chunk: int = 0, want_chunk_states: bool = False, nthreads: int = 0):
+    """Token-by-token forward.  q, k, v: [B, H, T, D]; beta: [B, H, T].
+
+    Returns a dict with ``o`` [B,H,T,D] and, on request, ``norms`` [B,H,T],
+    ``final_state`` [B,H,2,D,D] and ``chunk_states`` [B,H,T/chunk,2,D,D]
+    (the state in force before each chunk's first token).
+    """
+    q, k, v, beta = _f64(q), _f64(k), _f64(v), _f64(beta)
+    B, H, T, D = q.shape
+    assert k.shape == q.shape and v.shape == q.shape and beta.shape == (B, H, T)
+    o = np.zeros((B, H, T, D))
+    norms = np.zeros((B, H, T)) if want_norms else None
+    fs = np.zeros((B, H, 2, D, D)) if want_final_state else None
+    cs = None
+    if want_chunk_states:
+        assert chunk > 0 and T % chunk == 0
+        cs = np.zeros((B, H, T // chunk, 2, D, D))
+    init = None if init_state is None else _f64(init_state)
+    if init is not None:
+        assert init.shape == (B, H, 2, D, D)
+    rc = _load().gka_oracle_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), B, H, T, D,
+                                    float(a), int(r), _ptr(init), int(solve_from),
+                                    _ptr(o), _ptr(norms), _ptr(fs), int(chunk), _ptr(cs),
+                                    int(nthreads))
+    if rc != 0:
+        raise ValueError("gka_oracle_forward: bad arguments")
+    out = {"o": o}
+    if want_norms:
+        out["norms"] = norms
+    if want_final_state:
+        out["final_state"] = fs
+    if want_chunk_states:
+        out["chunk_states"] = cs
+    return out
+
+
+def decode_step(state, q, k, v, beta, a: float, r: int, nthreads: int = 0):
+    """One recurrent step.  state [B,H,2,D,D] (returned updated, new array);
+    q, k, v: [B,H,D]; beta [B,H].  Returns (o [B,H,D], state)."""
+    st = _f64(state).copy()
+    q, k, v, beta = _f64(q), _f64(k), _f64(v), _f64(beta)
+    B, H, D = q.shape
+    assert st.shape == (B, H, 2, D, D) and beta.shape == (B, H)
+    o = np.zeros((B, H, D))
+    rc = _load().gka_oracle_decode_step(_ptr(st), _ptr(q), _ptr(k), _ptr(v), _ptr(beta),
+                                        B, H, D, float(a), int(r), _ptr(o), int(nthreads))
+    if rc != 0:
+        raise ValueError("gka_oracle_decode_step: bad arguments")
+    return o, st
+
+
+def chunked_norms(k, beta, chunk: int, nthreads: int = 0) -> np.ndarray:
+    """||H_t||_F by the chunk-wise closed form.  k [B,H,T,D], beta [B,H,T]."""
+    k, beta = _f64(k), _f64(beta)
+    B, H, T, D = k.shape
+    out = np.zeros((B, H, T))
+    rc = _load().gka_oracle_chunked_norms(_ptr(k), _ptr(beta), B, H, T, D, int(chunk),
+                                          _ptr(out), int(nthreads))
+    if rc != 0:
+        raise ValueError("gka_oracle_chunked_norms: bad arguments")
+    return out
