@@ -1,0 +1,428 @@
+#!/usr/bin/env python
+"""Throughput benchmark of the GKA layer library on B200.
+
+Default workload: the chunked forward on B=8, heads=8, T=2048, D=128, bf16,
+chunk 64, a=0.5, r=20 (the shape of the paper's solver study), seeded
+synthetic inputs.  One step = one gka_forward call over the whole batch.
+A second measurement times the recurrent decode step on 256 x 32 heads with
+an fp32 state of 1 GiB (HBM-bound) and reports GB/s.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line on rank 0.  With --impl reference the float64 CPU
+oracle is timed on the host cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GKA fwd tokens/s (B8·T2048·H8·D128 bf16) & % bf16 tensor peak; decode GB/s"
+WORKLOAD = "bf16_b8h8t2048d128"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default=WORKLOAD)
+    p.add_argument("--no-decode", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--decode-steps", type=int, default=None)
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        d["_source"] = "measured"
+        return d
+    d = dict(FALLBACK_PEAKS)
+    d["_source"] = "fallback"
+    return d
+
+
+def flops_per_head_token(D, C, r):
+    """Algorithmic flops of the chunk form per (head, token), counting the causal
+    C x C products as dense tiles: Chebyshev (r-1)(2D^2+4CD), readout 2D^2+4CD,
+    state update 4D^2, norm 2D^2+2CD+2C^2."""
+    ch = (r - 1) * (2 * D * D + 4 * C * D)
+    out = 2 * D * D + 4 * C * D
+    upd = 4 * D * D
+    nrm = 2 * D * D + 2 * C * D + 2 * C * C
+    return ch, out, upd, nrm
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def _heads(x, n, w, with_d=True):
+    if with_d:
+        return x.reshape(w.B * w.H, w.T, w.D)[:n].reshape(1, n, w.T, w.D)
+    return x.reshape(w.B * w.H, w.T)[:n].reshape(1, n, w.T)
+
+
+def oracle_calibrate(w, budget_s, q, k, v, beta):
+    """Number of whole heads the oracle runs in about `budget_s` seconds with
+    all host threads (measured on one head per thread)."""
+    import oracle
+    nth = cpu_threads()
+    n0 = max(1, min(nth, w.B * w.H))
+    t0 = time.perf_counter()
+    oracle.forward(_heads(q, n0, w), _heads(k, n0, w), _heads(v, n0, w),
+                   _heads(beta, n0, w, False), w.a, w.r, nthreads=n0)
+    t_par = time.perf_counter() - t0
+    rounds = max(1, int(budget_s / max(t_par, 1e-3)))
+    return max(1, min(w.B * w.H, n0 * rounds))
+
+
+def oracle_sample(w, nheads, q, k, v, beta):
+    """Times the oracle on the first `nheads` whole heads of the workload;
+    returns (tokens/s in the metric's unit, seconds, threads)."""
+    import oracle
+    threads = min(cpu_threads(), nheads)
+    args = (_heads(q, nheads, w), _heads(k, nheads, w), _heads(v, nheads, w),
+            _heads(beta, nheads, w, False))
+    t0 = time.perf_counter()
+    oracle.forward(*args, w.a, w.r, nthreads=threads)
+    dt = time.perf_counter() - t0
+    tokens = nheads * w.T / w.H          # metric tokens: (batch, position) over all heads
+    return tokens / dt, dt, threads
+
+
+def run_reference(args, w, cfg, rank, world):
+    """The oracle, timed on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    from test_ridge_regression_b200.inputs import workload_inputs
+    q, k, v, beta = workload_inputs(w)
+    total = args.steps + args.warmup
+    budget = min(5.0, max(0.5, 150.0 / max(total, 1)))
+    nheads = oracle_calibrate(w, budget, q, k, v, beta)
+    vals = []
+    info = None
+    for i in range(total):
+        val, dt, threads = oracle_sample(w, nheads, q, k, v, beta)
+        if i >= args.warmup:
+            vals.append(val)
+            info = (nheads, threads)
+    value = statistics.mean(vals) if vals else 0.0
+    tok_step = w.B * w.T
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tok_step / value if value else None,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": cfg,
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": info[1] if info else 0,
+                         "kind": "oracle",
+                         "sample": f"{info[0]} whole heads x {w.T} tokens of the workload per "
+                                   f"step (float64 C oracle, OpenMP over heads)" if info else ""},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from test_ridge_regression_b200.inputs import WORKLOADS
+    w = WORKLOADS[args.workload]
+    cfg = {"workload": w.name, "B": w.B, "heads": w.H, "T": w.T, "D": w.D, "chunk": w.chunk,
+           "a": w.a, "r": w.r, "beta": f"sigmoid(N({w.beta_mu},{w.beta_sigma}))",
+           "global_batch": w.B * world, "seq_len": w.T, "parallelism": f"dp{world}",
+           "l2": "flushed (256 MiB write) before every timed step"}
+    if args.impl == "reference":
+        run_reference(args, w, cfg, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from test_ridge_regression_b200 import build, gka
+    from test_ridge_regression_b200.inputs import workload_inputs
+
+    build.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    peaks = load_peaks()
+    q, k, v, beta = workload_inputs(w)
+    qd, kd, vd, bd = (t.to(dev) for t in (q, k, v, beta))
+    od = torch.empty_like(vd)
+    ws = gka.alloc_workspace(w.B, w.H, w.T, w.D, w.chunk, w.dtype, dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def step():
+        gka.gka_forward(qd, kd, vd, bd, w.a, w.r, w.chunk, o=od, workspace=ws)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if gka.device_status() != 0:
+        raise RuntimeError("device status error after warm-up")
+
+    # ---- timed region: K steps, L2 flushed before each, events per step ----
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    gka.profiler_read()
+    gka.profiler_enable(True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.fill_(float(i))
+            starts[i].record()
+            step()
+            ends[i].record()
+        torch.cuda.synchronize()
+    barrier()
+    gka.profiler_enable(False)
+    kt = gka.profiler_read()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    tok_step = w.B * w.T
+    value = world * tok_step * args.steps / (total_ms / 1e3)
+    launches = sum(n for _, n in kt.values())
+
+    # ---- roofline of the dominant kernel ----
+    ch, out, upd, nrm = flops_per_head_token(w.D, w.chunk, w.r)
+    head_tok = w.B * w.H * w.T
+    dom = max(kt.items(), key=lambda kv: kv[1][0])
+    dom_name, (dom_ms, dom_n) = dom
+    per_launch_ms = dom_ms / dom_n
+    alg = {"chunk_solve": ch + out, "chunk_norm": nrm, "chunk_delta": upd}.get(dom_name, 0)
+    kernel_flops = alg * head_tok
+    sm_mhz_max = peaks.get("sm_max_mhz", 1965.0)
+    if dom_name == "chunk_solve" and getattr(gka, "SOLVE_ON_TENSOR_CORES", False):
+        bound, peak, punit = "tensor", peaks["bf16_tflops"], "TFLOP/s"
+        peak_note = f"bf16 dense, {peaks['_source']} burst"
+    else:
+        # CUDA-core fp32 FMA: 148 SMs x 128 lanes x 2 flop x max SM clock
+        bound, punit = "alu", "TFLOP/s"
+        peak = 148 * 128 * 2 * sm_mhz_max * 1e6 / 1e12
+        peak_note = "fp32 FMA: 148 SMs x 128 lanes x 2 flop x max SM clock"
+    achieved = kernel_flops / (per_launch_ms / 1e3) / 1e12
+    whole_flops = (ch + out + upd + nrm) * head_tok
+    roofline = {"bound": bound, "kernel": dom_name, "achieved": achieved, "peak": peak,
+                "unit": punit, "frac": achieved / peak, "traffic": None,
+                "peak_source": peak_note,
+                "algorithmic_per_launch": kernel_flops,
+                "step_frac_of_bf16_peak": whole_flops / (ms_per_step / 1e3) / 1e12
+                / peaks["bf16_tflops"]}
+
+    result = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": cfg, "roofline": roofline, "gpu_launches": launches,
+        "kernels_ms_per_step": {n: ms / args.steps for n, (ms, _) in kt.items()},
+        "clocks": clk.summary(),
+    }
+
+    # ---- end to end: pinned host buffers, copies inside the timed region ----
+    qh, kh, vh, bh = (t.pin_memory() for t in (q, k, v, beta))
+    oh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for _ in range(2):
+        qd.copy_(qh, non_blocking=True)
+        step()
+        oh.copy_(od, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        e_starts[i].record()
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        bd.copy_(bh, non_blocking=True)
+        step()
+        oh.copy_(od, non_blocking=True)
+        e_ends[i].record()
+    torch.cuda.synchronize()
+    barrier()
+    e_ms = sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends))
+    if world > 1:
+        t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e_ms = float(t.item())
+    h2d = sum(t.numel() * t.element_size() for t in (q, k, v, beta))
+    result["e2e"] = {"value": world * tok_step * args.steps / (e_ms / 1e3), "unit": "tokens/s",
+                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": oh.numel() * oh.element_size()}
+    del qh, kh, vh, bh, oh
+
+    # ---- decode step: HBM-bound, 256 x 32 heads, fp32 state ----
+    if not args.no_decode and world == 1:
+        result["decode"] = bench_decode(args, dev, peaks)
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1) ----
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        nheads = oracle_calibrate(w, 15.0, q, k, v, beta)
+        val, dt, threads = oracle_sample(w, nheads, q, k, v, beta)
+        result["cpu_baseline"] = {
+            "value": val, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{nheads} whole heads x {w.T} tokens of the workload ({dt:.1f} s, "
+                      f"float64 C oracle, OpenMP over heads)"}
+    if gka.device_status() != 0:
+        raise RuntimeError("device status error")
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def bench_decode(args, dev, peaks):
+    import torch
+    from test_ridge_regression_b200 import gka
+    from test_ridge_regression_b200.inputs import DECODE as w
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(w.seed)
+
+    def draw(b, h, t):
+        qq = torch.randn(b, h, t, w.D, generator=gen, device=dev)
+        kk = torch.randn(b, h, t, w.D, generator=gen, device=dev)
+        vv = torch.randn(b, h, t, w.D, generator=gen, device=dev)
+        bb = torch.sigmoid(w.beta_mu + w.beta_sigma * torch.randn(b, h, t, generator=gen,
+                                                                   device=dev))
+        qq = (qq / qq.norm(dim=-1, keepdim=True)).to(torch.bfloat16)
+        kk = (kk / kk.norm(dim=-1, keepdim=True)).to(torch.bfloat16)
+        return qq, kk, vv.to(torch.bfloat16), bb.contiguous()
+
+    # prefill through the forward path: the decode state is its final state
+    state = torch.empty(w.batch, w.H, 2, w.D, w.D, device=dev)
+    pq, pk, pv, pb = draw(w.batch, w.H, w.prefill)
+    gka.gka_forward(pq, pk, pv, pb, w.a, w.r, 64, final_state=state)
+    del pq, pk, pv, pb
+    torch.cuda.empty_cache()
+    nsets = 16
+    sets = [tuple(x[:, :, 0].contiguous() for x in draw(w.batch, w.H, 1)) for _ in range(nsets)]
+    o = torch.empty(w.batch, w.H, w.D, dtype=torch.bfloat16, device=dev)
+    steps = args.decode_steps or w.steps
+    for i in range(5):
+        qq, kk, vv, bb = sets[i % nsets]
+        gka.gka_decode_step(state, qq, kk, vv, bb, w.a, w.r, o=o)
+    torch.cuda.synchronize()
+    gka.profiler_read()
+    gka.profiler_enable(True)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        s.record()
+        for i in range(steps):
+            qq, kk, vv, bb = sets[i % nsets]
+            gka.gka_decode_step(state, qq, kk, vv, bb, w.a, w.r, o=o)
+        e.record()
+        torch.cuda.synchronize()
+    gka.profiler_enable(False)
+    kt = gka.profiler_read()
+    ms = s.elapsed_time(e) / steps
+    heads = w.batch * w.H
+    bytes_step = heads * (4 * w.D * w.D * 4 + 4 * w.D * 2 + 4)
+    k_ms, k_n = kt["decode_step"]
+    achieved = bytes_step / (k_ms / k_n / 1e3) / 1e9
+    return {
+        "workload": w.name, "steps": steps, "ms_per_step": ms,
+        "tokens_per_s": w.batch / (ms / 1e3), "GB_per_s": bytes_step / (ms / 1e3) / 1e9,
+        "roofline": {"bound": "hbm", "kernel": "decode_step", "achieved": achieved,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "algorithmic_per_launch": bytes_step,
+                     "peak_source": f"{peaks['_source']} copy bandwidth"},
+        "gpu_launches": k_n, "clocks": clk.summary(),
+    }
+
+
+if __name__ == "__main__":
+    main()

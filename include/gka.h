@@ -1,0 +1,160 @@
+/*
+ * gka.h - C ABI of the Gated KalmaNet (GKA) layer library for NVIDIA B200
+ * (sm_100a).
+ *
+ * The layer ("Gated KalmaNet: A Fading Memory Layer Through Test-Time Ridge
+ * Regression", arXiv 2511.21016; ai.info page, Key Contributions 2-3 and
+ * Methodology in Plain English) keeps, per (batch, head) and per token t,
+ *     H_t = beta_t H_{t-1} + k_t k_t^T         (gated fading Gram state)
+ *     M_t = beta_t M_{t-1} + v_t k_t^T         (value state, the paper's U_t)
+ * sets the adaptive ridge lambda_t = a ||H_t||_F (condition number at most
+ * (a+1)/a), approximately solves (H_t + lambda_t I) x_t = q_t with r steps of
+ * the Chebyshev iteration on the interval [a ||H_t||_F, (1+a) ||H_t||_F]
+ * started from x = 0, and emits o_t = M_t x_t.  The Chebyshev weights follow
+ * the schedule of the pith.science appendix (Lemma 3): omega_0 = 2,
+ * omega_i = 1/(1 - rho^2 omega_{i-1}/4), rho = 1/(1+2a).
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the
+ *     library allocates no device memory and frees nothing.  Every call is
+ *     asynchronous on `stream` (a cudaStream_t passed as void*; NULL = the
+ *     legacy default stream).  Buffers must stay alive until the stream has
+ *     run the call.
+ *   - Layouts are dense row-major: q, k, v, o are [B, H, T, D] with D
+ *     fastest; beta is [B, H, T] fp32.  States are fp32 [B, H, 2, D, D]:
+ *     H then M, each row-major (M maps keys to values: o = M x).
+ *   - Every tensor pointer must be 16-byte aligned.
+ *   - Return value: GKA_OK (0) or a negative gka_status.  On an error no
+ *     kernel has been launched and no output has been written, except for
+ *     GKA_ERR_CUDA, which reports a failed launch (the CUDA error code is
+ *     kept for gka_last_cuda_error()).
+ *   - Supported: D in {32, 64, 128}; chunk in {16, 32, 64, 128}; 1 <= r <= 256;
+ *     a > 0 and finite.
+ */
+#ifndef GKA_H
+#define GKA_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { GKA_F32 = 0, GKA_BF16 = 1 } gka_dtype;
+
+typedef enum {
+    GKA_OK = 0,
+    GKA_ERR_INVALID_ARG = -1,            /* null pointer, negative size, a <= 0, r < 1 ... */
+    GKA_ERR_UNSUPPORTED = -2,            /* D, chunk or r outside the supported set */
+    GKA_ERR_T_NOT_MULTIPLE_OF_CHUNK = -3,/* the chunk-wise form needs N = T / chunk chunks */
+    GKA_ERR_WORKSPACE_TOO_SMALL = -4,
+    GKA_ERR_CUDA = -5,                   /* a CUDA call failed; see gka_last_cuda_error() */
+    GKA_ERR_DEVICE_TIMEOUT = -6,         /* a bounded device-side wait gave up */
+    GKA_ERR_MISALIGNED = -7              /* a pointer is not 16-byte aligned */
+} gka_status;
+
+/* Byte offsets of the regions of the gka_forward workspace (diagnostics and
+ * tests read the intermediate results through this).  Every offset is a
+ * multiple of 256. */
+typedef struct {
+    size_t states_offset;   /* fp32 [B, H, N+1, 2, D, D]: H_s, M_s in force before chunk n;
+                               slot N holds the state after the last token */
+    size_t decay_offset;    /* fp32 [B, H, N]: product of beta over chunk n */
+    size_t norms_offset;    /* fp32 [B, H, T]: ||H_t||_F */
+    size_t states_bf16_offset; /* bf16 [B, H, N, 2, D, D] copy of the chunk-start states
+                                  (tensor-core path only; 0 bytes otherwise) */
+    size_t total_bytes;
+} gka_workspace_layout;
+
+/* Workspace bytes gka_forward needs for this problem (0 on invalid sizes). */
+size_t gka_forward_workspace_bytes(int B, int H, int T, int D, int chunk, gka_dtype dt);
+
+/* Fills *out with the workspace layout for this problem.  Returns a gka_status. */
+int gka_forward_workspace_layout(int B, int H, int T, int D, int chunk, gka_dtype dt,
+                                 gka_workspace_layout *out);
+
+/*
+ * Chunk-wise GKA forward (ai.info page, Key Contributions 3 and Methodology:
+ * the sequence is cut into N = T / chunk chunks; only each chunk's start
+ * state is computed sequentially; ||H_t||_F comes from a closed form through
+ * the Gram matrix of the keys; everything within a chunk runs in parallel).
+ * Steps, each a kernel on `stream`:
+ *   1. chunk-state scan: H_s, M_s before every chunk (fp32), into workspace;
+ *   2. per-token ||H_t||_F, into workspace;
+ *   3. r-step Chebyshev solve for every token and 4. the readout o_t = M_t x_t.
+ * The result does not depend on `chunk` beyond floating-point rounding.
+ *
+ *   q, k, v     [B, H, T, D] in `dt` (fp32 or bf16); k and q are used as given
+ *               (callers l2-normalise them, as the GKA block does)
+ *   beta        [B, H, T] fp32 in [0, 1]: decay of the previous state
+ *   o           [B, H, T, D] in `dt` (written)
+ *   a, r        ridge factor (> 0) and Chebyshev steps (r - 1 matrix-vector
+ *               products per token)
+ *   chunk       chunk length C; T must be a multiple of it
+ *   final_state nullable fp32 [B, H, 2, D, D]: state after the last token
+ *               (written), e.g. to continue with gka_decode_step
+ *   workspace   device scratch of at least gka_forward_workspace_bytes()
+ *               bytes, 256-byte aligned; contents on entry are ignored
+ */
+int gka_forward(const void *q, const void *k, const void *v, const float *beta, void *o,
+                int B, int H, int T, int D, gka_dtype dt, float a, int r, int chunk,
+                float *final_state, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * One recurrent decode step for B*H heads (ai.info page, Key Contributions 4:
+ * the recurrent form used for inference), in place on the fp32 state:
+ *   H <- beta H + k k^T;  n = ||H||_F;  x = r-step Chebyshev for
+ *   (H + a n I) x = q on [a n, (1+a) n];  M <- beta M + v k^T;  o = M x.
+ *   state  fp32 [B, H, 2, D, D] (read and written)
+ *   q, k, v, o  [B, H, D] in `dt`;  beta [B, H] fp32.
+ * A head whose H is all zero after the update gets o = 0.
+ */
+int gka_decode_step(float *state, const void *q, const void *k, const void *v,
+                    const float *beta, void *o, int B, int H, int D, gka_dtype dt,
+                    float a, int r, void *stream);
+
+/* Synchronises `stream`, then returns GKA_ERR_DEVICE_TIMEOUT if any kernel of
+ * this library on the current device gave up a bounded wait since the last
+ * call (and clears the flag), GKA_ERR_CUDA if the stream reports an error,
+ * else GKA_OK. */
+int gka_device_status(void *stream);
+
+/* CUDA error code (cudaError_t) behind the last GKA_ERR_CUDA, 0 if none. */
+int gka_last_cuda_error(void);
+
+/* Static text for a gka_status value. */
+const char *gka_status_string(int status);
+
+/* Library ABI version: 100 * major + minor. */
+int gka_version(void);
+
+/* Launch profiler.  Kernels of the library, by index into gka_kernel_times. */
+enum {
+    GKA_KERNEL_CHUNK_DELTA = 0,   /* chunk-state increments (scan step 1a) */
+    GKA_KERNEL_STATE_SCAN = 1,    /* sequential state scan over chunks (step 1b) */
+    GKA_KERNEL_CHUNK_NORM = 2,    /* per-token ||H_t||_F */
+    GKA_KERNEL_CHUNK_SOLVE = 3,   /* Chebyshev solve + readout */
+    GKA_KERNEL_DECODE_STEP = 4,   /* recurrent decode step */
+    GKA_KERNEL_COUNT = 8
+};
+
+typedef struct {
+    double ms[GKA_KERNEL_COUNT];  /* summed device time per kernel */
+    int launches[GKA_KERNEL_COUNT];
+} gka_kernel_times;
+
+/* While enabled (on != 0), every kernel launch is bracketed by two CUDA
+ * events recorded on its stream (host-side bookkeeping; no device memory).
+ * Not thread-safe against concurrent launches from several host threads
+ * beyond a mutex around the bookkeeping. */
+int gka_profiler_enable(int on);
+
+/* Waits for the recorded events, fills *out with the per-kernel sums since
+ * the last read, and forgets them. */
+int gka_profiler_read(gka_kernel_times *out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GKA_H */

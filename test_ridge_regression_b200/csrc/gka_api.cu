@@ -1,0 +1,341 @@
+// C ABI of the GKA library: argument checks, workspace layout, launches.
+// The declarations and the contract of every entry point are in include/gka.h.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+#include <vector>
+
+#include "../../include/gka.h"
+#include "chunk_simt.cuh"
+#include "common.cuh"
+#include "decode.cuh"
+
+namespace gka {
+
+// Set by a kernel whose bounded wait gave up; read and cleared by
+// gka_device_status().  One per device (module-scope device variable).
+__device__ int g_timeout_flag = 0;
+
+static std::atomic<int> g_last_cuda_error{0};
+
+// ---------------------------------------------------------------------------
+// Launch profiler: when enabled, every kernel launch of the library is
+// bracketed by a pair of CUDA events recorded on the launch stream.  Elapsed
+// times are summed per kernel when gka_profiler_read() is called.
+// ---------------------------------------------------------------------------
+struct ProfRecord {
+    int kernel;
+    cudaEvent_t start, stop;
+};
+static bool g_prof_on = false;
+static std::vector<ProfRecord> g_prof_pending;
+static std::vector<cudaEvent_t> g_prof_pool;
+static std::mutex g_prof_mu;
+
+static cudaEvent_t prof_event() {
+    if (!g_prof_pool.empty()) {
+        cudaEvent_t e = g_prof_pool.back();
+        g_prof_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+struct ProfScope {
+    int kernel;
+    cudaStream_t s;
+    cudaEvent_t start = nullptr;
+    ProfScope(int k, cudaStream_t st) : kernel(k), s(st) {
+        if (!g_prof_on) return;
+        std::lock_guard<std::mutex> g(g_prof_mu);
+        start = prof_event();
+        if (start) cudaEventRecord(start, s);
+    }
+    ~ProfScope() {
+        if (!start) return;
+        std::lock_guard<std::mutex> g(g_prof_mu);
+        cudaEvent_t stop = prof_event();
+        if (!stop) return;
+        cudaEventRecord(stop, s);
+        g_prof_pending.push_back({kernel, start, stop});
+    }
+};
+
+static int cuda_fail(cudaError_t e) {
+    g_last_cuda_error.store((int)e);
+    return GKA_ERR_CUDA;
+}
+
+static int check_launch() {
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? GKA_OK : cuda_fail(e);
+}
+
+static bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+static size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+static bool supported_d(int D) { return D == 32 || D == 64 || D == 128; }
+static bool supported_c(int C) { return C == 16 || C == 32 || C == 64 || C == 128; }
+
+// Chebyshev constants of one call (pith.science appendix, Lemma 3: omega_0 = 2,
+// omega_i = 1/(1 - rho^2 omega_{i-1}/4)); computed in double, stored in float.
+static ChebParams make_cheb(float a, int r) {
+    ChebParams P;
+    memset(&P, 0, sizeof(P));
+    P.a = a;
+    P.half_1p2a = (float)((1.0 + 2.0 * (double)a) * 0.5);
+    P.r = r;
+    const double rho = 1.0 / (1.0 + 2.0 * (double)a);
+    double w = 2.0;
+    P.omega[0] = (float)w;
+    for (int i = 1; i < r && i < kMaxSteps; ++i) {
+        w = 1.0 / (1.0 - rho * rho * w / 4.0);
+        P.omega[i] = (float)w;
+    }
+    return P;
+}
+
+static int layout(int B, int H, int T, int D, int C, gka_dtype dt, gka_workspace_layout *L) {
+    if (B < 0 || H < 0 || T < 0) return GKA_ERR_INVALID_ARG;
+    if (dt != GKA_F32 && dt != GKA_BF16) return GKA_ERR_INVALID_ARG;
+    if (!supported_d(D) || !supported_c(C)) return GKA_ERR_UNSUPPORTED;
+    if (T % C != 0) return GKA_ERR_T_NOT_MULTIPLE_OF_CHUNK;
+    const size_t BH = (size_t)B * H, N = (size_t)(T / C);
+    size_t off = 0;
+    L->states_offset = off;
+    off = round256(off + sizeof(float) * BH * (N + 1) * 2 * D * D);
+    L->decay_offset = off;
+    off = round256(off + sizeof(float) * BH * N);
+    L->norms_offset = off;
+    off = round256(off + sizeof(float) * BH * (size_t)T);
+    L->states_bf16_offset = off;
+    L->total_bytes = off;
+    return GKA_OK;
+}
+
+template <typename K>
+static cudaError_t set_smem(K kernel, size_t bytes) {
+    if (bytes <= 48 * 1024) return cudaSuccess;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+template <typename Tin, int D>
+static int forward_simt(const Tin *q, const Tin *k, const Tin *v, const float *beta, Tin *o,
+                        int B, int H, int T, int C, const ChebParams &P, float *final_state,
+                        char *ws, const gka_workspace_layout &L, cudaStream_t s) {
+    const int BH = B * H, N = T / C;
+    float *states = reinterpret_cast<float *>(ws + L.states_offset);
+    float *decay = reinterpret_cast<float *>(ws + L.decay_offset);
+    float *norms = reinterpret_cast<float *>(ws + L.norms_offset);
+    cudaError_t e;
+
+    const size_t sm_delta = sizeof(float) * 3 * (size_t)C * D;
+    if ((e = set_smem(k_chunk_delta<Tin, D>, sm_delta)) != cudaSuccess) return cuda_fail(e);
+    { ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
+    k_chunk_delta<Tin, D><<<dim3(N, BH), kSimtThreads, sm_delta, s>>>(k, v, beta, states, decay, T,
+                                                                        N, C); }
+    if (int rc = check_launch()) return rc;
+
+    const int DD2 = 2 * D * D;
+    { ProfScope ps(GKA_KERNEL_STATE_SCAN, s);
+    k_state_scan<<<dim3((DD2 + 255) / 256, BH), 256, 0, s>>>(states, decay, final_state, N, DD2); }
+    if (int rc = check_launch()) return rc;
+
+    const size_t sm_norm = sizeof(float) * ((size_t)D * D + (size_t)C * (D + 1));
+    if ((e = set_smem(k_chunk_norm<Tin, D>, sm_norm)) != cudaSuccess) return cuda_fail(e);
+    { ProfScope ps(GKA_KERNEL_CHUNK_NORM, s);
+    k_chunk_norm<Tin, D><<<dim3(N, BH), kSimtThreads, sm_norm, s>>>(k, beta, states, norms, T, N,
+                                                                    C); }
+    if (int rc = check_launch()) return rc;
+
+    const size_t sm_solve = SolveSmem<D>::bytes(C);
+    if ((e = set_smem(k_chunk_solve<Tin, D>, sm_solve)) != cudaSuccess) return cuda_fail(e);
+    { ProfScope ps(GKA_KERNEL_CHUNK_SOLVE, s);
+    k_chunk_solve<Tin, D><<<dim3(C / kSolveTG, N, BH), kSimtThreads, sm_solve, s>>>(
+        q, k, v, beta, states, norms, o, T, N, C, P); }
+    return check_launch();
+}
+
+template <typename Tin>
+static int forward_dispatch(const void *q, const void *k, const void *v, const float *beta,
+                            void *o, int B, int H, int T, int D, int C, const ChebParams &P,
+                            float *final_state, char *ws, const gka_workspace_layout &L,
+                            cudaStream_t s) {
+    auto Q = static_cast<const Tin *>(q);
+    auto K = static_cast<const Tin *>(k);
+    auto V = static_cast<const Tin *>(v);
+    auto O = static_cast<Tin *>(o);
+    switch (D) {
+        case 32: return forward_simt<Tin, 32>(Q, K, V, beta, O, B, H, T, C, P, final_state, ws, L, s);
+        case 64: return forward_simt<Tin, 64>(Q, K, V, beta, O, B, H, T, C, P, final_state, ws, L, s);
+        default: return forward_simt<Tin, 128>(Q, K, V, beta, O, B, H, T, C, P, final_state, ws, L, s);
+    }
+}
+
+static int timeout_flag_ptr(int **ptr) {
+    cudaError_t e = cudaGetSymbolAddress((void **)ptr, g_timeout_flag);
+    return e == cudaSuccess ? GKA_OK : cuda_fail(e);
+}
+
+template <typename Tin, int D>
+static int decode_launch(float *state, const void *q, const void *k, const void *v,
+                         const float *beta, void *o, int BH, const ChebParams &P, cudaStream_t s) {
+    int *flag = nullptr;
+    if (int rc = timeout_flag_ptr(&flag)) return rc;
+    const size_t smem = sizeof(float) * D * D;
+    cudaError_t e = set_smem(k_decode_step<Tin, D>, smem);
+    if (e != cudaSuccess) return cuda_fail(e);
+    ProfScope ps(GKA_KERNEL_DECODE_STEP, s);
+    k_decode_step<Tin, D><<<BH, 4 * D, smem, s>>>(
+        state, static_cast<const Tin *>(q), static_cast<const Tin *>(k),
+        static_cast<const Tin *>(v), beta, static_cast<Tin *>(o), P, flag);
+    return check_launch();
+}
+
+template <typename Tin>
+static int decode_dispatch(float *state, const void *q, const void *k, const void *v,
+                           const float *beta, void *o, int BH, int D, const ChebParams &P,
+                           cudaStream_t s) {
+    switch (D) {
+        case 32: return decode_launch<Tin, 32>(state, q, k, v, beta, o, BH, P, s);
+        case 64: return decode_launch<Tin, 64>(state, q, k, v, beta, o, BH, P, s);
+        default: return decode_launch<Tin, 128>(state, q, k, v, beta, o, BH, P, s);
+    }
+}
+
+}  // namespace gka
+
+using namespace gka;
+
+extern "C" {
+
+size_t gka_forward_workspace_bytes(int B, int H, int T, int D, int chunk, gka_dtype dt) {
+    gka_workspace_layout L;
+    return layout(B, H, T, D, chunk, dt, &L) == GKA_OK ? L.total_bytes : 0;
+}
+
+int gka_forward_workspace_layout(int B, int H, int T, int D, int chunk, gka_dtype dt,
+                                 gka_workspace_layout *out) {
+    if (!out) return GKA_ERR_INVALID_ARG;
+    return layout(B, H, T, D, chunk, dt, out);
+}
+
+int gka_forward(const void *q, const void *k, const void *v, const float *beta, void *o, int B,
+                int H, int T, int D, gka_dtype dt, float a, int r, int chunk, float *final_state,
+                void *workspace, size_t workspace_bytes, void *stream) {
+    gka_workspace_layout L;
+    if (int rc = layout(B, H, T, D, chunk, dt, &L)) return rc;
+    if (!(a > 0.f) || !isfinite(a) || r < 1) return GKA_ERR_INVALID_ARG;
+    if (r > kMaxSteps) return GKA_ERR_UNSUPPORTED;
+    if ((size_t)B * H > 65535) return GKA_ERR_UNSUPPORTED;
+    const size_t BH = (size_t)B * H;
+    if (BH == 0) return GKA_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        if (final_state) {
+            cudaError_t e = cudaMemsetAsync(final_state, 0, sizeof(float) * BH * 2 * D * D, s);
+            if (e != cudaSuccess) return cuda_fail(e);
+        }
+        return GKA_OK;
+    }
+    if (!q || !k || !v || !beta || !o || !workspace) return GKA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(beta) || !aligned16(o) ||
+        (final_state && !aligned16(final_state)) || ((uintptr_t)workspace & 255u))
+        return GKA_ERR_MISALIGNED;
+    if (workspace_bytes < L.total_bytes) return GKA_ERR_WORKSPACE_TOO_SMALL;
+    const ChebParams P = make_cheb(a, r);
+    char *ws = static_cast<char *>(workspace);
+    if (dt == GKA_BF16)
+        return forward_dispatch<__nv_bfloat16>(q, k, v, beta, o, B, H, T, D, chunk, P,
+                                               final_state, ws, L, s);
+    return forward_dispatch<float>(q, k, v, beta, o, B, H, T, D, chunk, P, final_state, ws, L, s);
+}
+
+int gka_decode_step(float *state, const void *q, const void *k, const void *v, const float *beta,
+                    void *o, int B, int H, int D, gka_dtype dt, float a, int r, void *stream) {
+    if (B < 0 || H < 0) return GKA_ERR_INVALID_ARG;
+    if (dt != GKA_F32 && dt != GKA_BF16) return GKA_ERR_INVALID_ARG;
+    if (!supported_d(D)) return GKA_ERR_UNSUPPORTED;
+    if (!(a > 0.f) || !isfinite(a) || r < 1) return GKA_ERR_INVALID_ARG;
+    if (r > kMaxSteps) return GKA_ERR_UNSUPPORTED;
+    const size_t BH = (size_t)B * H;
+    if (BH == 0) return GKA_OK;
+    if (BH > 0x7fffffffu) return GKA_ERR_UNSUPPORTED;
+    if (!state || !q || !k || !v || !beta || !o) return GKA_ERR_INVALID_ARG;
+    if (!aligned16(state) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(beta) ||
+        !aligned16(o))
+        return GKA_ERR_MISALIGNED;
+    const ChebParams P = make_cheb(a, r);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dt == GKA_BF16) return decode_dispatch<__nv_bfloat16>(state, q, k, v, beta, o, (int)BH, D, P, s);
+    return decode_dispatch<float>(state, q, k, v, beta, o, (int)BH, D, P, s);
+}
+
+int gka_device_status(void *stream) {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    int flag = 0;
+    e = cudaMemcpyFromSymbol(&flag, g_timeout_flag, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (flag) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbol(g_timeout_flag, &zero, sizeof(int));
+        if (e != cudaSuccess) return cuda_fail(e);
+        return GKA_ERR_DEVICE_TIMEOUT;
+    }
+    return GKA_OK;
+}
+
+int gka_last_cuda_error(void) { return g_last_cuda_error.load(); }
+
+const char *gka_status_string(int status) {
+    switch (status) {
+        case GKA_OK: return "ok";
+        case GKA_ERR_INVALID_ARG: return "invalid argument";
+        case GKA_ERR_UNSUPPORTED: return "unsupported size or parameter";
+        case GKA_ERR_T_NOT_MULTIPLE_OF_CHUNK: return "T is not a multiple of chunk";
+        case GKA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+        case GKA_ERR_CUDA: return "CUDA error";
+        case GKA_ERR_DEVICE_TIMEOUT: return "a bounded device wait timed out";
+        case GKA_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+        default: return "unknown status";
+    }
+}
+
+int gka_version(void) { return 100; }
+
+int gka_profiler_enable(int on) {
+    std::lock_guard<std::mutex> g(g_prof_mu);
+    g_prof_on = on != 0;
+    return GKA_OK;
+}
+
+int gka_profiler_read(gka_kernel_times *out) {
+    if (!out) return GKA_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> g(g_prof_mu);
+    memset(out, 0, sizeof(*out));
+    int rc = GKA_OK;
+    for (const ProfRecord &p : g_prof_pending) {
+        float ms = 0.f;
+        cudaError_t e = cudaEventSynchronize(p.stop);
+        if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, p.start, p.stop);
+        if (e != cudaSuccess) rc = cuda_fail(e);
+        if (p.kernel >= 0 && p.kernel < GKA_KERNEL_COUNT) {
+            out->ms[p.kernel] += ms;
+            out->launches[p.kernel] += 1;
+        }
+        g_prof_pool.push_back(p.start);
+        g_prof_pool.push_back(p.stop);
+    }
+    g_prof_pending.clear();
+    return rc;
+}
+
+}  // extern "C"

@@ -1,0 +1,185 @@
+"""Python binding of libgka.so: argument marshalling only.
+
+Every step of the layer runs in the library's CUDA kernels; this module checks
+tensor shapes, dtypes and devices, hands raw device pointers and the current
+CUDA stream to the C ABI (include/gka.h) and raises on a non-zero status.
+There is no fallback: if the library is missing or a call fails, it raises.
+"""
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+
+import torch
+
+_PKG = Path(__file__).resolve().parent
+LIB_PATH = _PKG / "libgka.so"
+
+GKA_F32, GKA_BF16 = 0, 1
+_DT = {torch.float32: GKA_F32, torch.bfloat16: GKA_BF16}
+
+
+class GkaError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        msg = _lib().gka_status_string(status).decode()
+        if status == -5:
+            msg += f" (cudaError {_lib().gka_last_cuda_error()})"
+        super().__init__(f"{fn}: {msg} [{status}]")
+
+
+KERNEL_NAMES = ["chunk_delta", "state_scan", "chunk_norm", "chunk_solve", "decode_step"]
+
+
+class KernelTimes(ctypes.Structure):
+    _fields_ = [("ms", ctypes.c_double * 8), ("launches", ctypes.c_int * 8)]
+
+
+class WorkspaceLayout(ctypes.Structure):
+    _fields_ = [("states_offset", ctypes.c_size_t), ("decay_offset", ctypes.c_size_t),
+                ("norms_offset", ctypes.c_size_t), ("states_bf16_offset", ctypes.c_size_t),
+                ("total_bytes", ctypes.c_size_t)]
+
+
+_L = None
+
+
+def _lib():
+    global _L
+    if _L is None:
+        if not LIB_PATH.exists():
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m test_ridge_regression_b200.build`")
+        lib = ctypes.CDLL(str(LIB_PATH))
+        vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        lib.gka_forward_workspace_bytes.argtypes = [i, i, i, i, i, i]
+        lib.gka_forward_workspace_bytes.restype = sz
+        lib.gka_forward_workspace_layout.argtypes = [i, i, i, i, i, i, ctypes.POINTER(WorkspaceLayout)]
+        lib.gka_forward_workspace_layout.restype = i
+        lib.gka_forward.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, vp, sz, vp]
+        lib.gka_forward.restype = i
+        lib.gka_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+        lib.gka_decode_step.restype = i
+        lib.gka_device_status.argtypes = [vp]
+        lib.gka_device_status.restype = i
+        lib.gka_last_cuda_error.argtypes = []
+        lib.gka_last_cuda_error.restype = i
+        lib.gka_status_string.argtypes = [i]
+        lib.gka_status_string.restype = ctypes.c_char_p
+        lib.gka_version.argtypes = []
+        lib.gka_version.restype = i
+        lib.gka_profiler_enable.argtypes = [i]
+        lib.gka_profiler_enable.restype = i
+        lib.gka_profiler_read.argtypes = [ctypes.POINTER(KernelTimes)]
+        lib.gka_profiler_read.restype = i
+        _L = lib
+    return _L
+
+
+def lib():
+    """The loaded ctypes library (raises ImportError if it was not built)."""
+    return _lib()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(fn, rc):
+    if rc != 0:
+        raise GkaError(fn, rc)
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype not in _DT:
+        raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
+    return _DT[t.dtype]
+
+
+def _dev(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def workspace_bytes(B, H, T, D, chunk, dtype=torch.bfloat16) -> int:
+    return int(_lib().gka_forward_workspace_bytes(B, H, T, D, chunk, _DT[dtype]))
+
+
+def workspace_layout(B, H, T, D, chunk, dtype=torch.bfloat16) -> WorkspaceLayout:
+    out = WorkspaceLayout()
+    _check("gka_forward_workspace_layout",
+           _lib().gka_forward_workspace_layout(B, H, T, D, chunk, _DT[dtype], ctypes.byref(out)))
+    return out
+
+
+def alloc_workspace(B, H, T, D, chunk, dtype=torch.bfloat16, device=None) -> torch.Tensor:
+    n = workspace_bytes(B, H, T, D, chunk, dtype)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def gka_forward(q, k, v, beta, a: float, r: int, chunk: int, *, o=None, final_state=None,
+                workspace=None, stream=None):
+    """Chunk-wise GKA forward (see include/gka.h).  q, k, v: [B, H, T, D] fp32 or
+    bf16 CUDA tensors; beta: [B, H, T] fp32.  Returns o (same shape/dtype as v)."""
+    _dev(q, k, v, beta, o, final_state, workspace)
+    B, H, T, D = q.shape
+    if k.shape != q.shape or v.shape != q.shape or beta.shape != (B, H, T):
+        raise ValueError("shape mismatch")
+    dt = _dtype(q)
+    if k.dtype != q.dtype or v.dtype != q.dtype or beta.dtype != torch.float32:
+        raise TypeError("q, k, v must share a dtype; beta must be float32")
+    if o is None:
+        o = torch.empty_like(v)
+    if final_state is not None and (final_state.dtype != torch.float32 or
+                                    final_state.shape != (B, H, 2, D, D)):
+        raise ValueError("final_state must be float32 [B, H, 2, D, D]")
+    if workspace is None:
+        workspace = alloc_workspace(B, H, T, D, chunk, q.dtype, q.device)
+    rc = _lib().gka_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(o), B, H, T, D, dt,
+                            float(a), int(r), int(chunk), _ptr(final_state), _ptr(workspace),
+                            workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("gka_forward", rc)
+    return o
+
+
+def gka_decode_step(state, q, k, v, beta, a: float, r: int, *, o=None, stream=None):
+    """One recurrent step in place on state [B, H, 2, D, D] fp32; q, k, v: [B, H, D];
+    beta: [B, H] fp32.  Returns o [B, H, D]."""
+    _dev(state, q, k, v, beta, o)
+    B, H, D = q.shape
+    if state.dtype != torch.float32 or state.shape != (B, H, 2, D, D):
+        raise ValueError("state must be float32 [B, H, 2, D, D]")
+    if k.shape != q.shape or v.shape != q.shape or beta.shape != (B, H):
+        raise ValueError("shape mismatch")
+    dt = _dtype(q)
+    if o is None:
+        o = torch.empty_like(v)
+    rc = _lib().gka_decode_step(_ptr(state), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(o),
+                                B, H, D, dt, float(a), int(r), _stream(stream))
+    _check("gka_decode_step", rc)
+    return o
+
+
+def device_status(stream=None) -> int:
+    """Synchronises the stream and returns the library's device status code."""
+    return int(_lib().gka_device_status(_stream(stream)))
+
+
+def profiler_enable(on: bool = True) -> None:
+    """Bracket every library kernel launch with CUDA events on its stream."""
+    _check("gka_profiler_enable", _lib().gka_profiler_enable(1 if on else 0))
+
+
+def profiler_read() -> dict:
+    """Per-kernel {name: (total_ms, launches)} since the last read (waits on the events)."""
+    out = KernelTimes()
+    _check("gka_profiler_read", _lib().gka_profiler_read(ctypes.byref(out)))
+    return {name: (out.ms[i], out.launches[i]) for i, name in enumerate(KERNEL_NAMES)
+            if out.launches[i]}

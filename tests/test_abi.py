@@ -1,0 +1,109 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every function include/gka.h declares, and rejects bad arguments with the
+documented status codes before any CUDA call."""
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+
+ROOT = Path(__file__).resolve().parents[1]
+HEADER = ROOT / "include" / "gka.h"
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from test_ridge_regression_b200 import build, gka
+    build.build()
+    return gka.lib()
+
+
+def declared_functions():
+    text = HEADER.read_text()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(gka_[a-z0-9_]+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for must in ["gka_forward", "gka_decode_step", "gka_forward_workspace_bytes",
+                 "gka_forward_workspace_layout", "gka_device_status", "gka_last_cuda_error",
+                 "gka_status_string", "gka_version"]:
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code in range(-7, 1):
+        assert len(lib.gka_status_string(code)) > 0
+    assert lib.gka_version() >= 100
+
+
+def test_workspace_layout(lib):
+    from test_ridge_regression_b200 import gka
+    import torch
+    B, H, T, D, C = 2, 3, 256, 64, 64
+    L = gka.workspace_layout(B, H, T, D, C, torch.float32)
+    N = T // C
+    assert L.states_offset == 0
+    assert L.decay_offset >= 4 * B * H * (N + 1) * 2 * D * D
+    assert L.norms_offset >= L.decay_offset + 4 * B * H * N
+    assert L.total_bytes >= L.norms_offset + 4 * B * H * T
+    for off in (L.states_offset, L.decay_offset, L.norms_offset, L.total_bytes):
+        assert off % 256 == 0
+    assert gka.workspace_bytes(B, H, T, D, C, torch.float32) == L.total_bytes
+    # invalid sizes give 0 bytes
+    assert lib.gka_forward_workspace_bytes(1, 1, 100, 64, 64, 0) == 0
+    assert lib.gka_forward_workspace_bytes(1, 1, 128, 48, 64, 0) == 0
+
+
+FAKE = ctypes.c_void_p(1 << 20)       # never dereferenced: every call below fails validation
+FAKE_MIS = ctypes.c_void_p((1 << 20) + 4)
+
+
+def fwd(lib, *, q=FAKE, beta=FAKE, B=1, H=1, T=128, D=64, dt=0, a=0.5, r=4, C=64, ws=FAKE,
+        ws_bytes=1 << 40):
+    return lib.gka_forward(q, FAKE, FAKE, beta, FAKE, B, H, T, D, dt, a, r, C, None, ws,
+                           ws_bytes, None)
+
+
+def test_forward_argument_errors(lib):
+    assert fwd(lib, T=100) == -3                 # T not a multiple of chunk
+    assert fwd(lib, D=48) == -2                  # unsupported head dim
+    assert fwd(lib, C=96) == -2                  # unsupported chunk
+    assert fwd(lib, r=0) == -1
+    assert fwd(lib, r=1000) == -2
+    assert fwd(lib, a=0.0) == -1
+    assert fwd(lib, a=float("nan")) == -1
+    assert fwd(lib, a=float("inf")) == -1
+    assert fwd(lib, B=-1) == -1
+    assert fwd(lib, dt=7) == -1
+    assert fwd(lib, q=None) == -1
+    assert fwd(lib, q=FAKE_MIS) == -7
+    assert fwd(lib, ws_bytes=16) == -4
+    assert fwd(lib, B=1000, H=1000) == -2        # more than 65535 heads
+    assert fwd(lib, B=0) == 0                    # nothing to do, no launch
+
+
+def test_decode_argument_errors(lib):
+    def dec(state=FAKE, B=2, H=2, D=128, dt=1, a=0.5, r=20):
+        return lib.gka_decode_step(state, FAKE, FAKE, FAKE, FAKE, FAKE, B, H, D, dt, a, r, None)
+    assert dec(D=96) == -2
+    assert dec(r=0) == -1
+    assert dec(a=-1.0) == -1
+    assert dec(state=None) == -1
+    assert dec(state=FAKE_MIS) == -7
+    assert dec(B=0) == 0
+
+
+def test_binding_raises_without_cuda_tensors():
+    import torch
+    from test_ridge_regression_b200 import gka
+    x = torch.zeros(1, 1, 64, 32)
+    with pytest.raises(ValueError):
+        gka.gka_forward(x, x, x, torch.ones(1, 1, 64), 0.5, 4, 64)

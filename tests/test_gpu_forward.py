@@ -1,0 +1,177 @@
+"""GPU parity of gka_forward (through the C ABI) against the float64 oracle on
+the same seeded inputs.
+
+Metric: max over (batch, head) of the relative Frobenius error of o over the
+head's [T, D] slab; bars 1e-4 (fp32 inputs) and 2e-2 (bf16 inputs, fp32
+accumulation).  Intermediate results (chunk-start states, per-token norms) are
+read back from the workspace and compared too.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import TOL, cuda, f64, head_rel_err
+from test_ridge_regression_b200 import build, gka
+from test_ridge_regression_b200.inputs import WORKLOADS, make_inputs, workload_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    build.build()
+
+
+def run_forward(q, k, v, beta, a, r, C):
+    B, H, T, D = q.shape
+    qd, kd, vd, bd = cuda(q, k, v, beta)
+    ws = gka.alloc_workspace(B, H, T, D, C, q.dtype)
+    fs = torch.full((B, H, 2, D, D), float("nan"), device="cuda")
+    o = gka.gka_forward(qd, kd, vd, bd, a, r, C, final_state=fs, workspace=ws)
+    assert gka.device_status() == 0
+    return o, fs, ws
+
+
+def ws_views(ws, B, H, T, D, C, dtype):
+    L = gka.workspace_layout(B, H, T, D, C, dtype)
+    N = T // C
+    states = ws[L.states_offset:L.states_offset + 4 * B * H * (N + 1) * 2 * D * D]
+    states = states.view(torch.float32).view(B, H, N + 1, 2, D, D)
+    norms = ws[L.norms_offset:L.norms_offset + 4 * B * H * T].view(torch.float32).view(B, H, T)
+    return states, norms
+
+
+def check_against_oracle(q, k, v, beta, a, r, C, *, check_ws=True):
+    B, H, T, D = q.shape
+    o, fs, ws = run_forward(q, k, v, beta, a, r, C)
+    ref = oracle.forward(q, k, v, beta, a, r, want_norms=True, want_final_state=True,
+                         chunk=C, want_chunk_states=True)
+    tol = TOL[q.dtype]
+    err = head_rel_err(o, ref["o"])
+    print(f"o rel err {err:.3e} (bar {tol:g})")
+    assert err <= tol
+    ferr = head_rel_err(fs, ref["final_state"])
+    assert ferr <= 1e-5, ferr
+    if check_ws:
+        states, norms = ws_views(ws, B, H, T, D, C, q.dtype)
+        assert head_rel_err(norms, ref["norms"]) <= 1e-5
+        cs = f64(states[:, :, :T // C])
+        assert np.all(cs[:, :, 0] == 0)
+        if T // C > 1:
+            assert head_rel_err(cs[:, :, 1:], ref["chunk_states"][:, :, 1:], head_dims=3) <= 1e-5
+    return err
+
+
+def test_tiny_fp32_workload():
+    w = WORKLOADS["tiny_fp32_b1h2t256d32"]
+    q, k, v, beta = workload_inputs(w)
+    check_against_oracle(q, k, v, beta, w.a, w.r, w.chunk)
+
+
+@pytest.mark.parametrize("D", [32, 64, 128])
+@pytest.mark.parametrize("C", [16, 32, 64, 128])
+def test_fp32_dims_and_chunks(D, C):
+    q, k, v, beta = make_inputs(1, 2, 256, D, torch.float32, 2.0, 1.0, seed=100 + D + C)
+    check_against_oracle(q, k, v, beta, 0.5, 8, C)
+
+
+@pytest.mark.parametrize("name", ["bf16_b8h8t2048d128", "bf16_b4h16t8192d128_a0.1",
+                                  "bf16_b1h8t131072d128"])
+def test_bf16_workload_distributions_small(name):
+    # the workload's dtype, a, r, chunk and beta distribution at B=1, H=2, T=4 chunks + more
+    w = WORKLOADS[name]
+    q, k, v, beta = workload_inputs(w, B=1, H=2, T=6 * w.chunk)
+    check_against_oracle(q, k, v, beta, w.a, w.r, w.chunk)
+
+
+def test_beta_zero_resets():
+    q, k, v, beta = make_inputs(1, 2, 256, 64, torch.float32, 1.0, 1.0, seed=7)
+    beta[0, 0, 64] = 0.0      # first token of a chunk
+    beta[0, 0, 100] = 0.0     # inside a chunk
+    beta[0, 1, 0] = 0.0       # very first token
+    beta[0, 1, 130:140] = 0.0 # a run of resets
+    check_against_oracle(q, k, v, beta, 0.5, 10, 64)
+
+
+def test_unnormalised_keys_and_strong_forgetting():
+    g = torch.Generator().manual_seed(3)
+    q = torch.randn(1, 2, 256, 128, generator=g)
+    k = 3.0 * torch.randn(1, 2, 256, 128, generator=g)
+    v = torch.randn(1, 2, 256, 128, generator=g)
+    beta = torch.sigmoid(-1.0 + torch.randn(1, 2, 256, generator=g))
+    check_against_oracle(q, k, v, beta, 0.1, 30, 64)
+
+
+def test_chunk_size_does_not_change_result():
+    q, k, v, beta = make_inputs(2, 2, 512, 128, torch.bfloat16, 3.0, 1.0, seed=11)
+    o64, fs64, _ = run_forward(q, k, v, beta, 0.5, 20, 64)
+    o128, fs128, _ = run_forward(q, k, v, beta, 0.5, 20, 128)
+    assert head_rel_err(o64, o128) <= 1e-2
+    assert head_rel_err(fs64, fs128) <= 1e-5
+
+
+def test_empty_sequence_and_no_heads():
+    D = 64
+    q = torch.zeros(1, 2, 0, D, device="cuda")
+    beta = torch.zeros(1, 2, 0, device="cuda")
+    fs = torch.full((1, 2, 2, D, D), 7.0, device="cuda")
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    o = gka.gka_forward(q, q, q, beta, 0.5, 4, 64, final_state=fs, workspace=ws)
+    torch.cuda.synchronize()
+    assert o.numel() == 0 and torch.all(fs == 0)
+    q0 = torch.zeros(0, 2, 64, D, device="cuda")
+    gka.gka_forward(q0, q0, q0, torch.zeros(0, 2, 64, device="cuda"), 0.5, 4, 64, workspace=ws)
+    assert gka.device_status() == 0
+
+
+def test_error_codes_on_device_tensors():
+    q = torch.zeros(1, 1, 100, 64, device="cuda")
+    beta = torch.ones(1, 1, 100, device="cuda")
+    with pytest.raises(gka.GkaError) as e:
+        gka.gka_forward(q, q, q, beta, 0.5, 4, 64, workspace=torch.empty(1 << 20, dtype=torch.uint8,
+                                                                             device="cuda"))
+    assert e.value.status == -3
+    q = torch.zeros(1, 1, 128, 64, device="cuda")
+    beta = torch.ones(1, 1, 128, device="cuda")
+    with pytest.raises(gka.GkaError) as e:
+        gka.gka_forward(q, q, q, beta, 0.5, 4, 64, workspace=torch.empty(256, dtype=torch.uint8,
+                                                                             device="cuda"))
+    assert e.value.status == -4
+
+
+# ---------------------------------------------------------------------------
+# Full-size workloads in the launch configuration the benchmark times; the
+# oracle checks a sample of heads (heads are independent), over the whole
+# sequence or, for the longest ones, over a window of outputs after running
+# the state recurrence through the whole prefix.
+# ---------------------------------------------------------------------------
+
+def _sampled(name, heads, window):
+    w = WORKLOADS[name]
+    q, k, v, beta = workload_inputs(w)
+    o, fs, _ = run_forward(q, k, v, beta, w.a, w.r, w.chunk)
+    o = o.cpu()
+    worst = 0.0
+    for (b, h) in heads:
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        start = w.T - window if window else 0
+        ref = oracle.forward(q[sl], k[sl], v[sl], beta[sl], w.a, w.r, solve_from=start,
+                             want_final_state=True)
+        err = head_rel_err(o[sl][:, :, start:], ref["o"][:, :, start:])
+        worst = max(worst, err)
+        assert head_rel_err(fs[sl], ref["final_state"]) <= 1e-4
+    print(f"{name}: sampled o rel err {worst:.3e}")
+    assert worst <= TOL[w.dtype]
+
+
+def test_full_b8h8t2048_sampled():
+    _sampled("bf16_b8h8t2048d128", [(0, 0), (7, 7), (3, 5)], window=0)
+
+
+def test_full_b4h16t8192_sampled():
+    _sampled("bf16_b4h16t8192d128_a0.1", [(0, 0), (3, 15)], window=1024)
+
+
+def test_full_b1h8t131072_sampled():
+    _sampled("bf16_b1h8t131072d128", [(0, 3)], window=512)
