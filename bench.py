@@ -42,6 +42,8 @@ def parse():
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--decode-steps", type=int, default=None)
+    p.add_argument("--decode-batch", type=int, default=None,
+                   help="fewer decode sequences (profiling runs); default: the workload's 256")
     return p.parse_args()
 
 
@@ -367,7 +369,10 @@ def main():
 def bench_decode(args, dev, peaks):
     import torch
     from test_ridge_regression_b200 import gka
+    from dataclasses import replace
     from test_ridge_regression_b200.inputs import DECODE as w
+    if args.decode_batch:
+        w = replace(w, batch=args.decode_batch)
     gen = torch.Generator(device=dev)
     gen.manual_seed(w.seed)
 

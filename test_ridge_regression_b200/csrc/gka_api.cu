@@ -5,6 +5,7 @@
 #include <string.h>
 
 #include <atomic>
+#include <map>
 #include <mutex>
 #include <vector>
 
@@ -119,10 +120,24 @@ static int layout(int B, int H, int T, int D, int C, gka_dtype dt, gka_workspace
     return GKA_OK;
 }
 
+// Opts a kernel into `bytes` of dynamic shared memory (beyond the 48 KiB
+// default, which also counts the kernel's static shared memory).  Remembered
+// per (kernel, device) so the attribute call happens once.
+static std::mutex g_smem_mu;
+static std::map<std::pair<const void *, int>, size_t> g_smem_set;
+
 template <typename K>
 static cudaError_t set_smem(K kernel, size_t bytes) {
-    if (bytes <= 48 * 1024) return cudaSuccess;
-    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const auto key = std::make_pair(reinterpret_cast<const void *>(kernel), dev);
+    std::lock_guard<std::mutex> g(g_smem_mu);
+    auto it = g_smem_set.find(key);
+    if (it != g_smem_set.end() && it->second >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) g_smem_set[key] = bytes;
+    return e;
 }
 
 template <typename Tin, int D>
