@@ -34,22 +34,22 @@ k_chunk_delta(const Tin *__restrict__ k, const Tin *__restrict__ v,
     float *Ks = sm;            // [C][D] keys
     float *Kw = Ks + C * D;    // [C][D] w_i k_i
     float *Vw = Kw + C * D;    // [C][D] w_i v_i
-    __shared__ float ell[256];
-    __shared__ float wtot[kSimtThreads / 32];
+    __shared__ double ell[256];
+    __shared__ double wtot[kSimtThreads / 32];
 
     const int n = blockIdx.x, bh = blockIdx.y;
     const size_t tok0 = (size_t)bh * T + (size_t)n * C;
     chunk_log_prefix(beta + tok0, C, ell, wtot);
-    const float lend = ell[C - 1];
+    const double lend = ell[C - 1];
     for (int e = threadIdx.x; e < C * D; e += kSimtThreads) {
         const int i = e / D;
-        const float w = expf(lend - ell[i]);
+        const float w = decay_exp(lend - ell[i]);
         const float kv = load_f(k + tok0 * D + e);
         Ks[e] = kv;
         Kw[e] = w * kv;
         Vw[e] = w * load_f(v + tok0 * D + e);
     }
-    if (threadIdx.x == 0) decay[(size_t)bh * N + n] = expf(lend);
+    if (threadIdx.x == 0) decay[(size_t)bh * N + n] = decay_exp(lend);
     __syncthreads();
 
     constexpr int TS = D / 16;  // TS x TS outputs per thread, 16 x 16 threads
@@ -135,8 +135,9 @@ k_chunk_norm(const Tin *__restrict__ k, const float *__restrict__ beta,
     float *Hs = sm;                 // [D][D]
     float *Ks = Hs + D * D;         // [C][D+1]
     constexpr int KP = D + 1;
-    __shared__ float ell[256], bj[256], betaj[256], ui[256], Xj[256], Ej[256], Gjj[256];
-    __shared__ float wtot[kSimtThreads / 32];
+    __shared__ double ell[256];
+    __shared__ float bj[256], betaj[256], ui[256], Xj[256], Ej[256], Gjj[256];
+    __shared__ double wtot[kSimtThreads / 32];
     __shared__ float upart[256][D / 32 > 0 ? D / 32 : 1];
     __shared__ float hs2_part[kSimtThreads / 32];
 
@@ -153,8 +154,8 @@ k_chunk_norm(const Tin *__restrict__ k, const float *__restrict__ beta,
     }
     for (int e = tid; e < C * D; e += kSimtThreads) Ks[(e / D) * KP + e % D] = load_f(k + tok0 * D + e);
     for (int j = tid; j < C; j += kSimtThreads) {
-        bj[j] = expf(ell[j]);
-        betaj[j] = expf(j == 0 ? ell[0] : ell[j] - ell[j - 1]);
+        bj[j] = decay_exp(ell[j]);
+        betaj[j] = decay_exp(j == 0 ? ell[0] : ell[j] - ell[j - 1]);
     }
     ss = warp_sum(ss);
     if (lane == 0) hs2_part[warp] = ss;
@@ -195,7 +196,7 @@ k_chunk_norm(const Tin *__restrict__ k, const float *__restrict__ beta,
         for (int i = lane; i <= j; i += 32) {
             float dot = 0.f;
             for (int d = 0; d < D; ++d) dot = fmaf(Ks[i * KP + d], Ks[j * KP + d], dot);
-            const float w = expf(ell[j] - ell[i]);
+            const float w = decay_exp(ell[j] - ell[i]);
             xs = fmaf(w, ui[i], xs);
             if (i < j) es = fmaf(w * dot, dot, es);
         }
@@ -257,7 +258,7 @@ k_chunk_solve(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
     float *Qs = Xp + TG * D;           // [TG][D] q
     float *Ps = Qs + TG * D;           // [TG][C] w_{ji} (k_i . x_j)
     float *Ws = Ps + TG * C;           // [TG][C] w_{ji}, 0 for i > j
-    __shared__ float ell[256], wtot[kSimtThreads / 32];
+    __shared__ double ell[256], wtot[kSimtThreads / 32];
     __shared__ float s_b[TG], s_lam[TG], s_invd[TG];
 
     const int tid = threadIdx.x;
@@ -272,14 +273,14 @@ k_chunk_solve(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
     for (int e = tid; e < TG * D; e += kSimtThreads) Qs[e] = load_f(q + (tok0 + j0) * D + e);
     if (tid < TG) {
         const float nj = norms[tok0 + j0 + tid];
-        s_b[tid] = expf(ell[j0 + tid]);
+        s_b[tid] = decay_exp(ell[j0 + tid]);
         s_lam[tid] = P.a * nj;
         s_invd[tid] = nj > 0.f ? 1.f / (P.half_1p2a * nj) : 0.f;
     }
     __syncthreads();
     for (int e = tid; e < TG * C; e += kSimtThreads) {
         const int jj = e / C, i = e % C;
-        Ws[e] = (i <= j0 + jj) ? expf(ell[j0 + jj] - ell[i]) : 0.f;
+        Ws[e] = (i <= j0 + jj) ? decay_exp(ell[j0 + jj] - ell[i]) : 0.f;
     }
     for (int e = tid; e < TG * D; e += kSimtThreads) {
         Xc[e] = Qs[e] * s_invd[e / D];

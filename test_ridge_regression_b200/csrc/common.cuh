@@ -20,8 +20,9 @@ struct ChebParams {
 
 // Lower clamp of log(beta): beta = 0 becomes exp(-150), which underflows to 0
 // in every fp32 product it enters, and keeps differences of cumulative logs
-// finite (no inf - inf).
-constexpr float kLogBetaMin = -150.f;
+// finite (no inf - inf).  Cumulative logs are summed in double so that the
+// difference of two of them keeps full fp32 precision even after resets.
+constexpr double kLogBetaMin = -150.0;
 
 __device__ __forceinline__ float load_f(const float *p) { return *p; }
 __device__ __forceinline__ float load_f(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
@@ -35,27 +36,30 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
-// Inclusive prefix sum of clamped log(beta) over one chunk of C <= 256 tokens,
-// into ell[0..C-1].  Every thread of the block must call it; blockDim.x >= C.
-// wtot: shared scratch of blockDim.x / 32 floats.
-__device__ __forceinline__ void chunk_log_prefix(const float *beta, int C, float *ell,
-                                                 float *wtot) {
+// Inclusive prefix sum, in double, of clamped log(beta) over one chunk of
+// C <= 256 tokens, into ell[0..C-1].  Every thread of the block must call it;
+// blockDim.x >= C.  wtot: shared scratch of blockDim.x / 32 doubles.
+__device__ __forceinline__ void chunk_log_prefix(const float *beta, int C, double *ell,
+                                                 double *wtot) {
     const int t = threadIdx.x, lane = t & 31, w = t >> 5;
-    float x = 0.f;
-    if (t < C) x = fmaxf(logf(beta[t]), kLogBetaMin);
+    double x = 0.0;
+    if (t < C) x = fmax(log((double)beta[t]), kLogBetaMin);
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        float y = __shfl_up_sync(0xffffffffu, x, o);
+        double y = __shfl_up_sync(0xffffffffu, x, o);
         if (lane >= o) x += y;
     }
     if (lane == 31) wtot[w] = x;  // lanes past C carry the last valid prefix
     __syncthreads();
     if (t < C) {
-        float add = 0.f;
+        double add = 0.0;
         for (int i = 0; i < w; ++i) add += wtot[i];
         ell[t] = x + add;
     }
     __syncthreads();
 }
+
+// exp of a (non-positive) difference of cumulative logs, evaluated in fp32.
+__device__ __forceinline__ float decay_exp(double d) { return expf((float)d); }
 
 }  // namespace gka
