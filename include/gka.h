@@ -50,7 +50,8 @@ typedef enum {
     GKA_ERR_WORKSPACE_TOO_SMALL = -4,
     GKA_ERR_CUDA = -5,                   /* a CUDA call failed; see gka_last_cuda_error() */
     GKA_ERR_DEVICE_TIMEOUT = -6,         /* a bounded device-side wait gave up */
-    GKA_ERR_MISALIGNED = -7              /* a pointer is not 16-byte aligned */
+    GKA_ERR_MISALIGNED = -7,             /* a pointer is not 16-byte aligned */
+    GKA_ERR_EXCEEDS_STATIC_SCRATCH = -8  /* gka_forward_static_scratch: problem too large */
 } gka_status;
 
 /* Byte offsets of the regions of the gka_forward workspace (diagnostics and
@@ -99,6 +100,39 @@ int gka_forward_workspace_layout(int B, int H, int T, int D, int chunk, gka_dtyp
 int gka_forward(const void *q, const void *k, const void *v, const float *beta, void *o,
                 int B, int H, int T, int D, gka_dtype dt, float a, int r, int chunk,
                 float *final_state, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * gka_forward without a caller-provided workspace.  There is no counterpart
+ * of this call in the paper: it exists for callers that cannot allocate
+ * device memory themselves, for example a plugin or extension run inside a
+ * host application that owns every device allocation and hands it only its
+ * input and output buffers, or a latency-critical caller that cannot accept
+ * the implicit device synchronisation of cudaMalloc/cudaFree.
+ *
+ * The scratch comes from one device array of GKA_STATIC_SCRATCH_BYTES
+ * (64 MiB) inside the library; every GPU that loads the library holds it
+ * until the process exits.  This call allocates nothing: no cudaMalloc, no
+ * cudaFree, no allocating library routine.  Arguments, layouts and results
+ * are those of gka_forward; the caller still passes q, k, v, beta, o and the
+ * optional final_state.
+ *   - Problems whose gka_forward_workspace_bytes() exceeds
+ *     GKA_STATIC_SCRATCH_BYTES are rejected with
+ *     GKA_ERR_EXCEEDS_STATIC_SCRATCH before anything is launched.
+ *   - The first call on a device looks up the array's device address and
+ *     sets the kernels' shared-memory attributes for that device; make that
+ *     first call before any stream capture.
+ *   - All calls share the one array, and it keeps the contents of the last
+ *     call.  Nothing in it has to start at zero (every region is written
+ *     before it is read), so no clearing is needed.  Calls whose execution
+ *     overlaps on the GPU (on different streams, or from several host
+ *     threads) race on the array and corrupt each other's results: serialise
+ *     them on one stream.
+ */
+#define GKA_STATIC_SCRATCH_BYTES ((size_t)64 << 20)
+
+int gka_forward_static_scratch(const void *q, const void *k, const void *v, const float *beta,
+                               void *o, int B, int H, int T, int D, gka_dtype dt, float a, int r,
+                               int chunk, float *final_state, void *stream);
 
 /*
  * One recurrent decode step for B*H heads (ai.info page, Key Contributions 4:

@@ -224,6 +224,36 @@ static int decode_dispatch(float *state, const void *q, const void *k, const voi
     }
 }
 
+// ---------------------------------------------------------------------------
+// Library-owned scratch for gka_forward_static_scratch().  A file-scope
+// device array: every GPU that loads this library holds it until the process
+// exits.  Host code must not use the symbol itself as an address (in host code
+// it names a host-side stand-in); it takes the device address from
+// cudaGetSymbolAddress once per device and passes that to the kernels.
+// ---------------------------------------------------------------------------
+constexpr size_t kStaticScratchBytes = GKA_STATIC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 256;
+static std::mutex g_scratch_mu;
+static void *g_scratch_addr[kMaxDevices];
+
+static int static_scratch_address(void **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= kMaxDevices) return GKA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> g(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_static_scratch);
+        if (e != cudaSuccess) return cuda_fail(e);
+        g_scratch_addr[dev] = p;
+    }
+    *out = g_scratch_addr[dev];
+    return GKA_OK;
+}
+
 }  // namespace gka
 
 using namespace gka;
@@ -270,6 +300,18 @@ int gka_forward(const void *q, const void *k, const void *v, const float *beta, 
         return forward_dispatch<__nv_bfloat16>(q, k, v, beta, o, B, H, T, D, chunk, P,
                                                final_state, ws, L, s);
     return forward_dispatch<float>(q, k, v, beta, o, B, H, T, D, chunk, P, final_state, ws, L, s);
+}
+
+int gka_forward_static_scratch(const void *q, const void *k, const void *v, const float *beta,
+                               void *o, int B, int H, int T, int D, gka_dtype dt, float a, int r,
+                               int chunk, float *final_state, void *stream) {
+    gka_workspace_layout L;
+    if (int rc = layout(B, H, T, D, chunk, dt, &L)) return rc;
+    if (L.total_bytes > kStaticScratchBytes) return GKA_ERR_EXCEEDS_STATIC_SCRATCH;
+    void *scratch = nullptr;
+    if (int rc = static_scratch_address(&scratch)) return rc;
+    return gka_forward(q, k, v, beta, o, B, H, T, D, dt, a, r, chunk, final_state, scratch,
+                       kStaticScratchBytes, stream);
 }
 
 int gka_decode_step(float *state, const void *q, const void *k, const void *v, const float *beta,
@@ -320,6 +362,8 @@ const char *gka_status_string(int status) {
         case GKA_ERR_CUDA: return "CUDA error";
         case GKA_ERR_DEVICE_TIMEOUT: return "a bounded device wait timed out";
         case GKA_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+        case GKA_ERR_EXCEEDS_STATIC_SCRATCH:
+            return "problem needs more scratch than the library's static array holds";
         default: return "unknown status";
     }
 }

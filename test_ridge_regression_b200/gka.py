@@ -58,6 +58,9 @@ def _lib():
         lib.gka_forward_workspace_layout.restype = i
         lib.gka_forward.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, vp, sz, vp]
         lib.gka_forward.restype = i
+        lib.gka_forward_static_scratch.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i,
+                                                   vp, vp]
+        lib.gka_forward_static_scratch.restype = i
         lib.gka_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
         lib.gka_decode_step.restype = i
         lib.gka_device_status.argtypes = [vp]
@@ -146,6 +149,27 @@ def gka_forward(q, k, v, beta, a: float, r: int, chunk: int, *, o=None, final_st
                             float(a), int(r), int(chunk), _ptr(final_state), _ptr(workspace),
                             workspace.numel() * workspace.element_size(), _stream(stream))
     _check("gka_forward", rc)
+    return o
+
+
+def gka_forward_static_scratch(q, k, v, beta, a: float, r: int, chunk: int, *, o=None,
+                               final_state=None, stream=None):
+    """gka_forward whose scratch is the library's own static device array
+    (for callers that cannot allocate device memory; see include/gka.h).
+    Calls that overlap on the GPU race on that array."""
+    _dev(q, k, v, beta, o, final_state)
+    B, H, T, D = q.shape
+    if k.shape != q.shape or v.shape != q.shape or beta.shape != (B, H, T):
+        raise ValueError("shape mismatch")
+    dt = _dtype(q)
+    if k.dtype != q.dtype or v.dtype != q.dtype or beta.dtype != torch.float32:
+        raise TypeError("q, k, v must share a dtype; beta must be float32")
+    if o is None:
+        o = torch.empty_like(v)
+    rc = _lib().gka_forward_static_scratch(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(o), B, H,
+                                           T, D, dt, float(a), int(r), int(chunk),
+                                           _ptr(final_state), _stream(stream))
+    _check("gka_forward_static_scratch", rc)
     return o
 
 

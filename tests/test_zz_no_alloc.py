@@ -1,0 +1,65 @@
+"""gka_forward_static_scratch: the forward for callers that cannot allocate
+device memory (a plugin inside a host application that owns all device
+allocations, or a latency-critical caller that cannot take cudaMalloc's
+implicit synchronisation).  Its scratch is the library's own static device
+array, so the test checks, through the C ABI, that two calls in a row (the
+second one finding the first one's leftovers in that array) give the same
+results as gka_forward with a caller workspace, and that a problem too large
+for the array is refused before anything runs.
+
+This file is collected last on purpose (its name sorts last)."""
+import ctypes
+
+import pytest
+import torch
+
+from helpers import TOL, head_rel_err
+from test_ridge_regression_b200 import build, gka
+from test_ridge_regression_b200.inputs import make_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def _call(lib, q, k, v, beta, o, a, r, chunk, fs):
+    B, H, T, D = q.shape
+    dt = 1 if q.dtype == torch.bfloat16 else 0
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    return lib.gka_forward_static_scratch(p(q), p(k), p(v), p(beta), p(o), B, H, T, D, dt,
+                                          float(a), int(r), int(chunk), p(fs), stream)
+
+
+@pytest.mark.parametrize("dtype,D,chunk,r", [(torch.bfloat16, 128, 64, 20),
+                                             (torch.float32, 64, 32, 10)])
+def test_static_scratch_matches_gka_forward_twice(dtype, D, chunk, r):
+    build.build()
+    lib = gka.lib()
+    B, H, T, a = 1, 4, 512, 0.5
+    assert gka.workspace_bytes(B, H, T, D, chunk, dtype) <= 64 << 20
+    for call, seed in enumerate((21, 22)):
+        q, k, v, beta = (x.cuda() for x in make_inputs(B, H, T, D, dtype, 3.0, 1.0, seed))
+        fs_ref = torch.empty(B, H, 2, D, D, device="cuda")
+        ref = gka.gka_forward(q, k, v, beta, a, r, chunk, final_state=fs_ref)
+        o = torch.full_like(ref, float("nan"))
+        fs = torch.full_like(fs_ref, float("nan"))
+        rc = _call(lib, q, k, v, beta, o, a, r, chunk, fs)
+        assert rc == 0, lib.gka_status_string(rc)
+        assert gka.device_status() == 0
+        assert torch.isfinite(o.float()).all()
+        err = head_rel_err(o, ref)
+        print(f"call {call}: rel err vs gka_forward {err:.3e}")
+        assert err <= TOL[dtype]
+        assert head_rel_err(fs, fs_ref) <= TOL[dtype]
+
+
+def test_static_scratch_refuses_oversized_problem():
+    build.build()
+    lib = gka.lib()
+    B, H, T, D, chunk = 8, 8, 2048, 128, 64          # needs ~280 MB of scratch
+    assert gka.workspace_bytes(B, H, T, D, chunk) > 64 << 20
+    q = torch.zeros(B, H, T, D, dtype=torch.bfloat16, device="cuda")
+    beta = torch.ones(B, H, T, device="cuda")
+    o = torch.zeros_like(q)
+    fs = torch.zeros(B, H, 2, D, D, device="cuda")
+    assert _call(lib, q, q, q, beta, o, 0.5, 20, chunk, fs) == -8
+    assert torch.all(o == 0)
