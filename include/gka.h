@@ -29,7 +29,10 @@
  *     GKA_ERR_CUDA, which reports a failed launch (the CUDA error code is
  *     kept for gka_last_cuda_error()).
  *   - Supported: D in {32, 64, 128}; chunk in {16, 32, 64, 128}; 1 <= r <= 256;
- *     a > 0 and finite.
+ *     a > 0 and finite.  bf16 with D = 128 and chunk 64 or 128 runs the
+ *     Chebyshev solve and readout on the tensor cores (tcgen05, TMEM
+ *     accumulators, TMA-fed bf16 operands, fp32 accumulation and fp32
+ *     Chebyshev updates); every other case runs them on CUDA cores in fp32.
  */
 #ifndef GKA_H
 #define GKA_H
@@ -63,7 +66,8 @@ typedef struct {
     size_t decay_offset;    /* fp32 [B, H, N]: product of beta over chunk n */
     size_t norms_offset;    /* fp32 [B, H, T]: ||H_t||_F */
     size_t states_bf16_offset; /* bf16 [B, H, N, 2, D, D] copy of the chunk-start states
-                                  (tensor-core path only; 0 bytes otherwise) */
+                                  (tensor-core path only; 0 bytes otherwise); the region
+                                  ends at total_bytes */
     size_t total_bytes;
 } gka_workspace_layout;
 
@@ -169,6 +173,7 @@ enum {
     GKA_KERNEL_CHUNK_NORM = 2,    /* per-token ||H_t||_F */
     GKA_KERNEL_CHUNK_SOLVE = 3,   /* Chebyshev solve + readout */
     GKA_KERNEL_DECODE_STEP = 4,   /* recurrent decode step */
+    GKA_KERNEL_CHUNK_SOLVE_TC = 5,/* Chebyshev solve + readout on tensor cores (tcgen05) */
     GKA_KERNEL_COUNT = 8
 };
 

@@ -86,15 +86,18 @@ k_chunk_delta(const Tin *__restrict__ k, const Tin *__restrict__ v,
 // ---------------------------------------------------------------------------
 // Step 1b: the sequential part.  Per state element e (of [2, D, D]):
 //   S_0 = 0,  S_{n+1} = b^{(n)} S_n + dS_n   (in place over slots 1..N)
-// grid (ceil(2*D*D/256), B*H), block 256.  Optionally copies S_N out.
+// grid (ceil(2*D*D/256), B*H), block 256.  Optionally copies S_N out and
+// writes a bf16 copy of every chunk-start state S_n, n < N (tensor-core operands).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
 k_state_scan(float *__restrict__ states, const float *__restrict__ decay,
-             float *__restrict__ final_state, int N, int DD2) {
+             float *__restrict__ final_state, __nv_bfloat16 *__restrict__ states_bf16, int N,
+             int DD2) {
     const int bh = blockIdx.y;
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
     if (e >= DD2) return;
     float *base = states + (size_t)bh * (N + 1) * DD2 + e;
+    __nv_bfloat16 *bbase = states_bf16 ? states_bf16 + (size_t)bh * N * DD2 + e : nullptr;
     const float *dec = decay + (size_t)bh * N;
     float s = 0.f;
     base[0] = 0.f;
@@ -105,11 +108,13 @@ k_state_scan(float *__restrict__ states, const float *__restrict__ decay,
         for (int u = 0; u < 8; ++u) dl[u] = base[(size_t)(n + u + 1) * DD2];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
+            if (bbase) bbase[(size_t)(n + u) * DD2] = __float2bfloat16_rn(s);
             s = fmaf(dec[n + u], s, dl[u]);
             base[(size_t)(n + u + 1) * DD2] = s;
         }
     }
     for (; n < N; ++n) {
+        if (bbase) bbase[(size_t)n * DD2] = __float2bfloat16_rn(s);
         s = fmaf(dec[n], s, base[(size_t)(n + 1) * DD2]);
         base[(size_t)(n + 1) * DD2] = s;
     }

@@ -5,14 +5,18 @@
 #include <string.h>
 
 #include <atomic>
+#include <type_traits>
 #include <map>
 #include <mutex>
 #include <vector>
 
 #include "../../include/gka.h"
+#include <cudaTypedefs.h>
+
 #include "chunk_simt.cuh"
 #include "common.cuh"
 #include "decode.cuh"
+#include "solve_tc.cuh"
 
 namespace gka {
 
@@ -84,6 +88,12 @@ static size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
 static bool supported_d(int D) { return D == 32 || D == 64 || D == 128; }
 static bool supported_c(int C) { return C == 16 || C == 32 || C == 64 || C == 128; }
 
+// bf16 inputs, head dimension 128 and chunks of 64 or 128 tokens run the
+// tensor-core solve; everything else the CUDA-core one.
+static bool tensor_core_path(int D, int C, gka_dtype dt) {
+    return dt == GKA_BF16 && D == 128 && (C == 64 || C == 128);
+}
+
 // Chebyshev constants of one call (pith.science appendix, Lemma 3: omega_0 = 2,
 // omega_i = 1/(1 - rho^2 omega_{i-1}/4)); computed in double, stored in float.
 static ChebParams make_cheb(float a, int r) {
@@ -116,6 +126,7 @@ static int layout(int B, int H, int T, int D, int C, gka_dtype dt, gka_workspace
     L->norms_offset = off;
     off = round256(off + sizeof(float) * BH * (size_t)T);
     L->states_bf16_offset = off;
+    if (tensor_core_path(D, C, dt)) off = round256(off + 2 * BH * N * 2 * (size_t)D * D);
     L->total_bytes = off;
     return GKA_OK;
 }
@@ -159,7 +170,8 @@ static int forward_simt(const Tin *q, const Tin *k, const Tin *v, const float *b
 
     const int DD2 = 2 * D * D;
     { ProfScope ps(GKA_KERNEL_STATE_SCAN, s);
-    k_state_scan<<<dim3((DD2 + 255) / 256, BH), 256, 0, s>>>(states, decay, final_state, N, DD2); }
+    k_state_scan<<<dim3((DD2 + 255) / 256, BH), 256, 0, s>>>(states, decay, final_state, nullptr,
+                                                             N, DD2); }
     if (int rc = check_launch()) return rc;
 
     const size_t sm_norm = sizeof(float) * ((size_t)D * D + (size_t)C * (D + 1));
@@ -177,6 +189,91 @@ static int forward_simt(const Tin *q, const Tin *k, const Tin *v, const float *b
     return check_launch();
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }();
+    return fn;
+}
+
+// 2-D map over a row-major [rows][128] bf16 array: boxes of 64 columns
+// (128 bytes) x 64 rows, 128-byte swizzle (the tensor-core operand layout).
+static int bf16_rows_map(CUtensorMap *m, const void *base, uint64_t rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return cuda_fail(cudaErrorNotSupported);
+    cuuint64_t dims[2] = {128, rows};
+    cuuint64_t strides[1] = {128 * 2};
+    cuuint32_t box[2] = {64, 64};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
+                     strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? GKA_OK : cuda_fail(cudaErrorInvalidValue);
+}
+
+static int timeout_flag_ptr(int **ptr);
+
+static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
+                      const float *beta, __nv_bfloat16 *o, int B, int H, int T, int C,
+                      const ChebParams &P, float *final_state, char *ws,
+                      const gka_workspace_layout &L, cudaStream_t s) {
+    constexpr int D = 128;
+    const int BH = B * H, N = T / C;
+    float *states = reinterpret_cast<float *>(ws + L.states_offset);
+    float *decay = reinterpret_cast<float *>(ws + L.decay_offset);
+    float *norms = reinterpret_cast<float *>(ws + L.norms_offset);
+    __nv_bfloat16 *sbf = reinterpret_cast<__nv_bfloat16 *>(ws + L.states_bf16_offset);
+    int *flag = nullptr;
+    if (int rc = timeout_flag_ptr(&flag)) return rc;
+    TcMaps maps;
+    if (int rc = bf16_rows_map(&maps.k, k, (uint64_t)BH * T)) return rc;
+    if (int rc = bf16_rows_map(&maps.v, v, (uint64_t)BH * T)) return rc;
+    if (int rc = bf16_rows_map(&maps.state, sbf, (uint64_t)BH * N * 2 * D)) return rc;
+    cudaError_t e;
+
+    const size_t sm_delta = sizeof(float) * 3 * (size_t)C * D;
+    if ((e = set_smem(k_chunk_delta<__nv_bfloat16, D>, sm_delta)) != cudaSuccess) return cuda_fail(e);
+    { ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
+    k_chunk_delta<__nv_bfloat16, D><<<dim3(N, BH), kSimtThreads, sm_delta, s>>>(k, v, beta, states,
+                                                                                decay, T, N, C); }
+    if (int rc = check_launch()) return rc;
+
+    const int DD2 = 2 * D * D;
+    { ProfScope ps(GKA_KERNEL_STATE_SCAN, s);
+    k_state_scan<<<dim3((DD2 + 255) / 256, BH), 256, 0, s>>>(states, decay, final_state, sbf, N,
+                                                             DD2); }
+    if (int rc = check_launch()) return rc;
+
+    const size_t sm_norm = sizeof(float) * ((size_t)D * D + (size_t)C * (D + 1));
+    if ((e = set_smem(k_chunk_norm<__nv_bfloat16, D>, sm_norm)) != cudaSuccess) return cuda_fail(e);
+    { ProfScope ps(GKA_KERNEL_CHUNK_NORM, s);
+    k_chunk_norm<__nv_bfloat16, D><<<dim3(N, BH), kSimtThreads, sm_norm, s>>>(k, beta, states,
+                                                                              norms, T, N, C); }
+    if (int rc = check_launch()) return rc;
+
+    if ((e = set_smem(k_chunk_solve_tc<64>, TcSmem<64>::bytes)) != cudaSuccess) return cuda_fail(e);
+    { ProfScope ps(GKA_KERNEL_CHUNK_SOLVE_TC, s);
+    k_chunk_solve_tc<64><<<dim3(N, BH), kTcThreads, TcSmem<64>::bytes, s>>>(
+        maps, q, beta, norms, o, T, N, C, 0, P, flag); }
+    if (int rc = check_launch()) return rc;
+    if (C == 128) {
+        if ((e = set_smem(k_chunk_solve_tc<128>, TcSmem<128>::bytes)) != cudaSuccess)
+            return cuda_fail(e);
+        { ProfScope ps(GKA_KERNEL_CHUNK_SOLVE_TC, s);
+        k_chunk_solve_tc<128><<<dim3(N, BH), kTcThreads, TcSmem<128>::bytes, s>>>(
+            maps, q, beta, norms, o, T, N, C, 1, P, flag); }
+        if (int rc = check_launch()) return rc;
+    }
+    return GKA_OK;
+}
+
 template <typename Tin>
 static int forward_dispatch(const void *q, const void *k, const void *v, const float *beta,
                             void *o, int B, int H, int T, int D, int C, const ChebParams &P,
@@ -186,6 +283,10 @@ static int forward_dispatch(const void *q, const void *k, const void *v, const f
     auto K = static_cast<const Tin *>(k);
     auto V = static_cast<const Tin *>(v);
     auto O = static_cast<Tin *>(o);
+    if constexpr (std::is_same<Tin, __nv_bfloat16>::value) {
+        if (tensor_core_path(D, C, GKA_BF16))
+            return forward_tc(Q, K, V, beta, O, B, H, T, C, P, final_state, ws, L, s);
+    }
     switch (D) {
         case 32: return forward_simt<Tin, 32>(Q, K, V, beta, O, B, H, T, C, P, final_state, ws, L, s);
         case 64: return forward_simt<Tin, 64>(Q, K, V, beta, O, B, H, T, C, P, final_state, ws, L, s);

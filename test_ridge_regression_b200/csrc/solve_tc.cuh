@@ -1,0 +1,336 @@
+// Tensor-core (tcgen05 + TMEM + TMA) Chebyshev solve and readout of the
+// chunk-wise GKA forward, bf16 inputs, head dimension 128.
+//
+// Method: "Gated KalmaNet" (arXiv 2511.21016), ai.info page, Key
+// Contributions 2-3 and Methodology: the Chebyshev iteration needs only
+// products with H_t, and inside a chunk H_t x = b_t H_s x + sum_{i<=t}
+// w_{ti} (k_i . x) k_i, so every iteration of all tokens of a chunk is three
+// small GEMMs against the chunk-start state and the chunk's keys.
+//
+// One CTA (4 warps) solves one group of 64 tokens of one chunk; it needs the
+// chunk's first MG = 64 (group + 1) keys (later keys are masked for these
+// tokens).  Work is kept transposed so that every accumulator has M = 128
+// rows = the head dimension, one TMEM lane per thread:
+//   S^T = K X^T           (M = MG keys, N = 64 tokens, K = 128)      -> TMEM S
+//   Z1  = H_s X^T         (M = 128,     N = 64,        K = 128)      -> TMEM Z1
+//   P^T = W o S^T         (registers -> bf16 in shared memory, W_{ij} = w_{ji})
+//   Z3  = K^T P^T         (M = 128,     N = 64,        K = MG)       -> TMEM Z3
+//   y_j = b_j Z1[:,j] + Z3[:,j] + lambda_j x_j; three-term Chebyshev update in
+//   fp32 registers (thread d owns element d of all 64 iterates); the new
+//   iterate goes back to shared memory as bf16 (MN-major, 128B-swizzled) as
+//   the B operand of the next round.
+// The readout is the same three GEMMs with M_s in place of H_s and V in
+// place of K for the final product: o_j = b_j M_s x_j + sum_i w_{ji} (k_i.x_j) v_i.
+// H_s, K, V (bf16) arrive by TMA and stay in shared memory for all r rounds.
+#pragma once
+
+#include "common.cuh"
+#include "ptx.cuh"
+#include "tcgen05.cuh"
+
+namespace gka {
+
+constexpr int kTcThreads = 128;
+constexpr int kTcTokens = 64;     // tokens per CTA
+constexpr int kTcD = 128;         // head dimension of the tensor-core path
+constexpr uint32_t kTcWaitProbes = 1u << 22;
+
+template <int MG>
+struct TcSmem {
+    // byte offsets from a 1024-aligned base
+    static constexpr uint32_t HM = 0;                        // H_s, later M_s: 2 x [128][64] bf16
+    static constexpr uint32_t KT = HM + 32768;               // keys:   2 x [MG][64] bf16
+    static constexpr uint32_t VT = KT + MG * 256;            // values: 2 x [MG][64] bf16
+    static constexpr uint32_t XT = VT + MG * 256;            // X^T: [128][64] bf16, MN-major
+    static constexpr uint32_t PT = XT + 16384;               // P^T: [MG][64] bf16, MN-major
+    static constexpr uint32_t QS = PT + MG * 128;            // q: [64][128] bf16 row-major
+    static constexpr uint32_t SCAL = QS + 16384;             // per-token scalars
+    static constexpr uint32_t ELL = SCAL + 4 * 4 * kTcTokens; // double[MG] cumulative logs
+    static constexpr uint32_t BARS = ELL + 8 * MG + 8 * (kTcThreads / 32);
+    static constexpr uint32_t TBASE = BARS + 8 * 8;
+    static constexpr uint32_t END = TBASE + 16;
+    static constexpr size_t bytes = END + 1024;               // + alignment slack
+};
+
+struct TcMaps {
+    CUtensorMap k;       // [B*H*T rows][128] bf16, box 64 x 64, 128B swizzle
+    CUtensorMap v;       // same for v
+    CUtensorMap state;   // [B*H*N*2*128 rows][128] bf16 chunk-start states, box 64 x 64
+};
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+                 "r"(d)
+                 : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&p);
+}
+
+// Writes 16 consecutive values (columns c0..c0+15, c0 % 16 == 0) of `row` of a
+// 128B-swizzled [rows][64] bf16 tile as two 16-byte chunks.
+__device__ __forceinline__ void st_row16(uint32_t tile, uint32_t row, uint32_t c0, const float *v) {
+    const uint32_t base = tile + row * 128u;
+    const uint32_t ch0 = ((c0 >> 3) ^ row) & 7u, ch1 = ((c0 >> 3) + 1u ^ row) & 7u;
+    st_shared_v4(base + ch0 * 16u, pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
+                 pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+    st_shared_v4(base + ch1 * 16u, pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]),
+                 pack_bf16(v[12], v[13]), pack_bf16(v[14], v[15]));
+}
+
+// grid (N, B*H); group g = `group` of every chunk; MG = 64 * (group + 1).
+template <int MG>
+__global__ void __launch_bounds__(kTcThreads, 2)
+k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__restrict__ q,
+                 const float *__restrict__ beta, const float *__restrict__ norms,
+                 __nv_bfloat16 *__restrict__ o, int T, int N, int C, int group, const ChebParams P,
+                 int *__restrict__ timeout_flag) {
+    using L = TcSmem<MG>;
+    extern __shared__ uint8_t smraw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+    const uint32_t sb = smem_u32(sm);
+    float *s_bi = reinterpret_cast<float *>(sm + L::SCAL);   // b_j / d_j
+    float *s_invd = s_bi + kTcTokens;                        // 1 / d_j (0 if ||H|| = 0)
+    float *s_li = s_invd + kTcTokens;                        // lambda_j / d_j
+    float *s_b = s_li + kTcTokens;                           // b_j
+    double *ell = reinterpret_cast<double *>(sm + L::ELL);
+    double *wtot = ell + MG;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BARS);
+    uint64_t *bar_load = &bars[0], *bar_v = &bars[1], *bar_m = &bars[2], *bar_s = &bars[3],
+             *bar_z = &bars[4], *bar_fin = &bars[5];
+    uint32_t *tbase = reinterpret_cast<uint32_t *>(sm + L::TBASE);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n = blockIdx.x, bh = blockIdx.y;
+    const int j0 = group * kTcTokens;                      // first token of the group in the chunk
+    const size_t tok0 = (size_t)bh * T + (size_t)n * C;    // first token of the chunk
+    const int srow = (int)(((size_t)bh * N + n) * 2 * kTcD);   // H_s row in the state map
+
+    if (tid == 0) {
+        for (int i = 0; i < 6; ++i) mbar_init(&bars[i], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid == 0) {
+        mbar_arrive_expect_tx(bar_load, 32768 + MG * 256 + kTcTokens * kTcD * 2);
+        for (int h = 0; h < 2; ++h) {
+            for (int rb = 0; rb < 2; ++rb)
+                tc::tma_load_2d(sm + L::HM + h * 16384 + rb * 8192, &maps.state, h * 64,
+                                srow + rb * 64, bar_load);
+            for (int rb = 0; rb < MG / 64; ++rb)
+                tc::tma_load_2d(sm + L::KT + h * MG * 128 + rb * 8192, &maps.k, h * 64,
+                                (int)tok0 + rb * 64, bar_load);
+        }
+        bulk_g2s(sm + L::QS, q + (tok0 + j0) * kTcD, kTcTokens * kTcD * 2, bar_load);
+        mbar_arrive_expect_tx(bar_v, MG * 256);
+        for (int h = 0; h < 2; ++h)
+            for (int rb = 0; rb < MG / 64; ++rb)
+                tc::tma_load_2d(sm + L::VT + h * MG * 128 + rb * 8192, &maps.v, h * 64,
+                                (int)tok0 + rb * 64, bar_v);
+    }
+    if (warp == 0) {
+        tc::tmem_alloc(tbase, 256);
+        tc::tmem_relinquish();
+    }
+    chunk_log_prefix(beta + tok0, MG, ell, wtot);
+    if (tid < kTcTokens) {
+        const float nj = norms[tok0 + j0 + tid];
+        const float invd = nj > 0.f ? 1.f / (P.half_1p2a * nj) : 0.f;
+        const float b = decay_exp(ell[j0 + tid]);
+        s_b[tid] = b;
+        s_bi[tid] = b * invd;
+        s_invd[tid] = invd;
+        s_li[tid] = P.a * nj * invd;
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tbase;
+    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);   // this warp's TMEM lane quarter
+    const uint32_t T_Z1 = 0, T_Z3 = 64, T_S = 128, T_W = 192;
+
+    // rows of S (keys) held by this thread: M = 64 puts key 16w + l in lane
+    // 32w + l (l < 16); M = 128 puts key t in lane t.
+    const bool s_owner = (MG == 128) || (lane < 16);
+    const int key = (MG == 128) ? tid : warp * 16 + lane;
+
+    // W^T rows: W[i][j] = w_{ji} = exp(l_j - l_i) for i <= j, else 0
+    {
+        float wv[16];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int j = j0 + c * 16 + u;
+                wv[u] = (s_owner && key <= j) ? decay_exp(ell[j] - ell[key]) : 0.f;
+            }
+            tc::tmem_st16(tl + T_W + c * 16, wv);
+        }
+        tc::tmem_wait_st();
+    }
+
+    bool ok = mbar_wait_bounded(bar_load, 0, kTcWaitProbes);
+    const __nv_bfloat16 *qs = reinterpret_cast<const __nv_bfloat16 *>(sm + L::QS);
+
+    // x_1 = q / d, x_0 = 0; thread d keeps element d of all 64 iterates
+    float xc[kTcTokens], xp[kTcTokens];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const int jj = c * 16 + u;
+            xc[jj] = __bfloat162float(qs[jj * kTcD + tid]) * s_invd[jj];
+            xp[jj] = 0.f;
+        }
+        st_row16(sb + L::XT, tid, c * 16, &xc[c * 16]);
+    }
+    fence_proxy_async_smem();
+    tc::fence_before_sync();
+    ok = __syncthreads_and(ok);
+
+    constexpr uint32_t IDESC_S = tc::idesc_bf16(MG, 64, false, true);
+    constexpr uint32_t IDESC_Z1 = tc::idesc_bf16(128, 64, false, true);
+    constexpr uint32_t IDESC_Z3 = tc::idesc_bf16(128, 64, true, true);
+    const uint32_t a_hm = sb + L::HM, a_kt = sb + L::KT, a_vt = sb + L::VT, b_xt = sb + L::XT,
+                   b_pt = sb + L::PT;
+    bool m_requested = false;
+    uint32_t ph = 0;   // phase parity of bar_s / bar_z (both complete once per round)
+
+#pragma unroll 1
+    for (int it = 1; it <= P.r && ok; ++it) {
+        const bool out_pass = (it == P.r);
+        if (tid == 0) {
+            tc::fence_after_sync();
+            // S^T = K X^T
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                tc::mma_bf16(tmem + T_S,
+                             tc::sdesc(a_kt + (kk >> 2) * (MG * 128) + (kk & 3) * 32, 16, 1024),
+                             tc::sdesc(b_xt + kk * 2048, 8192, 1024), IDESC_S, kk > 0);
+            tc::commit(bar_s);
+            if (out_pass) {
+                if (!m_requested) {
+                    mbar_arrive_expect_tx(bar_m, 32768);
+                    for (int h = 0; h < 2; ++h)
+                        for (int rb = 0; rb < 2; ++rb)
+                            tc::tma_load_2d(sm + L::HM + h * 16384 + rb * 8192, &maps.state, h * 64,
+                                            srow + kTcD + rb * 64, bar_m);
+                    m_requested = true;
+                }
+                if (!mbar_wait_bounded(bar_m, 0, kTcWaitProbes)) ok = false;
+            }
+            // Z1 = H_s X^T (M_s X^T on the readout pass)
+            if (ok) {
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_bf16(tmem + T_Z1,
+                                 tc::sdesc(a_hm + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                                 tc::sdesc(b_xt + kk * 2048, 8192, 1024), IDESC_Z1, kk > 0);
+            }
+        }
+        // P^T = W o S^T  -> bf16, MN-major tile of MG rows
+        if (!mbar_wait_bounded(bar_s, ph, kTcWaitProbes)) ok = false;
+        tc::fence_after_sync();
+        if (out_pass && tid == 0 && ok) ok = mbar_wait_bounded(bar_v, 0, kTcWaitProbes);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            float sv[16], wv[16];
+            tc::tmem_ld16(tl + T_S + c * 16, sv);
+            tc::tmem_ld16(tl + T_W + c * 16, wv);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int u = 0; u < 16; ++u) sv[u] *= wv[u];
+            if (s_owner) st_row16(b_pt, key, c * 16, sv);
+        }
+        fence_proxy_async_smem();
+        tc::fence_before_sync();
+        ok = __syncthreads_and(ok);
+        if (!ok) break;
+        if (tid == 0) {
+            tc::fence_after_sync();
+            const uint32_t a3 = out_pass ? a_vt : a_kt;
+#pragma unroll
+            for (int kk = 0; kk < MG / 16; ++kk)
+                tc::mma_bf16(tmem + T_Z3, tc::sdesc(a3 + kk * 2048, MG * 128, 1024),
+                             tc::sdesc(b_pt + kk * 2048, 8192, 1024), IDESC_Z3, kk > 0);
+            tc::commit(bar_z);
+        }
+        if (!mbar_wait_bounded(bar_z, ph, kTcWaitProbes)) ok = false;
+        tc::fence_after_sync();
+        ph ^= 1u;
+        if (!out_pass) {
+            if (tid == 0 && it == P.r - 1) {
+                // H_s is no longer read: fetch M_s for the readout into the same buffer
+                mbar_arrive_expect_tx(bar_m, 32768);
+                for (int h = 0; h < 2; ++h)
+                    for (int rb = 0; rb < 2; ++rb)
+                        tc::tma_load_2d(sm + L::HM + h * 16384 + rb * 8192, &maps.state, h * 64,
+                                        srow + kTcD + rb * 64, bar_m);
+                m_requested = true;
+            }
+            const float w = P.omega[it];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                float z1[16], z3[16];
+                tc::tmem_ld16(tl + T_Z1 + c * 16, z1);
+                tc::tmem_ld16(tl + T_Z3 + c * 16, z3);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int jj = c * 16 + u;
+                    // (q - A x)/d = q/d - (b Z1 + Z3)/d - (lambda/d) x
+                    const float r = __bfloat162float(qs[jj * kTcD + tid]) * s_invd[jj] -
+                                    s_bi[jj] * z1[u] - s_invd[jj] * z3[u] - s_li[jj] * xc[jj];
+                    const float xn = fmaf(w, r + xc[jj] - xp[jj], xp[jj]);
+                    xp[jj] = xc[jj];
+                    xc[jj] = xn;
+                }
+                st_row16(sb + L::XT, tid, c * 16, &xc[c * 16]);
+            }
+            fence_proxy_async_smem();
+            tc::fence_before_sync();
+            ok = __syncthreads_and(ok);
+        } else if (ok) {
+            // o_j[d] = b_j (M_s x_j)[d] + sum_i w_{ji} (k_i . x_j) v_i[d]
+            __nv_bfloat16 *orow = o + (tok0 + j0) * kTcD + tid;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                float z1[16], z3[16];
+                tc::tmem_ld16(tl + T_Z1 + c * 16, z1);
+                tc::tmem_ld16(tl + T_Z3 + c * 16, z3);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int jj = c * 16 + u;
+                    const float val = s_invd[jj] > 0.f ? fmaf(s_b[jj], z1[u], z3[u]) : 0.f;
+                    orow[(size_t)jj * kTcD] = __float2bfloat16_rn(val);
+                }
+            }
+        }
+    }
+
+    // teardown: no MMA or copy of this CTA may be in flight when TMEM is freed
+    ok = __syncthreads_and(ok);
+    if (!ok) {
+        if (tid == 0) {
+            atomicExch(timeout_flag, 1);
+            tc::commit(bar_fin);
+            mbar_wait_bounded(bar_fin, 0, kTcWaitProbes);
+            mbar_wait_bounded(bar_load, 0, kTcWaitProbes);
+            mbar_wait_bounded(bar_v, 0, kTcWaitProbes);
+            if (m_requested) mbar_wait_bounded(bar_m, 0, kTcWaitProbes);
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, 256);
+    }
+}
+
+}  // namespace gka

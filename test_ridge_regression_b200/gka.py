@@ -28,7 +28,8 @@ class GkaError(RuntimeError):
         super().__init__(f"{fn}: {msg} [{status}]")
 
 
-KERNEL_NAMES = ["chunk_delta", "state_scan", "chunk_norm", "chunk_solve", "decode_step"]
+KERNEL_NAMES = ["chunk_delta", "state_scan", "chunk_norm", "chunk_solve", "decode_step",
+                "chunk_solve_tc"]
 
 
 class KernelTimes(ctypes.Structure):

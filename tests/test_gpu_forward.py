@@ -85,6 +85,30 @@ def test_bf16_workload_distributions_small(name):
     check_against_oracle(q, k, v, beta, w.a, w.r, w.chunk)
 
 
+@pytest.mark.parametrize("C", [16, 32])
+def test_bf16_cuda_core_chunks(C):
+    # bf16 with chunks outside {64, 128} runs the CUDA-core solve
+    q, k, v, beta = make_inputs(1, 2, 256, 128, torch.bfloat16, 3.0, 1.0, seed=300 + C)
+    check_against_oracle(q, k, v, beta, 0.5, 20, C)
+
+
+@pytest.mark.parametrize("C", [64, 128])
+@pytest.mark.parametrize("r", [1, 2, 3])
+def test_tensor_core_short_iterations(C, r):
+    # r = 1 (no matrix-vector product), 2 and 3 on the tensor-core path
+    q, k, v, beta = make_inputs(1, 2, 2 * C, 128, torch.bfloat16, 2.0, 1.0, seed=400 + r + C)
+    check_against_oracle(q, k, v, beta, 0.5, r, C)
+
+
+def test_tensor_core_resets_and_strong_forgetting():
+    q, k, v, beta = make_inputs(2, 2, 384, 128, torch.bfloat16, 0.0, 2.0, seed=17)
+    beta[0, 0, 64] = 0.0
+    beta[0, 1, 70:75] = 0.0
+    beta[1, 0, 0] = 0.0
+    check_against_oracle(q, k, v, beta, 0.1, 30, 64)
+    check_against_oracle(q, k, v, beta, 0.1, 30, 128)
+
+
 def test_beta_zero_resets():
     q, k, v, beta = make_inputs(1, 2, 256, 64, torch.float32, 1.0, 1.0, seed=7)
     beta[0, 0, 64] = 0.0      # first token of a chunk
