@@ -31,8 +31,9 @@
  *   - Supported: D in {32, 64, 128}; chunk in {16, 32, 64, 128}; 1 <= r <= 256;
  *     a > 0 and finite.  bf16 with D = 128 and chunk 64 or 128 runs the
  *     Chebyshev solve and readout on the tensor cores (tcgen05, TMEM
- *     accumulators, TMA-fed bf16 operands, fp32 accumulation and fp32
- *     Chebyshev updates); every other case runs them on CUDA cores in fp32.
+ *     accumulators, TMA-fed fp16 operands with power-of-two scales, fp32
+ *     accumulation and fp32 Chebyshev updates); every other case runs them on
+ *     CUDA cores in fp32.
  */
 #ifndef GKA_H
 #define GKA_H
@@ -65,9 +66,10 @@ typedef struct {
                                slot N holds the state after the last token */
     size_t decay_offset;    /* fp32 [B, H, N]: product of beta over chunk n */
     size_t norms_offset;    /* fp32 [B, H, T]: ||H_t||_F */
-    size_t states_bf16_offset; /* bf16 [B, H, N, 2, D, D] copy of the chunk-start states
-                                  (tensor-core path only; 0 bytes otherwise); the region
-                                  ends at total_bytes */
+    size_t states_lp_offset;   /* tensor-core path only (0 bytes otherwise): fp16
+                                  [B, H, N, 2, D, D] copies of the chunk-start states, each
+                                  scaled by a power of two, then the scales; the region ends
+                                  at total_bytes */
     size_t total_bytes;
 } gka_workspace_layout;
 

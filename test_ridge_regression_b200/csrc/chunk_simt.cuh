@@ -13,6 +13,8 @@
 // so H_j x = b_j H_s x + sum_{i<=j} w_{ji} (k_i . x) k_i never needs H_j.
 #pragma once
 
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 
 namespace gka {
@@ -29,7 +31,7 @@ template <typename Tin, int D>
 __global__ void __launch_bounds__(kSimtThreads)
 k_chunk_delta(const Tin *__restrict__ k, const Tin *__restrict__ v,
               const float *__restrict__ beta, float *__restrict__ states,
-              float *__restrict__ decay, int T, int N, int C) {
+              float *__restrict__ decay, float *__restrict__ bound_inc, int T, int N, int C) {
     extern __shared__ __align__(16) float sm[];
     float *Ks = sm;            // [C][D] keys
     float *Kw = Ks + C * D;    // [C][D] w_i k_i
@@ -51,6 +53,37 @@ k_chunk_delta(const Tin *__restrict__ k, const Tin *__restrict__ v,
     }
     if (threadIdx.x == 0) decay[(size_t)bh * N + n] = decay_exp(lend);
     __syncthreads();
+    if (bound_inc) {
+        // sum_i w_i ||k_i k_i^T||_F and sum_i w_i ||v_i k_i^T||_F: the increments of a
+        // bound on ||H_s||_F and ||M_s||_F (triangle inequality) used to scale the
+        // low-precision copies of the states
+        __shared__ float bpart[2][kSimtThreads / 32];
+        float bh2 = 0.f, bm2 = 0.f;
+        const int t = threadIdx.x;
+        if (t < C) {
+            float kw = 0.f, kk = 0.f, vv = 0.f;
+            for (int d0 = 0; d0 < D; ++d0) {
+                const int d = (d0 + t) % D;
+                kw = fmaf(Kw[t * D + d], Ks[t * D + d], kw);
+                kk = fmaf(Ks[t * D + d], Ks[t * D + d], kk);
+                vv = fmaf(Vw[t * D + d], Vw[t * D + d], vv);
+            }
+            bh2 = kw;
+            bm2 = sqrtf(vv) * sqrtf(kk);
+        }
+        bh2 = warp_sum(bh2);
+        bm2 = warp_sum(bm2);
+        if ((t & 31) == 0) {
+            bpart[0][t >> 5] = bh2;
+            bpart[1][t >> 5] = bm2;
+        }
+        __syncthreads();
+        if (t < 2) {
+            float sum = 0.f;
+            for (int w = 0; w < kSimtThreads / 32; ++w) sum += bpart[t][w];
+            bound_inc[((size_t)bh * N + n) * 2 + t] = sum;
+        }
+    }
 
     constexpr int TS = D / 16;  // TS x TS outputs per thread, 16 x 16 threads
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
@@ -87,37 +120,52 @@ k_chunk_delta(const Tin *__restrict__ k, const Tin *__restrict__ v,
 // Step 1b: the sequential part.  Per state element e (of [2, D, D]):
 //   S_0 = 0,  S_{n+1} = b^{(n)} S_n + dS_n   (in place over slots 1..N)
 // grid (ceil(2*D*D/256), B*H), block 256.  Optionally copies S_N out and
-// writes a bf16 copy of every chunk-start state S_n, n < N (tensor-core operands).
+// writes an fp16 copy of every chunk-start state S_n, n < N, scaled by a power
+// of two 2^e_n chosen from the running bound ||S_n||_F <= bound_n (the
+// tensor-core operands; e_n goes to state_exp[bh][n][H or M]).
 // ---------------------------------------------------------------------------
+// Exponent e such that |value| <= bound implies |value * 2^e| <= 2^14.
+__device__ __forceinline__ int lp_exponent(float bound) {
+    if (!(bound > 0.f)) return 0;
+    const int e = 14 - (ilogbf(bound) + 1);
+    return e < -120 ? -120 : (e > 120 ? 120 : e);
+}
+
 __global__ void __launch_bounds__(256)
 k_state_scan(float *__restrict__ states, const float *__restrict__ decay,
-             float *__restrict__ final_state, __nv_bfloat16 *__restrict__ states_bf16, int N,
-             int DD2) {
+             float *__restrict__ final_state, __half *__restrict__ states_lp,
+             const float *__restrict__ bound_inc, int *__restrict__ state_exp, int N, int DD2) {
     const int bh = blockIdx.y;
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
     if (e >= DD2) return;
     float *base = states + (size_t)bh * (N + 1) * DD2 + e;
-    __nv_bfloat16 *bbase = states_bf16 ? states_bf16 + (size_t)bh * N * DD2 + e : nullptr;
+    __half *lbase = states_lp ? states_lp + (size_t)bh * N * DD2 + e : nullptr;
+    const int mat = e < DD2 / 2 ? 0 : 1;          // H or M element
+    const bool writes_exp = (e == 0) || (e == DD2 / 2);
     const float *dec = decay + (size_t)bh * N;
-    float s = 0.f;
+    float s = 0.f, bound = 0.f;
     base[0] = 0.f;
+    // one step of the scan: chunk-start copy, then S_{n+1} = b_n S_n + dS_n
+    auto step = [&](int n, float dl) {
+        if (lbase) {
+            // low-precision copy of the chunk-start state, scaled by 2^e from its norm bound
+            const int ex = lp_exponent(bound);
+            lbase[(size_t)n * DD2] = __float2half_rn(ldexpf(s, ex));
+            if (writes_exp) state_exp[((size_t)bh * N + n) * 2 + mat] = ex;
+            bound = fmaf(dec[n], bound, bound_inc[((size_t)bh * N + n) * 2 + mat]);
+        }
+        s = fmaf(dec[n], s, dl);
+        base[(size_t)(n + 1) * DD2] = s;
+    };
     int n = 0;
-    for (; n + 8 <= N; n += 8) {
+    for (; n + 8 <= N; n += 8) {   // loads of a batch issued before its dependent stores
         float dl[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) dl[u] = base[(size_t)(n + u + 1) * DD2];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            if (bbase) bbase[(size_t)(n + u) * DD2] = __float2bfloat16_rn(s);
-            s = fmaf(dec[n + u], s, dl[u]);
-            base[(size_t)(n + u + 1) * DD2] = s;
-        }
+        for (int u = 0; u < 8; ++u) step(n + u, dl[u]);
     }
-    for (; n < N; ++n) {
-        if (bbase) bbase[(size_t)n * DD2] = __float2bfloat16_rn(s);
-        s = fmaf(dec[n], s, base[(size_t)(n + 1) * DD2]);
-        base[(size_t)(n + 1) * DD2] = s;
-    }
+    for (; n < N; ++n) step(n, base[(size_t)(n + 1) * DD2]);
     if (final_state) final_state[(size_t)bh * DD2 + e] = s;
 }
 

@@ -125,8 +125,12 @@ static int layout(int B, int H, int T, int D, int C, gka_dtype dt, gka_workspace
     off = round256(off + sizeof(float) * BH * N);
     L->norms_offset = off;
     off = round256(off + sizeof(float) * BH * (size_t)T);
-    L->states_bf16_offset = off;
-    if (tensor_core_path(D, C, dt)) off = round256(off + 2 * BH * N * 2 * (size_t)D * D);
+    L->states_lp_offset = off;
+    if (tensor_core_path(D, C, dt)) {
+        off = round256(off + 2 * BH * N * 2 * (size_t)D * D);   // fp16 states
+        off = round256(off + sizeof(float) * BH * N * 2);       // norm-bound increments
+        off = round256(off + sizeof(int) * BH * N * 2);         // state exponents
+    }
     L->total_bytes = off;
     return GKA_OK;
 }
@@ -164,14 +168,14 @@ static int forward_simt(const Tin *q, const Tin *k, const Tin *v, const float *b
     const size_t sm_delta = sizeof(float) * 3 * (size_t)C * D;
     if ((e = set_smem(k_chunk_delta<Tin, D>, sm_delta)) != cudaSuccess) return cuda_fail(e);
     { ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
-    k_chunk_delta<Tin, D><<<dim3(N, BH), kSimtThreads, sm_delta, s>>>(k, v, beta, states, decay, T,
-                                                                        N, C); }
+    k_chunk_delta<Tin, D><<<dim3(N, BH), kSimtThreads, sm_delta, s>>>(k, v, beta, states, decay,
+                                                                        nullptr, T, N, C); }
     if (int rc = check_launch()) return rc;
 
     const int DD2 = 2 * D * D;
     { ProfScope ps(GKA_KERNEL_STATE_SCAN, s);
     k_state_scan<<<dim3((DD2 + 255) / 256, BH), 256, 0, s>>>(states, decay, final_state, nullptr,
-                                                             N, DD2); }
+                                                             nullptr, nullptr, N, DD2); }
     if (int rc = check_launch()) return rc;
 
     const size_t sm_norm = sizeof(float) * ((size_t)D * D + (size_t)C * (D + 1));
@@ -203,16 +207,16 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-// 2-D map over a row-major [rows][128] bf16 array: boxes of 64 columns
+// 2-D map over a row-major [rows][128] 16-bit array: boxes of 64 columns
 // (128 bytes) x 64 rows, 128-byte swizzle (the tensor-core operand layout).
-static int bf16_rows_map(CUtensorMap *m, const void *base, uint64_t rows) {
+static int rows128_map(CUtensorMap *m, const void *base, uint64_t rows, CUtensorMapDataType ty) {
     auto enc = tensor_map_encoder();
     if (!enc) return cuda_fail(cudaErrorNotSupported);
     cuuint64_t dims[2] = {128, rows};
     cuuint64_t strides[1] = {128 * 2};
     cuuint32_t box[2] = {64, 64};
     cuuint32_t es[2] = {1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
+    CUresult r = enc(m, ty, 2, const_cast<void *>(base), dims,
                      strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? GKA_OK : cuda_fail(cudaErrorInvalidValue);
@@ -229,26 +233,33 @@ static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
     float *states = reinterpret_cast<float *>(ws + L.states_offset);
     float *decay = reinterpret_cast<float *>(ws + L.decay_offset);
     float *norms = reinterpret_cast<float *>(ws + L.norms_offset);
-    __nv_bfloat16 *sbf = reinterpret_cast<__nv_bfloat16 *>(ws + L.states_bf16_offset);
+    const size_t BHN2 = (size_t)BH * N * 2;
+    __half *slp = reinterpret_cast<__half *>(ws + L.states_lp_offset);
+    float *bound_inc = reinterpret_cast<float *>(ws + L.states_lp_offset +
+                                                 round256(2 * BHN2 * (size_t)D * D));
+    int *sexp = reinterpret_cast<int *>(reinterpret_cast<char *>(bound_inc) +
+                                        round256(sizeof(float) * BHN2));
     int *flag = nullptr;
     if (int rc = timeout_flag_ptr(&flag)) return rc;
     TcMaps maps;
-    if (int rc = bf16_rows_map(&maps.k, k, (uint64_t)BH * T)) return rc;
-    if (int rc = bf16_rows_map(&maps.v, v, (uint64_t)BH * T)) return rc;
-    if (int rc = bf16_rows_map(&maps.state, sbf, (uint64_t)BH * N * 2 * D)) return rc;
+    if (int rc = rows128_map(&maps.k, k, (uint64_t)BH * T, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)) return rc;
+    if (int rc = rows128_map(&maps.v, v, (uint64_t)BH * T, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)) return rc;
+    if (int rc = rows128_map(&maps.state, slp, (uint64_t)BH * N * 2 * D,
+                             CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+        return rc;
     cudaError_t e;
 
     const size_t sm_delta = sizeof(float) * 3 * (size_t)C * D;
     if ((e = set_smem(k_chunk_delta<__nv_bfloat16, D>, sm_delta)) != cudaSuccess) return cuda_fail(e);
     { ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
-    k_chunk_delta<__nv_bfloat16, D><<<dim3(N, BH), kSimtThreads, sm_delta, s>>>(k, v, beta, states,
-                                                                                decay, T, N, C); }
+    k_chunk_delta<__nv_bfloat16, D><<<dim3(N, BH), kSimtThreads, sm_delta, s>>>(
+        k, v, beta, states, decay, bound_inc, T, N, C); }
     if (int rc = check_launch()) return rc;
 
     const int DD2 = 2 * D * D;
     { ProfScope ps(GKA_KERNEL_STATE_SCAN, s);
-    k_state_scan<<<dim3((DD2 + 255) / 256, BH), 256, 0, s>>>(states, decay, final_state, sbf, N,
-                                                             DD2); }
+    k_state_scan<<<dim3((DD2 + 255) / 256, BH), 256, 0, s>>>(states, decay, final_state, slp,
+                                                             bound_inc, sexp, N, DD2); }
     if (int rc = check_launch()) return rc;
 
     const size_t sm_norm = sizeof(float) * ((size_t)D * D + (size_t)C * (D + 1));
@@ -261,14 +272,14 @@ static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
     if ((e = set_smem(k_chunk_solve_tc<64>, TcSmem<64>::bytes)) != cudaSuccess) return cuda_fail(e);
     { ProfScope ps(GKA_KERNEL_CHUNK_SOLVE_TC, s);
     k_chunk_solve_tc<64><<<dim3(N, BH), kTcThreads, TcSmem<64>::bytes, s>>>(
-        maps, q, beta, norms, o, T, N, C, 0, P, flag); }
+        maps, q, beta, norms, sexp, o, T, N, C, 0, P, flag); }
     if (int rc = check_launch()) return rc;
     if (C == 128) {
         if ((e = set_smem(k_chunk_solve_tc<128>, TcSmem<128>::bytes)) != cudaSuccess)
             return cuda_fail(e);
         { ProfScope ps(GKA_KERNEL_CHUNK_SOLVE_TC, s);
         k_chunk_solve_tc<128><<<dim3(N, BH), kTcThreads, TcSmem<128>::bytes, s>>>(
-            maps, q, beta, norms, o, T, N, C, 1, P, flag); }
+            maps, q, beta, norms, sexp, o, T, N, C, 1, P, flag); }
         if (int rc = check_launch()) return rc;
     }
     return GKA_OK;

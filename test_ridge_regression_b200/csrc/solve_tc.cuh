@@ -21,8 +21,20 @@
 //   the B operand of the next round.
 // The readout is the same three GEMMs with M_s in place of H_s and V in
 // place of K for the final product: o_j = b_j M_s x_j + sum_i w_{ji} (k_i.x_j) v_i.
-// H_s, K, V (bf16) arrive by TMA and stay in shared memory for all r rounds.
+// H_s, M_s, K, V arrive by TMA and stay in shared memory for all r rounds.
+//
+// Operand precision: every MMA operand is fp16 with a power-of-two scale, fp32
+// accumulation.  bf16 keys and values convert exactly (scaled by 2^-e so that
+// |k|, |v| < 1); the chunk-start states come from the scan already in fp16,
+// scaled by 2^e from a bound on their Frobenius norm; each token's iterate is
+// scaled by 2^e from the bound ||x_i|| <= ||q|| (1+2a) / (a d) that every
+// Chebyshev iterate satisfies.  All scales are undone in fp32 in the
+// epilogue.  fp16 keeps 3 more mantissa bits than bf16 at the same tensor-core
+// rate; rounding the iterate to bf16 instead would cost about 1e-2 relative
+// error at a = 0.1 (condition number 11).
 #pragma once
+
+#include <cuda_fp16.h>
 
 #include "common.cuh"
 #include "ptx.cuh"
@@ -45,8 +57,9 @@ struct TcSmem {
     static constexpr uint32_t PT = XT + 16384;               // P^T: [MG][64] bf16, MN-major
     static constexpr uint32_t QS = PT + MG * 128;            // q: [64][128] bf16 row-major
     static constexpr uint32_t SCAL = QS + 16384;             // per-token scalars
-    static constexpr uint32_t ELL = SCAL + 4 * 4 * kTcTokens; // double[MG] cumulative logs
-    static constexpr uint32_t BARS = ELL + 8 * MG + 8 * (kTcThreads / 32);
+    static constexpr uint32_t ELL = SCAL + 8 * 4 * kTcTokens; // double[MG] cumulative logs
+    static constexpr uint32_t RED = ELL + 8 * MG + 8 * (kTcThreads / 32);  // float[8] reductions
+    static constexpr uint32_t BARS = RED + 32;
     static constexpr uint32_t TBASE = BARS + 8 * 8;
     static constexpr uint32_t END = TBASE + 16;
     static constexpr size_t bytes = END + 1024;               // + alignment slack
@@ -55,7 +68,7 @@ struct TcSmem {
 struct TcMaps {
     CUtensorMap k;       // [B*H*T rows][128] bf16, box 64 x 64, 128B swizzle
     CUtensorMap v;       // same for v
-    CUtensorMap state;   // [B*H*N*2*128 rows][128] bf16 chunk-start states, box 64 x 64
+    CUtensorMap state;   // [B*H*N*2*128 rows][128] fp16 scaled chunk-start states, box 64 x 64
 };
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
@@ -65,20 +78,56 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                  : "memory");
 }
 
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-    const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+    const __half2 p = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<const uint32_t *>(&p);
 }
 
+// 2^-(floor(log2 x) + 1) for x > 0 (so that x * result < 1), else 1.
+__device__ __forceinline__ float inv_pow2_above(float x) {
+    return x > 0.f ? ldexpf(1.f, -(ilogbf(x) + 1)) : 1.f;
+}
+
+// In place: bf16 tile of `bytes` bytes -> fp16, scaled so that every |value| < 1.
+// Returns the scale.  Every thread of the block calls it.
+__device__ __forceinline__ float tile_bf16_to_f16_scaled(uint8_t *tile, int bytes, float *red) {
+    const int tid = threadIdx.x;
+    float mx = 0.f;
+    for (int c = tid * 16; c < bytes; c += kTcThreads * 16) {
+        const uint4 u = *reinterpret_cast<const uint4 *>(tile + c);
+        const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&u);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(__bfloat162float(e[i])));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    __syncthreads();
+    if ((tid & 31) == 0) red[tid >> 5] = mx;
+    __syncthreads();
+    mx = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    const float sc = inv_pow2_above(mx);
+    for (int c = tid * 16; c < bytes; c += kTcThreads * 16) {
+        uint4 u = *reinterpret_cast<const uint4 *>(tile + c);
+        const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&u);
+        uint4 w;
+        w.x = pack_f16(__bfloat162float(e[0]) * sc, __bfloat162float(e[1]) * sc);
+        w.y = pack_f16(__bfloat162float(e[2]) * sc, __bfloat162float(e[3]) * sc);
+        w.z = pack_f16(__bfloat162float(e[4]) * sc, __bfloat162float(e[5]) * sc);
+        w.w = pack_f16(__bfloat162float(e[6]) * sc, __bfloat162float(e[7]) * sc);
+        *reinterpret_cast<uint4 *>(tile + c) = w;
+    }
+    return sc;
+}
+
 // Writes 16 consecutive values (columns c0..c0+15, c0 % 16 == 0) of `row` of a
-// 128B-swizzled [rows][64] bf16 tile as two 16-byte chunks.
+// 128B-swizzled [rows][64] fp16 tile as two 16-byte chunks.
 __device__ __forceinline__ void st_row16(uint32_t tile, uint32_t row, uint32_t c0, const float *v) {
     const uint32_t base = tile + row * 128u;
     const uint32_t ch0 = ((c0 >> 3) ^ row) & 7u, ch1 = ((c0 >> 3) + 1u ^ row) & 7u;
-    st_shared_v4(base + ch0 * 16u, pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
-                 pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
-    st_shared_v4(base + ch1 * 16u, pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]),
-                 pack_bf16(v[12], v[13]), pack_bf16(v[14], v[15]));
+    st_shared_v4(base + ch0 * 16u, pack_f16(v[0], v[1]), pack_f16(v[2], v[3]),
+                 pack_f16(v[4], v[5]), pack_f16(v[6], v[7]));
+    st_shared_v4(base + ch1 * 16u, pack_f16(v[8], v[9]), pack_f16(v[10], v[11]),
+                 pack_f16(v[12], v[13]), pack_f16(v[14], v[15]));
 }
 
 // grid (N, B*H); group g = `group` of every chunk; MG = 64 * (group + 1).
@@ -86,19 +135,23 @@ template <int MG>
 __global__ void __launch_bounds__(kTcThreads, 2)
 k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__restrict__ q,
                  const float *__restrict__ beta, const float *__restrict__ norms,
-                 __nv_bfloat16 *__restrict__ o, int T, int N, int C, int group, const ChebParams P,
-                 int *__restrict__ timeout_flag) {
+                 const int *__restrict__ state_exp, __nv_bfloat16 *__restrict__ o, int T, int N,
+                 int C, int group, const ChebParams P, int *__restrict__ timeout_flag) {
     using L = TcSmem<MG>;
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
     const uint32_t sb = smem_u32(sm);
-    float *s_bi = reinterpret_cast<float *>(sm + L::SCAL);   // b_j / d_j
-    float *s_invd = s_bi + kTcTokens;                        // 1 / d_j (0 if ||H|| = 0)
-    float *s_li = s_invd + kTcTokens;                        // lambda_j / d_j
-    float *s_b = s_li + kTcTokens;                           // b_j
+    float *s_cq = reinterpret_cast<float *>(sm + L::SCAL);   // 1/d_j (0 if ||H_j|| = 0)
+    float *s_c1 = s_cq + kTcTokens;                          // coefficient of Z1 in (A x)/d
+    float *s_c3 = s_c1 + kTcTokens;                          // coefficient of Z3 in (A x)/d
+    float *s_cl = s_c3 + kTcTokens;                          // lambda_j / d_j
+    float *s_sx = s_cl + kTcTokens;                          // iterate scale 2^e_j
+    float *s_o1 = s_sx + kTcTokens;                          // readout coefficient of Z1
+    float *s_o3 = s_o1 + kTcTokens;                          // readout coefficient of Z3
     double *ell = reinterpret_cast<double *>(sm + L::ELL);
     double *wtot = ell + MG;
+    float *red = reinterpret_cast<float *>(sm + L::RED);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BARS);
     uint64_t *bar_load = &bars[0], *bar_v = &bars[1], *bar_m = &bars[2], *bar_s = &bars[3],
              *bar_z = &bars[4], *bar_fin = &bars[5];
@@ -137,14 +190,34 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         tc::tmem_relinquish();
     }
     chunk_log_prefix(beta + tok0, MG, ell, wtot);
+    bool ok = mbar_wait_bounded(bar_load, 0, kTcWaitProbes);
+    ok = mbar_wait_bounded(bar_v, 0, kTcWaitProbes) && ok;
+    // keys and values: bf16 -> fp16 in place, scaled below 1
+    const float sK = tile_bf16_to_f16_scaled(sm + L::KT, MG * 256, red);
+    const float sV = tile_bf16_to_f16_scaled(sm + L::VT, MG * 256, red);
+    const __nv_bfloat16 *qs = reinterpret_cast<const __nv_bfloat16 *>(sm + L::QS);
     if (tid < kTcTokens) {
-        const float nj = norms[tok0 + j0 + tid];
+        const int j = tid;
+        const float nj = norms[tok0 + j0 + j];
         const float invd = nj > 0.f ? 1.f / (P.half_1p2a * nj) : 0.f;
-        const float b = decay_exp(ell[j0 + tid]);
-        s_b[tid] = b;
-        s_bi[tid] = b * invd;
-        s_invd[tid] = invd;
-        s_li[tid] = P.a * nj * invd;
+        const float b = decay_exp(ell[j0 + j]);
+        float qq = 0.f;
+        for (int d = 0; d < kTcD; ++d) {
+            const float x = __bfloat162float(qs[j * kTcD + ((d + j) & (kTcD - 1))]);
+            qq = fmaf(x, x, qq);
+        }
+        // every Chebyshev iterate obeys ||x|| <= ||q|| (1+2a) / (a d): scale it below 2^12
+        const float xb = sqrtf(qq) * invd * (2.f * P.half_1p2a / P.a);
+        const float sx = ldexpf(inv_pow2_above(xb), 12);
+        const float eH = ldexpf(1.f, -state_exp[((size_t)bh * N + n) * 2]);
+        const float eM = ldexpf(1.f, -state_exp[((size_t)bh * N + n) * 2 + 1]);
+        s_cq[j] = invd;
+        s_c1[j] = b * invd * eH / sx;
+        s_c3[j] = invd / (sK * sK * sx);
+        s_cl[j] = P.a * nj * invd;
+        s_sx[j] = sx;
+        s_o1[j] = invd > 0.f ? b * eM / sx : 0.f;
+        s_o3[j] = invd > 0.f ? 1.f / (sV * sK * sx) : 0.f;
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -173,28 +246,27 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         tc::tmem_wait_st();
     }
 
-    bool ok = mbar_wait_bounded(bar_load, 0, kTcWaitProbes);
-    const __nv_bfloat16 *qs = reinterpret_cast<const __nv_bfloat16 *>(sm + L::QS);
-
-    // x_1 = q / d, x_0 = 0; thread d keeps element d of all 64 iterates
+    // x_1 = q / d, x_0 = 0; thread d keeps element d of all 64 iterates in fp32
     float xc[kTcTokens], xp[kTcTokens];
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
+        float xs[16];
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
             const int jj = c * 16 + u;
-            xc[jj] = __bfloat162float(qs[jj * kTcD + tid]) * s_invd[jj];
+            xc[jj] = __bfloat162float(qs[jj * kTcD + tid]) * s_cq[jj];
             xp[jj] = 0.f;
+            xs[u] = xc[jj] * s_sx[jj];
         }
-        st_row16(sb + L::XT, tid, c * 16, &xc[c * 16]);
+        st_row16(sb + L::XT, tid, c * 16, xs);
     }
     fence_proxy_async_smem();
     tc::fence_before_sync();
     ok = __syncthreads_and(ok);
 
-    constexpr uint32_t IDESC_S = tc::idesc_bf16(MG, 64, false, true);
-    constexpr uint32_t IDESC_Z1 = tc::idesc_bf16(128, 64, false, true);
-    constexpr uint32_t IDESC_Z3 = tc::idesc_bf16(128, 64, true, true);
+    constexpr uint32_t IDESC_S = tc::idesc_f16(MG, 64, false, true);
+    constexpr uint32_t IDESC_Z1 = tc::idesc_f16(128, 64, false, true);
+    constexpr uint32_t IDESC_Z3 = tc::idesc_f16(128, 64, true, true);
     const uint32_t a_hm = sb + L::HM, a_kt = sb + L::KT, a_vt = sb + L::VT, b_xt = sb + L::XT,
                    b_pt = sb + L::PT;
     bool m_requested = false;
@@ -208,7 +280,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
             // S^T = K X^T
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-                tc::mma_bf16(tmem + T_S,
+                tc::mma_f16(tmem + T_S,
                              tc::sdesc(a_kt + (kk >> 2) * (MG * 128) + (kk & 3) * 32, 16, 1024),
                              tc::sdesc(b_xt + kk * 2048, 8192, 1024), IDESC_S, kk > 0);
             tc::commit(bar_s);
@@ -227,7 +299,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
             if (ok) {
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_bf16(tmem + T_Z1,
+                    tc::mma_f16(tmem + T_Z1,
                                  tc::sdesc(a_hm + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
                                  tc::sdesc(b_xt + kk * 2048, 8192, 1024), IDESC_Z1, kk > 0);
             }
@@ -235,7 +307,6 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         // P^T = W o S^T  -> bf16, MN-major tile of MG rows
         if (!mbar_wait_bounded(bar_s, ph, kTcWaitProbes)) ok = false;
         tc::fence_after_sync();
-        if (out_pass && tid == 0 && ok) ok = mbar_wait_bounded(bar_v, 0, kTcWaitProbes);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             float sv[16], wv[16];
@@ -255,7 +326,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
             const uint32_t a3 = out_pass ? a_vt : a_kt;
 #pragma unroll
             for (int kk = 0; kk < MG / 16; ++kk)
-                tc::mma_bf16(tmem + T_Z3, tc::sdesc(a3 + kk * 2048, MG * 128, 1024),
+                tc::mma_f16(tmem + T_Z3, tc::sdesc(a3 + kk * 2048, MG * 128, 1024),
                              tc::sdesc(b_pt + kk * 2048, 8192, 1024), IDESC_Z3, kk > 0);
             tc::commit(bar_z);
         }
@@ -279,17 +350,19 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
                 tc::tmem_ld16(tl + T_Z1 + c * 16, z1);
                 tc::tmem_ld16(tl + T_Z3 + c * 16, z3);
                 tc::tmem_wait_ld();
+                float xs[16];
 #pragma unroll
                 for (int u = 0; u < 16; ++u) {
                     const int jj = c * 16 + u;
-                    // (q - A x)/d = q/d - (b Z1 + Z3)/d - (lambda/d) x
-                    const float r = __bfloat162float(qs[jj * kTcD + tid]) * s_invd[jj] -
-                                    s_bi[jj] * z1[u] - s_invd[jj] * z3[u] - s_li[jj] * xc[jj];
+                    // (q - A x)/d = q/d - (b H_s x + intra)/d - (lambda/d) x, scales undone
+                    const float r = __bfloat162float(qs[jj * kTcD + tid]) * s_cq[jj] -
+                                    s_c1[jj] * z1[u] - s_c3[jj] * z3[u] - s_cl[jj] * xc[jj];
                     const float xn = fmaf(w, r + xc[jj] - xp[jj], xp[jj]);
                     xp[jj] = xc[jj];
                     xc[jj] = xn;
+                    xs[u] = xn * s_sx[jj];
                 }
-                st_row16(sb + L::XT, tid, c * 16, &xc[c * 16]);
+                st_row16(sb + L::XT, tid, c * 16, xs);
             }
             fence_proxy_async_smem();
             tc::fence_before_sync();
@@ -306,7 +379,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
 #pragma unroll
                 for (int u = 0; u < 16; ++u) {
                     const int jj = c * 16 + u;
-                    const float val = s_invd[jj] > 0.f ? fmaf(s_b[jj], z1[u], z3[u]) : 0.f;
+                    const float val = fmaf(s_o1[jj], z1[u], s_o3[jj] * z3[u]);
                     orow[(size_t)jj * kTcD] = __float2bfloat16_rn(val);
                 }
             }

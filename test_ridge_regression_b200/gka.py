@@ -38,7 +38,7 @@ class KernelTimes(ctypes.Structure):
 
 class WorkspaceLayout(ctypes.Structure):
     _fields_ = [("states_offset", ctypes.c_size_t), ("decay_offset", ctypes.c_size_t),
-                ("norms_offset", ctypes.c_size_t), ("states_bf16_offset", ctypes.c_size_t),
+                ("norms_offset", ctypes.c_size_t), ("states_lp_offset", ctypes.c_size_t),
                 ("total_bytes", ctypes.c_size_t)]
 
 
