@@ -281,15 +281,18 @@ def main():
     # ---- roofline of the dominant kernel ----
     ch, out, upd, nrm = flops_per_head_token(w.D, w.chunk, w.r)
     head_tok = w.B * w.H * w.T
+    # the dominant kernel: largest summed device time among the step's kernels
     dom = max(kt.items(), key=lambda kv: kv[1][0])
     dom_name, (dom_ms, dom_n) = dom
     per_launch_ms = dom_ms / dom_n
-    alg = {"chunk_solve": ch + out, "chunk_norm": nrm, "chunk_delta": upd}.get(dom_name, 0)
+    alg = {"chunk_solve": ch + out, "chunk_solve_tc": ch + out, "chunk_norm": nrm,
+           "chunk_delta": upd}.get(dom_name, 0)
     kernel_flops = alg * head_tok
     sm_mhz_max = peaks.get("sm_max_mhz", 1965.0)
-    if dom_name == "chunk_solve" and getattr(gka, "SOLVE_ON_TENSOR_CORES", False):
+    if dom_name == "chunk_solve_tc":
+        # fp16 operands, fp32 accumulation: the dense fp16 peak equals the bf16 one
         bound, peak, punit = "tensor", peaks["bf16_tflops"], "TFLOP/s"
-        peak_note = f"bf16 dense, {peaks['_source']} burst"
+        peak_note = f"dense bf16/fp16 tensor peak, {peaks['_source']} burst (cuBLAS bf16)"
     else:
         # CUDA-core fp32 FMA: 148 SMs x 128 lanes x 2 flop x max SM clock
         bound, punit = "alu", "TFLOP/s"
