@@ -63,9 +63,11 @@ typedef enum {
  * multiple of 256. */
 typedef struct {
     size_t states_offset;   /* fp32 [B, H, N+1, 2, D, D]: H_s, M_s in force before chunk n;
-                               slot N holds the state after the last token */
+                               slot N holds the state after the last token.  On the
+                               tensor-core path slots 1..N keep the per-chunk increments
+                               instead and the states live in the fp16 region below */
     size_t decay_offset;    /* fp32 [B, H, N]: product of beta over chunk n */
-    size_t norms_offset;    /* fp32 [B, H, T]: ||H_t||_F */
+    size_t norms_offset;    /* fp32 [B, H, T]: ||H_t||_F as used by the solve */
     size_t states_lp_offset;   /* tensor-core path only (0 bytes otherwise): fp16
                                   [B, H, N, 2, D, D] copies of the chunk-start states, each
                                   scaled by a power of two, then the scales; the region ends
@@ -86,9 +88,10 @@ int gka_forward_workspace_layout(int B, int H, int T, int D, int chunk, gka_dtyp
  * state is computed sequentially; ||H_t||_F comes from a closed form through
  * the Gram matrix of the keys; everything within a chunk runs in parallel).
  * Steps, each a kernel on `stream`:
- *   1. chunk-state scan: H_s, M_s before every chunk (fp32), into workspace;
+ *   1. chunk-state scan: H_s, M_s before every chunk, into workspace;
  *   2. per-token ||H_t||_F, into workspace;
- *   3. r-step Chebyshev solve for every token and 4. the readout o_t = M_t x_t.
+ *   3. r-step Chebyshev solve for every token and 4. the readout o_t = M_t x_t
+ *      (on the tensor-core path 2-4 are one kernel).
  * The result does not depend on `chunk` beyond floating-point rounding.
  *
  *   q, k, v     [B, H, T, D] in `dt` (fp32 or bf16); k and q are used as given

@@ -122,7 +122,8 @@ k_chunk_delta(const Tin *__restrict__ k, const Tin *__restrict__ v,
 // grid (ceil(2*D*D/256), B*H), block 256.  Optionally copies S_N out and
 // writes an fp16 copy of every chunk-start state S_n, n < N, scaled by a power
 // of two 2^e_n chosen from the running bound ||S_n||_F <= bound_n (the
-// tensor-core operands; e_n goes to state_exp[bh][n][H or M]).
+// tensor-core operands; e_n goes to state_exp[bh][n][H or M]).  Without
+// write_fp32 the fp32 slots keep the increments and only S_N is written out.
 // ---------------------------------------------------------------------------
 // Exponent e such that |value| <= bound implies |value * 2^e| <= 2^14.
 __device__ __forceinline__ int lp_exponent(float bound) {
@@ -134,7 +135,8 @@ __device__ __forceinline__ int lp_exponent(float bound) {
 __global__ void __launch_bounds__(256)
 k_state_scan(float *__restrict__ states, const float *__restrict__ decay,
              float *__restrict__ final_state, __half *__restrict__ states_lp,
-             const float *__restrict__ bound_inc, int *__restrict__ state_exp, int N, int DD2) {
+             const float *__restrict__ bound_inc, int *__restrict__ state_exp, int N, int DD2,
+             bool write_fp32) {
     const int bh = blockIdx.y;
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
     if (e >= DD2) return;
@@ -155,7 +157,7 @@ k_state_scan(float *__restrict__ states, const float *__restrict__ decay,
             bound = fmaf(dec[n], bound, bound_inc[((size_t)bh * N + n) * 2 + mat]);
         }
         s = fmaf(dec[n], s, dl);
-        base[(size_t)(n + 1) * DD2] = s;
+        if (write_fp32) base[(size_t)(n + 1) * DD2] = s;
     };
     int n = 0;
     for (; n + 8 <= N; n += 8) {   // loads of a batch issued before its dependent stores

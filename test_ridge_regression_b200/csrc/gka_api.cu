@@ -16,6 +16,7 @@
 #include "chunk_simt.cuh"
 #include "common.cuh"
 #include "decode.cuh"
+#include "delta_tc.cuh"
 #include "solve_tc.cuh"
 
 namespace gka {
@@ -175,7 +176,7 @@ static int forward_simt(const Tin *q, const Tin *k, const Tin *v, const float *b
     const int DD2 = 2 * D * D;
     { ProfScope ps(GKA_KERNEL_STATE_SCAN, s);
     k_state_scan<<<dim3((DD2 + 255) / 256, BH), 256, 0, s>>>(states, decay, final_state, nullptr,
-                                                             nullptr, nullptr, N, DD2); }
+                                                             nullptr, nullptr, N, DD2, true); }
     if (int rc = check_launch()) return rc;
 
     const size_t sm_norm = sizeof(float) * ((size_t)D * D + (size_t)C * (D + 1));
@@ -249,24 +250,25 @@ static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
         return rc;
     cudaError_t e;
 
-    const size_t sm_delta = sizeof(float) * 3 * (size_t)C * D;
-    if ((e = set_smem(k_chunk_delta<__nv_bfloat16, D>, sm_delta)) != cudaSuccess) return cuda_fail(e);
-    { ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
-    k_chunk_delta<__nv_bfloat16, D><<<dim3(N, BH), kSimtThreads, sm_delta, s>>>(
-        k, v, beta, states, decay, bound_inc, T, N, C); }
+    if (C == 64) {
+        if ((e = set_smem(k_chunk_delta_tc<64>, DeltaSmem<64>::bytes)) != cudaSuccess)
+            return cuda_fail(e);
+        ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
+        k_chunk_delta_tc<64><<<dim3(N, BH), kTcThreads, DeltaSmem<64>::bytes, s>>>(
+            maps, beta, states, decay, bound_inc, T, N, flag);
+    } else {
+        if ((e = set_smem(k_chunk_delta_tc<128>, DeltaSmem<128>::bytes)) != cudaSuccess)
+            return cuda_fail(e);
+        ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
+        k_chunk_delta_tc<128><<<dim3(N, BH), kTcThreads, DeltaSmem<128>::bytes, s>>>(
+            maps, beta, states, decay, bound_inc, T, N, flag);
+    }
     if (int rc = check_launch()) return rc;
 
     const int DD2 = 2 * D * D;
     { ProfScope ps(GKA_KERNEL_STATE_SCAN, s);
     k_state_scan<<<dim3((DD2 + 255) / 256, BH), 256, 0, s>>>(states, decay, final_state, slp,
-                                                             bound_inc, sexp, N, DD2); }
-    if (int rc = check_launch()) return rc;
-
-    const size_t sm_norm = sizeof(float) * ((size_t)D * D + (size_t)C * (D + 1));
-    if ((e = set_smem(k_chunk_norm<__nv_bfloat16, D>, sm_norm)) != cudaSuccess) return cuda_fail(e);
-    { ProfScope ps(GKA_KERNEL_CHUNK_NORM, s);
-    k_chunk_norm<__nv_bfloat16, D><<<dim3(N, BH), kSimtThreads, sm_norm, s>>>(k, beta, states,
-                                                                              norms, T, N, C); }
+                                                             bound_inc, sexp, N, DD2, false); }
     if (int rc = check_launch()) return rc;
 
     if ((e = set_smem(k_chunk_solve_tc<64>, TcSmem<64>::bytes)) != cudaSuccess) return cuda_fail(e);

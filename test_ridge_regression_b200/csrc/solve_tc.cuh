@@ -59,7 +59,9 @@ struct TcSmem {
     static constexpr uint32_t SCAL = QS + 16384;             // per-token scalars
     static constexpr uint32_t ELL = SCAL + 8 * 4 * kTcTokens; // double[MG] cumulative logs
     static constexpr uint32_t RED = ELL + 8 * MG + 8 * (kTcThreads / 32);  // float[8] reductions
-    static constexpr uint32_t BARS = RED + 32;
+    static constexpr uint32_t NRM = RED + 32;                 // norm terms: u, E, X, Gjj [4][MG]
+    static constexpr uint32_t UPART = NRM + 16 * MG;          // [4 warps][MG] partial sums of u
+    static constexpr uint32_t BARS = UPART + 16 * MG;
     static constexpr uint32_t TBASE = BARS + 8 * 8;
     static constexpr uint32_t END = TBASE + 16;
     static constexpr size_t bytes = END + 1024;               // + alignment slack
@@ -130,11 +132,29 @@ __device__ __forceinline__ void st_row16(uint32_t tile, uint32_t row, uint32_t c
                  pack_f16(v[12], v[13]), pack_f16(v[14], v[15]));
 }
 
+// Sums each of the N per-lane values v[0..N) over the 32 lanes of the warp by
+// recursive halving (N - N/32 shuffles).  Afterwards lane l holds, in
+// v[0..N/32), the totals of the original indices l*N/32 .. l*N/32 + N/32 - 1.
+template <int N>
+__device__ __forceinline__ void reduce_scatter32(float (&v)[N], int lane) {
+#pragma unroll
+    for (int step = 0; step < 5; ++step) {
+        const int o = 16 >> step, h = N >> (step + 1);
+        const bool up = lane & o;
+#pragma unroll
+        for (int s = 0; s < h; ++s) {
+            const float send = up ? v[s] : v[s + h];
+            const float keep = up ? v[s + h] : v[s];
+            v[s] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+}
+
 // grid (N, B*H); group g = `group` of every chunk; MG = 64 * (group + 1).
 template <int MG>
 __global__ void __launch_bounds__(kTcThreads, 2)
 k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__restrict__ q,
-                 const float *__restrict__ beta, const float *__restrict__ norms,
+                 const float *__restrict__ beta, float *__restrict__ norms,
                  const int *__restrict__ state_exp, __nv_bfloat16 *__restrict__ o, int T, int N,
                  int C, int group, const ChebParams P, int *__restrict__ timeout_flag) {
     using L = TcSmem<MG>;
@@ -154,7 +174,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     float *red = reinterpret_cast<float *>(sm + L::RED);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BARS);
     uint64_t *bar_load = &bars[0], *bar_v = &bars[1], *bar_m = &bars[2], *bar_s = &bars[3],
-             *bar_z = &bars[4], *bar_fin = &bars[5];
+             *bar_z = &bars[4], *bar_fin = &bars[5], *bar_n = &bars[6];
     uint32_t *tbase = reinterpret_cast<uint32_t *>(sm + L::TBASE);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -164,7 +184,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     const int srow = (int)(((size_t)bh * N + n) * 2 * kTcD);   // H_s row in the state map
 
     if (tid == 0) {
-        for (int i = 0; i < 6; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 7; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
     }
     __syncthreads();
@@ -196,9 +216,130 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     const float sK = tile_bf16_to_f16_scaled(sm + L::KT, MG * 256, red);
     const float sV = tile_bf16_to_f16_scaled(sm + L::VT, MG * 256, red);
     const __nv_bfloat16 *qs = reinterpret_cast<const __nv_bfloat16 *>(sm + L::QS);
+    const int eHexp = state_exp[((size_t)bh * N + n) * 2];
+    const int eMexp = state_exp[((size_t)bh * N + n) * 2 + 1];
+    fence_proxy_async_smem();
+    tc::fence_before_sync();
+    ok = __syncthreads_and(ok);
+    tc::fence_after_sync();
+    const uint32_t tmem = *tbase;
+    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);   // this warp's TMEM lane quarter
+    const uint32_t T_Z1 = 0, T_Z3 = 64, T_S = 128, T_W = 192;
+    const uint32_t a_hm = sb + L::HM, a_kt = sb + L::KT, a_vt = sb + L::VT, b_xt = sb + L::XT,
+                   b_pt = sb + L::PT;
+
+    // rows of S (keys) held by this thread: M = 64 puts key 16w + l in lane
+    // 32w + l (l < 16); M = 128 puts key t in lane t.
+    const bool s_owner = (MG == 128) || (lane < 16);
+    const int key = (MG == 128) ? tid : warp * 16 + lane;
+
+    // ---- per-token ||H_j||_F (ai.info, Methodology: closed form through the
+    // key Gram matrix).  Zn = H_s K^T gives u_i = k_i^T H_s k_i, G = K K^T the
+    // intra-chunk terms:  ||H_j||^2 = b_j^2 ||H_s||^2 + 2 b_j X_j + R_j with
+    // X_j = sum_{i<=j} w_ji u_i and R_j = beta_j^2 R_{j-1} + 2 E_j + G_jj^2,
+    // E_j = sum_{i<j} w_ji G_ij^2 (R_j = sum_{i,l<=j} w_ji w_jl G_il^2).
+    if (tid == 0 && ok) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t kdesc = tc::sdesc(a_kt + (kk >> 2) * (MG * 128) + (kk & 3) * 32, 16, 1024);
+            tc::mma_f16(tmem + 0, tc::sdesc(a_hm + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                        kdesc, tc::idesc_f16(128, MG, false, false), kk > 0);
+            tc::mma_f16(tmem + 128, kdesc, kdesc, tc::idesc_f16(MG, MG, false, false), kk > 0);
+        }
+        tc::commit(bar_n);
+    }
+    float *s_u = reinterpret_cast<float *>(sm + L::NRM);
+    float *s_E = s_u + MG, *s_X = s_E + MG, *s_G = s_X + MG;
+    float *upart = reinterpret_cast<float *>(sm + L::UPART);
+    {
+        // ||H_s||_F^2 from the (scaled) fp16 copy
+        float hs = 0.f;
+        for (int c = tid * 16; c < 32768; c += kTcThreads * 16) {
+            const uint4 u4 = *reinterpret_cast<const uint4 *>(sm + L::HM + c);
+            const __half *e = reinterpret_cast<const __half *>(&u4);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float x = __half2float(e[i]);
+                hs = fmaf(x, x, hs);
+            }
+        }
+        hs = warp_sum(hs);
+        if (lane == 0) red[4 + warp] = hs;
+    }
+    if (!mbar_wait_bounded(bar_n, 0, kTcWaitProbes)) ok = false;
+    tc::fence_after_sync();
+    {
+        // u_i: thread d forms k_i[d] (H_s k_i)[d] for every key i, then a sum over d
+        const __half *kt = reinterpret_cast<const __half *>(sm + L::KT);
+        const int hoff = (tid >> 6) * (MG * 64), c = tid & 63;
+        float pv[MG];
+#pragma unroll
+        for (int cb = 0; cb < MG; cb += 16) {
+            float zn[16];
+            tc::tmem_ld16(tl + cb, zn);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int u = 0; u < 16; ++u)
+                pv[cb + u] = zn[u] * __half2float(kt[hoff + tc::sw128_offset(cb + u, c) / 2]);
+        }
+        reduce_scatter32<MG>(pv, lane);
+#pragma unroll
+        for (int s2 = 0; s2 < MG / 32; ++s2) upart[warp * MG + lane * (MG / 32) + s2] = pv[s2];
+    }
+    __syncthreads();
+    const float inv_uscale = ldexpf(1.f, -eHexp) / (sK * sK);
+    if (tid < MG) s_u[tid] = (upart[tid] + upart[MG + tid] + upart[2 * MG + tid] +
+                              upart[3 * MG + tid]) * inv_uscale;
+    __syncthreads();
+    {
+        // row `key` of G: E_key, X_key, G_key,key
+        const float gs = 1.f / (sK * sK);
+        float es = 0.f, xs = 0.f, gjj = 0.f;
+#pragma unroll
+        for (int cb = 0; cb < MG; cb += 16) {
+            float g[16];
+            tc::tmem_ld16(tl + 128 + cb, g);
+            tc::tmem_wait_ld();
+            if (s_owner) {
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int i = cb + u;
+                    if (i <= key) {
+                        const float w = decay_exp(ell[key] - ell[i]);
+                        const float gi = g[u] * gs;
+                        xs = fmaf(w, s_u[i], xs);
+                        if (i < key) es = fmaf(w * gi, gi, es);
+                        else gjj = gi;
+                    }
+                }
+            }
+        }
+        if (s_owner) {
+            s_E[key] = es;
+            s_X[key] = xs;
+            s_G[key] = gjj;
+        }
+    }
+    __syncthreads();
+    float *s_n = s_o3;   // per-token norms, then overwritten by the readout coefficient
+    if (tid == 0) {
+        const float hs2 = (red[4] + red[5] + red[6] + red[7]) * ldexpf(1.f, -2 * eHexp);
+        float R = 0.f;
+        for (int j = 0; j < MG; ++j) {
+            const float bj = decay_exp(j == 0 ? ell[0] : ell[j] - ell[j - 1]);
+            R = fmaf(bj * bj, R, fmaf(2.f, s_E[j], s_G[j] * s_G[j]));
+            if (j >= j0) {
+                const float b = decay_exp(ell[j]);
+                const float n2 = fmaf(b * b, hs2, fmaf(2.f * b, s_X[j], R));
+                s_n[j - j0] = sqrtf(fmaxf(n2, 0.f));
+            }
+        }
+    }
+    __syncthreads();
     if (tid < kTcTokens) {
         const int j = tid;
-        const float nj = norms[tok0 + j0 + j];
+        const float nj = s_n[j];
+        norms[tok0 + j0 + j] = nj;
         const float invd = nj > 0.f ? 1.f / (P.half_1p2a * nj) : 0.f;
         const float b = decay_exp(ell[j0 + j]);
         float qq = 0.f;
@@ -209,8 +350,8 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         // every Chebyshev iterate obeys ||x|| <= ||q|| (1+2a) / (a d): scale it below 2^12
         const float xb = sqrtf(qq) * invd * (2.f * P.half_1p2a / P.a);
         const float sx = ldexpf(inv_pow2_above(xb), 12);
-        const float eH = ldexpf(1.f, -state_exp[((size_t)bh * N + n) * 2]);
-        const float eM = ldexpf(1.f, -state_exp[((size_t)bh * N + n) * 2 + 1]);
+        const float eH = ldexpf(1.f, -eHexp);
+        const float eM = ldexpf(1.f, -eMexp);
         s_cq[j] = invd;
         s_c1[j] = b * invd * eH / sx;
         s_c3[j] = invd / (sK * sK * sx);
@@ -219,17 +360,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         s_o1[j] = invd > 0.f ? b * eM / sx : 0.f;
         s_o3[j] = invd > 0.f ? 1.f / (sV * sK * sx) : 0.f;
     }
-    tc::fence_before_sync();
     __syncthreads();
-    tc::fence_after_sync();
-    const uint32_t tmem = *tbase;
-    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);   // this warp's TMEM lane quarter
-    const uint32_t T_Z1 = 0, T_Z3 = 64, T_S = 128, T_W = 192;
-
-    // rows of S (keys) held by this thread: M = 64 puts key 16w + l in lane
-    // 32w + l (l < 16); M = 128 puts key t in lane t.
-    const bool s_owner = (MG == 128) || (lane < 16);
-    const int key = (MG == 128) ? tid : warp * 16 + lane;
 
     // W^T rows: W[i][j] = w_{ji} = exp(l_j - l_i) for i <= j, else 0
     {
@@ -267,8 +398,6 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     constexpr uint32_t IDESC_S = tc::idesc_f16(MG, 64, false, true);
     constexpr uint32_t IDESC_Z1 = tc::idesc_f16(128, 64, false, true);
     constexpr uint32_t IDESC_Z3 = tc::idesc_f16(128, 64, true, true);
-    const uint32_t a_hm = sb + L::HM, a_kt = sb + L::KT, a_vt = sb + L::VT, b_xt = sb + L::XT,
-                   b_pt = sb + L::PT;
     bool m_requested = false;
     uint32_t ph = 0;   // phase parity of bar_s / bar_z (both complete once per round)
 

@@ -33,13 +33,28 @@ def run_forward(q, k, v, beta, a, r, C):
     return o, fs, ws
 
 
+def tensor_core_path(dtype, D, C):
+    """The rule include/gka.h states for the tensor-core solve."""
+    return dtype == torch.bfloat16 and D == 128 and C in (64, 128)
+
+
 def ws_views(ws, B, H, T, D, C, dtype):
+    """Chunk-start states [B,H,N,2,D,D] (fp32; on the tensor-core path the fp16
+    copies with their power-of-two scales undone) and norms [B,H,T]."""
     L = gka.workspace_layout(B, H, T, D, C, dtype)
     N = T // C
+    norms = ws[L.norms_offset:L.norms_offset + 4 * B * H * T].view(torch.float32).view(B, H, T)
+    if tensor_core_path(dtype, D, C):
+        n16 = B * H * N * 2 * D * D
+        lp = ws[L.states_lp_offset:L.states_lp_offset + 2 * n16].view(torch.float16)
+        lp = lp.view(B, H, N, 2, D, D).double()
+        off = L.states_lp_offset + ((2 * n16 + 255) // 256) * 256
+        off += ((4 * B * H * N * 2 + 255) // 256) * 256
+        ex = ws[off:off + 4 * B * H * N * 2].view(torch.int32).view(B, H, N, 2).double()
+        return lp * torch.pow(2.0, -ex)[..., None, None], norms
     states = ws[L.states_offset:L.states_offset + 4 * B * H * (N + 1) * 2 * D * D]
     states = states.view(torch.float32).view(B, H, N + 1, 2, D, D)
-    norms = ws[L.norms_offset:L.norms_offset + 4 * B * H * T].view(torch.float32).view(B, H, T)
-    return states, norms
+    return states[:, :, :N], norms
 
 
 def check_against_oracle(q, k, v, beta, a, r, C, *, check_ws=True):
@@ -54,12 +69,16 @@ def check_against_oracle(q, k, v, beta, a, r, C, *, check_ws=True):
     ferr = head_rel_err(fs, ref["final_state"])
     assert ferr <= 1e-5, ferr
     if check_ws:
+        # intermediate results: fp32 on the CUDA-core path; on the tensor-core path
+        # the states are fp16 copies (relative rounding 2^-11) and the norms use them
+        tc = tensor_core_path(q.dtype, D, C)
         states, norms = ws_views(ws, B, H, T, D, C, q.dtype)
-        assert head_rel_err(norms, ref["norms"]) <= 1e-5
-        cs = f64(states[:, :, :T // C])
+        assert head_rel_err(norms, ref["norms"]) <= (1e-3 if tc else 1e-5)
+        cs = f64(states)
         assert np.all(cs[:, :, 0] == 0)
         if T // C > 1:
-            assert head_rel_err(cs[:, :, 1:], ref["chunk_states"][:, :, 1:], head_dims=3) <= 1e-5
+            assert head_rel_err(cs[:, :, 1:], ref["chunk_states"][:, :, 1:],
+                                head_dims=3) <= (1e-3 if tc else 1e-5)
     return err
 
 
