@@ -55,7 +55,7 @@ struct TcSmem {
     static constexpr uint32_t VT = KT + MG * 256;            // values: 2 x [MG][64] bf16
     static constexpr uint32_t XT = VT + MG * 256;            // X^T: [128][64] bf16, MN-major
     static constexpr uint32_t PT = XT + 16384;               // P^T: [MG][64] bf16, MN-major
-    static constexpr uint32_t QS = PT + MG * 128;            // q: [64][128] bf16 row-major
+    static constexpr uint32_t QS = PT + MG * 128;            // q: [64][128] bf16, then q^T
     static constexpr uint32_t SCAL = QS + 16384;             // per-token scalars
     static constexpr uint32_t ELL = SCAL + 8 * 4 * kTcTokens; // double[MG] cumulative logs
     static constexpr uint32_t RED = ELL + 8 * MG + 8 * (kTcThreads / 32);  // float[8] reductions
@@ -88,6 +88,33 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
 // 2^-(floor(log2 x) + 1) for x > 0 (so that x * result < 1), else 1.
 __device__ __forceinline__ float inv_pow2_above(float x) {
     return x > 0.f ? ldexpf(1.f, -(ilogbf(x) + 1)) : 1.f;
+}
+
+// 16 consecutive fp32 values from shared memory (16-byte aligned), as 4 vector loads.
+__device__ __forceinline__ void ld_f32x16(const float *p, float *v) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float4 t = reinterpret_cast<const float4 *>(p)[i];
+        v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
+    }
+}
+
+// Tokens 16c..16c+15 of row `row` of the 128B-swizzled bf16 q^T tile, as fp32.
+__device__ __forceinline__ void load_qrow16(uint32_t tile, uint32_t row, int c, float *v) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint32_t ch = ((uint32_t)(2 * c + h) ^ row) & 7u;
+        uint32_t a, b, cc, d;
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(a), "=r"(b), "=r"(cc), "=r"(d)
+                     : "r"(tile + row * 128u + ch * 16u));
+        const uint32_t w4[4] = {a, b, cc, d};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            v[8 * h + 2 * i] = __uint_as_float(w4[i] << 16);
+            v[8 * h + 2 * i + 1] = __uint_as_float(w4[i] & 0xffff0000u);
+        }
+    }
 }
 
 // In place: bf16 tile of `bytes` bytes -> fp16, scaled so that every |value| < 1.
@@ -162,12 +189,10 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
     const uint32_t sb = smem_u32(sm);
-    float *s_cq = reinterpret_cast<float *>(sm + L::SCAL);   // 1/d_j (0 if ||H_j|| = 0)
-    float *s_c1 = s_cq + kTcTokens;                          // coefficient of Z1 in (A x)/d
-    float *s_c3 = s_c1 + kTcTokens;                          // coefficient of Z3 in (A x)/d
-    float *s_cl = s_c3 + kTcTokens;                          // lambda_j / d_j
-    float *s_sx = s_cl + kTcTokens;                          // iterate scale 2^e_j
-    float *s_o1 = s_sx + kTcTokens;                          // readout coefficient of Z1
+    float *s_cq = reinterpret_cast<float *>(sm + L::SCAL);   // coefficient of q (scaled domain)
+    float *s_c1 = s_cq + kTcTokens;                          // coefficient of Z1
+    float *s_c3 = s_c1 + kTcTokens;                          // coefficient of Z3
+    float *s_o1 = s_c3 + kTcTokens;                          // readout coefficient of Z1
     float *s_o3 = s_o1 + kTcTokens;                          // readout coefficient of Z3
     double *ell = reinterpret_cast<double *>(sm + L::ELL);
     double *wtot = ell + MG;
@@ -224,7 +249,8 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     tc::fence_after_sync();
     const uint32_t tmem = *tbase;
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);   // this warp's TMEM lane quarter
-    const uint32_t T_Z1 = 0, T_Z3 = 64, T_S = 128, T_W = 192;
+    // TMEM columns: Z1 | S, then Z3 (S is consumed before MMA3 writes Z3) | W | x_prev
+    const uint32_t T_Z1 = 0, T_S = 64, T_Z3 = 64, T_W = 128, T_XP = 192;
     const uint32_t a_hm = sb + L::HM, a_kt = sb + L::KT, a_vt = sb + L::VT, b_xt = sb + L::XT,
                    b_pt = sb + L::PT;
 
@@ -347,20 +373,37 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
             const float x = __bfloat162float(qs[j * kTcD + ((d + j) & (kTcD - 1))]);
             qq = fmaf(x, x, qq);
         }
-        // every Chebyshev iterate obeys ||x|| <= ||q|| (1+2a) / (a d): scale it below 2^12
+        // every Chebyshev iterate obeys ||x|| <= ||q|| (1+2a) / (a d): the iterate is
+        // kept as x~ = sx x with sx a power of two that puts ||x~|| below 2^12
         const float xb = sqrtf(qq) * invd * (2.f * P.half_1p2a / P.a);
         const float sx = ldexpf(inv_pow2_above(xb), 12);
         const float eH = ldexpf(1.f, -eHexp);
         const float eM = ldexpf(1.f, -eMexp);
-        s_cq[j] = invd;
-        s_c1[j] = b * invd * eH / sx;
-        s_c3[j] = invd / (sK * sK * sx);
-        s_cl[j] = P.a * nj * invd;
-        s_sx[j] = sx;
+        // (q - A x)/d in the scaled domain: cq q - c1 Z1 - c3 Z3 - cl x~
+        s_cq[j] = sx * invd;
+        s_c1[j] = b * invd * eH;
+        s_c3[j] = invd / (sK * sK);
         s_o1[j] = invd > 0.f ? b * eM / sx : 0.f;
         s_o3[j] = invd > 0.f ? 1.f / (sV * sK * sx) : 0.f;
     }
     __syncthreads();
+
+    // q^T: transpose the token-major q tile in place into [128 d][64 tokens]
+    // (128B-swizzled rows) so that thread d reads 8 tokens per 16-byte load
+    {
+        uint32_t qv[kTcTokens / 2];
+#pragma unroll
+        for (int jj = 0; jj < kTcTokens; jj += 2) {
+            const __nv_bfloat16 lo = qs[jj * kTcD + tid], hi = qs[(jj + 1) * kTcD + tid];
+            qv[jj / 2] = (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch)
+            st_shared_v4(sb + L::QS + tid * 128u + ((ch ^ tid) & 7u) * 16u, qv[4 * ch],
+                         qv[4 * ch + 1], qv[4 * ch + 2], qv[4 * ch + 3]);
+    }
+    const float cl = 2.f * P.a / (1.f + 2.f * P.a);   // lambda / d for every token with H != 0
 
     // W^T rows: W[i][j] = w_{ji} = exp(l_j - l_i) for i <= j, else 0
     {
@@ -377,19 +420,22 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         tc::tmem_wait_st();
     }
 
-    // x_1 = q / d, x_0 = 0; thread d keeps element d of all 64 iterates in fp32
-    float xc[kTcTokens], xp[kTcTokens];
+    // x_1 = q / d, x_0 = 0 (scaled by sx): thread d keeps element d of the 64
+    // current iterates in registers and of the previous ones in TMEM
+    float xc[kTcTokens];
+    {
+        const float zero16[16] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f,
+                                  0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        float xs[16];
+        for (int c = 0; c < 4; ++c) {
+            float qv[16];
+            load_qrow16(sb + L::QS, tid, c, qv);
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-            const int jj = c * 16 + u;
-            xc[jj] = __bfloat162float(qs[jj * kTcD + tid]) * s_cq[jj];
-            xp[jj] = 0.f;
-            xs[u] = xc[jj] * s_sx[jj];
+            for (int u = 0; u < 16; ++u) xc[c * 16 + u] = qv[u] * s_cq[c * 16 + u];
+            st_row16(sb + L::XT, tid, c * 16, &xc[c * 16]);
+            tc::tmem_st16(tl + T_XP + c * 16, zero16);
         }
-        st_row16(sb + L::XT, tid, c * 16, xs);
+        tc::tmem_wait_st();
     }
     fence_proxy_async_smem();
     tc::fence_before_sync();
@@ -433,18 +479,23 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
                                  tc::sdesc(b_xt + kk * 2048, 8192, 1024), IDESC_Z1, kk > 0);
             }
         }
-        // P^T = W o S^T  -> bf16, MN-major tile of MG rows
+        // P^T = W o S^T  -> fp16, MN-major tile of MG rows
         if (!mbar_wait_bounded(bar_s, ph, kTcWaitProbes)) ok = false;
         tc::fence_after_sync();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            float sv[16], wv[16];
+        for (int c = 0; c < 4; c += 2) {
+            float sv[32], wv[32];
             tc::tmem_ld16(tl + T_S + c * 16, sv);
+            tc::tmem_ld16(tl + T_S + c * 16 + 16, sv + 16);
             tc::tmem_ld16(tl + T_W + c * 16, wv);
+            tc::tmem_ld16(tl + T_W + c * 16 + 16, wv + 16);
             tc::tmem_wait_ld();
 #pragma unroll
-            for (int u = 0; u < 16; ++u) sv[u] *= wv[u];
-            if (s_owner) st_row16(b_pt, key, c * 16, sv);
+            for (int u = 0; u < 32; ++u) sv[u] *= wv[u];
+            if (s_owner) {
+                st_row16(b_pt, key, c * 16, sv);
+                st_row16(b_pt, key, c * 16 + 16, sv + 16);
+            }
         }
         fence_proxy_async_smem();
         tc::fence_before_sync();
@@ -475,24 +526,31 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
             const float w = P.omega[it];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                float z1[16], z3[16];
+                float z1[16], z3[16], xp[16], qv[16];
                 tc::tmem_ld16(tl + T_Z1 + c * 16, z1);
                 tc::tmem_ld16(tl + T_Z3 + c * 16, z3);
+                tc::tmem_ld16(tl + T_XP + c * 16, xp);
+                load_qrow16(sb + L::QS, tid, c, qv);
+                float cq[16], c1[16], c3[16];
+                ld_f32x16(s_cq + c * 16, cq);
+                ld_f32x16(s_c1 + c * 16, c1);
+                ld_f32x16(s_c3 + c * 16, c3);
                 tc::tmem_wait_ld();
-                float xs[16];
+                float xn[16];
 #pragma unroll
                 for (int u = 0; u < 16; ++u) {
                     const int jj = c * 16 + u;
-                    // (q - A x)/d = q/d - (b H_s x + intra)/d - (lambda/d) x, scales undone
-                    const float r = __bfloat162float(qs[jj * kTcD + tid]) * s_cq[jj] -
-                                    s_c1[jj] * z1[u] - s_c3[jj] * z3[u] - s_cl[jj] * xc[jj];
-                    const float xn = fmaf(w, r + xc[jj] - xp[jj], xp[jj]);
-                    xp[jj] = xc[jj];
-                    xc[jj] = xn;
-                    xs[u] = xn * s_sx[jj];
+                    // (q - A x)/d, scaled: cq q - c1 (H_s x~) - c3 (intra x~) - (lambda/d) x~
+                    const float r = fmaf(cq[u], qv[u],
+                                         -fmaf(c1[u], z1[u], fmaf(c3[u], z3[u], cl * xc[jj])));
+                    xn[u] = fmaf(w, r + xc[jj] - xp[u], xp[u]);
                 }
-                st_row16(sb + L::XT, tid, c * 16, xs);
+                tc::tmem_st16(tl + T_XP + c * 16, &xc[c * 16]);
+#pragma unroll
+                for (int u = 0; u < 16; ++u) xc[c * 16 + u] = xn[u];
+                st_row16(sb + L::XT, tid, c * 16, xn);
             }
+            tc::tmem_wait_st();
             fence_proxy_async_smem();
             tc::fence_before_sync();
             ok = __syncthreads_and(ok);
@@ -501,16 +559,16 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
             __nv_bfloat16 *orow = o + (tok0 + j0) * kTcD + tid;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                float z1[16], z3[16];
+                float z1[16], z3[16], o1[16], o3[16];
                 tc::tmem_ld16(tl + T_Z1 + c * 16, z1);
                 tc::tmem_ld16(tl + T_Z3 + c * 16, z3);
+                ld_f32x16(s_o1 + c * 16, o1);
+                ld_f32x16(s_o3 + c * 16, o3);
                 tc::tmem_wait_ld();
 #pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const int jj = c * 16 + u;
-                    const float val = fmaf(s_o1[jj], z1[u], s_o3[jj] * z3[u]);
-                    orow[(size_t)jj * kTcD] = __float2bfloat16_rn(val);
-                }
+                for (int u = 0; u < 16; ++u)
+                    orow[(size_t)(c * 16 + u) * kTcD] =
+                        __float2bfloat16_rn(fmaf(o1[u], z1[u], o3[u] * z3[u]));
             }
         }
     }
