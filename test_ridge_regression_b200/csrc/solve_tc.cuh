@@ -61,7 +61,9 @@ struct TcSmem {
     static constexpr uint32_t RED = ELL + 8 * MG + 8 * (kTcThreads / 32);  // float[8] reductions
     static constexpr uint32_t NRM = RED + 32;                 // norm terms: u, E, X, Gjj [4][MG]
     static constexpr uint32_t UPART = NRM + 16 * MG;          // [4 warps][MG] partial sums of u
-    static constexpr uint32_t BARS = UPART + 16 * MG;
+    static constexpr uint32_t QPART = UPART + 16 * MG;        // [4 warps][64] partial |q_j|^2
+    static constexpr uint32_t DEC = QPART + 16 * kTcTokens;   // l2, b, beta^2: [3][MG] floats
+    static constexpr uint32_t BARS = DEC + 12 * MG;
     static constexpr uint32_t TBASE = BARS + 8 * 8;
     static constexpr uint32_t END = TBASE + 16;
     static constexpr size_t bytes = END + 1024;               // + alignment slack
@@ -235,6 +237,16 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         tc::tmem_relinquish();
     }
     chunk_log_prefix(beta + tok0, MG, ell, wtot);
+    // decays of every position: l2_t = l_t log2(e) (fp32, so w_ti = exp2(l2_t - l2_i)),
+    // b_t = exp(l_t), beta_t^2 (from the double prefix)
+    float *s_l2 = reinterpret_cast<float *>(sm + L::DEC);
+    float *s_bt = s_l2 + MG, *s_beta2 = s_bt + MG;
+    if (tid < MG) {
+        s_l2[tid] = (float)(ell[tid] * 1.4426950408889634);
+        s_bt[tid] = decay_exp(ell[tid]);
+        const float bt = decay_exp(tid == 0 ? ell[0] : ell[tid] - ell[tid - 1]);
+        s_beta2[tid] = bt * bt;
+    }
     bool ok = mbar_wait_bounded(bar_load, 0, kTcWaitProbes);
     ok = mbar_wait_bounded(bar_v, 0, kTcWaitProbes) && ok;
     // keys and values: bf16 -> fp16 in place, scaled below 1
@@ -331,7 +343,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
                 for (int u = 0; u < 16; ++u) {
                     const int i = cb + u;
                     if (i <= key) {
-                        const float w = decay_exp(ell[key] - ell[i]);
+                        const float w = exp2f(s_l2[key] - s_l2[i]);
                         const float gi = g[u] * gs;
                         xs = fmaf(w, s_u[i], xs);
                         if (i < key) es = fmaf(w * gi, gi, es);
@@ -352,14 +364,31 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         const float hs2 = (red[4] + red[5] + red[6] + red[7]) * ldexpf(1.f, -2 * eHexp);
         float R = 0.f;
         for (int j = 0; j < MG; ++j) {
-            const float bj = decay_exp(j == 0 ? ell[0] : ell[j] - ell[j - 1]);
-            R = fmaf(bj * bj, R, fmaf(2.f, s_E[j], s_G[j] * s_G[j]));
+            R = fmaf(s_beta2[j], R, fmaf(2.f, s_E[j], s_G[j] * s_G[j]));
             if (j >= j0) {
-                const float b = decay_exp(ell[j]);
+                const float b = s_bt[j];
                 const float n2 = fmaf(b * b, hs2, fmaf(2.f * b, s_X[j], R));
                 s_n[j - j0] = sqrtf(fmaxf(n2, 0.f));
             }
         }
+    }
+    // q column of this thread (token-major tile), kept packed for the transpose
+    // below; |q_j|^2 = sum_d q_j[d]^2 by a reduce-scatter over the warp
+    uint32_t qcol[kTcTokens / 2];
+    {
+        float sq[kTcTokens];
+#pragma unroll
+        for (int jj = 0; jj < kTcTokens; jj += 2) {
+            const __nv_bfloat16 lo = qs[jj * kTcD + tid], hi = qs[(jj + 1) * kTcD + tid];
+            qcol[jj / 2] = (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+            const float a0 = __bfloat162float(lo), a1 = __bfloat162float(hi);
+            sq[jj] = a0 * a0;
+            sq[jj + 1] = a1 * a1;
+        }
+        reduce_scatter32<kTcTokens>(sq, lane);
+        float *qpart = reinterpret_cast<float *>(sm + L::QPART);
+        qpart[warp * kTcTokens + 2 * lane] = sq[0];
+        qpart[warp * kTcTokens + 2 * lane + 1] = sq[1];
     }
     __syncthreads();
     if (tid < kTcTokens) {
@@ -367,12 +396,10 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         const float nj = s_n[j];
         norms[tok0 + j0 + j] = nj;
         const float invd = nj > 0.f ? 1.f / (P.half_1p2a * nj) : 0.f;
-        const float b = decay_exp(ell[j0 + j]);
-        float qq = 0.f;
-        for (int d = 0; d < kTcD; ++d) {
-            const float x = __bfloat162float(qs[j * kTcD + ((d + j) & (kTcD - 1))]);
-            qq = fmaf(x, x, qq);
-        }
+        const float b = s_bt[j0 + j];
+        const float *qpart = reinterpret_cast<const float *>(sm + L::QPART);
+        const float qq = qpart[j] + qpart[kTcTokens + j] + qpart[2 * kTcTokens + j] +
+                         qpart[3 * kTcTokens + j];
         // every Chebyshev iterate obeys ||x|| <= ||q|| (1+2a) / (a d): the iterate is
         // kept as x~ = sx x with sx a power of two that puts ||x~|| below 2^12
         const float xb = sqrtf(qq) * invd * (2.f * P.half_1p2a / P.a);
@@ -390,19 +417,10 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
 
     // q^T: transpose the token-major q tile in place into [128 d][64 tokens]
     // (128B-swizzled rows) so that thread d reads 8 tokens per 16-byte load
-    {
-        uint32_t qv[kTcTokens / 2];
 #pragma unroll
-        for (int jj = 0; jj < kTcTokens; jj += 2) {
-            const __nv_bfloat16 lo = qs[jj * kTcD + tid], hi = qs[(jj + 1) * kTcD + tid];
-            qv[jj / 2] = (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
-        }
-        __syncthreads();
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch)
-            st_shared_v4(sb + L::QS + tid * 128u + ((ch ^ tid) & 7u) * 16u, qv[4 * ch],
-                         qv[4 * ch + 1], qv[4 * ch + 2], qv[4 * ch + 3]);
-    }
+    for (int ch = 0; ch < 8; ++ch)
+        st_shared_v4(sb + L::QS + tid * 128u + ((ch ^ tid) & 7u) * 16u, qcol[4 * ch],
+                     qcol[4 * ch + 1], qcol[4 * ch + 2], qcol[4 * ch + 3]);
     const float cl = 2.f * P.a / (1.f + 2.f * P.a);   // lambda / d for every token with H != 0
 
     // W^T rows: W[i][j] = w_{ji} = exp(l_j - l_i) for i <= j, else 0
@@ -413,7 +431,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
                 const int j = j0 + c * 16 + u;
-                wv[u] = (s_owner && key <= j) ? decay_exp(ell[j] - ell[key]) : 0.f;
+                wv[u] = (s_owner && key <= j) ? exp2f(s_l2[j] - s_l2[key]) : 0.f;
             }
             tc::tmem_st16(tl + T_W + c * 16, wv);
         }
