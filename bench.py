@@ -71,60 +71,90 @@ def flops_per_head_token(D, C, r):
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+    """Samples the SM clock and the clock-event (throttle) reasons of the bench GPU
+    during a timed region: NVML polled every millisecond from a thread (reads
+    only), with nvidia-smi at 200 ms as a fallback."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
+    def __init__(self, cuda_index: int):
+        self.cuda_index = cuda_index
+        self.samples = []          # (sm_mhz, reasons bitmask)
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._proc = None
+
+    def _pci_id(self):
+        import torch
+        p = torch.cuda.get_device_properties(self.cuda_index)
+        return f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByPciBusId(self._pci_id().encode())
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+
+            def poll():
+                while not self._stop.is_set():
+                    try:
+                        mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                        why = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.samples.append((float(mhz), int(why)))
+                    except Exception:
+                        pass
+                    self._stop.wait(0.001)
+            self._thread = threading.Thread(target=poll, daemon=True)
+            self._thread.start()
         except Exception:
-            self.proc = None
+            self._start_smi()
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _start_smi(self):
+        try:
+            self._proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self._pci_id()}",
+                 "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.active",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+
+            def read():
+                for line in self._proc.stdout:
+                    parts = [x.strip() for x in line.split(",")]
+                    try:
+                        self.max_mhz = float(parts[1])
+                        self.samples.append((float(parts[0]), int(parts[2], 16)))
+                    except (ValueError, IndexError):
+                        pass
+            self._thread = threading.Thread(target=read, daemon=True)
+            self._thread.start()
+        except Exception:
+            self._proc = None
 
     def __exit__(self, *a):
-        if self.proc is not None:
-            self.proc.terminate()
+        self._stop.set()
+        if self._proc is not None:
+            self._proc.terminate()
             try:
-                self.proc.wait(timeout=5)
+                self._proc.wait(timeout=5)
             except Exception:
-                self.proc.kill()
+                self._proc.kill()
+        if self._thread is not None:
+            self._thread.join(timeout=2)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [x.strip() for x in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for nm, val in zip(names, parts[5:9]):
-                if val.lower() == "active":
-                    reasons.add(nm)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"]}
+        mhz = [m for m, _ in self.samples]
+        mask = 0
+        for _, w in self.samples:
+            mask |= w
+        reasons = sorted(name for bit, name in self.REASONS.items() if mask & bit)
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(mhz), "source": "nvml" if self._proc is None else "nvidia-smi"}
 
 
 def cpu_threads():
@@ -355,12 +385,17 @@ def main():
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1) ----
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        nheads = oracle_calibrate(w, 15.0, q, k, v, beta)
-        val, dt, threads = oracle_sample(w, nheads, q, k, v, beta)
+        nheads = oracle_calibrate(w, 10.0, q, k, v, beta)
+        vals, total, reps = [], 0.0, 0
+        while total < 10.0 and reps < 50:   # the whole sample, repeated to about 10 s
+            val, dt, threads = oracle_sample(w, nheads, q, k, v, beta)
+            vals.append(val)
+            total += dt
+            reps += 1
         result["cpu_baseline"] = {
-            "value": val, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"{nheads} whole heads x {w.T} tokens of the workload ({dt:.1f} s, "
-                      f"float64 C oracle, OpenMP over heads)"}
+            "value": statistics.mean(vals), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{nheads} whole heads x {w.T} tokens of the workload, {reps} runs, "
+                      f"{total:.1f} s (float64 C oracle, OpenMP over heads)"}
     if gka.device_status() != 0:
         raise RuntimeError("device status error")
     if rank == 0:

@@ -132,43 +132,61 @@ __device__ __forceinline__ int lp_exponent(float bound) {
     return e < -120 ? -120 : (e > 120 ? 120 : e);
 }
 
+constexpr int kScanTile = 256;   // chunks whose scales are prepared per pass
+
 __global__ void __launch_bounds__(256)
 k_state_scan(float *__restrict__ states, const float *__restrict__ decay,
              float *__restrict__ final_state, __half *__restrict__ states_lp,
              const float *__restrict__ bound_inc, int *__restrict__ state_exp, int N, int DD2,
              bool write_fp32) {
+    __shared__ float s_dec[kScanTile], s_scale[2][kScanTile];
+    __shared__ float s_bound[2];
     const int bh = blockIdx.y;
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
-    if (e >= DD2) return;
+    const bool active = e < DD2;
     float *base = states + (size_t)bh * (N + 1) * DD2 + e;
     __half *lbase = states_lp ? states_lp + (size_t)bh * N * DD2 + e : nullptr;
     const int mat = e < DD2 / 2 ? 0 : 1;          // H or M element
-    const bool writes_exp = (e == 0) || (e == DD2 / 2);
     const float *dec = decay + (size_t)bh * N;
-    float s = 0.f, bound = 0.f;
-    base[0] = 0.f;
-    // one step of the scan: chunk-start copy, then S_{n+1} = b_n S_n + dS_n
-    auto step = [&](int n, float dl) {
-        if (lbase) {
-            // low-precision copy of the chunk-start state, scaled by 2^e from its norm bound
-            const int ex = lp_exponent(bound);
-            lbase[(size_t)n * DD2] = __float2half_rn(ldexpf(s, ex));
-            if (writes_exp) state_exp[((size_t)bh * N + n) * 2 + mat] = ex;
-            bound = fmaf(dec[n], bound, bound_inc[((size_t)bh * N + n) * 2 + mat]);
+    if (threadIdx.x < 2) s_bound[threadIdx.x] = 0.f;
+    float s = 0.f;
+    if (active) base[0] = 0.f;
+    for (int n0 = 0; n0 < N; n0 += kScanTile) {
+        const int nt = min(kScanTile, N - n0);
+        __syncthreads();
+        for (int i = threadIdx.x; i < nt; i += blockDim.x) s_dec[i] = dec[n0 + i];
+        if (lbase && threadIdx.x < 2) {
+            // power-of-two scales of the chunk-start states from the running bound
+            // ||S_n||_F <= bound_n (one thread per matrix; same for every block of bh)
+            const int m = threadIdx.x;
+            float bound = s_bound[m];
+            for (int i = 0; i < nt; ++i) {
+                const int ex = lp_exponent(bound);
+                s_scale[m][i] = ldexpf(1.f, ex);
+                if (blockIdx.x == 0) state_exp[((size_t)bh * N + n0 + i) * 2 + m] = ex;
+                bound = fmaf(dec[n0 + i], bound, bound_inc[((size_t)bh * N + n0 + i) * 2 + m]);
+            }
+            s_bound[m] = bound;
         }
-        s = fmaf(dec[n], s, dl);
-        if (write_fp32) base[(size_t)(n + 1) * DD2] = s;
-    };
-    int n = 0;
-    for (; n + 8 <= N; n += 8) {   // loads of a batch issued before its dependent stores
-        float dl[8];
+        __syncthreads();
+        if (!active) continue;
+        auto step = [&](int i, float dl) {
+            const int n = n0 + i;
+            if (lbase) lbase[(size_t)n * DD2] = __float2half_rn(s * s_scale[mat][i]);
+            s = fmaf(s_dec[i], s, dl);
+            if (write_fp32) base[(size_t)(n + 1) * DD2] = s;
+        };
+        int i = 0;
+        for (; i + 8 <= nt; i += 8) {   // loads of a batch issued before its dependent stores
+            float dl[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) dl[u] = base[(size_t)(n + u + 1) * DD2];
+            for (int u = 0; u < 8; ++u) dl[u] = base[(size_t)(n0 + i + u + 1) * DD2];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) step(n + u, dl[u]);
+            for (int u = 0; u < 8; ++u) step(i + u, dl[u]);
+        }
+        for (; i < nt; ++i) step(i, base[(size_t)(n0 + i + 1) * DD2]);
     }
-    for (; n < N; ++n) step(n, base[(size_t)(n + 1) * DD2]);
-    if (final_state) final_state[(size_t)bh * DD2 + e] = s;
+    if (active && final_state) final_state[(size_t)bh * DD2 + e] = s;
 }
 
 // ---------------------------------------------------------------------------

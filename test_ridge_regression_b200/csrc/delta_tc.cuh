@@ -32,7 +32,8 @@ struct DeltaSmem {
     static constexpr uint32_t VT = KT + C * 256;      // 2 x [C][64] values
     static constexpr uint32_t WH = VT + C * 256;      // 2 x [C][64] (w k)_hi
     static constexpr uint32_t WL = WH + C * 256;      // 2 x [C][64] (w k)_lo
-    static constexpr uint32_t ELL = WL + C * 256;     // double[C] cumulative logs
+    static constexpr uint32_t STAGE = WL + C * 256;   // 2 x [128][32] fp32 store staging (swizzled)
+    static constexpr uint32_t ELL = STAGE + 32768;    // double[C] cumulative logs
     static constexpr uint32_t RED = ELL + 8 * C + 8 * (kTcThreads / 32);
     static constexpr uint32_t BARS = RED + 64;
     static constexpr uint32_t TBASE = BARS + 32;
@@ -41,10 +42,15 @@ struct DeltaSmem {
     static constexpr size_t bytes = END + 1024 > 81920 ? END + 1024 : 81920;
 };
 
+struct DeltaMaps {
+    CUtensorMap k, v;    // [B*H*T][128] bf16, box 64 x 64, 128B swizzle
+    CUtensorMap out;     // fp32 states [B*H*(N+1)*2*128][128], box 32 x 128, 128B swizzle
+};
+
 // grid (N, B*H), block 128.
 template <int C>
 __global__ void __launch_bounds__(kTcThreads, 1)
-k_chunk_delta_tc(const __grid_constant__ TcMaps maps, const float *__restrict__ beta,
+k_chunk_delta_tc(const __grid_constant__ DeltaMaps maps, const float *__restrict__ beta,
                  float *__restrict__ states, float *__restrict__ decay,
                  float *__restrict__ bound_inc, int T, int N, int *__restrict__ timeout_flag) {
     using L = DeltaSmem<C>;
@@ -169,29 +175,41 @@ k_chunk_delta_tc(const __grid_constant__ TcMaps maps, const float *__restrict__ 
             bound_inc[((size_t)bh * N + n) * 2] = red[8] + red[9] + red[10] + red[11];
             bound_inc[((size_t)bh * N + n) * 2 + 1] = red[12] + red[13] + red[14] + red[15];
         }
-        // row d of dH and dM (thread d = TMEM lane d) to state slot n + 1
+        // row d of dH and dM (thread d = TMEM lane d) -> swizzled staging -> TMA store
+        // into state slot n + 1, 64 columns (two 32-column boxes) per round
         const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-        float *out = states + ((size_t)bh * (N + 1) + n + 1) * 2 * D * D + (size_t)tid * D;
         const float uh = 1.f / (sK * sK), um = 1.f / (sV * sK);
-#pragma unroll
-        for (int m = 0; m < 2; ++m) {
+        const int orow = (int)(((size_t)bh * (N + 1) + n + 1) * 2 * D);
+#pragma unroll 1
+        for (int round = 0; round < 4; ++round) {
+            const int m = round >> 1, cb0 = (round & 1) * 64;
             const float us = m == 0 ? uh : um;
 #pragma unroll
-            for (int cb = 0; cb < 128; cb += 32) {
+            for (int bx = 0; bx < 2; ++bx) {
                 float v0[16], v1[16];
-                tc::tmem_ld16(tl + m * 128 + cb, v0);
-                tc::tmem_ld16(tl + m * 128 + cb + 16, v1);
+                tc::tmem_ld16(tl + m * 128 + cb0 + bx * 32, v0);
+                tc::tmem_ld16(tl + m * 128 + cb0 + bx * 32 + 16, v1);
                 tc::tmem_wait_ld();
-                float4 *dst = reinterpret_cast<float4 *>(out + (size_t)m * D * D + cb);
+                const uint32_t rowb = sb + L::STAGE + bx * 16384 + tid * 128;
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    dst[q4] = make_float4(v0[4 * q4] * us, v0[4 * q4 + 1] * us, v0[4 * q4 + 2] * us,
-                                          v0[4 * q4 + 3] * us);
-                    dst[4 + q4] = make_float4(v1[4 * q4] * us, v1[4 * q4 + 1] * us,
-                                              v1[4 * q4 + 2] * us, v1[4 * q4 + 3] * us);
+                for (int j = 0; j < 8; ++j) {
+                    const float *vv = j < 4 ? v0 + 4 * j : v1 + 4 * (j - 4);
+                    st_shared_v4(rowb + ((j ^ tid) & 7) * 16, __float_as_uint(vv[0] * us),
+                                 __float_as_uint(vv[1] * us), __float_as_uint(vv[2] * us),
+                                 __float_as_uint(vv[3] * us));
                 }
             }
+            fence_proxy_async_smem();
+            __syncthreads();
+            if (tid == 0) {
+                tc::tma_store_2d(&maps.out, cb0, orow + m * D, sm + L::STAGE);
+                tc::tma_store_2d(&maps.out, cb0 + 32, orow + m * D, sm + L::STAGE + 16384);
+                tc::bulk_commit();
+                tc::bulk_wait_read0();
+            }
+            __syncthreads();
         }
+        if (tid == 0) tc::bulk_wait0();
     } else if (tid == 0) {
         atomicExch(timeout_flag, 1);
         tc::commit(bar_mma);   // drain: a second arrival after whatever is still in flight

@@ -210,12 +210,14 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 // 2-D map over a row-major [rows][128] 16-bit array: boxes of 64 columns
 // (128 bytes) x 64 rows, 128-byte swizzle (the tensor-core operand layout).
-static int rows128_map(CUtensorMap *m, const void *base, uint64_t rows, CUtensorMapDataType ty) {
+static int rows128_map(CUtensorMap *m, const void *base, uint64_t rows, CUtensorMapDataType ty,
+                       uint32_t box_cols = 64, uint32_t box_rows = 64) {
     auto enc = tensor_map_encoder();
     if (!enc) return cuda_fail(cudaErrorNotSupported);
     cuuint64_t dims[2] = {128, rows};
-    cuuint64_t strides[1] = {128 * 2};
-    cuuint32_t box[2] = {64, 64};
+    const uint32_t esize = ty == CU_TENSOR_MAP_DATA_TYPE_FLOAT32 ? 4 : 2;
+    cuuint64_t strides[1] = {128 * esize};
+    cuuint32_t box[2] = {box_cols, box_rows};
     cuuint32_t es[2] = {1, 1};
     CUresult r = enc(m, ty, 2, const_cast<void *>(base), dims,
                      strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -250,18 +252,24 @@ static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
         return rc;
     cudaError_t e;
 
+    DeltaMaps dmaps;
+    dmaps.k = maps.k;
+    dmaps.v = maps.v;
+    if (int rc = rows128_map(&dmaps.out, states, (uint64_t)BH * (N + 1) * 2 * D,
+                             CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 32, 128))
+        return rc;
     if (C == 64) {
         if ((e = set_smem(k_chunk_delta_tc<64>, DeltaSmem<64>::bytes)) != cudaSuccess)
             return cuda_fail(e);
         ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
         k_chunk_delta_tc<64><<<dim3(N, BH), kTcThreads, DeltaSmem<64>::bytes, s>>>(
-            maps, beta, states, decay, bound_inc, T, N, flag);
+            dmaps, beta, states, decay, bound_inc, T, N, flag);
     } else {
         if ((e = set_smem(k_chunk_delta_tc<128>, DeltaSmem<128>::bytes)) != cudaSuccess)
             return cuda_fail(e);
         ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
         k_chunk_delta_tc<128><<<dim3(N, BH), kTcThreads, DeltaSmem<128>::bytes, s>>>(
-            maps, beta, states, decay, bound_inc, T, N, flag);
+            dmaps, beta, states, decay, bound_inc, T, N, flag);
     }
     if (int rc = check_launch()) return rc;
 
