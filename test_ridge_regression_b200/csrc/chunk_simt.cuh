@@ -139,7 +139,7 @@ k_state_scan(float *__restrict__ states, const float *__restrict__ decay,
              float *__restrict__ final_state, __half *__restrict__ states_lp,
              const float *__restrict__ bound_inc, int *__restrict__ state_exp, int N, int DD2,
              bool write_fp32) {
-    __shared__ float s_dec[kScanTile], s_scale[2][kScanTile];
+    __shared__ float s_dec[kScanTile], s_scale[2][kScanTile], s_binc[2][kScanTile];
     __shared__ float s_bound[2];
     const int bh = blockIdx.y;
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
@@ -155,6 +155,10 @@ k_state_scan(float *__restrict__ states, const float *__restrict__ decay,
         const int nt = min(kScanTile, N - n0);
         __syncthreads();
         for (int i = threadIdx.x; i < nt; i += blockDim.x) s_dec[i] = dec[n0 + i];
+        if (lbase)
+            for (int i = threadIdx.x; i < 2 * nt; i += blockDim.x)
+                s_binc[i & 1][i >> 1] = bound_inc[((size_t)bh * N + n0) * 2 + i];
+        __syncthreads();
         if (lbase && threadIdx.x < 2) {
             // power-of-two scales of the chunk-start states from the running bound
             // ||S_n||_F <= bound_n (one thread per matrix; same for every block of bh)
@@ -164,7 +168,7 @@ k_state_scan(float *__restrict__ states, const float *__restrict__ decay,
                 const int ex = lp_exponent(bound);
                 s_scale[m][i] = ldexpf(1.f, ex);
                 if (blockIdx.x == 0) state_exp[((size_t)bh * N + n0 + i) * 2 + m] = ex;
-                bound = fmaf(dec[n0 + i], bound, bound_inc[((size_t)bh * N + n0 + i) * 2 + m]);
+                bound = fmaf(s_dec[i], bound, s_binc[m][i]);
             }
             s_bound[m] = bound;
         }

@@ -43,6 +43,7 @@
 namespace gka {
 
 constexpr int kTcThreads = 128;
+constexpr int kSolveThreads = 256;   // solve kernel: two warpgroups
 constexpr int kTcTokens = 64;     // tokens per CTA
 constexpr int kTcD = 128;         // head dimension of the tensor-core path
 constexpr uint32_t kTcWaitProbes = 1u << 22;
@@ -58,9 +59,10 @@ struct TcSmem {
     static constexpr uint32_t QS = PT + MG * 128;            // q: [64][128] bf16, then q^T
     static constexpr uint32_t SCAL = QS + 16384;             // per-token scalars
     static constexpr uint32_t ELL = SCAL + 8 * 4 * kTcTokens; // double[MG] cumulative logs
-    static constexpr uint32_t RED = ELL + 8 * MG + 8 * (kTcThreads / 32);  // float[8] reductions
-    static constexpr uint32_t NRM = RED + 32;                 // norm terms: u, E, X, Gjj [4][MG]
-    static constexpr uint32_t UPART = NRM + 16 * MG;          // [4 warps][MG] partial sums of u
+    static constexpr uint32_t RED = ELL + 8 * MG + 8 * (kSolveThreads / 32);  // float[16] reductions
+    static constexpr uint32_t NRM = RED + 64;                 // norm terms: u, E, X, Gjj [4][MG]
+    static constexpr uint32_t NRM2 = NRM + 16 * MG;           // second warpgroup's E, X [2][MG]
+    static constexpr uint32_t UPART = NRM2 + 8 * MG;          // [4 lane quarters][MG] partial u
     static constexpr uint32_t QPART = UPART + 16 * MG;        // [4 warps][64] partial |q_j|^2
     static constexpr uint32_t DEC = QPART + 16 * kTcTokens;   // l2, b, beta^2: [3][MG] floats
     static constexpr uint32_t BARS = DEC + 12 * MG;
@@ -120,11 +122,11 @@ __device__ __forceinline__ void load_qrow16(uint32_t tile, uint32_t row, int c, 
 }
 
 // In place: bf16 tile of `bytes` bytes -> fp16, scaled so that every |value| < 1.
-// Returns the scale.  Every thread of the block calls it.
+// Returns the scale.  Every thread of the block calls it (red: blockDim/32 floats).
 __device__ __forceinline__ float tile_bf16_to_f16_scaled(uint8_t *tile, int bytes, float *red) {
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, nthr = blockDim.x, nw = nthr >> 5;
     float mx = 0.f;
-    for (int c = tid * 16; c < bytes; c += kTcThreads * 16) {
+    for (int c = tid * 16; c < bytes; c += nthr * 16) {
         const uint4 u = *reinterpret_cast<const uint4 *>(tile + c);
         const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&u);
 #pragma unroll
@@ -135,9 +137,10 @@ __device__ __forceinline__ float tile_bf16_to_f16_scaled(uint8_t *tile, int byte
     __syncthreads();
     if ((tid & 31) == 0) red[tid >> 5] = mx;
     __syncthreads();
-    mx = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    mx = 0.f;
+    for (int w = 0; w < nw; ++w) mx = fmaxf(mx, red[w]);
     const float sc = inv_pow2_above(mx);
-    for (int c = tid * 16; c < bytes; c += kTcThreads * 16) {
+    for (int c = tid * 16; c < bytes; c += nthr * 16) {
         uint4 u = *reinterpret_cast<const uint4 *>(tile + c);
         const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&u);
         uint4 w;
@@ -180,13 +183,17 @@ __device__ __forceinline__ void reduce_scatter32(float (&v)[N], int lane) {
 }
 
 // grid (N, B*H); group g = `group` of every chunk; MG = 64 * (group + 1).
+// 8 warps: warpgroup wg (warps 4wg..4wg+3) owns tokens 32wg..32wg+31 of the
+// group; warp w reads TMEM lane quarter w % 4, so thread (wg, d) owns element d
+// of the iterates of its 32 tokens.
 template <int MG>
-__global__ void __launch_bounds__(kTcThreads, 2)
+__global__ void __launch_bounds__(kSolveThreads, 2)
 k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__restrict__ q,
                  const float *__restrict__ beta, float *__restrict__ norms,
                  const int *__restrict__ state_exp, __nv_bfloat16 *__restrict__ o, int T, int N,
                  int C, int group, const ChebParams P, int *__restrict__ timeout_flag) {
     using L = TcSmem<MG>;
+    constexpr int HALF = MG / 2;       // keys per warpgroup in the norm reductions
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -205,6 +212,9 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     uint32_t *tbase = reinterpret_cast<uint32_t *>(sm + L::TBASE);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int wg = warp >> 2, quarter = warp & 3;
+    const int d = quarter * 32 + lane;        // head-dimension row = TMEM lane of this thread
+    const int tcol = wg * 32;                 // first token (TMEM column) of this thread
     const int n = blockIdx.x, bh = blockIdx.y;
     const int j0 = group * kTcTokens;                      // first token of the group in the chunk
     const size_t tok0 = (size_t)bh * T + (size_t)n * C;    // first token of the chunk
@@ -260,7 +270,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     ok = __syncthreads_and(ok);
     tc::fence_after_sync();
     const uint32_t tmem = *tbase;
-    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);   // this warp's TMEM lane quarter
+    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);   // this warp's lane quarter
     // TMEM columns: Z1 | S, then Z3 (S is consumed before MMA3 writes Z3) | W | x_prev
     const uint32_t T_Z1 = 0, T_S = 64, T_Z3 = 64, T_W = 128, T_XP = 192;
     const uint32_t a_hm = sb + L::HM, a_kt = sb + L::KT, a_vt = sb + L::VT, b_xt = sb + L::XT,
@@ -269,7 +279,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     // rows of S (keys) held by this thread: M = 64 puts key 16w + l in lane
     // 32w + l (l < 16); M = 128 puts key t in lane t.
     const bool s_owner = (MG == 128) || (lane < 16);
-    const int key = (MG == 128) ? tid : warp * 16 + lane;
+    const int key = (MG == 128) ? d : quarter * 16 + lane;
 
     // ---- per-token ||H_j||_F (ai.info, Methodology: closed form through the
     // key Gram matrix).  Zn = H_s K^T gives u_i = k_i^T H_s k_i, G = K K^T the
@@ -287,12 +297,13 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         tc::commit(bar_n);
     }
     float *s_u = reinterpret_cast<float *>(sm + L::NRM);
-    float *s_E = s_u + MG, *s_X = s_E + MG, *s_G = s_X + MG;
+    float *s_E = s_u + MG, *s_X = s_E + MG, *s_G = s_X + MG;   // [MG] each; E and X: wg 0 part
+    float *s_E1 = reinterpret_cast<float *>(sm + L::NRM2), *s_X1 = s_E1 + MG;   // wg 1 part
     float *upart = reinterpret_cast<float *>(sm + L::UPART);
     {
         // ||H_s||_F^2 from the (scaled) fp16 copy
         float hs = 0.f;
-        for (int c = tid * 16; c < 32768; c += kTcThreads * 16) {
+        for (int c = tid * 16; c < 32768; c += kSolveThreads * 16) {
             const uint4 u4 = *reinterpret_cast<const uint4 *>(sm + L::HM + c);
             const __half *e = reinterpret_cast<const __half *>(&u4);
 #pragma unroll
@@ -302,27 +313,30 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
             }
         }
         hs = warp_sum(hs);
-        if (lane == 0) red[4 + warp] = hs;
+        if (lane == 0) red[8 + warp] = hs;
     }
     if (!mbar_wait_bounded(bar_n, 0, kTcWaitProbes)) ok = false;
     tc::fence_after_sync();
     {
-        // u_i: thread d forms k_i[d] (H_s k_i)[d] for every key i, then a sum over d
+        // u_i: thread (wg, d) forms k_i[d] (H_s k_i)[d] for its half of the keys,
+        // then a sum over d (warp reduce-scatter, then the four lane quarters)
         const __half *kt = reinterpret_cast<const __half *>(sm + L::KT);
-        const int hoff = (tid >> 6) * (MG * 64), c = tid & 63;
-        float pv[MG];
+        const int hoff = (d >> 6) * (MG * 64), c = d & 63;
+        float pv[HALF];
 #pragma unroll
-        for (int cb = 0; cb < MG; cb += 16) {
+        for (int cb = 0; cb < HALF; cb += 16) {
             float zn[16];
-            tc::tmem_ld16(tl + cb, zn);
+            tc::tmem_ld16(tl + wg * HALF + cb, zn);
             tc::tmem_wait_ld();
 #pragma unroll
             for (int u = 0; u < 16; ++u)
-                pv[cb + u] = zn[u] * __half2float(kt[hoff + tc::sw128_offset(cb + u, c) / 2]);
+                pv[cb + u] = zn[u] * __half2float(
+                                         kt[hoff + tc::sw128_offset(wg * HALF + cb + u, c) / 2]);
         }
-        reduce_scatter32<MG>(pv, lane);
+        reduce_scatter32<HALF>(pv, lane);
 #pragma unroll
-        for (int s2 = 0; s2 < MG / 32; ++s2) upart[warp * MG + lane * (MG / 32) + s2] = pv[s2];
+        for (int s2 = 0; s2 < HALF / 32; ++s2)
+            upart[quarter * MG + wg * HALF + lane * (HALF / 32) + s2] = pv[s2];
     }
     __syncthreads();
     const float inv_uscale = ldexpf(1.f, -eHexp) / (sK * sK);
@@ -330,65 +344,71 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
                               upart[3 * MG + tid]) * inv_uscale;
     __syncthreads();
     {
-        // row `key` of G: E_key, X_key, G_key,key
+        // row `key` of G over this warpgroup's half of the columns: E, X, G_key,key
         const float gs = 1.f / (sK * sK);
         float es = 0.f, xs = 0.f, gjj = 0.f;
+        bool has_diag = false;
 #pragma unroll
-        for (int cb = 0; cb < MG; cb += 16) {
+        for (int cb = 0; cb < HALF; cb += 16) {
             float g[16];
-            tc::tmem_ld16(tl + 128 + cb, g);
+            tc::tmem_ld16(tl + 128 + wg * HALF + cb, g);
             tc::tmem_wait_ld();
             if (s_owner) {
 #pragma unroll
                 for (int u = 0; u < 16; ++u) {
-                    const int i = cb + u;
+                    const int i = wg * HALF + cb + u;
                     if (i <= key) {
                         const float w = exp2f(s_l2[key] - s_l2[i]);
                         const float gi = g[u] * gs;
                         xs = fmaf(w, s_u[i], xs);
-                        if (i < key) es = fmaf(w * gi, gi, es);
-                        else gjj = gi;
+                        if (i < key) {
+                            es = fmaf(w * gi, gi, es);
+                        } else {
+                            gjj = gi;
+                            has_diag = true;
+                        }
                     }
                 }
             }
         }
         if (s_owner) {
-            s_E[key] = es;
-            s_X[key] = xs;
-            s_G[key] = gjj;
+            (wg == 0 ? s_E : s_E1)[key] = es;
+            (wg == 0 ? s_X : s_X1)[key] = xs;
+            if (has_diag) s_G[key] = gjj;
         }
     }
-    __syncthreads();
-    float *s_n = s_o3;   // per-token norms, then overwritten by the readout coefficient
-    if (tid == 0) {
-        const float hs2 = (red[4] + red[5] + red[6] + red[7]) * ldexpf(1.f, -2 * eHexp);
-        float R = 0.f;
-        for (int j = 0; j < MG; ++j) {
-            R = fmaf(s_beta2[j], R, fmaf(2.f, s_E[j], s_G[j] * s_G[j]));
-            if (j >= j0) {
-                const float b = s_bt[j];
-                const float n2 = fmaf(b * b, hs2, fmaf(2.f * b, s_X[j], R));
-                s_n[j - j0] = sqrtf(fmaxf(n2, 0.f));
-            }
-        }
-    }
-    // q column of this thread (token-major tile), kept packed for the transpose
-    // below; |q_j|^2 = sum_d q_j[d]^2 by a reduce-scatter over the warp
-    uint32_t qcol[kTcTokens / 2];
+    // q column of this thread's tokens (token-major tile), kept packed for the
+    // transpose below; |q_j|^2 = sum_d q_j[d]^2 by a reduce-scatter over the warp
+    uint32_t qcol[16];
     {
-        float sq[kTcTokens];
+        float sq[32];
 #pragma unroll
-        for (int jj = 0; jj < kTcTokens; jj += 2) {
-            const __nv_bfloat16 lo = qs[jj * kTcD + tid], hi = qs[(jj + 1) * kTcD + tid];
+        for (int jj = 0; jj < 32; jj += 2) {
+            const __nv_bfloat16 lo = qs[(tcol + jj) * kTcD + d], hi = qs[(tcol + jj + 1) * kTcD + d];
             qcol[jj / 2] = (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
             const float a0 = __bfloat162float(lo), a1 = __bfloat162float(hi);
             sq[jj] = a0 * a0;
             sq[jj + 1] = a1 * a1;
         }
-        reduce_scatter32<kTcTokens>(sq, lane);
-        float *qpart = reinterpret_cast<float *>(sm + L::QPART);
-        qpart[warp * kTcTokens + 2 * lane] = sq[0];
-        qpart[warp * kTcTokens + 2 * lane + 1] = sq[1];
+        reduce_scatter32<32>(sq, lane);
+        reinterpret_cast<float *>(sm + L::QPART)[quarter * kTcTokens + tcol + lane] = sq[0];
+    }
+    __syncthreads();
+    float *s_n = s_o3;   // per-token norms, then overwritten by the readout coefficient
+    if (tid == 0) {
+        float hs2 = 0.f;
+        for (int w = 0; w < kSolveThreads / 32; ++w) hs2 += red[8 + w];
+        hs2 *= ldexpf(1.f, -2 * eHexp);
+        float R = 0.f;
+        for (int j = 0; j < MG; ++j) {
+            const float E = s_E[j] + s_E1[j], X = s_X[j] + s_X1[j];
+            R = fmaf(s_beta2[j], R, fmaf(2.f, E, s_G[j] * s_G[j]));
+            if (j >= j0) {
+                const float b = s_bt[j];
+                const float n2 = fmaf(b * b, hs2, fmaf(2.f * b, X, R));
+                s_n[j - j0] = sqrtf(fmaxf(n2, 0.f));
+            }
+        }
     }
     __syncthreads();
     if (tid < kTcTokens) {
@@ -415,43 +435,43 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     }
     __syncthreads();
 
-    // q^T: transpose the token-major q tile in place into [128 d][64 tokens]
-    // (128B-swizzled rows) so that thread d reads 8 tokens per 16-byte load
+    // q^T: this thread's tokens of row d, written into the (now free) tile as
+    // [128 d][64 tokens] with 128B-swizzled rows: 8 tokens per 16-byte load later
 #pragma unroll
-    for (int ch = 0; ch < 8; ++ch)
-        st_shared_v4(sb + L::QS + tid * 128u + ((ch ^ tid) & 7u) * 16u, qcol[4 * ch],
+    for (int ch = 0; ch < 4; ++ch)
+        st_shared_v4(sb + L::QS + d * 128u + (((wg * 4 + ch) ^ d) & 7u) * 16u, qcol[4 * ch],
                      qcol[4 * ch + 1], qcol[4 * ch + 2], qcol[4 * ch + 3]);
     const float cl = 2.f * P.a / (1.f + 2.f * P.a);   // lambda / d for every token with H != 0
 
-    // W^T rows: W[i][j] = w_{ji} = exp(l_j - l_i) for i <= j, else 0
+    // W^T rows: W[i][j] = w_{ji} = exp(l_j - l_i) for i <= j, else 0 (this thread's tokens)
     {
         float wv[16];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
-                const int j = j0 + c * 16 + u;
+                const int j = j0 + tcol + c * 16 + u;
                 wv[u] = (s_owner && key <= j) ? exp2f(s_l2[j] - s_l2[key]) : 0.f;
             }
-            tc::tmem_st16(tl + T_W + c * 16, wv);
+            tc::tmem_st16(tl + T_W + tcol + c * 16, wv);
         }
-        tc::tmem_wait_st();
     }
 
-    // x_1 = q / d, x_0 = 0 (scaled by sx): thread d keeps element d of the 64
+    // x_1 = q / d, x_0 = 0 (scaled by sx): thread (wg, d) keeps element d of its 32
     // current iterates in registers and of the previous ones in TMEM
-    float xc[kTcTokens];
+    float xc[32];
     {
         const float zero16[16] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f,
                                   0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        __syncthreads();   // q^T complete
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
             float qv[16];
-            load_qrow16(sb + L::QS, tid, c, qv);
+            load_qrow16(sb + L::QS, d, wg * 2 + c, qv);
 #pragma unroll
-            for (int u = 0; u < 16; ++u) xc[c * 16 + u] = qv[u] * s_cq[c * 16 + u];
-            st_row16(sb + L::XT, tid, c * 16, &xc[c * 16]);
-            tc::tmem_st16(tl + T_XP + c * 16, zero16);
+            for (int u = 0; u < 16; ++u) xc[c * 16 + u] = qv[u] * s_cq[tcol + c * 16 + u];
+            st_row16(sb + L::XT, d, tcol + c * 16, &xc[c * 16]);
+            tc::tmem_st16(tl + T_XP + tcol + c * 16, zero16);
         }
         tc::tmem_wait_st();
     }
@@ -474,8 +494,8 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
                 tc::mma_f16(tmem + T_S,
-                             tc::sdesc(a_kt + (kk >> 2) * (MG * 128) + (kk & 3) * 32, 16, 1024),
-                             tc::sdesc(b_xt + kk * 2048, 8192, 1024), IDESC_S, kk > 0);
+                            tc::sdesc(a_kt + (kk >> 2) * (MG * 128) + (kk & 3) * 32, 16, 1024),
+                            tc::sdesc(b_xt + kk * 2048, 8192, 1024), IDESC_S, kk > 0);
             tc::commit(bar_s);
             if (out_pass) {
                 if (!m_requested) {
@@ -493,26 +513,25 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     tc::mma_f16(tmem + T_Z1,
-                                 tc::sdesc(a_hm + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                                 tc::sdesc(b_xt + kk * 2048, 8192, 1024), IDESC_Z1, kk > 0);
+                                tc::sdesc(a_hm + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                                tc::sdesc(b_xt + kk * 2048, 8192, 1024), IDESC_Z1, kk > 0);
             }
         }
-        // P^T = W o S^T  -> fp16, MN-major tile of MG rows
+        // P^T = W o S^T  -> fp16, MN-major tile of MG rows (this thread's 32 tokens)
         if (!mbar_wait_bounded(bar_s, ph, kTcWaitProbes)) ok = false;
         tc::fence_after_sync();
-#pragma unroll
-        for (int c = 0; c < 4; c += 2) {
+        {
             float sv[32], wv[32];
-            tc::tmem_ld16(tl + T_S + c * 16, sv);
-            tc::tmem_ld16(tl + T_S + c * 16 + 16, sv + 16);
-            tc::tmem_ld16(tl + T_W + c * 16, wv);
-            tc::tmem_ld16(tl + T_W + c * 16 + 16, wv + 16);
+            tc::tmem_ld16(tl + T_S + tcol, sv);
+            tc::tmem_ld16(tl + T_S + tcol + 16, sv + 16);
+            tc::tmem_ld16(tl + T_W + tcol, wv);
+            tc::tmem_ld16(tl + T_W + tcol + 16, wv + 16);
             tc::tmem_wait_ld();
 #pragma unroll
             for (int u = 0; u < 32; ++u) sv[u] *= wv[u];
             if (s_owner) {
-                st_row16(b_pt, key, c * 16, sv);
-                st_row16(b_pt, key, c * 16 + 16, sv + 16);
+                st_row16(b_pt, key, tcol, sv);
+                st_row16(b_pt, key, tcol + 16, sv + 16);
             }
         }
         fence_proxy_async_smem();
@@ -525,7 +544,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
 #pragma unroll
             for (int kk = 0; kk < MG / 16; ++kk)
                 tc::mma_f16(tmem + T_Z3, tc::sdesc(a3 + kk * 2048, MG * 128, 1024),
-                             tc::sdesc(b_pt + kk * 2048, 8192, 1024), IDESC_Z3, kk > 0);
+                            tc::sdesc(b_pt + kk * 2048, 8192, 1024), IDESC_Z3, kk > 0);
             tc::commit(bar_z);
         }
         if (!mbar_wait_bounded(bar_z, ph, kTcWaitProbes)) ok = false;
@@ -543,30 +562,37 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
             }
             const float w = P.omega[it];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 2; ++c) {
+                const int t0 = tcol + c * 16;
                 float z1[16], z3[16], xp[16], qv[16];
-                tc::tmem_ld16(tl + T_Z1 + c * 16, z1);
-                tc::tmem_ld16(tl + T_Z3 + c * 16, z3);
-                tc::tmem_ld16(tl + T_XP + c * 16, xp);
-                load_qrow16(sb + L::QS, tid, c, qv);
-                float cq[16], c1[16], c3[16];
-                ld_f32x16(s_cq + c * 16, cq);
-                ld_f32x16(s_c1 + c * 16, c1);
-                ld_f32x16(s_c3 + c * 16, c3);
+                tc::tmem_ld16(tl + T_Z1 + t0, z1);
+                tc::tmem_ld16(tl + T_Z3 + t0, z3);
+                tc::tmem_ld16(tl + T_XP + t0, xp);
+                load_qrow16(sb + L::QS, d, wg * 2 + c, qv);
                 tc::tmem_wait_ld();
                 float xn[16];
 #pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const int jj = c * 16 + u;
-                    // (q - A x)/d, scaled: cq q - c1 (H_s x~) - c3 (intra x~) - (lambda/d) x~
-                    const float r = fmaf(cq[u], qv[u],
-                                         -fmaf(c1[u], z1[u], fmaf(c3[u], z3[u], cl * xc[jj])));
-                    xn[u] = fmaf(w, r + xc[jj] - xp[u], xp[u]);
+                for (int u4 = 0; u4 < 16; u4 += 4) {
+                    const float4 cq = *reinterpret_cast<const float4 *>(s_cq + t0 + u4);
+                    const float4 c1 = *reinterpret_cast<const float4 *>(s_c1 + t0 + u4);
+                    const float4 c3 = *reinterpret_cast<const float4 *>(s_c3 + t0 + u4);
+                    const float cqv[4] = {cq.x, cq.y, cq.z, cq.w};
+                    const float c1v[4] = {c1.x, c1.y, c1.z, c1.w};
+                    const float c3v[4] = {c3.x, c3.y, c3.z, c3.w};
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        const int u = u4 + v;
+                        // (q - A x)/d, scaled: cq q - c1 (H_s x~) - c3 (intra x~) - (lambda/d) x~
+                        const float r = fmaf(cqv[v], qv[u], -fmaf(c1v[v], z1[u],
+                                                                  fmaf(c3v[v], z3[u],
+                                                                       cl * xc[c * 16 + u])));
+                        xn[u] = fmaf(w, r + xc[c * 16 + u] - xp[u], xp[u]);
+                    }
                 }
-                tc::tmem_st16(tl + T_XP + c * 16, &xc[c * 16]);
+                tc::tmem_st16(tl + T_XP + t0, &xc[c * 16]);
 #pragma unroll
                 for (int u = 0; u < 16; ++u) xc[c * 16 + u] = xn[u];
-                st_row16(sb + L::XT, tid, c * 16, xn);
+                st_row16(sb + L::XT, d, t0, xn);
             }
             tc::tmem_wait_st();
             fence_proxy_async_smem();
@@ -574,14 +600,15 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
             ok = __syncthreads_and(ok);
         } else if (ok) {
             // o_j[d] = b_j (M_s x_j)[d] + sum_i w_{ji} (k_i . x_j) v_i[d]
-            __nv_bfloat16 *orow = o + (tok0 + j0) * kTcD + tid;
+            __nv_bfloat16 *orow = o + (tok0 + j0 + tcol) * kTcD + d;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 2; ++c) {
+                const int t0 = tcol + c * 16;
                 float z1[16], z3[16], o1[16], o3[16];
-                tc::tmem_ld16(tl + T_Z1 + c * 16, z1);
-                tc::tmem_ld16(tl + T_Z3 + c * 16, z3);
-                ld_f32x16(s_o1 + c * 16, o1);
-                ld_f32x16(s_o3 + c * 16, o3);
+                tc::tmem_ld16(tl + T_Z1 + t0, z1);
+                tc::tmem_ld16(tl + T_Z3 + t0, z3);
+                ld_f32x16(s_o1 + t0, o1);
+                ld_f32x16(s_o3 + t0, o3);
                 tc::tmem_wait_ld();
 #pragma unroll
                 for (int u = 0; u < 16; ++u)
