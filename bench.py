@@ -311,13 +311,14 @@ def main():
     # ---- roofline of the dominant kernel ----
     ch, out, upd, nrm = flops_per_head_token(w.D, w.chunk, w.r)
     head_tok = w.B * w.H * w.T
-    # the dominant kernel: largest summed device time among the step's kernels
+    # the dominant kernel: largest summed device time among the step's kernels (it may
+    # be several launches per step, e.g. one per 64-token group of a 128-token chunk)
     dom = max(kt.items(), key=lambda kv: kv[1][0])
     dom_name, (dom_ms, dom_n) = dom
-    per_launch_ms = dom_ms / dom_n
+    per_step_ms = dom_ms / args.steps
     alg = {"chunk_solve": ch + out, "chunk_solve_tc": ch + out, "chunk_norm": nrm,
            "chunk_delta": upd}.get(dom_name, 0)
-    kernel_flops = alg * head_tok
+    kernel_flops = alg * head_tok            # per step
     sm_mhz_max = peaks.get("sm_max_mhz", 1965.0)
     if dom_name == "chunk_solve_tc":
         # fp16 operands, fp32 accumulation: the dense fp16 peak equals the bf16 one
@@ -328,12 +329,13 @@ def main():
         bound, punit = "alu", "TFLOP/s"
         peak = 148 * 128 * 2 * sm_mhz_max * 1e6 / 1e12
         peak_note = "fp32 FMA: 148 SMs x 128 lanes x 2 flop x max SM clock"
-    achieved = kernel_flops / (per_launch_ms / 1e3) / 1e12
+    achieved = kernel_flops / (per_step_ms / 1e3) / 1e12
     whole_flops = (ch + out + upd + nrm) * head_tok
     roofline = {"bound": bound, "kernel": dom_name, "achieved": achieved, "peak": peak,
                 "unit": punit, "frac": achieved / peak, "traffic": None,
                 "peak_source": peak_note,
-                "algorithmic_per_launch": kernel_flops,
+                "launches_per_step": dom_n / args.steps,
+                "algorithmic_per_step": kernel_flops,
                 "step_frac_of_bf16_peak": whole_flops / (ms_per_step / 1e3) / 1e12
                 / peaks["bf16_tflops"]}
 

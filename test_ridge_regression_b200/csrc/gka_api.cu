@@ -175,7 +175,7 @@ static int forward_simt(const Tin *q, const Tin *k, const Tin *v, const float *b
 
     const int DD2 = 2 * D * D;
     { ProfScope ps(GKA_KERNEL_STATE_SCAN, s);
-    k_state_scan<<<dim3((DD2 + 255) / 256, BH), 256, 0, s>>>(states, decay, final_state, nullptr,
+    k_state_scan<<<dim3((DD2 + 1023) / 1024, BH), 256, 0, s>>>(states, decay, final_state, nullptr,
                                                              nullptr, nullptr, N, DD2, true); }
     if (int rc = check_launch()) return rc;
 
@@ -275,7 +275,7 @@ static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
 
     const int DD2 = 2 * D * D;
     { ProfScope ps(GKA_KERNEL_STATE_SCAN, s);
-    k_state_scan<<<dim3((DD2 + 255) / 256, BH), 256, 0, s>>>(states, decay, final_state, slp,
+    k_state_scan<<<dim3((DD2 + 1023) / 1024, BH), 256, 0, s>>>(states, decay, final_state, slp,
                                                              bound_inc, sexp, N, DD2, false); }
     if (int rc = check_launch()) return rc;
 
