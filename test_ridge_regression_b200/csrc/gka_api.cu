@@ -279,19 +279,22 @@ static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
                                                              bound_inc, sexp, N, DD2, false); }
     if (int rc = check_launch()) return rc;
 
-    if ((e = set_smem(k_chunk_solve_tc<64>, TcSmem<64>::bytes)) != cudaSuccess) return cuda_fail(e);
-    { ProfScope ps(GKA_KERNEL_CHUNK_SOLVE_TC, s);
-    k_chunk_solve_tc<64><<<dim3(N, BH), kSolveThreads, TcSmem<64>::bytes, s>>>(
-        maps, q, beta, norms, sexp, o, T, N, C, 0, P, flag); }
-    if (int rc = check_launch()) return rc;
-    if (C == 128) {
-        if ((e = set_smem(k_chunk_solve_tc<128>, TcSmem<128>::bytes)) != cudaSuccess)
-            return cuda_fail(e);
-        { ProfScope ps(GKA_KERNEL_CHUNK_SOLVE_TC, s);
-        k_chunk_solve_tc<128><<<dim3(N, BH), kSolveThreads, TcSmem<128>::bytes, s>>>(
-            maps, q, beta, norms, sexp, o, T, N, C, 1, P, flag); }
-        if (int rc = check_launch()) return rc;
+    if (C == 64) {
+        // one CTA per 64-token chunk
+        auto kern = k_chunk_solve_tc<64, 64>;
+        if ((e = set_smem(kern, TcSmem<64, 64>::bytes)) != cudaSuccess) return cuda_fail(e);
+        ProfScope ps(GKA_KERNEL_CHUNK_SOLVE_TC, s);
+        kern<<<dim3(N, BH), kSolveThreads, TcSmem<64, 64>::bytes, s>>>(
+            maps, q, beta, norms, sexp, o, T, N, C, 0, P, flag);
+    } else {
+        // one CTA per 128-token chunk (N = 128 MMAs)
+        auto kern = k_chunk_solve_tc<128, 128>;
+        if ((e = set_smem(kern, TcSmem<128, 128>::bytes)) != cudaSuccess) return cuda_fail(e);
+        ProfScope ps(GKA_KERNEL_CHUNK_SOLVE_TC, s);
+        kern<<<dim3(N, BH), kSolveThreads, TcSmem<128, 128>::bytes, s>>>(
+            maps, q, beta, norms, sexp, o, T, N, C, 0, P, flag);
     }
+    if (int rc = check_launch()) return rc;
     return GKA_OK;
 }
 

@@ -44,31 +44,30 @@ namespace gka {
 
 constexpr int kTcThreads = 128;
 constexpr int kSolveThreads = 256;   // solve kernel: two warpgroups
-constexpr int kTcTokens = 64;     // tokens per CTA
 constexpr int kTcD = 128;         // head dimension of the tensor-core path
 constexpr uint32_t kTcWaitProbes = 1u << 22;
 
-template <int MG>
+template <int MG, int TOK>
 struct TcSmem {
     // byte offsets from a 1024-aligned base
-    static constexpr uint32_t HM = 0;                        // H_s, later M_s: 2 x [128][64] bf16
-    static constexpr uint32_t KT = HM + 32768;               // keys:   2 x [MG][64] bf16
-    static constexpr uint32_t VT = KT + MG * 256;            // values: 2 x [MG][64] bf16
-    static constexpr uint32_t XT = VT + MG * 256;            // X^T: [128][64] bf16, MN-major
-    static constexpr uint32_t PT = XT + 16384;               // P^T: [MG][64] bf16, MN-major
-    static constexpr uint32_t QS = PT + MG * 128;            // q: [64][128] bf16, then q^T
-    static constexpr uint32_t SCAL = QS + 16384;             // per-token scalars
-    static constexpr uint32_t ELL = SCAL + 8 * 4 * kTcTokens; // double[MG] cumulative logs
-    static constexpr uint32_t RED = ELL + 8 * MG + 8 * (kSolveThreads / 32);  // float[16] reductions
-    static constexpr uint32_t NRM = RED + 64;                 // norm terms: u, E, X, Gjj [4][MG]
-    static constexpr uint32_t NRM2 = NRM + 16 * MG;           // second warpgroup's E, X [2][MG]
-    static constexpr uint32_t UPART = NRM2 + 8 * MG;          // [4 lane quarters][MG] partial u
-    static constexpr uint32_t QPART = UPART + 16 * MG;        // [4 warps][64] partial |q_j|^2
-    static constexpr uint32_t DEC = QPART + 16 * kTcTokens;   // l2, b, beta^2: [3][MG] floats
+    static constexpr uint32_t HM = 0;                        // H_s, later M_s: 2 x [128][64] fp16
+    static constexpr uint32_t KT = HM + 32768;               // keys:   2 x [MG][64]
+    static constexpr uint32_t VT = KT + MG * 256;            // values: 2 x [MG][64]
+    static constexpr uint32_t XT = VT + MG * 256;            // X^T: TOK/64 x [128][64], MN-major
+    static constexpr uint32_t PT = XT + TOK * 256;           // P^T: TOK/64 x [MG][64], MN-major
+    static constexpr uint32_t QS = PT + TOK * MG * 2;        // q: [TOK][128] bf16, then q^T
+    static constexpr uint32_t SCAL = QS + TOK * 256;         // per-token scalars [5][TOK]
+    static constexpr uint32_t ELL = SCAL + 8 * 4 * TOK;      // double[MG] cumulative logs
+    static constexpr uint32_t RED = ELL + 8 * MG + 8 * (kSolveThreads / 32);  // float[16]
+    static constexpr uint32_t NRM = RED + 64;                // u, E, X, Gjj [4][MG]
+    static constexpr uint32_t NRM2 = NRM + 16 * MG;          // second warpgroup's E, X [2][MG]
+    static constexpr uint32_t UPART = NRM2 + 8 * MG;         // [4 lane quarters][MG] partial u
+    static constexpr uint32_t QPART = UPART + 16 * MG;       // [4 lane quarters][TOK] |q_j|^2
+    static constexpr uint32_t DEC = QPART + 16 * TOK;        // l2, b, beta^2: [3][MG] floats
     static constexpr uint32_t BARS = DEC + 12 * MG;
     static constexpr uint32_t TBASE = BARS + 8 * 8;
     static constexpr uint32_t END = TBASE + 16;
-    static constexpr size_t bytes = END + 1024;               // + alignment slack
+    static constexpr size_t bytes = END + 1024;              // + alignment slack
 };
 
 struct TcMaps {
@@ -182,27 +181,32 @@ __device__ __forceinline__ void reduce_scatter32(float (&v)[N], int lane) {
     }
 }
 
-// grid (N, B*H); group g = `group` of every chunk; MG = 64 * (group + 1).
-// 8 warps: warpgroup wg (warps 4wg..4wg+3) owns tokens 32wg..32wg+31 of the
-// group; warp w reads TMEM lane quarter w % 4, so thread (wg, d) owns element d
-// of the iterates of its 32 tokens.
-template <int MG>
-__global__ void __launch_bounds__(kSolveThreads, 2)
+// grid (N, B*H).  A CTA solves TOK tokens (64 or 128) of one chunk, starting at
+// token 64 * group, with the chunk's first MG keys (MG = 64 (group + 1) for
+// TOK = 64; MG = 128 for TOK = 128, a whole 128-token chunk in one CTA so that
+// every MMA has N = 128).  8 warps: warpgroup wg (warps 4wg..4wg+3) owns tokens
+// wg*TOK/2 .. (wg+1)*TOK/2 - 1; warp w reads TMEM lane quarter w % 4, so thread
+// (wg, d) owns element d of the iterates of its TOK/2 tokens.
+template <int MG, int TOK>
+__global__ void __launch_bounds__(kSolveThreads, TOK == 64 ? 2 : 1)
 k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__restrict__ q,
                  const float *__restrict__ beta, float *__restrict__ norms,
                  const int *__restrict__ state_exp, __nv_bfloat16 *__restrict__ o, int T, int N,
                  int C, int group, const ChebParams P, int *__restrict__ timeout_flag) {
-    using L = TcSmem<MG>;
+    using L = TcSmem<MG, TOK>;
     constexpr int HALF = MG / 2;       // keys per warpgroup in the norm reductions
+    constexpr int TPT = TOK / 2;       // tokens per thread
+    constexpr int NCH = TPT / 16;      // 16-token chunks per thread
+    constexpr uint32_t TMEM_COLS = 4 * TOK;
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
     const uint32_t sb = smem_u32(sm);
     float *s_cq = reinterpret_cast<float *>(sm + L::SCAL);   // coefficient of q (scaled domain)
-    float *s_c1 = s_cq + kTcTokens;                          // coefficient of Z1
-    float *s_c3 = s_c1 + kTcTokens;                          // coefficient of Z3
-    float *s_o1 = s_c3 + kTcTokens;                          // readout coefficient of Z1
-    float *s_o3 = s_o1 + kTcTokens;                          // readout coefficient of Z3
+    float *s_c1 = s_cq + TOK;                                // coefficient of Z1
+    float *s_c3 = s_c1 + TOK;                                // coefficient of Z3
+    float *s_o1 = s_c3 + TOK;                                // readout coefficient of Z1
+    float *s_o3 = s_o1 + TOK;                                // readout coefficient of Z3
     double *ell = reinterpret_cast<double *>(sm + L::ELL);
     double *wtot = ell + MG;
     float *red = reinterpret_cast<float *>(sm + L::RED);
@@ -214,9 +218,9 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wg = warp >> 2, quarter = warp & 3;
     const int d = quarter * 32 + lane;        // head-dimension row = TMEM lane of this thread
-    const int tcol = wg * 32;                 // first token (TMEM column) of this thread
+    const int tcol = wg * TPT;                // first token (TMEM column) of this thread
     const int n = blockIdx.x, bh = blockIdx.y;
-    const int j0 = group * kTcTokens;                      // first token of the group in the chunk
+    const int j0 = group * 64;                             // first token of the CTA in the chunk
     const size_t tok0 = (size_t)bh * T + (size_t)n * C;    // first token of the chunk
     const int srow = (int)(((size_t)bh * N + n) * 2 * kTcD);   // H_s row in the state map
 
@@ -226,7 +230,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     }
     __syncthreads();
     if (tid == 0) {
-        mbar_arrive_expect_tx(bar_load, 32768 + MG * 256 + kTcTokens * kTcD * 2);
+        mbar_arrive_expect_tx(bar_load, 32768 + MG * 256 + TOK * kTcD * 2);
         for (int h = 0; h < 2; ++h) {
             for (int rb = 0; rb < 2; ++rb)
                 tc::tma_load_2d(sm + L::HM + h * 16384 + rb * 8192, &maps.state, h * 64,
@@ -235,7 +239,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
                 tc::tma_load_2d(sm + L::KT + h * MG * 128 + rb * 8192, &maps.k, h * 64,
                                 (int)tok0 + rb * 64, bar_load);
         }
-        bulk_g2s(sm + L::QS, q + (tok0 + j0) * kTcD, kTcTokens * kTcD * 2, bar_load);
+        bulk_g2s(sm + L::QS, q + (tok0 + j0) * kTcD, TOK * kTcD * 2, bar_load);
         mbar_arrive_expect_tx(bar_v, MG * 256);
         for (int h = 0; h < 2; ++h)
             for (int rb = 0; rb < MG / 64; ++rb)
@@ -243,7 +247,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
                                 (int)tok0 + rb * 64, bar_v);
     }
     if (warp == 0) {
-        tc::tmem_alloc(tbase, 256);
+        tc::tmem_alloc(tbase, TMEM_COLS);
         tc::tmem_relinquish();
     }
     chunk_log_prefix(beta + tok0, MG, ell, wtot);
@@ -272,7 +276,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     const uint32_t tmem = *tbase;
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);   // this warp's lane quarter
     // TMEM columns: Z1 | S, then Z3 (S is consumed before MMA3 writes Z3) | W | x_prev
-    const uint32_t T_Z1 = 0, T_S = 64, T_Z3 = 64, T_W = 128, T_XP = 192;
+    const uint32_t T_Z1 = 0, T_S = TOK, T_Z3 = TOK, T_W = 2 * TOK, T_XP = 3 * TOK;
     const uint32_t a_hm = sb + L::HM, a_kt = sb + L::KT, a_vt = sb + L::VT, b_xt = sb + L::XT,
                    b_pt = sb + L::PT;
 
@@ -286,13 +290,15 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     // intra-chunk terms:  ||H_j||^2 = b_j^2 ||H_s||^2 + 2 b_j X_j + R_j with
     // X_j = sum_{i<=j} w_ji u_i and R_j = beta_j^2 R_{j-1} + 2 E_j + G_jj^2,
     // E_j = sum_{i<j} w_ji G_ij^2 (R_j = sum_{i,l<=j} w_ji w_jl G_il^2).
+    // Zn = H_s K^T in columns [0, MG), G = K K^T in [kGcol, kGcol + MG)
+    constexpr uint32_t kGcol = 128;
     if (tid == 0 && ok) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
             const uint64_t kdesc = tc::sdesc(a_kt + (kk >> 2) * (MG * 128) + (kk & 3) * 32, 16, 1024);
             tc::mma_f16(tmem + 0, tc::sdesc(a_hm + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
                         kdesc, tc::idesc_f16(128, MG, false, false), kk > 0);
-            tc::mma_f16(tmem + 128, kdesc, kdesc, tc::idesc_f16(MG, MG, false, false), kk > 0);
+            tc::mma_f16(tmem + kGcol, kdesc, kdesc, tc::idesc_f16(MG, MG, false, false), kk > 0);
         }
         tc::commit(bar_n);
     }
@@ -351,7 +357,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
 #pragma unroll
         for (int cb = 0; cb < HALF; cb += 16) {
             float g[16];
-            tc::tmem_ld16(tl + 128 + wg * HALF + cb, g);
+            tc::tmem_ld16(tl + kGcol + wg * HALF + cb, g);
             tc::tmem_wait_ld();
             if (s_owner) {
 #pragma unroll
@@ -379,19 +385,22 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     }
     // q column of this thread's tokens (token-major tile), kept packed for the
     // transpose below; |q_j|^2 = sum_d q_j[d]^2 by a reduce-scatter over the warp
-    uint32_t qcol[16];
+    uint32_t qcol[TPT / 2];
     {
-        float sq[32];
+        float sq[TPT];
 #pragma unroll
-        for (int jj = 0; jj < 32; jj += 2) {
+        for (int jj = 0; jj < TPT; jj += 2) {
             const __nv_bfloat16 lo = qs[(tcol + jj) * kTcD + d], hi = qs[(tcol + jj + 1) * kTcD + d];
             qcol[jj / 2] = (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
             const float a0 = __bfloat162float(lo), a1 = __bfloat162float(hi);
             sq[jj] = a0 * a0;
             sq[jj + 1] = a1 * a1;
         }
-        reduce_scatter32<32>(sq, lane);
-        reinterpret_cast<float *>(sm + L::QPART)[quarter * kTcTokens + tcol + lane] = sq[0];
+        reduce_scatter32<TPT>(sq, lane);
+#pragma unroll
+        for (int s2 = 0; s2 < TPT / 32; ++s2)
+            reinterpret_cast<float *>(sm + L::QPART)[quarter * TOK + tcol + lane * (TPT / 32) + s2] =
+                sq[s2];
     }
     __syncthreads();
     float *s_n = s_o3;   // per-token norms, then overwritten by the readout coefficient
@@ -403,7 +412,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         for (int j = 0; j < MG; ++j) {
             const float E = s_E[j] + s_E1[j], X = s_X[j] + s_X1[j];
             R = fmaf(s_beta2[j], R, fmaf(2.f, E, s_G[j] * s_G[j]));
-            if (j >= j0) {
+            if (j >= j0 && j < j0 + TOK) {
                 const float b = s_bt[j];
                 const float n2 = fmaf(b * b, hs2, fmaf(2.f * b, X, R));
                 s_n[j - j0] = sqrtf(fmaxf(n2, 0.f));
@@ -411,15 +420,14 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         }
     }
     __syncthreads();
-    if (tid < kTcTokens) {
+    if (tid < TOK) {
         const int j = tid;
         const float nj = s_n[j];
         norms[tok0 + j0 + j] = nj;
         const float invd = nj > 0.f ? 1.f / (P.half_1p2a * nj) : 0.f;
         const float b = s_bt[j0 + j];
         const float *qpart = reinterpret_cast<const float *>(sm + L::QPART);
-        const float qq = qpart[j] + qpart[kTcTokens + j] + qpart[2 * kTcTokens + j] +
-                         qpart[3 * kTcTokens + j];
+        const float qq = qpart[j] + qpart[TOK + j] + qpart[2 * TOK + j] + qpart[3 * TOK + j];
         // every Chebyshev iterate obeys ||x|| <= ||q|| (1+2a) / (a d): the iterate is
         // kept as x~ = sx x with sx a power of two that puts ||x~|| below 2^12
         const float xb = sqrtf(qq) * invd * (2.f * P.half_1p2a / P.a);
@@ -438,16 +446,18 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     // q^T: this thread's tokens of row d, written into the (now free) tile as
     // [128 d][64 tokens] with 128B-swizzled rows: 8 tokens per 16-byte load later
 #pragma unroll
-    for (int ch = 0; ch < 4; ++ch)
-        st_shared_v4(sb + L::QS + d * 128u + (((wg * 4 + ch) ^ d) & 7u) * 16u, qcol[4 * ch],
-                     qcol[4 * ch + 1], qcol[4 * ch + 2], qcol[4 * ch + 3]);
+    for (int ch = 0; ch < TPT / 8; ++ch) {
+        const int t = tcol + ch * 8;             // first of 8 tokens
+        st_shared_v4(sb + L::QS + (t >> 6) * 16384u + d * 128u + ((((t & 63) >> 3) ^ d) & 7u) * 16u,
+                     qcol[4 * ch], qcol[4 * ch + 1], qcol[4 * ch + 2], qcol[4 * ch + 3]);
+    }
     const float cl = 2.f * P.a / (1.f + 2.f * P.a);   // lambda / d for every token with H != 0
 
     // W^T rows: W[i][j] = w_{ji} = exp(l_j - l_i) for i <= j, else 0 (this thread's tokens)
     {
         float wv[16];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < NCH; ++c) {
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
                 const int j = j0 + tcol + c * 16 + u;
@@ -459,19 +469,20 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
 
     // x_1 = q / d, x_0 = 0 (scaled by sx): thread (wg, d) keeps element d of its 32
     // current iterates in registers and of the previous ones in TMEM
-    float xc[32];
+    float xc[TPT];
     {
         const float zero16[16] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f,
                                   0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         __syncthreads();   // q^T complete
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < NCH; ++c) {
+            const int t0 = tcol + c * 16;
             float qv[16];
-            load_qrow16(sb + L::QS, d, wg * 2 + c, qv);
+            load_qrow16(sb + L::QS + (t0 >> 6) * 16384u, d, (t0 & 63) >> 4, qv);
 #pragma unroll
-            for (int u = 0; u < 16; ++u) xc[c * 16 + u] = qv[u] * s_cq[tcol + c * 16 + u];
-            st_row16(sb + L::XT, d, tcol + c * 16, &xc[c * 16]);
-            tc::tmem_st16(tl + T_XP + tcol + c * 16, zero16);
+            for (int u = 0; u < 16; ++u) xc[c * 16 + u] = qv[u] * s_cq[t0 + u];
+            st_row16(sb + L::XT + (t0 >> 6) * 16384u, d, t0 & 63, &xc[c * 16]);
+            tc::tmem_st16(tl + T_XP + t0, zero16);
         }
         tc::tmem_wait_st();
     }
@@ -479,9 +490,10 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     tc::fence_before_sync();
     ok = __syncthreads_and(ok);
 
-    constexpr uint32_t IDESC_S = tc::idesc_f16(MG, 64, false, true);
-    constexpr uint32_t IDESC_Z1 = tc::idesc_f16(128, 64, false, true);
-    constexpr uint32_t IDESC_Z3 = tc::idesc_f16(128, 64, true, true);
+    constexpr uint32_t IDESC_S = tc::idesc_f16(MG, TOK, false, true);
+    constexpr uint32_t IDESC_Z1 = tc::idesc_f16(128, TOK, false, true);
+    constexpr uint32_t IDESC_Z3 = tc::idesc_f16(128, TOK, true, true);
+    constexpr uint32_t PT_BLOCK = MG * 128;   // bytes between 64-token blocks of P^T
     bool m_requested = false;
     uint32_t ph = 0;   // phase parity of bar_s / bar_z (both complete once per round)
 
@@ -495,7 +507,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
             for (int kk = 0; kk < 8; ++kk)
                 tc::mma_f16(tmem + T_S,
                             tc::sdesc(a_kt + (kk >> 2) * (MG * 128) + (kk & 3) * 32, 16, 1024),
-                            tc::sdesc(b_xt + kk * 2048, 8192, 1024), IDESC_S, kk > 0);
+                            tc::sdesc(b_xt + kk * 2048, 16384, 1024), IDESC_S, kk > 0);
             tc::commit(bar_s);
             if (out_pass) {
                 if (!m_requested) {
@@ -514,24 +526,27 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
                 for (int kk = 0; kk < 8; ++kk)
                     tc::mma_f16(tmem + T_Z1,
                                 tc::sdesc(a_hm + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                                tc::sdesc(b_xt + kk * 2048, 8192, 1024), IDESC_Z1, kk > 0);
+                                tc::sdesc(b_xt + kk * 2048, 16384, 1024), IDESC_Z1, kk > 0);
             }
         }
         // P^T = W o S^T  -> fp16, MN-major tile of MG rows (this thread's 32 tokens)
         if (!mbar_wait_bounded(bar_s, ph, kTcWaitProbes)) ok = false;
         tc::fence_after_sync();
-        {
+#pragma unroll
+        for (int c = 0; c < NCH; c += 2) {
+            const int t0 = tcol + c * 16;
             float sv[32], wv[32];
-            tc::tmem_ld16(tl + T_S + tcol, sv);
-            tc::tmem_ld16(tl + T_S + tcol + 16, sv + 16);
-            tc::tmem_ld16(tl + T_W + tcol, wv);
-            tc::tmem_ld16(tl + T_W + tcol + 16, wv + 16);
+            tc::tmem_ld16(tl + T_S + t0, sv);
+            tc::tmem_ld16(tl + T_S + t0 + 16, sv + 16);
+            tc::tmem_ld16(tl + T_W + t0, wv);
+            tc::tmem_ld16(tl + T_W + t0 + 16, wv + 16);
             tc::tmem_wait_ld();
 #pragma unroll
             for (int u = 0; u < 32; ++u) sv[u] *= wv[u];
             if (s_owner) {
-                st_row16(b_pt, key, tcol, sv);
-                st_row16(b_pt, key, tcol + 16, sv + 16);
+                const uint32_t pt = b_pt + (t0 >> 6) * PT_BLOCK;
+                st_row16(pt, key, t0 & 63, sv);
+                st_row16(pt, key, (t0 & 63) + 16, sv + 16);
             }
         }
         fence_proxy_async_smem();
@@ -544,7 +559,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
 #pragma unroll
             for (int kk = 0; kk < MG / 16; ++kk)
                 tc::mma_f16(tmem + T_Z3, tc::sdesc(a3 + kk * 2048, MG * 128, 1024),
-                            tc::sdesc(b_pt + kk * 2048, 8192, 1024), IDESC_Z3, kk > 0);
+                            tc::sdesc(b_pt + kk * 2048, PT_BLOCK, 1024), IDESC_Z3, kk > 0);
             tc::commit(bar_z);
         }
         if (!mbar_wait_bounded(bar_z, ph, kTcWaitProbes)) ok = false;
@@ -562,13 +577,13 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
             }
             const float w = P.omega[it];
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
+            for (int c = 0; c < NCH; ++c) {
                 const int t0 = tcol + c * 16;
                 float z1[16], z3[16], xp[16], qv[16];
                 tc::tmem_ld16(tl + T_Z1 + t0, z1);
                 tc::tmem_ld16(tl + T_Z3 + t0, z3);
                 tc::tmem_ld16(tl + T_XP + t0, xp);
-                load_qrow16(sb + L::QS, d, wg * 2 + c, qv);
+                load_qrow16(sb + L::QS + (t0 >> 6) * 16384u, d, (t0 & 63) >> 4, qv);
                 tc::tmem_wait_ld();
                 float xn[16];
 #pragma unroll
@@ -592,7 +607,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
                 tc::tmem_st16(tl + T_XP + t0, &xc[c * 16]);
 #pragma unroll
                 for (int u = 0; u < 16; ++u) xc[c * 16 + u] = xn[u];
-                st_row16(sb + L::XT, d, t0, xn);
+                st_row16(sb + L::XT + (t0 >> 6) * 16384u, d, t0 & 63, xn);
             }
             tc::tmem_wait_st();
             fence_proxy_async_smem();
@@ -602,7 +617,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
             // o_j[d] = b_j (M_s x_j)[d] + sum_i w_{ji} (k_i . x_j) v_i[d]
             __nv_bfloat16 *orow = o + (tok0 + j0 + tcol) * kTcD + d;
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
+            for (int c = 0; c < NCH; ++c) {
                 const int t0 = tcol + c * 16;
                 float z1[16], z3[16], o1[16], o3[16];
                 tc::tmem_ld16(tl + T_Z1 + t0, z1);
@@ -634,7 +649,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     __syncthreads();
     if (warp == 0) {
         tc::fence_after_sync();
-        tc::tmem_dealloc(tmem, 256);
+        tc::tmem_dealloc(tmem, TMEM_COLS);
     }
 }
 
