@@ -194,4 +194,172 @@ k_decode_step(float *__restrict__ state, const Tin *__restrict__ q, const Tin *_
     if (owner) store_f(o + (size_t)head * D + R, invd > 0.f ? orow : 0.f);
 }
 
+// ---------------------------------------------------------------------------
+// Persistent, software-pipelined decode step for D = 128: one CTA of 512
+// threads per SM walks its share of the heads.  While head i is updated and
+// iterated (H in registers), bulk async copies already bring H, M, q, k, v of
+// head i+1 into shared memory, so the HBM stream does not pause during the
+// r - 1 matrix-vector products.  Shared memory: one H buffer (64 KB) and two
+// M buffers (2 x 64 KB); the H buffer is refilled as soon as every thread has
+// copied H_i into its registers.
+// ---------------------------------------------------------------------------
+constexpr int kDecD = 128;
+constexpr int kDecThreads = 4 * kDecD;
+constexpr size_t kDecSmem = 3 * 65536 + 2 * 3 * 512 + 1024 + 1024;
+
+template <typename Tin>
+__global__ void __launch_bounds__(kDecThreads, 1)
+k_decode_pipelined(float *__restrict__ state, const Tin *__restrict__ q, const Tin *__restrict__ k,
+                   const Tin *__restrict__ v, const float *__restrict__ beta, Tin *__restrict__ o,
+                   int num_heads, const ChebParams P, int *__restrict__ timeout_flag) {
+    constexpr int D = kDecD, NW = kDecThreads / 32, CPL = D / 32;
+    constexpr uint32_t ROWB = D * sizeof(Tin);               // bytes of one q/k/v row
+    extern __shared__ __align__(128) uint8_t dsm[];
+    float *Hbuf = reinterpret_cast<float *>(dsm);             // [D][D]
+    float *Mbuf = Hbuf + D * D;                               // [2][D][D]
+    uint8_t *qkv = dsm + 3 * 65536;                           // [2][3][ROWB]
+    __shared__ __align__(16) float xbuf[2][D];
+    __shared__ float ks[D], vs[D];
+    __shared__ float red[NW];
+    __shared__ __align__(8) uint64_t barH, barM[2];
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int row0 = warp * 8, col0 = lane * CPL;
+    const int G = gridDim.x;
+    int head = blockIdx.x;
+    if (head >= num_heads) return;
+
+    auto issue = [&](int h, int buf, bool with_h) {
+        // H (if requested) into Hbuf, M and q, k, v into buffer `buf`
+        const float *Hg = state + (size_t)h * 2 * D * D;
+        if (with_h) {
+            mbar_arrive_expect_tx(&barH, D * D * 4);
+            bulk_g2s(Hbuf, Hg, D * D * 4, &barH);
+        }
+        mbar_arrive_expect_tx(&barM[buf], D * D * 4 + 3 * ROWB);
+        bulk_g2s(Mbuf + buf * D * D, Hg + D * D, D * D * 4, &barM[buf]);
+        uint8_t *dst = qkv + buf * 3 * ROWB;
+        bulk_g2s(dst, q + (size_t)h * D, ROWB, &barM[buf]);
+        bulk_g2s(dst + ROWB, k + (size_t)h * D, ROWB, &barM[buf]);
+        bulk_g2s(dst + 2 * ROWB, v + (size_t)h * D, ROWB, &barM[buf]);
+    };
+
+    if (tid == 0) {
+        mbar_init(&barH, 1);
+        mbar_init(&barM[0], 1);
+        mbar_init(&barM[1], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid == 0) issue(head, 0, true);
+
+    bool ok = true;
+    for (int i = 0; head < num_heads; ++i, head += G) {
+        const int buf = i & 1;
+        const int next = head + G;
+        const float bt = beta[head];
+        // H_i: shared -> registers, then the buffer goes back to the copy engine
+        if (!mbar_wait_bounded(&barH, i & 1, kDecodeWaitProbes)) ok = false;
+        float h[8][CPL];
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr) VecF<CPL>::ld(&Hbuf[(row0 + rr) * D + col0], h[rr]);
+        // q, k, v of this head (arrived with M_i on barM[buf])
+        if (!mbar_wait_bounded(&barM[buf], (i >> 1) & 1, kDecodeWaitProbes)) ok = false;
+        const Tin *qr = reinterpret_cast<const Tin *>(qkv + buf * 3 * ROWB);
+        for (int j = tid; j < D; j += kDecThreads) {
+            ks[j] = load_f(qr + D + j);
+            vs[j] = load_f(qr + 2 * D + j);
+        }
+        fence_proxy_async_smem();
+        ok = __syncthreads_and(ok);
+        if (!ok) break;
+        if (tid == 0 && next < num_heads) issue(next, buf ^ 1, true);
+
+        // H <- beta H + k k^T, written back at once
+        float *Hg = state + (size_t)head * 2 * D * D;
+        float ss = 0.f;
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr) {
+            const float kr = ks[row0 + rr];
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) {
+                h[rr][c] = fmaf(bt, h[rr][c], kr * ks[col0 + c]);
+                ss = fmaf(h[rr][c], h[rr][c], ss);
+            }
+            VecF<CPL>::st(Hg + (size_t)(row0 + rr) * D + col0, h[rr]);
+        }
+        ss = warp_sum(ss);
+        if (lane == 0) red[warp] = ss;
+        __syncthreads();
+        float n2 = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) n2 += red[w];
+        const float nrm = sqrtf(n2);
+        const float lam = P.a * nrm;
+        const float invd = nrm > 0.f ? 1.f / (P.half_1p2a * nrm) : 0.f;
+
+        // Chebyshev: the owner lane (lane % 4 == 0) of row R keeps x_prev, x_cur, q
+        const int R = row0 + rows8_sel(lane);
+        const bool owner = (lane & 3) == 0;
+        const float qR = load_f(qr + R);
+        float xprev = 0.f, xcur = qR * invd;
+        if (owner) xbuf[0][R] = xcur;
+        __syncthreads();
+        int cur = 0;
+#pragma unroll 1
+        for (int it = 1; it < P.r; ++it) {
+            float xv[CPL];
+            VecF<CPL>::ld(&xbuf[cur][col0], xv);
+            float part[8];
+#pragma unroll
+            for (int rr = 0; rr < 8; ++rr) {
+                float s2 = 0.f;
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) s2 = fmaf(h[rr][c], xv[c], s2);
+                part[rr] = s2;
+            }
+            const float y = fmaf(lam, xcur, rows8_reduce(part, lane));
+            const float xn = fmaf(P.omega[it], fmaf(qR - y, invd, xcur - xprev), xprev);
+            xprev = xcur;
+            xcur = xn;
+            if (owner) xbuf[cur ^ 1][R] = xn;
+            __syncthreads();
+            cur ^= 1;
+        }
+
+        // M <- beta M + v k^T and o = M x (M_i is in Mbuf[buf])
+        const float *Ms = Mbuf + buf * D * D;
+        float *Mg = Hg + D * D;
+        float xv[CPL];
+        VecF<CPL>::ld(&xbuf[cur][col0], xv);
+        float part[8];
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr) {
+            float m[CPL];
+            VecF<CPL>::ld(&Ms[(row0 + rr) * D + col0], m);
+            const float vr = vs[row0 + rr];
+            float s2 = 0.f;
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) {
+                m[c] = fmaf(bt, m[c], vr * ks[col0 + c]);
+                s2 = fmaf(m[c], xv[c], s2);
+            }
+            VecF<CPL>::st(Mg + (size_t)(row0 + rr) * D + col0, m);
+            part[rr] = s2;
+        }
+        const float orow = rows8_reduce(part, lane);
+        if (owner) store_f(o + (size_t)head * D + R, invd > 0.f ? orow : 0.f);
+        // every thread is done with Mbuf[buf], ks, vs, xbuf before they are reused
+        fence_proxy_async_smem();
+        __syncthreads();
+    }
+    if (!ok && tid == 0) {
+        atomicExch(timeout_flag, 1);
+        // let copies still in flight land before the CTA exits
+        mbar_wait_bounded(&barH, 0, kDecodeWaitProbes);
+        mbar_wait_bounded(&barM[0], 0, kDecodeWaitProbes);
+        mbar_wait_bounded(&barM[1], 0, kDecodeWaitProbes);
+    }
+}
+
 }  // namespace gka

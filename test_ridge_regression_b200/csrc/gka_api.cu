@@ -338,10 +338,41 @@ static int decode_launch(float *state, const void *q, const void *k, const void 
     return check_launch();
 }
 
+// Number of SMs of the current device (cached per device).
+static int sm_count() {
+    static int cache[256] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return 148;
+    if (!cache[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+template <typename Tin>
+static int decode_pipelined_launch(float *state, const void *q, const void *k, const void *v,
+                                   const float *beta, void *o, int BH, const ChebParams &P,
+                                   cudaStream_t s) {
+    int *flag = nullptr;
+    if (int rc = timeout_flag_ptr(&flag)) return rc;
+    cudaError_t e = set_smem(k_decode_pipelined<Tin>, kDecSmem);
+    if (e != cudaSuccess) return cuda_fail(e);
+    const int grid = BH < sm_count() ? BH : sm_count();
+    ProfScope ps(GKA_KERNEL_DECODE_STEP, s);
+    k_decode_pipelined<Tin><<<grid, kDecThreads, kDecSmem, s>>>(
+        state, static_cast<const Tin *>(q), static_cast<const Tin *>(k),
+        static_cast<const Tin *>(v), beta, static_cast<Tin *>(o), BH, P, flag);
+    return check_launch();
+}
+
 template <typename Tin>
 static int decode_dispatch(float *state, const void *q, const void *k, const void *v,
                            const float *beta, void *o, int BH, int D, const ChebParams &P,
                            cudaStream_t s) {
+    if (D == 128) return decode_pipelined_launch<Tin>(state, q, k, v, beta, o, BH, P, s);
     switch (D) {
         case 32: return decode_launch<Tin, 32>(state, q, k, v, beta, o, BH, P, s);
         case 64: return decode_launch<Tin, 64>(state, q, k, v, beta, o, BH, P, s);
