@@ -15,6 +15,7 @@
 
 #include "common.cuh"
 #include "ptx.cuh"
+#include "tcgen05.cuh"
 
 namespace gka {
 
@@ -195,170 +196,169 @@ k_decode_step(float *__restrict__ state, const Tin *__restrict__ q, const Tin *_
 }
 
 // ---------------------------------------------------------------------------
-// Persistent, software-pipelined decode step for D = 128: one CTA of 512
-// threads per SM walks its share of the heads.  While head i is updated and
-// iterated (H in registers), bulk async copies already bring H, M, q, k, v of
-// head i+1 into shared memory, so the HBM stream does not pause during the
-// r - 1 matrix-vector products.  Shared memory: one H buffer (64 KB) and two
-// M buffers (2 x 64 KB); the H buffer is refilled as soon as every thread has
-// copied H_i into its registers.
+// Decode step for D = 128, one row per thread: a CTA of 128 threads serves one
+// head and thread t owns row t of H (128 fp32 registers) for all r - 1
+// matrix-vector products, so a product needs no cross-thread reduction: x is
+// broadcast from shared memory and y_t = sum_c H[t][c] x[c] stays in the thread.
+// H and M move between HBM and a 64 KB shared buffer as 128-byte-swizzled TMA
+// tiles (bank-conflict-free row access); M is fetched into the buffer while the
+// products run, and the updated M and H leave through the same buffer with TMA
+// stores.  Three heads share an SM.
 // ---------------------------------------------------------------------------
 constexpr int kDecD = 128;
-constexpr int kDecThreads = 4 * kDecD;
-constexpr size_t kDecSmem = 3 * 65536 + 2 * 3 * 512 + 1024 + 1024;
+constexpr int kDecRowThreads = kDecD;
+constexpr size_t kDecRowSmem = 65536 + 1024;
+
+struct DecodeMaps {
+    CUtensorMap state;   // fp32 [B*H*2*128 rows][128], box 32 x 128, 128B swizzle
+};
+
+// Byte offset of fp32 element (row, 4*chunk) in the swizzled [128][128] tile
+// stored as four 32-column boxes.
+__device__ __forceinline__ uint32_t dec_tile_off(int row, int chunk) {
+    return (uint32_t)(chunk >> 3) * 16384u + (uint32_t)row * 128u +
+           (uint32_t)(((chunk & 7) ^ row) & 7) * 16u;
+}
 
 template <typename Tin>
-__global__ void __launch_bounds__(kDecThreads, 1)
-k_decode_pipelined(float *__restrict__ state, const Tin *__restrict__ q, const Tin *__restrict__ k,
-                   const Tin *__restrict__ v, const float *__restrict__ beta, Tin *__restrict__ o,
-                   int num_heads, const ChebParams P, int *__restrict__ timeout_flag) {
-    constexpr int D = kDecD, NW = kDecThreads / 32, CPL = D / 32;
-    constexpr uint32_t ROWB = D * sizeof(Tin);               // bytes of one q/k/v row
-    extern __shared__ __align__(128) uint8_t dsm[];
-    float *Hbuf = reinterpret_cast<float *>(dsm);             // [D][D]
-    float *Mbuf = Hbuf + D * D;                               // [2][D][D]
-    uint8_t *qkv = dsm + 3 * 65536;                           // [2][3][ROWB]
+__global__ void __launch_bounds__(kDecRowThreads, 3)
+k_decode_rows(const __grid_constant__ DecodeMaps maps, const Tin *__restrict__ q,
+              const Tin *__restrict__ k, const Tin *__restrict__ v, const float *__restrict__ beta,
+              Tin *__restrict__ o, const ChebParams P, int *__restrict__ timeout_flag) {
+    constexpr int D = kDecD, NW = kDecRowThreads / 32;
+    extern __shared__ uint8_t draw[];
+    uint8_t *buf = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(draw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
     __shared__ __align__(16) float xbuf[2][D];
-    __shared__ float ks[D], vs[D];
+    __shared__ __align__(16) float ks[D];
     __shared__ float red[NW];
-    __shared__ __align__(8) uint64_t barH, barM[2];
+    __shared__ __align__(8) uint64_t bar[2];
 
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int row0 = warp * 8, col0 = lane * CPL;
-    const int G = gridDim.x;
-    int head = blockIdx.x;
-    if (head >= num_heads) return;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int head = blockIdx.x;
+    const int hrow = head * 2 * D;          // first row of H in the state map; M follows
 
-    auto issue = [&](int h, int buf, bool with_h) {
-        // H (if requested) into Hbuf, M and q, k, v into buffer `buf`
-        const float *Hg = state + (size_t)h * 2 * D * D;
-        if (with_h) {
-            mbar_arrive_expect_tx(&barH, D * D * 4);
-            bulk_g2s(Hbuf, Hg, D * D * 4, &barH);
-        }
-        mbar_arrive_expect_tx(&barM[buf], D * D * 4 + 3 * ROWB);
-        bulk_g2s(Mbuf + buf * D * D, Hg + D * D, D * D * 4, &barM[buf]);
-        uint8_t *dst = qkv + buf * 3 * ROWB;
-        bulk_g2s(dst, q + (size_t)h * D, ROWB, &barM[buf]);
-        bulk_g2s(dst + ROWB, k + (size_t)h * D, ROWB, &barM[buf]);
-        bulk_g2s(dst + 2 * ROWB, v + (size_t)h * D, ROWB, &barM[buf]);
-    };
-
-    if (tid == 0) {
-        mbar_init(&barH, 1);
-        mbar_init(&barM[0], 1);
-        mbar_init(&barM[1], 1);
+    if (t == 0) {
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
         fence_mbar_init();
     }
     __syncthreads();
-    if (tid == 0) issue(head, 0, true);
-
-    bool ok = true;
-    for (int i = 0; head < num_heads; ++i, head += G) {
-        const int buf = i & 1;
-        const int next = head + G;
-        const float bt = beta[head];
-        // H_i: shared -> registers, then the buffer goes back to the copy engine
-        if (!mbar_wait_bounded(&barH, i & 1, kDecodeWaitProbes)) ok = false;
-        float h[8][CPL];
-#pragma unroll
-        for (int rr = 0; rr < 8; ++rr) VecF<CPL>::ld(&Hbuf[(row0 + rr) * D + col0], h[rr]);
-        // q, k, v of this head (arrived with M_i on barM[buf])
-        if (!mbar_wait_bounded(&barM[buf], (i >> 1) & 1, kDecodeWaitProbes)) ok = false;
-        const Tin *qr = reinterpret_cast<const Tin *>(qkv + buf * 3 * ROWB);
-        for (int j = tid; j < D; j += kDecThreads) {
-            ks[j] = load_f(qr + D + j);
-            vs[j] = load_f(qr + 2 * D + j);
-        }
-        fence_proxy_async_smem();
-        ok = __syncthreads_and(ok);
-        if (!ok) break;
-        if (tid == 0 && next < num_heads) issue(next, buf ^ 1, true);
-
-        // H <- beta H + k k^T, written back at once
-        float *Hg = state + (size_t)head * 2 * D * D;
-        float ss = 0.f;
-#pragma unroll
-        for (int rr = 0; rr < 8; ++rr) {
-            const float kr = ks[row0 + rr];
-#pragma unroll
-            for (int c = 0; c < CPL; ++c) {
-                h[rr][c] = fmaf(bt, h[rr][c], kr * ks[col0 + c]);
-                ss = fmaf(h[rr][c], h[rr][c], ss);
-            }
-            VecF<CPL>::st(Hg + (size_t)(row0 + rr) * D + col0, h[rr]);
-        }
-        ss = warp_sum(ss);
-        if (lane == 0) red[warp] = ss;
-        __syncthreads();
-        float n2 = 0.f;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) n2 += red[w];
-        const float nrm = sqrtf(n2);
-        const float lam = P.a * nrm;
-        const float invd = nrm > 0.f ? 1.f / (P.half_1p2a * nrm) : 0.f;
-
-        // Chebyshev: the owner lane (lane % 4 == 0) of row R keeps x_prev, x_cur, q
-        const int R = row0 + rows8_sel(lane);
-        const bool owner = (lane & 3) == 0;
-        const float qR = load_f(qr + R);
-        float xprev = 0.f, xcur = qR * invd;
-        if (owner) xbuf[0][R] = xcur;
-        __syncthreads();
-        int cur = 0;
-#pragma unroll 1
-        for (int it = 1; it < P.r; ++it) {
-            float xv[CPL];
-            VecF<CPL>::ld(&xbuf[cur][col0], xv);
-            float part[8];
-#pragma unroll
-            for (int rr = 0; rr < 8; ++rr) {
-                float s2 = 0.f;
-#pragma unroll
-                for (int c = 0; c < CPL; ++c) s2 = fmaf(h[rr][c], xv[c], s2);
-                part[rr] = s2;
-            }
-            const float y = fmaf(lam, xcur, rows8_reduce(part, lane));
-            const float xn = fmaf(P.omega[it], fmaf(qR - y, invd, xcur - xprev), xprev);
-            xprev = xcur;
-            xcur = xn;
-            if (owner) xbuf[cur ^ 1][R] = xn;
-            __syncthreads();
-            cur ^= 1;
-        }
-
-        // M <- beta M + v k^T and o = M x (M_i is in Mbuf[buf])
-        const float *Ms = Mbuf + buf * D * D;
-        float *Mg = Hg + D * D;
-        float xv[CPL];
-        VecF<CPL>::ld(&xbuf[cur][col0], xv);
-        float part[8];
-#pragma unroll
-        for (int rr = 0; rr < 8; ++rr) {
-            float m[CPL];
-            VecF<CPL>::ld(&Ms[(row0 + rr) * D + col0], m);
-            const float vr = vs[row0 + rr];
-            float s2 = 0.f;
-#pragma unroll
-            for (int c = 0; c < CPL; ++c) {
-                m[c] = fmaf(bt, m[c], vr * ks[col0 + c]);
-                s2 = fmaf(m[c], xv[c], s2);
-            }
-            VecF<CPL>::st(Mg + (size_t)(row0 + rr) * D + col0, m);
-            part[rr] = s2;
-        }
-        const float orow = rows8_reduce(part, lane);
-        if (owner) store_f(o + (size_t)head * D + R, invd > 0.f ? orow : 0.f);
-        // every thread is done with Mbuf[buf], ks, vs, xbuf before they are reused
-        fence_proxy_async_smem();
-        __syncthreads();
+    if (t == 0) {
+        mbar_arrive_expect_tx(&bar[0], D * D * 4);
+        for (int b = 0; b < 4; ++b) tc::tma_load_2d(buf + b * 16384, &maps.state, b * 32, hrow, &bar[0]);
     }
-    if (!ok && tid == 0) {
-        atomicExch(timeout_flag, 1);
-        // let copies still in flight land before the CTA exits
-        mbar_wait_bounded(&barH, 0, kDecodeWaitProbes);
-        mbar_wait_bounded(&barM[0], 0, kDecodeWaitProbes);
-        mbar_wait_bounded(&barM[1], 0, kDecodeWaitProbes);
+    const float bt = beta[head];
+    ks[t] = load_f(k + (size_t)head * D + t);
+    const float vt = load_f(v + (size_t)head * D + t);
+    const float qt = load_f(q + (size_t)head * D + t);
+    bool ok = mbar_wait_bounded(&bar[0], 0, kDecodeWaitProbes);
+    __syncthreads();   // ks complete
+
+    // H row t -> registers, updated: h = beta h + k_t k
+    float h[D];
+    const float kt = ks[t];
+    float ss = 0.f;
+#pragma unroll
+    for (int c = 0; c < D / 4; ++c) {
+        const float4 hv = *reinterpret_cast<const float4 *>(buf + dec_tile_off(t, c));
+        const float4 kv = *reinterpret_cast<const float4 *>(&ks[4 * c]);
+        h[4 * c + 0] = fmaf(bt, hv.x, kt * kv.x);
+        h[4 * c + 1] = fmaf(bt, hv.y, kt * kv.y);
+        h[4 * c + 2] = fmaf(bt, hv.z, kt * kv.z);
+        h[4 * c + 3] = fmaf(bt, hv.w, kt * kv.w);
+        ss = fmaf(h[4 * c], h[4 * c], ss);
+        ss = fmaf(h[4 * c + 1], h[4 * c + 1], ss);
+        ss = fmaf(h[4 * c + 2], h[4 * c + 2], ss);
+        ss = fmaf(h[4 * c + 3], h[4 * c + 3], ss);
+    }
+    ss = warp_sum(ss);
+    if (lane == 0) red[warp] = ss;
+    // buffer free: fetch M while the products run
+    fence_proxy_async_smem();
+    ok = __syncthreads_and(ok);
+    if (t == 0 && ok) {
+        mbar_arrive_expect_tx(&bar[1], D * D * 4);
+        for (int b = 0; b < 4; ++b)
+            tc::tma_load_2d(buf + b * 16384, &maps.state, b * 32, hrow + D, &bar[1]);
+    }
+    float n2 = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) n2 += red[w];
+    const float nrm = sqrtf(n2);
+    const float lam = P.a * nrm;
+    const float invd = nrm > 0.f ? 1.f / (P.half_1p2a * nrm) : 0.f;
+
+    // Chebyshev: thread t keeps element t of x_prev, x_cur
+    float xprev = 0.f, xcur = qt * invd;
+    xbuf[0][t] = xcur;
+    __syncthreads();
+    int cur = 0;
+#pragma unroll 1
+    for (int it = 1; it < P.r; ++it) {
+        float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+#pragma unroll
+        for (int c = 0; c < D / 4; ++c) {
+            const float4 xv = *reinterpret_cast<const float4 *>(&xbuf[cur][4 * c]);
+            y0 = fmaf(h[4 * c], xv.x, y0);
+            y1 = fmaf(h[4 * c + 1], xv.y, y1);
+            y2 = fmaf(h[4 * c + 2], xv.z, y2);
+            y3 = fmaf(h[4 * c + 3], xv.w, y3);
+        }
+        const float y = fmaf(lam, xcur, (y0 + y1) + (y2 + y3));
+        const float xn = fmaf(P.omega[it], fmaf(qt - y, invd, xcur - xprev), xprev);
+        xprev = xcur;
+        xcur = xn;
+        xbuf[cur ^ 1][t] = xn;
+        __syncthreads();
+        cur ^= 1;
+    }
+
+    // M row t: m = beta m + v_t k, o_t = m . x; the updated row goes back in place
+    if (!mbar_wait_bounded(&bar[1], 0, kDecodeWaitProbes)) ok = false;
+    float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
+#pragma unroll
+    for (int c = 0; c < D / 4; ++c) {
+        float4 *p = reinterpret_cast<float4 *>(buf + dec_tile_off(t, c));
+        float4 mv = *p;
+        const float4 kv = *reinterpret_cast<const float4 *>(&ks[4 * c]);
+        const float4 xv = *reinterpret_cast<const float4 *>(&xbuf[cur][4 * c]);
+        mv.x = fmaf(bt, mv.x, vt * kv.x);
+        mv.y = fmaf(bt, mv.y, vt * kv.y);
+        mv.z = fmaf(bt, mv.z, vt * kv.z);
+        mv.w = fmaf(bt, mv.w, vt * kv.w);
+        o0 = fmaf(mv.x, xv.x, o0);
+        o1 = fmaf(mv.y, xv.y, o1);
+        o2 = fmaf(mv.z, xv.z, o2);
+        o3 = fmaf(mv.w, xv.w, o3);
+        *p = mv;
+    }
+    store_f(o + (size_t)head * D + t, invd > 0.f ? (o0 + o1) + (o2 + o3) : 0.f);
+    fence_proxy_async_smem();
+    ok = __syncthreads_and(ok);
+    if (t == 0 && ok) {
+        for (int b = 0; b < 4; ++b) tc::tma_store_2d(&maps.state, b * 32, hrow + D, buf + b * 16384);
+        tc::bulk_commit();
+        tc::bulk_wait_read0();
+    }
+    __syncthreads();
+    // updated H row t back through the buffer
+#pragma unroll
+    for (int c = 0; c < D / 4; ++c)
+        *reinterpret_cast<float4 *>(buf + dec_tile_off(t, c)) =
+            make_float4(h[4 * c], h[4 * c + 1], h[4 * c + 2], h[4 * c + 3]);
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (t == 0) {
+        if (ok) {
+            for (int b = 0; b < 4; ++b) tc::tma_store_2d(&maps.state, b * 32, hrow, buf + b * 16384);
+            tc::bulk_commit();
+            tc::bulk_wait0();
+        } else {
+            atomicExch(timeout_flag, 1);
+            mbar_wait_bounded(&bar[0], 0, kDecodeWaitProbes);
+            mbar_wait_bounded(&bar[1], 0, kDecodeWaitProbes);
+        }
     }
 }
 

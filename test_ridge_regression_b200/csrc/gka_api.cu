@@ -353,18 +353,21 @@ static int sm_count() {
 }
 
 template <typename Tin>
-static int decode_pipelined_launch(float *state, const void *q, const void *k, const void *v,
-                                   const float *beta, void *o, int BH, const ChebParams &P,
-                                   cudaStream_t s) {
+static int decode_rows_launch(float *state, const void *q, const void *k, const void *v,
+                              const float *beta, void *o, int BH, const ChebParams &P,
+                              cudaStream_t s) {
     int *flag = nullptr;
     if (int rc = timeout_flag_ptr(&flag)) return rc;
-    cudaError_t e = set_smem(k_decode_pipelined<Tin>, kDecSmem);
+    DecodeMaps maps;
+    if (int rc = rows128_map(&maps.state, state, (uint64_t)BH * 2 * kDecD,
+                             CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 32, 128))
+        return rc;
+    cudaError_t e = set_smem(k_decode_rows<Tin>, kDecRowSmem);
     if (e != cudaSuccess) return cuda_fail(e);
-    const int grid = BH < sm_count() ? BH : sm_count();
     ProfScope ps(GKA_KERNEL_DECODE_STEP, s);
-    k_decode_pipelined<Tin><<<grid, kDecThreads, kDecSmem, s>>>(
-        state, static_cast<const Tin *>(q), static_cast<const Tin *>(k),
-        static_cast<const Tin *>(v), beta, static_cast<Tin *>(o), BH, P, flag);
+    k_decode_rows<Tin><<<BH, kDecRowThreads, kDecRowSmem, s>>>(
+        maps, static_cast<const Tin *>(q), static_cast<const Tin *>(k),
+        static_cast<const Tin *>(v), beta, static_cast<Tin *>(o), P, flag);
     return check_launch();
 }
 
@@ -372,7 +375,7 @@ template <typename Tin>
 static int decode_dispatch(float *state, const void *q, const void *k, const void *v,
                            const float *beta, void *o, int BH, int D, const ChebParams &P,
                            cudaStream_t s) {
-    if (D == 128) return decode_pipelined_launch<Tin>(state, q, k, v, beta, o, BH, P, s);
+    if (D == 128) return decode_rows_launch<Tin>(state, q, k, v, beta, o, BH, P, s);
     switch (D) {
         case 32: return decode_launch<Tin, 32>(state, q, k, v, beta, o, BH, P, s);
         case 64: return decode_launch<Tin, 64>(state, q, k, v, beta, o, BH, P, s);
