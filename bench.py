@@ -32,6 +32,36 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
                   "sm_max_mhz": 1965.0}
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one ncu capture per
+# kernel, with the SHA-1 of the kernel's source file at capture time: when the
+# source has changed since, the figure no longer describes the kernel and the
+# bench reports null.  Captures and commands: profiles/*.md.
+TRAFFIC = {
+    # full-size forward workload (B8 H8 T2048 D128, chunk 64), one launch
+    "chunk_solve_tc": {"bytes": 235.544576e6 + 24.613376e6, "workload": "bf16_b8h8t2048d128",
+                       "src": "test_ridge_regression_b200/csrc/solve_tc.cuh",
+                       "sha1": "fb4d6c766862ea733917bb5603f7f55c701a76e6"},
+    # decode captured on 64 x 32 heads (state above L2), scaled x4 to 256 x 32 heads
+    "decode_step": {"bytes": 4 * (270.054912e6 + 213.513472e6), "workload": "decode_bf16_b256h32d128",
+                    "src": "test_ridge_regression_b200/csrc/decode.cuh",
+                    "sha1": "9fed00ad526c1e277840c391aca09dea977665ff"},
+}
+
+
+def traffic_of(kernel, workload):
+    import hashlib
+    t = TRAFFIC.get(kernel)
+    if not t or t["workload"] != workload:
+        return None
+    try:
+        with open(os.path.join(ROOT, t["src"]), "rb") as f:
+            if hashlib.sha1(f.read()).hexdigest() != t["sha1"]:
+                return None
+    except OSError:
+        return None
+    return t["bytes"]
+
+
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
@@ -331,8 +361,10 @@ def main():
         peak_note = "fp32 FMA: 148 SMs x 128 lanes x 2 flop x max SM clock"
     achieved = kernel_flops / (per_step_ms / 1e3) / 1e12
     whole_flops = (ch + out + upd + nrm) * head_tok
+    tr = traffic_of(dom_name, w.name)
     roofline = {"bound": bound, "kernel": dom_name, "achieved": achieved, "peak": peak,
-                "unit": punit, "frac": achieved / peak, "traffic": None,
+                "unit": punit, "frac": achieved / peak,
+                "traffic": None if tr is None else tr * (dom_n / args.steps),
                 "peak_source": peak_note,
                 "launches_per_step": dom_n / args.steps,
                 "algorithmic_per_step": kernel_flops,
@@ -462,7 +494,8 @@ def bench_decode(args, dev, peaks):
         "tokens_per_s": w.batch / (ms / 1e3), "GB_per_s": bytes_step / (ms / 1e3) / 1e9,
         "roofline": {"bound": "hbm", "kernel": "decode_step", "achieved": achieved,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": traffic_of("decode_step", w.name) if w.batch == 256 else None,
                      "algorithmic_per_launch": bytes_step,
                      "peak_source": f"{peaks['_source']} copy bandwidth"},
         "gpu_launches": k_n, "clocks": clk.summary(),
