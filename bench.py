@@ -264,9 +264,8 @@ def run_reference(args, w, cfg, rank, world):
 
 def main():
     args = parse()
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from test_ridge_regression_b200 import dist as gdist
+    rank, world, local = gdist.rank_env()
     from test_ridge_regression_b200.inputs import WORKLOADS
     w = WORKLOADS[args.workload]
     cfg = {"workload": w.name, "B": w.B, "heads": w.H, "T": w.T, "D": w.D, "chunk": w.chunk,
@@ -286,16 +285,16 @@ def main():
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
-                                device_id=dev)
+        gdist.init("nccl", timeout_s=120, device=dev)
 
     def barrier():
         if world > 1:
             dist.barrier()
 
     peaks = load_peaks()
-    q, k, v, beta = workload_inputs(w)
+    # every rank runs its own batch (weak scaling over independent sequences)
+    from dataclasses import replace as _replace
+    q, k, v, beta = workload_inputs(_replace(w, seed=gdist.shard_seed(w.seed, rank)))
     qd, kd, vd, bd = (t.to(dev) for t in (q, k, v, beta))
     od = torch.empty_like(vd)
     ws = gka.alloc_workspace(w.B, w.H, w.T, w.D, w.chunk, w.dtype, dev)
@@ -328,11 +327,7 @@ def main():
     gka.profiler_enable(False)
     kt = gka.profiler_read()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = gdist.max_over_ranks(sum(step_ms), dev)
     ms_per_step = total_ms / args.steps
     tok_step = w.B * w.T
     value = world * tok_step * args.steps / (total_ms / 1e3)
@@ -403,11 +398,7 @@ def main():
         e_ends[i].record()
     torch.cuda.synchronize()
     barrier()
-    e_ms = sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends))
-    if world > 1:
-        t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e_ms = float(t.item())
+    e_ms = gdist.max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends)), dev)
     h2d = sum(t.numel() * t.element_size() for t in (q, k, v, beta))
     result["e2e"] = {"value": world * tok_step * args.steps / (e_ms / 1e3), "unit": "tokens/s",
                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": oh.numel() * oh.element_size()}

@@ -162,6 +162,14 @@ int gka_decode_step(float *state, const void *q, const void *k, const void *v,
  * else GKA_OK. */
 int gka_device_status(void *stream);
 
+/* Failure-reporting self-test (no counterpart in the paper): launches one
+ * thread that waits, with a short bound, on a barrier nothing completes, so
+ * the bounded wait gives up and raises the device flag exactly as a stuck
+ * kernel of this library would.  The following gka_device_status() then
+ * returns GKA_ERR_DEVICE_TIMEOUT (and clears the flag); the context stays
+ * usable.  Returns a gka_status for the launch. */
+int gka_selftest_timeout(void *stream);
+
 /* CUDA error code (cudaError_t) behind the last GKA_ERR_CUDA, 0 if none. */
 int gka_last_cuda_error(void);
 

@@ -413,6 +413,19 @@ static int static_scratch_address(void **out) {
     return GKA_OK;
 }
 
+// Failure-reporting self-test: one thread waits, with a short probe limit, on an
+// mbarrier phase that nothing completes; the bounded wait gives up, raises the
+// device flag and the kernel returns normally (no trap, no fault, the context
+// stays usable).
+__global__ void k_selftest_timeout(int *timeout_flag, uint32_t probes) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    if (!mbar_wait_bounded(&bar, 0, probes)) atomicExch(timeout_flag, 1);
+    mbar_arrive(&bar);   // complete the phase so the barrier is quiescent at exit
+}
+
 }  // namespace gka
 
 using namespace gka;
@@ -491,6 +504,13 @@ int gka_decode_step(float *state, const void *q, const void *k, const void *v, c
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (dt == GKA_BF16) return decode_dispatch<__nv_bfloat16>(state, q, k, v, beta, o, (int)BH, D, P, s);
     return decode_dispatch<float>(state, q, k, v, beta, o, (int)BH, D, P, s);
+}
+
+int gka_selftest_timeout(void *stream) {
+    int *flag = nullptr;
+    if (int rc = timeout_flag_ptr(&flag)) return rc;
+    k_selftest_timeout<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(flag, 1u << 12);
+    return check_launch();
 }
 
 int gka_device_status(void *stream) {

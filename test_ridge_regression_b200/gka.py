@@ -64,6 +64,8 @@ def _lib():
         lib.gka_forward_static_scratch.restype = i
         lib.gka_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
         lib.gka_decode_step.restype = i
+        lib.gka_selftest_timeout.argtypes = [vp]
+        lib.gka_selftest_timeout.restype = i
         lib.gka_device_status.argtypes = [vp]
         lib.gka_device_status.restype = i
         lib.gka_last_cuda_error.argtypes = []
@@ -190,6 +192,11 @@ def gka_decode_step(state, q, k, v, beta, a: float, r: int, *, o=None, stream=No
                                 B, H, D, dt, float(a), int(r), _stream(stream))
     _check("gka_decode_step", rc)
     return o
+
+
+def selftest_timeout(stream=None) -> None:
+    """Launch the bounded-wait self-test (see include/gka.h)."""
+    _check("gka_selftest_timeout", _lib().gka_selftest_timeout(_stream(stream)))
 
 
 def device_status(stream=None) -> int:
