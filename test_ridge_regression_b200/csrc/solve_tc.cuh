@@ -63,8 +63,8 @@ struct TcSmem {
     static constexpr uint32_t NRM2 = NRM + 16 * MG;          // second warpgroup's E, X [2][MG]
     static constexpr uint32_t UPART = NRM2 + 8 * MG;         // [4 lane quarters][MG] partial u
     static constexpr uint32_t QPART = UPART + 16 * MG;       // [4 lane quarters][TOK] |q_j|^2
-    static constexpr uint32_t DEC = QPART + 16 * TOK;        // l2, b, beta^2: [3][MG] floats
-    static constexpr uint32_t BARS = DEC + 12 * MG;
+    static constexpr uint32_t DEC = QPART + 16 * TOK;        // l2, b, beta, beta^2: [4][MG] floats
+    static constexpr uint32_t BARS = DEC + 16 * MG;
     static constexpr uint32_t TBASE = BARS + 8 * 8;
     static constexpr uint32_t END = TBASE + 16;
     static constexpr size_t bytes = END + 1024;              // + alignment slack
@@ -252,13 +252,16 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     }
     chunk_log_prefix(beta + tok0, MG, ell, wtot);
     // decays of every position: l2_t = l_t log2(e) (fp32, so w_ti = exp2(l2_t - l2_i)),
-    // b_t = exp(l_t), beta_t^2 (from the double prefix)
+    // b_t = exp(l_t), beta_t and beta_t^2 (from the double prefix).  Runs of
+    // weights w_ti over consecutive i or t are products of beta: w_{t,i-1} =
+    // w_ti beta_i and w_{t+1,i} = w_ti beta_{t+1}.
     float *s_l2 = reinterpret_cast<float *>(sm + L::DEC);
-    float *s_bt = s_l2 + MG, *s_beta2 = s_bt + MG;
+    float *s_bt = s_l2 + MG, *s_bet = s_bt + MG, *s_beta2 = s_bet + MG;
     if (tid < MG) {
         s_l2[tid] = (float)(ell[tid] * 1.4426950408889634);
         s_bt[tid] = decay_exp(ell[tid]);
         const float bt = decay_exp(tid == 0 ? ell[0] : ell[tid] - ell[tid - 1]);
+        s_bet[tid] = bt;
         s_beta2[tid] = bt * bt;
     }
     bool ok = mbar_wait_bounded(bar_load, 0, kTcWaitProbes);
@@ -354,26 +357,24 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         const float gs = 1.f / (sK * sK);
         float es = 0.f, xs = 0.f, gjj = 0.f;
         bool has_diag = false;
+        float g[HALF];
 #pragma unroll
-        for (int cb = 0; cb < HALF; cb += 16) {
-            float g[16];
-            tc::tmem_ld16(tl + kGcol + wg * HALF + cb, g);
-            tc::tmem_wait_ld();
-            if (s_owner) {
+        for (int cb = 0; cb < HALF; cb += 16) tc::tmem_ld16(tl + kGcol + wg * HALF + cb, g + cb);
+        tc::tmem_wait_ld();
+        if (s_owner) {
+            // i from the top of this half down: w = w_{key,i}, zero while i > key
+            const int lo = wg * HALF, hi = lo + HALF - 1;
+            float w = key > hi ? exp2f(s_l2[key] - s_l2[hi + 1]) : 0.f;
 #pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const int i = wg * HALF + cb + u;
-                    if (i <= key) {
-                        const float w = exp2f(s_l2[key] - s_l2[i]);
-                        const float gi = g[u] * gs;
-                        xs = fmaf(w, s_u[i], xs);
-                        if (i < key) {
-                            es = fmaf(w * gi, gi, es);
-                        } else {
-                            gjj = gi;
-                            has_diag = true;
-                        }
-                    }
+            for (int u = HALF - 1; u >= 0; --u) {
+                const int i = lo + u;
+                w = (i == key) ? 1.f : w * s_bet[min(i + 1, MG - 1)];   // w = 0 when i + 1 == MG
+                const float gi = g[u] * gs;
+                xs = fmaf(w, s_u[i], xs);
+                if (i < key) es = fmaf(w * gi, gi, es);
+                if (i == key) {
+                    gjj = gi;
+                    has_diag = true;
                 }
             }
         }
@@ -403,26 +404,49 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
                 sq[s2];
     }
     __syncthreads();
-    float *s_n = s_o3;   // per-token norms, then overwritten by the readout coefficient
-    if (tid == 0) {
-        float hs2 = 0.f;
-        for (int w = 0; w < kSolveThreads / 32; ++w) hs2 += red[8 + w];
-        hs2 *= ldexpf(1.f, -2 * eHexp);
-        float R = 0.f;
-        for (int j = 0; j < MG; ++j) {
-            const float E = s_E[j] + s_E1[j], X = s_X[j] + s_X1[j];
-            R = fmaf(s_beta2[j], R, fmaf(2.f, E, s_G[j] * s_G[j]));
-            if (j >= j0 && j < j0 + TOK) {
-                const float b = s_bt[j];
-                const float n2 = fmaf(b * b, hs2, fmaf(2.f * b, X, R));
-                s_n[j - j0] = sqrtf(fmaxf(n2, 0.f));
+    // R_j = beta_j^2 R_{j-1} + (2 E_j + G_jj^2), R_{-1} = 0: an affine recurrence,
+    // scanned by warp 0 (lane l owns MG/32 consecutive positions) into s_u (free now)
+    float *s_R = s_u;
+    if (warp == 0) {
+        constexpr int PER = MG / 32;
+        float ca[PER], cb2[PER];
+        float A = 1.f, Bc = 0.f;   // this lane's positions composed: R_out = A R_in + Bc
+#pragma unroll
+        for (int p = 0; p < PER; ++p) {
+            const int j = lane * PER + p;
+            ca[p] = s_beta2[j];
+            cb2[p] = fmaf(2.f, s_E[j] + s_E1[j], s_G[j] * s_G[j]);
+            Bc = fmaf(ca[p], Bc, cb2[p]);
+            A *= ca[p];
+        }
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {   // inclusive scan of the compositions
+            const float Ap = __shfl_up_sync(0xffffffffu, A, o);
+            const float Bp = __shfl_up_sync(0xffffffffu, Bc, o);
+            if (lane >= o) {
+                Bc = fmaf(A, Bp, Bc);
+                A *= Ap;
             }
+        }
+        float R = __shfl_up_sync(0xffffffffu, Bc, 1);   // R just before this lane's positions
+        if (lane == 0) R = 0.f;
+#pragma unroll
+        for (int p = 0; p < PER; ++p) {
+            R = fmaf(ca[p], R, cb2[p]);
+            s_R[lane * PER + p] = R;
         }
     }
     __syncthreads();
     if (tid < TOK) {
         const int j = tid;
-        const float nj = s_n[j];
+        float hs2 = 0.f;
+#pragma unroll
+        for (int w = 0; w < kSolveThreads / 32; ++w) hs2 += red[8 + w];
+        hs2 *= ldexpf(1.f, -2 * eHexp);
+        const float bj = s_bt[j0 + j];
+        const float n2 = fmaf(bj * bj, hs2,
+                              fmaf(2.f * bj, s_X[j0 + j] + s_X1[j0 + j], s_R[j0 + j]));
+        const float nj = sqrtf(fmaxf(n2, 0.f));
         norms[tok0 + j0 + j] = nj;
         const float invd = nj > 0.f ? 1.f / (P.half_1p2a * nj) : 0.f;
         const float b = s_bt[j0 + j];
@@ -455,13 +479,17 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
 
     // W^T rows: W[i][j] = w_{ji} = exp(l_j - l_i) for i <= j, else 0 (this thread's tokens)
     {
+        // w = w_{j,key} along this thread's tokens j (zero while j < key)
+        const int js = j0 + tcol;
+        float w = (s_owner && key <= js) ? exp2f(s_l2[js] - s_l2[key]) : 0.f;
         float wv[16];
 #pragma unroll
         for (int c = 0; c < NCH; ++c) {
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
-                const int j = j0 + tcol + c * 16 + u;
-                wv[u] = (s_owner && key <= j) ? exp2f(s_l2[j] - s_l2[key]) : 0.f;
+                const int j = js + c * 16 + u;
+                if (c * 16 + u > 0) w = (j == key && s_owner) ? 1.f : w * s_bet[j];
+                wv[u] = w;
             }
             tc::tmem_st16(tl + T_W + tcol + c * 16, wv);
         }
