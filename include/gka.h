@@ -70,8 +70,10 @@ typedef struct {
     size_t norms_offset;    /* fp32 [B, H, T]: ||H_t||_F as used by the solve */
     size_t states_lp_offset;   /* tensor-core path only (0 bytes otherwise): fp16
                                   [B, H, N, 2, D, D] copies of the chunk-start states, each
-                                  scaled by a power of two, then the scales; the region ends
-                                  at total_bytes */
+                                  scaled by a power of two, then the scales, then four fp32
+                                  [B, H, T] planes of per-token decays (log2 of the
+                                  chunk-relative cumulative decay, its exp, beta, beta^2);
+                                  the region ends at total_bytes */
     size_t total_bytes;
 } gka_workspace_layout;
 

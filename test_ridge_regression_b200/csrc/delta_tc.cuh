@@ -14,7 +14,9 @@
 // MMAs: dH = K^T (W K)_hi + K^T (W K)_lo, the same for dM with V^T.
 // Thread d reads row d of each fp32 accumulator from TMEM and writes it to
 // the state slot n + 1.  The CTA also writes the chunk decay b_{C-1} and the
-// increments of the norm bounds used to scale the scan's fp16 state copies.
+// increments of the norm bounds used to scale the scan's fp16 state copies,
+// and every token's decays for the solve: l_t log2(e), b_t = exp(l_t),
+// beta_t and beta_t^2 (l_t the chunk-relative cumulative log, summed in double).
 #pragma once
 
 #include <cuda_fp16.h>
@@ -52,7 +54,8 @@ template <int C>
 __global__ void __launch_bounds__(kTcThreads, 1)
 k_chunk_delta_tc(const __grid_constant__ DeltaMaps maps, const float *__restrict__ beta,
                  float *__restrict__ states, float *__restrict__ decay,
-                 float *__restrict__ bound_inc, int T, int N, int *__restrict__ timeout_flag) {
+                 float *__restrict__ bound_inc, float *__restrict__ tokdec, size_t plane, int T,
+                 int N, int *__restrict__ timeout_flag) {
     using L = DeltaSmem<C>;
     constexpr int D = kTcD;
     extern __shared__ uint8_t smraw[];
@@ -90,6 +93,13 @@ k_chunk_delta_tc(const __grid_constant__ DeltaMaps maps, const float *__restrict
         tc::tmem_relinquish();
     }
     chunk_log_prefix(beta + tok0, C, ell, wtot);
+    if (tid < C) {
+        const float bt = decay_exp(tid == 0 ? ell[0] : ell[tid] - ell[tid - 1]);
+        tokdec[tok0 + tid] = (float)(ell[tid] * 1.4426950408889634);
+        tokdec[plane + tok0 + tid] = decay_exp(ell[tid]);
+        tokdec[2 * plane + tok0 + tid] = bt;
+        tokdec[3 * plane + tok0 + tid] = bt * bt;
+    }
     bool ok = mbar_wait_bounded(bar_load, 0, kTcWaitProbes);
     const float sK = tile_bf16_to_f16_scaled(sm + L::KT, C * 256, red);
     const float sV = tile_bf16_to_f16_scaled(sm + L::VT, C * 256, red);

@@ -131,6 +131,7 @@ static int layout(int B, int H, int T, int D, int C, gka_dtype dt, gka_workspace
         off = round256(off + 2 * BH * N * 2 * (size_t)D * D);   // fp16 states
         off = round256(off + sizeof(float) * BH * N * 2);       // norm-bound increments
         off = round256(off + sizeof(int) * BH * N * 2);         // state exponents
+        off = round256(off + 4 * sizeof(float) * BH * (size_t)T);   // per-token decays
     }
     L->total_bytes = off;
     return GKA_OK;
@@ -242,6 +243,10 @@ static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
                                                  round256(2 * BHN2 * (size_t)D * D));
     int *sexp = reinterpret_cast<int *>(reinterpret_cast<char *>(bound_inc) +
                                         round256(sizeof(float) * BHN2));
+    // per-token decays, 4 planes of B*H*T floats: l2, b, beta, beta^2
+    const size_t plane = (size_t)BH * T;
+    float *tokdec = reinterpret_cast<float *>(reinterpret_cast<char *>(sexp) +
+                                              round256(sizeof(int) * BHN2));
     int *flag = nullptr;
     if (int rc = timeout_flag_ptr(&flag)) return rc;
     TcMaps maps;
@@ -263,13 +268,13 @@ static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
             return cuda_fail(e);
         ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
         k_chunk_delta_tc<64><<<dim3(N, BH), kTcThreads, DeltaSmem<64>::bytes, s>>>(
-            dmaps, beta, states, decay, bound_inc, T, N, flag);
+            dmaps, beta, states, decay, bound_inc, tokdec, plane, T, N, flag);
     } else {
         if ((e = set_smem(k_chunk_delta_tc<128>, DeltaSmem<128>::bytes)) != cudaSuccess)
             return cuda_fail(e);
         ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
         k_chunk_delta_tc<128><<<dim3(N, BH), kTcThreads, DeltaSmem<128>::bytes, s>>>(
-            dmaps, beta, states, decay, bound_inc, T, N, flag);
+            dmaps, beta, states, decay, bound_inc, tokdec, plane, T, N, flag);
     }
     if (int rc = check_launch()) return rc;
 
@@ -285,14 +290,14 @@ static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
         if ((e = set_smem(kern, TcSmem<64, 64>::bytes)) != cudaSuccess) return cuda_fail(e);
         ProfScope ps(GKA_KERNEL_CHUNK_SOLVE_TC, s);
         kern<<<dim3(N, BH), kSolveThreads, TcSmem<64, 64>::bytes, s>>>(
-            maps, q, beta, norms, sexp, o, T, N, C, 0, P, flag);
+            maps, q, tokdec, plane, norms, sexp, o, T, N, C, 0, P, flag);
     } else {
         // one CTA per 128-token chunk (N = 128 MMAs)
         auto kern = k_chunk_solve_tc<128, 128>;
         if ((e = set_smem(kern, TcSmem<128, 128>::bytes)) != cudaSuccess) return cuda_fail(e);
         ProfScope ps(GKA_KERNEL_CHUNK_SOLVE_TC, s);
         kern<<<dim3(N, BH), kSolveThreads, TcSmem<128, 128>::bytes, s>>>(
-            maps, q, beta, norms, sexp, o, T, N, C, 0, P, flag);
+            maps, q, tokdec, plane, norms, sexp, o, T, N, C, 0, P, flag);
     }
     if (int rc = check_launch()) return rc;
     return GKA_OK;

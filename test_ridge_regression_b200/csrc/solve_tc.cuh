@@ -51,24 +51,29 @@ template <int MG, int TOK>
 struct TcSmem {
     // byte offsets from a 1024-aligned base
     static constexpr uint32_t HM = 0;                        // H_s, later M_s: 2 x [128][64] fp16
-    static constexpr uint32_t KT = HM + 32768;               // keys:   2 x [MG][64]
-    static constexpr uint32_t VT = KT + MG * 256;            // values: 2 x [MG][64]
-    static constexpr uint32_t XT = VT + MG * 256;            // X^T: TOK/64 x [128][64], MN-major
+    static constexpr uint32_t VT = HM + 32768;               // values: 2 x [MG][64]
+    static constexpr uint32_t KT = VT + MG * 256;            // keys:   2 x [MG][64]
+    static constexpr uint32_t XT = KT + MG * 256;            // X^T: TOK/64 x [128][64], MN-major
     static constexpr uint32_t PT = XT + TOK * 256;           // P^T: TOK/64 x [MG][64], MN-major
     static constexpr uint32_t QS = PT + TOK * MG * 2;        // q: [TOK][128] bf16, then q^T
     static constexpr uint32_t SCAL = QS + TOK * 256;         // per-token scalars [5][TOK]
-    static constexpr uint32_t ELL = SCAL + 8 * 4 * TOK;      // double[MG] cumulative logs
-    static constexpr uint32_t RED = ELL + 8 * MG + 8 * (kSolveThreads / 32);  // float[16]
+    static constexpr uint32_t RED = SCAL + 8 * 4 * TOK;      // float[16]
     static constexpr uint32_t NRM = RED + 64;                // u, E, X, Gjj [4][MG]
     static constexpr uint32_t NRM2 = NRM + 16 * MG;          // second warpgroup's E, X [2][MG]
     static constexpr uint32_t UPART = NRM2 + 8 * MG;         // [4 lane quarters][MG] partial u
     static constexpr uint32_t QPART = UPART + 16 * MG;       // [4 lane quarters][TOK] |q_j|^2
     static constexpr uint32_t DEC = QPART + 16 * TOK;        // l2, b, beta, beta^2: [4][MG] floats
+    // [2 rounds][3][TOK] w * (cq, c1, c3) of the rounds: over UPART and QPART,
+    // set-up scratch that is dead once the rounds start
+    static constexpr uint32_t COEF = UPART;
+    static_assert(24 * TOK <= DEC - UPART, "coefficient tables overrun the set-up scratch");
     static constexpr uint32_t BARS = DEC + 16 * MG;
     static constexpr uint32_t TBASE = BARS + 8 * 8;
     static constexpr uint32_t END = TBASE + 16;
     static constexpr size_t bytes = END + 1024;              // + alignment slack
 };
+// two 64-token CTAs must fit one SM (228 KiB, of which 1 KiB per CTA is reserved)
+static_assert(TcSmem<64, 64>::bytes <= 233472 / 2 - 1024, "64-token solve: two CTAs per SM");
 
 struct TcMaps {
     CUtensorMap k;       // [B*H*T rows][128] bf16, box 64 x 64, 128B swizzle
@@ -190,7 +195,7 @@ __device__ __forceinline__ void reduce_scatter32(float (&v)[N], int lane) {
 template <int MG, int TOK>
 __global__ void __launch_bounds__(kSolveThreads, TOK == 64 ? 2 : 1)
 k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__restrict__ q,
-                 const float *__restrict__ beta, float *__restrict__ norms,
+                 const float *__restrict__ tokdec, size_t plane, float *__restrict__ norms,
                  const int *__restrict__ state_exp, __nv_bfloat16 *__restrict__ o, int T, int N,
                  int C, int group, const ChebParams P, int *__restrict__ timeout_flag) {
     using L = TcSmem<MG, TOK>;
@@ -207,12 +212,11 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     float *s_c3 = s_c1 + TOK;                                // coefficient of Z3
     float *s_o1 = s_c3 + TOK;                                // readout coefficient of Z1
     float *s_o3 = s_o1 + TOK;                                // readout coefficient of Z3
-    double *ell = reinterpret_cast<double *>(sm + L::ELL);
-    double *wtot = ell + MG;
+    float *s_coef = reinterpret_cast<float *>(sm + L::COEF);
     float *red = reinterpret_cast<float *>(sm + L::RED);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BARS);
     uint64_t *bar_load = &bars[0], *bar_v = &bars[1], *bar_m = &bars[2], *bar_s = &bars[3],
-             *bar_z = &bars[4], *bar_fin = &bars[5], *bar_n = &bars[6];
+             *bar_z = &bars[4], *bar_fin = &bars[5], *bar_n = &bars[6], *bar_z1 = &bars[7];
     uint32_t *tbase = reinterpret_cast<uint32_t *>(sm + L::TBASE);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -225,12 +229,12 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     const int srow = (int)(((size_t)bh * N + n) * 2 * kTcD);   // H_s row in the state map
 
     if (tid == 0) {
-        for (int i = 0; i < 7; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 8; ++i) mbar_init(&bars[i], i == 5 ? 2 : 1);   // bar_fin: 2
         fence_mbar_init();
     }
     __syncthreads();
     if (tid == 0) {
-        mbar_arrive_expect_tx(bar_load, 32768 + MG * 256 + TOK * kTcD * 2);
+        mbar_arrive_expect_tx(bar_load, 32768 + MG * 256 + TOK * kTcD * 2 + 16 * MG);
         for (int h = 0; h < 2; ++h) {
             for (int rb = 0; rb < 2; ++rb)
                 tc::tma_load_2d(sm + L::HM + h * 16384 + rb * 8192, &maps.state, h * 64,
@@ -240,6 +244,8 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
                                 (int)tok0 + rb * 64, bar_load);
         }
         bulk_g2s(sm + L::QS, q + (tok0 + j0) * kTcD, TOK * kTcD * 2, bar_load);
+        for (int pl = 0; pl < 4; ++pl)
+            bulk_g2s(sm + L::DEC + pl * 4 * MG, tokdec + pl * plane + tok0, 4 * MG, bar_load);
         mbar_arrive_expect_tx(bar_v, MG * 256);
         for (int h = 0; h < 2; ++h)
             for (int rb = 0; rb < MG / 64; ++rb)
@@ -250,20 +256,12 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         tc::tmem_alloc(tbase, TMEM_COLS);
         tc::tmem_relinquish();
     }
-    chunk_log_prefix(beta + tok0, MG, ell, wtot);
-    // decays of every position: l2_t = l_t log2(e) (fp32, so w_ti = exp2(l2_t - l2_i)),
-    // b_t = exp(l_t), beta_t and beta_t^2 (from the double prefix).  Runs of
-    // weights w_ti over consecutive i or t are products of beta: w_{t,i-1} =
-    // w_ti beta_i and w_{t+1,i} = w_ti beta_{t+1}.
+    // decays of every position (from the state pass): l2_t = l_t log2(e) with l_t
+    // the chunk-relative cumulative log (w_ti = exp2(l2_t - l2_i)), b_t = exp(l_t),
+    // beta_t and beta_t^2.  Runs of weights w_ti over consecutive i or t are
+    // products of beta: w_{t,i-1} = w_ti beta_i and w_{t+1,i} = w_ti beta_{t+1}.
     float *s_l2 = reinterpret_cast<float *>(sm + L::DEC);
     float *s_bt = s_l2 + MG, *s_bet = s_bt + MG, *s_beta2 = s_bet + MG;
-    if (tid < MG) {
-        s_l2[tid] = (float)(ell[tid] * 1.4426950408889634);
-        s_bt[tid] = decay_exp(ell[tid]);
-        const float bt = decay_exp(tid == 0 ? ell[0] : ell[tid] - ell[tid - 1]);
-        s_bet[tid] = bt;
-        s_beta2[tid] = bt * bt;
-    }
     bool ok = mbar_wait_bounded(bar_load, 0, kTcWaitProbes);
     ok = mbar_wait_bounded(bar_v, 0, kTcWaitProbes) && ok;
     // keys and values: bf16 -> fp16 in place, scaled below 1
@@ -283,10 +281,20 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     const uint32_t a_hm = sb + L::HM, a_kt = sb + L::KT, a_vt = sb + L::VT, b_xt = sb + L::XT,
                    b_pt = sb + L::PT;
 
-    // rows of S (keys) held by this thread: M = 64 puts key 16w + l in lane
+    // Rows of S = K X^T (keys) held by this thread.  With MG = 64 the S product is
+    // issued with M = 128 and an A operand that starts 32 rows (4 KB) before the key
+    // tile: key t lands in TMEM lane 32 + t (lane quarters 1 and 2), and lanes 0-31
+    // and 96-127 receive products of the neighbouring tiles (values, X^T: finite fp16
+    // data not written meanwhile), which nothing reads.  This costs the same tensor
+    // time as M = 64 and leaves lane quarters 0 and 3 out of the P phase.  MG = 128:
+    // key t in lane t.
+    constexpr bool kSOffset = (MG == 64);
+    const bool s_owner = kSOffset ? (quarter == 1 || quarter == 2) : true;
+    const int key = kSOffset ? d - 32 : d;
+    // rows of G = K K^T (norm set-up, M = MG): M = 64 puts key 16w + l in lane
     // 32w + l (l < 16); M = 128 puts key t in lane t.
-    const bool s_owner = (MG == 128) || (lane < 16);
-    const int key = (MG == 128) ? d : quarter * 16 + lane;
+    const bool g_owner = (MG == 128) || (lane < 16);
+    const int gkey = (MG == 128) ? d : quarter * 16 + lane;
 
     // ---- per-token ||H_j||_F (ai.info, Methodology: closed form through the
     // key Gram matrix).  Zn = H_s K^T gives u_i = k_i^T H_s k_i, G = K K^T the
@@ -353,7 +361,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
                               upart[3 * MG + tid]) * inv_uscale;
     __syncthreads();
     {
-        // row `key` of G over this warpgroup's half of the columns: E, X, G_key,key
+        // row `gkey` of G over this warpgroup's half of the columns: E, X, G_gkey,gkey
         const float gs = 1.f / (sK * sK);
         float es = 0.f, xs = 0.f, gjj = 0.f;
         bool has_diag = false;
@@ -361,27 +369,27 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
 #pragma unroll
         for (int cb = 0; cb < HALF; cb += 16) tc::tmem_ld16(tl + kGcol + wg * HALF + cb, g + cb);
         tc::tmem_wait_ld();
-        if (s_owner) {
-            // i from the top of this half down: w = w_{key,i}, zero while i > key
+        if (g_owner) {
+            // i from the top of this half down: w = w_{gkey,i}, zero while i > gkey
             const int lo = wg * HALF, hi = lo + HALF - 1;
-            float w = key > hi ? exp2f(s_l2[key] - s_l2[hi + 1]) : 0.f;
+            float w = gkey > hi ? exp2f(s_l2[gkey] - s_l2[hi + 1]) : 0.f;
 #pragma unroll
             for (int u = HALF - 1; u >= 0; --u) {
                 const int i = lo + u;
-                w = (i == key) ? 1.f : w * s_bet[min(i + 1, MG - 1)];   // w = 0 when i + 1 == MG
+                w = (i == gkey) ? 1.f : w * s_bet[min(i + 1, MG - 1)];   // w = 0 when i + 1 == MG
                 const float gi = g[u] * gs;
                 xs = fmaf(w, s_u[i], xs);
-                if (i < key) es = fmaf(w * gi, gi, es);
-                if (i == key) {
+                if (i < gkey) es = fmaf(w * gi, gi, es);
+                if (i == gkey) {
                     gjj = gi;
                     has_diag = true;
                 }
             }
         }
-        if (s_owner) {
-            (wg == 0 ? s_E : s_E1)[key] = es;
-            (wg == 0 ? s_X : s_X1)[key] = xs;
-            if (has_diag) s_G[key] = gjj;
+        if (g_owner) {
+            (wg == 0 ? s_E : s_E1)[gkey] = es;
+            (wg == 0 ? s_X : s_X1)[gkey] = xs;
+            if (has_diag) s_G[gkey] = gjj;
         }
     }
     // q column of this thread's tokens (token-major tile), kept packed for the
@@ -514,27 +522,43 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         }
         tc::tmem_wait_st();
     }
+    if (P.r > 1) {   // round 1's coefficient table (s_cq, s_c1, s_c3 are consecutive)
+        for (int e = tid; e < 3 * TOK; e += kSolveThreads) s_coef[3 * TOK + e] = P.omega[1] * s_cq[e];
+    }
     fence_proxy_async_smem();
     tc::fence_before_sync();
     ok = __syncthreads_and(ok);
 
-    constexpr uint32_t IDESC_S = tc::idesc_f16(MG, TOK, false, true);
+    constexpr uint32_t IDESC_S = tc::idesc_f16(kSOffset ? 128 : MG, TOK, false, true);
+    const uint32_t a_s = a_kt - (kSOffset ? 4096u : 0u);   // A operand start of S
     constexpr uint32_t IDESC_Z1 = tc::idesc_f16(128, TOK, false, true);
     constexpr uint32_t IDESC_Z3 = tc::idesc_f16(128, TOK, true, true);
     constexpr uint32_t PT_BLOCK = MG * 128;   // bytes between 64-token blocks of P^T
+    // P-phase warps and the issuer of the intra-chunk product Z3
+    constexpr int kZ3Issuer = kSOffset ? 96 : 128;   // lane 0 of warp 3 (MG 64) or 4 (MG 128)
+    constexpr int kPBarThreads = kSOffset ? 5 * 32 : kSolveThreads - 32;
+    const bool p_warp = kSOffset ? s_owner : (warp != 0);
+    const bool in_pbar = p_warp || warp == kZ3Issuer / 32;
     bool m_requested = false;
-    uint32_t ph = 0;   // phase parity of bar_s / bar_z (both complete once per round)
+    uint32_t ph = 0;   // phase parity of bar_s / bar_z1 / bar_z (each completes once per round)
 
+    // Round structure.  Thread 0 issues S = K X^T (commit bar_s) and Z1 = H_s X^T
+    // (commit bar_z1); issuing blocks it for about as long as the tensor core works,
+    // so warp 0 takes no part in the P phase.  MG = 64: the key rows of S sit in
+    // lane quarters 1-2, so warps 1, 2, 5, 6 form P and warp 3 issues Z3.  MG = 128:
+    // warps 1-7 form P, warp 4 also covering warp 0's lane quarter, and warp 4
+    // issues Z3.  The P warps and the Z3 issuer meet at a named barrier, so Z3 =
+    // K^T P^T (commit bar_z) need not wait for the Z1 issue to finish.
 #pragma unroll 1
     for (int it = 1; it <= P.r && ok; ++it) {
         const bool out_pass = (it == P.r);
+        const float w_next = P.omega[it + 1 < kMaxSteps ? it + 1 : 0];   // next round's weight
         if (tid == 0) {
             tc::fence_after_sync();
-            // S^T = K X^T
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
                 tc::mma_f16(tmem + T_S,
-                            tc::sdesc(a_kt + (kk >> 2) * (MG * 128) + (kk & 3) * 32, 16, 1024),
+                            tc::sdesc(a_s + (kk >> 2) * (MG * 128) + (kk & 3) * 32, 16, 1024),
                             tc::sdesc(b_xt + kk * 2048, 16384, 1024), IDESC_S, kk > 0);
             tc::commit(bar_s);
             if (out_pass) {
@@ -556,40 +580,48 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
                                 tc::sdesc(a_hm + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
                                 tc::sdesc(b_xt + kk * 2048, 16384, 1024), IDESC_Z1, kk > 0);
             }
+            tc::commit(bar_z1);
         }
-        // P^T = W o S^T  -> fp16, MN-major tile of MG rows (this thread's 32 tokens)
-        if (!mbar_wait_bounded(bar_s, ph, kTcWaitProbes)) ok = false;
-        tc::fence_after_sync();
+        // the issuing lane's warp reconverges before anyone in it waits on a barrier
+        // that this lane's issue completes (a suspended wait would stall the issue)
+        if (warp == 0) __syncwarp();
+        if (in_pbar) {
+            if (p_warp) {
+                // P^T = W o S^T -> fp16, MN-major tile of MG rows
+                if (!mbar_wait_bounded(bar_s, ph, kTcWaitProbes)) ok = false;
+                tc::fence_after_sync();
+                const bool both = !kSOffset && warp == 4;
+#pragma unroll 1
+                for (int hh = 0; hh < (both ? 2 : 1); ++hh) {
+                    const int tb = both ? hh * TPT : tcol;
 #pragma unroll
-        for (int c = 0; c < NCH; c += 2) {
-            const int t0 = tcol + c * 16;
-            float sv[32], wv[32];
-            tc::tmem_ld16(tl + T_S + t0, sv);
-            tc::tmem_ld16(tl + T_S + t0 + 16, sv + 16);
-            tc::tmem_ld16(tl + T_W + t0, wv);
-            tc::tmem_ld16(tl + T_W + t0 + 16, wv + 16);
-            tc::tmem_wait_ld();
+                    for (int c = 0; c < NCH; ++c) {
+                        const int t0 = tb + c * 16;
+                        float sv[16], wv[16];
+                        tc::tmem_ld16(tl + T_S + t0, sv);
+                        tc::tmem_ld16(tl + T_W + t0, wv);
+                        tc::tmem_wait_ld();
 #pragma unroll
-            for (int u = 0; u < 32; ++u) sv[u] *= wv[u];
-            if (s_owner) {
-                const uint32_t pt = b_pt + (t0 >> 6) * PT_BLOCK;
-                st_row16(pt, key, t0 & 63, sv);
-                st_row16(pt, key, (t0 & 63) + 16, sv + 16);
+                        for (int u = 0; u < 16; ++u) sv[u] *= wv[u];
+                        st_row16(b_pt + (t0 >> 6) * PT_BLOCK, key, t0 & 63, sv);
+                    }
+                }
+                fence_proxy_async_smem();
+                tc::fence_before_sync();
             }
-        }
-        fence_proxy_async_smem();
-        tc::fence_before_sync();
-        ok = __syncthreads_and(ok);
-        if (!ok) break;
-        if (tid == 0) {
-            tc::fence_after_sync();
-            const uint32_t a3 = out_pass ? a_vt : a_kt;
+            named_barrier_sync(1, kPBarThreads);
+            if (tid == kZ3Issuer) {
+                tc::fence_after_sync();
+                const uint32_t a3 = out_pass ? a_vt : a_kt;
 #pragma unroll
-            for (int kk = 0; kk < MG / 16; ++kk)
-                tc::mma_f16(tmem + T_Z3, tc::sdesc(a3 + kk * 2048, MG * 128, 1024),
-                            tc::sdesc(b_pt + kk * 2048, PT_BLOCK, 1024), IDESC_Z3, kk > 0);
-            tc::commit(bar_z);
+                for (int kk = 0; kk < MG / 16; ++kk)
+                    tc::mma_f16(tmem + T_Z3, tc::sdesc(a3 + kk * 2048, MG * 128, 1024),
+                                tc::sdesc(b_pt + kk * 2048, PT_BLOCK, 1024), IDESC_Z3, kk > 0);
+                tc::commit(bar_z);
+            }
+            if (warp == kZ3Issuer / 32) __syncwarp();
         }
+        if (!mbar_wait_bounded(bar_z1, ph, kTcWaitProbes)) ok = false;
         if (!mbar_wait_bounded(bar_z, ph, kTcWaitProbes)) ok = false;
         tc::fence_after_sync();
         ph ^= 1u;
@@ -603,7 +635,13 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
                                         srow + kTcD + rb * 64, bar_m);
                 m_requested = true;
             }
-            const float w = P.omega[it];
+            // x_new = (1 - w) x_prev + w (1 - lambda/d) x + w cq q - w c1 Z1 - w c3 Z3
+            // (the three-term update with the residual (q - A x)/d written out); the
+            // per-token products w cq, w c1, w c3 of this round come from the table
+            const float cA = 1.f - P.omega[it], cB = P.omega[it] * (1.f - cl);
+            const float *kq = s_coef + (it & 1) * 3 * TOK, *k1 = kq + TOK, *k3 = k1 + TOK;
+            // the previous round's x_prev stores (not waited for at its end) land first
+            tc::tmem_wait_st();
 #pragma unroll
             for (int c = 0; c < NCH; ++c) {
                 const int t0 = tcol + c * 16;
@@ -616,20 +654,17 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
                 float xn[16];
 #pragma unroll
                 for (int u4 = 0; u4 < 16; u4 += 4) {
-                    const float4 cq = *reinterpret_cast<const float4 *>(s_cq + t0 + u4);
-                    const float4 c1 = *reinterpret_cast<const float4 *>(s_c1 + t0 + u4);
-                    const float4 c3 = *reinterpret_cast<const float4 *>(s_c3 + t0 + u4);
-                    const float cqv[4] = {cq.x, cq.y, cq.z, cq.w};
-                    const float c1v[4] = {c1.x, c1.y, c1.z, c1.w};
-                    const float c3v[4] = {c3.x, c3.y, c3.z, c3.w};
+                    const float4 gq = *reinterpret_cast<const float4 *>(kq + t0 + u4);
+                    const float4 g1 = *reinterpret_cast<const float4 *>(k1 + t0 + u4);
+                    const float4 g3 = *reinterpret_cast<const float4 *>(k3 + t0 + u4);
+                    const float gqv[4] = {gq.x, gq.y, gq.z, gq.w};
+                    const float g1v[4] = {g1.x, g1.y, g1.z, g1.w};
+                    const float g3v[4] = {g3.x, g3.y, g3.z, g3.w};
 #pragma unroll
                     for (int v = 0; v < 4; ++v) {
                         const int u = u4 + v;
-                        // (q - A x)/d, scaled: cq q - c1 (H_s x~) - c3 (intra x~) - (lambda/d) x~
-                        const float r = fmaf(cqv[v], qv[u], -fmaf(c1v[v], z1[u],
-                                                                  fmaf(c3v[v], z3[u],
-                                                                       cl * xc[c * 16 + u])));
-                        xn[u] = fmaf(w, r + xc[c * 16 + u] - xp[u], xp[u]);
+                        const float t = fmaf(gqv[v], qv[u], -fmaf(g1v[v], z1[u], g3v[v] * z3[u]));
+                        xn[u] = fmaf(cA, xp[u], fmaf(cB, xc[c * 16 + u], t));
                     }
                 }
                 tc::tmem_st16(tl + T_XP + t0, &xc[c * 16]);
@@ -637,7 +672,11 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
                 for (int u = 0; u < 16; ++u) xc[c * 16 + u] = xn[u];
                 st_row16(sb + L::XT + (t0 >> 6) * 16384u, d, t0 & 63, xn);
             }
-            tc::tmem_wait_st();
+            // the next round's coefficient table (the other buffer)
+            if (it + 1 < P.r) {
+                for (int e = tid; e < 3 * TOK; e += kSolveThreads)
+                    s_coef[((it + 1) & 1) * 3 * TOK + e] = w_next * s_cq[e];
+            }
             fence_proxy_async_smem();
             tc::fence_before_sync();
             ok = __syncthreads_and(ok);
@@ -661,9 +700,11 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         }
     }
 
-    // teardown: no MMA or copy of this CTA may be in flight when TMEM is freed
+    // teardown: no MMA, copy or TMEM store of this CTA may be in flight when TMEM is freed
+    tc::tmem_wait_st();
     ok = __syncthreads_and(ok);
     if (!ok) {
+        if (tid == kZ3Issuer) tc::commit(bar_fin);   // bar_fin counts two arrivals
         if (tid == 0) {
             atomicExch(timeout_flag, 1);
             tc::commit(bar_fin);
