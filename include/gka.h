@@ -189,6 +189,7 @@ enum {
     GKA_KERNEL_CHUNK_SOLVE = 3,   /* Chebyshev solve + readout */
     GKA_KERNEL_DECODE_STEP = 4,   /* recurrent decode step */
     GKA_KERNEL_CHUNK_SOLVE_TC = 5,/* Chebyshev solve + readout on tensor cores (tcgen05) */
+    GKA_KERNEL_STATE_PASS_TC = 6, /* chunk-state increments and scan in one pass (tcgen05) */
     GKA_KERNEL_COUNT = 8
 };
 

@@ -18,6 +18,7 @@
 #include "decode.cuh"
 #include "delta_tc.cuh"
 #include "solve_tc.cuh"
+#include "state_tc.cuh"
 
 namespace gka {
 
@@ -91,6 +92,11 @@ static bool supported_c(int C) { return C == 16 || C == 32 || C == 64 || C == 12
 
 // bf16 inputs, head dimension 128 and chunks of 64 or 128 tokens run the
 // tensor-core solve; everything else the CUDA-core one.
+// On the tensor-core path, the chunk states come from one sequential pass per
+// (head, matrix) when there are at least this many heads (B*H) to spread over
+// the SMs; with fewer, from the chunk-parallel increments plus an element-wise
+// scan, which keeps every SM busy.
+constexpr int kStatePassMinHeads = 16;
 static bool tensor_core_path(int D, int C, gka_dtype dt) {
     return dt == GKA_BF16 && D == 128 && (C == 64 || C == 128);
 }
@@ -263,26 +269,46 @@ static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
     if (int rc = rows128_map(&dmaps.out, states, (uint64_t)BH * (N + 1) * 2 * D,
                              CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 32, 128))
         return rc;
-    if (C == 64) {
-        if ((e = set_smem(k_chunk_delta_tc<64>, DeltaSmem<64>::bytes)) != cudaSuccess)
-            return cuda_fail(e);
-        ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
-        k_chunk_delta_tc<64><<<dim3(N, BH), kTcThreads, DeltaSmem<64>::bytes, s>>>(
-            dmaps, beta, states, decay, bound_inc, tokdec, plane, T, N, flag);
+    if (BH >= kStatePassMinHeads) {
+        StateMaps smaps;
+        smaps.k = maps.k;
+        smaps.v = maps.v;
+        if (C == 64) {
+            if ((e = set_smem(k_state_pass_tc<64>, StateSmem<64>::bytes)) != cudaSuccess)
+                return cuda_fail(e);
+            ProfScope ps(GKA_KERNEL_STATE_PASS_TC, s);
+            k_state_pass_tc<64><<<dim3(2, BH), kStateThreads, StateSmem<64>::bytes, s>>>(
+                smaps, beta, slp, sexp, decay, tokdec, plane, final_state, T, N, flag);
+        } else {
+            if ((e = set_smem(k_state_pass_tc<128>, StateSmem<128>::bytes)) != cudaSuccess)
+                return cuda_fail(e);
+            ProfScope ps(GKA_KERNEL_STATE_PASS_TC, s);
+            k_state_pass_tc<128><<<dim3(2, BH), kStateThreads, StateSmem<128>::bytes, s>>>(
+                smaps, beta, slp, sexp, decay, tokdec, plane, final_state, T, N, flag);
+        }
+        if (int rc = check_launch()) return rc;
     } else {
-        if ((e = set_smem(k_chunk_delta_tc<128>, DeltaSmem<128>::bytes)) != cudaSuccess)
-            return cuda_fail(e);
-        ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
-        k_chunk_delta_tc<128><<<dim3(N, BH), kTcThreads, DeltaSmem<128>::bytes, s>>>(
-            dmaps, beta, states, decay, bound_inc, tokdec, plane, T, N, flag);
-    }
-    if (int rc = check_launch()) return rc;
+        if (C == 64) {
+            if ((e = set_smem(k_chunk_delta_tc<64>, DeltaSmem<64>::bytes)) != cudaSuccess)
+                return cuda_fail(e);
+            ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
+            k_chunk_delta_tc<64><<<dim3(N, BH), kTcThreads, DeltaSmem<64>::bytes, s>>>(
+                dmaps, beta, states, decay, bound_inc, tokdec, plane, T, N, flag);
+        } else {
+            if ((e = set_smem(k_chunk_delta_tc<128>, DeltaSmem<128>::bytes)) != cudaSuccess)
+                return cuda_fail(e);
+            ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
+            k_chunk_delta_tc<128><<<dim3(N, BH), kTcThreads, DeltaSmem<128>::bytes, s>>>(
+                dmaps, beta, states, decay, bound_inc, tokdec, plane, T, N, flag);
+        }
+        if (int rc = check_launch()) return rc;
 
-    const int DD2 = 2 * D * D;
-    { ProfScope ps(GKA_KERNEL_STATE_SCAN, s);
-    k_state_scan<<<dim3((DD2 + 1023) / 1024, BH), 256, 0, s>>>(states, decay, final_state, slp,
-                                                             bound_inc, sexp, N, DD2, false); }
-    if (int rc = check_launch()) return rc;
+        const int DD2 = 2 * D * D;
+        { ProfScope ps(GKA_KERNEL_STATE_SCAN, s);
+        k_state_scan<<<dim3((DD2 + 1023) / 1024, BH), 256, 0, s>>>(states, decay, final_state, slp,
+                                                                 bound_inc, sexp, N, DD2, false); }
+        if (int rc = check_launch()) return rc;
+    }
 
     if (C == 64) {
         // one CTA per 64-token chunk

@@ -29,7 +29,7 @@ class GkaError(RuntimeError):
 
 
 KERNEL_NAMES = ["chunk_delta", "state_scan", "chunk_norm", "chunk_solve", "decode_step",
-                "chunk_solve_tc"]
+                "chunk_solve_tc", "state_pass_tc"]
 
 
 class KernelTimes(ctypes.Structure):
