@@ -4,26 +4,31 @@
 // Method: "Gated KalmaNet" (arXiv 2511.21016), ai.info page, Methodology:
 // only the chunk-start states are carried across chunks,
 //   S_0 = 0,   S_{n+1} = b_n S_n + dS_n,
-//   dH_n = K^T diag(w) K,   dM_n = V^T diag(w) K,   w_i = exp(l_{C-1} - l_i),
-// with l the chunk-relative cumulative log of beta and b_n = exp(l_{C-1}).
+//   dH_n = K^T diag(w) K,   dM_n = V^T diag(w) K,   w_i = prod_{m > i} beta_m,
+// with b_n = prod_m beta_m over chunk n (the exp of the chunk's summed log decay).
 //
 // One CTA per (head, matrix): blockIdx.x = 0 carries H, 1 carries M.  The
-// fp32 state lives in registers for the whole sequence (thread (h, d) owns
-// row d, columns 64h..64h+63), so no state ever goes through memory in fp32.
+// fp32 state lives in registers for the whole sequence (arithmetic thread
+// (h, d) owns row d, columns 64h..64h+63), so no state goes through memory in
+// fp32.  Warps 0-7 do the arithmetic; warp 8 only issues the TMA loads and the
+// MMAs, so that waiting on the tensor core stalls no arithmetic warp.
 // Per chunk:
 //   - K (and V) arrive by TMA, bf16, two chunks ahead; beta with them;
-//   - every warp forms the chunk's log-decay prefix (fp32 logs summed in
-//     double) in registers; the H CTA writes the per-token decays the solve
-//     reads and the chunk decay;
+//   - every arithmetic warp forms w (suffix products of beta) for itself; warp
+//     0 of the H CTA also writes the per-token decays the solve reads (from
+//     fp32 logs summed in double) and the chunk decay;
 //   - the weighted keys w_i k_i are split into bf16 parts (three for 64-token
 //     chunks, about fp32; two for 128-token chunks, 16 mantissa bits) in the
 //     swizzled layout of the key tile; dS = A^T (wK) with A = K or V as loaded
 //     (bf16 is exact) accumulates the parts on tcgen05 into one of two TMEM
-//     buffers, while the threads write the fp16 copy of S_n and fold in
-//     dS_{n-1} from the other buffer;
-//   - the fp16 copy is scaled by 2^e_n with e_n from the running bound
-//     ||S_n||_F <= bound_n, bound_{n+1} = b_n bound_n + sum_i w_i |k_i|^2 (H)
-//     or sum_i w_i |v_i| |k_i| (M), so that every copied value is <= 2^14.
+//     buffers, while the arithmetic warps write the fp16 copy of S_n and fold
+//     in dS_{n-1} from the other buffer;
+//   - the fp16 copy is scaled by 2^e_n with e_n from a running bound
+//     ||S_n||_F <= bound_n, bound_{n+1} = b_n bound_n + inc_n, with
+//     inc_n = sum_i w_i |k_i|^2 >= ||dH_n||_F for H and
+//     inc_n = sum_i w_i (|v_i|^2 + |k_i|^2) / 2 >= sum_i w_i |v_i| |k_i| >= ||dM_n||_F
+//     for M (both linear in the elements, so no per-row reduction), which keeps
+//     every copied value <= 2^14.
 // The state after the last chunk goes to final_state (nullable).
 #pragma once
 
@@ -36,7 +41,9 @@
 
 namespace gka {
 
-constexpr int kStateThreads = 256;
+constexpr int kStateEpiThreads = 256;                    // arithmetic warps 0-7
+constexpr int kStateThreads = kStateEpiThreads + 32;     // + the issuing warp 8
+constexpr int kStateIssuer = kStateEpiThreads;           // its lane 0
 constexpr uint32_t kStateWaitProbes = 1u << 22;
 
 // Exponent e such that |value| <= bound implies |value * 2^e| <= 2^14.
@@ -55,7 +62,7 @@ struct StateSmem {
     static constexpr uint32_t PARTS = VS + 2 * TILE;        // NP tiles of (w k) parts
     static constexpr uint32_t BETA = PARTS + NP * TILE;     // 2 stages of beta [C] floats
     static constexpr uint32_t WW = BETA + 2 * 4 * C;        // per-warp w [8][C] floats
-    static constexpr uint32_t RED = WW + 8 * 4 * C;         // per-warp partial bound increments
+    static constexpr uint32_t RED = WW + 8 * 4 * C;         // [2][8] partial bound increments
     static constexpr uint32_t BARS = RED + 64;              // load[2], mma[2], fin
     static constexpr uint32_t TBASE = BARS + 8 * 8;
     static constexpr uint32_t END = TBASE + 16;
@@ -66,16 +73,19 @@ struct StateMaps {
     CUtensorMap k, v;    // [B*H*T][128] bf16, box 64 x 64, 128B swizzle
 };
 
-// Pairs of consecutive values as packed bf16x2 / fp16x2 words (low half first).
-__device__ __forceinline__ uint32_t pack_bf16(__nv_bfloat16 lo, __nv_bfloat16 hi) {
-    return (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+// A pair of floats as packed bf16x2 (first value in the low half), and back.
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+    const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&p);
 }
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
     const __half2 p = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<const uint32_t *>(&p);
 }
 
-// grid (2, B*H), block 256.  T = N * C.
+// grid (2, B*H), block kStateThreads.  T = N * C.
 template <int C>
 __global__ void __launch_bounds__(kStateThreads, 1)
 k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict__ beta,
@@ -93,23 +103,24 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
     uint64_t *bar_load = bars, *bar_mma = bars + 2, *bar_fin = bars + 4;
     uint32_t *tbase = reinterpret_cast<uint32_t *>(sm + L::TBASE);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quarter = warp & 3, half = warp >> 2;
+    const bool arith = warp < 8;
+    const int quarter = warp & 3, half = (warp >> 2) & 1;
     const int d = quarter * 32 + lane;          // state row of this thread = its TMEM lane
     const int m = blockIdx.x, bh = blockIdx.y;  // m = 0: H, 1: M
     const bool is_m = m == 1;
     const size_t tokbase = (size_t)bh * T;
-    float *s_beta = reinterpret_cast<float *>(sm + L::BETA);       // [2][C]
-    float *s_ww = reinterpret_cast<float *>(sm + L::WW) + warp * C;  // this warp's w [C]
-    float *s_red = reinterpret_cast<float *>(sm + L::RED);         // [2][8]
+    float *s_beta = reinterpret_cast<float *>(sm + L::BETA);              // [2][C]
+    float *s_ww = reinterpret_cast<float *>(sm + L::WW) + (warp & 7) * C;  // this warp's w
+    float *s_red = reinterpret_cast<float *>(sm + L::RED);                // [2][8]
 
-    if (tid == 0) {
+    if (tid == kStateIssuer) {
         for (int i = 0; i < 5; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
     }
     __syncthreads();
 
-    int last_load[2] = {-1, -1};   // thread 0: chunk last loaded into each stage
-    // thread 0: chunk c (keys, values for M, beta) into stage c & 1
+    int last_load[2] = {-1, -1};   // issuer: chunk last loaded into each stage
+    // issuer: chunk c (keys, values for M, beta) into stage c & 1
     auto issue_load = [&](int c) {
         const int st = c & 1;
         uint64_t *bar = &bar_load[st];
@@ -124,7 +135,20 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
         bulk_g2s(s_beta + st * C, beta + tokbase + (size_t)c * C, 4 * C, bar);
         last_load[st] = c;
     };
-    if (tid == 0) {
+    // issuer: dS_c = A^T (w K) into TMEM buffer c & 1 (A = K or V of stage c & 1)
+    auto issue_mma = [&](uint32_t tmem, int c) {
+        constexpr uint32_t ID = tc::idesc_bf16(128, 128, true, true);
+        const uint32_t a = sb + (is_m ? L::VS : L::KS) + (c & 1) * TILE;
+#pragma unroll
+        for (int p = 0; p < NP; ++p)
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)
+                tc::mma_f16(tmem + (c & 1) * 128, tc::sdesc(a + kk * 2048, C * 128, 1024),
+                            tc::sdesc(sb + L::PARTS + p * TILE + kk * 2048, C * 128, 1024), ID,
+                            (p | kk) != 0);
+        tc::commit(&bar_mma[c & 1]);
+    };
+    if (tid == kStateIssuer) {
         issue_load(0);
         if (N > 1) issue_load(1);
     }
@@ -138,134 +162,131 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
     const uint32_t tmem = *tbase;
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(half * 64);
 
-    // Log-decay prefix of chunk c, by every warp for itself: w_t into s_ww, the
-    // chunk decay into bn.  The H CTA's warp 0 also writes the per-token decays
-    // (l_t log2 e, exp(l_t), beta_t, beta_t^2) and the chunk decay.
+    // Decays of chunk c, by every arithmetic warp for itself: w_t = prod_{m>t}
+    // beta_m into s_ww (suffix products: lane l holds tokens l*PER..), the chunk
+    // decay into bn.  Warp 0 of the H CTA also writes the per-token decays
+    // (l_t log2 e, exp(l_t), beta_t, beta_t^2; l from fp32 logs summed in double)
+    // and the chunk decay.
     auto prefix = [&](int c, float &bn) {
         const float *bt = s_beta + (c & 1) * C;
-        double x[PER];
-        double run = 0.0;
+        float bv[PER], sfx[PER];
+        float run = 1.f;
 #pragma unroll
-        for (int p = 0; p < PER; ++p) {
-            run += fmax((double)logf(bt[lane * PER + p]), kLogBetaMin);
-            x[p] = run;
+        for (int p = 0; p < PER; ++p) bv[p] = bt[lane * PER + p];
+#pragma unroll
+        for (int p = PER - 1; p >= 0; --p) {
+            sfx[p] = run;          // product over this lane's tokens after p
+            run *= bv[p];
         }
-        double tot = run;
+        float tot = run;           // -> product over the tokens of lanes >= this lane
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const double y = __shfl_up_sync(0xffffffffu, tot, o);
-            if (lane >= o) tot += y;
+            const float y = __shfl_down_sync(0xffffffffu, tot, o);
+            if (lane + o < 32) tot *= y;
         }
-        const double excl = tot - run;
+        float above = __shfl_down_sync(0xffffffffu, tot, 1);   // lanes > this lane
+        if (lane == 31) above = 1.f;
 #pragma unroll
-        for (int p = 0; p < PER; ++p) x[p] += excl;   // l of token lane*PER + p
-        const double lend = __shfl_sync(0xffffffffu, tot, 31);
-#pragma unroll
-        for (int p = 0; p < PER; ++p) s_ww[lane * PER + p] = decay_exp(lend - x[p]);
-        bn = decay_exp(lend);
+        for (int p = 0; p < PER; ++p) s_ww[lane * PER + p] = sfx[p] * above;
+        bn = __shfl_sync(0xffffffffu, tot, 0);
         if (!is_m && warp == 0) {
-            double prev = __shfl_up_sync(0xffffffffu, x[PER - 1], 1);
+            double x[PER];
+            double acc = 0.0;
+#pragma unroll
+            for (int p = 0; p < PER; ++p) {
+                acc += fmax((double)logf(bv[p]), kLogBetaMin);
+                x[p] = acc;
+            }
+            double t2 = acc;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const double y = __shfl_up_sync(0xffffffffu, t2, o);
+                if (lane >= o) t2 += y;
+            }
+            const double excl = t2 - acc;
+            double prev = __shfl_up_sync(0xffffffffu, t2, 1);
             if (lane == 0) prev = 0.0;
 #pragma unroll
             for (int p = 0; p < PER; ++p) {
+                const double l = x[p] + excl;
                 const size_t g = tokbase + (size_t)c * C + lane * PER + p;
-                const float b1 = decay_exp(x[p] - (p == 0 ? prev : x[p - 1]));
-                tokdec[g] = (float)(x[p] * 1.4426950408889634);
-                tokdec[plane + g] = decay_exp(x[p]);
+                const float b1 = decay_exp(l - prev);
+                tokdec[g] = (float)(l * 1.4426950408889634);
+                tokdec[plane + g] = decay_exp(l);
                 tokdec[2 * plane + g] = b1;
                 tokdec[3 * plane + g] = b1 * b1;
+                prev = l;
             }
             if (lane == 0) decay[(size_t)bh * N + c] = bn;
         }
         __syncwarp();
     };
 
-    // B operand of chunk c: the parts of w_i k_i (bf16, the key tile's swizzled
-    // layout: the 16-byte chunk at a byte offset holds the same elements in
+    // B operand of chunk c: the bf16 parts of w_i k_i, in the swizzled layout of
+    // the key tile (the 16-byte chunk at a byte offset holds the same elements in
     // every tile), and this CTA's bound increment into s_red[c & 1][warp].
-    // 16 consecutive threads take the 16 chunks of one key row.
     auto prep = [&](int c) {
         const uint8_t *kt = sm + L::KS + (c & 1) * TILE;
         const uint8_t *vt = sm + L::VS + (c & 1) * TILE;
         float acc = 0.f;
-#pragma unroll 1
-        for (int item = tid; item < C * 16; item += kStateThreads) {
+#pragma unroll
+        for (int j = 0; j < C / 16; ++j) {
+            const int item = tid + j * kStateEpiThreads;   // C rows x 16 chunks of 16 bytes
             const int r = item >> 4, l16 = item & 15;
             const uint32_t off = (uint32_t)((l16 >> 3) * (C * 128) + r * 128 + (l16 & 7) * 16);
             const uint4 u = *reinterpret_cast<const uint4 *>(kt + off);
-            const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&u);
+            const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
             const float w = s_ww[r];
-            float kk = 0.f;
-            __nv_bfloat16 h0[8], h1[8], h2[8];
+            float sq = 0.f;
+            uint32_t p0[4], p1[4], p2[4];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float x = __bfloat162float(e[i]);
-                kk = fmaf(x, x, kk);
-                const float y = w * x;
-                h0[i] = __float2bfloat16_rn(y);
-                const float r1 = y - __bfloat162float(h0[i]);
-                h1[i] = __float2bfloat16_rn(r1);
-                if (NP == 3) h2[i] = __float2bfloat16_rn(r1 - __bfloat162float(h1[i]));
+            for (int q = 0; q < 4; ++q) {
+                const float x0 = bf16_lo(uw[q]), x1 = bf16_hi(uw[q]);
+                sq = fmaf(x0, x0, fmaf(x1, x1, sq));
+                const float y0 = w * x0, y1 = w * x1;
+                p0[q] = bf16x2_bits(y0, y1);
+                const float r0 = y0 - bf16_lo(p0[q]), r1 = y1 - bf16_hi(p0[q]);
+                p1[q] = bf16x2_bits(r0, r1);
+                if (NP == 3) p2[q] = bf16x2_bits(r0 - bf16_lo(p1[q]), r1 - bf16_hi(p1[q]));
             }
-            uint4 p0, p1;
-            p0.x = pack_bf16(h0[0], h0[1]); p0.y = pack_bf16(h0[2], h0[3]);
-            p0.z = pack_bf16(h0[4], h0[5]); p0.w = pack_bf16(h0[6], h0[7]);
-            p1.x = pack_bf16(h1[0], h1[1]); p1.y = pack_bf16(h1[2], h1[3]);
-            p1.z = pack_bf16(h1[4], h1[5]); p1.w = pack_bf16(h1[6], h1[7]);
-            *reinterpret_cast<uint4 *>(sm + L::PARTS + off) = p0;
-            *reinterpret_cast<uint4 *>(sm + L::PARTS + TILE + off) = p1;
-            if (NP == 3) {
-                uint4 p2;
-                p2.x = pack_bf16(h2[0], h2[1]); p2.y = pack_bf16(h2[2], h2[3]);
-                p2.z = pack_bf16(h2[4], h2[5]); p2.w = pack_bf16(h2[6], h2[7]);
-                *reinterpret_cast<uint4 *>(sm + L::PARTS + 2 * TILE + off) = p2;
-            }
-            float vv = 0.f;
+            *reinterpret_cast<uint4 *>(sm + L::PARTS + off) = make_uint4(p0[0], p0[1], p0[2], p0[3]);
+            *reinterpret_cast<uint4 *>(sm + L::PARTS + TILE + off) =
+                make_uint4(p1[0], p1[1], p1[2], p1[3]);
+            if (NP == 3)
+                *reinterpret_cast<uint4 *>(sm + L::PARTS + 2 * TILE + off) =
+                    make_uint4(p2[0], p2[1], p2[2], p2[3]);
             if (is_m) {
                 const uint4 uv = *reinterpret_cast<const uint4 *>(vt + off);
-                const __nv_bfloat16 *ev = reinterpret_cast<const __nv_bfloat16 *>(&uv);
+                const uint32_t vw[4] = {uv.x, uv.y, uv.z, uv.w};
+                float sv = 0.f;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float x = __bfloat162float(ev[i]);
-                    vv = fmaf(x, x, vv);
+                for (int q = 0; q < 4; ++q) {
+                    const float x0 = bf16_lo(vw[q]), x1 = bf16_hi(vw[q]);
+                    sv = fmaf(x0, x0, fmaf(x1, x1, sv));
                 }
+                acc = fmaf(0.5f * w, sq + sv, acc);
+            } else {
+                acc = fmaf(w, sq, acc);
             }
-#pragma unroll
-            for (int o = 1; o < 16; o <<= 1) {
-                kk += __shfl_xor_sync(0xffffffffu, kk, o);
-                vv += __shfl_xor_sync(0xffffffffu, vv, o);
-            }
-            if (l16 == 0) acc += is_m ? w * sqrtf(kk) * sqrtf(vv) : w * kk;
         }
         acc = warp_sum(acc);
         if (lane == 0) s_red[(c & 1) * 8 + warp] = acc;
     };
 
-    // thread 0: dS_c = A^T (w K) into TMEM buffer c & 1 (A = K or V of stage c & 1)
-    auto issue_mma = [&](int c) {
-        constexpr uint32_t ID = tc::idesc_bf16(128, 128, true, true);
-        const uint32_t a = sb + (is_m ? L::VS : L::KS) + (c & 1) * TILE;
-#pragma unroll
-        for (int p = 0; p < NP; ++p)
-#pragma unroll
-            for (int kk = 0; kk < C / 16; ++kk)
-                tc::mma_f16(tmem + (c & 1) * 128, tc::sdesc(a + kk * 2048, C * 128, 1024),
-                            tc::sdesc(sb + L::PARTS + p * TILE + kk * 2048, C * 128, 1024), ID,
-                            (p | kk) != 0);
-        tc::commit(&bar_mma[c & 1]);
-    };
-
     // ---- prologue: chunk 0's operands and product ----
-    bool ok = mbar_wait_bounded(&bar_load[0], 0, kStateWaitProbes);
+    bool ok = true;
     float b_next = 0.f;
-    prefix(0, b_next);
-    prep(0);
-    fence_proxy_async_smem();
+    if (arith) {
+        ok = mbar_wait_bounded(&bar_load[0], 0, kStateWaitProbes);
+        prefix(0, b_next);
+        prep(0);
+        fence_proxy_async_smem();
+    }
     ok = __syncthreads_and(ok);
     float binc_next = 0.f;
 #pragma unroll
     for (int w = 0; w < 8; ++w) binc_next += s_red[w];
-    if (tid == 0 && ok) issue_mma(0);
+    if (tid == kStateIssuer && ok) issue_mma(tmem, 0);
 
     float st[64];
 #pragma unroll
@@ -275,11 +296,28 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
 
 #pragma unroll 1
     for (int n = 0; n < N && ok; ++n) {
+        if (!arith) {
+            // issuer warp: stage n & 1 is free once dS_n is done; chunk n + 1's
+            // product is issued as soon as its operands are ready
+            if (lane == 0) {
+                if (!mbar_wait_bounded(&bar_mma[n & 1], (n >> 1) & 1, kStateWaitProbes)) ok = false;
+                if (n + 2 < N) issue_load(n + 2);
+            }
+            __syncwarp();
+            if (n + 1 < N) {
+                ok = named_barrier_and(2, kStateThreads, ok);
+                if (tid == kStateIssuer && ok) {
+                    tc::fence_after_sync();
+                    issue_mma(tmem, n + 1);
+                }
+                __syncwarp();
+            }
+            continue;
+        }
         const float bn = b_next, bincn = binc_next;   // chunk n's decay and bound increment
-        // dS_n is ready; stage n & 1 and the parts are free again
+        // dS_n is ready; the parts and stage n & 1 are free again
         if (!mbar_wait_bounded(&bar_mma[n & 1], (n >> 1) & 1, kStateWaitProbes)) ok = false;
         tc::fence_after_sync();
-        if (tid == 0 && n + 2 < N) issue_load(n + 2);
         if (n + 1 < N) {
             // chunk n + 1's operands; its product runs during this chunk's update
             if (!mbar_wait_bounded(&bar_load[(n + 1) & 1], ((n + 1) >> 1) & 1, kStateWaitProbes))
@@ -288,12 +326,10 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
             prep(n + 1);
             fence_proxy_async_smem();
             tc::fence_before_sync();
-            ok = __syncthreads_and(ok);
-            tc::fence_after_sync();
+            ok = named_barrier_and(2, kStateThreads, ok);
             binc_next = 0.f;
 #pragma unroll
             for (int w = 0; w < 8; ++w) binc_next += s_red[((n + 1) & 1) * 8 + w];
-            if (tid == 0 && ok) issue_mma(n + 1);
         }
         // fp16 copy of the chunk-start state S_n, scaled by 2^e_n
         const int ex = lp_exponent_tc(bound);
@@ -323,7 +359,7 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
         bound = fmaf(bn, bound, bincn);
     }
 
-    if (ok && final_state) {
+    if (arith && ok && final_state) {
         float *dst = final_state + ((size_t)bh * 2 + m) * DD + (size_t)d * D + half * 64;
 #pragma unroll
         for (int j = 0; j < 16; ++j)
@@ -334,7 +370,7 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
     // teardown: no MMA or copy of this CTA may be in flight when TMEM is freed
     tc::fence_before_sync();
     ok = __syncthreads_and(ok);
-    if (!ok && tid == 0) {
+    if (!ok && tid == kStateIssuer) {
         atomicExch(timeout_flag, 1);
         tc::commit(bar_fin);
         mbar_wait_bounded(bar_fin, 0, kStateWaitProbes);
