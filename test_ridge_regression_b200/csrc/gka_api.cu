@@ -273,18 +273,21 @@ static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
         StateMaps smaps;
         smaps.k = maps.k;
         smaps.v = maps.v;
+        if (int rc = rows128_map(&smaps.out, slp, (uint64_t)BH * N * 2 * D,
+                                 CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 64, 128))
+            return rc;
         if (C == 64) {
             if ((e = set_smem(k_state_pass_tc<64>, StateSmem<64>::bytes)) != cudaSuccess)
                 return cuda_fail(e);
             ProfScope ps(GKA_KERNEL_STATE_PASS_TC, s);
             k_state_pass_tc<64><<<dim3(2, BH), kStateThreads, StateSmem<64>::bytes, s>>>(
-                smaps, beta, slp, sexp, decay, tokdec, plane, final_state, T, N, flag);
+                smaps, beta, sexp, decay, tokdec, plane, final_state, T, N, flag);
         } else {
             if ((e = set_smem(k_state_pass_tc<128>, StateSmem<128>::bytes)) != cudaSuccess)
                 return cuda_fail(e);
             ProfScope ps(GKA_KERNEL_STATE_PASS_TC, s);
             k_state_pass_tc<128><<<dim3(2, BH), kStateThreads, StateSmem<128>::bytes, s>>>(
-                smaps, beta, slp, sexp, decay, tokdec, plane, final_state, T, N, flag);
+                smaps, beta, sexp, decay, tokdec, plane, final_state, T, N, flag);
         }
         if (int rc = check_launch()) return rc;
     } else {

@@ -9,20 +9,22 @@
 //
 // One CTA per (head, matrix): blockIdx.x = 0 carries H, 1 carries M.  The
 // fp32 state lives in registers for the whole sequence (arithmetic thread
-// (h, d) owns row d, columns 64h..64h+63), so no state goes through memory in
-// fp32.  Warps 0-7 do the arithmetic; warp 8 only issues the TMA loads and the
-// MMAs, so that waiting on the tensor core stalls no arithmetic warp.
+// (g, d) owns row d, columns 32g..32g+31), so no state goes through memory in
+// fp32.  Warps 0-15 do the arithmetic; warp 16 issues the TMA loads, the MMAs
+// and the TMA stores and forms each chunk's decays, so that neither waiting on
+// the tensor core nor that bookkeeping stalls an arithmetic warp.
 // Per chunk:
 //   - K (and V) arrive by TMA, bf16, two chunks ahead; beta with them;
-//   - every arithmetic warp forms w (suffix products of beta) for itself; warp
-//     0 of the H CTA also writes the per-token decays the solve reads (from
-//     fp32 logs summed in double) and the chunk decay;
+//   - the issuing warp forms w (suffix products of beta) and b_n, published
+//     through an mbarrier; in the H CTA it also writes the per-token decays the
+//     solve reads (from fp32 logs summed in double) and the chunk decay;
 //   - the weighted keys w_i k_i are split into bf16 parts (three for 64-token
 //     chunks, about fp32; two for 128-token chunks, 16 mantissa bits) in the
 //     swizzled layout of the key tile; dS = A^T (wK) with A = K or V as loaded
 //     (bf16 is exact) accumulates the parts on tcgen05 into one of two TMEM
-//     buffers, while the arithmetic warps write the fp16 copy of S_n and fold
-//     in dS_{n-1} from the other buffer;
+//     buffers, while the arithmetic warps stage the fp16 copy of S_n in shared
+//     memory (written out by one TMA store) and fold in dS_{n-1} from the
+//     other buffer;
 //   - the fp16 copy is scaled by 2^e_n with e_n from a running bound
 //     ||S_n||_F <= bound_n, bound_{n+1} = b_n bound_n + inc_n, with
 //     inc_n = sum_i w_i |k_i|^2 >= ||dH_n||_F for H and
@@ -41,9 +43,8 @@
 
 namespace gka {
 
-constexpr int kStateEpiThreads = 256;                    // arithmetic warps 0-7
-constexpr int kStateThreads = kStateEpiThreads + 32;     // + the issuing warp 8
-constexpr int kStateIssuer = kStateEpiThreads;           // its lane 0
+constexpr int kStateEpiThreads = 512;                    // arithmetic warps 0-15
+constexpr int kStateThreads = kStateEpiThreads + 32;     // + the issuing warp 16
 constexpr uint32_t kStateWaitProbes = 1u << 22;
 
 // Exponent e such that |value| <= bound implies |value * 2^e| <= 2^14.
@@ -60,10 +61,16 @@ struct StateSmem {
     static constexpr uint32_t KS = 0;                       // 2 stages of keys
     static constexpr uint32_t VS = KS + 2 * TILE;           // 2 stages of values (M CTA)
     static constexpr uint32_t PARTS = VS + 2 * TILE;        // NP tiles of (w k) parts
-    static constexpr uint32_t BETA = PARTS + NP * TILE;     // 2 stages of beta [C] floats
-    static constexpr uint32_t WW = BETA + 2 * 4 * C;        // per-warp w [8][C] floats
-    static constexpr uint32_t RED = WW + 8 * 4 * C;         // [2][8] partial bound increments
-    static constexpr uint32_t BARS = RED + 64;              // load[2], mma[2], fin
+    // fp16 staging of one state copy, [2 column halves][128 rows][64], 128B-swizzled:
+    // own space for 64-token chunks; with 128-token chunks the H CTA stages in
+    // its (unused) value stages and the M CTA in the key stage of the chunk it
+    // has just prepared (free until that stage is loaded again)
+    static constexpr uint32_t OUT = C == 64 ? PARTS + NP * TILE : 0;
+    static constexpr uint32_t BETA = C == 64 ? OUT + 32768 : PARTS + NP * TILE;  // [2][C]
+    static constexpr uint32_t W = BETA + 2 * 4 * C;         // [2][C] w of the chunks in flight
+    static constexpr uint32_t BN = W + 2 * 4 * C;           // [2] chunk decays (16 bytes)
+    static constexpr uint32_t RED = BN + 16;                // [2][16] partial bound increments
+    static constexpr uint32_t BARS = RED + 128;             // load[2] mma[2] fin w[2] out
     static constexpr uint32_t TBASE = BARS + 8 * 8;
     static constexpr uint32_t END = TBASE + 16;
     static constexpr size_t bytes = END + 1024;             // + alignment slack
@@ -71,6 +78,7 @@ struct StateSmem {
 
 struct StateMaps {
     CUtensorMap k, v;    // [B*H*T][128] bf16, box 64 x 64, 128B swizzle
+    CUtensorMap out;     // fp16 state copies [B*H*N*2*128][128], box 64 x 128, 128B swizzle
 };
 
 // A pair of floats as packed bf16x2 (first value in the low half), and back.
@@ -89,9 +97,9 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
 template <int C>
 __global__ void __launch_bounds__(kStateThreads, 1)
 k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict__ beta,
-                __half *__restrict__ slp, int *__restrict__ state_exp,
-                float *__restrict__ decay, float *__restrict__ tokdec, size_t plane,
-                float *__restrict__ final_state, int T, int N, int *__restrict__ timeout_flag) {
+                int *__restrict__ state_exp, float *__restrict__ decay,
+                float *__restrict__ tokdec, size_t plane, float *__restrict__ final_state,
+                int T, int N, int *__restrict__ timeout_flag) {
     using L = StateSmem<C>;
     constexpr int D = 128, NP = L::NP, PER = C / 32;
     constexpr uint32_t TILE = L::TILE;
@@ -100,21 +108,30 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
                                               ~static_cast<uintptr_t>(1023));
     const uint32_t sb = smem_u32(sm);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BARS);
-    uint64_t *bar_load = bars, *bar_mma = bars + 2, *bar_fin = bars + 4;
+    uint64_t *bar_load = bars, *bar_mma = bars + 2, *bar_fin = bars + 4, *bar_w = bars + 5,
+             *bar_out = bars + 7;
     uint32_t *tbase = reinterpret_cast<uint32_t *>(sm + L::TBASE);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const bool arith = warp < 8;
-    const int quarter = warp & 3, half = (warp >> 2) & 1;
+    const bool arith = warp < 16;
+    const int quarter = warp & 3, cg = (warp >> 2) & 3;   // lane quarter, 32-column group
     const int d = quarter * 32 + lane;          // state row of this thread = its TMEM lane
     const int m = blockIdx.x, bh = blockIdx.y;  // m = 0: H, 1: M
     const bool is_m = m == 1;
     const size_t tokbase = (size_t)bh * T;
-    float *s_beta = reinterpret_cast<float *>(sm + L::BETA);              // [2][C]
-    float *s_ww = reinterpret_cast<float *>(sm + L::WW) + (warp & 7) * C;  // this warp's w
-    float *s_red = reinterpret_cast<float *>(sm + L::RED);                // [2][8]
+    float *s_beta = reinterpret_cast<float *>(sm + L::BETA);   // [2][C]
+    float *s_w = reinterpret_cast<float *>(sm + L::W);         // [2][C]
+    float *s_bn = reinterpret_cast<float *>(sm + L::BN);       // [2]
+    float *s_red = reinterpret_cast<float *>(sm + L::RED);     // [2][16]
+    // staging of chunk n's fp16 state copy
+    auto out_stage = [&](int n) -> uint32_t {
+        return C == 64 ? L::OUT : (is_m ? L::KS + ((n + 1) & 1) * TILE : L::VS);
+    };
 
-    if (tid == kStateIssuer) {
+    if (tid == kStateEpiThreads) {
         for (int i = 0; i < 5; ++i) mbar_init(&bars[i], 1);
+        mbar_init(&bar_w[0], 32);
+        mbar_init(&bar_w[1], 32);
+        mbar_init(bar_out, kStateEpiThreads);
         fence_mbar_init();
     }
     __syncthreads();
@@ -148,7 +165,7 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
                             (p | kk) != 0);
         tc::commit(&bar_mma[c & 1]);
     };
-    if (tid == kStateIssuer) {
+    if (tid == kStateEpiThreads) {
         issue_load(0);
         if (N > 1) issue_load(1);
     }
@@ -160,14 +177,12 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tbase;
-    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(half * 64);
+    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(cg * 32);
 
-    // Decays of chunk c, by every arithmetic warp for itself: w_t = prod_{m>t}
-    // beta_m into s_ww (suffix products: lane l holds tokens l*PER..), the chunk
-    // decay into bn.  Warp 0 of the H CTA also writes the per-token decays
-    // (l_t log2 e, exp(l_t), beta_t, beta_t^2; l from fp32 logs summed in double)
-    // and the chunk decay.
-    auto prefix = [&](int c, float &bn) {
+    // Issuing warp: chunk c's decays w_t = prod_{m>t} beta_m (suffix products;
+    // lane l holds tokens l*PER..) into s_w[c & 1], b_c into s_bn[c & 1], then
+    // every lane arrives on bar_w[c & 1].
+    auto decays = [&](int c) {
         const float *bt = s_beta + (c & 1) * C;
         float bv[PER], sfx[PER];
         float run = 1.f;
@@ -187,56 +202,66 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
         float above = __shfl_down_sync(0xffffffffu, tot, 1);   // lanes > this lane
         if (lane == 31) above = 1.f;
 #pragma unroll
-        for (int p = 0; p < PER; ++p) s_ww[lane * PER + p] = sfx[p] * above;
-        bn = __shfl_sync(0xffffffffu, tot, 0);
-        if (!is_m && warp == 0) {
-            double x[PER];
-            double acc = 0.0;
+        for (int p = 0; p < PER; ++p) s_w[(c & 1) * C + lane * PER + p] = sfx[p] * above;
+        if (lane == 0) s_bn[c & 1] = tot;
+        __syncwarp();
+        mbar_arrive(&bar_w[c & 1]);
+    };
+
+    // Issuing warp of the H CTA: chunk c's per-token decays for the solve
+    // (l_t log2 e, exp(l_t), beta_t, beta_t^2; l from fp32 logs summed in
+    // double) and the chunk decay.
+    auto token_decays = [&](int c) {
+        const float *bt = s_beta + (c & 1) * C;
+        double x[PER];
+        double acc = 0.0;
 #pragma unroll
-            for (int p = 0; p < PER; ++p) {
-                acc += fmax((double)logf(bv[p]), kLogBetaMin);
-                x[p] = acc;
-            }
-            double t2 = acc;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const double y = __shfl_up_sync(0xffffffffu, t2, o);
-                if (lane >= o) t2 += y;
-            }
-            const double excl = t2 - acc;
-            double prev = __shfl_up_sync(0xffffffffu, t2, 1);
-            if (lane == 0) prev = 0.0;
-#pragma unroll
-            for (int p = 0; p < PER; ++p) {
-                const double l = x[p] + excl;
-                const size_t g = tokbase + (size_t)c * C + lane * PER + p;
-                const float b1 = decay_exp(l - prev);
-                tokdec[g] = (float)(l * 1.4426950408889634);
-                tokdec[plane + g] = decay_exp(l);
-                tokdec[2 * plane + g] = b1;
-                tokdec[3 * plane + g] = b1 * b1;
-                prev = l;
-            }
-            if (lane == 0) decay[(size_t)bh * N + c] = bn;
+        for (int p = 0; p < PER; ++p) {
+            acc += fmax((double)logf(bt[lane * PER + p]), kLogBetaMin);
+            x[p] = acc;
         }
+        double t2 = acc;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const double y = __shfl_up_sync(0xffffffffu, t2, o);
+            if (lane >= o) t2 += y;
+        }
+        const double excl = t2 - acc;
+        double prev = __shfl_up_sync(0xffffffffu, t2, 1);
+        if (lane == 0) prev = 0.0;
+#pragma unroll
+        for (int p = 0; p < PER; ++p) {
+            const double l = x[p] + excl;
+            const size_t g = tokbase + (size_t)c * C + lane * PER + p;
+            const float b1 = decay_exp(l - prev);
+            tokdec[g] = (float)(l * 1.4426950408889634);
+            tokdec[plane + g] = decay_exp(l);
+            tokdec[2 * plane + g] = b1;
+            tokdec[3 * plane + g] = b1 * b1;
+            prev = l;
+        }
+        const double lend = __shfl_sync(0xffffffffu, t2, 31);
+        if (lane == 0) decay[(size_t)bh * N + c] = decay_exp(lend);
         __syncwarp();
     };
 
-    // B operand of chunk c: the bf16 parts of w_i k_i, in the swizzled layout of
-    // the key tile (the 16-byte chunk at a byte offset holds the same elements in
-    // every tile), and this CTA's bound increment into s_red[c & 1][warp].
+    // Arithmetic warps: B operand of chunk c, the bf16 parts of w_i k_i, in the
+    // swizzled layout of the key tile (the 16-byte chunk at a byte offset holds
+    // the same elements in every tile), and this warp's share of the bound
+    // increment into s_red[c & 1][warp].
     auto prep = [&](int c) {
         const uint8_t *kt = sm + L::KS + (c & 1) * TILE;
         const uint8_t *vt = sm + L::VS + (c & 1) * TILE;
+        const float *wc = s_w + (c & 1) * C;
         float acc = 0.f;
 #pragma unroll
-        for (int j = 0; j < C / 16; ++j) {
+        for (int j = 0; j < C * 16 / kStateEpiThreads; ++j) {
             const int item = tid + j * kStateEpiThreads;   // C rows x 16 chunks of 16 bytes
             const int r = item >> 4, l16 = item & 15;
             const uint32_t off = (uint32_t)((l16 >> 3) * (C * 128) + r * 128 + (l16 & 7) * 16);
             const uint4 u = *reinterpret_cast<const uint4 *>(kt + off);
             const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
-            const float w = s_ww[r];
+            const float w = wc[r];
             float sq = 0.f;
             uint32_t p0[4], p1[4], p2[4];
 #pragma unroll
@@ -270,113 +295,143 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
             }
         }
         acc = warp_sum(acc);
-        if (lane == 0) s_red[(c & 1) * 8 + warp] = acc;
+        if (lane == 0) s_red[(c & 1) * 16 + warp] = acc;
+    };
+    auto bound_inc = [&](int c) {
+        float s = 0.f;
+#pragma unroll
+        for (int w = 0; w < 16; ++w) s += s_red[(c & 1) * 16 + w];
+        return s;
     };
 
     // ---- prologue: chunk 0's operands and product ----
     bool ok = true;
-    float b_next = 0.f;
     if (arith) {
-        ok = mbar_wait_bounded(&bar_load[0], 0, kStateWaitProbes);
-        prefix(0, b_next);
+        ok = mbar_wait_bounded(&bar_w[0], 0, kStateWaitProbes);
+        ok = mbar_wait_bounded(&bar_load[0], 0, kStateWaitProbes) && ok;
         prep(0);
         fence_proxy_async_smem();
+    } else {
+        ok = mbar_wait_bounded(&bar_load[0], 0, kStateWaitProbes);
+        decays(0);
+        if (!is_m) token_decays(0);
     }
     ok = __syncthreads_and(ok);
-    float binc_next = 0.f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) binc_next += s_red[w];
-    if (tid == kStateIssuer && ok) issue_mma(tmem, 0);
+    if (tid == kStateEpiThreads && ok) issue_mma(tmem, 0);
 
-    float st[64];
+    float st[32];
 #pragma unroll
-    for (int i = 0; i < 64; ++i) st[i] = 0.f;
+    for (int i = 0; i < 32; ++i) st[i] = 0.f;
     float bound = 0.f;
     const size_t DD = (size_t)D * D;
 
+    // `ok` changes only at barriers, so every thread leaves the loop together;
+    // a wait that gives up sets `fail`, which the next barrier folds into `ok`
+    bool fail = false;
 #pragma unroll 1
     for (int n = 0; n < N && ok; ++n) {
+        const int ph = (n >> 1) & 1, ph1 = ((n + 1) >> 1) & 1;
         if (!arith) {
-            // issuer warp: stage n & 1 is free once dS_n is done; chunk n + 1's
-            // product is issued as soon as its operands are ready
+            // issuing warp: chunk n + 1's decays as soon as it has landed; stage
+            // n & 1 is free once dS_n is done and the previous TMA store has read
+            // its staging; chunk n + 1's product once its operands are ready;
+            // chunk n's fp16 copy once it is staged
+            if (n + 1 < N) {
+                if (!mbar_wait_bounded(&bar_load[(n + 1) & 1], ph1, kStateWaitProbes)) fail = true;
+                decays(n + 1);
+                if (!is_m) token_decays(n + 1);
+            }
             if (lane == 0) {
-                if (!mbar_wait_bounded(&bar_mma[n & 1], (n >> 1) & 1, kStateWaitProbes)) ok = false;
+                if (!mbar_wait_bounded(&bar_mma[n & 1], ph, kStateWaitProbes)) fail = true;
+                tc::bulk_wait_read0();
                 if (n + 2 < N) issue_load(n + 2);
             }
             __syncwarp();
-            if (n + 1 < N) {
-                ok = named_barrier_and(2, kStateThreads, ok);
-                if (tid == kStateIssuer && ok) {
-                    tc::fence_after_sync();
-                    issue_mma(tmem, n + 1);
+            ok = named_barrier_and(2, kStateThreads, ok && !fail);
+            if (!ok) break;
+            if (lane == 0) {
+                tc::fence_after_sync();
+                if (n + 1 < N) issue_mma(tmem, n + 1);
+                if (!mbar_wait_bounded(bar_out, n & 1, kStateWaitProbes)) fail = true;
+                if (!fail) {
+                    const int row = (int)(((size_t)bh * N + n) * 2 + m) * D;
+                    tc::tma_store_2d(&maps.out, 0, row, sm + out_stage(n));
+                    tc::tma_store_2d(&maps.out, 64, row, sm + out_stage(n) + 16384);
+                    tc::bulk_commit();
                 }
-                __syncwarp();
             }
+            __syncwarp();
             continue;
         }
-        const float bn = b_next, bincn = binc_next;   // chunk n's decay and bound increment
+        const float bn = s_bn[n & 1];
+        const float bincn = bound_inc(n);
         // dS_n is ready; the parts and stage n & 1 are free again
-        if (!mbar_wait_bounded(&bar_mma[n & 1], (n >> 1) & 1, kStateWaitProbes)) ok = false;
+        if (!mbar_wait_bounded(&bar_mma[n & 1], ph, kStateWaitProbes)) fail = true;
         tc::fence_after_sync();
         if (n + 1 < N) {
             // chunk n + 1's operands; its product runs during this chunk's update
-            if (!mbar_wait_bounded(&bar_load[(n + 1) & 1], ((n + 1) >> 1) & 1, kStateWaitProbes))
-                ok = false;
-            prefix(n + 1, b_next);
+            if (!mbar_wait_bounded(&bar_w[(n + 1) & 1], ph1, kStateWaitProbes)) fail = true;
+            if (!mbar_wait_bounded(&bar_load[(n + 1) & 1], ph1, kStateWaitProbes)) fail = true;
             prep(n + 1);
             fence_proxy_async_smem();
-            tc::fence_before_sync();
-            ok = named_barrier_and(2, kStateThreads, ok);
-            binc_next = 0.f;
-#pragma unroll
-            for (int w = 0; w < 8; ++w) binc_next += s_red[((n + 1) & 1) * 8 + w];
         }
-        // fp16 copy of the chunk-start state S_n, scaled by 2^e_n
+        tc::fence_before_sync();
+        ok = named_barrier_and(2, kStateThreads, ok && !fail);
+        if (!ok) break;
+        // fp16 copy of the chunk-start state S_n, scaled by 2^e_n, staged in the
+        // TMA box layout: [column half][row][64], 16-byte chunk j of row d at j ^ (d % 8)
         const int ex = lp_exponent_tc(bound);
         {
             const float sc = ldexpf(1.f, ex);
-            __half *dst = slp + (((size_t)bh * N + n) * 2 + m) * DD + (size_t)d * D + half * 64;
+            uint8_t *row = sm + out_stage(n) + (cg >> 1) * 16384 + d * 128;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                uint4 w4;
-                w4.x = pack_h2(st[8 * j] * sc, st[8 * j + 1] * sc);
-                w4.y = pack_h2(st[8 * j + 2] * sc, st[8 * j + 3] * sc);
-                w4.z = pack_h2(st[8 * j + 4] * sc, st[8 * j + 5] * sc);
-                w4.w = pack_h2(st[8 * j + 6] * sc, st[8 * j + 7] * sc);
-                *reinterpret_cast<uint4 *>(dst + 8 * j) = w4;
+            for (int j = 0; j < 4; ++j) {
+                const int chunk = ((cg & 1) * 4 + j) ^ (d & 7);
+                *reinterpret_cast<uint4 *>(row + chunk * 16) = make_uint4(
+                    pack_h2(st[8 * j] * sc, st[8 * j + 1] * sc),
+                    pack_h2(st[8 * j + 2] * sc, st[8 * j + 3] * sc),
+                    pack_h2(st[8 * j + 4] * sc, st[8 * j + 5] * sc),
+                    pack_h2(st[8 * j + 6] * sc, st[8 * j + 7] * sc));
             }
+            fence_proxy_async_smem();
+            mbar_arrive(bar_out);
             if (tid == 0) state_exp[((size_t)bh * N + n) * 2 + m] = ex;
         }
         // S_{n+1} = b_n S_n + dS_n
         {
-            float dl[64];
+            float dl[32];
 #pragma unroll
-            for (int cb = 0; cb < 64; cb += 16) tc::tmem_ld16(tl + (n & 1) * 128 + cb, dl + cb);
+            for (int cb = 0; cb < 32; cb += 16) tc::tmem_ld16(tl + (n & 1) * 128 + cb, dl + cb);
             tc::tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 64; ++i) st[i] = fmaf(bn, st[i], dl[i]);
+            for (int i = 0; i < 32; ++i) st[i] = fmaf(bn, st[i], dl[i]);
         }
         bound = fmaf(bn, bound, bincn);
     }
 
+    ok = ok && !fail;
     if (arith && ok && final_state) {
-        float *dst = final_state + ((size_t)bh * 2 + m) * DD + (size_t)d * D + half * 64;
+        float *dst = final_state + ((size_t)bh * 2 + m) * DD + (size_t)d * D + cg * 32;
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
+        for (int j = 0; j < 8; ++j)
             *reinterpret_cast<float4 *>(dst + 4 * j) =
                 make_float4(st[4 * j], st[4 * j + 1], st[4 * j + 2], st[4 * j + 3]);
     }
 
-    // teardown: no MMA or copy of this CTA may be in flight when TMEM is freed
+    // teardown: no MMA or copy of this CTA may be in flight when TMEM or shared
+    // memory is released
     tc::fence_before_sync();
     ok = __syncthreads_and(ok);
-    if (!ok && tid == kStateIssuer) {
-        atomicExch(timeout_flag, 1);
-        tc::commit(bar_fin);
-        mbar_wait_bounded(bar_fin, 0, kStateWaitProbes);
-        for (int s2 = 0; s2 < 2; ++s2)
-            if (last_load[s2] >= 0)
-                mbar_wait_bounded(&bar_load[s2], (last_load[s2] >> 1) & 1, kStateWaitProbes);
+    if (tid == kStateEpiThreads) {
+        tc::bulk_wait0();
+        if (!ok) {
+            atomicExch(timeout_flag, 1);
+            tc::commit(bar_fin);
+            mbar_wait_bounded(bar_fin, 0, kStateWaitProbes);
+            for (int s2 = 0; s2 < 2; ++s2)
+                if (last_load[s2] >= 0)
+                    mbar_wait_bounded(&bar_load[s2], (last_load[s2] >> 1) & 1, kStateWaitProbes);
+        }
     }
     tc::fence_before_sync();
     __syncthreads();
