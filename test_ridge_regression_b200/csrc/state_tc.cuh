@@ -11,11 +11,12 @@
 // fp32 state lives in registers for the whole sequence (arithmetic thread
 // (g, d) owns row d, columns 32g..32g+31), so no state goes through memory in
 // fp32.  Warps 0-15 do the arithmetic; warp 16 issues the TMA loads, the MMAs
-// and the TMA stores and forms each chunk's decays, so that neither waiting on
-// the tensor core nor that bookkeeping stalls an arithmetic warp.
+// and the TMA stores; warp 17 forms each chunk's decays as soon as the chunk
+// has landed, so that neither waiting on the tensor core nor that bookkeeping
+// stalls an arithmetic warp.
 // Per chunk:
 //   - K (and V) arrive by TMA, bf16, two chunks ahead; beta with them;
-//   - the issuing warp forms w (suffix products of beta) and b_n, published
+//   - the decay warp forms w (suffix products of beta) and b_n, published
 //     through an mbarrier; in the H CTA it also writes the per-token decays the
 //     solve reads (from fp32 logs summed in double) and the chunk decay;
 //   - the weighted keys w_i k_i are split into bf16 parts (three for 64-token
@@ -24,7 +25,8 @@
 //     (bf16 is exact) accumulates the parts on tcgen05 into one of two TMEM
 //     buffers, while the arithmetic warps stage the fp16 copy of S_n in shared
 //     memory (written out by one TMA store) and fold in dS_{n-1} from the
-//     other buffer;
+//     other buffer; with 64-token chunks the parts are double-buffered too, so
+//     the next chunk's parts are formed while the current product runs;
 //   - the fp16 copy is scaled by 2^e_n with e_n from a running bound
 //     ||S_n||_F <= bound_n, bound_{n+1} = b_n bound_n + inc_n, with
 //     inc_n = sum_i w_i |k_i|^2 >= ||dH_n||_F for H and
@@ -44,7 +46,8 @@
 namespace gka {
 
 constexpr int kStateEpiThreads = 512;                    // arithmetic warps 0-15
-constexpr int kStateThreads = kStateEpiThreads + 32;     // + the issuing warp 16
+constexpr int kStateBarThreads = kStateEpiThreads + 32;  // + the issuing warp 16
+constexpr int kStateThreads = kStateBarThreads + 32;     // + the decay warp 17
 constexpr uint32_t kStateWaitProbes = 1u << 22;
 
 // Exponent e such that |value| <= bound implies |value * 2^e| <= 2^14.
@@ -57,16 +60,17 @@ __device__ __forceinline__ int lp_exponent_tc(float bound) {
 template <int C>
 struct StateSmem {
     static constexpr int NP = C == 64 ? 3 : 2;              // bf16 parts of w k
+    static constexpr int NPB = C == 64 ? 2 : 1;             // buffers of parts
     static constexpr uint32_t TILE = C * 256;               // one [C][128] bf16 tile (2 halves)
     static constexpr uint32_t KS = 0;                       // 2 stages of keys
     static constexpr uint32_t VS = KS + 2 * TILE;           // 2 stages of values (M CTA)
-    static constexpr uint32_t PARTS = VS + 2 * TILE;        // NP tiles of (w k) parts
+    static constexpr uint32_t PARTS = VS + 2 * TILE;        // NPB x NP tiles of (w k) parts
     // fp16 staging of one state copy, [2 column halves][128 rows][64], 128B-swizzled:
     // own space for 64-token chunks; with 128-token chunks the H CTA stages in
     // its (unused) value stages and the M CTA in the key stage of the chunk it
     // has just prepared (free until that stage is loaded again)
-    static constexpr uint32_t OUT = C == 64 ? PARTS + NP * TILE : 0;
-    static constexpr uint32_t BETA = C == 64 ? OUT + 32768 : PARTS + NP * TILE;  // [2][C]
+    static constexpr uint32_t OUT = C == 64 ? PARTS + NPB * NP * TILE : 0;
+    static constexpr uint32_t BETA = C == 64 ? OUT + 32768 : PARTS + NPB * NP * TILE;  // [2][C]
     static constexpr uint32_t W = BETA + 2 * 4 * C;         // [2][C] w of the chunks in flight
     static constexpr uint32_t BN = W + 2 * 4 * C;           // [2] chunk decays (16 bytes)
     static constexpr uint32_t RED = BN + 16;                // [2][16] partial bound increments
@@ -122,6 +126,8 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
     float *s_w = reinterpret_cast<float *>(sm + L::W);         // [2][C]
     float *s_bn = reinterpret_cast<float *>(sm + L::BN);       // [2]
     float *s_red = reinterpret_cast<float *>(sm + L::RED);     // [2][16]
+    // parts buffer of chunk c
+    auto parts = [&](int c) -> uint32_t { return L::PARTS + (c & (L::NPB - 1)) * NP * TILE; };
     // staging of chunk n's fp16 state copy
     auto out_stage = [&](int n) -> uint32_t {
         return C == 64 ? L::OUT : (is_m ? L::KS + ((n + 1) & 1) * TILE : L::VS);
@@ -161,7 +167,7 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
 #pragma unroll
             for (int kk = 0; kk < C / 16; ++kk)
                 tc::mma_f16(tmem + (c & 1) * 128, tc::sdesc(a + kk * 2048, C * 128, 1024),
-                            tc::sdesc(sb + L::PARTS + p * TILE + kk * 2048, C * 128, 1024), ID,
+                            tc::sdesc(sb + parts(c) + p * TILE + kk * 2048, C * 128, 1024), ID,
                             (p | kk) != 0);
         tc::commit(&bar_mma[c & 1]);
     };
@@ -179,7 +185,7 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
     const uint32_t tmem = *tbase;
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(cg * 32);
 
-    // Issuing warp: chunk c's decays w_t = prod_{m>t} beta_m (suffix products;
+    // Decay warp: chunk c's decays w_t = prod_{m>t} beta_m (suffix products;
     // lane l holds tokens l*PER..) into s_w[c & 1], b_c into s_bn[c & 1], then
     // every lane arrives on bar_w[c & 1].
     auto decays = [&](int c) {
@@ -208,7 +214,7 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
         mbar_arrive(&bar_w[c & 1]);
     };
 
-    // Issuing warp of the H CTA: chunk c's per-token decays for the solve
+    // Decay warp of the H CTA: chunk c's per-token decays for the solve
     // (l_t log2 e, exp(l_t), beta_t, beta_t^2; l from fp32 logs summed in
     // double) and the chunk decay.
     auto token_decays = [&](int c) {
@@ -274,11 +280,11 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
                 p1[q] = bf16x2_bits(r0, r1);
                 if (NP == 3) p2[q] = bf16x2_bits(r0 - bf16_lo(p1[q]), r1 - bf16_hi(p1[q]));
             }
-            *reinterpret_cast<uint4 *>(sm + L::PARTS + off) = make_uint4(p0[0], p0[1], p0[2], p0[3]);
-            *reinterpret_cast<uint4 *>(sm + L::PARTS + TILE + off) =
-                make_uint4(p1[0], p1[1], p1[2], p1[3]);
+            uint8_t *pb = sm + parts(c);
+            *reinterpret_cast<uint4 *>(pb + off) = make_uint4(p0[0], p0[1], p0[2], p0[3]);
+            *reinterpret_cast<uint4 *>(pb + TILE + off) = make_uint4(p1[0], p1[1], p1[2], p1[3]);
             if (NP == 3)
-                *reinterpret_cast<uint4 *>(sm + L::PARTS + 2 * TILE + off) =
+                *reinterpret_cast<uint4 *>(pb + 2 * TILE + off) =
                     make_uint4(p2[0], p2[1], p2[2], p2[3]);
             if (is_m) {
                 const uint4 uv = *reinterpret_cast<const uint4 *>(vt + off);
@@ -305,13 +311,17 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
     };
 
     // ---- prologue: chunk 0's operands and product ----
+    const bool issuer_warp = warp == 16, decay_warp = warp == 17;
+    constexpr bool kDblParts = L::NPB == 2;
     bool ok = true;
+    float b_next = 1.f;   // arithmetic warps: decay of the next chunk to fold in
     if (arith) {
         ok = mbar_wait_bounded(&bar_w[0], 0, kStateWaitProbes);
         ok = mbar_wait_bounded(&bar_load[0], 0, kStateWaitProbes) && ok;
+        b_next = s_bn[0];
         prep(0);
         fence_proxy_async_smem();
-    } else {
+    } else if (decay_warp) {
         ok = mbar_wait_bounded(&bar_load[0], 0, kStateWaitProbes);
         decays(0);
         if (!is_m) token_decays(0);
@@ -325,29 +335,36 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
     float bound = 0.f;
     const size_t DD = (size_t)D * D;
 
-    // `ok` changes only at barriers, so every thread leaves the loop together;
-    // a wait that gives up sets `fail`, which the next barrier folds into `ok`
+    // Decay warp: chunk c's decays as soon as it has landed.  Stage c & 1 is
+    // reloaded only after the product of chunk c - 2 is done, which comes after
+    // every read of the w and b_n buffers this overwrites.
+    if (decay_warp) {
+#pragma unroll 1
+        for (int c = 1; c < N && ok; ++c) {
+            if (!mbar_wait_bounded(&bar_load[c & 1], (c >> 1) & 1, kStateWaitProbes)) ok = false;
+            decays(c);
+            if (!is_m) token_decays(c);
+        }
+    }
+
+    // Arithmetic and issuing warps.  `ok` changes only at barriers, so they
+    // leave the loop together; a wait that gives up sets `fail`, which the next
+    // barrier folds into `ok`.
     bool fail = false;
 #pragma unroll 1
-    for (int n = 0; n < N && ok; ++n) {
+    for (int n = 0; n < N && ok && !decay_warp; ++n) {
         const int ph = (n >> 1) & 1, ph1 = ((n + 1) >> 1) & 1;
-        if (!arith) {
-            // issuing warp: chunk n + 1's decays as soon as it has landed; stage
-            // n & 1 is free once dS_n is done and the previous TMA store has read
-            // its staging; chunk n + 1's product once its operands are ready;
+        if (issuer_warp) {
+            // stage n & 1 is free once dS_n is done and the previous TMA store has
+            // read its staging; chunk n + 1's product once its operands are ready;
             // chunk n's fp16 copy once it is staged
-            if (n + 1 < N) {
-                if (!mbar_wait_bounded(&bar_load[(n + 1) & 1], ph1, kStateWaitProbes)) fail = true;
-                decays(n + 1);
-                if (!is_m) token_decays(n + 1);
-            }
             if (lane == 0) {
                 if (!mbar_wait_bounded(&bar_mma[n & 1], ph, kStateWaitProbes)) fail = true;
                 tc::bulk_wait_read0();
                 if (n + 2 < N) issue_load(n + 2);
             }
             __syncwarp();
-            ok = named_barrier_and(2, kStateThreads, ok && !fail);
+            ok = named_barrier_and(2, kStateBarThreads, ok && !fail);
             if (!ok) break;
             if (lane == 0) {
                 tc::fence_after_sync();
@@ -363,20 +380,27 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
             __syncwarp();
             continue;
         }
-        const float bn = s_bn[n & 1];
-        const float bincn = bound_inc(n);
-        // dS_n is ready; the parts and stage n & 1 are free again
-        if (!mbar_wait_bounded(&bar_mma[n & 1], ph, kStateWaitProbes)) fail = true;
-        tc::fence_after_sync();
+        const float bn = b_next, bincn = bound_inc(n);   // chunk n's decay and bound increment
         if (n + 1 < N) {
-            // chunk n + 1's operands; its product runs during this chunk's update
+            // chunk n + 1's operands (with double-buffered parts, formed while
+            // chunk n's product still runs)
             if (!mbar_wait_bounded(&bar_w[(n + 1) & 1], ph1, kStateWaitProbes)) fail = true;
             if (!mbar_wait_bounded(&bar_load[(n + 1) & 1], ph1, kStateWaitProbes)) fail = true;
+            b_next = s_bn[(n + 1) & 1];
+            if (kDblParts) {
+                prep(n + 1);
+                fence_proxy_async_smem();
+            }
+        }
+        // dS_n is ready (and, with single-buffered parts, the parts are free)
+        if (!mbar_wait_bounded(&bar_mma[n & 1], ph, kStateWaitProbes)) fail = true;
+        tc::fence_after_sync();
+        if (!kDblParts && n + 1 < N) {
             prep(n + 1);
             fence_proxy_async_smem();
         }
         tc::fence_before_sync();
-        ok = named_barrier_and(2, kStateThreads, ok && !fail);
+        ok = named_barrier_and(2, kStateBarThreads, ok && !fail);
         if (!ok) break;
         // fp16 copy of the chunk-start state S_n, scaled by 2^e_n, staged in the
         // TMA box layout: [column half][row][64], 16-byte chunk j of row d at j ^ (d % 8)
