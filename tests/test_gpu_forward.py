@@ -67,6 +67,7 @@ def check_against_oracle(q, k, v, beta, a, r, C, *, check_ws=True):
     print(f"o rel err {err:.3e} (bar {tol:g})")
     assert err <= tol
     ferr = head_rel_err(fs, ref["final_state"])
+    print(f"final state rel err {ferr:.3e} (bar 1e-05)")
     assert ferr <= 1e-5, ferr
     if check_ws:
         # intermediate results: fp32 on the CUDA-core path; on the tensor-core path
