@@ -96,7 +96,7 @@ static bool supported_c(int C) { return C == 16 || C == 32 || C == 64 || C == 12
 // (head, matrix) when there are at least this many heads (B*H) to spread over
 // the SMs; with fewer, from the chunk-parallel increments plus an element-wise
 // scan, which keeps every SM busy.
-constexpr int kStatePassMinHeads = 16;
+constexpr int kStatePassMinHeads = 24;
 static bool tensor_core_path(int D, int C, gka_dtype dt) {
     return dt == GKA_BF16 && D == 128 && (C == 64 || C == 128);
 }

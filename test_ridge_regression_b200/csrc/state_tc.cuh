@@ -59,7 +59,7 @@ __device__ __forceinline__ int lp_exponent_tc(float bound) {
 
 template <int C>
 struct StateSmem {
-    static constexpr int NP = 2;                            // bf16 parts of w k
+    static constexpr int NP = 2;                            // bf16 parts of w k (hi, lo)
     static constexpr int NPB = C == 64 ? 2 : 1;             // buffers of parts
     static constexpr uint32_t TILE = C * 256;               // one [C][128] bf16 tile (2 halves)
     static constexpr uint32_t KS = 0;                       // 2 stages of keys
@@ -269,7 +269,7 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
             const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
             const float w = wc[r];
             float sq = 0.f;
-            uint32_t p0[4], p1[4], p2[4];
+            uint32_t p0[4], p1[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const float x0 = bf16_lo(uw[q]), x1 = bf16_hi(uw[q]);
@@ -278,14 +278,10 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
                 p0[q] = bf16x2_bits(y0, y1);
                 const float r0 = y0 - bf16_lo(p0[q]), r1 = y1 - bf16_hi(p0[q]);
                 p1[q] = bf16x2_bits(r0, r1);
-                if (NP == 3) p2[q] = bf16x2_bits(r0 - bf16_lo(p1[q]), r1 - bf16_hi(p1[q]));
             }
             uint8_t *pb = sm + parts(c);
             *reinterpret_cast<uint4 *>(pb + off) = make_uint4(p0[0], p0[1], p0[2], p0[3]);
             *reinterpret_cast<uint4 *>(pb + TILE + off) = make_uint4(p1[0], p1[1], p1[2], p1[3]);
-            if (NP == 3)
-                *reinterpret_cast<uint4 *>(pb + 2 * TILE + off) =
-                    make_uint4(p2[0], p2[1], p2[2], p2[3]);
             if (is_m) {
                 const uint4 uv = *reinterpret_cast<const uint4 *>(vt + off);
                 const uint32_t vw[4] = {uv.x, uv.y, uv.z, uv.w};
