@@ -38,15 +38,17 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # bench reports null.  Captures and commands: profiles/*.md.
 TRAFFIC = {
     # full-size forward workload (B8 H8 T2048 D128, chunk 64), one launch
-    "chunk_solve_tc": {"bytes": 235.544576e6 + 24.613376e6, "workload": "bf16_b8h8t2048d128",
+    "chunk_solve_tc": {"bytes": 237.137408e6 + 23.863296e6, "workload": "bf16_b8h8t2048d128",
                        "src": "test_ridge_regression_b200/csrc/solve_tc.cuh",
-                       "sha1": "fb4d6c766862ea733917bb5603f7f55c701a76e6"},
+                       "sha1": "a3018159b4407640d7472ad4d3710aceb9045606"},
+    "state_pass_tc": {"bytes": 67.718912e6 + 80.975616e6, "workload": "bf16_b8h8t2048d128",
+                      "src": "test_ridge_regression_b200/csrc/state_tc.cuh",
+                      "sha1": "6b699f228b0797f72e56fce9c3607b1f777213e9"},
     # decode captured on 64 x 32 heads (state above L2), scaled x4 to 256 x 32 heads
     "decode_step": {"bytes": 4 * (270.054912e6 + 213.513472e6), "workload": "decode_bf16_b256h32d128",
                     "src": "test_ridge_regression_b200/csrc/decode.cuh",
                     "sha1": "9fed00ad526c1e277840c391aca09dea977665ff"},
 }
-
 
 def traffic_of(kernel, workload):
     import hashlib
@@ -342,7 +344,7 @@ def main():
     dom_name, (dom_ms, dom_n) = dom
     per_step_ms = dom_ms / args.steps
     alg = {"chunk_solve": ch + out, "chunk_solve_tc": ch + out, "chunk_norm": nrm,
-           "chunk_delta": upd}.get(dom_name, 0)
+           "chunk_delta": upd, "state_pass_tc": upd}.get(dom_name, 0)
     kernel_flops = alg * head_tok            # per step
     sm_mhz_max = peaks.get("sm_max_mhz", 1965.0)
     if dom_name == "chunk_solve_tc":
