@@ -59,8 +59,7 @@ k_chunk_delta_tc(const __grid_constant__ DeltaMaps maps, const float *__restrict
     using L = DeltaSmem<C>;
     constexpr int D = kTcD;
     extern __shared__ uint8_t smraw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
-                                              ~static_cast<uintptr_t>(1023));
+    uint8_t *sm = smem_align1024(smraw);
     const uint32_t sb = smem_u32(sm);
     double *ell = reinterpret_cast<double *>(sm + L::ELL);
     double *wtot = ell + C;

@@ -9,6 +9,13 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The first 1024-byte boundary at or after p (dynamic shared memory), derived by
+// pointer arithmetic on p so that the compiler still knows it is shared memory
+// (accesses through it stay shared loads and stores, not generic ones).
+__device__ __forceinline__ uint8_t *smem_align1024(uint8_t *p) {
+    return p + ((1024u - (smem_u32(p) & 1023u)) & 1023u);
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
                  : "memory");

@@ -204,8 +204,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     constexpr int NCH = TPT / 16;      // 16-token chunks per thread
     constexpr uint32_t TMEM_COLS = 4 * TOK;
     extern __shared__ uint8_t smraw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
-                                              ~static_cast<uintptr_t>(1023));
+    uint8_t *sm = smem_align1024(smraw);
     const uint32_t sb = smem_u32(sm);
     float *s_cq = reinterpret_cast<float *>(sm + L::SCAL);   // coefficient of q (scaled domain)
     float *s_c1 = s_cq + TOK;                                // coefficient of Z1

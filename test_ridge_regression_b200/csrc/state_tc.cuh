@@ -108,8 +108,7 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
     constexpr int D = 128, NP = L::NP, PER = C / 32;
     constexpr uint32_t TILE = L::TILE;
     extern __shared__ uint8_t smraw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
-                                              ~static_cast<uintptr_t>(1023));
+    uint8_t *sm = smem_align1024(smraw);
     const uint32_t sb = smem_u32(sm);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BARS);
     uint64_t *bar_load = bars, *bar_mma = bars + 2, *bar_fin = bars + 4, *bar_w = bars + 5,
