@@ -125,6 +125,20 @@ __device__ __forceinline__ void load_qrow16(uint32_t tile, uint32_t row, int c, 
     }
 }
 
+// Tokens 8c..8c+7 of row `row` of the 128B-swizzled bf16 q^T tile, as fp32.
+__device__ __forceinline__ void load_qrow8(uint32_t tile, uint32_t row, int c, float *v) {
+    uint32_t a, b, cc, dd;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(a), "=r"(b), "=r"(cc), "=r"(dd)
+                 : "r"(tile + row * 128u + (((uint32_t)c ^ row) & 7u) * 16u));
+    const uint32_t w4[4] = {a, b, cc, dd};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(w4[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w4[i] & 0xffff0000u);
+    }
+}
+
 // In place: bf16 tile of `bytes` bytes -> fp16, scaled so that every |value| < 1.
 // Returns the scale.  Every thread of the block calls it (red: blockDim/32 floats).
 __device__ __forceinline__ float tile_bf16_to_f16_scaled(uint8_t *tile, int bytes, float *red) {
@@ -155,6 +169,13 @@ __device__ __forceinline__ float tile_bf16_to_f16_scaled(uint8_t *tile, int byte
         *reinterpret_cast<uint4 *>(tile + c) = w;
     }
     return sc;
+}
+
+// Writes 8 consecutive values (columns c0..c0+7, c0 % 8 == 0) of `row` of a
+// 128B-swizzled [rows][64] fp16 tile as one 16-byte chunk.
+__device__ __forceinline__ void st_row8(uint32_t tile, uint32_t row, uint32_t c0, const float *v) {
+    st_shared_v4(tile + row * 128u + (((c0 >> 3) ^ row) & 7u) * 16u, pack_f16(v[0], v[1]),
+                 pack_f16(v[2], v[3]), pack_f16(v[4], v[5]), pack_f16(v[6], v[7]));
 }
 
 // Writes 16 consecutive values (columns c0..c0+15, c0 % 16 == 0) of `row` of a
@@ -641,18 +662,19 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
             const float *kq = s_coef + (it & 1) * 3 * TOK, *k1 = kq + TOK, *k3 = k1 + TOK;
             // the previous round's x_prev stores (not waited for at its end) land first
             tc::tmem_wait_st();
+            // 8 tokens at a time (few live temporaries next to the 32 iterates)
 #pragma unroll
-            for (int c = 0; c < NCH; ++c) {
-                const int t0 = tcol + c * 16;
-                float z1[16], z3[16], xp[16], qv[16];
-                tc::tmem_ld16(tl + T_Z1 + t0, z1);
-                tc::tmem_ld16(tl + T_Z3 + t0, z3);
-                tc::tmem_ld16(tl + T_XP + t0, xp);
-                load_qrow16(sb + L::QS + (t0 >> 6) * 16384u, d, (t0 & 63) >> 4, qv);
+            for (int c = 0; c < TPT / 8; ++c) {
+                const int t0 = tcol + c * 8;
+                float z1[8], z3[8], xp[8], qv[8];
+                tc::tmem_ld8(tl + T_Z1 + t0, z1);
+                tc::tmem_ld8(tl + T_Z3 + t0, z3);
+                tc::tmem_ld8(tl + T_XP + t0, xp);
+                load_qrow8(sb + L::QS + (t0 >> 6) * 16384u, d, (t0 & 63) >> 3, qv);
                 tc::tmem_wait_ld();
-                float xn[16];
+                float xn[8];
 #pragma unroll
-                for (int u4 = 0; u4 < 16; u4 += 4) {
+                for (int u4 = 0; u4 < 8; u4 += 4) {
                     const float4 gq = *reinterpret_cast<const float4 *>(kq + t0 + u4);
                     const float4 g1 = *reinterpret_cast<const float4 *>(k1 + t0 + u4);
                     const float4 g3 = *reinterpret_cast<const float4 *>(k3 + t0 + u4);
@@ -663,13 +685,13 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
                     for (int v = 0; v < 4; ++v) {
                         const int u = u4 + v;
                         const float t = fmaf(gqv[v], qv[u], -fmaf(g1v[v], z1[u], g3v[v] * z3[u]));
-                        xn[u] = fmaf(cA, xp[u], fmaf(cB, xc[c * 16 + u], t));
+                        xn[u] = fmaf(cA, xp[u], fmaf(cB, xc[c * 8 + u], t));
                     }
                 }
-                tc::tmem_st16(tl + T_XP + t0, &xc[c * 16]);
+                tc::tmem_st8(tl + T_XP + t0, &xc[c * 8]);
 #pragma unroll
-                for (int u = 0; u < 16; ++u) xc[c * 16 + u] = xn[u];
-                st_row16(sb + L::XT + (t0 >> 6) * 16384u, d, t0 & 63, xn);
+                for (int u = 0; u < 8; ++u) xc[c * 8 + u] = xn[u];
+                st_row8(sb + L::XT + (t0 >> 6) * 16384u, d, t0 & 63, xn);
             }
             // the next round's coefficient table (the other buffer)
             if (it + 1 < P.r) {
