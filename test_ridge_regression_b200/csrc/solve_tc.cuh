@@ -641,10 +641,16 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
             }
             if (warp == kZ3Issuer / 32) __syncwarp();
         }
+        // x_new = (1 - w) x_prev + w (1 - lambda/d) x + w cq q - w c1 Z1 - w c3 Z3 (the
+        // three-term update with the residual (q - A x)/d written out; the per-token
+        // products w cq, w c1, w c3 of this round come from the table), in two parts:
+        // A, as soon as Z1 = H_s X^T is done (while the P phase and the intra-chunk
+        // product run): part = (1 - w) x_prev + w (1 - lambda/d) x + w cq q - w c1 Z1,
+        // kept in the x_prev columns of TMEM; B, once Z3 is done: x_new = part - w c3 Z3.
+        const float cA = 1.f - P.omega[it], cB = P.omega[it] * (1.f - cl);
+        const float *kq = s_coef + (it & 1) * 3 * TOK, *k1 = kq + TOK, *k3 = k1 + TOK;
         if (!mbar_wait_bounded(bar_z1, ph, kTcWaitProbes)) ok = false;
-        if (!mbar_wait_bounded(bar_z, ph, kTcWaitProbes)) ok = false;
         tc::fence_after_sync();
-        ph ^= 1u;
         if (!out_pass) {
             if (tid == 0 && it == P.r - 1) {
                 // H_s is no longer read: fetch M_s for the readout into the same buffer
@@ -655,40 +661,54 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
                                         srow + kTcD + rb * 64, bar_m);
                 m_requested = true;
             }
-            // x_new = (1 - w) x_prev + w (1 - lambda/d) x + w cq q - w c1 Z1 - w c3 Z3
-            // (the three-term update with the residual (q - A x)/d written out); the
-            // per-token products w cq, w c1, w c3 of this round come from the table
-            const float cA = 1.f - P.omega[it], cB = P.omega[it] * (1.f - cl);
-            const float *kq = s_coef + (it & 1) * 3 * TOK, *k1 = kq + TOK, *k3 = k1 + TOK;
             // the previous round's x_prev stores (not waited for at its end) land first
             tc::tmem_wait_st();
-            // 8 tokens at a time (few live temporaries next to the 32 iterates)
 #pragma unroll
-            for (int c = 0; c < TPT / 8; ++c) {
+            for (int c = 0; c < TPT / 8; ++c) {   // 8 tokens at a time
                 const int t0 = tcol + c * 8;
-                float z1[8], z3[8], xp[8], qv[8];
+                float z1[8], xp[8], qv[8];
                 tc::tmem_ld8(tl + T_Z1 + t0, z1);
-                tc::tmem_ld8(tl + T_Z3 + t0, z3);
                 tc::tmem_ld8(tl + T_XP + t0, xp);
                 load_qrow8(sb + L::QS + (t0 >> 6) * 16384u, d, (t0 & 63) >> 3, qv);
                 tc::tmem_wait_ld();
-                float xn[8];
+                float part[8];
 #pragma unroll
                 for (int u4 = 0; u4 < 8; u4 += 4) {
                     const float4 gq = *reinterpret_cast<const float4 *>(kq + t0 + u4);
                     const float4 g1 = *reinterpret_cast<const float4 *>(k1 + t0 + u4);
-                    const float4 g3 = *reinterpret_cast<const float4 *>(k3 + t0 + u4);
                     const float gqv[4] = {gq.x, gq.y, gq.z, gq.w};
                     const float g1v[4] = {g1.x, g1.y, g1.z, g1.w};
-                    const float g3v[4] = {g3.x, g3.y, g3.z, g3.w};
 #pragma unroll
                     for (int v = 0; v < 4; ++v) {
                         const int u = u4 + v;
-                        const float t = fmaf(gqv[v], qv[u], -fmaf(g1v[v], z1[u], g3v[v] * z3[u]));
-                        xn[u] = fmaf(cA, xp[u], fmaf(cB, xc[c * 8 + u], t));
+                        part[u] = fmaf(cA, xp[u],
+                                       fmaf(cB, xc[c * 8 + u], fmaf(gqv[v], qv[u], -g1v[v] * z1[u])));
                     }
                 }
-                tc::tmem_st8(tl + T_XP + t0, &xc[c * 8]);
+                tc::tmem_st8(tl + T_XP + t0, part);
+            }
+        }
+        if (!mbar_wait_bounded(bar_z, ph, kTcWaitProbes)) ok = false;
+        tc::fence_after_sync();
+        ph ^= 1u;
+        if (!out_pass) {
+            tc::tmem_wait_st();   // this thread's parts are in TMEM
+#pragma unroll
+            for (int c = 0; c < TPT / 8; ++c) {
+                const int t0 = tcol + c * 8;
+                float z3[8], part[8];
+                tc::tmem_ld8(tl + T_Z3 + t0, z3);
+                tc::tmem_ld8(tl + T_XP + t0, part);
+                tc::tmem_wait_ld();
+                float xn[8];
+#pragma unroll
+                for (int u4 = 0; u4 < 8; u4 += 4) {
+                    const float4 g3 = *reinterpret_cast<const float4 *>(k3 + t0 + u4);
+                    const float g3v[4] = {g3.x, g3.y, g3.z, g3.w};
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) xn[u4 + v] = fmaf(-g3v[v], z3[u4 + v], part[u4 + v]);
+                }
+                tc::tmem_st8(tl + T_XP + t0, &xc[c * 8]);   // x_prev of the next round
 #pragma unroll
                 for (int u = 0; u < 8; ++u) xc[c * 8 + u] = xn[u];
                 st_row8(sb + L::XT + (t0 >> 6) * 16384u, d, t0 & 63, xn);
