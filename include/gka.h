@@ -113,6 +113,36 @@ int gka_forward(const void *q, const void *k, const void *v, const float *beta, 
                 float *final_state, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * gka_forward from HOST buffers, with the copies overlapped with the compute
+ * (no counterpart in the paper: a transfer pipeline around the forward).
+ * The B*H independent sequences, flattened to pairs p = b*H + h, are cut into
+ * slices of `slice` pairs (the last may be shorter); slice i's inputs are
+ * copied in on one internal stream while slice i-1 is computed on `stream`
+ * and slice i-2's output is copied out on another, through two device slots.
+ *
+ *   q, k, v, beta, o, final_state   HOST pointers, layouts as for gka_forward
+ *               (final_state nullable).  Page-locked (pinned) memory is needed
+ *               for the copies to overlap; pageable memory works but serialises.
+ *   slice       pairs per slice; 0 picks one (about a quarter of B*H, at
+ *               least 24 pairs; the first slice's copy in and the last one's
+ *               compute and copy out are not overlapped)
+ *   workspace   device scratch of at least gka_forward_host_workspace_bytes()
+ *               bytes, 256-byte aligned: two slots of device inputs and outputs
+ *               plus one gka_forward workspace of a slice
+ * Asynchronous with respect to the host: o and final_state are complete when
+ * `stream` has completed the work enqueued before the call returns.  Work
+ * already on `stream` finishes before any slot is reused.  Calls from several
+ * host threads are serialised while they enqueue; calls that overlap on the
+ * GPU must not share a workspace.
+ */
+size_t gka_forward_host_workspace_bytes(int B, int H, int T, int D, int chunk, gka_dtype dt,
+                                        int slice);
+int gka_forward_host(const void *q, const void *k, const void *v, const float *beta, void *o,
+                     int B, int H, int T, int D, gka_dtype dt, float a, int r, int chunk,
+                     float *final_state, int slice, void *workspace, size_t workspace_bytes,
+                     void *stream);
+
+/*
  * gka_forward without a caller-provided workspace.  There is no counterpart
  * of this call in the paper: it exists for callers that cannot allocate
  * device memory themselves, for example a plugin or extension run inside a

@@ -61,6 +61,11 @@ def _lib():
         lib.gka_forward.restype = i
         lib.gka_forward_static_scratch.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i,
                                                    vp, vp]
+        lib.gka_forward_host_workspace_bytes.argtypes = [i, i, i, i, i, i, i]
+        lib.gka_forward_host_workspace_bytes.restype = sz
+        lib.gka_forward_host.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, i, vp,
+                                         sz, vp]
+        lib.gka_forward_host.restype = i
         lib.gka_forward_static_scratch.restype = i
         lib.gka_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
         lib.gka_decode_step.restype = i
@@ -152,6 +157,46 @@ def gka_forward(q, k, v, beta, a: float, r: int, chunk: int, *, o=None, final_st
                             float(a), int(r), int(chunk), _ptr(final_state), _ptr(workspace),
                             workspace.numel() * workspace.element_size(), _stream(stream))
     _check("gka_forward", rc)
+    return o
+
+
+def host_workspace_bytes(B, H, T, D, chunk, dtype=torch.bfloat16, slice_pairs=0) -> int:
+    return int(_lib().gka_forward_host_workspace_bytes(B, H, T, D, chunk, _DT[dtype], slice_pairs))
+
+
+def alloc_host_workspace(B, H, T, D, chunk, dtype=torch.bfloat16, slice_pairs=0,
+                         device=None) -> torch.Tensor:
+    n = host_workspace_bytes(B, H, T, D, chunk, dtype, slice_pairs)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def gka_forward_host(q, k, v, beta, a: float, r: int, chunk: int, *, o=None, final_state=None,
+                     slice_pairs=0, workspace=None, stream=None):
+    """gka_forward from HOST tensors with the copies overlapped with the compute
+    (see include/gka.h).  q, k, v: [B, H, T, D] fp32 or bf16 CPU tensors (pinned
+    for overlap), beta: [B, H, T] fp32.  Returns o on the host; it is complete
+    once `stream` (default: the current CUDA stream) has completed."""
+    for t in (q, k, v, beta, o, final_state):
+        if t is not None and (t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous host tensors")
+    B, H, T, D = q.shape
+    if k.shape != q.shape or v.shape != q.shape or beta.shape != (B, H, T):
+        raise ValueError("shape mismatch")
+    dt = _dtype(q)
+    if k.dtype != q.dtype or v.dtype != q.dtype or beta.dtype != torch.float32:
+        raise TypeError("q, k, v must share a dtype; beta must be float32")
+    if o is None:
+        o = torch.empty(q.shape, dtype=q.dtype, pin_memory=q.is_pinned())
+    if final_state is not None and (final_state.dtype != torch.float32 or
+                                    final_state.shape != (B, H, 2, D, D)):
+        raise ValueError("final_state must be float32 [B, H, 2, D, D]")
+    if workspace is None:
+        workspace = alloc_host_workspace(B, H, T, D, chunk, q.dtype, slice_pairs)
+    rc = _lib().gka_forward_host(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(o), B, H, T, D, dt,
+                                 float(a), int(r), int(chunk), _ptr(final_state), int(slice_pairs),
+                                 _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                 _stream(stream))
+    _check("gka_forward_host", rc)
     return o
 
 

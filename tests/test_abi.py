@@ -107,3 +107,22 @@ def test_binding_raises_without_cuda_tensors():
     x = torch.zeros(1, 1, 64, 32)
     with pytest.raises(ValueError):
         gka.gka_forward(x, x, x, torch.ones(1, 1, 64), 0.5, 4, 64)
+
+
+def test_host_forward_plan_and_argument_errors(lib):
+    vp = ctypes.c_void_p
+    B, H, T, D, C, BF16 = 2, 8, 128, 128, 64, 1
+    n_auto = lib.gka_forward_host_workspace_bytes(B, H, T, D, C, BF16, 0)
+    n4 = lib.gka_forward_host_workspace_bytes(B, H, T, D, C, BF16, 4)
+    assert n_auto > 0 and 0 < n4 < n_auto
+    assert lib.gka_forward_host_workspace_bytes(B, H, T, D, C, BF16, -1) == 0
+    assert lib.gka_forward_host_workspace_bytes(B, H, 100, D, C, BF16, 0) == 0   # T % C
+    fake = vp(1 << 20)
+    args = (fake, fake, fake, fake, fake, B, H, T, D, BF16, ctypes.c_float(0.5), 8, C)
+    # no workspace, too small a workspace, misaligned workspace, bad a, bad slice
+    assert lib.gka_forward_host(*args, None, 0, None, 0, None) == -1
+    assert lib.gka_forward_host(*args, None, 0, fake, 256, None) == -4
+    assert lib.gka_forward_host(*args, None, 0, vp((1 << 20) + 16), n_auto, None) == -7
+    bad_a = args[:10] + (ctypes.c_float(0.0),) + args[11:]
+    assert lib.gka_forward_host(*bad_a, None, 0, fake, n_auto, None) == -1
+    assert lib.gka_forward_host(*args, None, -3, fake, n_auto, None) == -1
