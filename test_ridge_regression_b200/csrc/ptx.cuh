@@ -83,6 +83,31 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
     return false;
 }
 
+// One probe of phase `parity` that may suspend the calling thread for up to
+// `hint_ns` nanoseconds; it resumes as soon as the phase completes, so a waiting
+// warp takes no issue slots from the warps that still work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait with suspending probes: gives up after `max_probes` probes
+// (at most about max_probes * hint_ns nanoseconds) and returns false.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity,
+                                                uint32_t max_probes, uint32_t hint_ns) {
+    for (uint32_t i = 0; i < max_probes; ++i)
+        if (mbar_try_wait_sleep(bar, parity, hint_ns)) return true;
+    return false;
+}
+
 // Bulk (non-tensor) async copy global -> shared, completing on `bar`.
 // dst, src 16-byte aligned; bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes,

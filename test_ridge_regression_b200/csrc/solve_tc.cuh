@@ -46,6 +46,10 @@ constexpr int kTcThreads = 128;
 constexpr int kSolveThreads = 256;   // solve kernel: two warpgroups
 constexpr int kTcD = 128;         // head dimension of the tensor-core path
 constexpr uint32_t kTcWaitProbes = 1u << 22;
+// waits inside the solve suspend for up to kTcSleepNs per probe (a waiting warp
+// then takes no issue slots); kTcSleepProbes probes bound a wait at about a second
+constexpr uint32_t kTcSleepNs = 1000;
+constexpr uint32_t kTcSleepProbes = 1u << 20;
 
 template <int MG, int TOK>
 struct TcSmem {
@@ -88,6 +92,14 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                  : "memory");
 }
 
+__device__ __forceinline__ uint4 ld_shared_u4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr));
+    return v;
+}
+
 __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
     const __half2 p = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<const uint32_t *>(&p);
@@ -122,20 +134,6 @@ __device__ __forceinline__ void load_qrow16(uint32_t tile, uint32_t row, int c, 
             v[8 * h + 2 * i] = __uint_as_float(w4[i] << 16);
             v[8 * h + 2 * i + 1] = __uint_as_float(w4[i] & 0xffff0000u);
         }
-    }
-}
-
-// Tokens 8c..8c+7 of row `row` of the 128B-swizzled bf16 q^T tile, as fp32.
-__device__ __forceinline__ void load_qrow8(uint32_t tile, uint32_t row, int c, float *v) {
-    uint32_t a, b, cc, dd;
-    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(a), "=r"(b), "=r"(cc), "=r"(dd)
-                 : "r"(tile + row * 128u + (((uint32_t)c ^ row) & 7u) * 16u));
-    const uint32_t w4[4] = {a, b, cc, dd};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        v[2 * i] = __uint_as_float(w4[i] << 16);
-        v[2 * i + 1] = __uint_as_float(w4[i] & 0xffff0000u);
     }
 }
 
@@ -239,7 +237,9 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
              *bar_z = &bars[4], *bar_fin = &bars[5], *bar_n = &bars[6], *bar_z1 = &bars[7];
     uint32_t *tbase = reinterpret_cast<uint32_t *>(sm + L::TBASE);
 
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // the warp index read through a shuffle is known to be warp-uniform, so TMEM
+    // addresses and warp-role branches derived from it stay in uniform registers
+    const int tid = threadIdx.x, warp = __shfl_sync(0xffffffffu, tid >> 5, 0), lane = tid & 31;
     const int wg = warp >> 2, quarter = warp & 3;
     const int d = quarter * 32 + lane;        // head-dimension row = TMEM lane of this thread
     const int tcol = wg * TPT;                // first token (TMEM column) of this thread
@@ -282,8 +282,8 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     // products of beta: w_{t,i-1} = w_ti beta_i and w_{t+1,i} = w_ti beta_{t+1}.
     float *s_l2 = reinterpret_cast<float *>(sm + L::DEC);
     float *s_bt = s_l2 + MG, *s_bet = s_bt + MG, *s_beta2 = s_bet + MG;
-    bool ok = mbar_wait_bounded(bar_load, 0, kTcWaitProbes);
-    ok = mbar_wait_bounded(bar_v, 0, kTcWaitProbes) && ok;
+    bool ok = mbar_wait_sleep(bar_load, 0, kTcSleepProbes, kTcSleepNs);
+    ok = mbar_wait_sleep(bar_v, 0, kTcSleepProbes, kTcSleepNs) && ok;
     // keys and values: bf16 -> fp16 in place, scaled below 1
     const float sK = tile_bf16_to_f16_scaled(sm + L::KT, MG * 256, red);
     const float sV = tile_bf16_to_f16_scaled(sm + L::VT, MG * 256, red);
@@ -352,7 +352,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         hs = warp_sum(hs);
         if (lane == 0) red[8 + warp] = hs;
     }
-    if (!mbar_wait_bounded(bar_n, 0, kTcWaitProbes)) ok = false;
+    if (!mbar_wait_sleep(bar_n, 0, kTcSleepProbes, kTcSleepNs)) ok = false;
     tc::fence_after_sync();
     {
         // u_i: thread (wg, d) forms k_i[d] (H_s k_i)[d] for its half of the keys,
@@ -542,8 +542,9 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         }
         tc::tmem_wait_st();
     }
-    if (P.r > 1) {   // round 1's coefficient table (s_cq, s_c1, s_c3 are consecutive)
-        for (int e = tid; e < 3 * TOK; e += kSolveThreads) s_coef[3 * TOK + e] = P.omega[1] * s_cq[e];
+    if (P.r > 1) {   // round 1's table omega (cq, -c1, -c3) (s_cq, s_c1, s_c3 are consecutive)
+        for (int e = tid; e < 3 * TOK; e += kSolveThreads)
+            s_coef[3 * TOK + e] = (e < TOK ? P.omega[1] : -P.omega[1]) * s_cq[e];
     }
     fence_proxy_async_smem();
     tc::fence_before_sync();
@@ -608,7 +609,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         if (in_pbar) {
             if (p_warp) {
                 // P^T = W o S^T -> fp16, MN-major tile of MG rows
-                if (!mbar_wait_bounded(bar_s, ph, kTcWaitProbes)) ok = false;
+                if (!mbar_wait_sleep(bar_s, ph, kTcSleepProbes, kTcSleepNs)) ok = false;
                 tc::fence_after_sync();
                 const bool both = !kSOffset && warp == 4;
 #pragma unroll 1
@@ -622,7 +623,12 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
                         tc::tmem_ld16(tl + T_W + t0, wv);
                         tc::tmem_wait_ld();
 #pragma unroll
-                        for (int u = 0; u < 16; ++u) sv[u] *= wv[u];
+                        for (int u = 0; u < 16; u += 2) {
+                            const float2 p2 = __fmul2_rn(make_float2(sv[u], sv[u + 1]),
+                                                         make_float2(wv[u], wv[u + 1]));
+                            sv[u] = p2.x;
+                            sv[u + 1] = p2.y;
+                        }
                         st_row16(b_pt + (t0 >> 6) * PT_BLOCK, key, t0 & 63, sv);
                     }
                 }
@@ -643,13 +649,15 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         }
         // x_new = (1 - w) x_prev + w (1 - lambda/d) x + w cq q - w c1 Z1 - w c3 Z3 (the
         // three-term update with the residual (q - A x)/d written out; the per-token
-        // products w cq, w c1, w c3 of this round come from the table), in two parts:
+        // products w cq, -w c1, -w c3 of this round come from the table), in two parts:
         // A, as soon as Z1 = H_s X^T is done (while the P phase and the intra-chunk
         // product run): part = (1 - w) x_prev + w (1 - lambda/d) x + w cq q - w c1 Z1,
         // kept in the x_prev columns of TMEM; B, once Z3 is done: x_new = part - w c3 Z3.
-        const float cA = 1.f - P.omega[it], cB = P.omega[it] * (1.f - cl);
+        // Pairs of tokens go through the packed f32x2 FMA pipe.
+        const float cAs = 1.f - P.omega[it], cBs = P.omega[it] * (1.f - cl);
+        const float2 cA = make_float2(cAs, cAs), cB = make_float2(cBs, cBs);
         const float *kq = s_coef + (it & 1) * 3 * TOK, *k1 = kq + TOK, *k3 = k1 + TOK;
-        if (!mbar_wait_bounded(bar_z1, ph, kTcWaitProbes)) ok = false;
+        if (!mbar_wait_sleep(bar_z1, ph, kTcSleepProbes, kTcSleepNs)) ok = false;
         tc::fence_after_sync();
         if (!out_pass) {
             if (tid == 0 && it == P.r - 1) {
@@ -666,29 +674,38 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
 #pragma unroll
             for (int c = 0; c < TPT / 8; ++c) {   // 8 tokens at a time
                 const int t0 = tcol + c * 8;
-                float z1[8], xp[8], qv[8];
+                float z1[8], xp[8];
                 tc::tmem_ld8(tl + T_Z1 + t0, z1);
                 tc::tmem_ld8(tl + T_XP + t0, xp);
-                load_qrow8(sb + L::QS + (t0 >> 6) * 16384u, d, (t0 & 63) >> 3, qv);
+                const uint4 qw4 = ld_shared_u4(sb + L::QS + (t0 >> 6) * 16384u + d * 128u +
+                                               ((((uint32_t)(t0 & 63) >> 3) ^ d) & 7u) * 16u);
+                const float4 gq[2] = {*reinterpret_cast<const float4 *>(kq + t0),
+                                      *reinterpret_cast<const float4 *>(kq + t0 + 4)};
+                const float4 g1[2] = {*reinterpret_cast<const float4 *>(k1 + t0),
+                                      *reinterpret_cast<const float4 *>(k1 + t0 + 4)};
                 tc::tmem_wait_ld();
+                const uint32_t qw[4] = {qw4.x, qw4.y, qw4.z, qw4.w};
                 float part[8];
 #pragma unroll
-                for (int u4 = 0; u4 < 8; u4 += 4) {
-                    const float4 gq = *reinterpret_cast<const float4 *>(kq + t0 + u4);
-                    const float4 g1 = *reinterpret_cast<const float4 *>(k1 + t0 + u4);
-                    const float gqv[4] = {gq.x, gq.y, gq.z, gq.w};
-                    const float g1v[4] = {g1.x, g1.y, g1.z, g1.w};
-#pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        const int u = u4 + v;
-                        part[u] = fmaf(cA, xp[u],
-                                       fmaf(cB, xc[c * 8 + u], fmaf(gqv[v], qv[u], -g1v[v] * z1[u])));
-                    }
+                for (int p = 0; p < 4; ++p) {   // tokens 2p, 2p + 1
+                    const float2 gqp = (p & 1) ? make_float2(gq[p >> 1].z, gq[p >> 1].w)
+                                               : make_float2(gq[p >> 1].x, gq[p >> 1].y);
+                    const float2 g1p = (p & 1) ? make_float2(g1[p >> 1].z, g1[p >> 1].w)
+                                               : make_float2(g1[p >> 1].x, g1[p >> 1].y);
+                    // q^T holds bf16 pairs: the low half is token 2p, the high half 2p + 1
+                    const float2 qv = make_float2(__uint_as_float(qw[p] << 16),
+                                                  __uint_as_float(qw[p] & 0xffff0000u));
+                    float2 t = __fmul2_rn(g1p, make_float2(z1[2 * p], z1[2 * p + 1]));
+                    t = __ffma2_rn(gqp, qv, t);
+                    t = __ffma2_rn(cB, make_float2(xc[c * 8 + 2 * p], xc[c * 8 + 2 * p + 1]), t);
+                    t = __ffma2_rn(cA, make_float2(xp[2 * p], xp[2 * p + 1]), t);
+                    part[2 * p] = t.x;
+                    part[2 * p + 1] = t.y;
                 }
                 tc::tmem_st8(tl + T_XP + t0, part);
             }
         }
-        if (!mbar_wait_bounded(bar_z, ph, kTcWaitProbes)) ok = false;
+        if (!mbar_wait_sleep(bar_z, ph, kTcSleepProbes, kTcSleepNs)) ok = false;
         tc::fence_after_sync();
         ph ^= 1u;
         if (!out_pass) {
@@ -699,24 +716,27 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
                 float z3[8], part[8];
                 tc::tmem_ld8(tl + T_Z3 + t0, z3);
                 tc::tmem_ld8(tl + T_XP + t0, part);
+                const float4 g3[2] = {*reinterpret_cast<const float4 *>(k3 + t0),
+                                      *reinterpret_cast<const float4 *>(k3 + t0 + 4)};
                 tc::tmem_wait_ld();
-                float xn[8];
+                // x becomes the next round's x_prev (the part just read is dead), and the
+                // new iterate takes x's registers
+                tc::tmem_st8(tl + T_XP + t0, &xc[c * 8]);
 #pragma unroll
-                for (int u4 = 0; u4 < 8; u4 += 4) {
-                    const float4 g3 = *reinterpret_cast<const float4 *>(k3 + t0 + u4);
-                    const float g3v[4] = {g3.x, g3.y, g3.z, g3.w};
-#pragma unroll
-                    for (int v = 0; v < 4; ++v) xn[u4 + v] = fmaf(-g3v[v], z3[u4 + v], part[u4 + v]);
+                for (int p = 0; p < 4; ++p) {
+                    const float2 g3p = (p & 1) ? make_float2(g3[p >> 1].z, g3[p >> 1].w)
+                                               : make_float2(g3[p >> 1].x, g3[p >> 1].y);
+                    const float2 t = __ffma2_rn(g3p, make_float2(z3[2 * p], z3[2 * p + 1]),
+                                                make_float2(part[2 * p], part[2 * p + 1]));
+                    xc[c * 8 + 2 * p] = t.x;
+                    xc[c * 8 + 2 * p + 1] = t.y;
                 }
-                tc::tmem_st8(tl + T_XP + t0, &xc[c * 8]);   // x_prev of the next round
-#pragma unroll
-                for (int u = 0; u < 8; ++u) xc[c * 8 + u] = xn[u];
-                st_row8(sb + L::XT + (t0 >> 6) * 16384u, d, t0 & 63, xn);
+                st_row8(sb + L::XT + (t0 >> 6) * 16384u, d, t0 & 63, &xc[c * 8]);
             }
             // the next round's coefficient table (the other buffer)
             if (it + 1 < P.r) {
                 for (int e = tid; e < 3 * TOK; e += kSolveThreads)
-                    s_coef[((it + 1) & 1) * 3 * TOK + e] = w_next * s_cq[e];
+                    s_coef[((it + 1) & 1) * 3 * TOK + e] = (e < TOK ? w_next : -w_next) * s_cq[e];
             }
             fence_proxy_async_smem();
             tc::fence_before_sync();
