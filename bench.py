@@ -38,12 +38,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # bench reports null.  Captures and commands: profiles/*.md.
 TRAFFIC = {
     # full-size forward workload (B8 H8 T2048 D128, chunk 64), one launch
-    "chunk_solve_tc": {"bytes": 237.137408e6 + 23.863296e6, "workload": "bf16_b8h8t2048d128",
+    "chunk_solve_tc": {"bytes": 237.114112e6 + 20.744704e6, "workload": "bf16_b8h8t2048d128",
                        "src": "test_ridge_regression_b200/csrc/solve_tc.cuh",
-                       "sha1": "a3018159b4407640d7472ad4d3710aceb9045606"},
-    "state_pass_tc": {"bytes": 67.718912e6 + 80.975616e6, "workload": "bf16_b8h8t2048d128",
+                       "sha1": "9b1ad4883c334e9fcf528712492ca30eaace8ea0"},
+    "state_pass_tc": {"bytes": 67.709696e6 + 80.729088e6, "workload": "bf16_b8h8t2048d128",
                       "src": "test_ridge_regression_b200/csrc/state_tc.cuh",
-                      "sha1": "6b699f228b0797f72e56fce9c3607b1f777213e9"},
+                      "sha1": "d95a1373693a3001898b1cb7297e3fc496592228"},
     # decode captured on 64 x 32 heads (state above L2), scaled x4 to 256 x 32 heads
     "decode_step": {"bytes": 4 * (270.054912e6 + 213.513472e6), "workload": "decode_bf16_b256h32d128",
                     "src": "test_ridge_regression_b200/csrc/decode.cuh",
