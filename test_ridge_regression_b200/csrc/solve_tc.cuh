@@ -60,17 +60,17 @@ struct TcSmem {
     static constexpr uint32_t XT = KT + MG * 256;            // X^T: TOK/64 x [128][64], MN-major
     static constexpr uint32_t PT = XT + TOK * 256;           // P^T: TOK/64 x [MG][64], MN-major
     static constexpr uint32_t QS = PT + TOK * MG * 2;        // q: [TOK][128] bf16, then q^T
-    static constexpr uint32_t SCAL = QS + TOK * 256;         // per-token scalars [5][TOK]
+    static constexpr uint32_t SCAL = QS + TOK * 256;         // per-token scalars [3][TOK]
     static constexpr uint32_t RED = SCAL + 8 * 4 * TOK;      // float[16]
     static constexpr uint32_t NRM = RED + 64;                // u, E, X, Gjj [4][MG]
     static constexpr uint32_t NRM2 = NRM + 16 * MG;          // second warpgroup's E, X [2][MG]
     static constexpr uint32_t UPART = NRM2 + 8 * MG;         // [4 lane quarters][MG] partial u
     static constexpr uint32_t QPART = UPART + 16 * MG;       // [4 lane quarters][TOK] |q_j|^2
     static constexpr uint32_t DEC = QPART + 16 * TOK;        // l2, b, beta, beta^2: [4][MG] floats
-    // [2 rounds][3][TOK] w * (cq, c1, c3) of the rounds: over UPART and QPART,
-    // set-up scratch that is dead once the rounds start
+    // [2 rounds][TOK] -w c1 of the rounds: over UPART and QPART, set-up scratch
+    // that is dead once the rounds start
     static constexpr uint32_t COEF = UPART;
-    static_assert(24 * TOK <= DEC - UPART, "coefficient tables overrun the set-up scratch");
+    static_assert(8 * TOK <= DEC - UPART, "coefficient tables overrun the set-up scratch");
     static constexpr uint32_t BARS = DEC + 16 * MG;
     static constexpr uint32_t TBASE = BARS + 8 * 8;
     static constexpr uint32_t END = TBASE + 16;
@@ -225,11 +225,9 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = smem_align1024(smraw);
     const uint32_t sb = smem_u32(sm);
-    float *s_cq = reinterpret_cast<float *>(sm + L::SCAL);   // coefficient of q (scaled domain)
-    float *s_c1 = s_cq + TOK;                                // coefficient of Z1
-    float *s_c3 = s_c1 + TOK;                                // coefficient of Z3
+    float *s_c1 = reinterpret_cast<float *>(sm + L::SCAL);   // coefficient of Z1 (scaled domain)
+    float *s_c3 = s_c1 + TOK;                                // coefficient of Z3 (folded into W)
     float *s_o1 = s_c3 + TOK;                                // readout coefficient of Z1
-    float *s_o3 = s_o1 + TOK;                                // readout coefficient of Z3
     float *s_coef = reinterpret_cast<float *>(sm + L::COEF);
     float *red = reinterpret_cast<float *>(sm + L::RED);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BARS);
@@ -479,21 +477,41 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         const float invd = nj > 0.f ? 1.f / (P.half_1p2a * nj) : 0.f;
         const float b = s_bt[j0 + j];
         const float *qpart = reinterpret_cast<const float *>(sm + L::QPART);
-        const float qq = qpart[j] + qpart[TOK + j] + qpart[2 * TOK + j] + qpart[3 * TOK + j];
-        // every Chebyshev iterate obeys ||x|| <= ||q|| (1+2a) / (a d): the iterate is
-        // kept as x~ = sx x with sx a power of two that puts ||x~|| below 2^12
-        const float xb = sqrtf(qq) * invd * (2.f * P.half_1p2a / P.a);
-        const float sx = ldexpf(inv_pow2_above(xb), 12);
+        const float qn = sqrtf(qpart[j] + qpart[TOK + j] + qpart[2 * TOK + j] + qpart[3 * TOK + j]);
         const float eH = ldexpf(1.f, -eHexp);
         const float eM = ldexpf(1.f, -eMexp);
-        // (q - A x)/d in the scaled domain: cq q - c1 Z1 - c3 Z3 - cl x~
-        s_cq[j] = sx * invd;
+        // The iterate of token j is kept as x~ = (sigma / invd_j) x with sigma a power of
+        // two common to the CTA.  Every Chebyshev iterate obeys ||x|| <= ||q|| (1+2a) /
+        // (a d), so ||x~|| <= sigma ||q|| (1+2a) / a for every token, and in the scaled
+        // domain (q - A x) / d reads sigma q - c1 Z1 - c3 Z3 - cl x~: the coefficient of
+        // q is the same for all tokens.  c3 is folded into the decay weights below.
+        const float c3 = invd / (sK * sK);
         s_c1[j] = b * invd * eH;
-        s_c3[j] = invd / (sK * sK);
-        s_o1[j] = invd > 0.f ? b * eM / sx : 0.f;
-        s_o3[j] = invd > 0.f ? 1.f / (sV * sK * sx) : 0.f;
+        s_c3[j] = c3;
+        s_o1[j] = b * eM * invd;   // readout coefficient of Z1, times 1 / sigma below
+        float mq = qn, mc = c3;
+#pragma unroll
+        for (int o2 = 16; o2 > 0; o2 >>= 1) {
+            mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, o2));
+            mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, o2));
+        }
+        if (lane == 0) {
+            red[warp] = mq;
+            red[4 + warp] = mc;
+        }
     }
     __syncthreads();
+    // sigma puts every ||x~|| below 2^12; sc3 (a power of two) scales the largest c3
+    // below 1 so that the weighted products c3 w S stay in fp16 range
+    float qmax = 0.f, c3max = 0.f;
+#pragma unroll
+    for (int w = 0; w < TOK / 32; ++w) {
+        qmax = fmaxf(qmax, red[w]);
+        c3max = fmaxf(c3max, red[4 + w]);
+    }
+    const float sigma = ldexpf(inv_pow2_above(qmax * (2.f * P.half_1p2a / P.a)), 12);
+    const float sc3 = inv_pow2_above(c3max);
+    if (tid < TOK) s_o1[tid] *= 1.f / sigma;
 
     // q^T: this thread's tokens of row d, written into the (now free) tile as
     // [128 d][64 tokens] with 128B-swizzled rows: 8 tokens per 16-byte load later
@@ -505,7 +523,8 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     }
     const float cl = 2.f * P.a / (1.f + 2.f * P.a);   // lambda / d for every token with H != 0
 
-    // W^T rows: W[i][j] = w_{ji} = exp(l_j - l_i) for i <= j, else 0 (this thread's tokens)
+    // W^T rows: W[i][j] = sc3 c3_j w_{ji}, w_{ji} = exp(l_j - l_i) for i <= j, else 0
+    // (this thread's tokens); Z3 then carries c3 and its update coefficient is -w / sc3
     {
         // w = w_{j,key} along this thread's tokens j (zero while j < key)
         const int js = j0 + tcol;
@@ -517,13 +536,13 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
             for (int u = 0; u < 16; ++u) {
                 const int j = js + c * 16 + u;
                 if (c * 16 + u > 0) w = (j == key && s_owner) ? 1.f : w * s_bet[j];
-                wv[u] = w;
+                wv[u] = w * (s_c3[tcol + c * 16 + u] * sc3);   // c3_j w_ji, scaled by sc3
             }
             tc::tmem_st16(tl + T_W + tcol + c * 16, wv);
         }
     }
 
-    // x_1 = q / d, x_0 = 0 (scaled by sx): thread (wg, d) keeps element d of its 32
+    // x_1 = q / d, x_0 = 0 (x~_1 = sigma q): thread (wg, d) keeps element d of its 32
     // current iterates in registers and of the previous ones in TMEM
     float xc[TPT];
     {
@@ -536,15 +555,14 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
             float qv[16];
             load_qrow16(sb + L::QS + (t0 >> 6) * 16384u, d, (t0 & 63) >> 4, qv);
 #pragma unroll
-            for (int u = 0; u < 16; ++u) xc[c * 16 + u] = qv[u] * s_cq[t0 + u];
+            for (int u = 0; u < 16; ++u) xc[c * 16 + u] = qv[u] * sigma;
             st_row16(sb + L::XT + (t0 >> 6) * 16384u, d, t0 & 63, &xc[c * 16]);
             tc::tmem_st16(tl + T_XP + t0, zero16);
         }
         tc::tmem_wait_st();
     }
-    if (P.r > 1) {   // round 1's table omega (cq, -c1, -c3) (s_cq, s_c1, s_c3 are consecutive)
-        for (int e = tid; e < 3 * TOK; e += kSolveThreads)
-            s_coef[3 * TOK + e] = (e < TOK ? P.omega[1] : -P.omega[1]) * s_cq[e];
+    if (P.r > 1) {   // round 1's table: -w c1 per token
+        for (int e = tid; e < TOK; e += kSolveThreads) s_coef[TOK + e] = -P.omega[1] * s_c1[e];
     }
     fence_proxy_async_smem();
     tc::fence_before_sync();
@@ -649,14 +667,17 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         }
         // x_new = (1 - w) x_prev + w (1 - lambda/d) x + w cq q - w c1 Z1 - w c3 Z3 (the
         // three-term update with the residual (q - A x)/d written out; the per-token
-        // products w cq, -w c1, -w c3 of this round come from the table), in two parts:
+        // product -w c1 of this round comes from the table; the q and Z3 coefficients
+        // w sigma and -w / sc3 are common to all tokens), in two parts:
         // A, as soon as Z1 = H_s X^T is done (while the P phase and the intra-chunk
         // product run): part = (1 - w) x_prev + w (1 - lambda/d) x + w cq q - w c1 Z1,
         // kept in the x_prev columns of TMEM; B, once Z3 is done: x_new = part - w c3 Z3.
         // Pairs of tokens go through the packed f32x2 FMA pipe.
         const float cAs = 1.f - P.omega[it], cBs = P.omega[it] * (1.f - cl);
+        const float kqs = P.omega[it] * sigma, k3s = -P.omega[it] / sc3;
         const float2 cA = make_float2(cAs, cAs), cB = make_float2(cBs, cBs);
-        const float *kq = s_coef + (it & 1) * 3 * TOK, *k1 = kq + TOK, *k3 = k1 + TOK;
+        const float2 kq = make_float2(kqs, kqs), k3 = make_float2(k3s, k3s);
+        const float *k1 = s_coef + (it & 1) * TOK;
         if (!mbar_wait_sleep(bar_z1, ph, kTcSleepProbes, kTcSleepNs)) ok = false;
         tc::fence_after_sync();
         if (!out_pass) {
@@ -679,8 +700,6 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
                 tc::tmem_ld8(tl + T_XP + t0, xp);
                 const uint4 qw4 = ld_shared_u4(sb + L::QS + (t0 >> 6) * 16384u + d * 128u +
                                                ((((uint32_t)(t0 & 63) >> 3) ^ d) & 7u) * 16u);
-                const float4 gq[2] = {*reinterpret_cast<const float4 *>(kq + t0),
-                                      *reinterpret_cast<const float4 *>(kq + t0 + 4)};
                 const float4 g1[2] = {*reinterpret_cast<const float4 *>(k1 + t0),
                                       *reinterpret_cast<const float4 *>(k1 + t0 + 4)};
                 tc::tmem_wait_ld();
@@ -688,15 +707,13 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
                 float part[8];
 #pragma unroll
                 for (int p = 0; p < 4; ++p) {   // tokens 2p, 2p + 1
-                    const float2 gqp = (p & 1) ? make_float2(gq[p >> 1].z, gq[p >> 1].w)
-                                               : make_float2(gq[p >> 1].x, gq[p >> 1].y);
                     const float2 g1p = (p & 1) ? make_float2(g1[p >> 1].z, g1[p >> 1].w)
                                                : make_float2(g1[p >> 1].x, g1[p >> 1].y);
                     // q^T holds bf16 pairs: the low half is token 2p, the high half 2p + 1
                     const float2 qv = make_float2(__uint_as_float(qw[p] << 16),
                                                   __uint_as_float(qw[p] & 0xffff0000u));
                     float2 t = __fmul2_rn(g1p, make_float2(z1[2 * p], z1[2 * p + 1]));
-                    t = __ffma2_rn(gqp, qv, t);
+                    t = __ffma2_rn(kq, qv, t);
                     t = __ffma2_rn(cB, make_float2(xc[c * 8 + 2 * p], xc[c * 8 + 2 * p + 1]), t);
                     t = __ffma2_rn(cA, make_float2(xp[2 * p], xp[2 * p + 1]), t);
                     part[2 * p] = t.x;
@@ -716,17 +733,13 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
                 float z3[8], part[8];
                 tc::tmem_ld8(tl + T_Z3 + t0, z3);
                 tc::tmem_ld8(tl + T_XP + t0, part);
-                const float4 g3[2] = {*reinterpret_cast<const float4 *>(k3 + t0),
-                                      *reinterpret_cast<const float4 *>(k3 + t0 + 4)};
                 tc::tmem_wait_ld();
                 // x becomes the next round's x_prev (the part just read is dead), and the
                 // new iterate takes x's registers
                 tc::tmem_st8(tl + T_XP + t0, &xc[c * 8]);
 #pragma unroll
                 for (int p = 0; p < 4; ++p) {
-                    const float2 g3p = (p & 1) ? make_float2(g3[p >> 1].z, g3[p >> 1].w)
-                                               : make_float2(g3[p >> 1].x, g3[p >> 1].y);
-                    const float2 t = __ffma2_rn(g3p, make_float2(z3[2 * p], z3[2 * p + 1]),
+                    const float2 t = __ffma2_rn(k3, make_float2(z3[2 * p], z3[2 * p + 1]),
                                                 make_float2(part[2 * p], part[2 * p + 1]));
                     xc[c * 8 + 2 * p] = t.x;
                     xc[c * 8 + 2 * p + 1] = t.y;
@@ -735,28 +748,29 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
             }
             // the next round's coefficient table (the other buffer)
             if (it + 1 < P.r) {
-                for (int e = tid; e < 3 * TOK; e += kSolveThreads)
-                    s_coef[((it + 1) & 1) * 3 * TOK + e] = (e < TOK ? w_next : -w_next) * s_cq[e];
+                for (int e = tid; e < TOK; e += kSolveThreads)
+                    s_coef[((it + 1) & 1) * TOK + e] = -w_next * s_c1[e];
             }
             fence_proxy_async_smem();
             tc::fence_before_sync();
             ok = __syncthreads_and(ok);
         } else if (ok) {
-            // o_j[d] = b_j (M_s x_j)[d] + sum_i w_{ji} (k_i . x_j) v_i[d]
+            // o_j[d] = b_j (M_s x_j)[d] + sum_i w_{ji} (k_i . x_j) v_i[d]; Z3 carries
+            // sc3 c3_j, so its readout coefficient sK / (sV sigma sc3) is common to all tokens
+            const float o3 = sK / (sV * sigma * sc3);
             __nv_bfloat16 *orow = o + (tok0 + j0 + tcol) * kTcD + d;
 #pragma unroll
             for (int c = 0; c < NCH; ++c) {
                 const int t0 = tcol + c * 16;
-                float z1[16], z3[16], o1[16], o3[16];
+                float z1[16], z3[16], o1[16];
                 tc::tmem_ld16(tl + T_Z1 + t0, z1);
                 tc::tmem_ld16(tl + T_Z3 + t0, z3);
                 ld_f32x16(s_o1 + t0, o1);
-                ld_f32x16(s_o3 + t0, o3);
                 tc::tmem_wait_ld();
 #pragma unroll
                 for (int u = 0; u < 16; ++u)
                     orow[(size_t)(c * 16 + u) * kTcD] =
-                        __float2bfloat16_rn(fmaf(o1[u], z1[u], o3[u] * z3[u]));
+                        __float2bfloat16_rn(fmaf(o1[u], z1[u], o3 * z3[u]));
             }
         }
     }
