@@ -100,8 +100,8 @@ k_chunk_delta_tc(const __grid_constant__ DeltaMaps maps, const float *__restrict
         tokdec[3 * plane + tok0 + tid] = bt * bt;
     }
     bool ok = mbar_wait_bounded(bar_load, 0, kTcWaitProbes);
-    const float sK = tile_bf16_to_f16_scaled(sm + L::KT, C * 256, red);
-    const float sV = tile_bf16_to_f16_scaled(sm + L::VT, C * 256, red);
+    const float sK = tile_bf16_to_f16_scaled<C * 256, kTcThreads>(sm + L::KT, red);
+    const float sV = tile_bf16_to_f16_scaled<C * 256, kTcThreads>(sm + L::VT, red);
 
     // (w k)_hi and (w k)_lo tiles, same swizzled layout as the key tile: the
     // 16-byte chunk at byte c of half h belongs to key row (c % (C*128)) / 128

@@ -137,16 +137,25 @@ __device__ __forceinline__ void load_qrow16(uint32_t tile, uint32_t row, int c, 
     }
 }
 
-// In place: bf16 tile of `bytes` bytes -> fp16, scaled so that every |value| < 1.
-// Returns the scale.  Every thread of the block calls it (red: blockDim/32 floats).
-__device__ __forceinline__ float tile_bf16_to_f16_scaled(uint8_t *tile, int bytes, float *red) {
-    const int tid = threadIdx.x, nthr = blockDim.x, nw = nthr >> 5;
+// In place: bf16 tile of BYTES bytes -> fp16, scaled so that every |value| < 1.
+// Returns the scale.  All NTHR threads of the block call it (red: NTHR/32 floats);
+// each thread keeps the 16-byte pieces it reads for the max and converts them from
+// registers.
+template <int BYTES, int NTHR>
+__device__ __forceinline__ float tile_bf16_to_f16_scaled(uint8_t *tile, float *red) {
+    constexpr int PER = BYTES / (NTHR * 16);   // 16-byte pieces per thread
+    static_assert(BYTES % (NTHR * 16) == 0, "tile size");
+    const int tid = threadIdx.x, nw = NTHR >> 5;
+    uint4 u[PER];
     float mx = 0.f;
-    for (int c = tid * 16; c < bytes; c += nthr * 16) {
-        const uint4 u = *reinterpret_cast<const uint4 *>(tile + c);
-        const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&u);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(__bfloat162float(e[i])));
+    for (int i = 0; i < PER; ++i) {
+        u[i] = *reinterpret_cast<const uint4 *>(tile + (i * NTHR + tid) * 16);
+        const uint32_t w4[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(w4[e] << 16)),
+                                 fabsf(__uint_as_float(w4[e] & 0xffff0000u))));
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -156,15 +165,16 @@ __device__ __forceinline__ float tile_bf16_to_f16_scaled(uint8_t *tile, int byte
     mx = 0.f;
     for (int w = 0; w < nw; ++w) mx = fmaxf(mx, red[w]);
     const float sc = inv_pow2_above(mx);
-    for (int c = tid * 16; c < bytes; c += nthr * 16) {
-        uint4 u = *reinterpret_cast<const uint4 *>(tile + c);
-        const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&u);
-        uint4 w;
-        w.x = pack_f16(__bfloat162float(e[0]) * sc, __bfloat162float(e[1]) * sc);
-        w.y = pack_f16(__bfloat162float(e[2]) * sc, __bfloat162float(e[3]) * sc);
-        w.z = pack_f16(__bfloat162float(e[4]) * sc, __bfloat162float(e[5]) * sc);
-        w.w = pack_f16(__bfloat162float(e[6]) * sc, __bfloat162float(e[7]) * sc);
-        *reinterpret_cast<uint4 *>(tile + c) = w;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const uint32_t w4[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
+        uint32_t o4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            o4[e] = pack_f16(__uint_as_float(w4[e] << 16) * sc,
+                             __uint_as_float(w4[e] & 0xffff0000u) * sc);
+        *reinterpret_cast<uint4 *>(tile + (i * NTHR + tid) * 16) =
+            make_uint4(o4[0], o4[1], o4[2], o4[3]);
     }
     return sc;
 }
@@ -280,14 +290,13 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     // products of beta: w_{t,i-1} = w_ti beta_i and w_{t+1,i} = w_ti beta_{t+1}.
     float *s_l2 = reinterpret_cast<float *>(sm + L::DEC);
     float *s_bt = s_l2 + MG, *s_bet = s_bt + MG, *s_beta2 = s_bet + MG;
-    bool ok = mbar_wait_sleep(bar_load, 0, kTcSleepProbes, kTcSleepNs);
-    ok = mbar_wait_sleep(bar_v, 0, kTcSleepProbes, kTcSleepNs) && ok;
-    // keys and values: bf16 -> fp16 in place, scaled below 1
-    const float sK = tile_bf16_to_f16_scaled(sm + L::KT, MG * 256, red);
-    const float sV = tile_bf16_to_f16_scaled(sm + L::VT, MG * 256, red);
-    const __nv_bfloat16 *qs = reinterpret_cast<const __nv_bfloat16 *>(sm + L::QS);
     const int eHexp = state_exp[((size_t)bh * N + n) * 2];
     const int eMexp = state_exp[((size_t)bh * N + n) * 2 + 1];
+    bool ok = mbar_wait_sleep(bar_load, 0, kTcSleepProbes, kTcSleepNs);
+    // keys: bf16 -> fp16 in place, scaled below 1 (the values follow while the norm
+    // products run)
+    const float sK = tile_bf16_to_f16_scaled<MG * 256, kSolveThreads>(sm + L::KT, red);
+    const __nv_bfloat16 *qs = reinterpret_cast<const __nv_bfloat16 *>(sm + L::QS);
     fence_proxy_async_smem();
     tc::fence_before_sync();
     ok = __syncthreads_and(ok);
@@ -331,6 +340,9 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         }
         tc::commit(bar_n);
     }
+    // values: bf16 -> fp16 in place, scaled below 1 (first read by the readout)
+    ok = mbar_wait_sleep(bar_v, 0, kTcSleepProbes, kTcSleepNs) && ok;
+    const float sV = tile_bf16_to_f16_scaled<MG * 256, kSolveThreads>(sm + L::VT, red);
     float *s_u = reinterpret_cast<float *>(sm + L::NRM);
     float *s_E = s_u + MG, *s_X = s_E + MG, *s_G = s_X + MG;   // [MG] each; E and X: wg 0 part
     float *s_E1 = reinterpret_cast<float *>(sm + L::NRM2), *s_X1 = s_E1 + MG;   // wg 1 part
@@ -349,6 +361,25 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         }
         hs = warp_sum(hs);
         if (lane == 0) red[8 + warp] = hs;
+    }
+    // While the norm products run: the q column of this thread's tokens (token-major tile), kept packed for the
+    // transpose below; |q_j|^2 = sum_d q_j[d]^2 by a reduce-scatter over the warp
+    uint32_t qcol[TPT / 2];
+    {
+        float sq[TPT];
+#pragma unroll
+        for (int jj = 0; jj < TPT; jj += 2) {
+            const __nv_bfloat16 lo = qs[(tcol + jj) * kTcD + d], hi = qs[(tcol + jj + 1) * kTcD + d];
+            qcol[jj / 2] = (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+            const float a0 = __bfloat162float(lo), a1 = __bfloat162float(hi);
+            sq[jj] = a0 * a0;
+            sq[jj + 1] = a1 * a1;
+        }
+        reduce_scatter32<TPT>(sq, lane);
+#pragma unroll
+        for (int s2 = 0; s2 < TPT / 32; ++s2)
+            reinterpret_cast<float *>(sm + L::QPART)[quarter * TOK + tcol + lane * (TPT / 32) + s2] =
+                sq[s2];
     }
     if (!mbar_wait_sleep(bar_n, 0, kTcSleepProbes, kTcSleepNs)) ok = false;
     tc::fence_after_sync();
@@ -409,25 +440,6 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
             (wg == 0 ? s_X : s_X1)[gkey] = xs;
             if (has_diag) s_G[gkey] = gjj;
         }
-    }
-    // q column of this thread's tokens (token-major tile), kept packed for the
-    // transpose below; |q_j|^2 = sum_d q_j[d]^2 by a reduce-scatter over the warp
-    uint32_t qcol[TPT / 2];
-    {
-        float sq[TPT];
-#pragma unroll
-        for (int jj = 0; jj < TPT; jj += 2) {
-            const __nv_bfloat16 lo = qs[(tcol + jj) * kTcD + d], hi = qs[(tcol + jj + 1) * kTcD + d];
-            qcol[jj / 2] = (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
-            const float a0 = __bfloat162float(lo), a1 = __bfloat162float(hi);
-            sq[jj] = a0 * a0;
-            sq[jj + 1] = a1 * a1;
-        }
-        reduce_scatter32<TPT>(sq, lane);
-#pragma unroll
-        for (int s2 = 0; s2 < TPT / 32; ++s2)
-            reinterpret_cast<float *>(sm + L::QPART)[quarter * TOK + tcol + lane * (TPT / 32) + s2] =
-                sq[s2];
     }
     __syncthreads();
     // R_j = beta_j^2 R_{j-1} + (2 E_j + G_jj^2), R_{-1} = 0: an affine recurrence,
