@@ -147,6 +147,37 @@ def test_unnormalised_keys_and_strong_forgetting():
     check_against_oracle(q, k, v, beta, 0.1, 30, 64)
 
 
+def test_tensor_core_zero_keys_and_queries():
+    # zero keys at the start of a sequence and after a reset leave ||H_t|| = 0 (output 0
+    # by definition), zero queries give x = 0; the other tokens of the same chunks share
+    # the chunk's iterate scale and decay weights with them
+    q, k, v, beta = make_inputs(1, 2, 256, 128, torch.bfloat16, 2.0, 1.0, seed=21)
+    k[0, 0, :5] = 0.0
+    beta[0, 1, 100] = 0.0
+    k[0, 1, 100:103] = 0.0
+    q[0, 0, 70:74] = 0.0
+    q[0, 1, 130] = 0.0
+    for C in (64, 128):
+        check_against_oracle(q, k, v, beta, 0.5, 20, C)
+
+
+def test_tensor_core_query_scale_spread():
+    # the iterate scale is one power of two per chunk, set by the largest query: token
+    # queries spanning 2^-10 .. 2^10 within a chunk keep their relative accuracy, token
+    # by token (not only in the head's Frobenius norm, which the large tokens dominate)
+    q, k, v, beta = make_inputs(1, 2, 256, 128, torch.bfloat16, 2.0, 1.0, seed=22)
+    g = torch.Generator().manual_seed(5)
+    scale = torch.pow(2.0, torch.randint(-10, 11, (1, 2, 256, 1), generator=g).float())
+    q = (q.float() * scale).to(torch.bfloat16)
+    ref = oracle.forward(q, k, v, beta, 0.5, 20)["o"]
+    for C in (64, 128):
+        o, _, _ = run_forward(q, k, v, beta, 0.5, 20, C)
+        got, want = f64(o), f64(ref)
+        per_tok = np.linalg.norm(got - want, axis=-1) / np.linalg.norm(want, axis=-1)
+        print(f"chunk {C}: worst per-token rel err {per_tok.max():.3e}")
+        assert per_tok.max() <= TOL[torch.bfloat16]
+
+
 def test_chunk_size_does_not_change_result():
     q, k, v, beta = make_inputs(2, 2, 512, 128, torch.bfloat16, 3.0, 1.0, seed=11)
     o64, fs64, _ = run_forward(q, k, v, beta, 0.5, 20, 64)
