@@ -320,14 +320,14 @@ static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
         if ((e = set_smem(kern, TcSmem<64, 64>::bytes)) != cudaSuccess) return cuda_fail(e);
         ProfScope ps(GKA_KERNEL_CHUNK_SOLVE_TC, s);
         kern<<<dim3(N, BH), kSolveThreads, TcSmem<64, 64>::bytes, s>>>(
-            maps, q, tokdec, plane, norms, sexp, o, T, N, C, 0, P, flag);
+            maps, q, tokdec, plane, norms, sexp, o, T, N, C, P, flag);
     } else {
         // one CTA per 128-token chunk (N = 128 MMAs)
         auto kern = k_chunk_solve_tc<128, 128>;
         if ((e = set_smem(kern, TcSmem<128, 128>::bytes)) != cudaSuccess) return cuda_fail(e);
         ProfScope ps(GKA_KERNEL_CHUNK_SOLVE_TC, s);
         kern<<<dim3(N, BH), kSolveThreads, TcSmem<128, 128>::bytes, s>>>(
-            maps, q, tokdec, plane, norms, sexp, o, T, N, C, 0, P, flag);
+            maps, q, tokdec, plane, norms, sexp, o, T, N, C, P, flag);
     }
     if (int rc = check_launch()) return rc;
     return GKA_OK;
@@ -373,19 +373,6 @@ static int decode_launch(float *state, const void *q, const void *k, const void 
     return check_launch();
 }
 
-// Number of SMs of the current device (cached per device).
-static int sm_count() {
-    static int cache[256] = {0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return 148;
-    if (!cache[dev]) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-            n = 148;
-        cache[dev] = n;
-    }
-    return cache[dev];
-}
 
 template <typename Tin>
 static int decode_rows_launch(float *state, const void *q, const void *k, const void *v,

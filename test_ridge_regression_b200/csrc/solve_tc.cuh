@@ -7,31 +7,31 @@
 // w_{ti} (k_i . x) k_i, so every iteration of all tokens of a chunk is three
 // small GEMMs against the chunk-start state and the chunk's keys.
 //
-// One CTA (4 warps) solves one group of 64 tokens of one chunk; it needs the
-// chunk's first MG = 64 (group + 1) keys (later keys are masked for these
-// tokens).  Work is kept transposed so that every accumulator has M = 128
-// rows = the head dimension, one TMEM lane per thread:
-//   S^T = K X^T           (M = MG keys, N = 64 tokens, K = 128)      -> TMEM S
-//   Z1  = H_s X^T         (M = 128,     N = 64,        K = 128)      -> TMEM Z1
-//   P^T = W o S^T         (registers -> bf16 in shared memory, W_{ij} = w_{ji})
-//   Z3  = K^T P^T         (M = 128,     N = 64,        K = MG)       -> TMEM Z3
-//   y_j = b_j Z1[:,j] + Z3[:,j] + lambda_j x_j; three-term Chebyshev update in
-//   fp32 registers (thread d owns element d of all 64 iterates); the new
-//   iterate goes back to shared memory as bf16 (MN-major, 128B-swizzled) as
-//   the B operand of the next round.
-// The readout is the same three GEMMs with M_s in place of H_s and V in
-// place of K for the final product: o_j = b_j M_s x_j + sum_i w_{ji} (k_i.x_j) v_i.
-// H_s, M_s, K, V arrive by TMA and stay in shared memory for all r rounds.
+// One CTA (8 warps) solves one chunk of TOK = MG = C tokens (64 or 128).  Work is
+// kept transposed so that every accumulator has M = 128 rows, one TMEM lane per
+// thread:
+//   S^T = K X^T           (keys x tokens, K = 128)                    -> TMEM S
+//   Z1  = H_s X^T         (M = 128, N = TOK, K = 128)                  -> TMEM Z1
+//   P^T = W o S^T         (registers -> fp16 in shared memory, W_{ij} = w_{ji},
+//                          with each token's factor c3_j folded in)
+//   Z3  = K^T P^T         (M = 128, N = TOK, K = MG)                   -> TMEM Z3
+//   the three-term Chebyshev update in fp32 registers (thread d owns element d of
+//   its warpgroup's TOK/2 iterates); the new iterate goes back to shared memory as
+//   fp16 (MN-major, 128B-swizzled), the B operand of the next round.
+// The readout is the same three GEMMs with M_s in place of H_s and V in place of
+// K for the final product: o_j = b_j M_s x_j + sum_i w_{ji} (k_i.x_j) v_i.  H_s, K,
+// V and q arrive by TMA or bulk copies and stay in shared memory for all r rounds;
+// M_s replaces H_s for the readout.
 //
-// Operand precision: every MMA operand is fp16 with a power-of-two scale, fp32
-// accumulation.  bf16 keys and values convert exactly (scaled by 2^-e so that
-// |k|, |v| < 1); the chunk-start states come from the scan already in fp16,
-// scaled by 2^e from a bound on their Frobenius norm; each token's iterate is
-// scaled by 2^e from the bound ||x_i|| <= ||q|| (1+2a) / (a d) that every
-// Chebyshev iterate satisfies.  All scales are undone in fp32 in the
-// epilogue.  fp16 keeps 3 more mantissa bits than bf16 at the same tensor-core
-// rate; rounding the iterate to bf16 instead would cost about 1e-2 relative
-// error at a = 0.1 (condition number 11).
+// Operand precision: every MMA operand is fp16 with a scale, fp32 accumulation.
+// bf16 keys and values convert exactly (scaled by 2^-e so that |k|, |v| < 1); the
+// chunk-start states come from the state kernels already in fp16, scaled by 2^e
+// from a bound on their Frobenius norm; token j's iterate is kept as sigma x / invd_j
+// with sigma a power of two per chunk from the bound ||x_i|| <= ||q|| (1+2a) / (a d)
+// that every Chebyshev iterate satisfies, which makes the coefficient of q the same
+// for every token.  All scales are undone in fp32.  fp16 keeps 3 more mantissa
+// bits than bf16 at the same tensor-core rate; rounding the iterate to bf16 instead
+// would cost about 1e-2 relative error at a = 0.1 (condition number 11).
 #pragma once
 
 #include <cuda_fp16.h>
@@ -215,9 +215,7 @@ __device__ __forceinline__ void reduce_scatter32(float (&v)[N], int lane) {
     }
 }
 
-// grid (N, B*H).  A CTA solves TOK tokens (64 or 128) of one chunk, starting at
-// token 64 * group, with the chunk's first MG keys (MG = 64 (group + 1) for
-// TOK = 64; MG = 128 for TOK = 128, a whole 128-token chunk in one CTA so that
+// grid (N, B*H).  A CTA solves the TOK = MG tokens of one chunk (64, or 128 so that
 // every MMA has N = 128).  8 warps: warpgroup wg (warps 4wg..4wg+3) owns tokens
 // wg*TOK/2 .. (wg+1)*TOK/2 - 1; warp w reads TMEM lane quarter w % 4, so thread
 // (wg, d) owns element d of the iterates of its TOK/2 tokens.
@@ -226,7 +224,7 @@ __global__ void __launch_bounds__(kSolveThreads, TOK == 64 ? 2 : 1)
 k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__restrict__ q,
                  const float *__restrict__ tokdec, size_t plane, float *__restrict__ norms,
                  const int *__restrict__ state_exp, __nv_bfloat16 *__restrict__ o, int T, int N,
-                 int C, int group, const ChebParams P, int *__restrict__ timeout_flag) {
+                 int C, const ChebParams P, int *__restrict__ timeout_flag) {
     using L = TcSmem<MG, TOK>;
     constexpr int HALF = MG / 2;       // keys per warpgroup in the norm reductions
     constexpr int TPT = TOK / 2;       // tokens per thread
@@ -252,7 +250,6 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     const int d = quarter * 32 + lane;        // head-dimension row = TMEM lane of this thread
     const int tcol = wg * TPT;                // first token (TMEM column) of this thread
     const int n = blockIdx.x, bh = blockIdx.y;
-    const int j0 = group * 64;                             // first token of the CTA in the chunk
     const size_t tok0 = (size_t)bh * T + (size_t)n * C;    // first token of the chunk
     const int srow = (int)(((size_t)bh * N + n) * 2 * kTcD);   // H_s row in the state map
 
@@ -271,7 +268,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
                 tc::tma_load_2d(sm + L::KT + h * MG * 128 + rb * 8192, &maps.k, h * 64,
                                 (int)tok0 + rb * 64, bar_load);
         }
-        bulk_g2s(sm + L::QS, q + (tok0 + j0) * kTcD, TOK * kTcD * 2, bar_load);
+        bulk_g2s(sm + L::QS, q + tok0 * kTcD, TOK * kTcD * 2, bar_load);
         for (int pl = 0; pl < 4; ++pl)
             bulk_g2s(sm + L::DEC + pl * 4 * MG, tokdec + pl * plane + tok0, 4 * MG, bar_load);
         mbar_arrive_expect_tx(bar_v, MG * 256);
@@ -481,13 +478,13 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
 #pragma unroll
         for (int w = 0; w < kSolveThreads / 32; ++w) hs2 += red[8 + w];
         hs2 *= ldexpf(1.f, -2 * eHexp);
-        const float bj = s_bt[j0 + j];
+        const float bj = s_bt[j];
         const float n2 = fmaf(bj * bj, hs2,
-                              fmaf(2.f * bj, s_X[j0 + j] + s_X1[j0 + j], s_R[j0 + j]));
+                              fmaf(2.f * bj, s_X[j] + s_X1[j], s_R[j]));
         const float nj = sqrtf(fmaxf(n2, 0.f));
-        norms[tok0 + j0 + j] = nj;
+        norms[tok0 + j] = nj;
         const float invd = nj > 0.f ? 1.f / (P.half_1p2a * nj) : 0.f;
-        const float b = s_bt[j0 + j];
+        const float b = s_bt[j];
         const float *qpart = reinterpret_cast<const float *>(sm + L::QPART);
         const float qn = sqrtf(qpart[j] + qpart[TOK + j] + qpart[2 * TOK + j] + qpart[3 * TOK + j]);
         const float eH = ldexpf(1.f, -eHexp);
@@ -539,7 +536,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     // (this thread's tokens); Z3 then carries c3 and its update coefficient is -w / sc3
     {
         // w = w_{j,key} along this thread's tokens j (zero while j < key)
-        const int js = j0 + tcol;
+        const int js = tcol;
         float w = (s_owner && key <= js) ? exp2f(s_l2[js] - s_l2[key]) : 0.f;
         float wv[16];
 #pragma unroll
@@ -770,7 +767,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
             // o_j[d] = b_j (M_s x_j)[d] + sum_i w_{ji} (k_i . x_j) v_i[d]; Z3 carries
             // sc3 c3_j, so its readout coefficient sK / (sV sigma sc3) is common to all tokens
             const float o3 = sK / (sV * sigma * sc3);
-            __nv_bfloat16 *orow = o + (tok0 + j0 + tcol) * kTcD + d;
+            __nv_bfloat16 *orow = o + (tok0 + tcol) * kTcD + d;
 #pragma unroll
             for (int c = 0; c < NCH; ++c) {
                 const int t0 = tcol + c * 16;
