@@ -31,7 +31,7 @@
  *   - Supported: D in {32, 64, 128}; chunk in {16, 32, 64, 128}; 1 <= r <= 256;
  *     a > 0 and finite.  bf16 with D = 128 and chunk 64 or 128 runs the
  *     Chebyshev solve and readout on the tensor cores (tcgen05, TMEM
- *     accumulators, TMA-fed fp16 operands with power-of-two scales, fp32
+ *     accumulators, TMA-fed fp16 operands with per-tile or per-token scales, fp32
  *     accumulation and fp32 Chebyshev updates); every other case runs them on
  *     CUDA cores in fp32.
  */
