@@ -38,10 +38,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # bench reports null.  Captures and commands: profiles/*.md.
 TRAFFIC = {
     # full-size forward workload (B8 H8 T2048 D128, chunk 64), one launch
-    "chunk_solve_tc": {"bytes": 237.114112e6 + 20.744704e6, "workload": "bf16_b8h8t2048d128",
+    "chunk_solve_tc": {"bytes": 237.317120e6 + 21.281024e6, "workload": "bf16_b8h8t2048d128",
                        "src": "test_ridge_regression_b200/csrc/solve_tc.cuh",
-                       "sha1": "9b1ad4883c334e9fcf528712492ca30eaace8ea0"},
-    "state_pass_tc": {"bytes": 67.709696e6 + 80.729088e6, "workload": "bf16_b8h8t2048d128",
+                       "sha1": "a0eacd99a75638e4884b12f42cc63c5490c24b17"},
+    "state_pass_tc": {"bytes": 67.709696e6 + 79.886080e6, "workload": "bf16_b8h8t2048d128",
                       "src": "test_ridge_regression_b200/csrc/state_tc.cuh",
                       "sha1": "d95a1373693a3001898b1cb7297e3fc496592228"},
     # decode captured on 64 x 32 heads (state above L2), scaled x4 to 256 x 32 heads
