@@ -23,6 +23,14 @@
  * The decay beta_t multiplies the old state (the pages' gate gamma_t of the
  * weighted ridge objective, Eq. 3, with eta_{t,i} = prod_{j=i+1..t} gamma_j).
  *
+ * Write-gated variant (ai.info page, Main Findings, "The beta_t-augmented
+ * variant", and Future Directions): a per-token input-selectivity gate in
+ * [0, 1] scales the token's write into both states.  Named g_t here, since
+ * beta_t already names the decay:
+ *   H_t = beta_t H_{t-1} + g_t k_t k_t^T,   M_t = beta_t M_{t-1} + g_t v_t k_t^T
+ * Every entry point below takes the gate as a nullable array; NULL means
+ * g_t = 1 for every token (the layer of the paper's experiments).
+ *
  * All arithmetic is float64.  Matrices are dense row-major.
  */
 #include <math.h>
@@ -87,21 +95,23 @@ void gka_oracle_cheb_solve(const double *A, const double *q, int D,
 }
 
 /*
- * One token of the recurrence on one head, in place on (H, M).
+ * One token of the recurrence on one head, in place on (H, M), with decay
+ * beta and write gate g.
  * Writes the token's output o (D) and returns n_t = ||H_t||_F.
  * If solve == 0 only the state update and the norm are done.
  * work: D*D + 4*D doubles.
  */
 static double gka_token(double *H, double *M, const double *q, const double *k,
-                        const double *v, double beta, int D, double a, int r,
+                        const double *v, double beta, double g, int D, double a, int r,
                         int solve, double *o, double *work)
 {
     /* state update (ai.info, Methodology: running weighted covariances
-     * with a decay factor) */
+     * with a decay factor; Main Findings: the write gate g scales the
+     * token's own term) */
     for (int i = 0; i < D; ++i)
         for (int j = 0; j < D; ++j) {
-            H[(size_t)i * D + j] = beta * H[(size_t)i * D + j] + k[i] * k[j];
-            M[(size_t)i * D + j] = beta * M[(size_t)i * D + j] + v[i] * k[j];
+            H[(size_t)i * D + j] = beta * H[(size_t)i * D + j] + g * k[i] * k[j];
+            M[(size_t)i * D + j] = beta * M[(size_t)i * D + j] + g * v[i] * k[j];
         }
     /* Frobenius norm and adaptive ridge (ai.info, Key Contributions 2) */
     double n2 = 0.0;
@@ -130,6 +140,7 @@ static double gka_token(double *H, double *M, const double *q, const double *k,
 
 /*
  * Token-by-token forward over [B, Hh, T, D] inputs (row-major, D fastest).
+ *   gate        nullable, [B, Hh, T]: write gate g_t (NULL: 1 everywhere)
  *   init_state  nullable, [B, Hh, 2, D, D]: H then M at t = -1 (zero if NULL)
  *   solve_from  tokens t < solve_from only advance the state (o not written)
  *   o           [B, Hh, T, D]
@@ -142,7 +153,7 @@ static double gka_token(double *H, double *M, const double *q, const double *k,
  * Returns 0, or -1 on bad arguments.
  */
 int gka_oracle_forward(const double *q, const double *k, const double *v,
-                       const double *beta, int B, int Hh, int T, int D,
+                       const double *beta, const double *gate, int B, int Hh, int T, int D,
                        double a, int r, const double *init_state,
                        int solve_from, double *o, double *norms,
                        double *final_state, int chunk, double *chunk_states,
@@ -166,8 +177,9 @@ int gka_oracle_forward(const double *q, const double *k, const double *v,
                 memcpy(chunk_states + ((size_t)h * nchunks + t / chunk) * 2 * DD, H,
                        sizeof(double) * 2 * DD);
             size_t row = ((size_t)h * T + t) * D;
+            double g = gate ? gate[(size_t)h * T + t] : 1.0;
             double n = gka_token(H, M, q + row, k + row, v + row, beta[(size_t)h * T + t],
-                                 D, a, r, t >= solve_from, o + row, work);
+                                 g, D, a, r, t >= solve_from, o + row, work);
             if (norms) norms[(size_t)h * T + t] = n;
         }
         if (final_state) memcpy(final_state + (size_t)h * 2 * DD, H, sizeof(double) * 2 * DD);
@@ -180,10 +192,11 @@ int gka_oracle_forward(const double *q, const double *k, const double *v,
 /*
  * One recurrent decode step for [B, Hh] heads: the same token update as the
  * forward, applied in place to state [B, Hh, 2, D, D] (H then M).
- * q, k, v, o: [B, Hh, D];  beta: [B, Hh].
+ * q, k, v, o: [B, Hh, D];  beta: [B, Hh];  gate: nullable [B, Hh].
  */
 int gka_oracle_decode_step(double *state, const double *q, const double *k,
-                           const double *v, const double *beta, int B, int Hh,
+                           const double *v, const double *beta, const double *gate,
+                           int B, int Hh,
                            int D, double a, int r, double *o, int nthreads)
 {
     if (B < 0 || Hh < 0 || D <= 0 || r < 1 || !(a > 0.0)) return -1;
@@ -197,7 +210,7 @@ int gka_oracle_decode_step(double *state, const double *q, const double *k,
         double *work = (double *)malloc(sizeof(double) * (DD + 4 * (size_t)D));
         double *H = state + (size_t)h * 2 * DD;
         gka_token(H, H + DD, q + (size_t)h * D, k + (size_t)h * D, v + (size_t)h * D,
-                  beta[h], D, a, r, 1, o + (size_t)h * D, work);
+                  beta[h], gate ? gate[h] : 1.0, D, a, r, 1, o + (size_t)h * D, work);
         free(work);
     }
     return 0;
@@ -210,15 +223,18 @@ int gka_oracle_decode_step(double *state, const double *q, const double *k,
  * Within a chunk with start state H_s and positions j = 0..C-1:
  *   b_j    = prod_{m <= j} beta_m               (decay of H_s to token j)
  *   w_{ji} = prod_{i < m <= j} beta_m, i <= j   (decay of token i to token j)
- *   H_j    = b_j H_s + sum_{i<=j} w_{ji} k_i k_i^T
- *   ||H_j||_F^2 = b_j^2 ||H_s||_F^2 + 2 b_j sum_{i<=j} w_{ji} k_i^T H_s k_i
- *               + sum_{i,l<=j} w_{ji} w_{jl} (k_i^T k_l)^2
- * and the next chunk starts from H_s' = b_{C-1} H_s + sum_i w_{C-1,i} k_i k_i^T.
- * The products are formed directly (no logarithms).  T must be a multiple
- * of C.  norms: [B, Hh, T].
+ *   H_j    = b_j H_s + sum_{i<=j} w_{ji} g_i k_i k_i^T
+ *   ||H_j||_F^2 = b_j^2 ||H_s||_F^2 + 2 b_j sum_{i<=j} w_{ji} g_i k_i^T H_s k_i
+ *               + sum_{i,l<=j} w_{ji} g_i w_{jl} g_l (k_i^T k_l)^2
+ * and the next chunk starts from
+ *   H_s' = b_{C-1} H_s + sum_i w_{C-1,i} g_i k_i k_i^T.
+ * g is the write gate (nullable, [B, Hh, T]; NULL: 1).  The products are
+ * formed directly (no logarithms).  T must be a multiple of C.
+ * norms: [B, Hh, T].
  */
-int gka_oracle_chunked_norms(const double *k, const double *beta, int B, int Hh,
-                             int T, int D, int C, double *norms, int nthreads)
+int gka_oracle_chunked_norms(const double *k, const double *beta, const double *gate,
+                             int B, int Hh, int T, int D, int C, double *norms,
+                             int nthreads)
 {
     if (B < 0 || Hh < 0 || T < 0 || D <= 0 || C <= 0 || T % C != 0) return -1;
     long nh = (long)B * Hh;
@@ -237,7 +253,8 @@ int gka_oracle_chunked_norms(const double *k, const double *beta, int B, int Hh,
         for (int c0 = 0; c0 < T; c0 += C) {
             const double *K = k + ((size_t)h * T + c0) * D;
             const double *bt = beta + (size_t)h * T + c0;
-            /* decays */
+            const double *gt = gate ? gate + (size_t)h * T + c0 : NULL;
+            /* decays, each column i times the write gate of token i */
             for (int j = 0; j < C; ++j) {
                 double p = 1.0;
                 for (int m = 0; m <= j; ++m) p *= bt[m];
@@ -247,6 +264,7 @@ int gka_oracle_chunked_norms(const double *k, const double *beta, int B, int Hh,
                     if (i <= j) {
                         wji = 1.0;
                         for (int m = i + 1; m <= j; ++m) wji *= bt[m];
+                        if (gt) wji *= gt[i];
                     }
                     w[(size_t)j * C + i] = wji;
                 }

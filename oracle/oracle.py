@@ -47,13 +47,13 @@ def _load():
         lib.gka_oracle_omegas.restype = None
         lib.gka_oracle_cheb_solve.argtypes = [_dp, _dp, i, d, d, i, _dp, _dp]
         lib.gka_oracle_cheb_solve.restype = None
-        lib.gka_oracle_forward.argtypes = [_dp, _dp, _dp, _dp, i, i, i, i, d, i,
+        lib.gka_oracle_forward.argtypes = [_dp, _dp, _dp, _dp, _dp, i, i, i, i, d, i,
                                            _dp, i, _dp, _dp, _dp, i, _dp, i]
         lib.gka_oracle_forward.restype = i
-        lib.gka_oracle_decode_step.argtypes = [_dp, _dp, _dp, _dp, _dp, i, i, i,
+        lib.gka_oracle_decode_step.argtypes = [_dp, _dp, _dp, _dp, _dp, _dp, i, i, i,
                                                d, i, _dp, i]
         lib.gka_oracle_decode_step.restype = i
-        lib.gka_oracle_chunked_norms.argtypes = [_dp, _dp, i, i, i, i, i, _dp, i]
+        lib.gka_oracle_chunked_norms.argtypes = [_dp, _dp, _dp, i, i, i, i, i, _dp, i]
         lib.gka_oracle_chunked_norms.restype = i
         lib.gka_oracle_max_threads.argtypes = []
         lib.gka_oracle_max_threads.restype = i
@@ -95,10 +95,19 @@ def cheb_solve(A, q, mu: float, L: float, r: int) -> np.ndarray:
     return x
 
 
-def forward(q, k, v, beta, a: float, r: int, *, init_state=None, solve_from: int = 0,
-            want_norms: bool = False, want_final_state: bool = False,
+def _gate(gate, shape):
+    if gate is None:
+        return None
+    g = _f64(gate)
+    assert g.shape == shape, (g.shape, shape)
+    return g
+
+
+def forward(q, k, v, beta, a: float, r: int, *, gate=None, init_state=None,
+            solve_from: int = 0, want_norms: bool = False, want_final_state: bool = False,
             chunk: int = 0, want_chunk_states: bool = False, nthreads: int = 0):
-    """Token-by-token forward.  q, k, v: [B, H, T, D]; beta: [B, H, T].
+    """Token-by-token forward.  q, k, v: [B, H, T, D]; beta: [B, H, T];
+    gate: optional write gate [B, H, T] (None: 1 for every token).
 
     Returns a dict with ``o`` [B,H,T,D] and, on request, ``norms`` [B,H,T],
     ``final_state`` [B,H,2,D,D] and ``chunk_states`` [B,H,T/chunk,2,D,D]
@@ -114,10 +123,11 @@ def forward(q, k, v, beta, a: float, r: int, *, init_state=None, solve_from: int
     if want_chunk_states:
         assert chunk > 0 and T % chunk == 0
         cs = np.zeros((B, H, T // chunk, 2, D, D))
+    g = _gate(gate, (B, H, T))
     init = None if init_state is None else _f64(init_state)
     if init is not None:
         assert init.shape == (B, H, 2, D, D)
-    rc = _load().gka_oracle_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), B, H, T, D,
+    rc = _load().gka_oracle_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), B, H, T, D,
                                     float(a), int(r), _ptr(init), int(solve_from),
                                     _ptr(o), _ptr(norms), _ptr(fs), int(chunk), _ptr(cs),
                                     int(nthreads))
@@ -133,27 +143,31 @@ def forward(q, k, v, beta, a: float, r: int, *, init_state=None, solve_from: int
     return out
 
 
-def decode_step(state, q, k, v, beta, a: float, r: int, nthreads: int = 0):
+def decode_step(state, q, k, v, beta, a: float, r: int, nthreads: int = 0, gate=None):
     """One recurrent step.  state [B,H,2,D,D] (returned updated, new array);
-    q, k, v: [B,H,D]; beta [B,H].  Returns (o [B,H,D], state)."""
+    q, k, v: [B,H,D]; beta [B,H]; gate: optional write gate [B,H].
+    Returns (o [B,H,D], state)."""
     st = _f64(state).copy()
     q, k, v, beta = _f64(q), _f64(k), _f64(v), _f64(beta)
     B, H, D = q.shape
     assert st.shape == (B, H, 2, D, D) and beta.shape == (B, H)
     o = np.zeros((B, H, D))
+    g = _gate(gate, (B, H))
     rc = _load().gka_oracle_decode_step(_ptr(st), _ptr(q), _ptr(k), _ptr(v), _ptr(beta),
-                                        B, H, D, float(a), int(r), _ptr(o), int(nthreads))
+                                        _ptr(g), B, H, D, float(a), int(r), _ptr(o), int(nthreads))
     if rc != 0:
         raise ValueError("gka_oracle_decode_step: bad arguments")
     return o, st
 
 
-def chunked_norms(k, beta, chunk: int, nthreads: int = 0) -> np.ndarray:
-    """||H_t||_F by the chunk-wise closed form.  k [B,H,T,D], beta [B,H,T]."""
+def chunked_norms(k, beta, chunk: int, nthreads: int = 0, gate=None) -> np.ndarray:
+    """||H_t||_F by the chunk-wise closed form.  k [B,H,T,D], beta [B,H,T],
+    gate: optional write gate [B,H,T]."""
     k, beta = _f64(k), _f64(beta)
     B, H, T, D = k.shape
+    g = _gate(gate, (B, H, T))
     out = np.zeros((B, H, T))
-    rc = _load().gka_oracle_chunked_norms(_ptr(k), _ptr(beta), B, H, T, D, int(chunk),
+    rc = _load().gka_oracle_chunked_norms(_ptr(k), _ptr(beta), _ptr(g), B, H, T, D, int(chunk),
                                           _ptr(out), int(nthreads))
     if rc != 0:
         raise ValueError("gka_oracle_chunked_norms: bad arguments")

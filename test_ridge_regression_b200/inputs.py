@@ -10,6 +10,12 @@ l2 norm before the layer, Fig. 2 of the paper), then cast to the compute
 dtype; v ~ N(0, 1) cast to the dtype; beta = sigmoid(N(mu, sigma)) in fp32.
 All draws come from one torch CPU generator seeded per workload, in the order
 q, k, v, beta.
+
+Write gate (the paper's beta_t-augmented variant; ai.info page, Main Findings):
+g = sigmoid(N(mu, sigma)) in fp32, mu = 0 and sigma = 1.5 by default (the pages
+give no distribution for the learned gate; this spreads it over (0, 1) around
+1/2), from its own generator seeded with the workload seed + 1_000_000, so the
+other inputs do not change when a gate is drawn.
 """
 from __future__ import annotations
 
@@ -85,6 +91,13 @@ def make_inputs(B: int, H: int, T: int, D: int, dtype: torch.dtype, beta_mu: flo
     beta = torch.sigmoid(beta_mu + beta_sigma * torch.randn(B, H, T, generator=g,
                                                             dtype=torch.float32))
     return q.contiguous(), k.contiguous(), v.contiguous(), beta.contiguous()
+
+
+def make_gate(shape, seed: int, mu: float = 0.0, sigma: float = 1.5) -> torch.Tensor:
+    """Write gate in (0, 1), fp32 CPU tensor of ``shape`` ([B, H, T] or [B, H])."""
+    g = _gen(seed + 1_000_000)
+    return torch.sigmoid(mu + sigma * torch.randn(*shape, generator=g,
+                                                  dtype=torch.float32)).contiguous()
 
 
 def workload_inputs(w: Workload, *, B: int | None = None, H: int | None = None,
