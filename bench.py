@@ -72,6 +72,8 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default=WORKLOAD)
     p.add_argument("--no-decode", action="store_true")
+    p.add_argument("--no-write-gate", action="store_true",
+                   help="skip the write-gated forward leg")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--decode-steps", type=int, default=None)
     p.add_argument("--decode-batch", type=int, default=None,
@@ -419,6 +421,11 @@ def main():
         raise RuntimeError("device status error after the end-to-end steps")
     del qh, kh, vh, bh, oh
 
+    # ---- write-gated forward on the same inputs plus a gate ----
+    if not args.no_write_gate:
+        result["write_gate"] = bench_write_gate(args, w, dev, qd, kd, vd, bd, od, ws, flush,
+                                                rank, world, barrier)
+
     # ---- decode step: HBM-bound, 256 x 32 heads, fp32 state ----
     if not args.no_decode and world == 1:
         result["decode"] = bench_decode(args, dev, peaks)
@@ -442,6 +449,49 @@ def main():
         print(json.dumps(result), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def bench_write_gate(args, w, dev, qd, kd, vd, bd, od, ws, flush, rank, world, barrier):
+    """The paper's beta_t-augmented variant (a per-token write gate in [0, 1],
+    gka_forward_gated) on the workload's inputs: K steps timed like the main ones,
+    then the same K steps under the launch profiler for the per-kernel times."""
+    import torch
+    from test_ridge_regression_b200 import dist as gdist
+    from test_ridge_regression_b200 import gka
+    from test_ridge_regression_b200.inputs import make_gate
+    gd = make_gate((w.B, w.H, w.T), gdist.shard_seed(w.seed, rank)).to(dev)
+
+    def step():
+        gka.gka_forward_gated(qd, kd, vd, bd, gd, w.a, w.r, w.chunk, o=od, workspace=ws)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    barrier()
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        starts[i].record()
+        step()
+        ends[i].record()
+    torch.cuda.synchronize()
+    barrier()
+    total_ms = gdist.max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)), dev)
+    gka.profiler_read()
+    gka.profiler_enable(True)
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        step()
+    torch.cuda.synchronize()
+    gka.profiler_enable(False)
+    kt = gka.profiler_read()
+    if gka.device_status() != 0:
+        raise RuntimeError("device status error after the write-gated steps")
+    return {"gate": "sigmoid(N(0,1.5)) per token, fp32", "ms_per_step": total_ms / args.steps,
+            "tokens_per_s": world * w.B * w.T * args.steps / (total_ms / 1e3),
+            "kernels_ms_per_step": {n: ms / args.steps for n, (ms, _) in kt.items()},
+            "gpu_launches": sum(n for _, n in kt.values())}
 
 
 def bench_decode(args, dev, peaks):

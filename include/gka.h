@@ -113,6 +113,29 @@ int gka_forward(const void *q, const void *k, const void *v, const float *beta, 
                 float *final_state, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Write-gated forward: the paper's beta_t-augmented variant (ai.info page,
+ * Main Findings, "The beta_t-augmented variant", and Future Directions: a
+ * learned per-token input-selectivity gate in [0, 1] scales the token's write
+ * into both states).  With the gate named g_t (beta_t names the decay here):
+ *     H_t = beta_t H_{t-1} + g_t k_t k_t^T,   M_t = beta_t M_{t-1} + g_t v_t k_t^T,
+ * and everything else as in gka_forward (lambda_t = a ||H_t||_F, the same
+ * Chebyshev solve, o_t = M_t x_t).
+ *   gate   nullable fp32 [B, H, T], values in [0, 1], 16-byte aligned; NULL
+ *          means g_t = 1 for every token, and the call is then exactly
+ *          gka_forward (same kernels, same results bit for bit)
+ * Every other argument, the workspace size and the error behaviour are those
+ * of gka_forward.  The kernels fold g_i into the weight of token i's write
+ * (the chunk increments, the decode update) or scale token i's key and value
+ * rows by sqrt(g_i) where both sides of a product read the same row (the
+ * per-token norm, the solve and the readout); the two are equal in exact
+ * arithmetic.
+ */
+int gka_forward_gated(const void *q, const void *k, const void *v, const float *beta,
+                      const float *gate, void *o, int B, int H, int T, int D, gka_dtype dt,
+                      float a, int r, int chunk, float *final_state, void *workspace,
+                      size_t workspace_bytes, void *stream);
+
+/*
  * gka_forward from HOST buffers, with the copies overlapped with the compute
  * (no counterpart in the paper: a transfer pipeline around the forward).
  * The B*H independent sequences, flattened to pairs p = b*H + h, are cut into
@@ -187,6 +210,16 @@ int gka_forward_static_scratch(const void *q, const void *k, const void *v, cons
 int gka_decode_step(float *state, const void *q, const void *k, const void *v,
                     const float *beta, void *o, int B, int H, int D, gka_dtype dt,
                     float a, int r, void *stream);
+
+/*
+ * Write-gated decode step (the recurrent form of gka_forward_gated):
+ *   H <- beta H + g k k^T;  M <- beta M + g v k^T;  the rest as gka_decode_step.
+ *   gate   nullable fp32 [B, H] in [0, 1], 16-byte aligned (NULL: g = 1, exactly
+ *          gka_decode_step).
+ */
+int gka_decode_step_gated(float *state, const void *q, const void *k, const void *v,
+                          const float *beta, const float *gate, void *o, int B, int H, int D,
+                          gka_dtype dt, float a, int r, void *stream);
 
 /* Synchronises `stream`, then returns GKA_ERR_DEVICE_TIMEOUT if any kernel of
  * this library on the current device gave up a bounded wait since the last

@@ -11,6 +11,10 @@
 //   H_j    = b_j H_s + sum_{i<=j} w_{ji} k_i k_i^T
 //   M_j    = b_j M_s + sum_{i<=j} w_{ji} v_i k_i^T
 // so H_j x = b_j H_s x + sum_{i<=j} w_{ji} (k_i . x) k_i never needs H_j.
+// With the write gate g_i (the paper's beta_t-augmented variant, ai.info page,
+// Main Findings; `gate` nullable, NULL = 1) every w_{ji} above becomes
+// w_{ji} g_i: the increments take g_i into the weight, the norm and the solve
+// read sqrt(g_i) k_i and sqrt(g_i) v_i (the same products in exact arithmetic).
 #pragma once
 
 #include <cuda_fp16.h>
@@ -30,7 +34,8 @@ constexpr int kSimtThreads = 256;
 template <typename Tin, int D>
 __global__ void __launch_bounds__(kSimtThreads)
 k_chunk_delta(const Tin *__restrict__ k, const Tin *__restrict__ v,
-              const float *__restrict__ beta, float *__restrict__ states,
+              const float *__restrict__ beta, const float *__restrict__ gate,
+              float *__restrict__ states,
               float *__restrict__ decay, float *__restrict__ bound_inc, int T, int N, int C) {
     extern __shared__ __align__(16) float sm[];
     float *Ks = sm;            // [C][D] keys
@@ -45,7 +50,8 @@ k_chunk_delta(const Tin *__restrict__ k, const Tin *__restrict__ v,
     const double lend = ell[C - 1];
     for (int e = threadIdx.x; e < C * D; e += kSimtThreads) {
         const int i = e / D;
-        const float w = decay_exp(lend - ell[i]);
+        float w = decay_exp(lend - ell[i]);
+        if (gate) w *= gate[tok0 + i];
         const float kv = load_f(k + tok0 * D + e);
         Ks[e] = kv;
         Kw[e] = w * kv;
@@ -221,7 +227,7 @@ k_state_scan(float *__restrict__ states, const float *__restrict__ decay,
 template <typename Tin, int D>
 __global__ void __launch_bounds__(kSimtThreads)
 k_chunk_norm(const Tin *__restrict__ k, const float *__restrict__ beta,
-             const float *__restrict__ states, float *__restrict__ norms, int T, int N,
+             const float *__restrict__ gate, const float *__restrict__ states, float *__restrict__ norms, int T, int N,
              int C) {
     extern __shared__ __align__(16) float sm[];
     float *Hs = sm;                 // [D][D]
@@ -244,7 +250,11 @@ k_chunk_norm(const Tin *__restrict__ k, const float *__restrict__ beta,
         Hs[e] = h;
         ss = fmaf(h, h, ss);
     }
-    for (int e = tid; e < C * D; e += kSimtThreads) Ks[(e / D) * KP + e % D] = load_f(k + tok0 * D + e);
+    for (int e = tid; e < C * D; e += kSimtThreads) {
+        float kv = load_f(k + tok0 * D + e);
+        if (gate) kv *= sqrtf(gate[tok0 + e / D]);
+        Ks[(e / D) * KP + e % D] = kv;
+    }
     for (int j = tid; j < C; j += kSimtThreads) {
         bj[j] = decay_exp(ell[j]);
         betaj[j] = decay_exp(j == 0 ? ell[0] : ell[j] - ell[j - 1]);
@@ -336,7 +346,8 @@ struct SolveSmem {
 template <typename Tin, int D>
 __global__ void __launch_bounds__(kSimtThreads)
 k_chunk_solve(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
-              const float *__restrict__ beta, const float *__restrict__ states,
+              const float *__restrict__ beta, const float *__restrict__ gate,
+              const float *__restrict__ states,
               const float *__restrict__ norms, Tin *__restrict__ o, int T, int N, int C,
               const ChebParams P) {
     constexpr int TG = kSolveTG;
@@ -361,7 +372,15 @@ k_chunk_solve(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
 
     const float *Hg = states + ((size_t)bh * (N + 1) + n) * 2 * D * D;
     for (int e = tid; e < D * D; e += kSimtThreads) Ms[(e / D) * KP + e % D] = Hg[e];
-    for (int e = tid; e < jend * D; e += kSimtThreads) Ks[(e / D) * KP + e % D] = load_f(k + tok0 * D + e);
+    // keys (and at the readout values) of token i scaled by sqrt(g_i)
+    auto load_rows = [&](const Tin *src) {
+        for (int e = tid; e < jend * D; e += kSimtThreads) {
+            float x = load_f(src + tok0 * D + e);
+            if (gate) x *= sqrtf(gate[tok0 + e / D]);
+            Ks[(e / D) * KP + e % D] = x;
+        }
+    };
+    load_rows(k);
     for (int e = tid; e < TG * D; e += kSimtThreads) Qs[e] = load_f(q + (tok0 + j0) * D + e);
     if (tid < TG) {
         const float nj = norms[tok0 + j0 + tid];
@@ -455,7 +474,7 @@ k_chunk_solve(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
         const int row = e / D, col = e % D;   // M[row][col]; stored as Ms[col][row]
         Ms[col * KP + row] = Mg[e];
     }
-    for (int e = tid; e < jend * D; e += kSimtThreads) Ks[(e / D) * KP + e % D] = load_f(v + tok0 * D + e);
+    load_rows(v);
     __syncthreads();
     float acc[NJ];
     apply(acc);

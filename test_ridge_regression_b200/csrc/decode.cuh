@@ -5,6 +5,8 @@
 //   H <- beta H + k k^T;  n = ||H||_F;  lambda = a n;
 //   x = r-step Chebyshev for (H + lambda I) x = q on [a n, (1+a) n];
 //   M <- beta M + v k^T;  o = M x.
+// With the write gate g (the paper's beta_t-augmented variant, ai.info page,
+// Main Findings; nullable, NULL = 1) the writes are g k k^T and g v k^T.
 //
 // The step is bound by HBM traffic: each head reads and writes 2 * D * D fp32
 // state words once.  One CTA of 4*D threads serves one head.  H stays in
@@ -84,7 +86,8 @@ constexpr uint32_t kDecodeWaitProbes = 1u << 22;
 template <typename Tin, int D>
 __global__ void __launch_bounds__(4 * D, 2)
 k_decode_step(float *__restrict__ state, const Tin *__restrict__ q, const Tin *__restrict__ k,
-              const Tin *__restrict__ v, const float *__restrict__ beta, Tin *__restrict__ o,
+              const Tin *__restrict__ v, const float *__restrict__ beta,
+              const float *__restrict__ gate, Tin *__restrict__ o,
               const ChebParams P, int *__restrict__ timeout_flag) {
     constexpr int NT = 4 * D, NW = NT / 32, CPL = D / 32;
     extern __shared__ __align__(128) float Msm[];   // [D][D] M tile
@@ -107,9 +110,10 @@ k_decode_step(float *__restrict__ state, const Tin *__restrict__ q, const Tin *_
         bulk_g2s(Msm, Mg, D * D * 4, &mbar);
     }
     const float bt = beta[head];
+    const float gt = gate ? gate[head] : 1.f;   // write gate: g k k^T and g v k^T
     for (int i = tid; i < D; i += NT) {
         ks[i] = load_f(k + (size_t)head * D + i);
-        vs[i] = load_f(v + (size_t)head * D + i);
+        vs[i] = load_f(v + (size_t)head * D + i) * gt;
     }
     __syncthreads();
 
@@ -121,7 +125,7 @@ k_decode_step(float *__restrict__ state, const Tin *__restrict__ q, const Tin *_
     for (int rr = 0; rr < 8; ++rr) {
         float *rowp = Hg + (size_t)(row0 + rr) * D + col0;
         VecF<CPL>::ld(rowp, h[rr]);
-        const float kr = ks[row0 + rr];
+        const float kr = ks[row0 + rr] * gt;
 #pragma unroll
         for (int c = 0; c < CPL; ++c) {
             h[rr][c] = fmaf(bt, h[rr][c], kr * ks[col0 + c]);
@@ -224,7 +228,7 @@ template <typename Tin>
 __global__ void __launch_bounds__(kDecRowThreads, 3)
 k_decode_rows(const __grid_constant__ DecodeMaps maps, const Tin *__restrict__ q,
               const Tin *__restrict__ k, const Tin *__restrict__ v, const float *__restrict__ beta,
-              Tin *__restrict__ o, const ChebParams P, int *__restrict__ timeout_flag) {
+              const float *__restrict__ gate, Tin *__restrict__ o, const ChebParams P, int *__restrict__ timeout_flag) {
     constexpr int D = kDecD, NW = kDecRowThreads / 32;
     extern __shared__ uint8_t draw[];
     uint8_t *buf = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(draw) + 1023) &
@@ -249,15 +253,16 @@ k_decode_rows(const __grid_constant__ DecodeMaps maps, const Tin *__restrict__ q
         for (int b = 0; b < 4; ++b) tc::tma_load_2d(buf + b * 16384, &maps.state, b * 32, hrow, &bar[0]);
     }
     const float bt = beta[head];
+    const float gt = gate ? gate[head] : 1.f;   // write gate: g k k^T and g v k^T
     ks[t] = load_f(k + (size_t)head * D + t);
-    const float vt = load_f(v + (size_t)head * D + t);
+    const float vt = load_f(v + (size_t)head * D + t) * gt;
     const float qt = load_f(q + (size_t)head * D + t);
     bool ok = mbar_wait_bounded(&bar[0], 0, kDecodeWaitProbes);
     __syncthreads();   // ks complete
 
     // H row t -> registers, updated: h = beta h + k_t k
     float h[D];
-    const float kt = ks[t];
+    const float kt = ks[t] * gt;
     float ss = 0.f;
 #pragma unroll
     for (int c = 0; c < D / 4; ++c) {

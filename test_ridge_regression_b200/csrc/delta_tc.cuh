@@ -5,7 +5,8 @@
 // chunk n is  S_{n+1} = b_{C-1} S_n + dS_n  with
 //   dH_n = sum_i w_{C-1,i} k_i k_i^T = K^T diag(w) K,
 //   dM_n = sum_i w_{C-1,i} v_i k_i^T = V^T diag(w) K,
-// two 128 x 128 x C products per chunk; the scan kernel adds them up.
+// two 128 x 128 x C products per chunk; the scan kernel adds them up.  With
+// the write gate g (nullable) every weight w_{C-1,i} is w_{C-1,i} g_i.
 //
 // One CTA (4 warps) per chunk.  K and V arrive by TMA (bf16) and are turned
 // into fp16 with a power-of-two scale below 1 (exact).  The weighted keys
@@ -36,7 +37,8 @@ struct DeltaSmem {
     static constexpr uint32_t WL = WH + C * 256;      // 2 x [C][64] (w k)_lo
     static constexpr uint32_t STAGE = WL + C * 256;   // 2 x [128][32] fp32 store staging (swizzled)
     static constexpr uint32_t ELL = STAGE + 32768;    // double[C] cumulative logs
-    static constexpr uint32_t RED = ELL + 8 * C + 8 * (kTcThreads / 32);
+    static constexpr uint32_t WT = ELL + 8 * C + 8 * (kTcThreads / 32);   // float[C] weights
+    static constexpr uint32_t RED = WT + 4 * C;
     static constexpr uint32_t BARS = RED + 64;
     static constexpr uint32_t TBASE = BARS + 32;
     static constexpr uint32_t END = TBASE + 16;
@@ -53,7 +55,7 @@ struct DeltaMaps {
 template <int C>
 __global__ void __launch_bounds__(kTcThreads, 1)
 k_chunk_delta_tc(const __grid_constant__ DeltaMaps maps, const float *__restrict__ beta,
-                 float *__restrict__ states, float *__restrict__ decay,
+                 const float *__restrict__ gate, float *__restrict__ states, float *__restrict__ decay,
                  float *__restrict__ bound_inc, float *__restrict__ tokdec, size_t plane, int T,
                  int N, int *__restrict__ timeout_flag) {
     using L = DeltaSmem<C>;
@@ -63,6 +65,7 @@ k_chunk_delta_tc(const __grid_constant__ DeltaMaps maps, const float *__restrict
     const uint32_t sb = smem_u32(sm);
     double *ell = reinterpret_cast<double *>(sm + L::ELL);
     double *wtot = ell + C;
+    float *s_wt = reinterpret_cast<float *>(sm + L::WT);   // w_{C-1,i} g_i
     float *red = reinterpret_cast<float *>(sm + L::RED);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BARS);
     uint64_t *bar_load = &bars[0], *bar_mma = &bars[1];
@@ -98,6 +101,9 @@ k_chunk_delta_tc(const __grid_constant__ DeltaMaps maps, const float *__restrict
         tokdec[plane + tok0 + tid] = decay_exp(ell[tid]);
         tokdec[2 * plane + tok0 + tid] = bt;
         tokdec[3 * plane + tok0 + tid] = bt * bt;
+        float w = decay_exp(ell[C - 1] - ell[tid]);
+        if (gate) w *= gate[tok0 + tid];   // write gate of token tid
+        s_wt[tid] = w;
     }
     bool ok = mbar_wait_bounded(bar_load, 0, kTcWaitProbes);
     const float sK = tile_bf16_to_f16_scaled<C * 256, kTcThreads>(sm + L::KT, red);
@@ -108,7 +114,7 @@ k_chunk_delta_tc(const __grid_constant__ DeltaMaps maps, const float *__restrict
     const double lend = ell[C - 1];
     for (int c = tid * 16; c < C * 256; c += kTcThreads * 16) {
         const int row = (c % (C * 128)) >> 7;
-        const float w = decay_exp(lend - ell[row]);
+        const float w = s_wt[row];
         const uint4 u = *reinterpret_cast<const uint4 *>(sm + L::KT + c);
         const __half *e = reinterpret_cast<const __half *>(&u);
         float hv[8], lv[8];
@@ -151,7 +157,7 @@ k_chunk_delta_tc(const __grid_constant__ DeltaMaps maps, const float *__restrict
     {
         float bhs = 0.f, bms = 0.f;
         for (int i = tid; i < C; i += kTcThreads) {
-            const float w = decay_exp(lend - ell[i]);
+            const float w = s_wt[i];
             float kk2 = 0.f, vv2 = 0.f;
             for (int h = 0; h < 2; ++h) {
                 const __half *kr = reinterpret_cast<const __half *>(sm + L::KT + h * C * 128 + i * 128);

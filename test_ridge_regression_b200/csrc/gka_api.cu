@@ -165,8 +165,9 @@ static cudaError_t set_smem(K kernel, size_t bytes) {
 }
 
 template <typename Tin, int D>
-static int forward_simt(const Tin *q, const Tin *k, const Tin *v, const float *beta, Tin *o,
-                        int B, int H, int T, int C, const ChebParams &P, float *final_state,
+static int forward_simt(const Tin *q, const Tin *k, const Tin *v, const float *beta,
+                        const float *gate, Tin *o, int B, int H, int T, int C,
+                        const ChebParams &P, float *final_state,
                         char *ws, const gka_workspace_layout &L, cudaStream_t s) {
     const int BH = B * H, N = T / C;
     float *states = reinterpret_cast<float *>(ws + L.states_offset);
@@ -177,8 +178,8 @@ static int forward_simt(const Tin *q, const Tin *k, const Tin *v, const float *b
     const size_t sm_delta = sizeof(float) * 3 * (size_t)C * D;
     if ((e = set_smem(k_chunk_delta<Tin, D>, sm_delta)) != cudaSuccess) return cuda_fail(e);
     { ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
-    k_chunk_delta<Tin, D><<<dim3(N, BH), kSimtThreads, sm_delta, s>>>(k, v, beta, states, decay,
-                                                                        nullptr, T, N, C); }
+    k_chunk_delta<Tin, D><<<dim3(N, BH), kSimtThreads, sm_delta, s>>>(k, v, beta, gate, states,
+                                                                        decay, nullptr, T, N, C); }
     if (int rc = check_launch()) return rc;
 
     const int DD2 = 2 * D * D;
@@ -190,15 +191,15 @@ static int forward_simt(const Tin *q, const Tin *k, const Tin *v, const float *b
     const size_t sm_norm = sizeof(float) * ((size_t)D * D + (size_t)C * (D + 1));
     if ((e = set_smem(k_chunk_norm<Tin, D>, sm_norm)) != cudaSuccess) return cuda_fail(e);
     { ProfScope ps(GKA_KERNEL_CHUNK_NORM, s);
-    k_chunk_norm<Tin, D><<<dim3(N, BH), kSimtThreads, sm_norm, s>>>(k, beta, states, norms, T, N,
-                                                                    C); }
+    k_chunk_norm<Tin, D><<<dim3(N, BH), kSimtThreads, sm_norm, s>>>(k, beta, gate, states, norms,
+                                                                    T, N, C); }
     if (int rc = check_launch()) return rc;
 
     const size_t sm_solve = SolveSmem<D>::bytes(C);
     if ((e = set_smem(k_chunk_solve<Tin, D>, sm_solve)) != cudaSuccess) return cuda_fail(e);
     { ProfScope ps(GKA_KERNEL_CHUNK_SOLVE, s);
     k_chunk_solve<Tin, D><<<dim3(C / kSolveTG, N, BH), kSimtThreads, sm_solve, s>>>(
-        q, k, v, beta, states, norms, o, T, N, C, P); }
+        q, k, v, beta, gate, states, norms, o, T, N, C, P); }
     return check_launch();
 }
 
@@ -236,7 +237,7 @@ static int rows128_map(CUtensorMap *m, const void *base, uint64_t rows, CUtensor
 static int timeout_flag_ptr(int **ptr);
 
 static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
-                      const float *beta, __nv_bfloat16 *o, int B, int H, int T, int C,
+                      const float *beta, const float *gate, __nv_bfloat16 *o, int B, int H, int T, int C,
                       const ChebParams &P, float *final_state, char *ws,
                       const gka_workspace_layout &L, cudaStream_t s) {
     constexpr int D = 128;
@@ -282,13 +283,13 @@ static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
                 return cuda_fail(e);
             ProfScope ps(GKA_KERNEL_STATE_PASS_TC, s);
             k_state_pass_tc<64><<<dim3(2, BH), kStateThreads, StateSmem<64>::bytes, s>>>(
-                smaps, beta, sexp, decay, tokdec, plane, final_state, T, N, flag);
+                smaps, beta, gate, sexp, decay, tokdec, plane, final_state, T, N, flag);
         } else {
             if ((e = set_smem(k_state_pass_tc<128>, StateSmem<128>::bytes)) != cudaSuccess)
                 return cuda_fail(e);
             ProfScope ps(GKA_KERNEL_STATE_PASS_TC, s);
             k_state_pass_tc<128><<<dim3(2, BH), kStateThreads, StateSmem<128>::bytes, s>>>(
-                smaps, beta, sexp, decay, tokdec, plane, final_state, T, N, flag);
+                smaps, beta, gate, sexp, decay, tokdec, plane, final_state, T, N, flag);
         }
         if (int rc = check_launch()) return rc;
     } else {
@@ -297,13 +298,13 @@ static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
                 return cuda_fail(e);
             ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
             k_chunk_delta_tc<64><<<dim3(N, BH), kTcThreads, DeltaSmem<64>::bytes, s>>>(
-                dmaps, beta, states, decay, bound_inc, tokdec, plane, T, N, flag);
+                dmaps, beta, gate, states, decay, bound_inc, tokdec, plane, T, N, flag);
         } else {
             if ((e = set_smem(k_chunk_delta_tc<128>, DeltaSmem<128>::bytes)) != cudaSuccess)
                 return cuda_fail(e);
             ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
             k_chunk_delta_tc<128><<<dim3(N, BH), kTcThreads, DeltaSmem<128>::bytes, s>>>(
-                dmaps, beta, states, decay, bound_inc, tokdec, plane, T, N, flag);
+                dmaps, beta, gate, states, decay, bound_inc, tokdec, plane, T, N, flag);
         }
         if (int rc = check_launch()) return rc;
 
@@ -320,14 +321,14 @@ static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
         if ((e = set_smem(kern, TcSmem<64, 64>::bytes)) != cudaSuccess) return cuda_fail(e);
         ProfScope ps(GKA_KERNEL_CHUNK_SOLVE_TC, s);
         kern<<<dim3(N, BH), kSolveThreads, TcSmem<64, 64>::bytes, s>>>(
-            maps, q, tokdec, plane, norms, sexp, o, T, N, C, P, flag);
+            maps, q, gate, tokdec, plane, norms, sexp, o, T, N, C, P, flag);
     } else {
         // one CTA per 128-token chunk (N = 128 MMAs)
         auto kern = k_chunk_solve_tc<128, 128>;
         if ((e = set_smem(kern, TcSmem<128, 128>::bytes)) != cudaSuccess) return cuda_fail(e);
         ProfScope ps(GKA_KERNEL_CHUNK_SOLVE_TC, s);
         kern<<<dim3(N, BH), kSolveThreads, TcSmem<128, 128>::bytes, s>>>(
-            maps, q, tokdec, plane, norms, sexp, o, T, N, C, P, flag);
+            maps, q, gate, tokdec, plane, norms, sexp, o, T, N, C, P, flag);
     }
     if (int rc = check_launch()) return rc;
     return GKA_OK;
@@ -335,7 +336,7 @@ static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
 
 template <typename Tin>
 static int forward_dispatch(const void *q, const void *k, const void *v, const float *beta,
-                            void *o, int B, int H, int T, int D, int C, const ChebParams &P,
+                            const float *gate, void *o, int B, int H, int T, int D, int C, const ChebParams &P,
                             float *final_state, char *ws, const gka_workspace_layout &L,
                             cudaStream_t s) {
     auto Q = static_cast<const Tin *>(q);
@@ -344,12 +345,12 @@ static int forward_dispatch(const void *q, const void *k, const void *v, const f
     auto O = static_cast<Tin *>(o);
     if constexpr (std::is_same<Tin, __nv_bfloat16>::value) {
         if (tensor_core_path(D, C, GKA_BF16))
-            return forward_tc(Q, K, V, beta, O, B, H, T, C, P, final_state, ws, L, s);
+            return forward_tc(Q, K, V, beta, gate, O, B, H, T, C, P, final_state, ws, L, s);
     }
     switch (D) {
-        case 32: return forward_simt<Tin, 32>(Q, K, V, beta, O, B, H, T, C, P, final_state, ws, L, s);
-        case 64: return forward_simt<Tin, 64>(Q, K, V, beta, O, B, H, T, C, P, final_state, ws, L, s);
-        default: return forward_simt<Tin, 128>(Q, K, V, beta, O, B, H, T, C, P, final_state, ws, L, s);
+        case 32: return forward_simt<Tin, 32>(Q, K, V, beta, gate, O, B, H, T, C, P, final_state, ws, L, s);
+        case 64: return forward_simt<Tin, 64>(Q, K, V, beta, gate, O, B, H, T, C, P, final_state, ws, L, s);
+        default: return forward_simt<Tin, 128>(Q, K, V, beta, gate, O, B, H, T, C, P, final_state, ws, L, s);
     }
 }
 
@@ -360,7 +361,7 @@ static int timeout_flag_ptr(int **ptr) {
 
 template <typename Tin, int D>
 static int decode_launch(float *state, const void *q, const void *k, const void *v,
-                         const float *beta, void *o, int BH, const ChebParams &P, cudaStream_t s) {
+                         const float *beta, const float *gate, void *o, int BH, const ChebParams &P, cudaStream_t s) {
     int *flag = nullptr;
     if (int rc = timeout_flag_ptr(&flag)) return rc;
     const size_t smem = sizeof(float) * D * D;
@@ -369,14 +370,14 @@ static int decode_launch(float *state, const void *q, const void *k, const void 
     ProfScope ps(GKA_KERNEL_DECODE_STEP, s);
     k_decode_step<Tin, D><<<BH, 4 * D, smem, s>>>(
         state, static_cast<const Tin *>(q), static_cast<const Tin *>(k),
-        static_cast<const Tin *>(v), beta, static_cast<Tin *>(o), P, flag);
+        static_cast<const Tin *>(v), beta, gate, static_cast<Tin *>(o), P, flag);
     return check_launch();
 }
 
 
 template <typename Tin>
 static int decode_rows_launch(float *state, const void *q, const void *k, const void *v,
-                              const float *beta, void *o, int BH, const ChebParams &P,
+                              const float *beta, const float *gate, void *o, int BH, const ChebParams &P,
                               cudaStream_t s) {
     int *flag = nullptr;
     if (int rc = timeout_flag_ptr(&flag)) return rc;
@@ -389,19 +390,19 @@ static int decode_rows_launch(float *state, const void *q, const void *k, const 
     ProfScope ps(GKA_KERNEL_DECODE_STEP, s);
     k_decode_rows<Tin><<<BH, kDecRowThreads, kDecRowSmem, s>>>(
         maps, static_cast<const Tin *>(q), static_cast<const Tin *>(k),
-        static_cast<const Tin *>(v), beta, static_cast<Tin *>(o), P, flag);
+        static_cast<const Tin *>(v), beta, gate, static_cast<Tin *>(o), P, flag);
     return check_launch();
 }
 
 template <typename Tin>
 static int decode_dispatch(float *state, const void *q, const void *k, const void *v,
-                           const float *beta, void *o, int BH, int D, const ChebParams &P,
+                           const float *beta, const float *gate, void *o, int BH, int D, const ChebParams &P,
                            cudaStream_t s) {
-    if (D == 128) return decode_rows_launch<Tin>(state, q, k, v, beta, o, BH, P, s);
+    if (D == 128) return decode_rows_launch<Tin>(state, q, k, v, beta, gate, o, BH, P, s);
     switch (D) {
-        case 32: return decode_launch<Tin, 32>(state, q, k, v, beta, o, BH, P, s);
-        case 64: return decode_launch<Tin, 64>(state, q, k, v, beta, o, BH, P, s);
-        default: return decode_launch<Tin, 128>(state, q, k, v, beta, o, BH, P, s);
+        case 32: return decode_launch<Tin, 32>(state, q, k, v, beta, gate, o, BH, P, s);
+        case 64: return decode_launch<Tin, 64>(state, q, k, v, beta, gate, o, BH, P, s);
+        default: return decode_launch<Tin, 128>(state, q, k, v, beta, gate, o, BH, P, s);
     }
 }
 
@@ -468,6 +469,14 @@ int gka_forward_workspace_layout(int B, int H, int T, int D, int chunk, gka_dtyp
 int gka_forward(const void *q, const void *k, const void *v, const float *beta, void *o, int B,
                 int H, int T, int D, gka_dtype dt, float a, int r, int chunk, float *final_state,
                 void *workspace, size_t workspace_bytes, void *stream) {
+    return gka_forward_gated(q, k, v, beta, nullptr, o, B, H, T, D, dt, a, r, chunk, final_state,
+                             workspace, workspace_bytes, stream);
+}
+
+int gka_forward_gated(const void *q, const void *k, const void *v, const float *beta,
+                      const float *gate, void *o, int B, int H, int T, int D, gka_dtype dt,
+                      float a, int r, int chunk, float *final_state, void *workspace,
+                      size_t workspace_bytes, void *stream) {
     gka_workspace_layout L;
     if (int rc = layout(B, H, T, D, chunk, dt, &L)) return rc;
     if (!(a > 0.f) || !isfinite(a) || r < 1) return GKA_ERR_INVALID_ARG;
@@ -485,15 +494,17 @@ int gka_forward(const void *q, const void *k, const void *v, const float *beta, 
     }
     if (!q || !k || !v || !beta || !o || !workspace) return GKA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(beta) || !aligned16(o) ||
-        (final_state && !aligned16(final_state)) || ((uintptr_t)workspace & 255u))
+        (gate && !aligned16(gate)) || (final_state && !aligned16(final_state)) ||
+        ((uintptr_t)workspace & 255u))
         return GKA_ERR_MISALIGNED;
     if (workspace_bytes < L.total_bytes) return GKA_ERR_WORKSPACE_TOO_SMALL;
     const ChebParams P = make_cheb(a, r);
     char *ws = static_cast<char *>(workspace);
     if (dt == GKA_BF16)
-        return forward_dispatch<__nv_bfloat16>(q, k, v, beta, o, B, H, T, D, chunk, P,
+        return forward_dispatch<__nv_bfloat16>(q, k, v, beta, gate, o, B, H, T, D, chunk, P,
                                                final_state, ws, L, s);
-    return forward_dispatch<float>(q, k, v, beta, o, B, H, T, D, chunk, P, final_state, ws, L, s);
+    return forward_dispatch<float>(q, k, v, beta, gate, o, B, H, T, D, chunk, P, final_state, ws,
+                                   L, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -665,6 +676,12 @@ int gka_forward_static_scratch(const void *q, const void *k, const void *v, cons
 
 int gka_decode_step(float *state, const void *q, const void *k, const void *v, const float *beta,
                     void *o, int B, int H, int D, gka_dtype dt, float a, int r, void *stream) {
+    return gka_decode_step_gated(state, q, k, v, beta, nullptr, o, B, H, D, dt, a, r, stream);
+}
+
+int gka_decode_step_gated(float *state, const void *q, const void *k, const void *v,
+                          const float *beta, const float *gate, void *o, int B, int H, int D,
+                          gka_dtype dt, float a, int r, void *stream) {
     if (B < 0 || H < 0) return GKA_ERR_INVALID_ARG;
     if (dt != GKA_F32 && dt != GKA_BF16) return GKA_ERR_INVALID_ARG;
     if (!supported_d(D)) return GKA_ERR_UNSUPPORTED;
@@ -675,12 +692,13 @@ int gka_decode_step(float *state, const void *q, const void *k, const void *v, c
     if (BH > 0x7fffffffu) return GKA_ERR_UNSUPPORTED;
     if (!state || !q || !k || !v || !beta || !o) return GKA_ERR_INVALID_ARG;
     if (!aligned16(state) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(beta) ||
-        !aligned16(o))
+        !aligned16(o) || (gate && !aligned16(gate)))
         return GKA_ERR_MISALIGNED;
     const ChebParams P = make_cheb(a, r);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (dt == GKA_BF16) return decode_dispatch<__nv_bfloat16>(state, q, k, v, beta, o, (int)BH, D, P, s);
-    return decode_dispatch<float>(state, q, k, v, beta, o, (int)BH, D, P, s);
+    if (dt == GKA_BF16)
+        return decode_dispatch<__nv_bfloat16>(state, q, k, v, beta, gate, o, (int)BH, D, P, s);
+    return decode_dispatch<float>(state, q, k, v, beta, gate, o, (int)BH, D, P, s);
 }
 
 int gka_selftest_timeout(void *stream) {

@@ -179,6 +179,56 @@ __device__ __forceinline__ float tile_bf16_to_f16_scaled(uint8_t *tile, float *r
     return sc;
 }
 
+// The same conversion for a tile of two 64-column halves of ROWS rows each
+// (TMA box layout: the 16-byte piece at byte offset o belongs to row
+// (o mod ROWS*128) / 128), with row r first multiplied by sqrt(g[r]) (g: the
+// write gates of the tile's tokens; nullptr: the plain conversion above).
+template <int BYTES, int NTHR, int ROWS>
+__device__ __forceinline__ float tile_bf16_to_f16_rows_scaled(uint8_t *tile, float *red,
+                                                              const float *__restrict__ g) {
+    if (g == nullptr) return tile_bf16_to_f16_scaled<BYTES, NTHR>(tile, red);
+    constexpr int PER = BYTES / (NTHR * 16);
+    static_assert(BYTES % (NTHR * 16) == 0 && BYTES == 2 * ROWS * 128, "tile size");
+    const int tid = threadIdx.x, nw = NTHR >> 5;
+    float rs[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) rs[i] = sqrtf(__ldg(g + (((i * NTHR + tid) % (ROWS * 8)) >> 3)));
+    uint4 u[PER];
+    float mx = 0.f;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        u[i] = *reinterpret_cast<const uint4 *>(tile + (i * NTHR + tid) * 16);
+        const uint32_t w4[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
+        float m = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            m = fmaxf(m, fmaxf(fabsf(__uint_as_float(w4[e] << 16)),
+                               fabsf(__uint_as_float(w4[e] & 0xffff0000u))));
+        mx = fmaxf(mx, m * rs[i]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    __syncthreads();
+    if ((tid & 31) == 0) red[tid >> 5] = mx;
+    __syncthreads();
+    mx = 0.f;
+    for (int w = 0; w < nw; ++w) mx = fmaxf(mx, red[w]);
+    const float sc = inv_pow2_above(mx);
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const uint32_t w4[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
+        const float f = rs[i] * sc;
+        uint32_t o4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            o4[e] = pack_f16(__uint_as_float(w4[e] << 16) * f,
+                             __uint_as_float(w4[e] & 0xffff0000u) * f);
+        *reinterpret_cast<uint4 *>(tile + (i * NTHR + tid) * 16) =
+            make_uint4(o4[0], o4[1], o4[2], o4[3]);
+    }
+    return sc;
+}
+
 // Writes 8 consecutive values (columns c0..c0+7, c0 % 8 == 0) of `row` of a
 // 128B-swizzled [rows][64] fp16 tile as one 16-byte chunk.
 __device__ __forceinline__ void st_row8(uint32_t tile, uint32_t row, uint32_t c0, const float *v) {
@@ -222,7 +272,7 @@ __device__ __forceinline__ void reduce_scatter32(float (&v)[N], int lane) {
 template <int MG, int TOK>
 __global__ void __launch_bounds__(kSolveThreads, TOK == 64 ? 2 : 1)
 k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__restrict__ q,
-                 const float *__restrict__ tokdec, size_t plane, float *__restrict__ norms,
+                 const float *__restrict__ gate, const float *__restrict__ tokdec, size_t plane, float *__restrict__ norms,
                  const int *__restrict__ state_exp, __nv_bfloat16 *__restrict__ o, int T, int N,
                  int C, const ChebParams P, int *__restrict__ timeout_flag) {
     using L = TcSmem<MG, TOK>;
@@ -291,8 +341,11 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     const int eMexp = state_exp[((size_t)bh * N + n) * 2 + 1];
     bool ok = mbar_wait_sleep(bar_load, 0, kTcSleepProbes, kTcSleepNs);
     // keys: bf16 -> fp16 in place, scaled below 1 (the values follow while the norm
-    // products run)
-    const float sK = tile_bf16_to_f16_scaled<MG * 256, kSolveThreads>(sm + L::KT, red);
+    // products run); with the write gate, key and value rows of token i are taken
+    // times sqrt(g_i), which puts g_i into every product that pairs them
+    const float *gate_rows = gate ? gate + tok0 : nullptr;
+    const float sK = tile_bf16_to_f16_rows_scaled<MG * 256, kSolveThreads, MG>(sm + L::KT, red,
+                                                                               gate_rows);
     const __nv_bfloat16 *qs = reinterpret_cast<const __nv_bfloat16 *>(sm + L::QS);
     fence_proxy_async_smem();
     tc::fence_before_sync();
@@ -339,7 +392,8 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     }
     // values: bf16 -> fp16 in place, scaled below 1 (first read by the readout)
     ok = mbar_wait_sleep(bar_v, 0, kTcSleepProbes, kTcSleepNs) && ok;
-    const float sV = tile_bf16_to_f16_scaled<MG * 256, kSolveThreads>(sm + L::VT, red);
+    const float sV = tile_bf16_to_f16_rows_scaled<MG * 256, kSolveThreads, MG>(sm + L::VT, red,
+                                                                               gate_rows);
     float *s_u = reinterpret_cast<float *>(sm + L::NRM);
     float *s_E = s_u + MG, *s_X = s_E + MG, *s_G = s_X + MG;   // [MG] each; E and X: wg 0 part
     float *s_E1 = reinterpret_cast<float *>(sm + L::NRM2), *s_X1 = s_E1 + MG;   // wg 1 part

@@ -4,8 +4,10 @@
 // Method: "Gated KalmaNet" (arXiv 2511.21016), ai.info page, Methodology:
 // only the chunk-start states are carried across chunks,
 //   S_0 = 0,   S_{n+1} = b_n S_n + dS_n,
-//   dH_n = K^T diag(w) K,   dM_n = V^T diag(w) K,   w_i = prod_{m > i} beta_m,
-// with b_n = prod_m beta_m over chunk n (the exp of the chunk's summed log decay).
+//   dH_n = K^T diag(w) K,   dM_n = V^T diag(w) K,   w_i = g_i prod_{m > i} beta_m,
+// with b_n = prod_m beta_m over chunk n (the exp of the chunk's summed log decay)
+// and g_i the write gate of token i (the paper's beta_t-augmented variant,
+// ai.info page, Main Findings; `gate` nullable, NULL = 1).
 //
 // One CTA per (head, matrix): blockIdx.x = 0 carries H, 1 carries M.  The
 // fp32 state lives in registers for the whole sequence (arithmetic thread
@@ -71,7 +73,8 @@ struct StateSmem {
     // has just prepared (free until that stage is loaded again)
     static constexpr uint32_t OUT = C == 64 ? PARTS + NPB * NP * TILE : 0;
     static constexpr uint32_t BETA = C == 64 ? OUT + 32768 : PARTS + NPB * NP * TILE;  // [2][C]
-    static constexpr uint32_t W = BETA + 2 * 4 * C;         // [2][C] w of the chunks in flight
+    static constexpr uint32_t GATE = BETA + 2 * 4 * C;      // [2][C] write gates
+    static constexpr uint32_t W = GATE + 2 * 4 * C;         // [2][C] w of the chunks in flight
     static constexpr uint32_t BN = W + 2 * 4 * C;           // [2] chunk decays (16 bytes)
     static constexpr uint32_t RED = BN + 16;                // [2][16] partial bound increments
     static constexpr uint32_t BARS = RED + 128;             // load[2] mma[2] fin w[2] out
@@ -101,7 +104,7 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
 template <int C>
 __global__ void __launch_bounds__(kStateThreads, 1)
 k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict__ beta,
-                int *__restrict__ state_exp, float *__restrict__ decay,
+                const float *__restrict__ gate, int *__restrict__ state_exp, float *__restrict__ decay,
                 float *__restrict__ tokdec, size_t plane, float *__restrict__ final_state,
                 int T, int N, int *__restrict__ timeout_flag) {
     using L = StateSmem<C>;
@@ -122,6 +125,7 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
     const bool is_m = m == 1;
     const size_t tokbase = (size_t)bh * T;
     float *s_beta = reinterpret_cast<float *>(sm + L::BETA);   // [2][C]
+    float *s_gate = reinterpret_cast<float *>(sm + L::GATE);   // [2][C], with a gate
     float *s_w = reinterpret_cast<float *>(sm + L::W);         // [2][C]
     float *s_bn = reinterpret_cast<float *>(sm + L::BN);       // [2]
     float *s_red = reinterpret_cast<float *>(sm + L::RED);     // [2][16]
@@ -142,11 +146,11 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
     __syncthreads();
 
     int last_load[2] = {-1, -1};   // issuer: chunk last loaded into each stage
-    // issuer: chunk c (keys, values for M, beta) into stage c & 1
+    // issuer: chunk c (keys, values for M, beta, gates) into stage c & 1
     auto issue_load = [&](int c) {
         const int st = c & 1;
         uint64_t *bar = &bar_load[st];
-        mbar_arrive_expect_tx(bar, TILE * (is_m ? 2u : 1u) + 4u * C);
+        mbar_arrive_expect_tx(bar, TILE * (is_m ? 2u : 1u) + (gate ? 8u : 4u) * C);
         const int row0 = (int)(tokbase + (size_t)c * C);
         for (int h = 0; h < 2; ++h)
             for (int rb = 0; rb < C / 64; ++rb) {
@@ -155,6 +159,7 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
                 if (is_m) tc::tma_load_2d(sm + L::VS + o, &maps.v, h * 64, row0 + rb * 64, bar);
             }
         bulk_g2s(s_beta + st * C, beta + tokbase + (size_t)c * C, 4 * C, bar);
+        if (gate) bulk_g2s(s_gate + st * C, gate + tokbase + (size_t)c * C, 4 * C, bar);
         last_load[st] = c;
     };
     // issuer: dS_c = A^T (w K) into TMEM buffer c & 1 (A = K or V of stage c & 1)
@@ -184,7 +189,7 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
     const uint32_t tmem = *tbase;
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(cg * 32);
 
-    // Decay warp: chunk c's decays w_t = prod_{m>t} beta_m (suffix products;
+    // Decay warp: chunk c's weights w_t = g_t prod_{m>t} beta_m (suffix products;
     // lane l holds tokens l*PER..) into s_w[c & 1], b_c into s_bn[c & 1], then
     // every lane arrives on bar_w[c & 1].
     auto decays = [&](int c) {
@@ -207,7 +212,11 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
         float above = __shfl_down_sync(0xffffffffu, tot, 1);   // lanes > this lane
         if (lane == 31) above = 1.f;
 #pragma unroll
-        for (int p = 0; p < PER; ++p) s_w[(c & 1) * C + lane * PER + p] = sfx[p] * above;
+        for (int p = 0; p < PER; ++p) {
+            float w = sfx[p] * above;
+            if (gate) w *= s_gate[(c & 1) * C + lane * PER + p];
+            s_w[(c & 1) * C + lane * PER + p] = w;
+        }
         if (lane == 0) s_bn[c & 1] = tot;
         __syncwarp();
         mbar_arrive(&bar_w[c & 1]);

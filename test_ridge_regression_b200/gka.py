@@ -59,6 +59,9 @@ def _lib():
         lib.gka_forward_workspace_layout.restype = i
         lib.gka_forward.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, vp, sz, vp]
         lib.gka_forward.restype = i
+        lib.gka_forward_gated.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, vp,
+                                          sz, vp]
+        lib.gka_forward_gated.restype = i
         lib.gka_forward_static_scratch.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i,
                                                    vp, vp]
         lib.gka_forward_host_workspace_bytes.argtypes = [i, i, i, i, i, i, i]
@@ -69,6 +72,8 @@ def _lib():
         lib.gka_forward_static_scratch.restype = i
         lib.gka_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
         lib.gka_decode_step.restype = i
+        lib.gka_decode_step_gated.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+        lib.gka_decode_step_gated.restype = i
         lib.gka_selftest_timeout.argtypes = [vp]
         lib.gka_selftest_timeout.restype = i
         lib.gka_device_status.argtypes = [vp]
@@ -160,6 +165,34 @@ def gka_forward(q, k, v, beta, a: float, r: int, chunk: int, *, o=None, final_st
     return o
 
 
+def gka_forward_gated(q, k, v, beta, gate, a: float, r: int, chunk: int, *, o=None,
+                      final_state=None, workspace=None, stream=None):
+    """Write-gated forward (see include/gka.h): as gka_forward, with gate [B, H, T]
+    fp32 in [0, 1] scaling each token's write into H and M (None: no gate)."""
+    _dev(q, k, v, beta, gate, o, final_state, workspace)
+    B, H, T, D = q.shape
+    if k.shape != q.shape or v.shape != q.shape or beta.shape != (B, H, T):
+        raise ValueError("shape mismatch")
+    if gate is not None and (gate.shape != (B, H, T) or gate.dtype != torch.float32):
+        raise ValueError("gate must be float32 [B, H, T]")
+    dt = _dtype(q)
+    if k.dtype != q.dtype or v.dtype != q.dtype or beta.dtype != torch.float32:
+        raise TypeError("q, k, v must share a dtype; beta must be float32")
+    if o is None:
+        o = torch.empty_like(v)
+    if final_state is not None and (final_state.dtype != torch.float32 or
+                                    final_state.shape != (B, H, 2, D, D)):
+        raise ValueError("final_state must be float32 [B, H, 2, D, D]")
+    if workspace is None:
+        workspace = alloc_workspace(B, H, T, D, chunk, q.dtype, q.device)
+    rc = _lib().gka_forward_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(gate), _ptr(o),
+                                  B, H, T, D, dt, float(a), int(r), int(chunk), _ptr(final_state),
+                                  _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                  _stream(stream))
+    _check("gka_forward_gated", rc)
+    return o
+
+
 def host_workspace_bytes(B, H, T, D, chunk, dtype=torch.bfloat16, slice_pairs=0) -> int:
     return int(_lib().gka_forward_host_workspace_bytes(B, H, T, D, chunk, _DT[dtype], slice_pairs))
 
@@ -236,6 +269,28 @@ def gka_decode_step(state, q, k, v, beta, a: float, r: int, *, o=None, stream=No
     rc = _lib().gka_decode_step(_ptr(state), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(o),
                                 B, H, D, dt, float(a), int(r), _stream(stream))
     _check("gka_decode_step", rc)
+    return o
+
+
+def gka_decode_step_gated(state, q, k, v, beta, gate, a: float, r: int, *, o=None,
+                          stream=None):
+    """Write-gated decode step in place on state [B, H, 2, D, D] fp32; gate [B, H]
+    fp32 in [0, 1] (None: no gate).  Returns o [B, H, D]."""
+    _dev(state, q, k, v, beta, gate, o)
+    B, H, D = q.shape
+    if state.dtype != torch.float32 or state.shape != (B, H, 2, D, D):
+        raise ValueError("state must be float32 [B, H, 2, D, D]")
+    if k.shape != q.shape or v.shape != q.shape or beta.shape != (B, H):
+        raise ValueError("shape mismatch")
+    if gate is not None and (gate.shape != (B, H) or gate.dtype != torch.float32):
+        raise ValueError("gate must be float32 [B, H]")
+    dt = _dtype(q)
+    if o is None:
+        o = torch.empty_like(v)
+    rc = _lib().gka_decode_step_gated(_ptr(state), _ptr(q), _ptr(k), _ptr(v), _ptr(beta),
+                                      _ptr(gate), _ptr(o), B, H, D, dt, float(a), int(r),
+                                      _stream(stream))
+    _check("gka_decode_step_gated", rc)
     return o
 
 

@@ -27,7 +27,8 @@ def declared_functions():
 
 def test_header_declares_entry_points():
     names = declared_functions()
-    for must in ["gka_forward", "gka_decode_step", "gka_forward_workspace_bytes",
+    for must in ["gka_forward", "gka_decode_step", "gka_forward_gated", "gka_decode_step_gated",
+                 "gka_forward_workspace_bytes",
                  "gka_forward_workspace_layout", "gka_device_status", "gka_last_cuda_error",
                  "gka_status_string", "gka_version"]:
         assert must in names
@@ -99,6 +100,23 @@ def test_decode_argument_errors(lib):
     assert dec(state=None) == -1
     assert dec(state=FAKE_MIS) == -7
     assert dec(B=0) == 0
+
+
+def test_gated_entry_points_validate_like_the_ungated_ones(lib):
+    def fwdg(gate=None, T=128, D=64, r=4):
+        return lib.gka_forward_gated(FAKE, FAKE, FAKE, FAKE, gate, FAKE, 1, 1, T, D, 0, 0.5, r,
+                                     64, None, FAKE, 1 << 40, None)
+    assert fwdg(T=100) == -3
+    assert fwdg(D=48) == -2
+    assert fwdg(r=0) == -1
+    assert fwdg(gate=FAKE_MIS) == -7             # the gate must be 16-byte aligned too
+
+    def decg(gate=None, D=128, r=20):
+        return lib.gka_decode_step_gated(FAKE, FAKE, FAKE, FAKE, FAKE, gate, FAKE, 2, 2, D, 1,
+                                         0.5, r, None)
+    assert decg(D=96) == -2
+    assert decg(r=0) == -1
+    assert decg(gate=FAKE_MIS) == -7
 
 
 def test_binding_raises_without_cuda_tensors():
