@@ -76,3 +76,13 @@ def test_host_forward_twice_with_one_workspace():
     assert torch.equal(o1, o2)
     o_ref, _ = device_reference(q, k, v, beta, 0.5, 6, 64)
     assert torch.equal(o1, o_ref)
+
+
+def test_host_forward_default_schedule_64_pairs():
+    # the default schedule at 64 pairs is 24, 24, 16: two slices take the one-pass state
+    # kernel, the last the two-pass states, against one device call (one pass)
+    q, k, v, beta = make_inputs(8, 8, 128, 128, torch.bfloat16, 3.0, 1.0, seed=1204)
+    o_ref, fs_ref = device_reference(q, k, v, beta, 0.5, 10, 64)
+    o, fs = host_run(q, k, v, beta, 0.5, 10, 64, 0)
+    assert head_rel_err(o.float(), o_ref.float()) <= 5e-3
+    assert head_rel_err(fs, fs_ref) <= 1e-5
