@@ -8,6 +8,7 @@ Parity status: every function is pinned by ``tests/test_oracle_pins.py``
 (closed forms, the exact ridge solve, the page's rate table, invariances).
 """
 from .oracle import (  # noqa: F401
+    backward,
     build,
     cheb_solve,
     chunked_norms,

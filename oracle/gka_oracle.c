@@ -319,3 +319,138 @@ int gka_oracle_max_threads(void)
     return 1;
 #endif
 }
+
+/*
+ * Backward pass by implicit differentiation (ai.info page, Key Contributions
+ * 3 and Methodology: the backward treats x_t as the solution of the linear
+ * system that the Chebyshev iteration approximately solves and reuses the
+ * iteration on the upstream gradient; Main Findings: Lemma 2, dq_t = dq^_t;
+ * pith.science appendix, Eq. 50, the key gradient with its ||H_t||_F term).
+ *
+ * With g_o = dL/do_t (the upstream gradient), x_t the forward iterate and
+ * A_t = H_t + a ||H_t||_F I:
+ *   u_t = M_t^T g_o                 (dL/dx_t)
+ *   y_t = r-step Chebyshev for A_t y = u_t   (the same iteration as the forward)
+ *   dq_t = y_t
+ *   dL/dH_t = -y_t x_t^T - c_t H_t,  c_t = a (y_t . x_t) / ||H_t||_F
+ *     (from dx = -A^-1 dA x and d||H||_F = <H, dH> / ||H||_F)
+ *   dL/dM_t = g_o x_t^T
+ * then back through H_t = beta_t H_{t-1} + g_t k_t k_t^T (and M) with the
+ * adjoint states  Hb_t = dL/dH_t + beta_{t+1} Hb_{t+1},  Mb_t likewise:
+ *   dk_t = g_t ((Hb_t + Hb_t^T) k_t + Mb_t^T v_t),   dv_t = g_t Mb_t k_t,
+ *   dbeta_t = <Hb_t, H_{t-1}> + <Mb_t, M_{t-1}>,
+ *   dg_t = k_t^T Hb_t k_t + v_t^T Mb_t k_t       (the write gate g, if any).
+ * A token with ||H_t||_F = 0 has x_t = 0 and contributes nothing.
+ *
+ * Inputs as for gka_oracle_forward plus dout [B, Hh, T, D]; outputs dq, dk,
+ * dv [B, Hh, T, D], dbeta [B, Hh, T] and, when gate is given, dgate
+ * [B, Hh, T] (nullable).  Keeps every H_t and M_t of a head in memory
+ * (T * 2 * D * D doubles per thread): meant for test sizes.
+ * Returns 0, -1 on bad arguments, -2 if memory runs out.
+ */
+int gka_oracle_backward(const double *q, const double *k, const double *v,
+                        const double *beta, const double *gate, const double *dout,
+                        int B, int Hh, int T, int D, double a, int r,
+                        double *dq, double *dk, double *dv, double *dbeta,
+                        double *dgate, int nthreads)
+{
+    if (B < 0 || Hh < 0 || T < 0 || D <= 0 || r < 1 || !(a > 0.0)) return -1;
+    long nh = (long)B * Hh;
+    size_t DD = (size_t)D * D;
+    int fail = 0;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (long h = 0; h < nh; ++h) {
+        /* S[t] = (H_t, M_t) for t = 0..T-1, plus the zero state at index -1 */
+        double *S = (double *)calloc((size_t)(T + 1) * 2 * DD, sizeof(double));
+        double *X = (double *)malloc(sizeof(double) * ((size_t)T * D + 1));
+        double *Y = (double *)malloc(sizeof(double) * ((size_t)T * D + 1));
+        double *cn = (double *)malloc(sizeof(double) * ((size_t)T + 1));
+        double *work = (double *)malloc(sizeof(double) * (DD + 4 * (size_t)D));
+        double *A = (double *)malloc(sizeof(double) * DD);
+        double *u = (double *)malloc(sizeof(double) * D);
+        double *o = (double *)malloc(sizeof(double) * D);
+        double *Hb = (double *)calloc(2 * DD, sizeof(double));
+        if (!S || !X || !Y || !cn || !work || !A || !u || !o || !Hb) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+            fail = 1;
+            free(S); free(X); free(Y); free(cn); free(work); free(A); free(u); free(o); free(Hb);
+            continue;
+        }
+        double *Mb = Hb + DD;
+        const double *bt = beta + (size_t)h * T;
+        const double *gt = gate ? gate + (size_t)h * T : NULL;
+        /* forward sweep: states, iterates x_t, adjoint solves y_t */
+        for (int t = 0; t < T; ++t) {
+            double *Ht = S + (size_t)(t + 1) * 2 * DD, *Mt = Ht + DD;
+            memcpy(Ht, S + (size_t)t * 2 * DD, sizeof(double) * 2 * DD);
+            size_t row = ((size_t)h * T + t) * D;
+            double n = gka_token(Ht, Mt, q + row, k + row, v + row, bt[t], gt ? gt[t] : 1.0,
+                                 D, a, r, 1, o, work);
+            double *xt = X + (size_t)t * D, *yt = Y + (size_t)t * D;
+            if (n == 0.0) {
+                for (int i = 0; i < D; ++i) xt[i] = yt[i] = 0.0;
+                cn[t] = 0.0;
+                continue;
+            }
+            /* gka_token left the forward iterate at work + D*D */
+            memcpy(xt, work + DD, sizeof(double) * D);
+            const double *g = dout + row;
+            for (int j = 0; j < D; ++j) {
+                double s = 0.0;
+                for (int i = 0; i < D; ++i) s += Mt[(size_t)i * D + j] * g[i];
+                u[j] = s;
+            }
+            memcpy(A, Ht, sizeof(double) * DD);
+            for (int i = 0; i < D; ++i) A[(size_t)i * D + i] += a * n;
+            gka_oracle_cheb_solve(A, u, D, a * n, (1.0 + a) * n, r, yt, work);
+            double yx = 0.0;
+            for (int i = 0; i < D; ++i) yx += yt[i] * xt[i];
+            cn[t] = a * yx / n;
+        }
+        /* reverse sweep over the adjoint states */
+        for (int t = T - 1; t >= 0; --t) {
+            const double *Ht = S + (size_t)(t + 1) * 2 * DD, *Mt = Ht + DD;
+            const double *Hp = S + (size_t)t * 2 * DD, *Mp = Hp + DD;
+            const double bnext = (t + 1 < T) ? bt[t + 1] : 0.0;
+            const double *xt = X + (size_t)t * D, *yt = Y + (size_t)t * D;
+            size_t row = ((size_t)h * T + t) * D;
+            const double *g = dout + row;
+            for (int i = 0; i < D; ++i)
+                for (int j = 0; j < D; ++j) {
+                    size_t e = (size_t)i * D + j;
+                    Hb[e] = bnext * Hb[e] - yt[i] * xt[j] - cn[t] * Ht[e];
+                    Mb[e] = bnext * Mb[e] + g[i] * xt[j];
+                }
+            const double *kt = k + row, *vt = v + row;
+            const double gw = gt ? gt[t] : 1.0;
+            double db = 0.0, dg = 0.0;
+            for (size_t e = 0; e < DD; ++e) db += Hb[e] * Hp[e] + Mb[e] * Mp[e];
+            for (int i = 0; i < D; ++i) {
+                double sk = 0.0, sv = 0.0;
+                for (int j = 0; j < D; ++j) {
+                    sk += (Hb[(size_t)i * D + j] + Hb[(size_t)j * D + i]) * kt[j]
+                          + Mb[(size_t)j * D + i] * vt[j];
+                    sv += Mb[(size_t)i * D + j] * kt[j];
+                }
+                dk[row + i] = gw * sk;
+                dv[row + i] = gw * sv;
+                double hk = 0.0, mk = 0.0;
+                for (int j = 0; j < D; ++j) {
+                    hk += Hb[(size_t)i * D + j] * kt[j];
+                    mk += Mb[(size_t)i * D + j] * kt[j];
+                }
+                dg += kt[i] * hk + vt[i] * mk;
+                dq[row + i] = yt[i];
+            }
+            dbeta[(size_t)h * T + t] = db;
+            if (dgate) dgate[(size_t)h * T + t] = dg;
+        }
+        free(S); free(X); free(Y); free(cn); free(work); free(A); free(u); free(o); free(Hb);
+    }
+    return fail ? -2 : 0;
+}

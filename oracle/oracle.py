@@ -55,6 +55,9 @@ def _load():
         lib.gka_oracle_decode_step.restype = i
         lib.gka_oracle_chunked_norms.argtypes = [_dp, _dp, _dp, i, i, i, i, i, _dp, i]
         lib.gka_oracle_chunked_norms.restype = i
+        lib.gka_oracle_backward.argtypes = [_dp, _dp, _dp, _dp, _dp, _dp, i, i, i, i, d, i,
+                                            _dp, _dp, _dp, _dp, _dp, i]
+        lib.gka_oracle_backward.restype = i
         lib.gka_oracle_max_threads.argtypes = []
         lib.gka_oracle_max_threads.restype = i
         _lib = lib
@@ -171,4 +174,27 @@ def chunked_norms(k, beta, chunk: int, nthreads: int = 0, gate=None) -> np.ndarr
                                           _ptr(out), int(nthreads))
     if rc != 0:
         raise ValueError("gka_oracle_chunked_norms: bad arguments")
+    return out
+
+
+def backward(q, k, v, beta, dout, a: float, r: int, *, gate=None, nthreads: int = 0):
+    """Implicit-differentiation backward of the layer (see the C file).  q, k, v,
+    dout: [B, H, T, D]; beta (and the optional gate): [B, H, T].  Returns a dict
+    with dq, dk, dv [B, H, T, D], dbeta [B, H, T] and, with a gate, dgate [B, H, T]."""
+    q, k, v, beta, dout = _f64(q), _f64(k), _f64(v), _f64(beta), _f64(dout)
+    B, H, T, D = q.shape
+    assert k.shape == q.shape and v.shape == q.shape and dout.shape == q.shape
+    assert beta.shape == (B, H, T)
+    g = _gate(gate, (B, H, T))
+    out = {n: np.zeros((B, H, T, D)) for n in ("dq", "dk", "dv")}
+    out["dbeta"] = np.zeros((B, H, T))
+    dg = np.zeros((B, H, T)) if g is not None else None
+    rc = _load().gka_oracle_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(dout),
+                                     B, H, T, D, float(a), int(r), _ptr(out["dq"]),
+                                     _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dbeta"]),
+                                     _ptr(dg), int(nthreads))
+    if rc != 0:
+        raise ValueError(f"gka_oracle_backward failed ({rc})")
+    if dg is not None:
+        out["dgate"] = dg
     return out
