@@ -221,6 +221,38 @@ int gka_decode_step_gated(float *state, const void *q, const void *k, const void
                           const float *beta, const float *gate, void *o, int B, int H, int D,
                           gka_dtype dt, float a, int r, void *stream);
 
+/*
+ * Backward pass of gka_forward / gka_forward_gated by implicit
+ * differentiation (ai.info page, Key Contributions 3 and Methodology: the
+ * backward differentiates through the linear system that the Chebyshev
+ * iteration approximately solves and reuses the iteration on the upstream
+ * gradient; Main Findings: Lemma 2, dq_t = dq^_t, and the full intra-chunk
+ * interaction of the backward; pith.science appendix, Eq. 50).  With x_t the
+ * forward's r-step iterate, g_t = dL/do_t and A_t = H_t + a ||H_t||_F I:
+ *   y_t = r-step Chebyshev for A_t y = M_t^T g_t,   dq_t = y_t,
+ *   dL/dH_t = -y_t x_t^T - a (y_t . x_t) / ||H_t||_F H_t,   dL/dM_t = g_t x_t^T,
+ * carried back through the decayed, write-gated recurrence to dk, dv, dbeta
+ * and dgate.  It recomputes the forward quantities it needs (chunk states,
+ * norms, iterates) itself; every step runs on CUDA cores in fp32.
+ *   q, k, v, beta, gate  the forward's inputs (gate nullable)
+ *   dout        [B, H, T, D] in `dt`: dL/do
+ *   dq, dk, dv  [B, H, T, D] in `dt` (written)
+ *   dbeta       [B, H, T] fp32 (written)
+ *   dgate       [B, H, T] fp32 (written); non-NULL exactly when gate is
+ *   chunk       16 or 32 (the backward's own chunking; the result does not
+ *               depend on it beyond rounding); T must be a multiple of it
+ *   workspace   at least gka_backward_workspace_bytes(), 256-byte aligned
+ * A token whose H_t is zero (zero keys) has x_t = 0 and passes no gradient.
+ * Errors as for gka_forward; GKA_ERR_UNSUPPORTED for chunk 64 or 128,
+ * GKA_ERR_INVALID_ARG when exactly one of gate and dgate is NULL.
+ */
+size_t gka_backward_workspace_bytes(int B, int H, int T, int D, int chunk, gka_dtype dt);
+int gka_backward(const void *q, const void *k, const void *v, const float *beta,
+                 const float *gate, const void *dout, void *dq, void *dk, void *dv,
+                 float *dbeta, float *dgate, int B, int H, int T, int D, gka_dtype dt,
+                 float a, int r, int chunk, void *workspace, size_t workspace_bytes,
+                 void *stream);
+
 /* Synchronises `stream`, then returns GKA_ERR_DEVICE_TIMEOUT if any kernel of
  * this library on the current device gave up a bounded wait since the last
  * call (and clears the flag), GKA_ERR_CUDA if the stream reports an error,
@@ -253,7 +285,12 @@ enum {
     GKA_KERNEL_DECODE_STEP = 4,   /* recurrent decode step */
     GKA_KERNEL_CHUNK_SOLVE_TC = 5,/* Chebyshev solve + readout on tensor cores (tcgen05) */
     GKA_KERNEL_STATE_PASS_TC = 6, /* chunk-state increments and scan in one pass (tcgen05) */
-    GKA_KERNEL_COUNT = 8
+    GKA_KERNEL_BWD_SOLVE = 7,     /* backward: u = M^T dL/do and the Chebyshev solve for dq */
+    GKA_KERNEL_BWD_DELTA = 8,     /* backward: per-chunk increments of the adjoint state */
+    GKA_KERNEL_ADJOINT_SCAN = 9,  /* backward: adjoint states, last chunk first */
+    GKA_KERNEL_BWD_ROWS = 10,     /* backward: chunk rows against H_s, M_s and the adjoints */
+    GKA_KERNEL_BWD_GRADS = 11,    /* backward: dk, dv, dbeta, dgate of each chunk */
+    GKA_KERNEL_COUNT = 16
 };
 
 typedef struct {

@@ -327,6 +327,8 @@ k_chunk_norm(const Tin *__restrict__ k, const float *__restrict__ beta,
 // ---------------------------------------------------------------------------
 // Steps 3 + 4: r-step Chebyshev solve of (H_j + lambda_j I) x = q_j for TG
 // tokens of one chunk, then o_j = b_j M_s x_j + sum_{i<=j} w_{ji} (k_i.x_j) v_i.
+// With x_out (nullable, fp32 [B*H*T, D]) the kernel writes the iterates x_j there
+// instead and skips the readout (the backward pass recomputes them this way).
 // Chebyshev (ai.info, Key Contributions 2; pith.science appendix, Lemma 3):
 //   x_1 = q/d,  x_{i+1} = x_{i-1} + omega_i ((q - A x_i)/d + x_i - x_{i-1}),
 //   A = H_j + lambda_j I,  d = (1+2a) n_j / 2,  lambda_j = a n_j.
@@ -348,8 +350,8 @@ __global__ void __launch_bounds__(kSimtThreads)
 k_chunk_solve(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
               const float *__restrict__ beta, const float *__restrict__ gate,
               const float *__restrict__ states,
-              const float *__restrict__ norms, Tin *__restrict__ o, int T, int N, int C,
-              const ChebParams P) {
+              const float *__restrict__ norms, Tin *__restrict__ o, float *__restrict__ x_out,
+              int T, int N, int C, const ChebParams P) {
     constexpr int TG = kSolveTG;
     constexpr int KP = D + 1;
     constexpr int NJ = TG * D / kSimtThreads;   // tokens per thread in the D-parallel phase
@@ -466,6 +468,10 @@ k_chunk_solve(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
         __syncthreads();
     }
 
+    if (x_out) {
+        for (int e = tid; e < TG * D; e += kSimtThreads) x_out[(tok0 + j0) * D + e] = Xc[e];
+        return;
+    }
     // readout: P with the keys, then swap in M_s^T and the values
     form_p();
     __syncthreads();

@@ -14,6 +14,7 @@
 #include "../../include/gka.h"
 #include <cudaTypedefs.h>
 
+#include "backward_simt.cuh"
 #include "chunk_simt.cuh"
 #include "common.cuh"
 #include "decode.cuh"
@@ -199,7 +200,7 @@ static int forward_simt(const Tin *q, const Tin *k, const Tin *v, const float *b
     if ((e = set_smem(k_chunk_solve<Tin, D>, sm_solve)) != cudaSuccess) return cuda_fail(e);
     { ProfScope ps(GKA_KERNEL_CHUNK_SOLVE, s);
     k_chunk_solve<Tin, D><<<dim3(C / kSolveTG, N, BH), kSimtThreads, sm_solve, s>>>(
-        q, k, v, beta, gate, states, norms, o, T, N, C, P); }
+        q, k, v, beta, gate, states, norms, o, nullptr, T, N, C, P); }
     return check_launch();
 }
 
@@ -351,6 +352,124 @@ static int forward_dispatch(const void *q, const void *k, const void *v, const f
         case 32: return forward_simt<Tin, 32>(Q, K, V, beta, gate, O, B, H, T, C, P, final_state, ws, L, s);
         case 64: return forward_simt<Tin, 64>(Q, K, V, beta, gate, O, B, H, T, C, P, final_state, ws, L, s);
         default: return forward_simt<Tin, 128>(Q, K, V, beta, gate, O, B, H, T, C, P, final_state, ws, L, s);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Backward pass (CUDA cores): workspace layout and launches.
+// ---------------------------------------------------------------------------
+static bool supported_bwd_c(int C) { return C == 16 || C == 32; }
+
+struct BwdLayout {
+    gka_workspace_layout fwd;   // the forward's regions (chunk states, decays, norms)
+    size_t xs, ys, cvec, adj, rows, tokq, chq, total;
+};
+
+static int bwd_layout(int B, int H, int T, int D, int C, gka_dtype dt, BwdLayout *L) {
+    if (!supported_bwd_c(C) && supported_c(C)) return GKA_ERR_UNSUPPORTED;
+    if (int rc = layout(B, H, T, D, C, dt, &L->fwd)) return rc;
+    const size_t BH = (size_t)B * H, N = (size_t)(T / C), TD = BH * (size_t)T * D;
+    size_t off = round256(L->fwd.total_bytes);
+    L->xs = off;   off = round256(off + sizeof(float) * TD);
+    L->ys = off;   off = round256(off + sizeof(float) * TD);
+    L->cvec = off; off = round256(off + sizeof(float) * BH * T);
+    L->adj = off;  off = round256(off + sizeof(float) * BH * (N + 1) * 2 * D * D);
+    L->rows = off; off = round256(off + 4 * sizeof(float) * TD);
+    L->tokq = off; off = round256(off + 4 * sizeof(float) * BH * T);
+    L->chq = off;  off = round256(off + 2 * sizeof(float) * BH * N);
+    L->total = off;
+    return GKA_OK;
+}
+
+template <typename Tin, int D>
+static int backward_simt(const Tin *q, const Tin *k, const Tin *v, const float *beta,
+                         const float *gate, const Tin *dout, Tin *dq, Tin *dk, Tin *dv,
+                         float *dbeta, float *dgate, int B, int H, int T, int C,
+                         const ChebParams &P, char *ws, const BwdLayout &L, cudaStream_t s) {
+    const int BH = B * H, N = T / C;
+    float *states = reinterpret_cast<float *>(ws + L.fwd.states_offset);
+    float *decay = reinterpret_cast<float *>(ws + L.fwd.decay_offset);
+    float *norms = reinterpret_cast<float *>(ws + L.fwd.norms_offset);
+    float *xs = reinterpret_cast<float *>(ws + L.xs), *ys = reinterpret_cast<float *>(ws + L.ys);
+    float *cvec = reinterpret_cast<float *>(ws + L.cvec), *adj = reinterpret_cast<float *>(ws + L.adj);
+    float *rows = reinterpret_cast<float *>(ws + L.rows), *tokq = reinterpret_cast<float *>(ws + L.tokq);
+    float *chq = reinterpret_cast<float *>(ws + L.chq);
+    cudaError_t e;
+    const int DD2 = 2 * D * D;
+
+    // forward recompute: chunk states, norms and the iterates x_t
+    const size_t sm_delta = sizeof(float) * 3 * (size_t)C * D;
+    if ((e = set_smem(k_chunk_delta<Tin, D>, sm_delta)) != cudaSuccess) return cuda_fail(e);
+    { ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
+    k_chunk_delta<Tin, D><<<dim3(N, BH), kSimtThreads, sm_delta, s>>>(k, v, beta, gate, states,
+                                                                        decay, nullptr, T, N, C); }
+    if (int rc = check_launch()) return rc;
+    { ProfScope ps(GKA_KERNEL_STATE_SCAN, s);
+    k_state_scan<<<dim3((DD2 + 1023) / 1024, BH), 256, 0, s>>>(states, decay, nullptr, nullptr,
+                                                             nullptr, nullptr, N, DD2, true); }
+    if (int rc = check_launch()) return rc;
+    const size_t sm_norm = sizeof(float) * ((size_t)D * D + (size_t)C * (D + 1));
+    if ((e = set_smem(k_chunk_norm<Tin, D>, sm_norm)) != cudaSuccess) return cuda_fail(e);
+    { ProfScope ps(GKA_KERNEL_CHUNK_NORM, s);
+    k_chunk_norm<Tin, D><<<dim3(N, BH), kSimtThreads, sm_norm, s>>>(k, beta, gate, states, norms,
+                                                                    T, N, C); }
+    if (int rc = check_launch()) return rc;
+    const size_t sm_solve = SolveSmem<D>::bytes(C);
+    if ((e = set_smem(k_chunk_solve<Tin, D>, sm_solve)) != cudaSuccess) return cuda_fail(e);
+    { ProfScope ps(GKA_KERNEL_CHUNK_SOLVE, s);
+    k_chunk_solve<Tin, D><<<dim3(C / kSolveTG, N, BH), kSimtThreads, sm_solve, s>>>(
+        q, k, v, beta, gate, states, norms, nullptr, xs, T, N, C, P); }
+    if (int rc = check_launch()) return rc;
+
+    // adjoint solve: dq = y, c
+    if ((e = set_smem(k_bwd_solve<Tin, D>, sm_solve)) != cudaSuccess) return cuda_fail(e);
+    { ProfScope ps(GKA_KERNEL_BWD_SOLVE, s);
+    k_bwd_solve<Tin, D><<<dim3(C / kSolveTG, N, BH), kSimtThreads, sm_solve, s>>>(
+        k, v, beta, gate, dout, states, norms, xs, dq, ys, cvec, T, N, C, P); }
+    if (int rc = check_launch()) return rc;
+    // adjoint chunk increments and their reverse scan
+    const size_t sm_bd = sizeof(float) * 5 * (size_t)C * D;
+    if ((e = set_smem(k_bwd_delta<Tin, D>, sm_bd)) != cudaSuccess) return cuda_fail(e);
+    { ProfScope ps(GKA_KERNEL_BWD_DELTA, s);
+    k_bwd_delta<Tin, D><<<dim3(N, BH), kSimtThreads, sm_bd, s>>>(k, beta, gate, dout, states, xs,
+                                                                ys, cvec, adj, T, N, C); }
+    if (int rc = check_launch()) return rc;
+    { ProfScope ps(GKA_KERNEL_ADJOINT_SCAN, s);
+    k_adjoint_scan<<<dim3((DD2 / 4 + 255) / 256, BH), 256, 0, s>>>(adj, decay, N, DD2); }
+    if (int rc = check_launch()) return rc;
+    // the chunk rows against H_s, M_s and the adjoints
+    const size_t sm_rows = sizeof(float) * ((size_t)D * (D + 1) + 6 * (size_t)C * D);
+    if ((e = set_smem(k_bwd_rows<Tin, D>, sm_rows)) != cudaSuccess) return cuda_fail(e);
+    { ProfScope ps(GKA_KERNEL_BWD_ROWS, s);
+    k_bwd_rows<Tin, D><<<dim3(N, BH), kSimtThreads, sm_rows, s>>>(k, v, dout, states, adj, xs, ys,
+                                                                 rows, tokq, chq, T, N, C); }
+    if (int rc = check_launch()) return rc;
+    // gradients
+    const size_t sm_gr = BwdGradSmem<D>::bytes(C);
+    if ((e = set_smem(k_bwd_grads<Tin, D>, sm_gr)) != cudaSuccess) return cuda_fail(e);
+    { ProfScope ps(GKA_KERNEL_BWD_GRADS, s);
+    k_bwd_grads<Tin, D><<<dim3(N, BH), kSimtThreads, sm_gr, s>>>(
+        k, v, beta, gate, dout, xs, ys, cvec, rows, tokq, chq, dk, dv, dbeta, dgate, T, N, C); }
+    return check_launch();
+}
+
+template <typename Tin>
+static int backward_dispatch(const void *q, const void *k, const void *v, const float *beta,
+                             const float *gate, const void *dout, void *dq, void *dk, void *dv,
+                             float *dbeta, float *dgate, int B, int H, int T, int D, int C,
+                             const ChebParams &P, char *ws, const BwdLayout &L, cudaStream_t s) {
+    auto in = [](const void *p) { return static_cast<const Tin *>(p); };
+    auto out = [](void *p) { return static_cast<Tin *>(p); };
+    switch (D) {
+        case 32:
+            return backward_simt<Tin, 32>(in(q), in(k), in(v), beta, gate, in(dout), out(dq), out(dk),
+                                          out(dv), dbeta, dgate, B, H, T, C, P, ws, L, s);
+        case 64:
+            return backward_simt<Tin, 64>(in(q), in(k), in(v), beta, gate, in(dout), out(dq), out(dk),
+                                          out(dv), dbeta, dgate, B, H, T, C, P, ws, L, s);
+        default:
+            return backward_simt<Tin, 128>(in(q), in(k), in(v), beta, gate, in(dout), out(dq),
+                                           out(dk), out(dv), dbeta, dgate, B, H, T, C, P, ws, L, s);
     }
 }
 
@@ -701,6 +820,39 @@ int gka_decode_step_gated(float *state, const void *q, const void *k, const void
     return decode_dispatch<float>(state, q, k, v, beta, gate, o, (int)BH, D, P, s);
 }
 
+size_t gka_backward_workspace_bytes(int B, int H, int T, int D, int chunk, gka_dtype dt) {
+    BwdLayout L;
+    return bwd_layout(B, H, T, D, chunk, dt, &L) == GKA_OK ? L.total : 0;
+}
+
+int gka_backward(const void *q, const void *k, const void *v, const float *beta, const float *gate,
+                 const void *dout, void *dq, void *dk, void *dv, float *dbeta, float *dgate, int B,
+                 int H, int T, int D, gka_dtype dt, float a, int r, int chunk, void *workspace,
+                 size_t workspace_bytes, void *stream) {
+    BwdLayout L;
+    if (int rc = bwd_layout(B, H, T, D, chunk, dt, &L)) return rc;
+    if (!(a > 0.f) || !isfinite(a) || r < 1) return GKA_ERR_INVALID_ARG;
+    if (r > kMaxSteps) return GKA_ERR_UNSUPPORTED;
+    if ((size_t)B * H > 65535) return GKA_ERR_UNSUPPORTED;
+    if ((dgate != nullptr) != (gate != nullptr)) return GKA_ERR_INVALID_ARG;
+    if ((size_t)B * H == 0 || T == 0) return GKA_OK;
+    if (!q || !k || !v || !beta || !dout || !dq || !dk || !dv || !dbeta || !workspace)
+        return GKA_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, beta, gate, dout, dq, dk, dv, dbeta, dgate};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return GKA_ERR_MISALIGNED;
+    if ((uintptr_t)workspace & 255u) return GKA_ERR_MISALIGNED;
+    if (workspace_bytes < L.total) return GKA_ERR_WORKSPACE_TOO_SMALL;
+    const ChebParams P = make_cheb(a, r);
+    char *ws = static_cast<char *>(workspace);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dt == GKA_BF16)
+        return backward_dispatch<__nv_bfloat16>(q, k, v, beta, gate, dout, dq, dk, dv, dbeta, dgate,
+                                                B, H, T, D, chunk, P, ws, L, s);
+    return backward_dispatch<float>(q, k, v, beta, gate, dout, dq, dk, dv, dbeta, dgate, B, H, T, D,
+                                    chunk, P, ws, L, s);
+}
+
 int gka_selftest_timeout(void *stream) {
     int *flag = nullptr;
     if (int rc = timeout_flag_ptr(&flag)) return rc;
@@ -742,7 +894,7 @@ const char *gka_status_string(int status) {
     }
 }
 
-int gka_version(void) { return 100; }
+int gka_version(void) { return 110; }
 
 int gka_profiler_enable(int on) {
     std::lock_guard<std::mutex> g(g_prof_mu);

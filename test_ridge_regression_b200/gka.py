@@ -29,11 +29,13 @@ class GkaError(RuntimeError):
 
 
 KERNEL_NAMES = ["chunk_delta", "state_scan", "chunk_norm", "chunk_solve", "decode_step",
-                "chunk_solve_tc", "state_pass_tc"]
+                "chunk_solve_tc", "state_pass_tc", "bwd_solve", "bwd_delta", "adjoint_scan",
+                "bwd_rows", "bwd_grads"]
+_KERNEL_COUNT = 16
 
 
 class KernelTimes(ctypes.Structure):
-    _fields_ = [("ms", ctypes.c_double * 8), ("launches", ctypes.c_int * 8)]
+    _fields_ = [("ms", ctypes.c_double * _KERNEL_COUNT), ("launches", ctypes.c_int * _KERNEL_COUNT)]
 
 
 class WorkspaceLayout(ctypes.Structure):
@@ -74,6 +76,10 @@ def _lib():
         lib.gka_decode_step.restype = i
         lib.gka_decode_step_gated.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
         lib.gka_decode_step_gated.restype = i
+        lib.gka_backward_workspace_bytes.argtypes = [i, i, i, i, i, i]
+        lib.gka_backward_workspace_bytes.restype = sz
+        lib.gka_backward.argtypes = [vp] * 11 + [i, i, i, i, i, f, i, i, vp, sz, vp]
+        lib.gka_backward.restype = i
         lib.gka_selftest_timeout.argtypes = [vp]
         lib.gka_selftest_timeout.restype = i
         lib.gka_device_status.argtypes = [vp]
@@ -292,6 +298,41 @@ def gka_decode_step_gated(state, q, k, v, beta, gate, a: float, r: int, *, o=Non
                                       _stream(stream))
     _check("gka_decode_step_gated", rc)
     return o
+
+
+def backward_workspace_bytes(B, H, T, D, chunk, dtype=torch.bfloat16) -> int:
+    return int(_lib().gka_backward_workspace_bytes(B, H, T, D, chunk, _DT[dtype]))
+
+
+def gka_backward(q, k, v, beta, dout, a: float, r: int, chunk: int = 32, *, gate=None,
+                 workspace=None, stream=None):
+    """Implicit-differentiation backward (see include/gka.h).  q, k, v, dout:
+    [B, H, T, D] fp32 or bf16 CUDA tensors; beta (and the optional gate):
+    [B, H, T] fp32.  Returns a dict with dq, dk, dv (dtype of q), dbeta and, with a
+    gate, dgate (fp32)."""
+    _dev(q, k, v, beta, gate, dout, workspace)
+    B, H, T, D = q.shape
+    if any(t.shape != q.shape for t in (k, v, dout)) or beta.shape != (B, H, T):
+        raise ValueError("shape mismatch")
+    if gate is not None and (gate.shape != (B, H, T) or gate.dtype != torch.float32):
+        raise ValueError("gate must be float32 [B, H, T]")
+    dt = _dtype(q)
+    if any(t.dtype != q.dtype for t in (k, v, dout)) or beta.dtype != torch.float32:
+        raise TypeError("q, k, v, dout must share a dtype; beta must be float32")
+    out = {n: torch.empty_like(q) for n in ("dq", "dk", "dv")}
+    out["dbeta"] = torch.empty_like(beta)
+    if gate is not None:
+        out["dgate"] = torch.empty_like(gate)
+    if workspace is None:
+        n = backward_workspace_bytes(B, H, T, D, chunk, q.dtype)
+        workspace = torch.empty(max(n, 256), dtype=torch.uint8, device=q.device)
+    rc = _lib().gka_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(gate), _ptr(dout),
+                             _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dbeta"]),
+                             _ptr(out.get("dgate")), B, H, T, D, dt, float(a), int(r), int(chunk),
+                             _ptr(workspace), workspace.numel() * workspace.element_size(),
+                             _stream(stream))
+    _check("gka_backward", rc)
+    return out
 
 
 def selftest_timeout(stream=None) -> None:

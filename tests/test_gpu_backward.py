@@ -1,0 +1,108 @@
+"""GPU parity of gka_backward (implicit-differentiation backward, through the C
+ABI) against the float64 oracle's backward on the same seeded inputs.
+
+Metric: max over (batch, head) of the relative Frobenius error over the head's
+slab, for dq, dk, dv ([T, D]) and dbeta, dgate ([T]).  The backward computes in
+fp32 on CUDA cores; bars: 1e-4 with fp32 inputs; with bf16 inputs dq, dk, dv
+are rounded to bf16 (relative rounding 2^-9), bar 2e-2, and dbeta / dgate stay
+fp32, bar 1e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import cuda, head_rel_err
+from test_ridge_regression_b200 import build, gka
+from test_ridge_regression_b200.inputs import make_gate, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    build.build()
+
+
+def _dout(shape, dtype, seed):
+    g = torch.Generator().manual_seed(seed)
+    return torch.randn(*shape, generator=g).to(dtype)
+
+
+def check_backward(q, k, v, beta, a, r, C, gate=None, seed=0):
+    dout = _dout(q.shape, q.dtype, 9000 + seed)
+    dev = cuda(q, k, v, beta, dout)
+    gd = gate.cuda() if gate is not None else None
+    got = gka.gka_backward(dev[0], dev[1], dev[2], dev[3], dev[4], a, r, C, gate=gd)
+    assert gka.device_status() == 0
+    ref = oracle.backward(q, k, v, beta, dout, a, r, gate=gate)
+    fp32 = q.dtype == torch.float32
+    errs = {}
+    for name in ref:
+        bar = 1e-4 if fp32 else (1e-3 if name in ("dbeta", "dgate") else 2e-2)
+        errs[name] = head_rel_err(got[name], ref[name])
+        assert np.all(np.isfinite(got[name].float().cpu().numpy())), name
+        assert errs[name] <= bar, (name, errs[name], bar)
+    print(" ".join(f"{n} {e:.2e}" for n, e in errs.items()))
+    return got, ref
+
+
+@pytest.mark.parametrize("D", [32, 64, 128])
+@pytest.mark.parametrize("C", [16, 32])
+def test_backward_fp32(D, C):
+    q, k, v, beta = make_inputs(1, 2, 128, D, torch.float32, 2.0, 1.0, seed=800 + D + C)
+    check_backward(q, k, v, beta, 0.5, 10, C, seed=D + C)
+
+
+def test_backward_bf16_d128():
+    q, k, v, beta = make_inputs(1, 2, 128, 128, torch.bfloat16, 3.0, 1.0, seed=820)
+    check_backward(q, k, v, beta, 0.5, 20, 32, seed=1)
+
+
+def test_backward_write_gate_and_resets():
+    q, k, v, beta = make_inputs(1, 2, 128, 64, torch.float32, 1.0, 1.0, seed=830)
+    gate = make_gate((1, 2, 128), 830)
+    gate[0, 0, 0] = 0.0
+    gate[0, 1, 40:48] = 0.0
+    beta[0, 0, 32] = 0.0      # first token of a chunk
+    beta[0, 1, 50] = 0.0      # inside a chunk
+    check_backward(q, k, v, beta, 0.5, 10, 32, gate=gate, seed=2)
+
+
+def test_backward_small_a_strong_forgetting():
+    q, k, v, beta = make_inputs(1, 2, 96, 128, torch.float32, 0.0, 2.0, seed=840)
+    check_backward(q, k, v, beta, 0.1, 30, 16, seed=3)
+
+
+def test_backward_zero_keys_at_start():
+    q, k, v, beta = make_inputs(1, 2, 64, 32, torch.float32, 2.0, 1.0, seed=850)
+    k[0, 0, :3] = 0.0
+    got, _ = check_backward(q, k, v, beta, 0.5, 8, 16, seed=4)
+    assert torch.all(got["dq"][0, 0, :3] == 0)
+
+
+def test_backward_chunk_size_invariance():
+    q, k, v, beta = make_inputs(1, 2, 128, 64, torch.float32, 2.0, 1.0, seed=860)
+    dout = _dout(q.shape, q.dtype, 5)
+    dev = cuda(q, k, v, beta, dout)
+    g16 = gka.gka_backward(*dev, 0.5, 10, 16)
+    g32 = gka.gka_backward(*dev, 0.5, 10, 32)
+    for n in g16:
+        assert head_rel_err(g16[n], g32[n]) <= 1e-5, n
+
+
+def test_backward_larger_bf16():
+    q, k, v, beta = make_inputs(2, 4, 512, 128, torch.bfloat16, 3.0, 1.0, seed=870)
+    check_backward(q, k, v, beta, 0.5, 20, 32, seed=6)
+
+
+def test_backward_error_codes():
+    q = torch.zeros(1, 1, 64, 64, device="cuda")
+    beta = torch.ones(1, 1, 64, device="cuda")
+    with pytest.raises(gka.GkaError) as e:
+        gka.gka_backward(q, q, q, beta, q, 0.5, 4, 64)
+    assert e.value.status == -2
+    with pytest.raises(gka.GkaError) as e:
+        gka.gka_backward(q[:, :, :48], q[:, :, :48], q[:, :, :48], beta[:, :, :48], q[:, :, :48],
+                         0.5, 4, 32)
+    assert e.value.status == -3
