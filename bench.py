@@ -74,6 +74,7 @@ def parse():
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-write-gate", action="store_true",
                    help="skip the write-gated forward leg")
+    p.add_argument("--no-backward", action="store_true", help="skip the backward leg")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--decode-steps", type=int, default=None)
     p.add_argument("--decode-batch", type=int, default=None,
@@ -426,6 +427,11 @@ def main():
         result["write_gate"] = bench_write_gate(args, w, dev, qd, kd, vd, bd, od, ws, flush,
                                                 rank, world, barrier)
 
+    # ---- backward pass (implicit differentiation) on the same inputs ----
+    if not args.no_backward:
+        result["backward"] = bench_backward(args, w, dev, qd, kd, vd, bd, flush, rank, world,
+                                            barrier, peaks)
+
     # ---- decode step: HBM-bound, 256 x 32 heads, fp32 state ----
     if not args.no_decode and world == 1:
         result["decode"] = bench_decode(args, dev, peaks)
@@ -492,6 +498,80 @@ def bench_write_gate(args, w, dev, qd, kd, vd, bd, od, ws, flush, rank, world, b
             "tokens_per_s": world * w.B * w.T * args.steps / (total_ms / 1e3),
             "kernels_ms_per_step": {n: ms / args.steps for n, (ms, _) in kt.items()},
             "gpu_launches": sum(n for _, n in kt.values())}
+
+
+BWD_CHUNK = 32
+
+
+def bwd_flops_per_head_token(D, C, r):
+    """Algorithmic flops of each backward kernel per (head, token), causal C x C
+    products counted as dense tiles (2 flops per multiply-add)."""
+    ch = (r - 1) * (2 * D * D + 4 * C * D)
+    return {
+        "chunk_solve": ch,                                  # forward iterates, recomputed
+        "bwd_solve": (2 * D * D + 4 * C * D) + ch,          # u = M^T g, then the iteration
+        "bwd_delta": 6 * D * D,                             # three rank-C products per chunk
+        "bwd_rows": 14 * D * D,                             # seven row-times-matrix products
+        "bwd_grads": 16 * C * D,                            # four C x C x D dots, four C x C x D sums
+        "chunk_delta": 4 * D * D, "chunk_norm": 2 * D * D + 2 * C * D + 2 * C * C,
+    }
+
+
+def bench_backward(args, w, dev, qd, kd, vd, bd, flush, rank, world, barrier, peaks):
+    """gka_backward on the workload's inputs with a seeded upstream gradient: K steps
+    timed like the forward's, then the same steps under the launch profiler."""
+    import torch
+    from test_ridge_regression_b200 import dist as gdist
+    from test_ridge_regression_b200 import gka
+    g = torch.Generator(device=dev).manual_seed(gdist.shard_seed(w.seed, rank) + 77)
+    dout = torch.randn(qd.shape, generator=g, device=dev).to(qd.dtype)
+    ws = torch.empty(gka.backward_workspace_bytes(w.B, w.H, w.T, w.D, BWD_CHUNK, w.dtype),
+                     dtype=torch.uint8, device=dev)
+    steps = max(1, min(args.steps, 10))
+
+    def step():
+        return gka.gka_backward(qd, kd, vd, bd, dout, w.a, w.r, BWD_CHUNK, workspace=ws)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    torch.cuda.synchronize()
+    barrier()
+    for i in range(steps):
+        flush.fill_(float(i))
+        starts[i].record()
+        step()
+        ends[i].record()
+    torch.cuda.synchronize()
+    barrier()
+    total_ms = gdist.max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)), dev)
+    gka.profiler_read()
+    gka.profiler_enable(True)
+    for i in range(steps):
+        flush.fill_(float(i))
+        step()
+    torch.cuda.synchronize()
+    gka.profiler_enable(False)
+    kt = gka.profiler_read()
+    if gka.device_status() != 0:
+        raise RuntimeError("device status error after the backward steps")
+    per_kernel = {n: ms / steps for n, (ms, _) in kt.items()}
+    fl = bwd_flops_per_head_token(w.D, BWD_CHUNK, w.r)
+    head_tok = w.B * w.H * w.T
+    dom = max(per_kernel, key=per_kernel.get)
+    achieved = fl.get(dom, 0) * head_tok / (per_kernel[dom] / 1e3) / 1e12
+    peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+    total_fl = sum(fl[n] for n in per_kernel if n in fl) * head_tok
+    return {"chunk": BWD_CHUNK, "steps": steps, "ms_per_step": total_ms / steps,
+            "tokens_per_s": world * w.B * w.T * steps / (total_ms / 1e3),
+            "kernels_ms_per_step": per_kernel,
+            "gpu_launches": sum(n for _, n in kt.values()),
+            "roofline": {"bound": "alu", "kernel": dom, "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                         "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 flop x max SM clock",
+                         "algorithmic_per_step": fl.get(dom, 0) * head_tok},
+            "step_frac_of_fp32_peak": total_fl / (total_ms / steps / 1e3) / 1e12 / peak}
 
 
 def bench_decode(args, dev, peaks):

@@ -106,3 +106,26 @@ def test_backward_error_codes():
         gka.gka_backward(q[:, :, :48], q[:, :, :48], q[:, :, :48], beta[:, :, :48], q[:, :, :48],
                          0.5, 4, 32)
     assert e.value.status == -3
+
+
+def test_backward_full_b8h8t2048_sampled():
+    """The default forward workload (B8 H8 T2048 D128 bf16, a 0.5, r 20) through the
+    backward in the benchmark's launch configuration (chunk 32); the oracle checks a
+    sample of heads (heads are independent)."""
+    from test_ridge_regression_b200.inputs import WORKLOADS, workload_inputs
+    w = WORKLOADS["bf16_b8h8t2048d128"]
+    q, k, v, beta = workload_inputs(w)
+    dout = _dout(q.shape, q.dtype, 77)
+    got = gka.gka_backward(*cuda(q, k, v, beta, dout), w.a, w.r, 32)
+    assert gka.device_status() == 0
+    got = {n: t.cpu() for n, t in got.items()}
+    worst = {}
+    for (b, h) in [(0, 0), (7, 7)]:
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        ref = oracle.backward(q[sl], k[sl], v[sl], beta[sl], dout[sl], w.a, w.r, nthreads=1)
+        for name in ref:
+            bar = 1e-3 if name == "dbeta" else 2e-2
+            e = head_rel_err(got[name][sl], ref[name])
+            worst[name] = max(worst.get(name, 0.0), e)
+            assert e <= bar, (name, b, h, e)
+    print("full size sampled:", " ".join(f"{n} {e:.2e}" for n, e in worst.items()))
