@@ -38,16 +38,16 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # bench reports null.  Captures and commands: profiles/*.md.
 TRAFFIC = {
     # full-size forward workload (B8 H8 T2048 D128, chunk 64), one launch
-    "chunk_solve_tc": {"bytes": 237.317120e6 + 21.281024e6, "workload": "bf16_b8h8t2048d128",
+    "chunk_solve_tc": {"bytes": 237.268736e6 + 21.026560e6, "workload": "bf16_b8h8t2048d128",
                        "src": "test_ridge_regression_b200/csrc/solve_tc.cuh",
-                       "sha1": "a0eacd99a75638e4884b12f42cc63c5490c24b17"},
-    "state_pass_tc": {"bytes": 67.709696e6 + 79.886080e6, "workload": "bf16_b8h8t2048d128",
+                       "sha1": "a69f99e2165fff067707b5c625f3200655cd524d"},
+    "state_pass_tc": {"bytes": 67.715840e6 + 80.063488e6, "workload": "bf16_b8h8t2048d128",
                       "src": "test_ridge_regression_b200/csrc/state_tc.cuh",
-                      "sha1": "d95a1373693a3001898b1cb7297e3fc496592228"},
+                      "sha1": "3bd3bff3a2f8e7bf8df221195dc42f9281487e71"},
     # decode captured on 64 x 32 heads (state above L2), scaled x4 to 256 x 32 heads
-    "decode_step": {"bytes": 4 * (270.054912e6 + 213.513472e6), "workload": "decode_bf16_b256h32d128",
+    "decode_step": {"bytes": 4 * (270.059520e6 + 211.768320e6), "workload": "decode_bf16_b256h32d128",
                     "src": "test_ridge_regression_b200/csrc/decode.cuh",
-                    "sha1": "9fed00ad526c1e277840c391aca09dea977665ff"},
+                    "sha1": "584a95174601413ebccb32a81bd0bfb4d0217334"},
 }
 
 def traffic_of(kernel, workload):
