@@ -58,7 +58,7 @@ k_bwd_solve(const Tin *__restrict__ k, const Tin *__restrict__ v, const float *_
             const float *__restrict__ xs, Tin *__restrict__ dq, float *__restrict__ ys,
             float *__restrict__ cvec, int T, int N, int C, const ChebParams P) {
     constexpr int TG = kSolveTG;
-    constexpr int KP = D + 1;
+    constexpr int KP = SolveSmem<D>::KP;
     constexpr int NJ = TG * D / kSimtThreads;
     extern __shared__ __align__(16) float sm[];
     float *Ms = sm;                    // [D][KP]: M_s, then H_s
@@ -105,12 +105,7 @@ k_bwd_solve(const Tin *__restrict__ k, const Tin *__restrict__ v, const float *_
     auto form_p = [&]() {
         for (int p = tid; p < TG * jend; p += kSimtThreads) {
             const int jj = p / jend, i = p % jend;
-            const float *kr = Ks + i * KP;
-            const float *xr = Xc + jj * D;
-            float dot = 0.f;
-#pragma unroll 8
-            for (int d = 0; d < D; ++d) dot = fmaf(kr[d], xr[d], dot);
-            Ps[jj * C + i] = Ws[jj * C + i] * dot;
+            Ps[jj * C + i] = Ws[jj * C + i] * dot4<D>(Ks + i * KP, Xc + jj * D);
         }
     };
     // acc[u] = b_j sum_d Ms[d][c] x_j[d] + sum_i P[j][i] Ks[i][c]
@@ -330,15 +325,26 @@ k_adjoint_scan(float *__restrict__ adj, const float *__restrict__ decay, int N, 
     float *base = adj + (size_t)bh * (N + 1) * DD2 + e;
     const float *dec = decay + (size_t)bh * N;
     float4 carry = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int n = N - 1; n >= 0; --n) {
-        float4 *slot = reinterpret_cast<float4 *>(base + (size_t)n * DD2);
-        const float4 d = *slot;
-        *slot = carry;
-        const float b = dec[n];
-        carry.x = fmaf(b, carry.x, d.x);
-        carry.y = fmaf(b, carry.y, d.y);
-        carry.z = fmaf(b, carry.z, d.z);
-        carry.w = fmaf(b, carry.w, d.w);
+    // the loads of a batch of 8 slots are issued before the dependent stores
+    for (int n1 = N - 1; n1 >= 0; n1 -= 8) {
+        const int nb = n1 >= 7 ? 8 : n1 + 1;
+        float4 d[8];
+        float b[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (u < nb) {
+                d[u] = __ldcs(reinterpret_cast<const float4 *>(base + (size_t)(n1 - u) * DD2));
+                b[u] = dec[n1 - u];
+            }
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (u < nb) {
+                *reinterpret_cast<float4 *>(base + (size_t)(n1 - u) * DD2) = carry;
+                carry.x = fmaf(b[u], carry.x, d[u].x);
+                carry.y = fmaf(b[u], carry.y, d[u].y);
+                carry.z = fmaf(b[u], carry.z, d[u].z);
+                carry.w = fmaf(b[u], carry.w, d[u].w);
+            }
     }
 }
 
@@ -349,15 +355,28 @@ k_adjoint_scan(float *__restrict__ adj, const float *__restrict__ decay, int N, 
 //   (rows of [B*H*T, D] each), and per token uk_t = k_t^T H_s k_t,
 //   yhx_t = y_t^T H_s x_t, gmx_t = g_t^T M_s x_t, qe_t = k_t^T E^H k_t + v_t^T E^M k_t;
 //   per chunk hs2 = ||H_s||_F^2 and eh = <E^H, H_s> + <E^M, M_s>.
-// grid (N, B*H), block 256, shared memory (D * (D + 1) + 6 * C * D) floats.
+// Every product is out[t][c] = sum_d row_t[d] Mt[d][c] with the matrix staged in
+// shared memory in the orientation it needs (E^M transposed for R4, E^H
+// symmetrised for R2).  Warp w computes tokens w*C/8.., lane l the columns
+// l, l + 32, .. (conflict-free), in registers, reading 4 d at a time.
+// grid (N, B*H), block 256, shared memory BwdRowsSmem<D, C>::bytes.
 // ---------------------------------------------------------------------------
-template <typename Tin, int D>
+template <int D, int C>
+struct BwdRowsSmem {
+    static constexpr int DP = D + 4;   // 16-byte aligned rows
+    static constexpr size_t bytes = sizeof(float) * ((size_t)D * DP + 6 * (size_t)C * D);
+};
+
+template <typename Tin, int D, int C>
 __global__ void __launch_bounds__(kSimtThreads)
 k_bwd_rows(const Tin *__restrict__ k, const Tin *__restrict__ v, const Tin *__restrict__ dout,
            const float *__restrict__ states, const float *__restrict__ adj,
            const float *__restrict__ xs, const float *__restrict__ ys, float *__restrict__ R,
-           float *__restrict__ tokq, float *__restrict__ chq, int T, int N, int C) {
-    constexpr int DP = D + 1;
+           float *__restrict__ tokq, float *__restrict__ chq, int T, int N) {
+    constexpr int DP = BwdRowsSmem<D, C>::DP;
+    constexpr int TT = C / 8;          // tokens per warp
+    constexpr int CC = D / 32;         // columns per lane
+    static_assert(kSimtThreads == 256 && C % 8 == 0 && D % 32 == 0, "tiling");
     extern __shared__ __align__(16) float sm[];
     float *Mt = sm;              // [D][DP] one matrix at a time
     float *Kr = Mt + D * DP;     // [C][D] k_t
@@ -372,6 +391,7 @@ k_bwd_rows(const Tin *__restrict__ k, const Tin *__restrict__ v, const Tin *__re
     const int lane = tid & 31, warp = tid >> 5;
     const size_t tok0 = (size_t)bh * T + (size_t)n * C;
     const size_t plane = (size_t)gridDim.y * T;   // B*H*T
+    const size_t RD = plane * D;                  // one [B*H*T, D] array
     const float *Hs = states + ((size_t)bh * (N + 1) + n) * 2 * D * D, *Mst = Hs + D * D;
     const float *EH = adj + ((size_t)bh * (N + 1) + n) * 2 * D * D, *EM = EH + D * D;
     for (int e = tid; e < C * D; e += kSimtThreads) {
@@ -402,25 +422,62 @@ k_bwd_rows(const Tin *__restrict__ k, const Tin *__restrict__ v, const Tin *__re
         for (int w = 0; w < kSimtThreads / 32; ++w) s += red[tid][w];
         chq[((size_t)bh * N + n) * 2 + tid] = s;
     }
-    auto load_mat = [&](const float *src) {
+    // mode 0: Mt[d][c] = A[d][c]; 1: A[c][d]; 2: A[d][c] + A[c][d] (coalesced reads of A)
+    auto load_mat = [&](const float *A, int mode) {
         __syncthreads();
-        for (int e = tid; e < D * D; e += kSimtThreads) Mt[(e / D) * DP + e % D] = src[e];
-        __syncthreads();
-    };
-    // out[t][c] = sum_d row_t[d] (trans ? Mt[c][d] : Mt[d][c]) for every token t
-    auto rows_times = [&](const float *rows, bool trans, float *out, size_t gout) {
-        for (int p = tid; p < C * D; p += kSimtThreads) {
-            const int t = p / D, c = p % D;
-            const float *rw = rows + t * D;
-            float s = 0.f;
-            if (trans) {
-                for (int d = 0; d < D; ++d) s = fmaf(rw[d], Mt[c * DP + d], s);
-            } else {
-                for (int d = 0; d < D; ++d) s = fmaf(rw[d], Mt[d * DP + c], s);
-            }
-            if (out) out[p] = s;
-            if (gout != (size_t)-1) R[gout + tok0 * D + p] = s;
+        for (int e = tid; e < D * D; e += kSimtThreads) {
+            const int r = e / D, c = e % D;
+            if (mode == 1) Mt[c * DP + r] = A[e];
+            else Mt[r * DP + c] = A[e];
         }
+        __syncthreads();
+        if (mode == 2) {
+            for (int e = tid; e < D * D; e += kSimtThreads) {
+                const int r = e / D, c = e % D;
+                if (r < c) {
+                    const float x = Mt[r * DP + c] + Mt[c * DP + r];
+                    Mt[r * DP + c] = x;
+                    Mt[c * DP + r] = x;
+                } else if (r == c) {
+                    Mt[r * DP + c] *= 2.f;
+                }
+            }
+            __syncthreads();
+        }
+    };
+    // out[t][c] = sum_d rows[t][d] Mt[d][c] for this thread's TT x CC tile; written to
+    // shared memory (out) and/or the global array at gout
+    auto rows_times = [&](const float *rows, float *out, size_t gout) {
+        float acc[TT][CC];
+#pragma unroll
+        for (int a = 0; a < TT; ++a)
+#pragma unroll
+            for (int b = 0; b < CC; ++b) acc[a][b] = 0.f;
+        const int t0 = warp * TT;
+#pragma unroll 2
+        for (int d = 0; d < D; d += 4) {
+            float m[4][CC];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int b = 0; b < CC; ++b) m[u][b] = Mt[(d + u) * DP + lane + 32 * b];
+#pragma unroll
+            for (int a = 0; a < TT; ++a) {
+                const float4 r4 = *reinterpret_cast<const float4 *>(rows + (t0 + a) * D + d);
+#pragma unroll
+                for (int b = 0; b < CC; ++b)
+                    acc[a][b] = fmaf(r4.x, m[0][b], fmaf(r4.y, m[1][b],
+                                fmaf(r4.z, m[2][b], fmaf(r4.w, m[3][b], acc[a][b]))));
+            }
+        }
+#pragma unroll
+        for (int a = 0; a < TT; ++a)
+#pragma unroll
+            for (int b = 0; b < CC; ++b) {
+                const int p = (t0 + a) * D + lane + 32 * b;
+                if (out) out[p] = acc[a][b];
+                if (gout != (size_t)-1) R[gout + tok0 * D + p] = acc[a][b];
+            }
     };
     // per-token dot of two [C][D] arrays in shared memory, one warp per token
     auto tok_dot = [&](const float *A, const float *B, float *dst, float scale, bool add) {
@@ -431,35 +488,28 @@ k_bwd_rows(const Tin *__restrict__ k, const Tin *__restrict__ v, const Tin *__re
             s = warp_sum(s) * scale;
             if (lane == 0) dst[tok0 + t] = add ? dst[tok0 + t] + s : s;
         }
+        __syncthreads();
     };
-    const size_t RD = plane * D;   // one [B*H*T, D] array
-    // H_s: R1 = K H_s (H_s symmetric), uk = k . R1; H_s x -> yhx
-    load_mat(Hs);
-    rows_times(Kr, false, Tr, 0);
+    // H_s (symmetric): R1 = K H_s, uk = k . R1; x^T H_s -> yhx
+    load_mat(Hs, 0);
+    rows_times(Kr, Tr, 0);
     tok_dot(Tr, Kr, tokq, 1.f, false);
-    __syncthreads();
-    rows_times(Xr, false, Tr, (size_t)-1);
+    rows_times(Xr, Tr, (size_t)-1);
     tok_dot(Tr, Yr, tokq + plane, 1.f, false);
-    // M_s: g^T M_s x = (M_s^T g) . x
-    load_mat(Mst);
-    rows_times(Gr, false, Tr, (size_t)-1);
+    // M_s: g^T M_s x = (g^T M_s) . x
+    load_mat(Mst, 0);
+    rows_times(Gr, Tr, (size_t)-1);
     tok_dot(Tr, Xr, tokq + 2 * plane, 1.f, false);
-    // E^H: R2 = (E^H + E^H^T) k, qe = k^T E^H k = (k . R2) / 2
-    load_mat(EH);
-    for (int p = tid; p < C * D; p += kSimtThreads) {
-        const int t = p / D, c = p % D;
-        const float *rw = Kr + t * D;
-        float s = 0.f;
-        for (int d = 0; d < D; ++d) s = fmaf(rw[d], Mt[d * DP + c] + Mt[c * DP + d], s);
-        Tr[p] = s;
-        R[RD + tok0 * D + p] = s;
-    }
+    // E^H + E^H^T: R2, qe = k^T E^H k = (k . R2) / 2
+    load_mat(EH, 2);
+    rows_times(Kr, Tr, RD);
     tok_dot(Tr, Kr, tokq + 3 * plane, 0.5f, false);
-    // E^M: R3 = E^M^T v (rows v^T E^M), R4 = E^M k; qe += v . R4
-    load_mat(EM);
-    rows_times(Vr, false, nullptr, 2 * RD);
-    __syncthreads();
-    rows_times(Kr, true, Tr, 3 * RD);
+    // E^M: R3 = rows v^T E^M
+    load_mat(EM, 0);
+    rows_times(Vr, nullptr, 2 * RD);
+    // E^M^T: R4 = rows k^T E^M^T = (E^M k)^T; qe += v . R4
+    load_mat(EM, 1);
+    rows_times(Kr, Tr, 3 * RD);
     tok_dot(Tr, Vr, tokq + 3 * plane, 1.f, true);
 }
 

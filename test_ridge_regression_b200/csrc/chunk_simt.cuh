@@ -336,9 +336,25 @@ k_chunk_norm(const Tin *__restrict__ k, const float *__restrict__ beta,
 // ---------------------------------------------------------------------------
 constexpr int kSolveTG = 16;
 
+// Dot product of two 16-byte aligned rows of D floats in shared memory, 4 at a time.
+template <int D>
+__device__ __forceinline__ float dot4(const float *a, const float *b) {
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll 8
+    for (int d = 0; d < D; d += 8) {
+        const float4 a0 = *reinterpret_cast<const float4 *>(a + d);
+        const float4 b0 = *reinterpret_cast<const float4 *>(b + d);
+        const float4 a1 = *reinterpret_cast<const float4 *>(a + d + 4);
+        const float4 b1 = *reinterpret_cast<const float4 *>(b + d + 4);
+        s0 = fmaf(a0.x, b0.x, fmaf(a0.y, b0.y, fmaf(a0.z, b0.z, fmaf(a0.w, b0.w, s0))));
+        s1 = fmaf(a1.x, b1.x, fmaf(a1.y, b1.y, fmaf(a1.z, b1.z, fmaf(a1.w, b1.w, s1))));
+    }
+    return s0 + s1;
+}
+
 template <int D>
 struct SolveSmem {
-    static constexpr int KP = D + 1;
+    static constexpr int KP = D + 4;   // 16-byte aligned rows (float4 dots, conflict-free)
     static size_t bytes(int C) {
         return sizeof(float) * ((size_t)D * KP + (size_t)C * KP + 3 * kSolveTG * D +
                                 2 * kSolveTG * C);
@@ -353,7 +369,7 @@ k_chunk_solve(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
               const float *__restrict__ norms, Tin *__restrict__ o, float *__restrict__ x_out,
               int T, int N, int C, const ChebParams P) {
     constexpr int TG = kSolveTG;
-    constexpr int KP = D + 1;
+    constexpr int KP = SolveSmem<D>::KP;
     constexpr int NJ = TG * D / kSimtThreads;   // tokens per thread in the D-parallel phase
     extern __shared__ __align__(16) float sm[];
     float *Ms = sm;                    // [D][KP]: H_s (symmetric), later M_s^T
@@ -407,12 +423,7 @@ k_chunk_solve(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
     auto form_p = [&]() {
         for (int p = tid; p < TG * jend; p += kSimtThreads) {
             const int jj = p / jend, i = p % jend;
-            const float *kr = Ks + i * KP;
-            const float *xr = Xc + jj * D;
-            float dot = 0.f;
-#pragma unroll 8
-            for (int d = 0; d < D; ++d) dot = fmaf(kr[d], xr[d], dot);
-            Ps[jj * C + i] = Ws[jj * C + i] * dot;
+            Ps[jj * C + i] = Ws[jj * C + i] * dot4<D>(Ks + i * KP, Xc + jj * D);
         }
     };
     // acc[u] = b_j sum_d S[d][c] x_j[d] + sum_i P[j][i] R[i][c] for the thread's tokens

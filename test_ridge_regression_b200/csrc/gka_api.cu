@@ -240,7 +240,7 @@ static int timeout_flag_ptr(int **ptr);
 static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
                       const float *beta, const float *gate, __nv_bfloat16 *o, int B, int H, int T, int C,
                       const ChebParams &P, float *final_state, char *ws,
-                      const gka_workspace_layout &L, cudaStream_t s) {
+                      const gka_workspace_layout &L, cudaStream_t s, float *x_out = nullptr) {
     constexpr int D = 128;
     const int BH = B * H, N = T / C;
     float *states = reinterpret_cast<float *>(ws + L.states_offset);
@@ -322,14 +322,14 @@ static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
         if ((e = set_smem(kern, TcSmem<64, 64>::bytes)) != cudaSuccess) return cuda_fail(e);
         ProfScope ps(GKA_KERNEL_CHUNK_SOLVE_TC, s);
         kern<<<dim3(N, BH), kSolveThreads, TcSmem<64, 64>::bytes, s>>>(
-            maps, q, gate, tokdec, plane, norms, sexp, o, T, N, C, P, flag);
+            maps, q, gate, tokdec, plane, norms, sexp, o, x_out, T, N, C, P, flag);
     } else {
         // one CTA per 128-token chunk (N = 128 MMAs)
         auto kern = k_chunk_solve_tc<128, 128>;
         if ((e = set_smem(kern, TcSmem<128, 128>::bytes)) != cudaSuccess) return cuda_fail(e);
         ProfScope ps(GKA_KERNEL_CHUNK_SOLVE_TC, s);
         kern<<<dim3(N, BH), kSolveThreads, TcSmem<128, 128>::bytes, s>>>(
-            maps, q, gate, tokdec, plane, norms, sexp, o, T, N, C, P, flag);
+            maps, q, gate, tokdec, plane, norms, sexp, o, x_out, T, N, C, P, flag);
     }
     if (int rc = check_launch()) return rc;
     return GKA_OK;
@@ -362,7 +362,12 @@ static bool supported_bwd_c(int C) { return C == 16 || C == 32; }
 
 struct BwdLayout {
     gka_workspace_layout fwd;   // the forward's regions (chunk states, decays, norms)
-    size_t xs, ys, cvec, adj, rows, tokq, chq, total;
+    size_t xs, ys, cvec, adj, rows, tokq, chq;
+    // bf16, D = 128, T a multiple of 64: the forward iterates come from the tensor-core
+    // forward with 64-token chunks, whose own workspace starts at tc
+    bool tc_recompute;
+    gka_workspace_layout tcl;
+    size_t tc, total;
 };
 
 static int bwd_layout(int B, int H, int T, int D, int C, gka_dtype dt, BwdLayout *L) {
@@ -377,6 +382,12 @@ static int bwd_layout(int B, int H, int T, int D, int C, gka_dtype dt, BwdLayout
     L->rows = off; off = round256(off + 4 * sizeof(float) * TD);
     L->tokq = off; off = round256(off + 4 * sizeof(float) * BH * T);
     L->chq = off;  off = round256(off + 2 * sizeof(float) * BH * N);
+    L->tc_recompute = tensor_core_path(D, 64, dt) && T % 64 == 0;
+    L->tc = off;
+    if (L->tc_recompute) {
+        if (int rc = layout(B, H, T, D, 64, dt, &L->tcl)) return rc;
+        off = round256(off + L->tcl.total_bytes);
+    }
     L->total = off;
     return GKA_OK;
 }
@@ -397,7 +408,8 @@ static int backward_simt(const Tin *q, const Tin *k, const Tin *v, const float *
     cudaError_t e;
     const int DD2 = 2 * D * D;
 
-    // forward recompute: chunk states, norms and the iterates x_t
+    // forward recompute: chunk states, norms and the iterates x_t (bf16, D = 128: the
+    // iterates and norms from the tensor-core forward, the fp32 chunk states here)
     const size_t sm_delta = sizeof(float) * 3 * (size_t)C * D;
     if ((e = set_smem(k_chunk_delta<Tin, D>, sm_delta)) != cudaSuccess) return cuda_fail(e);
     { ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
@@ -408,18 +420,31 @@ static int backward_simt(const Tin *q, const Tin *k, const Tin *v, const float *
     k_state_scan<<<dim3((DD2 + 1023) / 1024, BH), 256, 0, s>>>(states, decay, nullptr, nullptr,
                                                              nullptr, nullptr, N, DD2, true); }
     if (int rc = check_launch()) return rc;
-    const size_t sm_norm = sizeof(float) * ((size_t)D * D + (size_t)C * (D + 1));
-    if ((e = set_smem(k_chunk_norm<Tin, D>, sm_norm)) != cudaSuccess) return cuda_fail(e);
-    { ProfScope ps(GKA_KERNEL_CHUNK_NORM, s);
-    k_chunk_norm<Tin, D><<<dim3(N, BH), kSimtThreads, sm_norm, s>>>(k, beta, gate, states, norms,
-                                                                    T, N, C); }
-    if (int rc = check_launch()) return rc;
     const size_t sm_solve = SolveSmem<D>::bytes(C);
-    if ((e = set_smem(k_chunk_solve<Tin, D>, sm_solve)) != cudaSuccess) return cuda_fail(e);
-    { ProfScope ps(GKA_KERNEL_CHUNK_SOLVE, s);
-    k_chunk_solve<Tin, D><<<dim3(C / kSolveTG, N, BH), kSimtThreads, sm_solve, s>>>(
-        q, k, v, beta, gate, states, norms, nullptr, xs, T, N, C, P); }
-    if (int rc = check_launch()) return rc;
+    bool tc_done = false;
+    if constexpr (std::is_same<Tin, __nv_bfloat16>::value && D == 128) {
+        if (L.tc_recompute) {
+            char *tws = ws + L.tc;
+            if (int rc = forward_tc(q, k, v, beta, gate, nullptr, B, H, T, 64, P, nullptr, tws,
+                                    L.tcl, s, xs))
+                return rc;
+            norms = reinterpret_cast<float *>(tws + L.tcl.norms_offset);
+            tc_done = true;
+        }
+    }
+    if (!tc_done) {
+        const size_t sm_norm = sizeof(float) * ((size_t)D * D + (size_t)C * (D + 1));
+        if ((e = set_smem(k_chunk_norm<Tin, D>, sm_norm)) != cudaSuccess) return cuda_fail(e);
+        { ProfScope ps(GKA_KERNEL_CHUNK_NORM, s);
+        k_chunk_norm<Tin, D><<<dim3(N, BH), kSimtThreads, sm_norm, s>>>(k, beta, gate, states,
+                                                                        norms, T, N, C); }
+        if (int rc = check_launch()) return rc;
+        if ((e = set_smem(k_chunk_solve<Tin, D>, sm_solve)) != cudaSuccess) return cuda_fail(e);
+        { ProfScope ps(GKA_KERNEL_CHUNK_SOLVE, s);
+        k_chunk_solve<Tin, D><<<dim3(C / kSolveTG, N, BH), kSimtThreads, sm_solve, s>>>(
+            q, k, v, beta, gate, states, norms, nullptr, xs, T, N, C, P); }
+        if (int rc = check_launch()) return rc;
+    }
 
     // adjoint solve: dq = y, c
     if ((e = set_smem(k_bwd_solve<Tin, D>, sm_solve)) != cudaSuccess) return cuda_fail(e);
@@ -438,11 +463,19 @@ static int backward_simt(const Tin *q, const Tin *k, const Tin *v, const float *
     k_adjoint_scan<<<dim3((DD2 / 4 + 255) / 256, BH), 256, 0, s>>>(adj, decay, N, DD2); }
     if (int rc = check_launch()) return rc;
     // the chunk rows against H_s, M_s and the adjoints
-    const size_t sm_rows = sizeof(float) * ((size_t)D * (D + 1) + 6 * (size_t)C * D);
-    if ((e = set_smem(k_bwd_rows<Tin, D>, sm_rows)) != cudaSuccess) return cuda_fail(e);
-    { ProfScope ps(GKA_KERNEL_BWD_ROWS, s);
-    k_bwd_rows<Tin, D><<<dim3(N, BH), kSimtThreads, sm_rows, s>>>(k, v, dout, states, adj, xs, ys,
-                                                                 rows, tokq, chq, T, N, C); }
+    if (C == 16) {
+        constexpr size_t sm_rows = BwdRowsSmem<D, 16>::bytes;
+        if ((e = set_smem(k_bwd_rows<Tin, D, 16>, sm_rows)) != cudaSuccess) return cuda_fail(e);
+        ProfScope ps(GKA_KERNEL_BWD_ROWS, s);
+        k_bwd_rows<Tin, D, 16><<<dim3(N, BH), kSimtThreads, sm_rows, s>>>(
+            k, v, dout, states, adj, xs, ys, rows, tokq, chq, T, N);
+    } else {
+        constexpr size_t sm_rows = BwdRowsSmem<D, 32>::bytes;
+        if ((e = set_smem(k_bwd_rows<Tin, D, 32>, sm_rows)) != cudaSuccess) return cuda_fail(e);
+        ProfScope ps(GKA_KERNEL_BWD_ROWS, s);
+        k_bwd_rows<Tin, D, 32><<<dim3(N, BH), kSimtThreads, sm_rows, s>>>(
+            k, v, dout, states, adj, xs, ys, rows, tokq, chq, T, N);
+    }
     if (int rc = check_launch()) return rc;
     // gradients
     const size_t sm_gr = BwdGradSmem<D>::bytes(C);

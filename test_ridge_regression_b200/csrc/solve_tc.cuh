@@ -273,8 +273,9 @@ template <int MG, int TOK>
 __global__ void __launch_bounds__(kSolveThreads, TOK == 64 ? 2 : 1)
 k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__restrict__ q,
                  const float *__restrict__ gate, const float *__restrict__ tokdec, size_t plane, float *__restrict__ norms,
-                 const int *__restrict__ state_exp, __nv_bfloat16 *__restrict__ o, int T, int N,
-                 int C, const ChebParams P, int *__restrict__ timeout_flag) {
+                 const int *__restrict__ state_exp, __nv_bfloat16 *__restrict__ o,
+                 float *__restrict__ x_out, int T, int N, int C, const ChebParams P,
+                 int *__restrict__ timeout_flag) {
     using L = TcSmem<MG, TOK>;
     constexpr int HALF = MG / 2;       // keys per warpgroup in the norm reductions
     constexpr int TPT = TOK / 2;       // tokens per thread
@@ -651,8 +652,11 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     // warps 1-7 form P, warp 4 also covering warp 0's lane quarter, and warp 4
     // issues Z3.  The P warps and the Z3 issuer meet at a named barrier, so Z3 =
     // K^T P^T (commit bar_z) need not wait for the Z1 issue to finish.
+    // With x_out (nullable, fp32 [B*H*T][128]) the rounds stop before the readout
+    // pass and the iterates x_j themselves are written (the backward recomputes them).
+    const int last_it = x_out ? P.r - 1 : P.r;
 #pragma unroll 1
-    for (int it = 1; it <= P.r && ok; ++it) {
+    for (int it = 1; it <= last_it && ok; ++it) {
         const bool out_pass = (it == P.r);
         const float w_next = P.omega[it + 1 < kMaxSteps ? it + 1 : 0];   // next round's weight
         if (tid == 0) {
@@ -744,7 +748,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         if (!mbar_wait_sleep(bar_z1, ph, kTcSleepProbes, kTcSleepNs)) ok = false;
         tc::fence_after_sync();
         if (!out_pass) {
-            if (tid == 0 && it == P.r - 1) {
+            if (tid == 0 && it == P.r - 1 && !x_out) {
                 // H_s is no longer read: fetch M_s for the readout into the same buffer
                 mbar_arrive_expect_tx(bar_m, 32768);
                 for (int h = 0; h < 2; ++h)
@@ -838,6 +842,14 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         }
     }
 
+    if (x_out && ok) {
+        // x_j = x~_j invd_j / sigma, invd_j = c3_j sK^2 (thread (wg, d): element d of
+        // its tokens; consecutive d of a token are consecutive threads)
+        const float xs = sK * sK / sigma;
+        float *xrow = x_out + (tok0 + tcol) * kTcD + d;
+#pragma unroll
+        for (int u = 0; u < TPT; ++u) xrow[(size_t)u * kTcD] = xc[u] * (s_c3[tcol + u] * xs);
+    }
     // teardown: no MMA, copy or TMEM store of this CTA may be in flight when TMEM is freed
     tc::tmem_wait_st();
     ok = __syncthreads_and(ok);

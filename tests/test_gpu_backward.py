@@ -3,9 +3,10 @@ ABI) against the float64 oracle's backward on the same seeded inputs.
 
 Metric: max over (batch, head) of the relative Frobenius error over the head's
 slab, for dq, dk, dv ([T, D]) and dbeta, dgate ([T]).  The backward computes in
-fp32 on CUDA cores; bars: 1e-4 with fp32 inputs; with bf16 inputs dq, dk, dv
-are rounded to bf16 (relative rounding 2^-9), bar 2e-2, and dbeta / dgate stay
-fp32, bar 1e-3.
+fp32 on CUDA cores; with bf16 inputs, D = 128 and T a multiple of 64 it takes the
+forward iterates and norms from the tensor-core forward (fp16 operands), so its
+gradients carry that forward's bf16-level error.  Bars: 1e-4 with fp32 inputs,
+2e-2 with bf16 inputs (dq, dk, dv are also rounded to bf16).
 """
 import numpy as np
 import pytest
@@ -39,7 +40,7 @@ def check_backward(q, k, v, beta, a, r, C, gate=None, seed=0):
     fp32 = q.dtype == torch.float32
     errs = {}
     for name in ref:
-        bar = 1e-4 if fp32 else (1e-3 if name in ("dbeta", "dgate") else 2e-2)
+        bar = 1e-4 if fp32 else 2e-2
         errs[name] = head_rel_err(got[name], ref[name])
         assert np.all(np.isfinite(got[name].float().cpu().numpy())), name
         assert errs[name] <= bar, (name, errs[name], bar)
@@ -55,8 +56,24 @@ def test_backward_fp32(D, C):
 
 
 def test_backward_bf16_d128():
+    # T = 128: the tensor-core forward supplies the iterates (4 heads: chunk increments)
     q, k, v, beta = make_inputs(1, 2, 128, 128, torch.bfloat16, 3.0, 1.0, seed=820)
     check_backward(q, k, v, beta, 0.5, 20, 32, seed=1)
+
+
+def test_backward_bf16_d128_cuda_core_recompute():
+    # T = 96 (not a multiple of 64): the CUDA-core forward supplies the iterates
+    q, k, v, beta = make_inputs(1, 2, 96, 128, torch.bfloat16, 3.0, 1.0, seed=821)
+    check_backward(q, k, v, beta, 0.5, 20, 32, seed=7)
+
+
+def test_backward_bf16_state_pass_gate_resets():
+    # 24 heads: the tensor-core forward's one-pass state kernel; a write gate, resets
+    q, k, v, beta = make_inputs(1, 24, 128, 128, torch.bfloat16, 2.0, 1.0, seed=822)
+    gate = make_gate((1, 24, 128), 822)
+    gate[0, 3, 10:20] = 0.0
+    beta[0, 5, 64] = 0.0
+    check_backward(q, k, v, beta, 0.5, 20, 32, gate=gate, seed=8)
 
 
 def test_backward_write_gate_and_resets():
@@ -124,8 +141,8 @@ def test_backward_full_b8h8t2048_sampled():
         sl = (slice(b, b + 1), slice(h, h + 1))
         ref = oracle.backward(q[sl], k[sl], v[sl], beta[sl], dout[sl], w.a, w.r, nthreads=1)
         for name in ref:
-            bar = 1e-3 if name == "dbeta" else 2e-2
             e = head_rel_err(got[name][sl], ref[name])
+            bar = 2e-2
             worst[name] = max(worst.get(name, 0.0), e)
             assert e <= bar, (name, b, h, e)
     print("full size sampled:", " ".join(f"{n} {e:.2e}" for n, e in worst.items()))
