@@ -56,7 +56,8 @@ k_bwd_solve(const Tin *__restrict__ k, const Tin *__restrict__ v, const float *_
             const float *__restrict__ gate, const Tin *__restrict__ dout,
             const float *__restrict__ states, const float *__restrict__ norms,
             const float *__restrict__ xs, Tin *__restrict__ dq, float *__restrict__ ys,
-            float *__restrict__ cvec, int T, int N, int C, const ChebParams P) {
+            float *__restrict__ cvec, Tin *__restrict__ u_out, int T, int N, int C,
+            const ChebParams P) {
     constexpr int TG = kSolveTG;
     constexpr int KP = SolveSmem<D>::KP;
     constexpr int NJ = TG * D / kSimtThreads;
@@ -148,6 +149,11 @@ k_bwd_solve(const Tin *__restrict__ k, const Tin *__restrict__ v, const float *_
         for (int u = 0; u < NJ; ++u) Qs[(jg * NJ + u) * D + c] = acc[u];
     }
     __syncthreads();
+    if (u_out) {
+        // u only (the solve runs elsewhere)
+        for (int e = tid; e < TG * D; e += kSimtThreads) store_f(u_out + (tok0 + j0) * D + e, Qs[e]);
+        return;
+    }
     for (int e = tid; e < D * D; e += kSimtThreads) Ms[(e / D) * KP + e % D] = Sg[e];
     for (int e = tid; e < TG * D; e += kSimtThreads) {
         Xc[e] = Qs[e] * s_invd[e / D];
@@ -194,6 +200,31 @@ k_bwd_solve(const Tin *__restrict__ k, const Tin *__restrict__ v, const float *_
             const float nj = norms[tok0 + j0 + jj];
             cvec[tok0 + j0 + jj] = nj > 0.f ? P.a * s / nj : 0.f;
         }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// k_bwd_yfinish: after an adjoint solve done elsewhere (y in ys), dq = y and
+// c_t = a (y_t . x_t) / n_t.  One warp per token; grid ceil(tokens / 8), block 256.
+// ---------------------------------------------------------------------------
+template <typename Tin, int D>
+__global__ void __launch_bounds__(kSimtThreads)
+k_bwd_yfinish(const float *__restrict__ ys, const float *__restrict__ xs,
+              const float *__restrict__ norms, Tin *__restrict__ dq, float *__restrict__ cvec,
+              size_t tokens, float a) {
+    const int lane = threadIdx.x & 31;
+    const size_t t = (size_t)blockIdx.x * (kSimtThreads / 32) + (threadIdx.x >> 5);
+    if (t >= tokens) return;
+    float s = 0.f;
+    for (int d = lane; d < D; d += 32) {
+        const float y = ys[t * D + d];
+        s = fmaf(y, xs[t * D + d], s);
+        store_f(dq + t * D + d, y);
+    }
+    s = warp_sum(s);
+    if (lane == 0) {
+        const float n = norms[t];
+        cvec[t] = n > 0.f ? a * s / n : 0.f;
     }
 }
 

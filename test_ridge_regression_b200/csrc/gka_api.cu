@@ -240,7 +240,10 @@ static int timeout_flag_ptr(int **ptr);
 static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
                       const float *beta, const float *gate, __nv_bfloat16 *o, int B, int H, int T, int C,
                       const ChebParams &P, float *final_state, char *ws,
-                      const gka_workspace_layout &L, cudaStream_t s, float *x_out = nullptr) {
+                      const gka_workspace_layout &L, cudaStream_t s, float *x_out = nullptr,
+                      bool solve_only = false) {
+    // x_out: write the iterates instead of o; solve_only: the chunk states in the
+    // workspace are current (an earlier call on the same keys, values and decays)
     constexpr int D = 128;
     const int BH = B * H, N = T / C;
     float *states = reinterpret_cast<float *>(ws + L.states_offset);
@@ -272,7 +275,9 @@ static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
     if (int rc = rows128_map(&dmaps.out, states, (uint64_t)BH * (N + 1) * 2 * D,
                              CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 32, 128))
         return rc;
-    if (BH >= kStatePassMinHeads) {
+    if (solve_only) {
+        // chunk states already in the workspace
+    } else if (BH >= kStatePassMinHeads) {
         StateMaps smaps;
         smaps.k = maps.k;
         smaps.v = maps.v;
@@ -367,7 +372,7 @@ struct BwdLayout {
     // forward with 64-token chunks, whose own workspace starts at tc
     bool tc_recompute;
     gka_workspace_layout tcl;
-    size_t tc, total;
+    size_t tc, u16, total;
 };
 
 static int bwd_layout(int B, int H, int T, int D, int C, gka_dtype dt, BwdLayout *L) {
@@ -387,6 +392,8 @@ static int bwd_layout(int B, int H, int T, int D, int C, gka_dtype dt, BwdLayout
     if (L->tc_recompute) {
         if (int rc = layout(B, H, T, D, 64, dt, &L->tcl)) return rc;
         off = round256(off + L->tcl.total_bytes);
+        L->u16 = off;   // u = M^T dL/do in bf16, the right-hand side of the adjoint solve
+        off = round256(off + 2 * TD);
     }
     L->total = off;
     return GKA_OK;
@@ -446,12 +453,25 @@ static int backward_simt(const Tin *q, const Tin *k, const Tin *v, const float *
         if (int rc = check_launch()) return rc;
     }
 
-    // adjoint solve: dq = y, c
+    // adjoint solve: dq = y, c (bf16, D = 128: u on CUDA cores, rounded to bf16, then the
+    // tensor-core solve on it with the tensor-core forward's chunk states)
     if ((e = set_smem(k_bwd_solve<Tin, D>, sm_solve)) != cudaSuccess) return cuda_fail(e);
+    Tin *u16 = tc_done ? reinterpret_cast<Tin *>(ws + L.u16) : nullptr;
     { ProfScope ps(GKA_KERNEL_BWD_SOLVE, s);
     k_bwd_solve<Tin, D><<<dim3(C / kSolveTG, N, BH), kSimtThreads, sm_solve, s>>>(
-        k, v, beta, gate, dout, states, norms, xs, dq, ys, cvec, T, N, C, P); }
+        k, v, beta, gate, dout, states, norms, xs, dq, ys, cvec, u16, T, N, C, P); }
     if (int rc = check_launch()) return rc;
+    if constexpr (std::is_same<Tin, __nv_bfloat16>::value && D == 128) {
+        if (tc_done) {
+            if (int rc = forward_tc(u16, k, v, beta, gate, nullptr, B, H, T, 64, P, nullptr,
+                                    ws + L.tc, L.tcl, s, ys, true))
+                return rc;
+            { ProfScope ps(GKA_KERNEL_BWD_SOLVE, s);
+            k_bwd_yfinish<Tin, D><<<(unsigned)(((size_t)BH * T + 7) / 8), kSimtThreads, 0, s>>>(
+                ys, xs, norms, dq, cvec, (size_t)BH * T, P.a); }
+            if (int rc = check_launch()) return rc;
+        }
+    }
     // adjoint chunk increments and their reverse scan
     const size_t sm_bd = sizeof(float) * 5 * (size_t)C * D;
     if ((e = set_smem(k_bwd_delta<Tin, D>, sm_bd)) != cudaSuccess) return cuda_fail(e);
