@@ -546,48 +546,57 @@ k_bwd_rows(const Tin *__restrict__ k, const Tin *__restrict__ v, const Tin *__re
 
 // ---------------------------------------------------------------------------
 // k_bwd_grads: dk, dv, dbeta and the write-gate gradient of one chunk.
-// grid (N, B*H), block 256, shared memory BwdGradSmem<D>::bytes(C).
+// Shared memory: the chunk's k, x, y, g rows (fp32, rows padded to 16 bytes),
+// the C x C matrices, and one region that holds the v rows until their dot
+// products are formed and the four coefficient matrices after.  Products run
+// in register tiles: the dot-product matrices in TI x TI tiles over rows
+// (l0 + 8i, s0 + 8j) (conflict-free 16-byte loads), the row outputs with a warp
+// per group of tokens and a lane per group of columns.
+// grid (N, B*H), block 256, shared memory BwdGradSmem<D, C>::bytes (2 CTAs per SM
+// at D = 128, C = 32).
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, int C>
 struct BwdGradSmem {
-    static constexpr int KP = D + 1;
-    static size_t bytes(int C) {
-        return sizeof(float) * (5 * (size_t)C * KP + 10 * (size_t)C * (C + 1) + 2 * (size_t)C * KP);
-    }
+    static constexpr int KP = D + 4;
+    static constexpr int CP = C + 1;
+    static constexpr size_t rows = (size_t)C * KP;
+    static constexpr size_t mats = (size_t)C * CP;
+    // k, x, y, g rows; v rows / Py Px Pk Pg; KX KY VG GK Wt Q
+    static constexpr size_t union_floats = rows > 4 * mats ? rows : 4 * mats;
+    static constexpr size_t bytes = sizeof(float) * (4 * rows + union_floats + 6 * mats);
 };
 
-template <typename Tin, int D>
-__global__ void __launch_bounds__(kSimtThreads)
+template <typename Tin, int D, int C>
+__global__ void __launch_bounds__(kSimtThreads, 2)
 k_bwd_grads(const Tin *__restrict__ k, const Tin *__restrict__ v, const float *__restrict__ beta,
             const float *__restrict__ gate, const Tin *__restrict__ dout,
             const float *__restrict__ xs, const float *__restrict__ ys,
             const float *__restrict__ cvec, const float *__restrict__ R,
             const float *__restrict__ tokq, const float *__restrict__ chq, Tin *__restrict__ dk,
             Tin *__restrict__ dv, float *__restrict__ dbeta, float *__restrict__ dgate, int T,
-            int N, int C) {
-    constexpr int KP = D + 1;
-    const int CP = C + 1;
+            int N) {
+    using L = BwdGradSmem<D, C>;
+    constexpr int KP = L::KP, CP = L::CP;
+    constexpr int TI = C / 8;          // dot tile edge; tokens per warp in the row outputs
+    constexpr int CC = D / 32;         // columns per lane in the row outputs
+    static_assert(kSimtThreads == 256 && (C == 16 || C == 32) && D % 32 == 0, "tiling");
     extern __shared__ __align__(16) float sm[];
-    float *Kr = sm;                  // [C][KP] k_t (as given)
-    float *Vr = Kr + C * KP;         // [C][KP] v_t
-    float *Xr = Vr + C * KP;         // [C][KP] x_t
-    float *Yr = Xr + C * KP;         // [C][KP] y_t
-    float *Gr = Yr + C * KP;         // [C][KP] g_t = dL/do_t
-    float *KX = Gr + C * KP;         // [C][CP] k_l . x_s
-    float *KY = KX + C * CP;         // [C][CP] k_l . y_s
-    float *VG = KY + C * CP;         // [C][CP] v_l . g_s
-    float *GK = VG + C * CP;         // [C][CP] k_l . k_i
-    float *Wt = GK + C * CP;         // [C][CP] w_sl at [l][s], 0 for s < l
-    float *Py = Wt + C * CP;         // [C][CP] coefficient matrices of the row outputs
-    float *Px = Py + C * CP;
-    float *Pk = Px + C * CP;
-    float *Pg = Pk + C * CP;
-    float *Qm = Pg + C * CP;         // [C][CP] Q[i][s], then w_sj Phi[j][s]
-    float *A0 = Qm + C * CP;         // [C][KP] dL/dk~ with the own row unwritten
-    float *B0 = A0 + C * KP;         // [C][KP] dL/dv~ likewise
-    __shared__ double ell[256], wtot[kSimtThreads / 32];
-    __shared__ float s_b[32], s_step[32], s_wend[32], s_w[32], s_c[32], s_f[32], s_R[32];
-    __shared__ float s_uk[32], s_yhx[32], s_gmx[32], s_qe[32], s_X1[32], s_bm1[32];
+    float *Kr = sm;                          // [C][KP] k_t (as given)
+    float *Xr = Kr + L::rows;                // [C][KP] x_t
+    float *Yr = Xr + L::rows;                // [C][KP] y_t
+    float *Gr = Yr + L::rows;                // [C][KP] g_t = dL/do_t
+    float *Un = Gr + L::rows;                // v rows, then Py Px Pk Pg
+    float *Vr = Un;
+    float *Py = Un, *Px = Py + L::mats, *Pk = Px + L::mats, *Pg = Pk + L::mats;
+    float *KX = Un + L::union_floats;        // [C][CP] k_l . x_s
+    float *KY = KX + L::mats;                // [C][CP] k_l . y_s
+    float *VG = KY + L::mats;                // [C][CP] v_l . g_s
+    float *GK = VG + L::mats;                // [C][CP] k_l . k_i
+    float *Wt = GK + L::mats;                // [C][CP] w_sl at [l][s], 0 for s < l
+    float *Qm = Wt + L::mats;                // [C][CP] Q[i][s]
+    __shared__ double ell[C], wtot[kSimtThreads / 32];
+    __shared__ float s_b[C], s_step[C], s_wend[C], s_w[C], s_c[C], s_f[C], s_R[C];
+    __shared__ float s_uk[C], s_yhx[C], s_gmx[C], s_qe[C], s_X1[C], s_bm1[C];
 
     const int n = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
     const int lane = tid & 31, warp = tid >> 5;
@@ -619,18 +628,40 @@ k_bwd_grads(const Tin *__restrict__ k, const Tin *__restrict__ v, const float *_
         Gr[t * KP + d] = load_f(dout + g);
     }
     for (int e = tid; e < C * C; e += kSimtThreads) {
-        const int l = e / C, s = e % C;
-        Wt[l * CP + s] = s >= l ? decay_exp(ell[s] - ell[l]) : 0.f;
+        const int l = e / C, s2 = e % C;
+        Wt[l * CP + s2] = s2 >= l ? decay_exp(ell[s2] - ell[l]) : 0.f;
     }
     __syncthreads();
-    // dot-product matrices
-    for (int e = tid; e < 4 * C * C; e += kSimtThreads) {
-        const int m = e / (C * C), l = (e / C) % C, s = e % C;
-        const float *A = (m == 1 || m == 3 || m == 0) ? Kr : Vr;
+    // dot-product matrices: 64 threads per matrix, a TI x TI tile each
+    {
+        const int m = tid >> 6, q = tid & 63, lt = q >> 3, st = q & 7;
+        const float *A = m == 2 ? Vr : Kr;
         const float *B = m == 0 ? Xr : (m == 1 ? Yr : (m == 2 ? Gr : Kr));
-        float acc = 0.f;
-        for (int d = 0; d < D; ++d) acc = fmaf(A[l * KP + d], B[s * KP + d], acc);
-        (m == 0 ? KX : m == 1 ? KY : m == 2 ? VG : GK)[l * CP + s] = acc;
+        float acc[TI][TI];
+#pragma unroll
+        for (int i = 0; i < TI; ++i)
+#pragma unroll
+            for (int j = 0; j < TI; ++j) acc[i][j] = 0.f;
+#pragma unroll 2
+        for (int d = 0; d < D; d += 4) {
+            float4 a4[TI], b4[TI];
+#pragma unroll
+            for (int i = 0; i < TI; ++i) {
+                a4[i] = *reinterpret_cast<const float4 *>(A + (lt + 8 * i) * KP + d);
+                b4[i] = *reinterpret_cast<const float4 *>(B + (st + 8 * i) * KP + d);
+            }
+#pragma unroll
+            for (int i = 0; i < TI; ++i)
+#pragma unroll
+                for (int j = 0; j < TI; ++j)
+                    acc[i][j] = fmaf(a4[i].x, b4[j].x, fmaf(a4[i].y, b4[j].y,
+                                fmaf(a4[i].z, b4[j].z, fmaf(a4[i].w, b4[j].w, acc[i][j]))));
+        }
+        float *dst = m == 0 ? KX : (m == 1 ? KY : (m == 2 ? VG : GK));
+#pragma unroll
+        for (int i = 0; i < TI; ++i)
+#pragma unroll
+            for (int j = 0; j < TI; ++j) dst[(lt + 8 * i) * CP + st + 8 * j] = acc[i][j];
     }
     if (tid == 0) {
         // f_l = sum_{s>=l} w_sl c_s b_s and R_m = sum_{s>=m} c_s w_sm^2 (suffix recurrences)
@@ -644,54 +675,83 @@ k_bwd_grads(const Tin *__restrict__ k, const Tin *__restrict__ v, const float *_
         }
         // X1_s = sum_{l<=s} w_sl w_l uk_l (the written keys' H_s quadratic forms)
         float x1 = 0.f;
-        for (int s = 0; s < C; ++s) {
-            x1 = fmaf(s == 0 ? 0.f : s_step[s], x1, s_w[s] * s_uk[s]);
-            s_X1[s] = x1;
+        for (int s2 = 0; s2 < C; ++s2) {
+            x1 = fmaf(s2 == 0 ? 0.f : s_step[s2], x1, s_w[s2] * s_uk[s2]);
+            s_X1[s2] = x1;
         }
     }
-    __syncthreads();
-    // coefficient matrices of the row outputs
+    __syncthreads();   // dot matrices complete; the v rows are dead from here on
+    // coefficient matrices of the row outputs (over the v rows)
     for (int e = tid; e < C * C; e += kSimtThreads) {
-        const int l = e / C, s = e % C;
-        const float w = Wt[l * CP + s];
-        Py[l * CP + s] = -w * KX[l * CP + s];
-        Px[l * CP + s] = w * (VG[l * CP + s] - KY[l * CP + s]);
-        Pg[l * CP + s] = w * KX[l * CP + s];
-        // Mw[l][i] = R_m w_ml w_mi, m = max(l, i); here i = s
-        const int m = l > s ? l : s;
-        const float wml = Wt[l * CP + m], wmi = Wt[s * CP + m];
-        Pk[l * CP + s] = -2.f * s_R[m] * wml * wmi * s_w[s] * GK[l * CP + s];
+        const int l = e / C, s2 = e % C;
+        const float w = Wt[l * CP + s2];
+        Py[l * CP + s2] = -w * KX[l * CP + s2];
+        Px[l * CP + s2] = w * (VG[l * CP + s2] - KY[l * CP + s2]);
+        Pg[l * CP + s2] = w * KX[l * CP + s2];
+        // Mw[l][i] = R_m w_ml w_mi, m = max(l, i); here i = s2
+        const int m = l > s2 ? l : s2;
+        Pk[l * CP + s2] = -2.f * s_R[m] * Wt[l * CP + m] * Wt[s2 * CP + m] * s_w[s2] * GK[l * CP + s2];
     }
     // Q[i][s] = sum_{l<=s} w_sl w_l w_i (k_l . k_i)^2, thread i over s
     if (tid < C) {
         const int i = tid;
         float qv = 0.f;
-        for (int s = 0; s < C; ++s) {
-            const float g2 = GK[s * CP + i];
-            qv = fmaf(s == 0 ? 0.f : s_step[s], qv, s_w[s] * s_w[i] * g2 * g2);
-            Qm[i * CP + s] = qv;
+        for (int s2 = 0; s2 < C; ++s2) {
+            const float g2 = GK[s2 * CP + i];
+            qv = fmaf(s2 == 0 ? 0.f : s_step[s2], qv, s_w[s2] * s_w[i] * g2 * g2);
+            Qm[i * CP + s2] = qv;
         }
     }
     __syncthreads();
-    // row outputs: thread (column c, token group) over tokens l
+    // row outputs: warp w takes tokens w + 8i, lane the columns lane + 32b
     {
-        const int c = tid % D;
-        for (int l = tid / D; l < C; l += kSimtThreads / D) {
-            float a0 = 0.f, b0 = 0.f;
-            for (int s = 0; s < C; ++s) {
-                a0 = fmaf(Py[l * CP + s], Yr[s * KP + c], a0);
-                a0 = fmaf(Px[l * CP + s], Xr[s * KP + c], a0);
-                a0 = fmaf(Pk[l * CP + s], Kr[s * KP + c], a0);
-                b0 = fmaf(Pg[l * CP + s], Gr[s * KP + c], b0);
+        float a0[TI][CC], b0[TI][CC];
+#pragma unroll
+        for (int i = 0; i < TI; ++i)
+#pragma unroll
+            for (int b = 0; b < CC; ++b) a0[i][b] = b0[i][b] = 0.f;
+#pragma unroll 4
+        for (int s2 = 0; s2 < C; ++s2) {
+            float yv[CC], xv[CC], kv[CC], gv[CC];
+#pragma unroll
+            for (int b = 0; b < CC; ++b) {
+                const int c = lane + 32 * b;
+                yv[b] = Yr[s2 * KP + c];
+                xv[b] = Xr[s2 * KP + c];
+                kv[b] = Kr[s2 * KP + c];
+                gv[b] = Gr[s2 * KP + c];
             }
-            const size_t g = (tok0 + l) * D + c;
-            a0 = fmaf(-2.f * s_f[l], R[g], a0);
-            a0 = fmaf(s_wend[l], R[RD + g] + R[2 * RD + g], a0);
-            b0 = fmaf(s_wend[l], R[3 * RD + g], b0);
-            A0[l * KP + c] = a0;
-            B0[l * KP + c] = b0;
-            store_f(dk + g, s_w[l] * a0);
-            store_f(dv + g, s_w[l] * b0);
+#pragma unroll
+            for (int i = 0; i < TI; ++i) {
+                const int l = warp + 8 * i;
+                const float py = Py[l * CP + s2], px = Px[l * CP + s2], pk = Pk[l * CP + s2],
+                            pg = Pg[l * CP + s2];
+#pragma unroll
+                for (int b = 0; b < CC; ++b) {
+                    a0[i][b] = fmaf(py, yv[b], fmaf(px, xv[b], fmaf(pk, kv[b], a0[i][b])));
+                    b0[i][b] = fmaf(pg, gv[b], b0[i][b]);
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < TI; ++i) {
+            const int l = warp + 8 * i;
+            const size_t row = (tok0 + l) * D;
+            float dgp = 0.f;
+#pragma unroll
+            for (int b = 0; b < CC; ++b) {
+                const int c = lane + 32 * b;
+                const size_t g = row + c;
+                float a = fmaf(-2.f * s_f[l], R[g], a0[i][b]);
+                a = fmaf(s_wend[l], R[RD + g] + R[2 * RD + g], a);
+                const float bb = fmaf(s_wend[l], R[3 * RD + g], b0[i][b]);
+                store_f(dk + g, s_w[l] * a);
+                store_f(dv + g, s_w[l] * bb);
+                dgp = fmaf(Kr[l * KP + c], a, fmaf(load_f(v + g), bb, dgp));
+            }
+            // write-gate gradient: (k . A0 + v . B0) / 2 over the row
+            dgp = warp_sum(dgp);
+            if (dgate && lane == 0) dgate[tok0 + l] = 0.5f * dgp;
         }
     }
     // dbeta_j = sum_{s>=j} w_sj Phi[j][s] + (adjoint from later chunks), with
@@ -701,45 +761,34 @@ k_bwd_grads(const Tin *__restrict__ k, const Tin *__restrict__ v, const float *_
     // matrices and of Q) and stores w_sj Phi[j][s] into Py[j][s] (free by now).
     __syncthreads();
     if (tid < C) {
-        const int s = tid;
+        const int s2 = tid;
         float t1 = 0.f, t2 = 0.f, t3 = 0.f, u1 = 0.f;
-        for (int j = 0; j <= s; ++j) {
+        for (int j = 0; j <= s2; ++j) {
             if (j > 0) {
                 const int i = j - 1;
                 const float st = s_step[i];
-                t1 = fmaf(st, t1, s_w[i] * KY[i * CP + s] * KX[i * CP + s]);
-                t3 = fmaf(st, t3, s_w[i] * VG[i * CP + s] * KX[i * CP + s]);
-                t2 = fmaf(st, t2, Qm[i * CP + s]);
+                t1 = fmaf(st, t1, s_w[i] * KY[i * CP + s2] * KX[i * CP + s2]);
+                t3 = fmaf(st, t3, s_w[i] * VG[i * CP + s2] * KX[i * CP + s2]);
+                t2 = fmaf(st, t2, Qm[i * CP + s2]);
                 u1 = fmaf(st, u1, s_w[i] * s_uk[i]);
             }
             const float bm = s_bm1[j];
-            const float phi = -(bm * s_yhx[s] + t1)
-                              - s_c[s] * (s_b[s] * bm * hs2 + s_b[s] * u1 + bm * s_X1[s] + t2)
-                              + (bm * s_gmx[s] + t3);
-            Py[j * CP + s] = Wt[j * CP + s] * phi;   // w_sj Phi[j][s]
+            const float phi = -(bm * s_yhx[s2] + t1)
+                              - s_c[s2] * (s_b[s2] * bm * hs2 + s_b[s2] * u1 + bm * s_X1[s2] + t2)
+                              + (bm * s_gmx[s2] + t3);
+            Py[j * CP + s2] = Wt[j * CP + s2] * phi;   // w_sj Phi[j][s]
         }
     }
     __syncthreads();
     if (tid < C) {
         const int j = tid;
         float acc = 0.f;
-        for (int s = j; s < C; ++s) acc += Py[j * CP + s];
+        for (int s2 = j; s2 < C; ++s2) acc += Py[j * CP + s2];
         // the adjoint from later chunks: w_{C-1,j} (b_{j-1} eh + sum_{i<j} w_{j-1,i} w_i qe_i)
         float qe = 0.f;
         for (int i = 0; i < j; ++i) qe = fmaf(s_step[i], qe, s_w[i] * s_qe[i]);
         acc = fmaf(s_wend[j], fmaf(s_bm1[j], eh, qe), acc);
         dbeta[tok0 + j] = acc;
-    }
-    __syncthreads();
-    // write-gate gradient: (k . A0 + v . B0) / 2, one warp per token
-    if (dgate) {
-        for (int t = warp; t < C; t += kSimtThreads / 32) {
-            float s = 0.f;
-            for (int d = lane; d < D; d += 32)
-                s = fmaf(Kr[t * KP + d], A0[t * KP + d], fmaf(Vr[t * KP + d], B0[t * KP + d], s));
-            s = warp_sum(s);
-            if (lane == 0) dgate[tok0 + t] = 0.5f * s;
-        }
     }
 }
 

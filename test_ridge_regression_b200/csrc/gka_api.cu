@@ -498,11 +498,19 @@ static int backward_simt(const Tin *q, const Tin *k, const Tin *v, const float *
     }
     if (int rc = check_launch()) return rc;
     // gradients
-    const size_t sm_gr = BwdGradSmem<D>::bytes(C);
-    if ((e = set_smem(k_bwd_grads<Tin, D>, sm_gr)) != cudaSuccess) return cuda_fail(e);
-    { ProfScope ps(GKA_KERNEL_BWD_GRADS, s);
-    k_bwd_grads<Tin, D><<<dim3(N, BH), kSimtThreads, sm_gr, s>>>(
-        k, v, beta, gate, dout, xs, ys, cvec, rows, tokq, chq, dk, dv, dbeta, dgate, T, N, C); }
+    if (C == 16) {
+        constexpr size_t sm_gr = BwdGradSmem<D, 16>::bytes;
+        if ((e = set_smem(k_bwd_grads<Tin, D, 16>, sm_gr)) != cudaSuccess) return cuda_fail(e);
+        ProfScope ps(GKA_KERNEL_BWD_GRADS, s);
+        k_bwd_grads<Tin, D, 16><<<dim3(N, BH), kSimtThreads, sm_gr, s>>>(
+            k, v, beta, gate, dout, xs, ys, cvec, rows, tokq, chq, dk, dv, dbeta, dgate, T, N);
+    } else {
+        constexpr size_t sm_gr = BwdGradSmem<D, 32>::bytes;
+        if ((e = set_smem(k_bwd_grads<Tin, D, 32>, sm_gr)) != cudaSuccess) return cuda_fail(e);
+        ProfScope ps(GKA_KERNEL_BWD_GRADS, s);
+        k_bwd_grads<Tin, D, 32><<<dim3(N, BH), kSimtThreads, sm_gr, s>>>(
+            k, v, beta, gate, dout, xs, ys, cvec, rows, tokq, chq, dk, dv, dbeta, dgate, T, N);
+    }
     return check_launch();
 }
 
