@@ -386,36 +386,137 @@ k_adjoint_scan(float *__restrict__ adj, const float *__restrict__ decay, int N, 
 //   (rows of [B*H*T, D] each), and per token uk_t = k_t^T H_s k_t,
 //   yhx_t = y_t^T H_s x_t, gmx_t = g_t^T M_s x_t, qe_t = k_t^T E^H k_t + v_t^T E^M k_t;
 //   per chunk hs2 = ||H_s||_F^2 and eh = <E^H, H_s> + <E^M, M_s>.
-// Every product is out[t][c] = sum_d row_t[d] Mt[d][c] with the matrix staged in
-// shared memory in the orientation it needs (E^M transposed for R4, E^H
-// symmetrised for R2).  Warp w computes tokens w*C/8.., lane l the columns
-// l, l + 32, .. (conflict-free), in registers, reading 4 d at a time.
-// grid (N, B*H), block 256, shared memory BwdRowsSmem<D, C>::bytes.
+// Every product is out[t][c] = sum_d row_t[d] Mt[d][c], the matrix staged in
+// shared memory half a column range at a time in the orientation the product
+// needs (E^M transposed for R4, E^H symmetrised for R2).  Warp w computes tokens
+// w*C/8.., lane l the columns l and l + 32 of the half, in registers; the
+// per-token dots are reduced from the registers.  k, v and g rows are kept as
+// their bf16 values when the inputs are bf16 (exact).
+// grid (N, B*H), block 256, shared memory BwdRowsSmem<Tin, D, C>::bytes (two CTAs
+// per SM at D = 128, C = 32).
 // ---------------------------------------------------------------------------
-template <int D, int C>
+template <typename Tin, int D, int C>
 struct BwdRowsSmem {
-    static constexpr int DP = D + 4;   // 16-byte aligned rows
-    static constexpr size_t bytes = sizeof(float) * ((size_t)D * DP + 6 * (size_t)C * D);
+    static constexpr int NH = D >= 64 ? 2 : 1;   // column ranges staged one after another
+    static constexpr int HC = D / NH;            // columns per staged range
+    static constexpr int DP = HC + 4;         // 16-byte aligned rows
+    static constexpr size_t mat = sizeof(float) * (size_t)D * DP;
+    static constexpr size_t in_rows = sizeof(Tin) * (size_t)C * D;     // k, v, g
+    static constexpr size_t f_rows = sizeof(float) * (size_t)C * D;    // x, y
+    static constexpr size_t bytes = mat + 3 * in_rows + 2 * f_rows;
 };
 
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// Mt[d][c'] = A'[d][h*HC + c'] for the column range h, A' = A (mode 0), A^T (1),
+// A + A^T (2); global reads are coalesced in every mode.  All threads call it.
+template <int D, int HC, int DP>
+__device__ __forceinline__ void bwd_stage(float *Mt, const float *__restrict__ A, int mode, int h) {
+    const int tid = threadIdx.x;
+    __syncthreads();
+    if (mode != 1) {
+        for (int e = tid; e < D * HC; e += kSimtThreads) {
+            const int d = e / HC, c = e % HC;
+            Mt[d * DP + c] = A[d * D + h * HC + c];
+        }
+    }
+    if (mode == 2) __syncthreads();
+    if (mode != 0) {
+        for (int e = tid; e < HC * D; e += kSimtThreads) {
+            const int c = e / D, d = e % D;
+            const float x = A[(h * HC + c) * D + d];
+            Mt[d * DP + c] = mode == 2 ? Mt[d * DP + c] + x : x;
+        }
+    }
+    __syncthreads();
+}
+
+// For the column range h staged in Mt: out[t][h*HC + c] = sum_d rows[t][d] Mt[d][c]
+// over this warp's TT tokens and this lane's CC columns; written to R + gout (if
+// gout != -1) and its dot with dotB[t][.] added to dacc.
+template <int D, int HC, int DP, int TT, typename RowT, typename DotT>
+__device__ __forceinline__ void bwd_half_product(const float *Mt, const RowT *rows,
+                                                 const DotT *dotB, int h, float *__restrict__ R,
+                                                 size_t gout, size_t tok0, float (&dacc)[TT]) {
+    constexpr int CC = HC / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float acc[TT][CC];
+#pragma unroll
+    for (int a = 0; a < TT; ++a)
+#pragma unroll
+        for (int b = 0; b < CC; ++b) acc[a][b] = 0.f;
+    const int t0 = warp * TT;
+#pragma unroll 2
+    for (int d = 0; d < D; d += 4) {
+        float m[4][CC];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int b = 0; b < CC; ++b) m[u][b] = Mt[(d + u) * DP + lane + 32 * b];
+#pragma unroll
+        for (int a = 0; a < TT; ++a) {
+            float r[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) r[u] = to_f(rows[(t0 + a) * D + d + u]);
+#pragma unroll
+            for (int b = 0; b < CC; ++b)
+                acc[a][b] = fmaf(r[0], m[0][b], fmaf(r[1], m[1][b],
+                            fmaf(r[2], m[2][b], fmaf(r[3], m[3][b], acc[a][b]))));
+        }
+    }
+#pragma unroll
+    for (int a = 0; a < TT; ++a)
+#pragma unroll
+        for (int b = 0; b < CC; ++b) {
+            const int p = (t0 + a) * D + h * HC + lane + 32 * b;
+            if (gout != (size_t)-1) R[gout + tok0 * D + p] = acc[a][b];
+            dacc[a] = fmaf(acc[a][b], to_f(dotB[p]), dacc[a]);
+        }
+}
+
+// One product over all column ranges; the per-token dot (times scale) written to
+// dst[tok0 + t] (or added), unless dst is null.
+template <int D, int HC, int DP, int NH, int TT, typename RowT, typename DotT>
+__device__ __forceinline__ void bwd_product(float *Mt, const float *__restrict__ A, int mode,
+                                            const RowT *rows, size_t gout, const DotT *dotB,
+                                            float *dst, float scale, bool add,
+                                            float *__restrict__ R, size_t tok0) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float dacc[TT];
+#pragma unroll
+    for (int a = 0; a < TT; ++a) dacc[a] = 0.f;
+    for (int h = 0; h < NH; ++h) {
+        bwd_stage<D, HC, DP>(Mt, A, mode, h);
+        bwd_half_product<D, HC, DP, TT>(Mt, rows, dotB, h, R, gout, tok0, dacc);
+    }
+#pragma unroll
+    for (int a = 0; a < TT; ++a) {
+        const float s = warp_sum(dacc[a]) * scale;
+        if (dst && lane == 0) {
+            const size_t t = tok0 + warp * TT + a;
+            dst[t] = add ? dst[t] + s : s;
+        }
+    }
+}
+
 template <typename Tin, int D, int C>
-__global__ void __launch_bounds__(kSimtThreads)
+__global__ void __launch_bounds__(kSimtThreads, 2)
 k_bwd_rows(const Tin *__restrict__ k, const Tin *__restrict__ v, const Tin *__restrict__ dout,
            const float *__restrict__ states, const float *__restrict__ adj,
            const float *__restrict__ xs, const float *__restrict__ ys, float *__restrict__ R,
            float *__restrict__ tokq, float *__restrict__ chq, int T, int N) {
-    constexpr int DP = BwdRowsSmem<D, C>::DP;
+    using L = BwdRowsSmem<Tin, D, C>;
+    constexpr int HC = L::HC, DP = L::DP, NH = L::NH;
     constexpr int TT = C / 8;          // tokens per warp
-    constexpr int CC = D / 32;         // columns per lane
-    static_assert(kSimtThreads == 256 && C % 8 == 0 && D % 32 == 0, "tiling");
-    extern __shared__ __align__(16) float sm[];
-    float *Mt = sm;              // [D][DP] one matrix at a time
-    float *Kr = Mt + D * DP;     // [C][D] k_t
-    float *Vr = Kr + C * D;      // [C][D] v_t
-    float *Xr = Vr + C * D;      // [C][D] x_t
-    float *Yr = Xr + C * D;      // [C][D] y_t
-    float *Gr = Yr + C * D;      // [C][D] g_t
-    float *Tr = Gr + C * D;      // [C][D] a product, reduced per token
+    static_assert(kSimtThreads == 256 && C % 8 == 0 && HC % 32 == 0, "tiling");
+    extern __shared__ __align__(16) uint8_t smb[];
+    float *Mt = reinterpret_cast<float *>(smb);                       // [D][DP] staged columns
+    Tin *Kr = reinterpret_cast<Tin *>(smb + L::mat);                  // [C][D] k_t
+    Tin *Vr = Kr + C * D;                                             // [C][D] v_t
+    Tin *Gr = Vr + C * D;                                             // [C][D] g_t
+    float *Xr = reinterpret_cast<float *>(smb + L::mat + 3 * L::in_rows);   // [C][D] x_t
+    float *Yr = Xr + C * D;                                                 // [C][D] y_t
     __shared__ float red[2][kSimtThreads / 32];
 
     const int n = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
@@ -427,11 +528,11 @@ k_bwd_rows(const Tin *__restrict__ k, const Tin *__restrict__ v, const Tin *__re
     const float *EH = adj + ((size_t)bh * (N + 1) + n) * 2 * D * D, *EM = EH + D * D;
     for (int e = tid; e < C * D; e += kSimtThreads) {
         const size_t g = tok0 * D + e;
-        Kr[e] = load_f(k + g);
-        Vr[e] = load_f(v + g);
+        Kr[e] = k[g];
+        Vr[e] = v[g];
+        Gr[e] = dout[g];
         Xr[e] = xs[g];
         Yr[e] = ys[g];
-        Gr[e] = load_f(dout + g);
     }
     {
         float h2 = 0.f, eh = 0.f;
@@ -453,95 +554,21 @@ k_bwd_rows(const Tin *__restrict__ k, const Tin *__restrict__ v, const Tin *__re
         for (int w = 0; w < kSimtThreads / 32; ++w) s += red[tid][w];
         chq[((size_t)bh * N + n) * 2 + tid] = s;
     }
-    // mode 0: Mt[d][c] = A[d][c]; 1: A[c][d]; 2: A[d][c] + A[c][d] (coalesced reads of A)
-    auto load_mat = [&](const float *A, int mode) {
-        __syncthreads();
-        for (int e = tid; e < D * D; e += kSimtThreads) {
-            const int r = e / D, c = e % D;
-            if (mode == 1) Mt[c * DP + r] = A[e];
-            else Mt[r * DP + c] = A[e];
-        }
-        __syncthreads();
-        if (mode == 2) {
-            for (int e = tid; e < D * D; e += kSimtThreads) {
-                const int r = e / D, c = e % D;
-                if (r < c) {
-                    const float x = Mt[r * DP + c] + Mt[c * DP + r];
-                    Mt[r * DP + c] = x;
-                    Mt[c * DP + r] = x;
-                } else if (r == c) {
-                    Mt[r * DP + c] *= 2.f;
-                }
-            }
-            __syncthreads();
-        }
-    };
-    // out[t][c] = sum_d rows[t][d] Mt[d][c] for this thread's TT x CC tile; written to
-    // shared memory (out) and/or the global array at gout
-    auto rows_times = [&](const float *rows, float *out, size_t gout) {
-        float acc[TT][CC];
-#pragma unroll
-        for (int a = 0; a < TT; ++a)
-#pragma unroll
-            for (int b = 0; b < CC; ++b) acc[a][b] = 0.f;
-        const int t0 = warp * TT;
-#pragma unroll 2
-        for (int d = 0; d < D; d += 4) {
-            float m[4][CC];
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-#pragma unroll
-                for (int b = 0; b < CC; ++b) m[u][b] = Mt[(d + u) * DP + lane + 32 * b];
-#pragma unroll
-            for (int a = 0; a < TT; ++a) {
-                const float4 r4 = *reinterpret_cast<const float4 *>(rows + (t0 + a) * D + d);
-#pragma unroll
-                for (int b = 0; b < CC; ++b)
-                    acc[a][b] = fmaf(r4.x, m[0][b], fmaf(r4.y, m[1][b],
-                                fmaf(r4.z, m[2][b], fmaf(r4.w, m[3][b], acc[a][b]))));
-            }
-        }
-#pragma unroll
-        for (int a = 0; a < TT; ++a)
-#pragma unroll
-            for (int b = 0; b < CC; ++b) {
-                const int p = (t0 + a) * D + lane + 32 * b;
-                if (out) out[p] = acc[a][b];
-                if (gout != (size_t)-1) R[gout + tok0 * D + p] = acc[a][b];
-            }
-    };
-    // per-token dot of two [C][D] arrays in shared memory, one warp per token
-    auto tok_dot = [&](const float *A, const float *B, float *dst, float scale, bool add) {
-        __syncthreads();
-        for (int t = warp; t < C; t += kSimtThreads / 32) {
-            float s = 0.f;
-            for (int d = lane; d < D; d += 32) s = fmaf(A[t * D + d], B[t * D + d], s);
-            s = warp_sum(s) * scale;
-            if (lane == 0) dst[tok0 + t] = add ? dst[tok0 + t] + s : s;
-        }
-        __syncthreads();
-    };
-    // H_s (symmetric): R1 = K H_s, uk = k . R1; x^T H_s -> yhx
-    load_mat(Hs, 0);
-    rows_times(Kr, Tr, 0);
-    tok_dot(Tr, Kr, tokq, 1.f, false);
-    rows_times(Xr, Tr, (size_t)-1);
-    tok_dot(Tr, Yr, tokq + plane, 1.f, false);
+    constexpr size_t none = (size_t)-1;
+    // H_s (symmetric): R1 = K H_s with uk = k . R1; x^T H_s with yhx = (x^T H_s) . y
+    bwd_product<D, HC, DP, NH, TT>(Mt, Hs, 0, Kr, 0, Kr, tokq, 1.f, false, R, tok0);
+    bwd_product<D, HC, DP, NH, TT>(Mt, Hs, 0, Xr, none, Yr, tokq + plane, 1.f, false, R, tok0);
     // M_s: g^T M_s x = (g^T M_s) . x
-    load_mat(Mst, 0);
-    rows_times(Gr, Tr, (size_t)-1);
-    tok_dot(Tr, Xr, tokq + 2 * plane, 1.f, false);
+    bwd_product<D, HC, DP, NH, TT>(Mt, Mst, 0, Gr, none, Xr, tokq + 2 * plane, 1.f, false, R,
+                                   tok0);
     // E^H + E^H^T: R2, qe = k^T E^H k = (k . R2) / 2
-    load_mat(EH, 2);
-    rows_times(Kr, Tr, RD);
-    tok_dot(Tr, Kr, tokq + 3 * plane, 0.5f, false);
-    // E^M: R3 = rows v^T E^M
-    load_mat(EM, 0);
-    rows_times(Vr, nullptr, 2 * RD);
+    bwd_product<D, HC, DP, NH, TT>(Mt, EH, 2, Kr, RD, Kr, tokq + 3 * plane, 0.5f, false, R, tok0);
+    // E^M: R3 = rows v^T E^M (its dot is not needed)
+    bwd_product<D, HC, DP, NH, TT>(Mt, EM, 0, Vr, 2 * RD, Vr, (float *)nullptr, 0.f, false, R,
+                                   tok0);
     // E^M^T: R4 = rows k^T E^M^T = (E^M k)^T; qe += v . R4
-    load_mat(EM, 1);
-    rows_times(Kr, Tr, 3 * RD);
-    tok_dot(Tr, Vr, tokq + 3 * plane, 1.f, true);
+    bwd_product<D, HC, DP, NH, TT>(Mt, EM, 1, Kr, 3 * RD, Vr, tokq + 3 * plane, 1.f, true, R,
+                                   tok0);
 }
 
 // ---------------------------------------------------------------------------

@@ -484,13 +484,13 @@ static int backward_simt(const Tin *q, const Tin *k, const Tin *v, const float *
     if (int rc = check_launch()) return rc;
     // the chunk rows against H_s, M_s and the adjoints
     if (C == 16) {
-        constexpr size_t sm_rows = BwdRowsSmem<D, 16>::bytes;
+        constexpr size_t sm_rows = BwdRowsSmem<Tin, D, 16>::bytes;
         if ((e = set_smem(k_bwd_rows<Tin, D, 16>, sm_rows)) != cudaSuccess) return cuda_fail(e);
         ProfScope ps(GKA_KERNEL_BWD_ROWS, s);
         k_bwd_rows<Tin, D, 16><<<dim3(N, BH), kSimtThreads, sm_rows, s>>>(
             k, v, dout, states, adj, xs, ys, rows, tokq, chq, T, N);
     } else {
-        constexpr size_t sm_rows = BwdRowsSmem<D, 32>::bytes;
+        constexpr size_t sm_rows = BwdRowsSmem<Tin, D, 32>::bytes;
         if ((e = set_smem(k_bwd_rows<Tin, D, 32>, sm_rows)) != cudaSuccess) return cuda_fail(e);
         ProfScope ps(GKA_KERNEL_BWD_ROWS, s);
         k_bwd_rows<Tin, D, 32><<<dim3(N, BH), kSimtThreads, sm_rows, s>>>(
