@@ -323,14 +323,14 @@ static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
 
     if (C == 64) {
         // one CTA per 64-token chunk
-        auto kern = k_chunk_solve_tc<64, 64>;
+        auto kern = x_out ? k_chunk_solve_tc<64, 64, true> : k_chunk_solve_tc<64, 64, false>;
         if ((e = set_smem(kern, TcSmem<64, 64>::bytes)) != cudaSuccess) return cuda_fail(e);
         ProfScope ps(GKA_KERNEL_CHUNK_SOLVE_TC, s);
         kern<<<dim3(N, BH), kSolveThreads, TcSmem<64, 64>::bytes, s>>>(
             maps, q, gate, tokdec, plane, norms, sexp, o, x_out, T, N, C, P, flag);
     } else {
         // one CTA per 128-token chunk (N = 128 MMAs)
-        auto kern = k_chunk_solve_tc<128, 128>;
+        auto kern = x_out ? k_chunk_solve_tc<128, 128, true> : k_chunk_solve_tc<128, 128, false>;
         if ((e = set_smem(kern, TcSmem<128, 128>::bytes)) != cudaSuccess) return cuda_fail(e);
         ProfScope ps(GKA_KERNEL_CHUNK_SOLVE_TC, s);
         kern<<<dim3(N, BH), kSolveThreads, TcSmem<128, 128>::bytes, s>>>(

@@ -269,7 +269,7 @@ __device__ __forceinline__ void reduce_scatter32(float (&v)[N], int lane) {
 // every MMA has N = 128).  8 warps: warpgroup wg (warps 4wg..4wg+3) owns tokens
 // wg*TOK/2 .. (wg+1)*TOK/2 - 1; warp w reads TMEM lane quarter w % 4, so thread
 // (wg, d) owns element d of the iterates of its TOK/2 tokens.
-template <int MG, int TOK>
+template <int MG, int TOK, bool XOUT = false>
 __global__ void __launch_bounds__(kSolveThreads, TOK == 64 ? 2 : 1)
 k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__restrict__ q,
                  const float *__restrict__ gate, const float *__restrict__ tokdec, size_t plane, float *__restrict__ norms,
@@ -652,9 +652,9 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     // warps 1-7 form P, warp 4 also covering warp 0's lane quarter, and warp 4
     // issues Z3.  The P warps and the Z3 issuer meet at a named barrier, so Z3 =
     // K^T P^T (commit bar_z) need not wait for the Z1 issue to finish.
-    // With x_out (nullable, fp32 [B*H*T][128]) the rounds stop before the readout
-    // pass and the iterates x_j themselves are written (the backward recomputes them).
-    const int last_it = x_out ? P.r - 1 : P.r;
+    // XOUT (x_out: fp32 [B*H*T][128]): the rounds stop before the readout pass and the
+    // iterates x_j themselves are written (the backward recomputes them this way).
+    const int last_it = XOUT ? P.r - 1 : P.r;
 #pragma unroll 1
     for (int it = 1; it <= last_it && ok; ++it) {
         const bool out_pass = (it == P.r);
@@ -748,7 +748,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         if (!mbar_wait_sleep(bar_z1, ph, kTcSleepProbes, kTcSleepNs)) ok = false;
         tc::fence_after_sync();
         if (!out_pass) {
-            if (tid == 0 && it == P.r - 1 && !x_out) {
+            if (tid == 0 && it == P.r - 1 && !XOUT) {
                 // H_s is no longer read: fetch M_s for the readout into the same buffer
                 mbar_arrive_expect_tx(bar_m, 32768);
                 for (int h = 0; h < 2; ++h)
@@ -842,7 +842,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         }
     }
 
-    if (x_out && ok) {
+    if (XOUT && ok) {
         // x_j = x~_j invd_j / sigma, invd_j = c3_j sK^2 (thread (wg, d): element d of
         // its tokens; consecutive d of a token are consecutive threads)
         const float xs = sK * sK / sigma;
