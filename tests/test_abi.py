@@ -28,6 +28,7 @@ def declared_functions():
 def test_header_declares_entry_points():
     names = declared_functions()
     for must in ["gka_forward", "gka_decode_step", "gka_forward_gated", "gka_decode_step_gated",
+                 "gka_backward", "gka_backward_workspace_bytes",
                  "gka_forward_workspace_bytes",
                  "gka_forward_workspace_layout", "gka_device_status", "gka_last_cuda_error",
                  "gka_status_string", "gka_version"]:
@@ -117,6 +118,27 @@ def test_gated_entry_points_validate_like_the_ungated_ones(lib):
     assert decg(D=96) == -2
     assert decg(r=0) == -1
     assert decg(gate=FAKE_MIS) == -7
+
+
+def test_backward_argument_errors(lib):
+    def bwd(gate=None, dgate=None, T=128, D=64, C=32, r=4, q=FAKE, ws_bytes=1 << 40, B=1):
+        return lib.gka_backward(q, FAKE, FAKE, FAKE, gate, FAKE, FAKE, FAKE, FAKE, FAKE, dgate,
+                                B, 1, T, D, 0, 0.5, r, C, FAKE, ws_bytes, None)
+    assert bwd(C=64) == -2                      # the backward takes chunks of 16 or 32
+    assert bwd(C=96) == -2
+    assert bwd(T=100) == -3
+    assert bwd(D=48) == -2
+    assert bwd(r=0) == -1
+    assert bwd(gate=FAKE) == -1                 # a gate needs its gradient buffer
+    assert bwd(dgate=FAKE) == -1                # and a gradient buffer needs a gate
+    assert bwd(q=FAKE_MIS) == -7
+    assert bwd(gate=FAKE_MIS, dgate=FAKE) == -7
+    assert bwd(ws_bytes=16) == -4
+    assert bwd(B=0) == 0
+    n16 = lib.gka_backward_workspace_bytes(1, 2, 128, 128, 16, 1)
+    n32 = lib.gka_backward_workspace_bytes(1, 2, 128, 128, 32, 1)
+    assert n16 > n32 > lib.gka_forward_workspace_bytes(1, 2, 128, 128, 64, 1) > 0
+    assert lib.gka_backward_workspace_bytes(1, 2, 128, 128, 64, 1) == 0
 
 
 def test_binding_raises_without_cuda_tensors():
