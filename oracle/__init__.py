@@ -16,4 +16,7 @@ from .oracle import (  # noqa: F401
     forward,
     max_threads,
     omegas,
+    solver_residuals,
+    solver_study,
+    SOLVERS,
 )

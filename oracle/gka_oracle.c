@@ -454,3 +454,160 @@ int gka_oracle_backward(const double *q, const double *k, const double *v,
     }
     return fail ? -2 : 0;
 }
+
+/*
+ * Solver study (ai.info page, Key Contributions 2 and Main Findings: CH is
+ * compared with gradient descent, accelerated gradient descent and conjugate
+ * gradient on the layer's systems; pith.science page, Fig. 1a and Fig. 8:
+ * residual norms per iteration in a random-regression setup, and for several
+ * regularisation strengths).
+ *
+ * For every token t the system A_t x = q_t of the layer (A_t = H_t + a n_t I,
+ * spectrum in [mu, L] = [a n_t, (1+a) n_t]) is solved from x_0 = 0 by
+ *   solver 0  Chebyshev (the layer's iteration)
+ *   solver 1  gradient descent with the fixed step 2/(L + mu)
+ *   solver 2  Nesterov's accelerated gradient descent for strongly convex
+ *             quadratics: y = x_i + m (x_i - x_{i-1}), x_{i+1} = y + (q - A y)/L,
+ *             m = (sqrt(kappa) - 1)/(sqrt(kappa) + 1), kappa = L / mu
+ *   solver 3  conjugate gradient (Hestenes-Stiefel)
+ * and resid[t][i] = ||q_t - A_t x_i|| / ||q_t|| for i = 0..r (the true residual,
+ * formed from x_i; resid[t][0] = 1).  A token with n_t = 0 or q_t = 0 gets zeros.
+ * Inputs as gka_oracle_forward (gate nullable); resid: [B, Hh, T, r + 1].
+ */
+static void solver_residuals(const double *A, const double *q, int D, double mu, double L,
+                             int r, int solver, double *res, double *work)
+{
+    double *x = work, *xp = work + D, *y = work + 2 * D, *Ay = work + 3 * D;
+    double *rr = work + 4 * D, *p = work + 5 * D, *Ap = work + 6 * D;
+    double qn = 0.0;
+    for (int i = 0; i < D; ++i) qn += q[i] * q[i];
+    qn = sqrt(qn);
+    if (qn == 0.0) {
+        for (int i = 0; i <= r; ++i) res[i] = 0.0;
+        return;
+    }
+    for (int i = 0; i < D; ++i) x[i] = xp[i] = 0.0;
+    res[0] = 1.0;
+    const double d = 0.5 * (L + mu), rho = (L - mu) / (L + mu);
+    const double kap = L / mu, m = (sqrt(kap) - 1.0) / (sqrt(kap) + 1.0);
+    double *omega = (double *)malloc(sizeof(double) * (size_t)(r > 1 ? r : 1));
+    gka_oracle_omegas(rho, r, omega);
+    double rs = 0.0;
+    if (solver == 3) {
+        for (int i = 0; i < D; ++i) rr[i] = p[i] = q[i];
+        for (int i = 0; i < D; ++i) rs += rr[i] * rr[i];
+    }
+    for (int it = 0; it < r; ++it) {
+        if (solver == 0) {
+            if (it == 0) {
+                for (int i = 0; i < D; ++i) x[i] = q[i] / d;
+            } else {
+                /* x_{it+1} = x_{it-1} + omega_it ((q - A x_it)/d + x_it - x_{it-1}) */
+                for (int i = 0; i < D; ++i) {
+                    double s = 0.0;
+                    for (int j = 0; j < D; ++j) s += A[(size_t)i * D + j] * x[j];
+                    Ay[i] = s;
+                }
+                for (int i = 0; i < D; ++i) {
+                    double xn = xp[i] + omega[it] * ((q[i] - Ay[i]) / d + x[i] - xp[i]);
+                    xp[i] = x[i];
+                    x[i] = xn;
+                }
+            }
+        } else if (solver == 1 || solver == 2) {
+            for (int i = 0; i < D; ++i) y[i] = solver == 2 ? x[i] + m * (x[i] - xp[i]) : x[i];
+            for (int i = 0; i < D; ++i) {
+                double s = 0.0;
+                for (int j = 0; j < D; ++j) s += A[(size_t)i * D + j] * y[j];
+                Ay[i] = s;
+            }
+            const double step = solver == 2 ? 1.0 / L : 1.0 / d;
+            for (int i = 0; i < D; ++i) {
+                xp[i] = x[i];
+                x[i] = y[i] + step * (q[i] - Ay[i]);
+            }
+        } else {
+            for (int i = 0; i < D; ++i) {
+                double s = 0.0;
+                for (int j = 0; j < D; ++j) s += A[(size_t)i * D + j] * p[j];
+                Ap[i] = s;
+            }
+            double pAp = 0.0;
+            for (int i = 0; i < D; ++i) pAp += p[i] * Ap[i];
+            const double alpha = pAp > 0.0 ? rs / pAp : 0.0;
+            double rs1 = 0.0;
+            for (int i = 0; i < D; ++i) {
+                x[i] += alpha * p[i];
+                rr[i] -= alpha * Ap[i];
+                rs1 += rr[i] * rr[i];
+            }
+            const double beta = rs > 0.0 ? rs1 / rs : 0.0;
+            for (int i = 0; i < D; ++i) p[i] = rr[i] + beta * p[i];
+            rs = rs1;
+        }
+        /* true residual of the new iterate */
+        double e2 = 0.0;
+        for (int i = 0; i < D; ++i) {
+            double s = 0.0;
+            for (int j = 0; j < D; ++j) s += A[(size_t)i * D + j] * x[j];
+            e2 += (q[i] - s) * (q[i] - s);
+        }
+        res[it + 1] = sqrt(e2) / qn;
+    }
+    free(omega);
+}
+
+int gka_oracle_solver_study(const double *q, const double *k, const double *beta,
+                            const double *gate, int B, int Hh, int T, int D, double a,
+                            int r, int solver, double *resid, int nthreads)
+{
+    if (B < 0 || Hh < 0 || T < 0 || D <= 0 || r < 1 || !(a > 0.0) || solver < 0 || solver > 3)
+        return -1;
+    long nh = (long)B * Hh;
+    size_t DD = (size_t)D * D;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (long h = 0; h < nh; ++h) {
+        double *H = (double *)calloc(DD, sizeof(double));
+        double *A = (double *)malloc(sizeof(double) * DD);
+        double *work = (double *)malloc(sizeof(double) * 8 * (size_t)D);
+        for (int t = 0; t < T; ++t) {
+            size_t row = ((size_t)h * T + t) * D;
+            const double g = gate ? gate[(size_t)h * T + t] : 1.0;
+            const double b = beta[(size_t)h * T + t];
+            const double *kt = k + row;
+            double n2 = 0.0;
+            for (int i = 0; i < D; ++i)
+                for (int j = 0; j < D; ++j) {
+                    double v = b * H[(size_t)i * D + j] + g * kt[i] * kt[j];
+                    H[(size_t)i * D + j] = v;
+                    n2 += v * v;
+                }
+            double *res = resid + ((size_t)h * T + t) * (size_t)(r + 1);
+            const double n = sqrt(n2);
+            if (n == 0.0) {
+                for (int i = 0; i <= r; ++i) res[i] = 0.0;
+                continue;
+            }
+            memcpy(A, H, sizeof(double) * DD);
+            for (int i = 0; i < D; ++i) A[(size_t)i * D + i] += a * n;
+            solver_residuals(A, q + row, D, a * n, (1.0 + a) * n, r, solver, res, work);
+        }
+        free(H); free(A); free(work);
+    }
+    return 0;
+}
+
+/*
+ * The residual history of one solver on one system A x = q (A: D x D symmetric
+ * with its spectrum in [mu, L]); res: r + 1 values (see gka_oracle_solver_study).
+ */
+void gka_oracle_solver_residuals(const double *A, const double *q, int D, double mu, double L,
+                                 int r, int solver, double *res)
+{
+    double *work = (double *)malloc(sizeof(double) * 8 * (size_t)D);
+    solver_residuals(A, q, D, mu, L, r, solver, res, work);
+    free(work);
+}

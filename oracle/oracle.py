@@ -58,6 +58,10 @@ def _load():
         lib.gka_oracle_backward.argtypes = [_dp, _dp, _dp, _dp, _dp, _dp, i, i, i, i, d, i,
                                             _dp, _dp, _dp, _dp, _dp, i]
         lib.gka_oracle_backward.restype = i
+        lib.gka_oracle_solver_study.argtypes = [_dp, _dp, _dp, _dp, i, i, i, i, d, i, i, _dp, i]
+        lib.gka_oracle_solver_study.restype = i
+        lib.gka_oracle_solver_residuals.argtypes = [_dp, _dp, i, d, d, i, i, _dp]
+        lib.gka_oracle_solver_residuals.restype = None
         lib.gka_oracle_max_threads.argtypes = []
         lib.gka_oracle_max_threads.restype = i
         _lib = lib
@@ -197,4 +201,33 @@ def backward(q, k, v, beta, dout, a: float, r: int, *, gate=None, nthreads: int 
         raise ValueError(f"gka_oracle_backward failed ({rc})")
     if dg is not None:
         out["dgate"] = dg
+    return out
+
+
+SOLVERS = ("chebyshev", "gd", "agd", "cg")
+
+
+def solver_study(q, k, beta, a: float, r: int, solver: str, *, gate=None, nthreads: int = 0):
+    """Relative residual ||q_t - A_t x_i|| / ||q_t||, i = 0..r, of ``solver`` (one of
+    SOLVERS) on every token's system A_t x = q_t.  Returns [B, H, T, r + 1]."""
+    q, k, beta = _f64(q), _f64(k), _f64(beta)
+    B, H, T, D = q.shape
+    g = _gate(gate, (B, H, T))
+    out = np.zeros((B, H, T, r + 1))
+    rc = _load().gka_oracle_solver_study(_ptr(q), _ptr(k), _ptr(beta), _ptr(g), B, H, T, D,
+                                         float(a), int(r), SOLVERS.index(solver), _ptr(out),
+                                         int(nthreads))
+    if rc != 0:
+        raise ValueError("gka_oracle_solver_study: bad arguments")
+    return out
+
+
+def solver_residuals(A, q, mu: float, L: float, r: int, solver: str) -> np.ndarray:
+    """Residual history ||q - A x_i|| / ||q||, i = 0..r, of ``solver`` on A x = q."""
+    A, q = _f64(A), _f64(q)
+    D = q.shape[0]
+    assert A.shape == (D, D)
+    out = np.zeros(r + 1)
+    _load().gka_oracle_solver_residuals(_ptr(A), _ptr(q), D, float(mu), float(L), int(r),
+                                        SOLVERS.index(solver), _ptr(out))
     return out
