@@ -75,6 +75,7 @@ def parse():
     p.add_argument("--no-write-gate", action="store_true",
                    help="skip the write-gated forward leg")
     p.add_argument("--no-backward", action="store_true", help="skip the backward leg")
+    p.add_argument("--no-solver-study", action="store_true", help="skip the solver-study leg")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--decode-steps", type=int, default=None)
     p.add_argument("--decode-batch", type=int, default=None,
@@ -432,6 +433,10 @@ def main():
         result["backward"] = bench_backward(args, w, dev, qd, kd, vd, bd, flush, rank, world,
                                             barrier, peaks)
 
+    # ---- solver study: Chebyshev vs gradient descent, Nesterov, conjugate gradient ----
+    if not args.no_solver_study and world == 1:
+        result["solver_study"] = bench_solver_study(w, qd, kd, bd)
+
     # ---- decode step: HBM-bound, 256 x 32 heads, fp32 state ----
     if not args.no_decode and world == 1:
         result["decode"] = bench_decode(args, dev, peaks)
@@ -572,6 +577,35 @@ def bench_backward(args, w, dev, qd, kd, vd, bd, flush, rank, world, barrier, pe
                          "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 flop x max SM clock",
                          "algorithmic_per_step": fl.get(dom, 0) * head_tok},
             "step_frac_of_fp32_peak": total_fl / (total_ms / steps / 1e3) / 1e12 / peak}
+
+
+def bench_solver_study(w, qd, kd, bd):
+    """Residual histories of the four solvers on every token of the workload (the
+    pages' Fig. 1a on its random-regression shape) and the final mean residual for
+    several regularisation strengths (Fig. 8); one timed run per solver at the
+    workload's a and r."""
+    import torch
+    from test_ridge_regression_b200 import gka
+    chunk = 64
+    out = {"chunk": chunk, "r": w.r, "a": w.a, "mean_residual": {}, "ms": {}}
+    for solver in gka.SOLVERS:
+        gka.gka_solver_study(qd, kd, bd, w.a, w.r, solver, chunk)   # warm-up
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        res = gka.gka_solver_study(qd, kd, bd, w.a, w.r, solver, chunk)
+        e.record()
+        torch.cuda.synchronize()
+        out["ms"][solver] = s.elapsed_time(e)
+        out["mean_residual"][solver] = [float(x) for x in res.double().mean(dim=(0, 1, 2))]
+    sweep = {}
+    for a in (0.5, 0.1, 0.05, 0.02):
+        sweep[str(a)] = {solver: float(gka.gka_solver_study(qd, kd, bd, a, 30, solver, chunk)
+                                       [..., -1].double().mean())
+                         for solver in gka.SOLVERS}
+    out["a_sweep_final_mean_residual_r30"] = sweep
+    if gka.device_status() != 0:
+        raise RuntimeError("device status error after the solver study")
+    return out
 
 
 def bench_decode(args, dev, peaks):

@@ -253,6 +253,34 @@ int gka_backward(const void *q, const void *k, const void *v, const float *beta,
                  float a, int r, int chunk, void *workspace, size_t workspace_bytes,
                  void *stream);
 
+/*
+ * Solver study (ai.info page, Key Contributions 2 and Main Findings: the
+ * layer's Chebyshev iteration compared with gradient descent, accelerated
+ * gradient descent and conjugate gradient; pith.science page, Fig. 1a and
+ * Fig. 8: residual norms per iteration, for several regularisation
+ * strengths).  For every token t, the system A_t x = q_t of the layer
+ * (A_t = H_t + a ||H_t||_F I, spectrum in [mu, L] = [a, 1 + a] ||H_t||_F) is
+ * solved from x_0 = 0 by
+ *   solver 0  Chebyshev (the layer's iteration)
+ *   solver 1  gradient descent, step 2 / (L + mu)
+ *   solver 2  Nesterov's method for strongly convex quadratics, step 1 / L,
+ *             momentum (sqrt(kappa) - 1) / (sqrt(kappa) + 1), kappa = L / mu
+ *   solver 3  conjugate gradient (Hestenes-Stiefel)
+ * and resid[t][i] = ||q_t - A_t x_i|| / ||q_t|| is written for i = 0..r (the
+ * true residual of each iterate, fp32 arithmetic on CUDA cores); zero for a
+ * token with H_t = 0 or q_t = 0.
+ *   q, k, beta, gate  as for gka_forward_gated (gate nullable); v is not needed
+ *   chunk       16, 32 or 64 (the chunk form of the products A x)
+ *   resid       fp32 [B, H, T, r + 1] (written)
+ *   workspace   at least gka_solver_study_workspace_bytes() bytes, 256-byte aligned
+ * Errors as for gka_forward; GKA_ERR_INVALID_ARG for a solver outside 0..3,
+ * GKA_ERR_UNSUPPORTED for chunk 128.
+ */
+size_t gka_solver_study_workspace_bytes(int B, int H, int T, int D, int chunk, gka_dtype dt);
+int gka_solver_study(const void *q, const void *k, const float *beta, const float *gate, int B,
+                     int H, int T, int D, gka_dtype dt, float a, int r, int chunk, int solver,
+                     float *resid, void *workspace, size_t workspace_bytes, void *stream);
+
 /* Synchronises `stream`, then returns GKA_ERR_DEVICE_TIMEOUT if any kernel of
  * this library on the current device gave up a bounded wait since the last
  * call (and clears the flag), GKA_ERR_CUDA if the stream reports an error,
@@ -290,6 +318,7 @@ enum {
     GKA_KERNEL_ADJOINT_SCAN = 9,  /* backward: adjoint states, last chunk first */
     GKA_KERNEL_BWD_ROWS = 10,     /* backward: chunk rows against H_s, M_s and the adjoints */
     GKA_KERNEL_BWD_GRADS = 11,    /* backward: dk, dv, dbeta, dgate of each chunk */
+    GKA_KERNEL_SOLVER_STUDY = 12, /* solver study: residual histories */
     GKA_KERNEL_COUNT = 16
 };
 

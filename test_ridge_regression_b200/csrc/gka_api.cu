@@ -21,6 +21,7 @@
 #include "delta_tc.cuh"
 #include "solve_tc.cuh"
 #include "state_tc.cuh"
+#include "study_simt.cuh"
 
 namespace gka {
 
@@ -534,6 +535,58 @@ static int backward_dispatch(const void *q, const void *k, const void *v, const 
     }
 }
 
+// ---------------------------------------------------------------------------
+// Solver study: the CUDA-core chunk states and norms, then one study kernel.
+// ---------------------------------------------------------------------------
+template <typename Tin, int D, int SOLVER>
+static int study_launch(const Tin *q, const Tin *k, const float *beta, const float *gate,
+                        const float *states, const float *norms, float *resid, int BH, int T,
+                        int N, int C, const ChebParams &P, cudaStream_t s) {
+    const size_t smem = sizeof(float) * ((size_t)D * SolveSmem<D>::KP +
+                                         (size_t)C * SolveSmem<D>::KP + (size_t)kSolveTG * D +
+                                         2 * (size_t)kSolveTG * C);
+    cudaError_t e = set_smem(k_solver_study<Tin, D, SOLVER>, smem);
+    if (e != cudaSuccess) return cuda_fail(e);
+    ProfScope ps(GKA_KERNEL_SOLVER_STUDY, s);
+    k_solver_study<Tin, D, SOLVER><<<dim3(C / kSolveTG, N, BH), kSimtThreads, smem, s>>>(
+        q, k, beta, gate, states, norms, resid, T, N, C, P);
+    return check_launch();
+}
+
+template <typename Tin, int D>
+static int study_simt(const Tin *q, const Tin *k, const float *beta, const float *gate, int B,
+                      int H, int T, int C, int solver, const ChebParams &P, float *resid, char *ws,
+                      const gka_workspace_layout &L, cudaStream_t s) {
+    const int BH = B * H, N = T / C;
+    float *states = reinterpret_cast<float *>(ws + L.states_offset);
+    float *decay = reinterpret_cast<float *>(ws + L.decay_offset);
+    float *norms = reinterpret_cast<float *>(ws + L.norms_offset);
+    cudaError_t e;
+    const size_t sm_delta = sizeof(float) * 3 * (size_t)C * D;
+    if ((e = set_smem(k_chunk_delta<Tin, D>, sm_delta)) != cudaSuccess) return cuda_fail(e);
+    { ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
+    k_chunk_delta<Tin, D><<<dim3(N, BH), kSimtThreads, sm_delta, s>>>(k, k, beta, gate, states,
+                                                                        decay, nullptr, T, N, C); }
+    if (int rc = check_launch()) return rc;
+    const int DD2 = 2 * D * D;
+    { ProfScope ps(GKA_KERNEL_STATE_SCAN, s);
+    k_state_scan<<<dim3((DD2 + 1023) / 1024, BH), 256, 0, s>>>(states, decay, nullptr, nullptr,
+                                                             nullptr, nullptr, N, DD2, true); }
+    if (int rc = check_launch()) return rc;
+    const size_t sm_norm = sizeof(float) * ((size_t)D * D + (size_t)C * (D + 1));
+    if ((e = set_smem(k_chunk_norm<Tin, D>, sm_norm)) != cudaSuccess) return cuda_fail(e);
+    { ProfScope ps(GKA_KERNEL_CHUNK_NORM, s);
+    k_chunk_norm<Tin, D><<<dim3(N, BH), kSimtThreads, sm_norm, s>>>(k, beta, gate, states, norms,
+                                                                    T, N, C); }
+    if (int rc = check_launch()) return rc;
+    switch (solver) {
+        case 0: return study_launch<Tin, D, 0>(q, k, beta, gate, states, norms, resid, BH, T, N, C, P, s);
+        case 1: return study_launch<Tin, D, 1>(q, k, beta, gate, states, norms, resid, BH, T, N, C, P, s);
+        case 2: return study_launch<Tin, D, 2>(q, k, beta, gate, states, norms, resid, BH, T, N, C, P, s);
+        default: return study_launch<Tin, D, 3>(q, k, beta, gate, states, norms, resid, BH, T, N, C, P, s);
+    }
+}
+
 static int timeout_flag_ptr(int **ptr) {
     cudaError_t e = cudaGetSymbolAddress((void **)ptr, g_timeout_flag);
     return e == cudaSuccess ? GKA_OK : cuda_fail(e);
@@ -912,6 +965,43 @@ int gka_backward(const void *q, const void *k, const void *v, const float *beta,
                                                 B, H, T, D, chunk, P, ws, L, s);
     return backward_dispatch<float>(q, k, v, beta, gate, dout, dq, dk, dv, dbeta, dgate, B, H, T, D,
                                     chunk, P, ws, L, s);
+}
+
+size_t gka_solver_study_workspace_bytes(int B, int H, int T, int D, int chunk, gka_dtype dt) {
+    if (chunk == 128) return 0;
+    gka_workspace_layout L;
+    return layout(B, H, T, D, chunk, dt, &L) == GKA_OK ? L.total_bytes : 0;
+}
+
+int gka_solver_study(const void *q, const void *k, const float *beta, const float *gate, int B,
+                     int H, int T, int D, gka_dtype dt, float a, int r, int chunk, int solver,
+                     float *resid, void *workspace, size_t workspace_bytes, void *stream) {
+    gka_workspace_layout L;
+    if (int rc = layout(B, H, T, D, chunk, dt, &L)) return rc;
+    if (chunk == 128) return GKA_ERR_UNSUPPORTED;   // the study's C x D tiles stop at 64
+    if (!(a > 0.f) || !isfinite(a) || r < 1 || solver < 0 || solver > 3) return GKA_ERR_INVALID_ARG;
+    if (r > kMaxSteps) return GKA_ERR_UNSUPPORTED;
+    if ((size_t)B * H > 65535) return GKA_ERR_UNSUPPORTED;
+    if ((size_t)B * H == 0 || T == 0) return GKA_OK;
+    if (!q || !k || !beta || !resid || !workspace) return GKA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(beta) || (gate && !aligned16(gate)) ||
+        !aligned16(resid) || ((uintptr_t)workspace & 255u))
+        return GKA_ERR_MISALIGNED;
+    if (workspace_bytes < L.total_bytes) return GKA_ERR_WORKSPACE_TOO_SMALL;
+    const ChebParams P = make_cheb(a, r);
+    char *ws = static_cast<char *>(workspace);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    auto run = [&](auto tag) -> int {
+        using Tin = decltype(tag);
+        auto Q = static_cast<const Tin *>(q);
+        auto K = static_cast<const Tin *>(k);
+        switch (D) {
+            case 32: return study_simt<Tin, 32>(Q, K, beta, gate, B, H, T, chunk, solver, P, resid, ws, L, s);
+            case 64: return study_simt<Tin, 64>(Q, K, beta, gate, B, H, T, chunk, solver, P, resid, ws, L, s);
+            default: return study_simt<Tin, 128>(Q, K, beta, gate, B, H, T, chunk, solver, P, resid, ws, L, s);
+        }
+    };
+    return dt == GKA_BF16 ? run(__nv_bfloat16()) : run(float());
 }
 
 int gka_selftest_timeout(void *stream) {

@@ -30,7 +30,7 @@ class GkaError(RuntimeError):
 
 KERNEL_NAMES = ["chunk_delta", "state_scan", "chunk_norm", "chunk_solve", "decode_step",
                 "chunk_solve_tc", "state_pass_tc", "bwd_solve", "bwd_delta", "adjoint_scan",
-                "bwd_rows", "bwd_grads"]
+                "bwd_rows", "bwd_grads", "solver_study"]
 _KERNEL_COUNT = 16
 
 
@@ -80,6 +80,10 @@ def _lib():
         lib.gka_backward_workspace_bytes.restype = sz
         lib.gka_backward.argtypes = [vp] * 11 + [i, i, i, i, i, f, i, i, vp, sz, vp]
         lib.gka_backward.restype = i
+        lib.gka_solver_study_workspace_bytes.argtypes = [i, i, i, i, i, i]
+        lib.gka_solver_study_workspace_bytes.restype = sz
+        lib.gka_solver_study.argtypes = [vp, vp, vp, vp, i, i, i, i, i, f, i, i, i, vp, vp, sz, vp]
+        lib.gka_solver_study.restype = i
         lib.gka_selftest_timeout.argtypes = [vp]
         lib.gka_selftest_timeout.restype = i
         lib.gka_device_status.argtypes = [vp]
@@ -333,6 +337,34 @@ def gka_backward(q, k, v, beta, dout, a: float, r: int, chunk: int = 32, *, gate
                              _stream(stream))
     _check("gka_backward", rc)
     return out
+
+
+SOLVERS = ("chebyshev", "gd", "agd", "cg")
+
+
+def gka_solver_study(q, k, beta, a: float, r: int, solver: str, chunk: int = 64, *, gate=None,
+                     workspace=None, stream=None):
+    """Residual history ||q_t - A_t x_i|| / ||q_t||, i = 0..r, of ``solver`` (one of
+    SOLVERS) on every token's system (see include/gka.h).  Returns [B, H, T, r + 1] fp32."""
+    _dev(q, k, beta, gate, workspace)
+    B, H, T, D = q.shape
+    if k.shape != q.shape or beta.shape != (B, H, T):
+        raise ValueError("shape mismatch")
+    if gate is not None and (gate.shape != (B, H, T) or gate.dtype != torch.float32):
+        raise ValueError("gate must be float32 [B, H, T]")
+    dt = _dtype(q)
+    if k.dtype != q.dtype or beta.dtype != torch.float32:
+        raise TypeError("q, k must share a dtype; beta must be float32")
+    resid = torch.empty(B, H, T, r + 1, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        n = int(_lib().gka_solver_study_workspace_bytes(B, H, T, D, chunk, dt))
+        workspace = torch.empty(max(n, 256), dtype=torch.uint8, device=q.device)
+    rc = _lib().gka_solver_study(_ptr(q), _ptr(k), _ptr(beta), _ptr(gate), B, H, T, D, dt,
+                                 float(a), int(r), int(chunk), SOLVERS.index(solver), _ptr(resid),
+                                 _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                 _stream(stream))
+    _check("gka_solver_study", rc)
+    return resid
 
 
 def selftest_timeout(stream=None) -> None:
