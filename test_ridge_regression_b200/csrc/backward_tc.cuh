@@ -1,0 +1,326 @@
+// Tensor-core row products of the backward pass (bf16 inputs, D = 128, chunks
+// of 32 tokens): the work of k_bwd_rows (backward_simt.cuh) as fp16 MMAs.
+//
+// Per chunk, with its fp32 matrices H_s, M_s (chunk-start states) and E^H, E^M
+// (adjoint states arriving from later chunks), and its rows k_t, v_t, g_t, x_t:
+//   R1 = H_s K^T,  Hx = H_s X^T,  Mg = M_s^T G^T,
+//   R2 = (E^H + E^H^T) K^T,  R3 = E^M^T V^T,  R4 = E^M K^T
+// as 128 x 32 tiles (row c = TMEM lane, column t = token), then
+//   R1, R2, R3, R4 to global (rows [B*H*T][128]), and per token
+//   uk = k . R1,  yhx = y . Hx,  gmx = x . Mg,  qe = k . R2 / 2 + v . R4,
+//   and per chunk hs2 = ||H_s||_F^2, eh = <E^H, H_s> + <E^M, M_s>.
+// Every matrix is converted in shared memory to fp16 with a power-of-two scale
+// that puts its largest entry below 1 (relative rounding 2^-11, as the forward's
+// fp16 state copies); k, v, g tiles likewise, x per token.  The accumulators are
+// fp32.  Two phases reuse the matrix tiles: (H_s, M_s) then (E^H, E^M).
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include "backward_simt.cuh"
+#include "common.cuh"
+#include "ptx.cuh"
+#include "solve_tc.cuh"
+#include "tcgen05.cuh"
+
+namespace gka {
+
+constexpr int kBrC = 32;   // tokens per chunk of this kernel
+
+struct BwdRowsTcSmem {
+    static constexpr uint32_t MA = 0;              // [2][128][64] fp16: H_s, then E^H
+    static constexpr uint32_t MB = MA + 32768;     // [2][128][64] fp16: M_s, then E^M
+    static constexpr uint32_t RK = MB + 32768;     // [2][32][64] fp16 rows of k
+    static constexpr uint32_t RV = RK + 8192;      // v
+    static constexpr uint32_t RG = RV + 8192;      // g
+    static constexpr uint32_t RX = RG + 8192;      // x (per-token scales)
+    static constexpr uint32_t XS = RX + 8192;      // float[32] x scales
+    static constexpr uint32_t RED = XS + 128;      // float[32][4] per-token partial sums
+    static constexpr uint32_t MRED = RED + 512;    // float[16] block reductions
+    static constexpr uint32_t BARS = MRED + 64;    // 3 mbarriers: phase A, phase B, drain
+    static constexpr uint32_t TBASE = BARS + 32;
+    static constexpr uint32_t END = TBASE + 16;
+    static constexpr size_t bytes = END + 1024;    // + alignment slack
+};
+
+// Largest value over the block (256 threads); red: 8 floats.
+__device__ __forceinline__ float block_max256(float v, float *red) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    float m = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) m = fmaxf(m, red[w]);
+    return m;
+}
+
+// fp32 row-major 128 x 128 matrix -> fp16 [2][128][64] swizzled tile, scaled by a
+// power of two below 1/max.  Thread (row r = tid / 2, column half h = tid % 2) holds
+// its 64 elements in registers between the max and the conversion.
+// dotw (nullable): accumulates sum A * W over the thread's elements into *dot;
+// sq2 (nullable): accumulates sum A^2.  Returns the scale.
+__device__ __forceinline__ float mat_to_f16_tile(const float *__restrict__ A, uint32_t tile,
+                                                 float *red, const float *__restrict__ dotw,
+                                                 float *dot, float *sq2) {
+    const int tid = threadIdx.x, r = tid >> 1, h = tid & 1;
+    const float4 *src = reinterpret_cast<const float4 *>(A + r * 128 + h * 64);
+    const float4 *wsrc = dotw ? reinterpret_cast<const float4 *>(dotw + r * 128 + h * 64) : nullptr;
+    float mx = 0.f, dp = 0.f, s2 = 0.f;
+    // all 16 loads of a pass are issued before their values are used
+    float4 x[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) x[i] = __ldg(src + i);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        mx = fmaxf(mx, fmaxf(fmaxf(fabsf(x[i].x), fabsf(x[i].y)), fmaxf(fabsf(x[i].z), fabsf(x[i].w))));
+        s2 = fmaf(x[i].x, x[i].x, fmaf(x[i].y, x[i].y, fmaf(x[i].z, x[i].z, fmaf(x[i].w, x[i].w, s2))));
+    }
+    if (wsrc) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float4 w = __ldg(wsrc + i);
+            dp = fmaf(x[i].x, w.x, fmaf(x[i].y, w.y, fmaf(x[i].z, w.z, fmaf(x[i].w, w.w, dp))));
+        }
+    }
+    if (dot) *dot += dp;
+    if (sq2) *sq2 += s2;
+    const float sc = inv_pow2_above(block_max256(mx, red));
+    const uint32_t base = tile + (uint32_t)h * 16384u;
+#pragma unroll
+    for (int c8 = 0; c8 < 8; ++c8) {
+        const float4 a = x[2 * c8], b = x[2 * c8 + 1];
+        const float v[8] = {a.x * sc, a.y * sc, a.z * sc, a.w * sc,
+                            b.x * sc, b.y * sc, b.z * sc, b.w * sc};
+        st_row8(base, (uint32_t)r, (uint32_t)(c8 * 8), v);
+    }
+    return sc;
+}
+
+// bf16 rows [32][128] (global) -> fp16 [2][32][64] swizzled tile with one power-of-two
+// scale (per_token: one scale per token row, written to xs).  Thread (token t = tid / 8,
+// 16 columns (tid % 8) * 16).  Returns the tile scale (1 with per_token).
+template <typename Src>
+__device__ __forceinline__ float rows_to_f16_tile(const Src *__restrict__ src, uint32_t tile,
+                                                  float *red, bool per_token, float *xs) {
+    const int tid = threadIdx.x, t = tid >> 3, c0 = (tid & 7) * 16;
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = to_f(src[t * 128 + c0 + i]);
+    float mx = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) mx = fmaxf(mx, fabsf(v[i]));
+    float sc;
+    if (per_token) {
+#pragma unroll
+        for (int o = 1; o < 8; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        sc = inv_pow2_above(mx);
+        if ((tid & 7) == 0) xs[t] = sc;
+    } else {
+        sc = inv_pow2_above(block_max256(mx, red));
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] *= sc;
+    const uint32_t base = tile + (uint32_t)(c0 >> 6) * (kBrC * 128u);
+    st_row8(base, (uint32_t)t, (uint32_t)(c0 & 63), v);
+    st_row8(base, (uint32_t)t, (uint32_t)((c0 & 63) + 8), v + 8);
+    return per_token ? 1.f : sc;
+}
+
+// grid (N, B*H), block 256.  T = N * 32.
+__global__ void __launch_bounds__(kSimtThreads, 2)
+k_bwd_rows_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
+              const __nv_bfloat16 *__restrict__ dout, const float *__restrict__ states,
+              const float *__restrict__ adj, const float *__restrict__ xs,
+              const float *__restrict__ ys, float *__restrict__ R, float *__restrict__ tokq,
+              float *__restrict__ chq, int T, int N, int *__restrict__ timeout_flag) {
+    using L = BwdRowsTcSmem;
+    constexpr int D = 128, C = kBrC;
+    extern __shared__ uint8_t smraw[];
+    uint8_t *sm = smem_align1024(smraw);
+    const uint32_t sb = smem_u32(sm);
+    float *xsc = reinterpret_cast<float *>(sm + L::XS);
+    float *red = reinterpret_cast<float *>(sm + L::RED);    // [32 tokens][4 quarters]
+    float *mred = reinterpret_cast<float *>(sm + L::MRED);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BARS);
+    uint32_t *tbase = reinterpret_cast<uint32_t *>(sm + L::TBASE);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3, wg = warp >> 2;
+    const int c = quarter * 32 + lane;       // matrix row = TMEM lane of this thread
+    const int n = blockIdx.x, bh = blockIdx.y;
+    const size_t tok0 = (size_t)bh * T + (size_t)n * C;
+    const size_t plane = (size_t)gridDim.y * T, RD = plane * D;
+    const float *Hs = states + ((size_t)bh * (N + 1) + n) * 2 * D * D, *Ms = Hs + D * D;
+    const float *EH = adj + ((size_t)bh * (N + 1) + n) * 2 * D * D, *EM = EH + D * D;
+
+    if (tid == 0) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        mbar_init(&bars[2], 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tc::tmem_alloc(tbase, 256);
+        tc::tmem_relinquish();
+    }
+    // rows and phase-A matrices
+    const float sK = rows_to_f16_tile(k + tok0 * D, sb + L::RK, mred, false, nullptr);
+    const float sV = rows_to_f16_tile(v + tok0 * D, sb + L::RV, mred, false, nullptr);
+    const float sG = rows_to_f16_tile(dout + tok0 * D, sb + L::RG, mred, false, nullptr);
+    rows_to_f16_tile(xs + tok0 * D, sb + L::RX, mred, true, xsc);
+    float hs2 = 0.f, eh = 0.f;
+    const float sH = mat_to_f16_tile(Hs, sb + L::MA, mred, nullptr, nullptr, &hs2);
+    const float sM = mat_to_f16_tile(Ms, sb + L::MB, mred, nullptr, nullptr, nullptr);
+    fence_proxy_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tbase;
+    constexpr uint32_t ID_K = tc::idesc_f16(128, C, false, false);   // A K-major
+    constexpr uint32_t ID_T = tc::idesc_f16(128, C, true, false);    // A MN-major (transposed)
+    auto adesc_k = [&](uint32_t a, int kk) { return tc::sdesc(a + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024); };
+    auto adesc_t = [&](uint32_t a, int kk) { return tc::sdesc(a + kk * 2048, 16384, 1024); };
+    auto bdesc = [&](uint32_t b, int kk) { return tc::sdesc(b + (kk >> 2) * (C * 128) + (kk & 3) * 32, 16, 1024); };
+    if (tid == 0) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            tc::mma_f16(tmem + 0, adesc_k(sb + L::MA, kk), bdesc(sb + L::RK, kk), ID_K, kk > 0);
+            tc::mma_f16(tmem + 32, adesc_k(sb + L::MA, kk), bdesc(sb + L::RX, kk), ID_K, kk > 0);
+            tc::mma_f16(tmem + 64, adesc_t(sb + L::MB, kk), bdesc(sb + L::RG, kk), ID_T, kk > 0);
+        }
+        tc::commit(&bars[0]);
+    }
+    bool ok = mbar_wait_bounded(&bars[0], 0, kTcWaitProbes);
+    tc::fence_after_sync();
+
+    // per-token sums over the 128 rows: this thread's 16 partials -> red[t][quarter]
+    auto token_sum = [&](float *part, float *dst, float scale, bool add) {
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const float s = warp_sum(part[u]);
+            if (lane == 0) red[(wg * 16 + u) * 4 + quarter] = s;
+        }
+        __syncthreads();
+        if (tid < C) {
+            const float s = (red[tid * 4] + red[tid * 4 + 1] + red[tid * 4 + 2] + red[tid * 4 + 3]) * scale;
+            if (ok) dst[tok0 + tid] = add ? dst[tok0 + tid] + s : s;
+        }
+        __syncthreads();
+    };
+    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(wg * 16);
+    {
+        // one product at a time (register budget: two CTAs per SM)
+        float acc[16], part[16];
+        tc::tmem_ld16(tl + 0, acc);
+        tc::tmem_wait_ld();
+        const float u1 = 1.f / (sH * sK);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const size_t g = (tok0 + wg * 16 + u) * D + c;
+            const float a1 = acc[u] * u1;
+            if (ok) R[g] = a1;
+            part[u] = a1 * __bfloat162float(k[g]);
+        }
+        token_sum(part, tokq, 1.f, false);
+        tc::tmem_ld16(tl + 32, acc);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const int t = wg * 16 + u;
+            const size_t g = (tok0 + t) * D + c;
+            part[u] = acc[u] / (sH * xsc[t]) * ys[g];
+        }
+        token_sum(part, tokq + plane, 1.f, false);
+        tc::tmem_ld16(tl + 64, acc);
+        tc::tmem_wait_ld();
+        const float u3 = 1.f / (sM * sG);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const size_t g = (tok0 + wg * 16 + u) * D + c;
+            part[u] = acc[u] * u3 * xs[g];
+        }
+        token_sum(part, tokq + 2 * plane, 1.f, false);
+    }
+    // phase B: the adjoints into the same tiles (the phase-A products are complete)
+    const float sEH = mat_to_f16_tile(EH, sb + L::MA, mred, Hs, &eh, nullptr);
+    const float sEM = mat_to_f16_tile(EM, sb + L::MB, mred, Ms, &eh, nullptr);
+    fence_proxy_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (tid == 0 && ok) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            tc::mma_f16(tmem + 96, adesc_k(sb + L::MA, kk), bdesc(sb + L::RK, kk), ID_K, kk > 0);
+            tc::mma_f16(tmem + 128, adesc_t(sb + L::MB, kk), bdesc(sb + L::RV, kk), ID_T, kk > 0);
+            tc::mma_f16(tmem + 160, adesc_k(sb + L::MB, kk), bdesc(sb + L::RK, kk), ID_K, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+            tc::mma_f16(tmem + 96, adesc_t(sb + L::MA, kk), bdesc(sb + L::RK, kk), ID_T, true);
+    }
+    if (tid == 0) tc::commit(&bars[1]);
+    if (!mbar_wait_bounded(&bars[1], 0, kTcWaitProbes)) ok = false;
+    tc::fence_after_sync();
+    {
+        float acc[16], part[16];
+        tc::tmem_ld16(tl + 96, acc);
+        tc::tmem_wait_ld();
+        const float u2 = 1.f / (sEH * sK), u3 = 1.f / (sEM * sV), u4 = 1.f / (sEM * sK);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const size_t g = (tok0 + wg * 16 + u) * D + c;
+            const float a2 = acc[u] * u2;
+            if (ok) R[RD + g] = a2;
+            part[u] = 0.5f * a2 * __bfloat162float(k[g]);
+        }
+        tc::tmem_ld16(tl + 128, acc);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const size_t g = (tok0 + wg * 16 + u) * D + c;
+            if (ok) R[2 * RD + g] = acc[u] * u3;
+        }
+        tc::tmem_ld16(tl + 160, acc);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const size_t g = (tok0 + wg * 16 + u) * D + c;
+            const float a4 = acc[u] * u4;
+            if (ok) R[3 * RD + g] = a4;
+            part[u] = fmaf(a4, __bfloat162float(v[g]), part[u]);
+        }
+        token_sum(part, tokq + 3 * plane, 1.f, false);
+    }
+    // chunk scalars
+    {
+        hs2 = warp_sum(hs2);
+        eh = warp_sum(eh);
+        if (lane == 0) {
+            mred[warp] = hs2;
+            mred[8 + warp] = eh;
+        }
+        __syncthreads();
+        if (tid < 2 && ok) {
+            float s = 0.f;
+            for (int w = 0; w < 8; ++w) s += mred[tid * 8 + w];
+            chq[((size_t)bh * N + n) * 2 + tid] = s;
+        }
+    }
+    if (!ok && tid == 0) {
+        // a wait gave up: flag it, and let every MMA this CTA issued finish before TMEM
+        // is released (a commit after them, waited for with a bound)
+        atomicExch(timeout_flag, 1);
+        tc::commit(&bars[2]);
+        mbar_wait_bounded(&bars[2], 0, kTcWaitProbes);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, 256);
+    }
+}
+
+}  // namespace gka

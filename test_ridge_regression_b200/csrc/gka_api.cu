@@ -15,6 +15,7 @@
 #include <cudaTypedefs.h>
 
 #include "backward_simt.cuh"
+#include "backward_tc.cuh"
 #include "chunk_simt.cuh"
 #include "common.cuh"
 #include "decode.cuh"
@@ -484,7 +485,24 @@ static int backward_simt(const Tin *q, const Tin *k, const Tin *v, const float *
     k_adjoint_scan<<<dim3((DD2 / 4 + 255) / 256, BH), 256, 0, s>>>(adj, decay, N, DD2); }
     if (int rc = check_launch()) return rc;
     // the chunk rows against H_s, M_s and the adjoints
-    if (C == 16) {
+    bool rows_done = false;
+    if constexpr (std::is_same<Tin, __nv_bfloat16>::value && D == 128) {
+        if (tc_done && C == kBrC) {
+            // bf16, D = 128: the row products as fp16 MMAs
+            int *flag = nullptr;
+            if (int rc = timeout_flag_ptr(&flag)) return rc;
+            if ((e = set_smem(k_bwd_rows_tc, BwdRowsTcSmem::bytes)) != cudaSuccess)
+                return cuda_fail(e);
+            { ProfScope ps(GKA_KERNEL_BWD_ROWS, s);
+            k_bwd_rows_tc<<<dim3(N, BH), kSimtThreads, BwdRowsTcSmem::bytes, s>>>(
+                k, v, dout, states, adj, xs, ys, rows, tokq, chq, T, N, flag); }
+            if (int rc = check_launch()) return rc;
+            rows_done = true;
+        }
+    }
+    if (rows_done) {
+        // the tensor-core row products ran
+    } else if (C == 16) {
         constexpr size_t sm_rows = BwdRowsSmem<Tin, D, 16>::bytes;
         if ((e = set_smem(k_bwd_rows<Tin, D, 16>, sm_rows)) != cudaSuccess) return cuda_fail(e);
         ProfScope ps(GKA_KERNEL_BWD_ROWS, s);
