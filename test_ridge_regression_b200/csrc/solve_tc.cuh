@@ -625,7 +625,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         }
         tc::tmem_wait_st();
     }
-    if (P.r > 1) {   // round 1's table: -w c1 per token
+    if (P.r > 1) {   // the first Chebyshev round's table: -w c1 per token
         for (int e = tid; e < TOK; e += kSolveThreads) s_coef[TOK + e] = -P.omega[1] * s_c1[e];
     }
     fence_proxy_async_smem();
