@@ -38,10 +38,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # bench reports null.  Captures and commands: profiles/*.md.
 TRAFFIC = {
     # full-size forward workload (B8 H8 T2048 D128, chunk 64), one launch
-    "chunk_solve_tc": {"bytes": 237.136640e6 + 20.724480e6, "workload": "bf16_b8h8t2048d128",
+    "chunk_solve_tc": {"bytes": 237.182720e6 + 20.763136e6, "workload": "bf16_b8h8t2048d128",
                        "src": "test_ridge_regression_b200/csrc/solve_tc.cuh",
-                       "sha1": "674083975df1535cbb33550a4555b31f8c1682c4"},
-    "state_pass_tc": {"bytes": 67.715840e6 + 80.063488e6, "workload": "bf16_b8h8t2048d128",
+                       "sha1": "45f1ba0509465c05e81305cbf9b066dcc0cd12f2"},
+    "state_pass_tc": {"bytes": 67.759872e6 + 80.081664e6, "workload": "bf16_b8h8t2048d128",
                       "src": "test_ridge_regression_b200/csrc/state_tc.cuh",
                       "sha1": "3bd3bff3a2f8e7bf8df221195dc42f9281487e71"},
     # decode captured on 64 x 32 heads (state above L2), scaled x4 to 256 x 32 heads
