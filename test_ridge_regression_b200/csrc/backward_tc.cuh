@@ -324,3 +324,182 @@ k_bwd_rows_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restri
 }
 
 }  // namespace gka
+
+namespace gka {
+
+// ---------------------------------------------------------------------------
+// k_bwd_delta_tc: the adjoint increments of one 32-token chunk on tcgen05
+// (the work of k_bwd_delta):
+//   dE^H = -(b o Y)^T X - (e o K~)^T K~ - (sum_s b_s^2 c_s) H_start,
+//   dE^M = (b o G)^T X,      e_i = sum_{s>=i} b_s c_s w_si,
+// two 128 x 128 x 32 accumulations (operands MN-major from token-row tiles, fp16
+// with power-of-two scales; the two products of dE^H scaled alike so that they
+// share one accumulator), the H_start term added in fp32 on the way out.
+// grid (N, B*H), block 256.
+// ---------------------------------------------------------------------------
+struct BwdDeltaTcSmem {
+    static constexpr uint32_t TY = 0;            // [2][32][64] fp16: -(b o y) rows
+    static constexpr uint32_t TX = TY + 8192;    // x rows
+    static constexpr uint32_t TE = TX + 8192;    // -(e o k~) rows
+    static constexpr uint32_t TK = TE + 8192;    // k~ rows
+    static constexpr uint32_t TG = TK + 8192;    // (b o g) rows
+    static constexpr uint32_t ELL = TG + 8192;   // double[32] + double[8]
+    static constexpr uint32_t SC = ELL + 320;    // float[32] b, float[32] e, float[32] sqrt(w)
+    static constexpr uint32_t MRED = SC + 384;   // float[16]
+    static constexpr uint32_t BARS = MRED + 64;  // 2 mbarriers: products, drain
+    static constexpr uint32_t TBASE = BARS + 16;
+    static constexpr uint32_t END = TBASE + 16;
+    static constexpr size_t bytes = END + 1024;
+};
+
+// rows [32][128] of src (fp32 or bf16) times a per-row weight -> fp16 swizzled
+// [2][32][64] tile, scaled by `sc` (a power of two); the caller picks the scale from
+// the maximum that rows_absmax returns.
+template <typename Src>
+__device__ __forceinline__ float rows_absmax(const Src *__restrict__ src, const float *wrow,
+                                             float *red) {
+    const int tid = threadIdx.x, t = tid >> 3, c0 = (tid & 7) * 16;
+    const float w = wrow ? wrow[t] : 1.f;
+    float mx = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) mx = fmaxf(mx, fabsf(to_f(src[t * 128 + c0 + i]) * w));
+    return block_max256(mx, red);
+}
+template <typename Src>
+__device__ __forceinline__ void rows_store_f16(const Src *__restrict__ src, const float *wrow,
+                                               float sc, uint32_t tile) {
+    const int tid = threadIdx.x, t = tid >> 3, c0 = (tid & 7) * 16;
+    const float w = (wrow ? wrow[t] : 1.f) * sc;
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = to_f(src[t * 128 + c0 + i]) * w;
+    const uint32_t base = tile + (uint32_t)(c0 >> 6) * (kBrC * 128u);
+    st_row8(base, (uint32_t)t, (uint32_t)(c0 & 63), v);
+    st_row8(base, (uint32_t)t, (uint32_t)((c0 & 63) + 8), v + 8);
+}
+
+__global__ void __launch_bounds__(kSimtThreads, 2)
+k_bwd_delta_tc(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ beta,
+               const float *__restrict__ gate, const __nv_bfloat16 *__restrict__ dout,
+               const float *__restrict__ states, const float *__restrict__ xs,
+               const float *__restrict__ ys, const float *__restrict__ cvec,
+               float *__restrict__ adj, int T, int N, int *__restrict__ timeout_flag) {
+    using L = BwdDeltaTcSmem;
+    constexpr int D = 128, C = kBrC;
+    extern __shared__ uint8_t smraw[];
+    uint8_t *sm = smem_align1024(smraw);
+    const uint32_t sb = smem_u32(sm);
+    double *ell = reinterpret_cast<double *>(sm + L::ELL);
+    double *wtot = ell + C;
+    float *s_b = reinterpret_cast<float *>(sm + L::SC), *s_e = s_b + C, *s_sg = s_e + C;
+    float *mred = reinterpret_cast<float *>(sm + L::MRED);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BARS);
+    uint32_t *tbase = reinterpret_cast<uint32_t *>(sm + L::TBASE);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n = blockIdx.x, bh = blockIdx.y;
+    const size_t tok0 = (size_t)bh * T + (size_t)n * C;
+    if (tid == 0) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tc::tmem_alloc(tbase, 256);
+        tc::tmem_relinquish();
+    }
+    chunk_log_prefix(beta + tok0, C, ell, wtot);
+    if (tid < C) s_sg[tid] = gate ? sqrtf(gate[tok0 + tid]) : 1.f;
+    if (tid == 0) {
+        float e = 0.f, c1 = 0.f;
+        for (int i = C - 1; i >= 0; --i) {
+            const float b = decay_exp(ell[i]);
+            const float bc = b * cvec[tok0 + i];
+            const float nxt = i + 1 < C ? decay_exp(ell[i + 1] - ell[i]) : 0.f;
+            e = fmaf(nxt, e, bc);
+            s_e[i] = e;
+            s_b[i] = b;
+            c1 = fmaf(b, bc, c1);
+        }
+        mred[15] = c1;
+    }
+    __syncthreads();
+    const float c1 = mred[15];
+    // scales: x and k~ by their maxima; y and (e k~) so that both products of dE^H
+    // carry the same overall scale S = min(sY sX, sE sK)
+    const float *xrow = xs + tok0 * D, *yrow = ys + tok0 * D;
+    const __nv_bfloat16 *krow = k + tok0 * D, *grow = dout + tok0 * D;
+    // k~ = sqrt(w) k: weight s_sg; e o k~: weight s_e * s_sg (formed below)
+    __shared__ float s_ek[kBrC];
+    if (tid < C) s_ek[tid] = s_e[tid] * s_sg[tid];
+    __syncthreads();
+    const float mX = rows_absmax(xrow, nullptr, mred);
+    const float mK = rows_absmax(krow, s_sg, mred);
+    const float mY = rows_absmax(yrow, s_b, mred);
+    const float mE = rows_absmax(krow, s_ek, mred);
+    const float mG = rows_absmax(grow, s_b, mred);
+    const float sX = inv_pow2_above(mX), sK = inv_pow2_above(mK);
+    const float sY0 = inv_pow2_above(mY), sE0 = inv_pow2_above(mE), sG = inv_pow2_above(mG);
+    const float S = fminf(sY0 * sX, sE0 * sK);
+    const float sY = S / sX, sE = S / sK;    // both <= their own limits (powers of two)
+    rows_store_f16(xrow, nullptr, sX, sb + L::TX);
+    rows_store_f16(krow, s_sg, sK, sb + L::TK);
+    rows_store_f16(yrow, s_b, -sY, sb + L::TY);
+    rows_store_f16(krow, s_ek, -sE, sb + L::TE);
+    rows_store_f16(grow, s_b, sG, sb + L::TG);
+    fence_proxy_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tbase;
+    constexpr uint32_t ID = tc::idesc_f16(128, 128, true, true);
+    auto desc = [&](uint32_t t, int kk) { return tc::sdesc(t + kk * 2048, C * 128, 1024); };
+    if (tid == 0) {
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk) {
+            tc::mma_f16(tmem + 0, desc(sb + L::TY, kk), desc(sb + L::TX, kk), ID, kk > 0);
+            tc::mma_f16(tmem + 0, desc(sb + L::TE, kk), desc(sb + L::TK, kk), ID, true);
+            tc::mma_f16(tmem + 128, desc(sb + L::TG, kk), desc(sb + L::TX, kk), ID, kk > 0);
+        }
+        tc::commit(&bars[0]);
+    }
+    bool ok = mbar_wait_bounded(&bars[0], 0, kTcWaitProbes);
+    tc::fence_after_sync();
+    // row p = TMEM lane of this thread, columns 64 wg .. 64 wg + 63
+    const int quarter = warp & 3, wg = warp >> 2, p = quarter * 32 + lane;
+    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(wg * 64);
+    const float *Hst = states + ((size_t)bh * (N + 1) + n) * 2 * D * D + (size_t)p * D + wg * 64;
+    float *outH = adj + ((size_t)bh * (N + 1) + n) * 2 * D * D + (size_t)p * D + wg * 64;
+    float *outM = outH + D * D;
+    const float uH = 1.f / S, uM = 1.f / (sG * sX);
+#pragma unroll
+    for (int cb = 0; cb < 64; cb += 16) {
+        float a[16], m[16];
+        tc::tmem_ld16(tl + cb, a);
+        tc::tmem_ld16(tl + 128 + cb, m);
+        tc::tmem_wait_ld();
+        if (ok) {
+#pragma unroll
+            for (int j = 0; j < 16; j += 4) {
+                const float4 h = *reinterpret_cast<const float4 *>(Hst + cb + j);
+                *reinterpret_cast<float4 *>(outH + cb + j) =
+                    make_float4(fmaf(-c1, h.x, a[j] * uH), fmaf(-c1, h.y, a[j + 1] * uH),
+                                fmaf(-c1, h.z, a[j + 2] * uH), fmaf(-c1, h.w, a[j + 3] * uH));
+                *reinterpret_cast<float4 *>(outM + cb + j) =
+                    make_float4(m[j] * uM, m[j + 1] * uM, m[j + 2] * uM, m[j + 3] * uM);
+            }
+        }
+    }
+    if (!ok && tid == 0) {
+        atomicExch(timeout_flag, 1);
+        tc::commit(&bars[1]);
+        mbar_wait_bounded(&bars[1], 0, kTcWaitProbes);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, 256);
+    }
+}
+
+}  // namespace gka

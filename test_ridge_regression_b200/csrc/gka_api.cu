@@ -475,12 +475,29 @@ static int backward_simt(const Tin *q, const Tin *k, const Tin *v, const float *
         }
     }
     // adjoint chunk increments and their reverse scan
-    const size_t sm_bd = sizeof(float) * 5 * (size_t)C * D;
-    if ((e = set_smem(k_bwd_delta<Tin, D>, sm_bd)) != cudaSuccess) return cuda_fail(e);
-    { ProfScope ps(GKA_KERNEL_BWD_DELTA, s);
-    k_bwd_delta<Tin, D><<<dim3(N, BH), kSimtThreads, sm_bd, s>>>(k, beta, gate, dout, states, xs,
-                                                                ys, cvec, adj, T, N, C); }
-    if (int rc = check_launch()) return rc;
+    bool delta_done = false;
+    if constexpr (std::is_same<Tin, __nv_bfloat16>::value && D == 128) {
+        if (tc_done && C == kBrC) {
+            // bf16, D = 128: the adjoint increments as fp16 MMAs
+            int *flag = nullptr;
+            if (int rc = timeout_flag_ptr(&flag)) return rc;
+            if ((e = set_smem(k_bwd_delta_tc, BwdDeltaTcSmem::bytes)) != cudaSuccess)
+                return cuda_fail(e);
+            { ProfScope ps(GKA_KERNEL_BWD_DELTA, s);
+            k_bwd_delta_tc<<<dim3(N, BH), kSimtThreads, BwdDeltaTcSmem::bytes, s>>>(
+                k, beta, gate, dout, states, xs, ys, cvec, adj, T, N, flag); }
+            if (int rc = check_launch()) return rc;
+            delta_done = true;
+        }
+    }
+    if (!delta_done) {
+        const size_t sm_bd = sizeof(float) * 5 * (size_t)C * D;
+        if ((e = set_smem(k_bwd_delta<Tin, D>, sm_bd)) != cudaSuccess) return cuda_fail(e);
+        { ProfScope ps(GKA_KERNEL_BWD_DELTA, s);
+        k_bwd_delta<Tin, D><<<dim3(N, BH), kSimtThreads, sm_bd, s>>>(k, beta, gate, dout, states,
+                                                                    xs, ys, cvec, adj, T, N, C); }
+        if (int rc = check_launch()) return rc;
+    }
     { ProfScope ps(GKA_KERNEL_ADJOINT_SCAN, s);
     k_adjoint_scan<<<dim3((DD2 / 4 + 255) / 256, BH), 256, 0, s>>>(adj, decay, N, DD2); }
     if (int rc = check_launch()) return rc;
