@@ -435,7 +435,7 @@ def main():
 
     # ---- solver study: Chebyshev vs gradient descent, Nesterov, conjugate gradient ----
     if not args.no_solver_study and world == 1:
-        result["solver_study"] = bench_solver_study(w, qd, kd, bd)
+        result["solver_study"] = bench_solver_study(w, qd, kd, bd, peaks)
 
     # ---- decode step: HBM-bound, 256 x 32 heads, fp32 state ----
     if not args.no_decode and world == 1:
@@ -565,21 +565,35 @@ def bench_backward(args, w, dev, qd, kd, vd, bd, flush, rank, world, barrier, pe
     fl = bwd_flops_per_head_token(w.D, BWD_CHUNK, w.r)
     head_tok = w.B * w.H * w.T
     dom = max(per_kernel, key=per_kernel.get)
-    achieved = fl.get(dom, 0) * head_tok / (per_kernel[dom] / 1e3) / 1e12
     peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
     total_fl = sum(fl[n] for n in per_kernel if n in fl) * head_tok
+    tc_rows = w.dtype == torch.bfloat16 and w.D == 128 and BWD_CHUNK == 32 and w.T % 64 == 0
+    if dom == "bwd_rows" and tc_rows:
+        # the row products run as fp16 MMAs; what they must move bounds them: per chunk the
+        # four fp32 D x D matrices, the k, v, g (bf16) and x, y (fp32) rows in, R1..R4 and
+        # the per-token scalars out
+        D, C = w.D, BWD_CHUNK
+        per_tok = 4 * D * D * 4 / C + 3 * D * 2 + 2 * D * 4 + 4 * D * 4 + 4 * 4
+        byts = per_tok * head_tok
+        ach = byts / (per_kernel[dom] / 1e3) / 1e9
+        roof = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": ach / peaks["hbm_gbs"], "traffic": None,
+                "peak_source": "measured copy bandwidth", "algorithmic_per_step": byts}
+    else:
+        achieved = fl.get(dom, 0) * head_tok / (per_kernel[dom] / 1e3) / 1e12
+        roof = {"bound": "alu", "kernel": dom, "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 flop x max SM clock",
+                "algorithmic_per_step": fl.get(dom, 0) * head_tok}
     return {"chunk": BWD_CHUNK, "steps": steps, "ms_per_step": total_ms / steps,
             "tokens_per_s": world * w.B * w.T * steps / (total_ms / 1e3),
             "kernels_ms_per_step": per_kernel,
             "gpu_launches": sum(n for _, n in kt.values()),
-            "roofline": {"bound": "alu", "kernel": dom, "achieved": achieved, "peak": peak,
-                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
-                         "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 flop x max SM clock",
-                         "algorithmic_per_step": fl.get(dom, 0) * head_tok},
+            "roofline": roof,
             "step_frac_of_fp32_peak": total_fl / (total_ms / steps / 1e3) / 1e12 / peak}
 
 
-def bench_solver_study(w, qd, kd, bd):
+def bench_solver_study(w, qd, kd, bd, peaks):
     """Residual histories of the four solvers on every token of the workload (the
     pages' Fig. 1a on its random-regression shape) and the final mean residual for
     several regularisation strengths (Fig. 8); one timed run per solver at the
@@ -603,6 +617,16 @@ def bench_solver_study(w, qd, kd, bd):
                                        [..., -1].double().mean())
                          for solver in gka.SOLVERS}
     out["a_sweep_final_mean_residual_r30"] = sweep
+    # ALU roofline of the study kernel (Chebyshev run): r products A x per token, each
+    # 2 D^2 + 4 C D flops in chunk form (CG takes two per step)
+    head_tok = w.B * w.H * w.T
+    fl = w.r * (2 * w.D * w.D + 4 * chunk * w.D) * head_tok
+    peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+    ach = fl / (out["ms"]["chebyshev"] / 1e3) / 1e12
+    out["roofline"] = {"bound": "alu", "kernel": "solver_study (chebyshev)", "achieved": ach,
+                       "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+                       "algorithmic_per_run": fl,
+                       "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 flop x max SM clock"}
     if gka.device_status() != 0:
         raise RuntimeError("device status error after the solver study")
     return out
