@@ -76,6 +76,14 @@ def test_backward_bf16_state_pass_gate_resets():
     check_backward(q, k, v, beta, 0.5, 20, 32, gate=gate, seed=8)
 
 
+@pytest.mark.parametrize("D,C", [(64, 32), (128, 16), (32, 16)])
+def test_backward_bf16_cuda_core_shapes(D, C):
+    # bf16 inputs with D != 128 (all on CUDA cores), or D = 128 with chunk 16 (tensor-core
+    # iterates and adjoint solve, the row products and increments on CUDA cores)
+    q, k, v, beta = make_inputs(1, 2, 128, D, torch.bfloat16, 2.0, 1.0, seed=880 + D + C)
+    check_backward(q, k, v, beta, 0.5, 12, C, seed=9 + D)
+
+
 def test_backward_write_gate_and_resets():
     q, k, v, beta = make_inputs(1, 2, 128, 64, torch.float32, 1.0, 1.0, seed=830)
     gate = make_gate((1, 2, 128), 830)
