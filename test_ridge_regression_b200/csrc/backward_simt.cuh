@@ -40,6 +40,7 @@
 
 #include "chunk_simt.cuh"
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace gka {
 
@@ -608,6 +609,7 @@ k_bwd_u(const Tin *__restrict__ k, const Tin *__restrict__ v, const float *__res
     const int lane = tid & 31, warp = tid >> 5;
     const size_t tok0 = (size_t)bh * T + (size_t)n * C;
     const float *Ms = states + ((size_t)bh * (N + 1) + n) * 2 * D * D + D * D;
+    if (tid == 32) bulk_prefetch_l2(Ms, D * D * 4);   // read once P is formed
     chunk_log_prefix(beta + tok0, C, ell, wtot);
     if (tid < C) s_b[tid] = decay_exp(ell[tid]);
     for (int e = tid; e < C * D; e += kSimtThreads) {

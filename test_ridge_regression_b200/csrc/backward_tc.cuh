@@ -160,6 +160,12 @@ k_bwd_rows_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restri
         mbar_init(&bars[2], 1);
         fence_mbar_init();
     }
+    if (tid == 32) {
+        // everything read after the rows: the four matrices and the fp32 y rows
+        bulk_prefetch_l2(Hs, 2 * D * D * 4);
+        bulk_prefetch_l2(EH, 2 * D * D * 4);
+        bulk_prefetch_l2(ys + tok0 * D, C * D * 4);
+    }
     if (warp == 0) {
         tc::tmem_alloc(tbase, 256);
         tc::tmem_relinquish();

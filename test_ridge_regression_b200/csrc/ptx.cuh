@@ -119,4 +119,10 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
         : "memory");
 }
 
+// Asks L2 to fetch `bytes` from global memory at src (16-byte aligned, a multiple
+// of 16 bytes) without waiting for it and without touching shared memory.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 }  // namespace gka
