@@ -8,6 +8,10 @@
 // two 128 x 128 x C products per chunk; the scan kernel adds them up.  With
 // the write gate g (nullable) every weight w_{C-1,i} is w_{C-1,i} g_i.
 //
+// C = 64 or 128 in the forward (tensor maps of 64-row boxes), C = 32 in the
+// backward's recompute of the chunk states (32-row boxes; no per-token decays
+// or norm bounds: tokdec and bound_inc are NULL there).
+//
 // One CTA (4 warps) per chunk.  K and V arrive by TMA (bf16) and are turned
 // into fp16 with a power-of-two scale below 1 (exact).  The weighted keys
 // diag(w) K are split into fp16 hi + lo parts (hi + lo carries 22 mantissa
@@ -47,7 +51,7 @@ struct DeltaSmem {
 };
 
 struct DeltaMaps {
-    CUtensorMap k, v;    // [B*H*T][128] bf16, box 64 x 64, 128B swizzle
+    CUtensorMap k, v;    // [B*H*T][128] bf16, box 64 x min(C, 64), 128B swizzle
     CUtensorMap out;     // fp32 states [B*H*(N+1)*2*128][128], box 32 x 128, 128B swizzle
 };
 
@@ -80,14 +84,15 @@ k_chunk_delta_tc(const __grid_constant__ DeltaMaps maps, const float *__restrict
         fence_mbar_init();
     }
     __syncthreads();
+    constexpr int BOX = C < 64 ? C : 64;   // rows per TMA box
     if (tid == 0) {
         mbar_arrive_expect_tx(bar_load, 2 * C * 256);
         for (int h = 0; h < 2; ++h)
-            for (int rb = 0; rb < C / 64; ++rb) {
-                tc::tma_load_2d(sm + L::KT + h * C * 128 + rb * 8192, &maps.k, h * 64,
-                                (int)tok0 + rb * 64, bar_load);
-                tc::tma_load_2d(sm + L::VT + h * C * 128 + rb * 8192, &maps.v, h * 64,
-                                (int)tok0 + rb * 64, bar_load);
+            for (int rb = 0; rb < C / BOX; ++rb) {
+                tc::tma_load_2d(sm + L::KT + h * C * 128 + rb * BOX * 128, &maps.k, h * 64,
+                                (int)tok0 + rb * BOX, bar_load);
+                tc::tma_load_2d(sm + L::VT + h * C * 128 + rb * BOX * 128, &maps.v, h * 64,
+                                (int)tok0 + rb * BOX, bar_load);
             }
     }
     if (warp == 0) {
@@ -96,11 +101,13 @@ k_chunk_delta_tc(const __grid_constant__ DeltaMaps maps, const float *__restrict
     }
     chunk_log_prefix(beta + tok0, C, ell, wtot);
     if (tid < C) {
-        const float bt = decay_exp(tid == 0 ? ell[0] : ell[tid] - ell[tid - 1]);
-        tokdec[tok0 + tid] = (float)(ell[tid] * 1.4426950408889634);
-        tokdec[plane + tok0 + tid] = decay_exp(ell[tid]);
-        tokdec[2 * plane + tok0 + tid] = bt;
-        tokdec[3 * plane + tok0 + tid] = bt * bt;
+        if (tokdec) {
+            const float bt = decay_exp(tid == 0 ? ell[0] : ell[tid] - ell[tid - 1]);
+            tokdec[tok0 + tid] = (float)(ell[tid] * 1.4426950408889634);
+            tokdec[plane + tok0 + tid] = decay_exp(ell[tid]);
+            tokdec[2 * plane + tok0 + tid] = bt;
+            tokdec[3 * plane + tok0 + tid] = bt * bt;
+        }
         float w = decay_exp(ell[C - 1] - ell[tid]);
         if (gate) w *= gate[tok0 + tid];   // write gate of token tid
         s_wt[tid] = w;
@@ -154,7 +161,7 @@ k_chunk_delta_tc(const __grid_constant__ DeltaMaps maps, const float *__restrict
         tc::commit(bar_mma);
     }
     // chunk decay and the norm-bound increments sum_i w_i ||k_i||^2, sum_i w_i ||v_i|| ||k_i||
-    {
+    if (bound_inc) {
         float bhs = 0.f, bms = 0.f;
         for (int i = tid; i < C; i += kTcThreads) {
             const float w = s_wt[i];
@@ -187,8 +194,10 @@ k_chunk_delta_tc(const __grid_constant__ DeltaMaps maps, const float *__restrict
     if (ok) {
         if (tid == 0) {
             decay[(size_t)bh * N + n] = decay_exp(lend);
-            bound_inc[((size_t)bh * N + n) * 2] = red[8] + red[9] + red[10] + red[11];
-            bound_inc[((size_t)bh * N + n) * 2 + 1] = red[12] + red[13] + red[14] + red[15];
+            if (bound_inc) {
+                bound_inc[((size_t)bh * N + n) * 2] = red[8] + red[9] + red[10] + red[11];
+                bound_inc[((size_t)bh * N + n) * 2 + 1] = red[12] + red[13] + red[14] + red[15];
+            }
         }
         // row d of dH and dM (thread d = TMEM lane d) -> swizzled staging -> TMA store
         // into state slot n + 1, 64 columns (two 32-column boxes) per round

@@ -419,12 +419,39 @@ static int backward_simt(const Tin *q, const Tin *k, const Tin *v, const float *
 
     // forward recompute: chunk states, norms and the iterates x_t (bf16, D = 128: the
     // iterates and norms from the tensor-core forward, the fp32 chunk states here)
-    const size_t sm_delta = sizeof(float) * 3 * (size_t)C * D;
-    if ((e = set_smem(k_chunk_delta<Tin, D>, sm_delta)) != cudaSuccess) return cuda_fail(e);
-    { ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
-    k_chunk_delta<Tin, D><<<dim3(N, BH), kSimtThreads, sm_delta, s>>>(k, v, beta, gate, states,
-                                                                        decay, nullptr, T, N, C); }
-    if (int rc = check_launch()) return rc;
+    bool delta_tc = false;
+    if constexpr (std::is_same<Tin, __nv_bfloat16>::value && D == 128) {
+        if (L.tc_recompute && C == 32) {
+            // the increments as fp16 MMAs (hi + lo weighted keys, fp32 accuracy)
+            int *flag = nullptr;
+            if (int rc = timeout_flag_ptr(&flag)) return rc;
+            DeltaMaps dm;
+            if (int rc = rows128_map(&dm.k, k, (uint64_t)BH * T, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                                     64, 32))
+                return rc;
+            if (int rc = rows128_map(&dm.v, v, (uint64_t)BH * T, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                                     64, 32))
+                return rc;
+            if (int rc = rows128_map(&dm.out, states, (uint64_t)BH * (N + 1) * 2 * D,
+                                     CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 32, 128))
+                return rc;
+            if ((e = set_smem(k_chunk_delta_tc<32>, DeltaSmem<32>::bytes)) != cudaSuccess)
+                return cuda_fail(e);
+            { ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
+            k_chunk_delta_tc<32><<<dim3(N, BH), kTcThreads, DeltaSmem<32>::bytes, s>>>(
+                dm, beta, gate, states, decay, nullptr, nullptr, 0, T, N, flag); }
+            if (int rc = check_launch()) return rc;
+            delta_tc = true;
+        }
+    }
+    if (!delta_tc) {
+        const size_t sm_delta = sizeof(float) * 3 * (size_t)C * D;
+        if ((e = set_smem(k_chunk_delta<Tin, D>, sm_delta)) != cudaSuccess) return cuda_fail(e);
+        { ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
+        k_chunk_delta<Tin, D><<<dim3(N, BH), kSimtThreads, sm_delta, s>>>(
+            k, v, beta, gate, states, decay, nullptr, T, N, C); }
+        if (int rc = check_launch()) return rc;
+    }
     { ProfScope ps(GKA_KERNEL_STATE_SCAN, s);
     k_state_scan<<<dim3((DD2 + 1023) / 1024, BH), 256, 0, s>>>(states, decay, nullptr, nullptr,
                                                              nullptr, nullptr, N, DD2, true); }
