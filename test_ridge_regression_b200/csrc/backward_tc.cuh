@@ -340,7 +340,10 @@ namespace gka {
 //   dE^M = (b o G)^T X,      e_i = sum_{s>=i} b_s c_s w_si,
 // two 128 x 128 x 32 accumulations (operands MN-major from token-row tiles, fp16
 // with power-of-two scales; the two products of dE^H scaled alike so that they
-// share one accumulator), the H_start term added in fp32 on the way out.
+// share one accumulator), the H_start term added in fp32 on the way out.  The
+// increments leave through shared memory: 32 columns of every row per round in a
+// [128][32] fp32 box (128B swizzle), written by TMA stores while the next round
+// fills the other of two buffers.
 // grid (N, B*H), block 256.
 // ---------------------------------------------------------------------------
 struct BwdDeltaTcSmem {
@@ -349,7 +352,9 @@ struct BwdDeltaTcSmem {
     static constexpr uint32_t TE = TX + 8192;    // -(e o k~) rows
     static constexpr uint32_t TK = TE + 8192;    // k~ rows
     static constexpr uint32_t TG = TK + 8192;    // (b o g) rows
-    static constexpr uint32_t ELL = TG + 8192;   // double[32] + double[8]
+    static constexpr uint32_t STG0 = TY;         // output staging: 2 x [128][32] fp32 over the
+    static constexpr uint32_t STG1 = TG + 8192;  // row tiles (free after the products), and its own
+    static constexpr uint32_t ELL = STG1 + 32768;   // double[32] + double[8]
     static constexpr uint32_t SC = ELL + 320;    // float[32] b, float[32] e, float[32] sqrt(w)
     static constexpr uint32_t MRED = SC + 384;   // float[16]
     static constexpr uint32_t BARS = MRED + 64;  // 2 mbarriers: products, drain
@@ -389,7 +394,9 @@ k_bwd_delta_tc(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ be
                const float *__restrict__ gate, const __nv_bfloat16 *__restrict__ dout,
                const float *__restrict__ states, const float *__restrict__ xs,
                const float *__restrict__ ys, const float *__restrict__ cvec,
-               float *__restrict__ adj, int T, int N, int *__restrict__ timeout_flag) {
+               const __grid_constant__ CUtensorMap adj_map, int T, int N,
+               int *__restrict__ timeout_flag) {
+    // adj_map: the adjoint states [B*H*(N+1)*2*128][128] fp32, box 32 x 128, 128B swizzle
     using L = BwdDeltaTcSmem;
     constexpr int D = 128, C = kBrC;
     extern __shared__ uint8_t smraw[];
@@ -470,31 +477,58 @@ k_bwd_delta_tc(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ be
     }
     bool ok = mbar_wait_bounded(&bars[0], 0, kTcWaitProbes);
     tc::fence_after_sync();
-    // row p = TMEM lane of this thread, columns 64 wg .. 64 wg + 63
+    ok = __syncthreads_and(ok);
+    // row p = TMEM lane of this thread; round (m, j) covers columns 64 wg + 32 j .. + 31
+    // of dE^H (m = 0, with the H_start term) or dE^M (m = 1)
     const int quarter = warp & 3, wg = warp >> 2, p = quarter * 32 + lane;
-    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(wg * 64);
-    const float *Hst = states + ((size_t)bh * (N + 1) + n) * 2 * D * D + (size_t)p * D + wg * 64;
-    float *outH = adj + ((size_t)bh * (N + 1) + n) * 2 * D * D + (size_t)p * D + wg * 64;
-    float *outM = outH + D * D;
+    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+    const float *Hst = states + ((size_t)bh * (N + 1) + n) * 2 * D * D + (size_t)p * D;
+    const int orow = (int)(((size_t)bh * (N + 1) + n) * 2 * D);
     const float uH = 1.f / S, uM = 1.f / (sG * sX);
+#pragma unroll 1
+    for (int round = 0; round < 4 && ok; ++round) {
+        const int m = round >> 1, col = wg * 64 + (round & 1) * 32;
+        // buffer round % 2; the stores that last read it (round - 2) were waited for
+        // before the previous round's barrier
+        const uint32_t rowb = sb + ((round & 1) ? L::STG1 : L::STG0) + wg * 16384 + p * 128;
+        float a[32];
+        tc::tmem_ld16(tl + m * 128 + col, a);
+        tc::tmem_ld16(tl + m * 128 + col + 16, a + 16);
+        float4 h[8];
+        if (m == 0) {
 #pragma unroll
-    for (int cb = 0; cb < 64; cb += 16) {
-        float a[16], m[16];
-        tc::tmem_ld16(tl + cb, a);
-        tc::tmem_ld16(tl + 128 + cb, m);
+            for (int c = 0; c < 8; ++c) h[c] = *reinterpret_cast<const float4 *>(Hst + col + 4 * c);
+        }
         tc::tmem_wait_ld();
-        if (ok) {
 #pragma unroll
-            for (int j = 0; j < 16; j += 4) {
-                const float4 h = *reinterpret_cast<const float4 *>(Hst + cb + j);
-                *reinterpret_cast<float4 *>(outH + cb + j) =
-                    make_float4(fmaf(-c1, h.x, a[j] * uH), fmaf(-c1, h.y, a[j + 1] * uH),
-                                fmaf(-c1, h.z, a[j + 2] * uH), fmaf(-c1, h.w, a[j + 3] * uH));
-                *reinterpret_cast<float4 *>(outM + cb + j) =
-                    make_float4(m[j] * uM, m[j + 1] * uM, m[j + 2] * uM, m[j + 3] * uM);
+        for (int c = 0; c < 8; ++c) {
+            float o0, o1, o2, o3;
+            if (m == 0) {
+                o0 = fmaf(-c1, h[c].x, a[4 * c] * uH);
+                o1 = fmaf(-c1, h[c].y, a[4 * c + 1] * uH);
+                o2 = fmaf(-c1, h[c].z, a[4 * c + 2] * uH);
+                o3 = fmaf(-c1, h[c].w, a[4 * c + 3] * uH);
+            } else {
+                o0 = a[4 * c] * uM;
+                o1 = a[4 * c + 1] * uM;
+                o2 = a[4 * c + 2] * uM;
+                o3 = a[4 * c + 3] * uM;
             }
+            st_shared_v4(rowb + ((c ^ p) & 7) * 16, __float_as_uint(o0), __float_as_uint(o1),
+                         __float_as_uint(o2), __float_as_uint(o3));
+        }
+        fence_proxy_async_smem();
+        if (tid == 0) tc::bulk_wait_read0();   // the previous round's stores have read their buffer
+        __syncthreads();
+        if (tid == 0) {
+            const uint32_t buf = (round & 1) ? L::STG1 : L::STG0;
+            const int x = (round & 1) * 32;
+            tc::tma_store_2d(&adj_map, x, orow + m * D, sm + buf);
+            tc::tma_store_2d(&adj_map, 64 + x, orow + m * D, sm + buf + 16384);
+            tc::bulk_commit();
         }
     }
+    if (tid == 0) tc::bulk_wait0();
     if (!ok && tid == 0) {
         atomicExch(timeout_flag, 1);
         tc::commit(&bars[1]);

@@ -517,11 +517,15 @@ static int backward_simt(const Tin *q, const Tin *k, const Tin *v, const float *
             // bf16, D = 128: the adjoint increments as fp16 MMAs
             int *flag = nullptr;
             if (int rc = timeout_flag_ptr(&flag)) return rc;
+            CUtensorMap adj_map;
+            if (int rc = rows128_map(&adj_map, adj, (uint64_t)BH * (N + 1) * 2 * D,
+                                     CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 32, 128))
+                return rc;
             if ((e = set_smem(k_bwd_delta_tc, BwdDeltaTcSmem::bytes)) != cudaSuccess)
                 return cuda_fail(e);
             { ProfScope ps(GKA_KERNEL_BWD_DELTA, s);
             k_bwd_delta_tc<<<dim3(N, BH), kSimtThreads, BwdDeltaTcSmem::bytes, s>>>(
-                k, beta, gate, dout, states, xs, ys, cvec, adj, T, N, flag); }
+                k, beta, gate, dout, states, xs, ys, cvec, adj_map, T, N, flag); }
             if (int rc = check_launch()) return rc;
             delta_done = true;
         }
