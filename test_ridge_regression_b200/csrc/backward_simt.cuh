@@ -573,105 +573,6 @@ k_bwd_rows(const Tin *__restrict__ k, const Tin *__restrict__ v, const Tin *__re
 }
 
 // ---------------------------------------------------------------------------
-// k_bwd_u: the right-hand side of the adjoint solve, one CTA per chunk:
-//   u_t = M_t^T g_t = b_t M_s^T g_t + sum_{i<=t} w_ti k~_i (v~_i . g_t),
-// written in the input dtype (the tensor-core solve reads it as its q).  M_s is
-// staged in column halves (as in k_bwd_rows) and M_s^T g formed in register tiles;
-// the intra-chunk term goes through the C x C matrix P[t][i] = w_ti (v~_i . g_t).
-// grid (N, B*H), block 256, shared memory BwdUSmem<Tin, D, C>::bytes.
-// ---------------------------------------------------------------------------
-template <typename Tin, int D, int C>
-struct BwdUSmem {
-    static constexpr int NH = D >= 64 ? 2 : 1, HC = D / NH, DP = HC + 4, KP = D + 4;
-    static constexpr size_t bytes = sizeof(float) * ((size_t)D * DP + 2 * (size_t)C * KP +
-                                                     (size_t)C * (C + 1)) +
-                                    sizeof(Tin) * (size_t)C * D;
-};
-
-template <typename Tin, int D, int C>
-__global__ void __launch_bounds__(kSimtThreads, 2)
-k_bwd_u(const Tin *__restrict__ k, const Tin *__restrict__ v, const float *__restrict__ beta,
-        const float *__restrict__ gate, const Tin *__restrict__ dout,
-        const float *__restrict__ states, Tin *__restrict__ u_out, int T, int N) {
-    using L = BwdUSmem<Tin, D, C>;
-    constexpr int NH = L::NH, HC = L::HC, DP = L::DP, KP = L::KP, CP = C + 1;
-    constexpr int TT = C / 8, CC = HC / 32;
-    static_assert(kSimtThreads == 256 && C % 8 == 0 && HC % 32 == 0, "tiling");
-    extern __shared__ __align__(16) uint8_t smb[];
-    float *Mt = reinterpret_cast<float *>(smb);   // [D][DP] columns of M_s
-    float *Kh = Mt + D * DP;                      // [C][KP] k~ = sqrt(w) k
-    float *Vh = Kh + C * KP;                      // [C][KP] v~
-    float *Pm = Vh + C * KP;                      // [C][CP] P[t][i]
-    Tin *Gr = reinterpret_cast<Tin *>(Pm + C * CP);   // [C][D] g
-    __shared__ double ell[C], wtot[kSimtThreads / 32];
-    __shared__ float s_b[C];
-    const int n = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
-    const int lane = tid & 31, warp = tid >> 5;
-    const size_t tok0 = (size_t)bh * T + (size_t)n * C;
-    const float *Ms = states + ((size_t)bh * (N + 1) + n) * 2 * D * D + D * D;
-    if (tid == 32) bulk_prefetch_l2(Ms, D * D * 4);   // read once P is formed
-    chunk_log_prefix(beta + tok0, C, ell, wtot);
-    if (tid < C) s_b[tid] = decay_exp(ell[tid]);
-    for (int e = tid; e < C * D; e += kSimtThreads) {
-        const int t = e / D, d = e % D;
-        const size_t g = tok0 * D + e;
-        const float sg = gate ? sqrtf(gate[tok0 + t]) : 1.f;
-        Kh[t * KP + d] = load_f(k + g) * sg;
-        Vh[t * KP + d] = load_f(v + g) * sg;
-        Gr[e] = dout[g];
-    }
-    __syncthreads();
-    // P[t][i] = w_ti (v~_i . g_t), i <= t
-    for (int e = tid; e < C * C; e += kSimtThreads) {
-        const int t = e / C, i = e % C;
-        float acc = 0.f;
-        if (i <= t) {
-            for (int d = 0; d < D; ++d) acc = fmaf(Vh[i * KP + d], to_f(Gr[t * D + d]), acc);
-            acc *= decay_exp(ell[t] - ell[i]);
-        }
-        Pm[t * CP + i] = acc;
-    }
-    const int t0 = warp * TT;
-    for (int h = 0; h < NH; ++h) {
-        bwd_stage<D, HC, DP>(Mt, Ms, 0, h);   // barriers inside: P and the rows are complete
-        float acc[TT][CC];
-#pragma unroll
-        for (int a = 0; a < TT; ++a)
-#pragma unroll
-            for (int b = 0; b < CC; ++b) acc[a][b] = 0.f;
-#pragma unroll 2
-        for (int d = 0; d < D; d += 4) {
-            float m[4][CC];
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-#pragma unroll
-                for (int b = 0; b < CC; ++b) m[q][b] = Mt[(d + q) * DP + lane + 32 * b];
-#pragma unroll
-            for (int a = 0; a < TT; ++a) {
-                float r[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) r[q] = to_f(Gr[(t0 + a) * D + d + q]);
-#pragma unroll
-                for (int b = 0; b < CC; ++b)
-                    acc[a][b] = fmaf(r[0], m[0][b], fmaf(r[1], m[1][b],
-                                fmaf(r[2], m[2][b], fmaf(r[3], m[3][b], acc[a][b]))));
-            }
-        }
-#pragma unroll
-        for (int a = 0; a < TT; ++a) {
-            const int t = t0 + a;
-#pragma unroll
-            for (int b = 0; b < CC; ++b) {
-                const int c = h * HC + lane + 32 * b;
-                float x = acc[a][b] * s_b[t];
-                for (int i = 0; i <= t; ++i) x = fmaf(Pm[t * CP + i], Kh[i * KP + c], x);
-                store_f(u_out + (tok0 + t) * D + c, x);
-            }
-        }
-    }
-}
-
-// ---------------------------------------------------------------------------
 // k_bwd_grads: dk, dv, dbeta and the write-gate gradient of one chunk.
 // Shared memory: the chunk's k, x, y, g rows (fp32, rows padded to 16 bytes),
 // the C x C matrices, and one region that holds the v rows until their dot

@@ -334,6 +334,135 @@ k_bwd_rows_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restri
 namespace gka {
 
 // ---------------------------------------------------------------------------
+// k_bwd_u_tc: the right-hand side of the adjoint solve for one 32-token chunk
+// (bf16 inputs, D = 128; the tensor-core solve then solves for y on it):
+//   u_t = M_t^T g_t = b_t M_s^T g_t + sum_{i<=t} w_ti k~_i (v~_i . g_t),
+// M_s^T G^T as eight 128 x 32 x 16 fp16 MMAs (M_s and the g rows converted with
+// power-of-two scales, as in k_bwd_rows_tc) while the CUDA cores form the
+// intra-chunk matrix P[t][i] = w_ti (v~_i . g_t); thread (row c, 16 tokens) adds
+// the two parts and writes u in bf16 (the precision the tensor-core solve reads).
+// grid (N, B*H), block 256.
+// ---------------------------------------------------------------------------
+struct BwdUTcSmem {
+    static constexpr int KP = 132;                 // fp32 row pitch of k~, v~
+    static constexpr uint32_t MB = 0;              // [2][128][64] fp16 M_s
+    static constexpr uint32_t RG = MB + 32768;     // [2][32][64] fp16 g rows
+    static constexpr uint32_t KH = RG + 8192;      // float[32][KP] k~
+    static constexpr uint32_t VH = KH + 32 * KP * 4;   // float[32][KP] v~
+    static constexpr uint32_t PM = VH + 32 * KP * 4;   // float[32][33] P
+    static constexpr uint32_t GR = PM + 32 * 33 * 4;   // bf16 [32][128] g
+    static constexpr uint32_t MRED = GR + 8192;    // float[16]
+    static constexpr uint32_t BARS = MRED + 64;    // 2 mbarriers: product, drain
+    static constexpr uint32_t TBASE = BARS + 16;
+    static constexpr uint32_t END = TBASE + 16;
+    static constexpr size_t bytes = END + 1024;    // + alignment slack
+};
+
+__global__ void __launch_bounds__(kSimtThreads, 2)
+k_bwd_u_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
+           const float *__restrict__ beta, const float *__restrict__ gate,
+           const __nv_bfloat16 *__restrict__ dout, const float *__restrict__ states,
+           __nv_bfloat16 *__restrict__ u_out, int T, int N, int *__restrict__ timeout_flag) {
+    using L = BwdUTcSmem;
+    constexpr int D = 128, C = kBrC, KP = L::KP, CP = C + 1;
+    extern __shared__ uint8_t smraw[];
+    uint8_t *sm = smem_align1024(smraw);
+    const uint32_t sb = smem_u32(sm);
+    float *Kh = reinterpret_cast<float *>(sm + L::KH);
+    float *Vh = reinterpret_cast<float *>(sm + L::VH);
+    float *Pm = reinterpret_cast<float *>(sm + L::PM);
+    __nv_bfloat16 *Gr = reinterpret_cast<__nv_bfloat16 *>(sm + L::GR);
+    float *mred = reinterpret_cast<float *>(sm + L::MRED);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BARS);
+    uint32_t *tbase = reinterpret_cast<uint32_t *>(sm + L::TBASE);
+    __shared__ double ell[C], wtot[kSimtThreads / 32];
+    __shared__ float s_b[C];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n = blockIdx.x, bh = blockIdx.y;
+    const size_t tok0 = (size_t)bh * T + (size_t)n * C;
+    const float *Ms = states + ((size_t)bh * (N + 1) + n) * 2 * D * D + D * D;
+
+    if (tid == 0) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tc::tmem_alloc(tbase, 32);
+        tc::tmem_relinquish();
+    }
+    chunk_log_prefix(beta + tok0, C, ell, wtot);
+    if (tid < C) s_b[tid] = decay_exp(ell[tid]);
+    for (int e = tid; e < C * D; e += kSimtThreads) {
+        const int t = e / D, d = e % D;
+        const size_t g = tok0 * D + e;
+        const float sg = gate ? sqrtf(gate[tok0 + t]) : 1.f;
+        Kh[t * KP + d] = __bfloat162float(k[g]) * sg;
+        Vh[t * KP + d] = __bfloat162float(v[g]) * sg;
+        Gr[e] = dout[g];
+    }
+    const float sG = rows_to_f16_tile(dout + tok0 * D, sb + L::RG, mred, false, nullptr);
+    const float sM = mat_to_f16_tile(Ms, sb + L::MB, mred, nullptr, nullptr, nullptr);
+    fence_proxy_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tbase;
+    if (tid == 0) {
+        constexpr uint32_t ID_T = tc::idesc_f16(128, C, true, false);   // A = M_s^T (MN-major)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+            tc::mma_f16(tmem, tc::sdesc(sb + L::MB + kk * 2048, 16384, 1024),
+                        tc::sdesc(sb + L::RG + (kk >> 2) * (C * 128) + (kk & 3) * 32, 16, 1024),
+                        ID_T, kk > 0);
+        tc::commit(&bars[0]);
+    }
+    // P[t][i] = w_ti (v~_i . g_t), i <= t, while the product runs
+    for (int e = tid; e < C * C; e += kSimtThreads) {
+        const int t = e / C, i = e % C;
+        float acc = 0.f;
+        if (i <= t) {
+            for (int d = 0; d < D; d += 4) {
+                const float4 vv = *reinterpret_cast<const float4 *>(Vh + i * KP + d);
+                const __nv_bfloat162 g01 = *reinterpret_cast<const __nv_bfloat162 *>(Gr + t * D + d);
+                const __nv_bfloat162 g23 = *reinterpret_cast<const __nv_bfloat162 *>(Gr + t * D + d + 2);
+                acc = fmaf(vv.x, __low2float(g01), fmaf(vv.y, __high2float(g01),
+                      fmaf(vv.z, __low2float(g23), fmaf(vv.w, __high2float(g23), acc))));
+            }
+            acc *= decay_exp(ell[t] - ell[i]);
+        }
+        Pm[t * CP + i] = acc;
+    }
+    __syncthreads();
+    bool ok = mbar_wait_bounded(&bars[0], 0, kTcWaitProbes);
+    tc::fence_after_sync();
+    // thread (row c = TMEM lane, tokens 16 wg .. 16 wg + 15)
+    const int quarter = warp & 3, wg = warp >> 2, c = quarter * 32 + lane;
+    float acc[16];
+    tc::tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(wg * 16), acc);
+    tc::tmem_wait_ld();
+    const float um = 1.f / (sM * sG);
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+        const int t = wg * 16 + u;
+        float x = acc[u] * um * s_b[t];
+        for (int i = 0; i <= t; ++i) x = fmaf(Pm[t * CP + i], Kh[i * KP + c], x);
+        if (ok) u_out[(tok0 + t) * D + c] = __float2bfloat16_rn(x);
+    }
+    if (!ok && tid == 0) {
+        atomicExch(timeout_flag, 1);
+        tc::commit(&bars[1]);
+        mbar_wait_bounded(&bars[1], 0, kTcWaitProbes);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, 32);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // k_bwd_delta_tc: the adjoint increments of one 32-token chunk on tcgen05
 // (the work of k_bwd_delta):
 //   dE^H = -(b o Y)^T X - (e o K~)^T K~ - (sum_s b_s^2 c_s) H_start,

@@ -485,14 +485,21 @@ static int backward_simt(const Tin *q, const Tin *k, const Tin *v, const float *
     // adjoint solve: dq = y, c (bf16, D = 128: u on CUDA cores, rounded to bf16, then the
     // tensor-core solve on it with the tensor-core forward's chunk states)
     Tin *u16 = tc_done ? reinterpret_cast<Tin *>(ws + L.u16) : nullptr;
-    if (u16 && C == 32) {
-        // u alone, one CTA per chunk (the solve runs on the tensor cores below)
-        constexpr size_t sm_u = BwdUSmem<Tin, D, 32>::bytes;
-        if ((e = set_smem(k_bwd_u<Tin, D, 32>, sm_u)) != cudaSuccess) return cuda_fail(e);
-        { ProfScope ps(GKA_KERNEL_BWD_SOLVE, s);
-        k_bwd_u<Tin, D, 32><<<dim3(N, BH), kSimtThreads, sm_u, s>>>(k, v, beta, gate, dout,
-                                                                   states, u16, T, N); }
-    } else {
+    bool u_done = false;
+    if constexpr (std::is_same<Tin, __nv_bfloat16>::value && D == 128) {
+        if (u16 && C == kBrC) {
+            // u alone, M_s^T G^T as fp16 MMAs
+            int *flag = nullptr;
+            if (int rc = timeout_flag_ptr(&flag)) return rc;
+            if ((e = set_smem(k_bwd_u_tc, BwdUTcSmem::bytes)) != cudaSuccess) return cuda_fail(e);
+            { ProfScope ps(GKA_KERNEL_BWD_SOLVE, s);
+            k_bwd_u_tc<<<dim3(N, BH), kSimtThreads, BwdUTcSmem::bytes, s>>>(
+                k, v, beta, gate, dout, states, u16, T, N, flag); }
+            u_done = true;
+        }
+    }
+    if (!u_done) {
+        // u (into u16 for the tensor-core solve, C = 16) or the whole adjoint solve
         if ((e = set_smem(k_bwd_solve<Tin, D>, sm_solve)) != cudaSuccess) return cuda_fail(e);
         { ProfScope ps(GKA_KERNEL_BWD_SOLVE, s);
         k_bwd_solve<Tin, D><<<dim3(C / kSolveTG, N, BH), kSimtThreads, sm_solve, s>>>(
