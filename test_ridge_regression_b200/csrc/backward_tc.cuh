@@ -12,7 +12,9 @@
 // Every matrix is converted in shared memory to fp16 with a power-of-two scale
 // that puts its largest entry below 1 (relative rounding 2^-11, as the forward's
 // fp16 state copies); k, v, g tiles likewise, x per token.  The accumulators are
-// fp32.  Two phases reuse the matrix tiles: (H_s, M_s) then (E^H, E^M).
+// fp32.  Two phases reuse the matrix tiles: (H_s, M_s) then (E^H, E^M); eh takes
+// H_s and M_s from the fp16 copies that E^H and E^M overwrite (E in fp32), so each
+// matrix is read from memory once.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -59,14 +61,14 @@ __device__ __forceinline__ float block_max256(float v, float *red) {
 // fp32 row-major 128 x 128 matrix -> fp16 [2][128][64] swizzled tile, scaled by a
 // power of two below 1/max.  Thread (row r = tid / 2, column half h = tid % 2) holds
 // its 64 elements in registers between the max and the conversion.
-// dotw (nullable): accumulates sum A * W over the thread's elements into *dot;
-// sq2 (nullable): accumulates sum A^2.  Returns the scale.
+// prev_scale > 0: the tile holds another matrix W as fp16 scaled by prev_scale; each
+// thread reads the entries it overwrites and accumulates sum A * W into *dot (W at
+// fp16 precision, A in fp32).  sq2 (nullable): accumulates sum A^2.  Returns the scale.
 __device__ __forceinline__ float mat_to_f16_tile(const float *__restrict__ A, uint32_t tile,
-                                                 float *red, const float *__restrict__ dotw,
-                                                 float *dot, float *sq2) {
+                                                 float *red, float prev_scale, float *dot,
+                                                 float *sq2) {
     const int tid = threadIdx.x, r = tid >> 1, h = tid & 1;
     const float4 *src = reinterpret_cast<const float4 *>(A + r * 128 + h * 64);
-    const float4 *wsrc = dotw ? reinterpret_cast<const float4 *>(dotw + r * 128 + h * 64) : nullptr;
     float mx = 0.f, dp = 0.f, s2 = 0.f;
     // all 16 loads of a pass are issued before their values are used
     float4 x[16];
@@ -77,24 +79,26 @@ __device__ __forceinline__ float mat_to_f16_tile(const float *__restrict__ A, ui
         mx = fmaxf(mx, fmaxf(fmaxf(fabsf(x[i].x), fabsf(x[i].y)), fmaxf(fabsf(x[i].z), fabsf(x[i].w))));
         s2 = fmaf(x[i].x, x[i].x, fmaf(x[i].y, x[i].y, fmaf(x[i].z, x[i].z, fmaf(x[i].w, x[i].w, s2))));
     }
-    if (wsrc) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float4 w = __ldg(wsrc + i);
-            dp = fmaf(x[i].x, w.x, fmaf(x[i].y, w.y, fmaf(x[i].z, w.z, fmaf(x[i].w, w.w, dp))));
-        }
-    }
-    if (dot) *dot += dp;
     if (sq2) *sq2 += s2;
     const float sc = inv_pow2_above(block_max256(mx, red));
     const uint32_t base = tile + (uint32_t)h * 16384u;
 #pragma unroll
     for (int c8 = 0; c8 < 8; ++c8) {
         const float4 a = x[2 * c8], b = x[2 * c8 + 1];
+        if (prev_scale > 0.f) {
+            const uint4 o = ld_shared_u4(base + (uint32_t)r * 128u + (((uint32_t)c8 ^ (uint32_t)r) & 7u) * 16u);
+            const float2 w0 = __half22float2(*reinterpret_cast<const __half2 *>(&o.x));
+            const float2 w1 = __half22float2(*reinterpret_cast<const __half2 *>(&o.y));
+            const float2 w2 = __half22float2(*reinterpret_cast<const __half2 *>(&o.z));
+            const float2 w3 = __half22float2(*reinterpret_cast<const __half2 *>(&o.w));
+            dp = fmaf(a.x, w0.x, fmaf(a.y, w0.y, fmaf(a.z, w1.x, fmaf(a.w, w1.y, dp))));
+            dp = fmaf(b.x, w2.x, fmaf(b.y, w2.y, fmaf(b.z, w3.x, fmaf(b.w, w3.y, dp))));
+        }
         const float v[8] = {a.x * sc, a.y * sc, a.z * sc, a.w * sc,
                             b.x * sc, b.y * sc, b.z * sc, b.w * sc};
         st_row8(base, (uint32_t)r, (uint32_t)(c8 * 8), v);
     }
+    if (prev_scale > 0.f) *dot += dp / prev_scale;
     return sc;
 }
 
@@ -176,8 +180,8 @@ k_bwd_rows_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restri
     const float sG = rows_to_f16_tile(dout + tok0 * D, sb + L::RG, mred, false, nullptr);
     rows_to_f16_tile(xs + tok0 * D, sb + L::RX, mred, true, xsc);
     float hs2 = 0.f, eh = 0.f;
-    const float sH = mat_to_f16_tile(Hs, sb + L::MA, mred, nullptr, nullptr, &hs2);
-    const float sM = mat_to_f16_tile(Ms, sb + L::MB, mred, nullptr, nullptr, nullptr);
+    const float sH = mat_to_f16_tile(Hs, sb + L::MA, mred, 0.f, nullptr, &hs2);
+    const float sM = mat_to_f16_tile(Ms, sb + L::MB, mred, 0.f, nullptr, nullptr);
     fence_proxy_async_smem();
     tc::fence_before_sync();
     __syncthreads();
@@ -249,8 +253,9 @@ k_bwd_rows_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restri
         token_sum(part, tokq + 2 * plane, 1.f, false);
     }
     // phase B: the adjoints into the same tiles (the phase-A products are complete)
-    const float sEH = mat_to_f16_tile(EH, sb + L::MA, mred, Hs, &eh, nullptr);
-    const float sEM = mat_to_f16_tile(EM, sb + L::MB, mred, Ms, &eh, nullptr);
+    // <E^H, H_s> + <E^M, M_s> against the fp16 copies of H_s, M_s that these overwrite
+    const float sEH = mat_to_f16_tile(EH, sb + L::MA, mred, sH, &eh, nullptr);
+    const float sEM = mat_to_f16_tile(EM, sb + L::MB, mred, sM, &eh, nullptr);
     fence_proxy_async_smem();
     tc::fence_before_sync();
     __syncthreads();
@@ -402,7 +407,7 @@ k_bwd_u_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict_
         Gr[e] = dout[g];
     }
     const float sG = rows_to_f16_tile(dout + tok0 * D, sb + L::RG, mred, false, nullptr);
-    const float sM = mat_to_f16_tile(Ms, sb + L::MB, mred, nullptr, nullptr, nullptr);
+    const float sM = mat_to_f16_tile(Ms, sb + L::MB, mred, 0.f, nullptr, nullptr);
     fence_proxy_async_smem();
     tc::fence_before_sync();
     __syncthreads();
