@@ -44,6 +44,11 @@ TRAFFIC = {
     "state_pass_tc": {"bytes": 67.759872e6 + 80.081664e6, "workload": "bf16_b8h8t2048d128",
                       "src": "test_ridge_regression_b200/csrc/state_tc.cuh",
                       "sha1": "3bd3bff3a2f8e7bf8df221195dc42f9281487e71"},
+    # backward row products captured at B2 H8 T2048 (1024 chunks), scaled x4 to the
+    # 4096 chunks of the full workload (per-chunk traffic does not depend on B)
+    "bwd_rows_tc": {"bytes": 4 * (397.614848e6 + 72.314624e6), "workload": "bf16_b8h8t2048d128",
+                    "src": "test_ridge_regression_b200/csrc/backward_tc.cuh",
+                    "sha1": "bae7a862a52575dedb40425feeb40e75c13d8c07"},
     # decode captured on 64 x 32 heads (state above L2), scaled x4 to 256 x 32 heads
     "decode_step": {"bytes": 4 * (270.059520e6 + 211.768320e6), "workload": "decode_bf16_b256h32d128",
                     "src": "test_ridge_regression_b200/csrc/decode.cuh",
@@ -564,7 +569,10 @@ def bench_backward(args, w, dev, qd, kd, vd, bd, flush, rank, world, barrier, pe
     per_kernel = {n: ms / steps for n, (ms, _) in kt.items()}
     fl = bwd_flops_per_head_token(w.D, BWD_CHUNK, w.r)
     head_tok = w.B * w.H * w.T
-    dom = max(per_kernel, key=per_kernel.get)
+    # roofline of the largest of the backward's own kernels (the forward recompute's
+    # kernels have theirs in the forward leg)
+    own = {n: t for n, t in per_kernel.items() if n.startswith("bwd_") or n == "adjoint_scan"}
+    dom = max(own or per_kernel, key=(own or per_kernel).get)
     peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
     total_fl = sum(fl[n] for n in per_kernel if n in fl) * head_tok
     tc_rows = w.dtype == torch.bfloat16 and w.D == 128 and BWD_CHUNK == 32 and w.T % 64 == 0
@@ -577,7 +585,8 @@ def bench_backward(args, w, dev, qd, kd, vd, bd, flush, rank, world, barrier, pe
         byts = per_tok * head_tok
         ach = byts / (per_kernel[dom] / 1e3) / 1e9
         roof = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": ach / peaks["hbm_gbs"], "traffic": None,
+                "unit": "GB/s", "frac": ach / peaks["hbm_gbs"],
+                "traffic": traffic_of("bwd_rows_tc", w.name),
                 "peak_source": "measured copy bandwidth", "algorithmic_per_step": byts}
     else:
         achieved = fl.get(dom, 0) * head_tok / (per_kernel[dom] / 1e3) / 1e12
