@@ -1,0 +1,78 @@
+"""Host logic of bench.py that needs no GPU: the source-hash gate on captured DRAM
+traffic, the peaks fallback, the clock summary and the algorithmic flop count the
+solve's roofline divides by."""
+import hashlib
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def test_traffic_is_reported_only_for_the_captured_source(tmp_path, monkeypatch):
+    src = tmp_path / "kern.cuh"
+    src.write_bytes(b"// kernel source at capture time\n")
+    entry = {"bytes": 123.0e6, "workload": "wl", "src": "kern.cuh",
+             "sha1": hashlib.sha1(src.read_bytes()).hexdigest()}
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setitem(bench.TRAFFIC, "kern", entry)
+    assert bench.traffic_of("kern", "wl") == 123.0e6
+    # another workload, or a kernel without a capture: no figure
+    assert bench.traffic_of("kern", "other") is None
+    assert bench.traffic_of("no_such_kernel", "wl") is None
+    # the source changed since the capture: no figure
+    src.write_bytes(b"// kernel source edited after the capture\n")
+    assert bench.traffic_of("kern", "wl") is None
+    # the source is gone: no figure
+    src.unlink()
+    assert bench.traffic_of("kern", "wl") is None
+
+
+def test_traffic_table_names_existing_sources():
+    for name, t in bench.TRAFFIC.items():
+        assert os.path.exists(os.path.join(ROOT, t["src"])), name
+        assert len(t["sha1"]) == 40 and t["bytes"] > 0, name
+
+
+def test_peaks_fall_back_without_measured_file(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    p = bench.load_peaks()
+    assert p["_source"] == "fallback"
+    assert p["hbm_gbs"] == bench.FALLBACK_PEAKS["hbm_gbs"]
+    (tmp_path / "MEASURED_PEAKS.json").write_text('{"hbm_gbs": 6000.0, "bf16_tflops": 1600.0}')
+    p = bench.load_peaks()
+    assert p["_source"] == "measured" and p["hbm_gbs"] == 6000.0
+
+
+def test_solve_flops_per_head_token():
+    # r rounds of three products per token at C = 64, D = 128 (K X^T: 2CD,
+    # H_s X^T: 2D^2, K^T P^T: 2CD): the r - 1 Chebyshev products plus the readout
+    D, C, r = 128, 64, 20
+    ch, out, upd, nrm = bench.flops_per_head_token(D, C, r)
+    assert ch + out == r * (2 * C * D + 2 * D * D + 2 * D * C) == 1_310_720
+    assert upd == 4 * D * D
+    assert nrm == 2 * D * D + 2 * C * D + 2 * C * C
+
+
+def test_clock_summary_flags_throttle_reasons():
+    s = bench.ClockSampler(0)
+    assert s.summary()["reasons"] == ["unsampled"]
+    s.max_mhz = 1965.0
+    s.samples = [(1965.0, 0), (1850.0, 0x4), (1900.0, 0)]
+    out = s.summary()
+    assert out["sm_mhz"] == 1900.0 and out["sm_max_mhz"] == 1965.0
+    assert out["reasons"] == ["sw_power_cap"] and out["samples"] == 3
+    s.samples.append((1200.0, 0x40 | 0x8))
+    assert s.summary()["reasons"] == ["hw_slowdown", "hw_thermal_slowdown", "sw_power_cap"]
+
+
+@pytest.mark.parametrize("D,C", [(128, 32), (64, 16)])
+def test_backward_flops_are_per_kernel(D, C):
+    fl = bench.bwd_flops_per_head_token(D, C, 20)
+    assert fl["bwd_rows"] == 7 * 2 * D * D
+    assert fl["bwd_delta"] == 3 * 2 * D * D
+    assert fl["bwd_solve"] == (2 * D * D + 4 * C * D) + fl["chunk_solve"]
