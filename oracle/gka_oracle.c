@@ -414,7 +414,7 @@ int gka_oracle_backward(const double *q, const double *k, const double *v,
         }
         /* reverse sweep over the adjoint states */
         for (int t = T - 1; t >= 0; --t) {
-            const double *Ht = S + (size_t)(t + 1) * 2 * DD, *Mt = Ht + DD;
+            const double *Ht = S + (size_t)(t + 1) * 2 * DD;
             const double *Hp = S + (size_t)t * 2 * DD, *Mp = Hp + DD;
             const double bnext = (t + 1 < T) ? bt[t + 1] : 0.0;
             const double *xt = X + (size_t)t * D, *yt = Y + (size_t)t * D;
