@@ -233,7 +233,12 @@ int gka_decode_step_gated(float *state, const void *q, const void *k, const void
  *   dL/dH_t = -y_t x_t^T - a (y_t . x_t) / ||H_t||_F H_t,   dL/dM_t = g_t x_t^T,
  * carried back through the decayed, write-gated recurrence to dk, dv, dbeta
  * and dgate.  It recomputes the forward quantities it needs (chunk states,
- * norms, iterates) itself; every step runs on CUDA cores in fp32.
+ * norms, iterates) itself.  With bf16 inputs, D = 128, chunk 32 and T a
+ * multiple of 64 the recompute, both Chebyshev solves, the chunk and adjoint
+ * increments, u = M_t^T g_t and the row products run on the tensor cores
+ * (fp16 operands with power-of-two scales, fp32 accumulation) and the scans
+ * and final gradients in fp32 on CUDA cores; otherwise every step runs on
+ * CUDA cores in fp32.
  *   q, k, v, beta, gate  the forward's inputs (gate nullable)
  *   dout        [B, H, T, D] in `dt`: dL/do
  *   dq, dk, dv  [B, H, T, D] in `dt` (written)
