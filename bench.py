@@ -35,7 +35,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one ncu capture per
 # kernel, with the SHA-1 of the kernel's source file at capture time: when the
 # source has changed since, the figure no longer describes the kernel and the
-# bench reports null.  Captures and commands: profiles/*.md.
+# bench reports null.  The captures' commands sit beside their summaries.
 TRAFFIC = {
     # full-size forward workload (B8 H8 T2048 D128, chunk 64), one launch
     "chunk_solve_tc": {"bytes": 237.182720e6 + 20.763136e6, "workload": "bf16_b8h8t2048d128",
@@ -82,6 +82,8 @@ def parse():
     p.add_argument("--no-backward", action="store_true", help="skip the backward leg")
     p.add_argument("--no-solver-study", action="store_true", help="skip the solver-study leg")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-configs", action="store_true",
+                   help="skip the legs of the other forward workloads")
     p.add_argument("--decode-steps", type=int, default=None)
     p.add_argument("--decode-batch", type=int, default=None,
                    help="fewer decode sequences (profiling runs); default: the workload's 256")
@@ -273,6 +275,120 @@ def run_reference(args, w, cfg, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# algorithmic flops per (head, token) of each forward kernel, from the four parts of
+# flops_per_head_token: the tensor-core solve also computes the per-token norm (fused)
+KERNEL_PARTS = {"chunk_solve_tc": ("ch", "out", "nrm"), "chunk_solve": ("ch", "out"),
+                "chunk_norm": ("nrm",), "chunk_delta": ("upd",), "state_pass_tc": ("upd",)}
+
+
+def kernel_flops_per_head_token(name, D, C, r):
+    ch, out, upd, nrm = flops_per_head_token(D, C, r)
+    parts = {"ch": ch, "out": out, "upd": upd, "nrm": nrm}
+    return sum(parts[x] for x in KERNEL_PARTS.get(name, ()))
+
+
+def alu_peak_tflops(peaks):
+    """fp32 FMA peak: 148 SMs x 128 lanes x 2 flop x max SM clock."""
+    return 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+
+
+def forward_roofline(w, kt, steps, ms_per_step, peaks):
+    """Roofline of the step's dominant kernel (largest summed device time) and the
+    whole step's fraction of the bf16 tensor peak."""
+    ch, out, upd, nrm = flops_per_head_token(w.D, w.chunk, w.r)
+    head_tok = w.B * w.H * w.T
+    dom_name, (dom_ms, dom_n) = max(kt.items(), key=lambda kv: kv[1][0])
+    per_step_ms = dom_ms / steps
+    kernel_flops = kernel_flops_per_head_token(dom_name, w.D, w.chunk, w.r) * head_tok
+    if dom_name == "chunk_solve_tc":
+        # fp16 operands, fp32 accumulation: the dense fp16 peak equals the bf16 one
+        bound, peak = "tensor", peaks["bf16_tflops"]
+        peak_note = f"dense bf16/fp16 tensor peak, {peaks['_source']} burst (cuBLAS bf16)"
+    else:
+        bound, peak = "alu", alu_peak_tflops(peaks)
+        peak_note = "fp32 FMA: 148 SMs x 128 lanes x 2 flop x max SM clock"
+    achieved = kernel_flops / (per_step_ms / 1e3) / 1e12
+    whole_flops = (ch + out + upd + nrm) * head_tok
+    tr = traffic_of(dom_name, w.name)
+    return {"bound": bound, "kernel": dom_name, "achieved": achieved, "peak": peak,
+            "unit": "TFLOP/s", "frac": achieved / peak,
+            "traffic": None if tr is None else tr * (dom_n / steps),
+            "peak_source": peak_note, "launches_per_step": dom_n / steps,
+            "algorithmic_per_step": kernel_flops,
+            "algorithmic_parts": "+".join(KERNEL_PARTS.get(dom_name, ())),
+            "step_frac_of_bf16_peak": whole_flops / (ms_per_step / 1e3) / 1e12
+            / peaks["bf16_tflops"]}
+
+
+def time_forward(step, steps, warmup, flush, dev, barrier):
+    """W warm-up steps, then K steps with L2 flushed before each, CUDA events per
+    step on the launch stream and the SM clock sampled meanwhile; then the same K
+    steps again under the library's launch profiler (per-kernel device times, kept
+    out of the step times).  Returns (per-step ms, kernel times, clock summary)."""
+    import torch
+    from test_ridge_regression_b200 import gka
+    for _ in range(max(warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if gka.device_status() != 0:
+        raise RuntimeError("device status error after warm-up")
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        for i in range(steps):
+            flush.fill_(float(i))
+            starts[i].record()
+            step()
+            ends[i].record()
+        torch.cuda.synchronize()
+    barrier()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    gka.profiler_read()
+    gka.profiler_enable(True)
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.fill_(float(i))
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    gka.profiler_enable(False)
+    kt = gka.profiler_read()
+    if gka.device_status() != 0:
+        raise RuntimeError("device status error after the timed steps")
+    return step_ms, kt, clk.summary()
+
+
+def bench_config(args, w, dev, peaks, flush):
+    """One other forward workload (N = 1): the same timing as the main line, its
+    own roofline and step fraction."""
+    import torch
+    from test_ridge_regression_b200 import gka
+    from test_ridge_regression_b200.inputs import workload_inputs
+    qd, kd, vd, bd = (t.to(dev) for t in workload_inputs(w))
+    od = torch.empty_like(vd)
+    ws = gka.alloc_workspace(w.B, w.H, w.T, w.D, w.chunk, w.dtype, dev)
+
+    def step():
+        gka.gka_forward(qd, kd, vd, bd, w.a, w.r, w.chunk, o=od, workspace=ws)
+
+    steps = max(1, min(args.steps, 20))
+    step_ms, kt, clk = time_forward(step, steps, args.warmup, flush, dev, lambda: None)
+    ms = sum(step_ms) / steps
+    out = {"workload": w.name, "B": w.B, "heads": w.H, "T": w.T, "D": w.D, "chunk": w.chunk,
+           "a": w.a, "r": w.r, "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32",
+           "beta": f"sigmoid(N({w.beta_mu},{w.beta_sigma}))", "steps": steps,
+           "ms_per_step": ms, "tokens_per_s": w.B * w.T / (ms / 1e3),
+           "kernels_ms_per_step": {n: t / steps for n, (t, _) in kt.items()},
+           "gpu_launches": sum(n for _, n in kt.values()),
+           "roofline": forward_roofline(w, kt, steps, ms, peaks), "clocks": clk}
+    del qd, kd, vd, bd, od, ws
+    torch.cuda.empty_cache()
+    return out
+
+
 def main():
     args = parse()
     from test_ridge_regression_b200 import dist as gdist
@@ -314,78 +430,13 @@ def main():
     def step():
         gka.gka_forward(qd, kd, vd, bd, w.a, w.r, w.chunk, o=od, workspace=ws)
 
-    for _ in range(max(args.warmup, 3)):
-        step()
-    torch.cuda.synchronize()
-    if gka.device_status() != 0:
-        raise RuntimeError("device status error after warm-up")
-
-    # ---- timed region: K steps, L2 flushed before each, events per step ----
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        for i in range(args.steps):
-            flush.fill_(float(i))
-            starts[i].record()
-            step()
-            ends[i].record()
-        torch.cuda.synchronize()
-    barrier()
-    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    # ---- per-kernel device times: the same K steps again with the library's launch
-    # profiler (CUDA events around every kernel on its stream), kept out of the step
-    # times above ----
-    gka.profiler_read()
-    gka.profiler_enable(True)
-    barrier()
-    torch.cuda.synchronize()
-    for i in range(args.steps):
-        flush.fill_(float(i))
-        step()
-    torch.cuda.synchronize()
-    barrier()
-    gka.profiler_enable(False)
-    kt = gka.profiler_read()
+    step_ms, kt, clocks = time_forward(step, args.steps, args.warmup, flush, dev, barrier)
     total_ms = gdist.max_over_ranks(sum(step_ms), dev)
     ms_per_step = total_ms / args.steps
     tok_step = w.B * w.T
     value = world * tok_step * args.steps / (total_ms / 1e3)
     launches = sum(n for _, n in kt.values())
-
-    # ---- roofline of the dominant kernel ----
-    ch, out, upd, nrm = flops_per_head_token(w.D, w.chunk, w.r)
-    head_tok = w.B * w.H * w.T
-    # the dominant kernel: largest summed device time among the step's kernels (it may
-    # be several launches per step, e.g. one per 64-token group of a 128-token chunk)
-    dom = max(kt.items(), key=lambda kv: kv[1][0])
-    dom_name, (dom_ms, dom_n) = dom
-    per_step_ms = dom_ms / args.steps
-    alg = {"chunk_solve": ch + out, "chunk_solve_tc": ch + out, "chunk_norm": nrm,
-           "chunk_delta": upd, "state_pass_tc": upd}.get(dom_name, 0)
-    kernel_flops = alg * head_tok            # per step
-    sm_mhz_max = peaks.get("sm_max_mhz", 1965.0)
-    if dom_name == "chunk_solve_tc":
-        # fp16 operands, fp32 accumulation: the dense fp16 peak equals the bf16 one
-        bound, peak, punit = "tensor", peaks["bf16_tflops"], "TFLOP/s"
-        peak_note = f"dense bf16/fp16 tensor peak, {peaks['_source']} burst (cuBLAS bf16)"
-    else:
-        # CUDA-core fp32 FMA: 148 SMs x 128 lanes x 2 flop x max SM clock
-        bound, punit = "alu", "TFLOP/s"
-        peak = 148 * 128 * 2 * sm_mhz_max * 1e6 / 1e12
-        peak_note = "fp32 FMA: 148 SMs x 128 lanes x 2 flop x max SM clock"
-    achieved = kernel_flops / (per_step_ms / 1e3) / 1e12
-    whole_flops = (ch + out + upd + nrm) * head_tok
-    tr = traffic_of(dom_name, w.name)
-    roofline = {"bound": bound, "kernel": dom_name, "achieved": achieved, "peak": peak,
-                "unit": punit, "frac": achieved / peak,
-                "traffic": None if tr is None else tr * (dom_n / args.steps),
-                "peak_source": peak_note,
-                "launches_per_step": dom_n / args.steps,
-                "algorithmic_per_step": kernel_flops,
-                "step_frac_of_bf16_peak": whole_flops / (ms_per_step / 1e3) / 1e12
-                / peaks["bf16_tflops"]}
+    roofline = forward_roofline(w, kt, args.steps, ms_per_step, peaks)
 
     result = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -393,7 +444,7 @@ def main():
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic", "config": cfg, "roofline": roofline, "gpu_launches": launches,
         "kernels_ms_per_step": {n: ms / args.steps for n, (ms, _) in kt.items()},
-        "clocks": clk.summary(),
+        "clocks": clocks,
     }
 
     # ---- end to end: the library's host-buffer forward (pinned host buffers; the
@@ -445,6 +496,12 @@ def main():
     # ---- decode step: HBM-bound, 256 x 32 heads, fp32 state ----
     if not args.no_decode and world == 1:
         result["decode"] = bench_decode(args, dev, peaks)
+
+    # ---- the other forward workloads (N = 1): every config, timed like the main line ----
+    if not args.no_configs and world == 1:
+        from test_ridge_regression_b200.inputs import WORKLOADS as _W
+        result["configs"] = {name: bench_config(args, cw, dev, peaks, flush)
+                             for name, cw in _W.items() if name != w.name}
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1) ----
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

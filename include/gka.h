@@ -182,9 +182,12 @@ int gka_forward_host(const void *q, const void *k, const void *v, const float *b
  *   - Problems whose gka_forward_workspace_bytes() exceeds
  *     GKA_STATIC_SCRATCH_BYTES are rejected with
  *     GKA_ERR_EXCEEDS_STATIC_SCRATCH before anything is launched.
- *   - The first call on a device looks up the array's device address and
- *     sets the kernels' shared-memory attributes for that device; make that
- *     first call before any stream capture.
+ *   - Every call looks up the array's device address in the calling
+ *     thread's current context (cudaGetSymbolAddress), so a context reset or
+ *     a second context on the same device gets its own copy of the array.
+ *     The first call on a device also sets the kernels' shared-memory
+ *     attributes for that device; make that first call before any stream
+ *     capture.
  *   - All calls share the one array, and it keeps the contents of the last
  *     call.  Nothing in it has to start at zero (every region is written
  *     before it is read), so no clearing is needed.  Calls whose execution

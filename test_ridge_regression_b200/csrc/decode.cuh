@@ -235,6 +235,7 @@ k_decode_rows(const __grid_constant__ DecodeMaps maps, const Tin *__restrict__ q
                                                ~static_cast<uintptr_t>(1023));
     __shared__ __align__(16) float xbuf[2][D];
     __shared__ __align__(16) float ks[D];
+    __shared__ float vs[D];   // g v_t, parked here through the products (frees a register)
     __shared__ float red[NW];
     __shared__ __align__(8) uint64_t bar[2];
 
@@ -255,7 +256,7 @@ k_decode_rows(const __grid_constant__ DecodeMaps maps, const Tin *__restrict__ q
     const float bt = beta[head];
     const float gt = gate ? gate[head] : 1.f;   // write gate: g k k^T and g v k^T
     ks[t] = load_f(k + (size_t)head * D + t);
-    const float vt = load_f(v + (size_t)head * D + t) * gt;
+    vs[t] = load_f(v + (size_t)head * D + t) * gt;
     const float qt = load_f(q + (size_t)head * D + t);
     bool ok = mbar_wait_bounded(&bar[0], 0, kDecodeWaitProbes);
     __syncthreads();   // ks complete
@@ -321,24 +322,28 @@ k_decode_rows(const __grid_constant__ DecodeMaps maps, const Tin *__restrict__ q
 
     // M row t: m = beta m + v_t k, o_t = m . x; the updated row goes back in place
     if (!mbar_wait_bounded(&bar[1], 0, kDecodeWaitProbes)) ok = false;
-    float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
-#pragma unroll
+    const float vt = vs[t];
+    const float bm = beta[head];   // reloaded (cached) rather than held through the products
+    // (h stays live through this loop for the store below: a partial unroll and two
+    // accumulators keep the loop's temporaries within the register budget, no spill)
+    float o0 = 0.f, o1 = 0.f;
+#pragma unroll 4
     for (int c = 0; c < D / 4; ++c) {
         float4 *p = reinterpret_cast<float4 *>(buf + dec_tile_off(t, c));
         float4 mv = *p;
         const float4 kv = *reinterpret_cast<const float4 *>(&ks[4 * c]);
         const float4 xv = *reinterpret_cast<const float4 *>(&xbuf[cur][4 * c]);
-        mv.x = fmaf(bt, mv.x, vt * kv.x);
-        mv.y = fmaf(bt, mv.y, vt * kv.y);
-        mv.z = fmaf(bt, mv.z, vt * kv.z);
-        mv.w = fmaf(bt, mv.w, vt * kv.w);
+        mv.x = fmaf(bm, mv.x, vt * kv.x);
+        mv.y = fmaf(bm, mv.y, vt * kv.y);
+        mv.z = fmaf(bm, mv.z, vt * kv.z);
+        mv.w = fmaf(bm, mv.w, vt * kv.w);
         o0 = fmaf(mv.x, xv.x, o0);
         o1 = fmaf(mv.y, xv.y, o1);
-        o2 = fmaf(mv.z, xv.z, o2);
-        o3 = fmaf(mv.w, xv.w, o3);
+        o0 = fmaf(mv.z, xv.z, o0);
+        o1 = fmaf(mv.w, xv.w, o1);
         *p = mv;
     }
-    store_f(o + (size_t)head * D + t, invd > 0.f ? (o0 + o1) + (o2 + o3) : 0.f);
+    store_f(o + (size_t)head * D + t, invd > 0.f ? o0 + o1 : 0.f);
     fence_proxy_async_smem();
     ok = __syncthreads_and(ok);
     if (t == 0 && ok) {

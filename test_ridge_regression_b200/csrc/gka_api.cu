@@ -726,28 +726,19 @@ static int decode_dispatch(float *state, const void *q, const void *k, const voi
 // device array: every GPU that loads this library holds it until the process
 // exits.  Host code must not use the symbol itself as an address (in host code
 // it names a host-side stand-in); it takes the device address from
-// cudaGetSymbolAddress once per device and passes that to the kernels.
+// cudaGetSymbolAddress on every call, in the caller's current context, and
+// passes that to the kernels.  (The address belongs to a context, not to a
+// device number, so a cached copy could outlive a cudaDeviceReset or belong to
+// another context of the same device.)
 // ---------------------------------------------------------------------------
 constexpr size_t kStaticScratchBytes = GKA_STATIC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
-constexpr int kMaxDevices = 256;
-static std::mutex g_scratch_mu;
-static void *g_scratch_addr[kMaxDevices];
-
 static int static_scratch_address(void **out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
     if (e != cudaSuccess) return cuda_fail(e);
-    if (dev < 0 || dev >= kMaxDevices) return GKA_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> g(g_scratch_mu);
-    if (!g_scratch_addr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_static_scratch);
-        if (e != cudaSuccess) return cuda_fail(e);
-        g_scratch_addr[dev] = p;
-    }
-    *out = g_scratch_addr[dev];
+    *out = p;
     return GKA_OK;
 }
 
@@ -867,6 +858,7 @@ static int host_plan(int B, int H, int T, int D, int chunk, gka_dtype dt, int sl
 }
 
 // Copy streams and events of one device, made once (non-blocking streams).
+constexpr int kMaxDevices = 256;
 struct HostPipe {
     cudaStream_t h2d = nullptr, d2h = nullptr;
     cudaEvent_t entry = nullptr, in_done[2] = {}, comp_done[2] = {}, out_done[2] = {};

@@ -61,6 +61,13 @@ def test_solve_flops_per_head_token():
     assert ch + out == r * (2 * C * D + 2 * D * D + 2 * D * C) == 1_310_720
     assert upd == 4 * D * D
     assert nrm == 2 * D * D + 2 * C * D + 2 * C * C
+    # the tensor-core solve also forms every token's norm (fused), so its own count
+    # is Chebyshev + readout + norm; the CUDA-core solve leaves the norm to its kernel
+    assert bench.kernel_flops_per_head_token("chunk_solve_tc", D, C, r) == 1_310_720 + 57_344
+    assert bench.kernel_flops_per_head_token("chunk_solve", D, C, r) == 1_310_720
+    assert bench.kernel_flops_per_head_token("chunk_norm", D, C, r) == nrm
+    assert bench.kernel_flops_per_head_token("state_pass_tc", D, C, r) == upd
+    assert bench.kernel_flops_per_head_token("state_scan", D, C, r) == 0
 
 
 def test_clock_summary_flags_throttle_reasons():
@@ -81,3 +88,20 @@ def test_backward_flops_are_per_kernel(D, C):
     assert fl["bwd_rows"] == 7 * 2 * D * D
     assert fl["bwd_delta"] == 3 * 2 * D * D
     assert fl["bwd_solve"] == (2 * D * D + 4 * C * D) + fl["chunk_solve"]
+
+
+def test_forward_roofline_counts_the_solve_with_its_norm():
+    from test_ridge_regression_b200.inputs import WORKLOADS
+    w = WORKLOADS["bf16_b8h8t2048d128"]
+    peaks = {"bf16_tflops": 1000.0, "sm_max_mhz": 1965.0, "_source": "test"}
+    # 20 steps, the solve 0.5 ms per step, the state pass 0.1 ms: the solve dominates
+    kt = {"chunk_solve_tc": (10.0, 20), "state_pass_tc": (2.0, 20)}
+    roof = bench.forward_roofline(w, kt, 20, 0.65, peaks)
+    head_tok = w.B * w.H * w.T
+    flops = (1_310_720 + 57_344) * head_tok
+    assert roof["kernel"] == "chunk_solve_tc" and roof["bound"] == "tensor"
+    assert roof["algorithmic_per_step"] == flops
+    assert abs(roof["achieved"] - flops / 0.5e-3 / 1e12) < 1e-6
+    assert abs(roof["frac"] - roof["achieved"] / 1000.0) < 1e-12
+    whole = 1_433_600 * head_tok
+    assert abs(roof["step_frac_of_bf16_peak"] - whole / 0.65e-3 / 1e12 / 1000.0) < 1e-12

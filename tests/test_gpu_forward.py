@@ -244,9 +244,35 @@ def test_full_b8h8t2048_sampled():
     _sampled("bf16_b8h8t2048d128", [(0, 0), (7, 7), (3, 5)], window=0)
 
 
+def _sampled_windows(name, heads, window, fractions=(0.25, 0.5, 0.75)):
+    """Outputs at several windows spread along the sequence (at the given fractions
+    of T and at its end), for a sample of heads, with the oracle's state recurrence
+    carried through every prefix in segments (init_state), and the final state."""
+    w = WORKLOADS[name]
+    q, k, v, beta = workload_inputs(w)
+    o, fs, _ = run_forward(q, k, v, beta, w.a, w.r, w.chunk)
+    o, fs = o.cpu(), fs.cpu()
+    pick = lambda x: torch.stack([x[b, h] for b, h in heads])[None]
+    qs, ks, vs, bs, os_, fss = (pick(x) for x in (q, k, v, beta, o, fs))
+    starts = sorted({int(f * w.T) // w.chunk * w.chunk for f in fractions} | {w.T - window})
+    state, pos, worst = None, 0, 0.0
+    for s0 in starts:
+        seg = slice(pos, s0 + window)
+        ref = oracle.forward(qs[:, :, seg], ks[:, :, seg], vs[:, :, seg], bs[:, :, seg], w.a, w.r,
+                             init_state=state, solve_from=s0 - pos, want_final_state=True,
+                             nthreads=len(heads))
+        err = head_rel_err(os_[:, :, s0:s0 + window], ref["o"][:, :, s0 - pos:])
+        print(f"{name}: window [{s0}, {s0 + window}) o rel err {err:.3e}")
+        worst = max(worst, err)
+        state, pos = ref["final_state"], s0 + window
+    assert pos == w.T
+    assert head_rel_err(fss, state) <= 1e-4
+    assert worst <= TOL[w.dtype]
+
+
 def test_full_b4h16t8192_sampled():
-    _sampled("bf16_b4h16t8192d128_a0.1", [(0, 0), (3, 15)], window=1024)
+    _sampled_windows("bf16_b4h16t8192d128_a0.1", [(0, 0), (1, 5), (2, 10), (3, 15)], window=512)
 
 
 def test_full_b1h8t131072_sampled():
-    _sampled("bf16_b1h8t131072d128", [(0, 3)], window=512)
+    _sampled_windows("bf16_b1h8t131072d128", [(0, 0), (0, 3), (0, 7)], window=512)

@@ -2,10 +2,12 @@
 device memory (a plugin inside a host application that owns all device
 allocations, or a latency-critical caller that cannot take cudaMalloc's
 implicit synchronisation).  Its scratch is the library's own static device
-array, so the test checks, through the C ABI, that two calls in a row (the
-second one finding the first one's leftovers in that array) give the same
-results as gka_forward with a caller workspace, and that a problem too large
-for the array is refused before anything runs.
+array, so the tests check, through the C ABI, that calls in a row (each one
+finding the previous call's leftovers in that array, at the same or at other
+offsets) give bit for bit the results of gka_forward with a caller workspace:
+both run the same deterministic kernels (no atomics, no reduction order that
+depends on the launch), so any difference is a scratch fault.  A problem too
+large for the array is refused before anything runs.
 
 This file is collected last on purpose (its name sorts last)."""
 import ctypes
@@ -29,6 +31,22 @@ def _call(lib, q, k, v, beta, o, a, r, chunk, fs):
                                           float(a), int(r), int(chunk), p(fs), stream)
 
 
+def _check_against_gka_forward(lib, B, H, T, D, dtype, chunk, r, a, seed):
+    q, k, v, beta = (x.cuda() for x in make_inputs(B, H, T, D, dtype, 3.0, 1.0, seed))
+    fs_ref = torch.empty(B, H, 2, D, D, device="cuda")
+    ref = gka.gka_forward(q, k, v, beta, a, r, chunk, final_state=fs_ref)
+    o = torch.full_like(ref, float("nan"))
+    fs = torch.full_like(fs_ref, float("nan"))
+    rc = _call(lib, q, k, v, beta, o, a, r, chunk, fs)
+    assert rc == 0, lib.gka_status_string(rc)
+    assert gka.device_status() == 0
+    # same kernels, same inputs: identical bits (a tolerance would hide a scratch fault)
+    assert torch.equal(o, ref), f"max |diff| {(o.float() - ref.float()).abs().max().item():.3e}"
+    assert torch.equal(fs, fs_ref)
+    # and both still agree with the layer within the bf16 / fp32 parity bar
+    assert head_rel_err(o, ref) <= TOL[dtype]
+
+
 @pytest.mark.parametrize("dtype,D,chunk,r", [(torch.bfloat16, 128, 64, 20),
                                              (torch.float32, 64, 32, 10)])
 def test_static_scratch_matches_gka_forward_twice(dtype, D, chunk, r):
@@ -36,20 +54,21 @@ def test_static_scratch_matches_gka_forward_twice(dtype, D, chunk, r):
     lib = gka.lib()
     B, H, T, a = 1, 4, 512, 0.5
     assert gka.workspace_bytes(B, H, T, D, chunk, dtype) <= 64 << 20
-    for call, seed in enumerate((21, 22)):
-        q, k, v, beta = (x.cuda() for x in make_inputs(B, H, T, D, dtype, 3.0, 1.0, seed))
-        fs_ref = torch.empty(B, H, 2, D, D, device="cuda")
-        ref = gka.gka_forward(q, k, v, beta, a, r, chunk, final_state=fs_ref)
-        o = torch.full_like(ref, float("nan"))
-        fs = torch.full_like(fs_ref, float("nan"))
-        rc = _call(lib, q, k, v, beta, o, a, r, chunk, fs)
-        assert rc == 0, lib.gka_status_string(rc)
-        assert gka.device_status() == 0
-        assert torch.isfinite(o.float()).all()
-        err = head_rel_err(o, ref)
-        print(f"call {call}: rel err vs gka_forward {err:.3e}")
-        assert err <= TOL[dtype]
-        assert head_rel_err(fs, fs_ref) <= TOL[dtype]
+    for seed in (21, 22):
+        _check_against_gka_forward(lib, B, H, T, D, dtype, chunk, r, a, seed)
+
+
+def test_static_scratch_one_pass_state_branch_after_other_shape():
+    """24 heads take the one-pass state kernel, which writes another subset of the
+    workspace than the chunk-parallel increments; the call before it has another
+    shape and chunk, so that its leftovers sit at other offsets of the array."""
+    build.build()
+    lib = gka.lib()
+    assert gka.workspace_bytes(1, 24, 512, 128, 64, torch.bfloat16) <= 64 << 20
+    assert gka.workspace_bytes(2, 4, 1024, 128, 128, torch.bfloat16) <= 64 << 20
+    _check_against_gka_forward(lib, 2, 4, 1024, 128, torch.bfloat16, 128, 20, 0.5, 31)
+    _check_against_gka_forward(lib, 1, 24, 512, 128, torch.bfloat16, 64, 20, 0.5, 32)
+    _check_against_gka_forward(lib, 1, 24, 512, 128, torch.bfloat16, 64, 20, 0.1, 33)
 
 
 def test_static_scratch_refuses_oversized_problem():
