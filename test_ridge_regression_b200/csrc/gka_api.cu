@@ -20,6 +20,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "delta_tc.cuh"
+#include "seg_tc.cuh"
 #include "solve_tc.cuh"
 #include "state_tc.cuh"
 #include "study_simt.cuh"
@@ -96,13 +97,18 @@ static bool supported_c(int C) { return C == 16 || C == 32 || C == 64 || C == 12
 
 // bf16 inputs, head dimension 128 and chunks of 64 or 128 tokens run the
 // tensor-core solve; everything else the CUDA-core one.
-// On the tensor-core path, the chunk states come from one sequential pass per
-// (head, matrix) when there are at least this many heads (B*H) to spread over
-// the SMs; with fewer, from the chunk-parallel increments plus an element-wise
-// scan, which keeps every SM busy.
-constexpr int kStatePassMinHeads = 24;
 static bool tensor_core_path(int D, int C, gka_dtype dt) {
     return dt == GKA_BF16 && D == 128 && (C == 64 || C == 128);
+}
+
+// On the tensor-core path the chunk states come from one sequential pass per
+// (head, matrix), one CTA each on an SM of its own.  With fewer than sms / 2
+// heads that leaves SMs idle, so every sequence is cut into S segments of whole
+// chunks (S <= N), as many as fill the SMs with 2 * B*H * S CTAs.
+static int state_segments(int BH, int N, int sms) {
+    int S = BH > 0 ? sms / (2 * BH) : 1;
+    if (S > N) S = N;
+    return S < 1 ? 1 : S;
 }
 
 // Chebyshev constants of one call (pith.science appendix, Lemma 3: omega_0 = 2,
@@ -271,55 +277,55 @@ static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
         return rc;
     cudaError_t e;
 
-    DeltaMaps dmaps;
-    dmaps.k = maps.k;
-    dmaps.v = maps.v;
-    if (int rc = rows128_map(&dmaps.out, states, (uint64_t)BH * (N + 1) * 2 * D,
-                             CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 32, 128))
-        return rc;
     if (solve_only) {
         // chunk states already in the workspace
-    } else if (BH >= kStatePassMinHeads) {
+    } else {
+        // One pass per (head, matrix) over the chunks; with few heads the sequences
+        // are cut into S segments (aggregates on the tensor cores, then a scan of
+        // the segment starts) so that S times more CTAs share the sequential pass.
         StateMaps smaps;
         smaps.k = maps.k;
         smaps.v = maps.v;
         if (int rc = rows128_map(&smaps.out, slp, (uint64_t)BH * N * 2 * D,
                                  CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 64, 128))
             return rc;
+        int dev = 0, sms = 148;
+        if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return cuda_fail(e);
+        const int S = state_segments(BH, N, sms);
+        // segment buffers in the fp32 state region (unused by this path otherwise):
+        // starts [BH][S][2][D][D], then decays [BH][S], increments and bounds [BH][S][2]
+        float *seg_start = states;
+        float *seg_dec = seg_start + (size_t)BH * S * 2 * D * D;
+        float *seg_inc = seg_dec + (size_t)BH * S;
+        float *seg_bound = seg_inc + (size_t)BH * S * 2;
+        if (S > 1) {
+            if ((e = set_smem(k_seg_delta_tc, SegSmem::bytes)) != cudaSuccess) return cuda_fail(e);
+            { ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
+            k_seg_delta_tc<<<dim3(S, BH), kSegThreads, SegSmem::bytes, s>>>(
+                smaps, beta, gate, seg_start, seg_dec, seg_inc, T, N, C, S, flag); }
+            if (int rc = check_launch()) return rc;
+            { ProfScope ps(GKA_KERNEL_STATE_SCAN, s);
+            k_seg_scan<<<dim3(2 * D * D / 1024, BH), 256, 0, s>>>(seg_start, seg_dec, seg_inc,
+                                                                 seg_bound, S); }
+            if (int rc = check_launch()) return rc;
+        }
         if (C == 64) {
             if ((e = set_smem(k_state_pass_tc<64>, StateSmem<64>::bytes)) != cudaSuccess)
                 return cuda_fail(e);
             ProfScope ps(GKA_KERNEL_STATE_PASS_TC, s);
-            k_state_pass_tc<64><<<dim3(2, BH), kStateThreads, StateSmem<64>::bytes, s>>>(
-                smaps, beta, gate, sexp, decay, tokdec, plane, final_state, T, N, flag);
+            k_state_pass_tc<64><<<dim3(2, BH * S), kStateThreads, StateSmem<64>::bytes, s>>>(
+                smaps, beta, gate, sexp, decay, tokdec, plane, final_state, T, N, S, seg_start,
+                seg_bound, flag);
         } else {
             if ((e = set_smem(k_state_pass_tc<128>, StateSmem<128>::bytes)) != cudaSuccess)
                 return cuda_fail(e);
             ProfScope ps(GKA_KERNEL_STATE_PASS_TC, s);
-            k_state_pass_tc<128><<<dim3(2, BH), kStateThreads, StateSmem<128>::bytes, s>>>(
-                smaps, beta, gate, sexp, decay, tokdec, plane, final_state, T, N, flag);
+            k_state_pass_tc<128><<<dim3(2, BH * S), kStateThreads, StateSmem<128>::bytes, s>>>(
+                smaps, beta, gate, sexp, decay, tokdec, plane, final_state, T, N, S, seg_start,
+                seg_bound, flag);
         }
-        if (int rc = check_launch()) return rc;
-    } else {
-        if (C == 64) {
-            if ((e = set_smem(k_chunk_delta_tc<64>, DeltaSmem<64>::bytes)) != cudaSuccess)
-                return cuda_fail(e);
-            ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
-            k_chunk_delta_tc<64><<<dim3(N, BH), kTcThreads, DeltaSmem<64>::bytes, s>>>(
-                dmaps, beta, gate, states, decay, bound_inc, tokdec, plane, T, N, flag);
-        } else {
-            if ((e = set_smem(k_chunk_delta_tc<128>, DeltaSmem<128>::bytes)) != cudaSuccess)
-                return cuda_fail(e);
-            ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
-            k_chunk_delta_tc<128><<<dim3(N, BH), kTcThreads, DeltaSmem<128>::bytes, s>>>(
-                dmaps, beta, gate, states, decay, bound_inc, tokdec, plane, T, N, flag);
-        }
-        if (int rc = check_launch()) return rc;
-
-        const int DD2 = 2 * D * D;
-        { ProfScope ps(GKA_KERNEL_STATE_SCAN, s);
-        k_state_scan<<<dim3((DD2 + 1023) / 1024, BH), 256, 0, s>>>(states, decay, final_state, slp,
-                                                                 bound_inc, sexp, N, DD2, false); }
         if (int rc = check_launch()) return rc;
     }
 

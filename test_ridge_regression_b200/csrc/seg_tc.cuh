@@ -1,0 +1,304 @@
+// Chunk states for few heads: the sequence of every head is cut into S
+// segments of whole chunks, so that S times more CTAs share the sequential
+// work of the one-pass state kernel.
+//
+// Method: "Gated KalmaNet" (arXiv 2511.21016), ai.info page, Methodology:
+// only the chunk-start states are carried across chunks, and the carry is
+// linear, S_{n+1} = b_n S_n + dS_n.  Over a segment of tokens [t0, t1) the
+// same carry composes to
+//   S(t1) = b_seg S(t0) + A_seg,   b_seg = prod_{t0 <= m < t1} beta_m,
+//   A_seg = sum_{t0 <= i < t1} w_i a_i k_i^T,  w_i = g_i prod_{i < m < t1} beta_m,
+// with a = k for H and a = v for M (g the write gate, NULL = 1): the segment's
+// aggregate is one product over all its tokens, A_seg = A^T diag(w) K, with no
+// sequential chain inside it.  Three steps:
+//   1. k_seg_delta_tc: A_seg of every segment (fp32), b_seg and the segment's
+//      norm-bound increment, one CTA per (segment, head) running through the
+//      segment's tokens in 64-token pieces on tcgen05, both matrices at once;
+//   2. k_seg_scan: the segment-start states S(t0) by the composed carry, in
+//      place of the aggregates (segments in order, element-wise), and the
+//      segment-start norm bounds;
+//   3. k_state_pass_tc from each segment's start state and bound, one CTA per
+//      (matrix, head, segment), writing every chunk's fp16 state copy exactly
+//      as the single pass over the whole sequence would.
+//
+// Step 1's operands: A = K or V as loaded (bf16 is exact) and the weighted
+// keys w_i k_i split into two bf16 parts (hi + lo, 16 mantissa bits), as in
+// the one-pass kernel; accumulation in fp32 (TMEM).  The weights come from
+// clamped log(beta) summed in double from the segment's end backwards, one
+// piece at a time.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "ptx.cuh"
+#include "state_tc.cuh"
+#include "tcgen05.cuh"
+
+namespace gka {
+
+constexpr int kSegThreads = 256;
+constexpr int kSegSub = 64;   // tokens per piece
+constexpr int kSegStages = 3; // pieces in flight (TMA)
+
+struct SegSmem {
+    static constexpr uint32_t TILE = kSegSub * 256;                // [64][128] bf16, 2 halves
+    static constexpr uint32_t KS = 0;                              // stages of keys
+    static constexpr uint32_t VS = KS + kSegStages * TILE;         // stages of values
+    static constexpr uint32_t PARTS = VS + kSegStages * TILE;      // 2 buffers x (hi, lo)
+    static constexpr uint32_t BETA = PARTS + 2 * 2 * TILE;         // [stages][64] floats
+    static constexpr uint32_t GATE = BETA + kSegStages * 4 * kSegSub;
+    static constexpr uint32_t W = GATE + kSegStages * 4 * kSegSub; // [2][64] weights
+    static constexpr uint32_t RED = W + 2 * 4 * kSegSub;           // [2][8] bound partials
+    static constexpr uint32_t BARS = RED + 64;                     // load[3] mma[2] fin
+    static constexpr uint32_t TBASE = BARS + 8 * 8;
+    static constexpr uint32_t END = TBASE + 16;
+    static constexpr size_t bytes = END + 1024;
+};
+
+// Chunks [n0, n1) of segment s of S over N chunks (every segment non-empty
+// when S <= N).
+__host__ __device__ __forceinline__ int seg_begin(int s, int S, int N) {
+    return (int)(((long long)s * N) / S);
+}
+
+// grid (S, B*H), block kSegThreads.  agg: fp32 [B*H][S][2][128][128] (H then M
+// of each segment); segdec: [B*H][S]; seginc: [B*H][S][2].
+__global__ void __launch_bounds__(kSegThreads, 1)
+k_seg_delta_tc(const __grid_constant__ StateMaps maps, const float *__restrict__ beta,
+               const float *__restrict__ gate, float *__restrict__ agg, float *__restrict__ segdec,
+               float *__restrict__ seginc, int T, int N, int C, int S,
+               int *__restrict__ timeout_flag) {
+    using L = SegSmem;
+    constexpr int D = 128;
+    constexpr uint32_t TILE = L::TILE;
+    extern __shared__ uint8_t smraw[];
+    uint8_t *sm = smem_align1024(smraw);
+    const uint32_t sb = smem_u32(sm);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BARS);
+    uint64_t *bar_load = bars, *bar_mma = bars + kSegStages, *bar_fin = bars + kSegStages + 2;
+    uint32_t *tbase = reinterpret_cast<uint32_t *>(sm + L::TBASE);
+    float *s_beta = reinterpret_cast<float *>(sm + L::BETA);
+    float *s_gate = reinterpret_cast<float *>(sm + L::GATE);
+    float *s_w = reinterpret_cast<float *>(sm + L::W);
+    float *s_red = reinterpret_cast<float *>(sm + L::RED);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int s = blockIdx.x, bh = blockIdx.y;
+    const int n0 = seg_begin(s, S, N), n1 = seg_begin(s + 1, S, N);
+    const int nsub = (n1 - n0) * C / kSegSub;   // pieces, processed from the last one back
+    const size_t tokbase = (size_t)bh * T + (size_t)n0 * C;
+
+    if (tid == 0) {
+        for (int i = 0; i < kSegStages + 3; ++i) mbar_init(&bars[i], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    int last_load[kSegStages];
+    for (int i = 0; i < kSegStages; ++i) last_load[i] = -1;
+    // piece c (counted from the segment's end) into stage c % kSegStages
+    auto issue_load = [&](int c) {
+        const int st = c % kSegStages;
+        uint64_t *bar = &bar_load[st];
+        mbar_arrive_expect_tx(bar, 2 * TILE + (gate ? 8u : 4u) * kSegSub);
+        const size_t t = tokbase + (size_t)(nsub - 1 - c) * kSegSub;
+        for (int h = 0; h < 2; ++h) {
+            tc::tma_load_2d(sm + L::KS + st * TILE + h * 8192, &maps.k, h * 64, (int)t, bar);
+            tc::tma_load_2d(sm + L::VS + st * TILE + h * 8192, &maps.v, h * 64, (int)t, bar);
+        }
+        bulk_g2s(s_beta + st * kSegSub, beta + t, 4 * kSegSub, bar);
+        if (gate) bulk_g2s(s_gate + st * kSegSub, gate + t, 4 * kSegSub, bar);
+        last_load[st] = c;
+    };
+    if (tid == 0)
+        for (int c = 0; c < kSegStages - 1 && c < nsub; ++c) issue_load(c);
+    if (warp == 0) {
+        tc::tmem_alloc(tbase, 256);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tbase;
+
+    double suf = 0.0;         // warp 0: summed log decay of the pieces after this one
+    float binc_h = 0.f, binc_m = 0.f;   // this thread's share of the bound increments
+    bool ok = true;
+#pragma unroll 1
+    for (int c = 0; c < nsub && ok; ++c) {
+        const int st = c % kSegStages;
+        if (!mbar_wait_bounded(&bar_load[st], (c / kSegStages) & 1, kStateWaitProbes)) ok = false;
+        if (warp == 0) {
+            // w_i = g_i exp(sum of the logs after token i in the segment); lane l
+            // holds tokens 2l, 2l + 1
+            const float *bt = s_beta + st * kSegSub;
+            const double l0 = fmax((double)logf(bt[2 * lane]), kLogBetaMin);
+            const double l1 = fmax((double)logf(bt[2 * lane + 1]), kLogBetaMin);
+            double after = 0.0;   // logs of the lanes above this one
+            double tot = l0 + l1;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const double y = __shfl_down_sync(0xffffffffu, tot, o);
+                if (lane + o < 32) tot += y;
+            }
+            after = __shfl_down_sync(0xffffffffu, tot, 1);
+            if (lane == 31) after = 0.0;
+            float w1 = decay_exp(suf + after), w0 = decay_exp(suf + after + l1);
+            if (gate) {
+                w0 *= s_gate[st * kSegSub + 2 * lane];
+                w1 *= s_gate[st * kSegSub + 2 * lane + 1];
+            }
+            s_w[(c & 1) * kSegSub + 2 * lane] = w0;
+            s_w[(c & 1) * kSegSub + 2 * lane + 1] = w1;
+            suf += __shfl_sync(0xffffffffu, tot, 0);
+        }
+        __syncthreads();
+        // the (w k) parts of piece c, in the swizzled layout of the key tile, and
+        // this thread's share of the bound increments
+        {
+            const uint8_t *kt = sm + L::KS + st * TILE;
+            const uint8_t *vt = sm + L::VS + st * TILE;
+            uint8_t *pb = sm + L::PARTS + (c & 1) * 2 * TILE;
+            const float *wc = s_w + (c & 1) * kSegSub;
+#pragma unroll
+            for (int j = 0; j < kSegSub * 16 / kSegThreads; ++j) {
+                const int item = tid + j * kSegThreads;   // 64 rows x 16 pieces of 16 bytes
+                const int r = item >> 4, l16 = item & 15;
+                const uint32_t off = (uint32_t)((l16 >> 3) * 8192 + r * 128 + (l16 & 7) * 16);
+                const uint4 u = *reinterpret_cast<const uint4 *>(kt + off);
+                const uint4 uv = *reinterpret_cast<const uint4 *>(vt + off);
+                const uint32_t uw[4] = {u.x, u.y, u.z, u.w}, vw[4] = {uv.x, uv.y, uv.z, uv.w};
+                const float w = wc[r];
+                float sq = 0.f, sv = 0.f;
+                uint32_t p0[4], p1[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float x0 = bf16_lo(uw[q]), x1 = bf16_hi(uw[q]);
+                    sq = fmaf(x0, x0, fmaf(x1, x1, sq));
+                    const float y0 = w * x0, y1 = w * x1;
+                    p0[q] = bf16x2_bits(y0, y1);
+                    p1[q] = bf16x2_bits(y0 - bf16_lo(p0[q]), y1 - bf16_hi(p0[q]));
+                    const float z0 = bf16_lo(vw[q]), z1 = bf16_hi(vw[q]);
+                    sv = fmaf(z0, z0, fmaf(z1, z1, sv));
+                }
+                *reinterpret_cast<uint4 *>(pb + off) = make_uint4(p0[0], p0[1], p0[2], p0[3]);
+                *reinterpret_cast<uint4 *>(pb + TILE + off) = make_uint4(p1[0], p1[1], p1[2], p1[3]);
+                binc_h = fmaf(w, sq, binc_h);
+                binc_m = fmaf(0.5f * w, sq + sv, binc_m);
+            }
+        }
+        fence_proxy_async_smem();
+        tc::fence_before_sync();
+        __syncthreads();
+        if (tid == 0 && ok) {
+            tc::fence_after_sync();
+            constexpr uint32_t ID = tc::idesc_bf16(128, 128, true, true);
+            const uint32_t ak = sb + L::KS + st * TILE, av = sb + L::VS + st * TILE;
+            const uint32_t ph = sb + L::PARTS + (c & 1) * 2 * TILE;
+#pragma unroll
+            for (int kk = 0; kk < kSegSub / 16; ++kk)
+#pragma unroll
+                for (int p = 0; p < 2; ++p) {
+                    const uint64_t bd = tc::sdesc(ph + p * TILE + kk * 2048, 8192, 1024);
+                    const bool acc = (c | kk | p) != 0;
+                    tc::mma_f16(tmem + 0, tc::sdesc(ak + kk * 2048, 8192, 1024), bd, ID, acc);
+                    tc::mma_f16(tmem + 128, tc::sdesc(av + kk * 2048, 8192, 1024), bd, ID, acc);
+                }
+            tc::commit(&bar_mma[c & 1]);
+            // the product of piece c - 1 is done: its stage takes piece c + 2, and
+            // (with the barrier at the top of the next round) its parts buffer is free
+            if (c >= 1 && !mbar_wait_bounded(&bar_mma[(c - 1) & 1], ((c - 1) >> 1) & 1,
+                                              kStateWaitProbes))
+                ok = false;
+            if (ok && c + kSegStages - 1 < nsub) issue_load(c + kSegStages - 1);
+        }
+        ok = __syncthreads_and(ok);
+    }
+    // the last product
+    if (tid == 0 && ok && nsub > 0 &&
+        !mbar_wait_bounded(&bar_mma[(nsub - 1) & 1], ((nsub - 1) >> 1) & 1, kStateWaitProbes))
+        ok = false;
+    binc_h = warp_sum(binc_h);
+    binc_m = warp_sum(binc_m);
+    if (lane == 0) {
+        s_red[warp] = binc_h;
+        s_red[8 + warp] = binc_m;
+    }
+    tc::fence_before_sync();
+    ok = __syncthreads_and(ok);
+    tc::fence_after_sync();
+    if (ok) {
+        if (tid == 0) {
+            float bh_ = 0.f, bm_ = 0.f;
+            for (int w = 0; w < kSegThreads / 32; ++w) {
+                bh_ += s_red[w];
+                bm_ += s_red[8 + w];
+            }
+            segdec[(size_t)bh * S + s] = decay_exp(suf);   // lane 0 of warp 0 holds suf
+            seginc[((size_t)bh * S + s) * 2] = bh_;
+            seginc[((size_t)bh * S + s) * 2 + 1] = bm_;
+        }
+        // rows of the two accumulators: warp w reads lane quarter w % 4, columns
+        // (w / 4) * 64 .. + 63 of H and of M
+        const int quarter = warp & 3, half = warp >> 2;
+        const int d = quarter * 32 + lane;
+        const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+        float *dst = agg + ((size_t)bh * S + s) * 2 * D * D + (size_t)d * D;
+#pragma unroll 1
+        for (int m = 0; m < 2; ++m)
+#pragma unroll
+            for (int cb = 0; cb < 64; cb += 16) {
+                float v[16];
+                tc::tmem_ld16(tl + m * 128 + half * 64 + cb, v);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    *reinterpret_cast<float4 *>(dst + (size_t)m * D * D + half * 64 + cb + 4 * j) =
+                        make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+            }
+    } else if (tid == 0) {
+        atomicExch(timeout_flag, 1);
+        tc::commit(bar_fin);   // drain whatever this thread issued
+        mbar_wait_bounded(bar_fin, 0, kStateWaitProbes);
+        for (int st = 0; st < kSegStages; ++st)
+            if (last_load[st] >= 0)
+                mbar_wait_bounded(&bar_load[st], (last_load[st] / kSegStages) & 1, kStateWaitProbes);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, 256);
+    }
+}
+
+// Step 2: segment-start states in place of the aggregates, element-wise over
+// the segments of a head in order: start_0 = 0, start_{s+1} = b_s start_s + A_s.
+// grid (2*D*D / (4 * 256), B*H), block 256 (four elements per thread).
+// Block (0, bh) also scans the two norm bounds into segbound [B*H][S][2].
+__global__ void __launch_bounds__(256)
+k_seg_scan(float *__restrict__ agg, const float *__restrict__ segdec,
+           const float *__restrict__ seginc, float *__restrict__ segbound, int S) {
+    constexpr int DD2 = 2 * 128 * 128;
+    const int bh = blockIdx.y;
+    const int e = (blockIdx.x * 256 + threadIdx.x) * 4;
+    float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
+    float *base = agg + (size_t)bh * S * DD2 + e;
+#pragma unroll 1
+    for (int s = 0; s < S; ++s) {
+        float4 *p = reinterpret_cast<float4 *>(base + (size_t)s * DD2);
+        const float4 a = *p;
+        *p = run;
+        const float b = segdec[(size_t)bh * S + s];
+        run = make_float4(fmaf(b, run.x, a.x), fmaf(b, run.y, a.y), fmaf(b, run.z, a.z),
+                          fmaf(b, run.w, a.w));
+    }
+    if (blockIdx.x == 0 && threadIdx.x < 2) {
+        float bd = 0.f;
+        for (int s = 0; s < S; ++s) {
+            segbound[((size_t)bh * S + s) * 2 + threadIdx.x] = bd;
+            bd = fmaf(segdec[(size_t)bh * S + s], bd, seginc[((size_t)bh * S + s) * 2 + threadIdx.x]);
+        }
+    }
+}
+
+}  // namespace gka

@@ -67,10 +67,10 @@ struct TcSmem {
     static constexpr uint32_t UPART = NRM2 + 8 * MG;         // [4 lane quarters][MG] partial u
     static constexpr uint32_t QPART = UPART + 16 * MG;       // [4 lane quarters][TOK] |q_j|^2
     static constexpr uint32_t DEC = QPART + 16 * TOK;        // l2, b, beta, beta^2: [4][MG] floats
-    // [2 rounds][TOK] -w c1 of the rounds: over UPART and QPART, set-up scratch
-    // that is dead once the rounds start
+    // [2 rounds][TOK] -w c1, then [2 rounds][TOK] -w / s_j of the rounds: over UPART
+    // and QPART, set-up scratch that is dead once the rounds start
     static constexpr uint32_t COEF = UPART;
-    static_assert(8 * TOK <= DEC - UPART, "coefficient tables overrun the set-up scratch");
+    static_assert(16 * TOK <= DEC - UPART, "coefficient tables overrun the set-up scratch");
     static constexpr uint32_t BARS = DEC + 16 * MG;
     static constexpr uint32_t TBASE = BARS + 8 * 8;
     static constexpr uint32_t END = TBASE + 16;
@@ -285,9 +285,11 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     uint8_t *sm = smem_align1024(smraw);
     const uint32_t sb = smem_u32(sm);
     float *s_c1 = reinterpret_cast<float *>(sm + L::SCAL);   // coefficient of Z1 (scaled domain)
-    float *s_c3 = s_c1 + TOK;                                // coefficient of Z3 (folded into W)
+    float *s_c3 = s_c1 + TOK;                                // c3_j s_j, folded into W
     float *s_o1 = s_c3 + TOK;                                // readout coefficient of Z1
-    float *s_coef = reinterpret_cast<float *>(sm + L::COEF);
+    float *s_t3 = s_o1 + TOK;                                // 1 / s_j, undoes s_j on Z3
+    float *s_coef = reinterpret_cast<float *>(sm + L::COEF);   // -w c1 per token
+    float *s_coef3 = s_coef + 2 * TOK;                         // -w / s_j per token
     float *red = reinterpret_cast<float *>(sm + L::RED);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BARS);
     uint64_t *bar_load = &bars[0], *bar_v = &bars[1], *bar_m = &bars[2], *bar_s = &bars[3],
@@ -529,17 +531,21 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     __syncthreads();
     if (tid < TOK) {
         const int j = tid;
-        float hs2 = 0.f;
+        float hs2s = 0.f;   // ||H_s||^2 of the scaled fp16 copy
 #pragma unroll
-        for (int w = 0; w < kSolveThreads / 32; ++w) hs2 += red[8 + w];
-        hs2 *= ldexpf(1.f, -2 * eHexp);
-        const float bj = s_bt[j];
-        const float n2 = fmaf(bj * bj, hs2,
-                              fmaf(2.f * bj, s_X[j] + s_X1[j], s_R[j]));
-        const float nj = sqrtf(fmaxf(n2, 0.f));
+        for (int w = 0; w < kSolveThreads / 32; ++w) hs2s += red[8 + w];
+        // in double: after long runs of strong decay without writes b_j^2 ||H_s||^2
+        // falls below the fp32 range while ||H_j|| itself (and, since the layer is
+        // invariant to scaling H and M together, the output) is still well defined
+        const double hs2 = (double)hs2s * ldexp(1.0, -2 * eHexp);
+        const float b = s_bt[j];
+        const double bj = b;
+        const double n2 = bj * bj * hs2 + 2.0 * bj * (double)(s_X[j] + s_X1[j]) + (double)s_R[j];
+        // a norm below 2^-120 (a state decayed that far since its last write) counts
+        // as a zero state, whose output is 0: 1 / ||H_j|| would leave the fp32 range
+        const float nj = n2 > 0x1p-240 ? (float)sqrt(n2) : 0.f;
         norms[tok0 + j] = nj;
         const float invd = nj > 0.f ? 1.f / (P.half_1p2a * nj) : 0.f;
-        const float b = s_bt[j];
         const float *qpart = reinterpret_cast<const float *>(sm + L::QPART);
         const float qn = sqrtf(qpart[j] + qpart[TOK + j] + qpart[2 * TOK + j] + qpart[3 * TOK + j]);
         const float eH = ldexpf(1.f, -eHexp);
@@ -548,33 +554,28 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         // two common to the CTA.  Every Chebyshev iterate obeys ||x|| <= ||q|| (1+2a) /
         // (a d), so ||x~|| <= sigma ||q|| (1+2a) / a for every token, and in the scaled
         // domain (q - A x) / d reads sigma q - c1 Z1 - c3 Z3 - cl x~: the coefficient of
-        // q is the same for all tokens.  c3 is folded into the decay weights below.
+        // q is the same for all tokens.  c3 is folded into the decay weights below,
+        // times a power of two s_j of the token's own (c3 s_j in [1/2, 1)), so that the
+        // weighted products c3 w S stay in fp16 range however far the tokens of one
+        // chunk differ in ||H_j||; Z3's column j then carries s_j, which the update
+        // and the readout take out again (exactly: 1 / s_j is a power of two).
         const float c3 = invd / (sK * sK);
+        const float s3 = inv_pow2_above(c3);
         s_c1[j] = b * invd * eH;
-        s_c3[j] = c3;
+        s_c3[j] = c3 * s3;
+        s_t3[j] = 1.f / s3;
         s_o1[j] = b * eM * invd;   // readout coefficient of Z1, times 1 / sigma below
-        float mq = qn, mc = c3;
+        float mq = qn;
 #pragma unroll
-        for (int o2 = 16; o2 > 0; o2 >>= 1) {
-            mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, o2));
-            mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, o2));
-        }
-        if (lane == 0) {
-            red[warp] = mq;
-            red[4 + warp] = mc;
-        }
+        for (int o2 = 16; o2 > 0; o2 >>= 1) mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, o2));
+        if (lane == 0) red[warp] = mq;
     }
     __syncthreads();
-    // sigma puts every ||x~|| below 2^12; sc3 (a power of two) scales the largest c3
-    // below 1 so that the weighted products c3 w S stay in fp16 range
-    float qmax = 0.f, c3max = 0.f;
+    // sigma puts every ||x~|| below 2^12
+    float qmax = 0.f;
 #pragma unroll
-    for (int w = 0; w < TOK / 32; ++w) {
-        qmax = fmaxf(qmax, red[w]);
-        c3max = fmaxf(c3max, red[4 + w]);
-    }
+    for (int w = 0; w < TOK / 32; ++w) qmax = fmaxf(qmax, red[w]);
     const float sigma = ldexpf(inv_pow2_above(qmax * (2.f * P.half_1p2a / P.a)), 12);
-    const float sc3 = inv_pow2_above(c3max);
     if (tid < TOK) s_o1[tid] *= 1.f / sigma;
 
     // q^T: this thread's tokens of row d, written into the (now free) tile as
@@ -587,8 +588,9 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     }
     const float cl = 2.f * P.a / (1.f + 2.f * P.a);   // lambda / d for every token with H != 0
 
-    // W^T rows: W[i][j] = sc3 c3_j w_{ji}, w_{ji} = exp(l_j - l_i) for i <= j, else 0
-    // (this thread's tokens); Z3 then carries c3 and its update coefficient is -w / sc3
+    // W^T rows: W[i][j] = s_j c3_j w_{ji}, w_{ji} = exp(l_j - l_i) for i <= j, else 0
+    // (this thread's tokens); Z3 then carries s_j c3_j and its update coefficient is
+    // -w / s_j
     {
         // w = w_{j,key} along this thread's tokens j (zero while j < key)
         const int js = tcol;
@@ -600,7 +602,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
             for (int u = 0; u < 16; ++u) {
                 const int j = js + c * 16 + u;
                 if (c * 16 + u > 0) w = (j == key && s_owner) ? 1.f : w * s_bet[j];
-                wv[u] = w * (s_c3[tcol + c * 16 + u] * sc3);   // c3_j w_ji, scaled by sc3
+                wv[u] = w * s_c3[tcol + c * 16 + u];   // s_j c3_j w_ji
             }
             tc::tmem_st16(tl + T_W + tcol + c * 16, wv);
         }
@@ -625,8 +627,11 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         }
         tc::tmem_wait_st();
     }
-    if (P.r > 1) {   // the first Chebyshev round's table: -w c1 per token
-        for (int e = tid; e < TOK; e += kSolveThreads) s_coef[TOK + e] = -P.omega[1] * s_c1[e];
+    if (P.r > 1) {   // the first Chebyshev round's tables: -w c1 and -w / s_j per token
+        for (int e = tid; e < TOK; e += kSolveThreads) {
+            s_coef[TOK + e] = -P.omega[1] * s_c1[e];
+            s_coef3[TOK + e] = -P.omega[1] * s_t3[e];
+        }
     }
     fence_proxy_async_smem();
     tc::fence_before_sync();
@@ -734,17 +739,17 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         }
         // x_new = (1 - w) x_prev + w (1 - lambda/d) x + w cq q - w c1 Z1 - w c3 Z3 (the
         // three-term update with the residual (q - A x)/d written out; the per-token
-        // product -w c1 of this round comes from the table; the q and Z3 coefficients
-        // w sigma and -w / sc3 are common to all tokens), in two parts:
+        // products -w c1 and -w / s_j of this round come from the tables; the q
+        // coefficient w sigma is common to all tokens), in two parts:
         // A, as soon as Z1 = H_s X^T is done (while the P phase and the intra-chunk
         // product run): part = (1 - w) x_prev + w (1 - lambda/d) x + w cq q - w c1 Z1,
         // kept in the x_prev columns of TMEM; B, once Z3 is done: x_new = part - w c3 Z3.
         // Pairs of tokens go through the packed f32x2 FMA pipe.
         const float cAs = 1.f - P.omega[it], cBs = P.omega[it] * (1.f - cl);
-        const float kqs = P.omega[it] * sigma, k3s = -P.omega[it] / sc3;
+        const float kqs = P.omega[it] * sigma;
         const float2 cA = make_float2(cAs, cAs), cB = make_float2(cBs, cBs);
-        const float2 kq = make_float2(kqs, kqs), k3 = make_float2(k3s, k3s);
-        const float *k1 = s_coef + (it & 1) * TOK;
+        const float2 kq = make_float2(kqs, kqs);
+        const float *k1 = s_coef + (it & 1) * TOK, *k3t = s_coef3 + (it & 1) * TOK;
         if (!mbar_wait_sleep(bar_z1, ph, kTcSleepProbes, kTcSleepNs)) ok = false;
         tc::fence_after_sync();
         if (!out_pass) {
@@ -800,12 +805,16 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
                 float z3[8], part[8];
                 tc::tmem_ld8(tl + T_Z3 + t0, z3);
                 tc::tmem_ld8(tl + T_XP + t0, part);
+                const float4 g3[2] = {*reinterpret_cast<const float4 *>(k3t + t0),
+                                      *reinterpret_cast<const float4 *>(k3t + t0 + 4)};
                 tc::tmem_wait_ld();
                 // x becomes the next round's x_prev (the part just read is dead), and the
                 // new iterate takes x's registers
                 tc::tmem_st8(tl + T_XP + t0, &xc[c * 8]);
 #pragma unroll
                 for (int p = 0; p < 4; ++p) {
+                    const float2 k3 = (p & 1) ? make_float2(g3[p >> 1].z, g3[p >> 1].w)
+                                              : make_float2(g3[p >> 1].x, g3[p >> 1].y);
                     const float2 t = __ffma2_rn(k3, make_float2(z3[2 * p], z3[2 * p + 1]),
                                                 make_float2(part[2 * p], part[2 * p + 1]));
                     xc[c * 8 + 2 * p] = t.x;
@@ -815,40 +824,45 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
             }
             // the next round's coefficient table (the other buffer)
             if (it + 1 < P.r) {
-                for (int e = tid; e < TOK; e += kSolveThreads)
+                for (int e = tid; e < TOK; e += kSolveThreads) {
                     s_coef[((it + 1) & 1) * TOK + e] = -w_next * s_c1[e];
+                    s_coef3[((it + 1) & 1) * TOK + e] = -w_next * s_t3[e];
+                }
             }
             fence_proxy_async_smem();
             tc::fence_before_sync();
             ok = __syncthreads_and(ok);
         } else if (ok) {
             // o_j[d] = b_j (M_s x_j)[d] + sum_i w_{ji} (k_i . x_j) v_i[d]; Z3 carries
-            // sc3 c3_j, so its readout coefficient sK / (sV sigma sc3) is common to all tokens
-            const float o3 = sK / (sV * sigma * sc3);
+            // s_j c3_j, so its readout coefficient is sK / (sV sigma) / s_j
+            const float o3 = sK / (sV * sigma);
             __nv_bfloat16 *orow = o + (tok0 + tcol) * kTcD + d;
 #pragma unroll
             for (int c = 0; c < NCH; ++c) {
                 const int t0 = tcol + c * 16;
-                float z1[16], z3[16], o1[16];
+                float z1[16], z3[16], o1[16], t3[16];
                 tc::tmem_ld16(tl + T_Z1 + t0, z1);
                 tc::tmem_ld16(tl + T_Z3 + t0, z3);
                 ld_f32x16(s_o1 + t0, o1);
+                ld_f32x16(s_t3 + t0, t3);
                 tc::tmem_wait_ld();
 #pragma unroll
                 for (int u = 0; u < 16; ++u)
                     orow[(size_t)(c * 16 + u) * kTcD] =
-                        __float2bfloat16_rn(fmaf(o1[u], z1[u], o3 * z3[u]));
+                        __float2bfloat16_rn(fmaf(o1[u], z1[u], (o3 * t3[u]) * z3[u]));
             }
         }
     }
 
     if (XOUT && ok) {
-        // x_j = x~_j invd_j / sigma, invd_j = c3_j sK^2 (thread (wg, d): element d of
-        // its tokens; consecutive d of a token are consecutive threads)
+        // x_j = x~_j invd_j / sigma, invd_j = c3_j sK^2 = (c3_j s_j) (1 / s_j) sK^2
+        // (thread (wg, d): element d of its tokens; consecutive d of a token are
+        // consecutive threads)
         const float xs = sK * sK / sigma;
         float *xrow = x_out + (tok0 + tcol) * kTcD + d;
 #pragma unroll
-        for (int u = 0; u < TPT; ++u) xrow[(size_t)u * kTcD] = xc[u] * (s_c3[tcol + u] * xs);
+        for (int u = 0; u < TPT; ++u)
+            xrow[(size_t)u * kTcD] = xc[u] * ((s_c3[tcol + u] * s_t3[tcol + u]) * xs);
     }
     // teardown: no MMA, copy or TMEM store of this CTA may be in flight when TMEM is freed
     tc::tmem_wait_st();

@@ -36,6 +36,11 @@
 //     for M (both linear in the elements, so no per-row reduction), which keeps
 //     every copied value <= 2^14.
 // The state after the last chunk goes to final_state (nullable).
+//
+// With S > 1 the sequence of every head is cut into S segments of whole chunks
+// (seg_tc.cuh): CTA (m, bh * S + s) runs segment s from its start state
+// seg_start[bh][s] and norm bound seg_bound[bh][s] (fp32, from the segment scan)
+// instead of from zero, and only the last segment writes final_state.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -100,13 +105,15 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
     return *reinterpret_cast<const uint32_t *>(&p);
 }
 
-// grid (2, B*H), block kStateThreads.  T = N * C.
+// grid (2, B*H*S), block kStateThreads.  T = N * C.  seg_start: fp32
+// [B*H][S][2][128][128], seg_bound: [B*H][S][2] (both unused when S == 1).
 template <int C>
 __global__ void __launch_bounds__(kStateThreads, 1)
 k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict__ beta,
                 const float *__restrict__ gate, int *__restrict__ state_exp, float *__restrict__ decay,
                 float *__restrict__ tokdec, size_t plane, float *__restrict__ final_state,
-                int T, int N, int *__restrict__ timeout_flag) {
+                int T, int N, int S, const float *__restrict__ seg_start,
+                const float *__restrict__ seg_bound, int *__restrict__ timeout_flag) {
     using L = StateSmem<C>;
     constexpr int D = 128, NP = L::NP, PER = C / 32;
     constexpr uint32_t TILE = L::TILE;
@@ -121,9 +128,12 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
     const bool arith = warp < 16;
     const int quarter = warp & 3, cg = (warp >> 2) & 3;   // lane quarter, 32-column group
     const int d = quarter * 32 + lane;          // state row of this thread = its TMEM lane
-    const int m = blockIdx.x, bh = blockIdx.y;  // m = 0: H, 1: M
+    const int m = blockIdx.x, bh = blockIdx.y / S, seg = blockIdx.y % S;  // m = 0: H, 1: M
     const bool is_m = m == 1;
-    const size_t tokbase = (size_t)bh * T;
+    // this CTA's chunks: n0 .. n0 + NL - 1 (the whole sequence when S == 1)
+    const int n0 = (int)(((long long)seg * N) / S);
+    const int NL = (int)(((long long)(seg + 1) * N) / S) - n0;
+    const size_t tokbase = (size_t)bh * T + (size_t)n0 * C;
     float *s_beta = reinterpret_cast<float *>(sm + L::BETA);   // [2][C]
     float *s_gate = reinterpret_cast<float *>(sm + L::GATE);   // [2][C], with a gate
     float *s_w = reinterpret_cast<float *>(sm + L::W);         // [2][C]
@@ -177,7 +187,7 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
     };
     if (tid == kStateEpiThreads) {
         issue_load(0);
-        if (N > 1) issue_load(1);
+        if (NL > 1) issue_load(1);
     }
     if (warp == 0) {
         tc::tmem_alloc(tbase, 256);
@@ -255,7 +265,7 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
             prev = l;
         }
         const double lend = __shfl_sync(0xffffffffu, t2, 31);
-        if (lane == 0) decay[(size_t)bh * N + c] = decay_exp(lend);
+        if (lane == 0) decay[(size_t)bh * N + n0 + c] = decay_exp(lend);
         __syncwarp();
     };
 
@@ -334,17 +344,28 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
     if (tid == kStateEpiThreads && ok) issue_mma(tmem, 0);
 
     float st[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) st[i] = 0.f;
     float bound = 0.f;
     const size_t DD = (size_t)D * D;
+    if (S > 1 && arith) {
+        // the segment's start state and norm bound (zero for the first segment)
+        const float *src = seg_start + (((size_t)bh * S + seg) * 2 + m) * DD + (size_t)d * D + cg * 32;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float4 x = *reinterpret_cast<const float4 *>(src + 4 * j);
+            st[4 * j] = x.x; st[4 * j + 1] = x.y; st[4 * j + 2] = x.z; st[4 * j + 3] = x.w;
+        }
+        bound = seg_bound[((size_t)bh * S + seg) * 2 + m];
+    } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) st[i] = 0.f;
+    }
 
     // Decay warp: chunk c's decays as soon as it has landed.  Stage c & 1 is
     // reloaded only after the product of chunk c - 2 is done, which comes after
     // every read of the w and b_n buffers this overwrites.
     if (decay_warp) {
 #pragma unroll 1
-        for (int c = 1; c < N && ok; ++c) {
+        for (int c = 1; c < NL && ok; ++c) {
             if (!mbar_wait_bounded(&bar_load[c & 1], (c >> 1) & 1, kStateWaitProbes)) ok = false;
             decays(c);
             if (!is_m) token_decays(c);
@@ -356,7 +377,7 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
     // barrier folds into `ok`.
     bool fail = false;
 #pragma unroll 1
-    for (int n = 0; n < N && ok && !decay_warp; ++n) {
+    for (int n = 0; n < NL && ok && !decay_warp; ++n) {
         const int ph = (n >> 1) & 1, ph1 = ((n + 1) >> 1) & 1;
         if (issuer_warp) {
             // stage n & 1 is free once dS_n is done and the previous TMA store has
@@ -365,17 +386,17 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
             if (lane == 0) {
                 if (!mbar_wait_bounded(&bar_mma[n & 1], ph, kStateWaitProbes)) fail = true;
                 tc::bulk_wait_read0();
-                if (n + 2 < N) issue_load(n + 2);
+                if (n + 2 < NL) issue_load(n + 2);
             }
             __syncwarp();
             ok = named_barrier_and(2, kStateBarThreads, ok && !fail);
             if (!ok) break;
             if (lane == 0) {
                 tc::fence_after_sync();
-                if (n + 1 < N) issue_mma(tmem, n + 1);
+                if (n + 1 < NL) issue_mma(tmem, n + 1);
                 if (!mbar_wait_bounded(bar_out, n & 1, kStateWaitProbes)) fail = true;
                 if (!fail) {
-                    const int row = (int)(((size_t)bh * N + n) * 2 + m) * D;
+                    const int row = (int)(((size_t)bh * N + n0 + n) * 2 + m) * D;
                     tc::tma_store_2d(&maps.out, 0, row, sm + out_stage(n));
                     tc::tma_store_2d(&maps.out, 64, row, sm + out_stage(n) + 16384);
                     tc::bulk_commit();
@@ -385,7 +406,7 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
             continue;
         }
         const float bn = b_next, bincn = bound_inc(n);   // chunk n's decay and bound increment
-        if (n + 1 < N) {
+        if (n + 1 < NL) {
             // chunk n + 1's operands (with double-buffered parts, formed while
             // chunk n's product still runs)
             if (!mbar_wait_bounded(&bar_w[(n + 1) & 1], ph1, kStateWaitProbes)) fail = true;
@@ -399,7 +420,7 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
         // dS_n is ready (and, with single-buffered parts, the parts are free)
         if (!mbar_wait_bounded(&bar_mma[n & 1], ph, kStateWaitProbes)) fail = true;
         tc::fence_after_sync();
-        if (!kDblParts && n + 1 < N) {
+        if (!kDblParts && n + 1 < NL) {
             prep(n + 1);
             fence_proxy_async_smem();
         }
@@ -423,7 +444,7 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
             }
             fence_proxy_async_smem();
             mbar_arrive(bar_out);
-            if (tid == 0) state_exp[((size_t)bh * N + n) * 2 + m] = ex;
+            if (tid == 0) state_exp[((size_t)bh * N + n0 + n) * 2 + m] = ex;
         }
         // S_{n+1} = b_n S_n + dS_n
         {
@@ -438,7 +459,7 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
     }
 
     ok = ok && !fail;
-    if (arith && ok && final_state) {
+    if (arith && ok && final_state && seg == S - 1) {
         float *dst = final_state + ((size_t)bh * 2 + m) * DD + (size_t)d * D + cg * 32;
 #pragma unroll
         for (int j = 0; j < 8; ++j)

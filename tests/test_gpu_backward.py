@@ -68,7 +68,7 @@ def test_backward_bf16_d128_cuda_core_recompute():
 
 
 def test_backward_bf16_state_pass_gate_resets():
-    # 24 heads: the tensor-core forward's one-pass state kernel; a write gate, resets
+    # 24 heads: the tensor-core forward's segmented states; a write gate, resets
     q, k, v, beta = make_inputs(1, 24, 128, 128, torch.bfloat16, 2.0, 1.0, seed=822)
     gate = make_gate((1, 24, 128), 822)
     gate[0, 3, 10:20] = 0.0

@@ -49,15 +49,15 @@ def test_host_forward_identical_to_device(dtype, D, C, slice_pairs):
 
 
 def test_host_forward_one_pass_slices_identical():
-    # 48 heads: the whole call and slices of 24 both take the one-pass state kernel
-    q, k, v, beta = make_inputs(2, 24, 192, 128, torch.bfloat16, 3.0, 1.0, seed=1201)
+    # 80 heads: the whole call and slices of 40 both take the one-pass state kernel
+    q, k, v, beta = make_inputs(2, 40, 192, 128, torch.bfloat16, 3.0, 1.0, seed=1201)
     o_ref, fs_ref = device_reference(q, k, v, beta, 0.5, 10, 64)
-    o, fs = host_run(q, k, v, beta, 0.5, 10, 64, 24)
+    o, fs = host_run(q, k, v, beta, 0.5, 10, 64, 40)
     assert torch.equal(o, o_ref) and torch.equal(fs, fs_ref)
 
 
 def test_host_forward_mixed_state_paths_and_pageable_memory():
-    # 48 heads in one device call (one pass) vs slices of 10 (two passes), pageable host memory
+    # 48 heads in one device call (one pass) vs slices of 10 (segmented), pageable host memory
     q, k, v, beta = make_inputs(2, 24, 192, 128, torch.bfloat16, 3.0, 1.0, seed=1202)
     o_ref, fs_ref = device_reference(q, k, v, beta, 0.5, 10, 64)
     o, fs = host_run(q, k, v, beta, 0.5, 10, 64, 10, pinned=False)
@@ -66,7 +66,7 @@ def test_host_forward_mixed_state_paths_and_pageable_memory():
 
 
 def test_host_forward_twice_with_one_workspace():
-    # 20 heads: the whole call and the slices of 8 both take the two-pass states
+    # 20 heads: the whole call and the slices of 8 both cut the two chunks into two segments
     q, k, v, beta = make_inputs(1, 20, 128, 128, torch.bfloat16, 2.0, 1.0, seed=1203)
     q, k, v, beta = (t.pin_memory() for t in (q, k, v, beta))
     ws = gka.alloc_host_workspace(1, 20, 128, 128, 64, torch.bfloat16, 8)
@@ -79,8 +79,8 @@ def test_host_forward_twice_with_one_workspace():
 
 
 def test_host_forward_default_schedule_64_pairs():
-    # the default schedule at 64 pairs is 24, 24, 16: two slices take the one-pass state
-    # kernel, the last the two-pass states, against one device call (one pass)
+    # the default schedule at 64 pairs is 24, 24, 16: every slice takes segmented states,
+    # against one device call (one pass)
     q, k, v, beta = make_inputs(8, 8, 128, 128, torch.bfloat16, 3.0, 1.0, seed=1204)
     o_ref, fs_ref = device_reference(q, k, v, beta, 0.5, 10, 64)
     o, fs = host_run(q, k, v, beta, 0.5, 10, 64, 0)

@@ -4,9 +4,10 @@ same gate: the paper's beta_t-augmented variant (ai.info page, Main Findings),
 H_t = beta_t H_{t-1} + g_t k_t k_t^T and M_t = beta_t M_{t-1} + g_t v_t k_t^T.
 
 Every kernel family is covered: the CUDA-core path (fp32, any D; bf16 with
-chunks 16/32), the tensor-core path with the chunk-parallel increments
-(fewer than 24 heads) and with the one-pass state kernel (24 heads or more),
-and both decode kernels.  Bars as for the ungated layer: 1e-4 (fp32 inputs),
+chunks 16/32), the tensor-core path with segmented chunk states (few heads:
+segment aggregates, a scan of the segment starts, one pass per segment) and
+with the one-pass state kernel over whole sequences (38 heads or more on 148
+SMs), and both decode kernels.  Bars as for the ungated layer: 1e-4 (fp32 inputs),
 2e-2 (bf16 inputs); a gate of ones reproduces the ungated kernels bit for bit.
 """
 import numpy as np
@@ -74,15 +75,15 @@ def test_gated_cuda_core_bf16(C):
 
 
 @pytest.mark.parametrize("C", [64, 128])
-def test_gated_tensor_core_chunk_increments(C):
-    # 4 heads (< 24): chunk-parallel increments + element-wise scan
+def test_gated_tensor_core_segmented_states(C):
+    # 4 heads, 4 chunks: the sequences cut into one-chunk segments
     check_gated(*gated_inputs(2, 2, 4 * C, 128, torch.bfloat16, 540 + C, 3.0), 0.5, 20, C)
 
 
 @pytest.mark.parametrize("C", [64, 128])
 def test_gated_tensor_core_state_pass(C):
-    # 24 heads: the one-pass state kernel
-    check_gated(*gated_inputs(1, 24, 2 * C, 128, torch.bfloat16, 560 + C, 3.0), 0.5, 20, C)
+    # 40 heads: the one-pass state kernel over whole sequences
+    check_gated(*gated_inputs(1, 40, 2 * C, 128, torch.bfloat16, 560 + C, 3.0), 0.5, 20, C)
 
 
 def test_gated_tensor_core_small_a_resets():
@@ -96,7 +97,7 @@ def test_gated_tensor_core_small_a_resets():
                                          (torch.bfloat16, 128, 32, 2),
                                          (torch.bfloat16, 128, 64, 2),
                                          (torch.bfloat16, 128, 128, 2),
-                                         (torch.bfloat16, 128, 64, 24)])
+                                         (torch.bfloat16, 128, 64, 40)])
 def test_unit_gate_and_null_gate_match_ungated_bit_for_bit(dtype, D, C, H):
     q, k, v, beta = make_inputs(1, H, 2 * C, D, dtype, 3.0, 1.0, seed=600 + C + H)
     qd, kd, vd, bd = cuda(q, k, v, beta)

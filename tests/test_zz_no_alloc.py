@@ -58,17 +58,19 @@ def test_static_scratch_matches_gka_forward_twice(dtype, D, chunk, r):
         _check_against_gka_forward(lib, B, H, T, D, dtype, chunk, r, a, seed)
 
 
-def test_static_scratch_one_pass_state_branch_after_other_shape():
-    """24 heads take the one-pass state kernel, which writes another subset of the
-    workspace than the chunk-parallel increments; the call before it has another
-    shape and chunk, so that its leftovers sit at other offsets of the array."""
+def test_static_scratch_both_state_paths_after_other_shapes():
+    """40 heads take the one-pass state kernel over whole sequences, 24 heads and
+    8 heads the segmented states, which also use the fp32 state region of the
+    workspace; each call follows one of another shape or chunk, so that the
+    leftovers sit at other offsets of the array."""
     build.build()
     lib = gka.lib()
-    assert gka.workspace_bytes(1, 24, 512, 128, 64, torch.bfloat16) <= 64 << 20
-    assert gka.workspace_bytes(2, 4, 1024, 128, 128, torch.bfloat16) <= 64 << 20
+    for shape in [(2, 4, 1024, 128, 128), (1, 40, 256, 128, 64), (1, 24, 512, 128, 64)]:
+        assert gka.workspace_bytes(*shape, torch.bfloat16) <= 64 << 20
     _check_against_gka_forward(lib, 2, 4, 1024, 128, torch.bfloat16, 128, 20, 0.5, 31)
-    _check_against_gka_forward(lib, 1, 24, 512, 128, torch.bfloat16, 64, 20, 0.5, 32)
+    _check_against_gka_forward(lib, 1, 40, 256, 128, torch.bfloat16, 64, 20, 0.5, 32)
     _check_against_gka_forward(lib, 1, 24, 512, 128, torch.bfloat16, 64, 20, 0.1, 33)
+    _check_against_gka_forward(lib, 1, 40, 256, 128, torch.bfloat16, 64, 20, 0.5, 34)
 
 
 def test_static_scratch_refuses_oversized_problem():
