@@ -294,21 +294,24 @@ static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
             (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
             return cuda_fail(e);
         const int S = state_segments(BH, N, sms);
+        // the aggregates (one CTA per SM each) may cut the sequences K times finer
+        const int K = S > 1 ? std::max(1, std::min(sms / (BH * S), N / S)) : 1;
+        const int S1 = K * S;
         // segment buffers in the fp32 state region (unused by this path otherwise):
-        // starts [BH][S][2][D][D], then decays [BH][S], increments and bounds [BH][S][2]
+        // starts [BH][S1][2][D][D], then decays [BH][S1], increments and bounds [BH][S1][2]
         float *seg_start = states;
-        float *seg_dec = seg_start + (size_t)BH * S * 2 * D * D;
-        float *seg_inc = seg_dec + (size_t)BH * S;
-        float *seg_bound = seg_inc + (size_t)BH * S * 2;
+        float *seg_dec = seg_start + (size_t)BH * S1 * 2 * D * D;
+        float *seg_inc = seg_dec + (size_t)BH * S1;
+        float *seg_bound = seg_inc + (size_t)BH * S1 * 2;
         if (S > 1) {
             if ((e = set_smem(k_seg_delta_tc, SegSmem::bytes)) != cudaSuccess) return cuda_fail(e);
             { ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
-            k_seg_delta_tc<<<dim3(S, BH), kSegThreads, SegSmem::bytes, s>>>(
-                smaps, beta, gate, seg_start, seg_dec, seg_inc, T, N, C, S, flag); }
+            k_seg_delta_tc<<<dim3(S1, BH), kSegThreads, SegSmem::bytes, s>>>(
+                smaps, beta, gate, seg_start, seg_dec, seg_inc, T, N, C, S1, flag); }
             if (int rc = check_launch()) return rc;
             { ProfScope ps(GKA_KERNEL_STATE_SCAN, s);
             k_seg_scan<<<dim3(2 * D * D / 1024, BH), 256, 0, s>>>(seg_start, seg_dec, seg_inc,
-                                                                 seg_bound, S); }
+                                                                 seg_bound, S1); }
             if (int rc = check_launch()) return rc;
         }
         if (C == 64) {
@@ -316,14 +319,14 @@ static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
                 return cuda_fail(e);
             ProfScope ps(GKA_KERNEL_STATE_PASS_TC, s);
             k_state_pass_tc<64><<<dim3(2, BH * S), kStateThreads, StateSmem<64>::bytes, s>>>(
-                smaps, beta, gate, sexp, decay, tokdec, plane, final_state, T, N, S, seg_start,
+                smaps, beta, gate, sexp, decay, tokdec, plane, final_state, T, N, S, K, seg_start,
                 seg_bound, flag);
         } else {
             if ((e = set_smem(k_state_pass_tc<128>, StateSmem<128>::bytes)) != cudaSuccess)
                 return cuda_fail(e);
             ProfScope ps(GKA_KERNEL_STATE_PASS_TC, s);
             k_state_pass_tc<128><<<dim3(2, BH * S), kStateThreads, StateSmem<128>::bytes, s>>>(
-                smaps, beta, gate, sexp, decay, tokdec, plane, final_state, T, N, S, seg_start,
+                smaps, beta, gate, sexp, decay, tokdec, plane, final_state, T, N, S, K, seg_start,
                 seg_bound, flag);
         }
         if (int rc = check_launch()) return rc;

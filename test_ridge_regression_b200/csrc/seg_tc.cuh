@@ -25,7 +25,9 @@
 // keys w_i k_i split into two bf16 parts (hi + lo, 16 mantissa bits), as in
 // the one-pass kernel; accumulation in fp32 (TMEM).  The weights come from
 // clamped log(beta) summed in double from the segment's end backwards, one
-// piece at a time.
+// piece at a time.  Step 1 may cut the sequences finer than step 3 (S1 = K S3
+// segments, so that it too fills the SMs); step 3 then starts its segment s
+// from step 2's start of segment K s.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -37,9 +39,11 @@
 
 namespace gka {
 
-constexpr int kSegThreads = 256;
-constexpr int kSegSub = 64;   // tokens per piece
-constexpr int kSegStages = 3; // pieces in flight (TMA)
+constexpr int kSegPrepWarps = 8;                          // warps forming the (w k) parts
+constexpr int kSegPrepThreads = 32 * kSegPrepWarps;
+constexpr int kSegThreads = kSegPrepThreads + 32;         // + the control warp
+constexpr int kSegSub = 64;    // tokens per piece
+constexpr int kSegStages = 4;  // stages of loaded pieces
 
 struct SegSmem {
     static constexpr uint32_t TILE = kSegSub * 256;                // [64][128] bf16, 2 halves
@@ -50,8 +54,8 @@ struct SegSmem {
     static constexpr uint32_t GATE = BETA + kSegStages * 4 * kSegSub;
     static constexpr uint32_t W = GATE + kSegStages * 4 * kSegSub; // [2][64] weights
     static constexpr uint32_t RED = W + 2 * 4 * kSegSub;           // [2][8] bound partials
-    static constexpr uint32_t BARS = RED + 64;                     // load[3] mma[2] fin
-    static constexpr uint32_t TBASE = BARS + 8 * 8;
+    static constexpr uint32_t BARS = RED + 64;    // load[stages] mma[2] wrdy[2] pdone[2] fin
+    static constexpr uint32_t TBASE = BARS + 8 * (kSegStages + 7);
     static constexpr uint32_t END = TBASE + 16;
     static constexpr size_t bytes = END + 1024;
 };
@@ -64,6 +68,12 @@ __host__ __device__ __forceinline__ int seg_begin(int s, int S, int N) {
 
 // grid (S, B*H), block kSegThreads.  agg: fp32 [B*H][S][2][128][128] (H then M
 // of each segment); segdec: [B*H][S]; seginc: [B*H][S][2].
+//
+// Warps 0-7 form the (w k) parts of each piece; warp 8 computes each piece's
+// weights as soon as the piece has landed, issues the TMA loads (kSegStages
+// pieces in flight) and the MMAs.  Per piece c (counted from the segment's end):
+//   load(c) -> weights(c) [warp 8] -> parts(c) [warps 0-7] -> MMA(c) [warp 8],
+// with parts(c) overlapping MMA(c - 1) and weights(c + 1) overlapping parts(c).
 __global__ void __launch_bounds__(kSegThreads, 1)
 k_seg_delta_tc(const __grid_constant__ StateMaps maps, const float *__restrict__ beta,
                const float *__restrict__ gate, float *__restrict__ agg, float *__restrict__ segdec,
@@ -76,26 +86,32 @@ k_seg_delta_tc(const __grid_constant__ StateMaps maps, const float *__restrict__
     uint8_t *sm = smem_align1024(smraw);
     const uint32_t sb = smem_u32(sm);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BARS);
-    uint64_t *bar_load = bars, *bar_mma = bars + kSegStages, *bar_fin = bars + kSegStages + 2;
+    uint64_t *bar_load = bars, *bar_mma = bars + kSegStages, *bar_wrdy = bar_mma + 2,
+             *bar_pdone = bar_wrdy + 2, *bar_fin = bar_pdone + 2;
     uint32_t *tbase = reinterpret_cast<uint32_t *>(sm + L::TBASE);
     float *s_beta = reinterpret_cast<float *>(sm + L::BETA);
     float *s_gate = reinterpret_cast<float *>(sm + L::GATE);
     float *s_w = reinterpret_cast<float *>(sm + L::W);
     float *s_red = reinterpret_cast<float *>(sm + L::RED);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const bool control = warp == kSegPrepWarps;
     const int s = blockIdx.x, bh = blockIdx.y;
     const int n0 = seg_begin(s, S, N), n1 = seg_begin(s + 1, S, N);
     const int nsub = (n1 - n0) * C / kSegSub;   // pieces, processed from the last one back
     const size_t tokbase = (size_t)bh * T + (size_t)n0 * C;
 
     if (tid == 0) {
-        for (int i = 0; i < kSegStages + 3; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < kSegStages; ++i) mbar_init(&bar_load[i], 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bar_mma[i], 1);
+            mbar_init(&bar_wrdy[i], 1);
+            mbar_init(&bar_pdone[i], kSegPrepWarps);
+        }
+        mbar_init(bar_fin, 1);
         fence_mbar_init();
     }
     __syncthreads();
-    int last_load[kSegStages];
-    for (int i = 0; i < kSegStages; ++i) last_load[i] = -1;
-    // piece c (counted from the segment's end) into stage c % kSegStages
+    // control lane 0: piece c (counted from the segment's end) into stage c % kSegStages
     auto issue_load = [&](int c) {
         const int st = c % kSegStages;
         uint64_t *bar = &bar_load[st];
@@ -107,10 +123,29 @@ k_seg_delta_tc(const __grid_constant__ StateMaps maps, const float *__restrict__
         }
         bulk_g2s(s_beta + st * kSegSub, beta + t, 4 * kSegSub, bar);
         if (gate) bulk_g2s(s_gate + st * kSegSub, gate + t, 4 * kSegSub, bar);
-        last_load[st] = c;
     };
-    if (tid == 0)
-        for (int c = 0; c < kSegStages - 1 && c < nsub; ++c) issue_load(c);
+    // control lane 0: dS += A^T (w k) of piece c into TMEM (H: columns 0-127, M: 128-255)
+    auto issue_mma = [&](uint32_t tmem, int c) {
+        constexpr uint32_t ID = tc::idesc_bf16(128, 128, true, true);
+        const int st = c % kSegStages;
+        const uint32_t ak = sb + L::KS + st * TILE, av = sb + L::VS + st * TILE;
+        const uint32_t ph = sb + L::PARTS + (c & 1) * 2 * TILE;
+#pragma unroll
+        for (int kk = 0; kk < kSegSub / 16; ++kk)
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                const uint64_t bd = tc::sdesc(ph + p * TILE + kk * 2048, 8192, 1024);
+                const bool acc = (c | kk | p) != 0;
+                tc::mma_f16(tmem + 0, tc::sdesc(ak + kk * 2048, 8192, 1024), bd, ID, acc);
+                tc::mma_f16(tmem + 128, tc::sdesc(av + kk * 2048, 8192, 1024), bd, ID, acc);
+            }
+        tc::commit(&bar_mma[c & 1]);
+    };
+    // pieces 0 and 1 now; piece c + 2 once the product of piece c - 2 has freed its
+    // stage (kSegStages = 4)
+    static_assert(kSegStages == 4, "load schedule");
+    if (control && lane == 0)
+        for (int c = 0; c < 2 && c < nsub; ++c) issue_load(c);
     if (warp == 0) {
         tc::tmem_alloc(tbase, 256);
         tc::tmem_relinquish();
@@ -120,27 +155,34 @@ k_seg_delta_tc(const __grid_constant__ StateMaps maps, const float *__restrict__
     tc::fence_after_sync();
     const uint32_t tmem = *tbase;
 
-    double suf = 0.0;         // warp 0: summed log decay of the pieces after this one
-    float binc_h = 0.f, binc_m = 0.f;   // this thread's share of the bound increments
     bool ok = true;
+    double suf = 0.0;   // control warp: summed log decay of the pieces after this one
+    float binc_h = 0.f, binc_m = 0.f;   // prep threads: shares of the bound increments
+    int last_load[kSegStages];   // control lane 0: piece last loaded into each stage
+    for (int i = 0; i < kSegStages; ++i) last_load[i] = i < nsub && i < 2 ? i : -1;
+    if (control) {
 #pragma unroll 1
-    for (int c = 0; c < nsub && ok; ++c) {
-        const int st = c % kSegStages;
-        if (!mbar_wait_bounded(&bar_load[st], (c / kSegStages) & 1, kStateWaitProbes)) ok = false;
-        if (warp == 0) {
-            // w_i = g_i exp(sum of the logs after token i in the segment); lane l
-            // holds tokens 2l, 2l + 1
+        for (int c = 0; c < nsub; ++c) {
+            const int st = c % kSegStages;
+            // (every wait's outcome is made warp-uniform, so the warp leaves together)
+            if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bar_load[st], (c / kSegStages) & 1,
+                                                           kStateWaitProbes))) {
+                ok = false;
+                break;
+            }
+            // weights(c) -> s_w[c & 1]: w_i = g_i exp(sum of the logs after token i in
+            // the segment); lane l holds tokens 2l, 2l + 1.  The buffer's last reader,
+            // parts(c - 2), finished before MMA(c - 2) was issued.
             const float *bt = s_beta + st * kSegSub;
             const double l0 = fmax((double)logf(bt[2 * lane]), kLogBetaMin);
             const double l1 = fmax((double)logf(bt[2 * lane + 1]), kLogBetaMin);
-            double after = 0.0;   // logs of the lanes above this one
-            double tot = l0 + l1;
+            double tot = l0 + l1;   // -> sum over the tokens of this lane and the lanes above
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const double y = __shfl_down_sync(0xffffffffu, tot, o);
                 if (lane + o < 32) tot += y;
             }
-            after = __shfl_down_sync(0xffffffffu, tot, 1);
+            double after = __shfl_down_sync(0xffffffffu, tot, 1);   // the lanes above
             if (lane == 31) after = 0.0;
             float w1 = decay_exp(suf + after), w0 = decay_exp(suf + after + l1);
             if (gate) {
@@ -150,18 +192,67 @@ k_seg_delta_tc(const __grid_constant__ StateMaps maps, const float *__restrict__
             s_w[(c & 1) * kSegSub + 2 * lane] = w0;
             s_w[(c & 1) * kSegSub + 2 * lane + 1] = w1;
             suf += __shfl_sync(0xffffffffu, tot, 0);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar_wrdy[c & 1]);
+            // MMA(c - 1) once its parts are formed
+            if (c >= 1) {
+                if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bar_pdone[(c - 1) & 1],
+                                                               ((c - 1) >> 1) & 1, kStateWaitProbes))) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) {
+                    tc::fence_after_sync();
+                    issue_mma(tmem, c - 1);
+                }
+            }
+            // MMA(c - 2) done: its stage takes piece c + 2
+            if (c >= 2 && !__all_sync(0xffffffffu, mbar_wait_bounded(&bar_mma[c & 1], ((c - 2) >> 1) & 1,
+                                                                     kStateWaitProbes))) {
+                ok = false;
+                break;
+            }
+            if (lane == 0 && c + 2 < nsub) {
+                issue_load(c + 2);
+                last_load[(c + 2) % kSegStages] = c + 2;
+            }
+            __syncwarp();
         }
-        __syncthreads();
-        // the (w k) parts of piece c, in the swizzled layout of the key tile, and
-        // this thread's share of the bound increments
-        {
+        // the last piece's product, then every product is done
+        if (ok && nsub > 0) {
+            if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bar_pdone[(nsub - 1) & 1],
+                                                           ((nsub - 1) >> 1) & 1, kStateWaitProbes)))
+                ok = false;
+            if (ok && lane == 0) {
+                tc::fence_after_sync();
+                issue_mma(tmem, nsub - 1);
+            }
+            __syncwarp();
+            if (ok && !__all_sync(0xffffffffu, mbar_wait_bounded(&bar_mma[(nsub - 1) & 1],
+                                                                 ((nsub - 1) >> 1) & 1, kStateWaitProbes)))
+                ok = false;
+        }
+    } else {
+        // parts(c): the (w k) parts of piece c in the swizzled layout of the key tile,
+        // and this thread's share of the bound increments
+#pragma unroll 1
+        for (int c = 0; c < nsub; ++c) {
+            const int st = c % kSegStages;
+            const bool got =
+                mbar_wait_bounded(&bar_load[st], (c / kSegStages) & 1, kStateWaitProbes) &&
+                mbar_wait_bounded(&bar_wrdy[c & 1], (c >> 1) & 1, kStateWaitProbes) &&
+                (c < 2 || mbar_wait_bounded(&bar_mma[c & 1], ((c - 2) >> 1) & 1, kStateWaitProbes));
+            if (!__all_sync(0xffffffffu, got)) {   // warp-uniform: the warp leaves together
+                ok = false;
+                break;
+            }
             const uint8_t *kt = sm + L::KS + st * TILE;
             const uint8_t *vt = sm + L::VS + st * TILE;
             uint8_t *pb = sm + L::PARTS + (c & 1) * 2 * TILE;
             const float *wc = s_w + (c & 1) * kSegSub;
 #pragma unroll
-            for (int j = 0; j < kSegSub * 16 / kSegThreads; ++j) {
-                const int item = tid + j * kSegThreads;   // 64 rows x 16 pieces of 16 bytes
+            for (int j = 0; j < kSegSub * 16 / kSegPrepThreads; ++j) {
+                const int item = tid + j * kSegPrepThreads;   // 64 rows x 16 pieces of 16 bytes
                 const int r = item >> 4, l16 = item & 15;
                 const uint32_t off = (uint32_t)((l16 >> 3) * 8192 + r * 128 + (l16 & 7) * 16);
                 const uint4 u = *reinterpret_cast<const uint4 *>(kt + off);
@@ -185,79 +276,56 @@ k_seg_delta_tc(const __grid_constant__ StateMaps maps, const float *__restrict__
                 binc_h = fmaf(w, sq, binc_h);
                 binc_m = fmaf(0.5f * w, sq + sv, binc_m);
             }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar_pdone[c & 1]);
         }
-        fence_proxy_async_smem();
-        tc::fence_before_sync();
-        __syncthreads();
-        if (tid == 0 && ok) {
-            tc::fence_after_sync();
-            constexpr uint32_t ID = tc::idesc_bf16(128, 128, true, true);
-            const uint32_t ak = sb + L::KS + st * TILE, av = sb + L::VS + st * TILE;
-            const uint32_t ph = sb + L::PARTS + (c & 1) * 2 * TILE;
-#pragma unroll
-            for (int kk = 0; kk < kSegSub / 16; ++kk)
-#pragma unroll
-                for (int p = 0; p < 2; ++p) {
-                    const uint64_t bd = tc::sdesc(ph + p * TILE + kk * 2048, 8192, 1024);
-                    const bool acc = (c | kk | p) != 0;
-                    tc::mma_f16(tmem + 0, tc::sdesc(ak + kk * 2048, 8192, 1024), bd, ID, acc);
-                    tc::mma_f16(tmem + 128, tc::sdesc(av + kk * 2048, 8192, 1024), bd, ID, acc);
-                }
-            tc::commit(&bar_mma[c & 1]);
-            // the product of piece c - 1 is done: its stage takes piece c + 2, and
-            // (with the barrier at the top of the next round) its parts buffer is free
-            if (c >= 1 && !mbar_wait_bounded(&bar_mma[(c - 1) & 1], ((c - 1) >> 1) & 1,
-                                              kStateWaitProbes))
-                ok = false;
-            if (ok && c + kSegStages - 1 < nsub) issue_load(c + kSegStages - 1);
+        binc_h = warp_sum(binc_h);
+        binc_m = warp_sum(binc_m);
+        if (lane == 0) {
+            s_red[warp] = binc_h;
+            s_red[8 + warp] = binc_m;
         }
-        ok = __syncthreads_and(ok);
-    }
-    // the last product
-    if (tid == 0 && ok && nsub > 0 &&
-        !mbar_wait_bounded(&bar_mma[(nsub - 1) & 1], ((nsub - 1) >> 1) & 1, kStateWaitProbes))
-        ok = false;
-    binc_h = warp_sum(binc_h);
-    binc_m = warp_sum(binc_m);
-    if (lane == 0) {
-        s_red[warp] = binc_h;
-        s_red[8 + warp] = binc_m;
     }
     tc::fence_before_sync();
     ok = __syncthreads_and(ok);
     tc::fence_after_sync();
     if (ok) {
-        if (tid == 0) {
-            float bh_ = 0.f, bm_ = 0.f;
-            for (int w = 0; w < kSegThreads / 32; ++w) {
-                bh_ += s_red[w];
-                bm_ += s_red[8 + w];
+        if (control) {
+            if (lane == 0) {
+                float bh_ = 0.f, bm_ = 0.f;
+                for (int w = 0; w < kSegPrepWarps; ++w) {
+                    bh_ += s_red[w];
+                    bm_ += s_red[8 + w];
+                }
+                segdec[(size_t)bh * S + s] = decay_exp(suf);
+                seginc[((size_t)bh * S + s) * 2] = bh_;
+                seginc[((size_t)bh * S + s) * 2 + 1] = bm_;
             }
-            segdec[(size_t)bh * S + s] = decay_exp(suf);   // lane 0 of warp 0 holds suf
-            seginc[((size_t)bh * S + s) * 2] = bh_;
-            seginc[((size_t)bh * S + s) * 2 + 1] = bm_;
-        }
-        // rows of the two accumulators: warp w reads lane quarter w % 4, columns
-        // (w / 4) * 64 .. + 63 of H and of M
-        const int quarter = warp & 3, half = warp >> 2;
-        const int d = quarter * 32 + lane;
-        const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
-        float *dst = agg + ((size_t)bh * S + s) * 2 * D * D + (size_t)d * D;
+        } else {
+            // rows of the two accumulators: warp w reads lane quarter w % 4, columns
+            // (w / 4) * 64 .. + 63 of H and of M
+            const int quarter = warp & 3, half = warp >> 2;
+            const int d = quarter * 32 + lane;
+            const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+            float *dst = agg + ((size_t)bh * S + s) * 2 * D * D + (size_t)d * D;
 #pragma unroll 1
-        for (int m = 0; m < 2; ++m)
+            for (int m = 0; m < 2; ++m)
 #pragma unroll
-            for (int cb = 0; cb < 64; cb += 16) {
-                float v[16];
-                tc::tmem_ld16(tl + m * 128 + half * 64 + cb, v);
-                tc::tmem_wait_ld();
+                for (int cb = 0; cb < 64; cb += 16) {
+                    float v[16];
+                    tc::tmem_ld16(tl + m * 128 + half * 64 + cb, v);
+                    tc::tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    *reinterpret_cast<float4 *>(dst + (size_t)m * D * D + half * 64 + cb + 4 * j) =
-                        make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-            }
-    } else if (tid == 0) {
+                    for (int j = 0; j < 4; ++j)
+                        *reinterpret_cast<float4 *>(dst + (size_t)m * D * D + half * 64 + cb + 4 * j) =
+                            make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                }
+        }
+    } else if (control && lane == 0) {
+        // a wait gave up: flag it, then drain the products and copies this lane issued
         atomicExch(timeout_flag, 1);
-        tc::commit(bar_fin);   // drain whatever this thread issued
+        tc::commit(bar_fin);
         mbar_wait_bounded(bar_fin, 0, kStateWaitProbes);
         for (int st = 0; st < kSegStages; ++st)
             if (last_load[st] >= 0)

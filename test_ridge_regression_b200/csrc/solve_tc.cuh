@@ -36,6 +36,8 @@
 
 #include <cuda_fp16.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "ptx.cuh"
 #include "tcgen05.cuh"
@@ -105,9 +107,14 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
     return *reinterpret_cast<const uint32_t *>(&p);
 }
 
-// 2^-(floor(log2 x) + 1) for x > 0 (so that x * result < 1), else 1.
+// 2^-(floor(log2 x) + 1) for x > 0 (so that x * result < 1), else 1; built from
+// x's exponent field (x below the normal range counts as 2^-127, and the result is
+// at least 2^-126).
 __device__ __forceinline__ float inv_pow2_above(float x) {
-    return x > 0.f ? ldexpf(1.f, -(ilogbf(x) + 1)) : 1.f;
+    if (!(x > 0.f)) return 1.f;
+    const int eb = (__float_as_int(x) >> 23) & 0xff;   // biased exponent of x
+    const int rb = 253 - eb;                           // biased exponent of 2^(126 - eb)
+    return __int_as_float((rb < 1 ? 1 : rb) << 23);
 }
 
 // 16 consecutive fp32 values from shared memory (16-byte aligned), as 4 vector loads.
@@ -285,9 +292,10 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     uint8_t *sm = smem_align1024(smraw);
     const uint32_t sb = smem_u32(sm);
     float *s_c1 = reinterpret_cast<float *>(sm + L::SCAL);   // coefficient of Z1 (scaled domain)
-    float *s_c3 = s_c1 + TOK;                                // c3_j s_j, folded into W
+    float *s_c3 = s_c1 + TOK;                                // c3_j
     float *s_o1 = s_c3 + TOK;                                // readout coefficient of Z1
     float *s_t3 = s_o1 + TOK;                                // 1 / s_j, undoes s_j on Z3
+    float *s_mn = s_t3 + TOK;                                // per-warp minima of c3 (set-up)
     float *s_coef = reinterpret_cast<float *>(sm + L::COEF);   // -w c1 per token
     float *s_coef3 = s_coef + 2 * TOK;                         // -w / s_j per token
     float *red = reinterpret_cast<float *>(sm + L::RED);
@@ -555,28 +563,51 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         // (a d), so ||x~|| <= sigma ||q|| (1+2a) / a for every token, and in the scaled
         // domain (q - A x) / d reads sigma q - c1 Z1 - c3 Z3 - cl x~: the coefficient of
         // q is the same for all tokens.  c3 is folded into the decay weights below,
-        // times a power of two s_j of the token's own (c3 s_j in [1/2, 1)), so that the
-        // weighted products c3 w S stay in fp16 range however far the tokens of one
-        // chunk differ in ||H_j||; Z3's column j then carries s_j, which the update
-        // and the readout take out again (exactly: 1 / s_j is a power of two).
+        // times a power of two s_j (s3_of below).
         const float c3 = invd / (sK * sK);
-        const float s3 = inv_pow2_above(c3);
         s_c1[j] = b * invd * eH;
-        s_c3[j] = c3 * s3;
-        s_t3[j] = 1.f / s3;
+        s_c3[j] = c3;
         s_o1[j] = b * eM * invd;   // readout coefficient of Z1, times 1 / sigma below
-        float mq = qn;
+        float mq = qn, mc = c3, mn = c3 > 0.f ? c3 : INFINITY;
 #pragma unroll
-        for (int o2 = 16; o2 > 0; o2 >>= 1) mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, o2));
-        if (lane == 0) red[warp] = mq;
+        for (int o2 = 16; o2 > 0; o2 >>= 1) {
+            mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, o2));
+            mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, o2));
+            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o2));
+        }
+        if (lane == 0) {
+            red[warp] = mq;
+            red[4 + warp] = mc;
+            s_mn[warp] = mn;
+        }
     }
     __syncthreads();
     // sigma puts every ||x~|| below 2^12
-    float qmax = 0.f;
+    float qmax = 0.f, c3max = 0.f, c3min = INFINITY;
 #pragma unroll
-    for (int w = 0; w < TOK / 32; ++w) qmax = fmaxf(qmax, red[w]);
+    for (int w = 0; w < TOK / 32; ++w) {
+        qmax = fmaxf(qmax, red[w]);
+        c3max = fmaxf(c3max, red[4 + w]);
+        c3min = fminf(c3min, s_mn[w]);
+    }
     const float sigma = ldexpf(inv_pow2_above(qmax * (2.f * P.half_1p2a / P.a)), 12);
-    if (tid < TOK) s_o1[tid] *= 1.f / sigma;
+    // The weighted products c3_j w S go to fp16 as s_j c3_j w S, and Z3's column j
+    // carries s_j, which the update and the readout take out again (exactly: s_j is a
+    // power of two).  Normally one s_j = sc3 serves the whole chunk, scaling its
+    // largest c3 below 1, and the update's Z3 coefficient is common to all tokens;
+    // when the chunk's norms spread so far that the smallest c3 sc3 would lose fp16
+    // precision (a state decayed far below its tokens' writes), every token takes its
+    // own s_j with c3_j s_j in [1/2, 1).  Both give the same bits where both apply.
+    // With 64-token chunks every token takes its own s_j always (measured faster than
+    // carrying both update loops; with 128-token chunks the common loop is faster).
+    constexpr bool kPerTokenAlways = TOK == 64;
+    const float sc3 = inv_pow2_above(c3max);
+    const bool s3_common = !kPerTokenAlways && c3max <= 0x1p12f * c3min;
+    auto s3_of = [&](float c3j) { return s3_common ? sc3 : inv_pow2_above(c3j); };
+    if (tid < TOK) {
+        s_o1[tid] *= 1.f / sigma;
+        s_t3[tid] = 1.f / s3_of(s_c3[tid]);
+    }
 
     // q^T: this thread's tokens of row d, written into the (now free) tile as
     // [128 d][64 tokens] with 128B-swizzled rows: 8 tokens per 16-byte load later
@@ -602,7 +633,8 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
             for (int u = 0; u < 16; ++u) {
                 const int j = js + c * 16 + u;
                 if (c * 16 + u > 0) w = (j == key && s_owner) ? 1.f : w * s_bet[j];
-                wv[u] = w * s_c3[tcol + c * 16 + u];   // s_j c3_j w_ji
+                const float c3j = s_c3[tcol + c * 16 + u];
+                wv[u] = w * (c3j * s3_of(c3j));   // s_j c3_j w_ji
             }
             tc::tmem_st16(tl + T_W + tcol + c * 16, wv);
         }
@@ -630,7 +662,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     if (P.r > 1) {   // the first Chebyshev round's tables: -w c1 and -w / s_j per token
         for (int e = tid; e < TOK; e += kSolveThreads) {
             s_coef[TOK + e] = -P.omega[1] * s_c1[e];
-            s_coef3[TOK + e] = -P.omega[1] * s_t3[e];
+            if (!s3_common) s_coef3[TOK + e] = -P.omega[1] * s_t3[e];
         }
     }
     fence_proxy_async_smem();
@@ -746,7 +778,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         // kept in the x_prev columns of TMEM; B, once Z3 is done: x_new = part - w c3 Z3.
         // Pairs of tokens go through the packed f32x2 FMA pipe.
         const float cAs = 1.f - P.omega[it], cBs = P.omega[it] * (1.f - cl);
-        const float kqs = P.omega[it] * sigma;
+        const float kqs = P.omega[it] * sigma, k3s = -P.omega[it] / sc3;
         const float2 cA = make_float2(cAs, cAs), cB = make_float2(cBs, cBs);
         const float2 kq = make_float2(kqs, kqs);
         const float *k1 = s_coef + (it & 1) * TOK, *k3t = s_coef3 + (it & 1) * TOK;
@@ -799,34 +831,51 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         ph ^= 1u;
         if (!out_pass) {
             tc::tmem_wait_st();   // this thread's parts are in TMEM
+            // x_new = part + k3_j Z3_j: k3 = -w / sc3 for the whole chunk, or -w / s_j from
+            // the table (two copies of the loop, so that the common case loads nothing)
+            auto update_b = [&](auto per_token) {
 #pragma unroll
-            for (int c = 0; c < TPT / 8; ++c) {
-                const int t0 = tcol + c * 8;
-                float z3[8], part[8];
-                tc::tmem_ld8(tl + T_Z3 + t0, z3);
-                tc::tmem_ld8(tl + T_XP + t0, part);
-                const float4 g3[2] = {*reinterpret_cast<const float4 *>(k3t + t0),
-                                      *reinterpret_cast<const float4 *>(k3t + t0 + 4)};
-                tc::tmem_wait_ld();
-                // x becomes the next round's x_prev (the part just read is dead), and the
-                // new iterate takes x's registers
-                tc::tmem_st8(tl + T_XP + t0, &xc[c * 8]);
+                for (int c = 0; c < TPT / 8; ++c) {
+                    const int t0 = tcol + c * 8;
+                    float z3[8], part[8];
+                    tc::tmem_ld8(tl + T_Z3 + t0, z3);
+                    tc::tmem_ld8(tl + T_XP + t0, part);
+                    float4 g3[2];
+                    if constexpr (decltype(per_token)::value) {
+                        g3[0] = *reinterpret_cast<const float4 *>(k3t + t0);
+                        g3[1] = *reinterpret_cast<const float4 *>(k3t + t0 + 4);
+                    }
+                    tc::tmem_wait_ld();
+                    // x becomes the next round's x_prev (the part just read is dead), and
+                    // the new iterate takes x's registers
+                    tc::tmem_st8(tl + T_XP + t0, &xc[c * 8]);
 #pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    const float2 k3 = (p & 1) ? make_float2(g3[p >> 1].z, g3[p >> 1].w)
-                                              : make_float2(g3[p >> 1].x, g3[p >> 1].y);
-                    const float2 t = __ffma2_rn(k3, make_float2(z3[2 * p], z3[2 * p + 1]),
-                                                make_float2(part[2 * p], part[2 * p + 1]));
-                    xc[c * 8 + 2 * p] = t.x;
-                    xc[c * 8 + 2 * p + 1] = t.y;
+                    for (int p = 0; p < 4; ++p) {
+                        float2 k3 = make_float2(k3s, k3s);
+                        if constexpr (decltype(per_token)::value)
+                            k3 = (p & 1) ? make_float2(g3[p >> 1].z, g3[p >> 1].w)
+                                         : make_float2(g3[p >> 1].x, g3[p >> 1].y);
+                        const float2 t = __ffma2_rn(k3, make_float2(z3[2 * p], z3[2 * p + 1]),
+                                                    make_float2(part[2 * p], part[2 * p + 1]));
+                        xc[c * 8 + 2 * p] = t.x;
+                        xc[c * 8 + 2 * p + 1] = t.y;
+                    }
+                    st_row8(sb + L::XT + (t0 >> 6) * 16384u, d, t0 & 63, &xc[c * 8]);
                 }
-                st_row8(sb + L::XT + (t0 >> 6) * 16384u, d, t0 & 63, &xc[c * 8]);
+            };
+            if constexpr (kPerTokenAlways) {
+                update_b(std::true_type{});
+            } else {
+                if (s3_common)
+                    update_b(std::false_type{});
+                else
+                    update_b(std::true_type{});
             }
             // the next round's coefficient table (the other buffer)
             if (it + 1 < P.r) {
                 for (int e = tid; e < TOK; e += kSolveThreads) {
                     s_coef[((it + 1) & 1) * TOK + e] = -w_next * s_c1[e];
-                    s_coef3[((it + 1) & 1) * TOK + e] = -w_next * s_t3[e];
+                    if (!s3_common) s_coef3[((it + 1) & 1) * TOK + e] = -w_next * s_t3[e];
                 }
             }
             fence_proxy_async_smem();
@@ -855,14 +904,12 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     }
 
     if (XOUT && ok) {
-        // x_j = x~_j invd_j / sigma, invd_j = c3_j sK^2 = (c3_j s_j) (1 / s_j) sK^2
-        // (thread (wg, d): element d of its tokens; consecutive d of a token are
-        // consecutive threads)
+        // x_j = x~_j invd_j / sigma, invd_j = c3_j sK^2 (thread (wg, d): element d of
+        // its tokens; consecutive d of a token are consecutive threads)
         const float xs = sK * sK / sigma;
         float *xrow = x_out + (tok0 + tcol) * kTcD + d;
 #pragma unroll
-        for (int u = 0; u < TPT; ++u)
-            xrow[(size_t)u * kTcD] = xc[u] * ((s_c3[tcol + u] * s_t3[tcol + u]) * xs);
+        for (int u = 0; u < TPT; ++u) xrow[(size_t)u * kTcD] = xc[u] * (s_c3[tcol + u] * xs);
     }
     // teardown: no MMA, copy or TMEM store of this CTA may be in flight when TMEM is freed
     tc::tmem_wait_st();

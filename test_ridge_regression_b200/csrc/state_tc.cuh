@@ -39,8 +39,9 @@
 //
 // With S > 1 the sequence of every head is cut into S segments of whole chunks
 // (seg_tc.cuh): CTA (m, bh * S + s) runs segment s from its start state
-// seg_start[bh][s] and norm bound seg_bound[bh][s] (fp32, from the segment scan)
-// instead of from zero, and only the last segment writes final_state.
+// seg_start[bh][K s] and norm bound seg_bound[bh][K s] (fp32, from the scan over
+// the K S finer segments of the aggregates) instead of from zero, and only the
+// last segment writes final_state.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -106,13 +107,13 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
 }
 
 // grid (2, B*H*S), block kStateThreads.  T = N * C.  seg_start: fp32
-// [B*H][S][2][128][128], seg_bound: [B*H][S][2] (both unused when S == 1).
+// [B*H][K*S][2][128][128], seg_bound: [B*H][K*S][2] (both unused when S == 1).
 template <int C>
 __global__ void __launch_bounds__(kStateThreads, 1)
 k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict__ beta,
                 const float *__restrict__ gate, int *__restrict__ state_exp, float *__restrict__ decay,
                 float *__restrict__ tokdec, size_t plane, float *__restrict__ final_state,
-                int T, int N, int S, const float *__restrict__ seg_start,
+                int T, int N, int S, int K, const float *__restrict__ seg_start,
                 const float *__restrict__ seg_bound, int *__restrict__ timeout_flag) {
     using L = StateSmem<C>;
     constexpr int D = 128, NP = L::NP, PER = C / 32;
@@ -348,13 +349,14 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
     const size_t DD = (size_t)D * D;
     if (S > 1 && arith) {
         // the segment's start state and norm bound (zero for the first segment)
-        const float *src = seg_start + (((size_t)bh * S + seg) * 2 + m) * DD + (size_t)d * D + cg * 32;
+        const size_t e0 = (size_t)bh * S * K + (size_t)seg * K;   // this segment's start entry
+        const float *src = seg_start + (e0 * 2 + m) * DD + (size_t)d * D + cg * 32;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const float4 x = *reinterpret_cast<const float4 *>(src + 4 * j);
             st[4 * j] = x.x; st[4 * j + 1] = x.y; st[4 * j + 2] = x.z; st[4 * j + 3] = x.w;
         }
-        bound = seg_bound[((size_t)bh * S + seg) * 2 + m];
+        bound = seg_bound[e0 * 2 + m];
     } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i) st[i] = 0.f;
