@@ -23,9 +23,9 @@
 //
 // Step 1's operands: A = K or V as loaded (bf16 is exact) and the weighted
 // keys w_i k_i split into two bf16 parts (hi + lo, 16 mantissa bits), as in
-// the one-pass kernel; accumulation in fp32 (TMEM).  The weights come from
-// clamped log(beta) summed in double from the segment's end backwards, one
-// piece at a time.  Step 1 may cut the sequences finer than step 3 (S1 = K S3
+// the one-pass kernel; accumulation in fp32 (TMEM).  The weights are products of
+// beta from the segment's end backwards: fp32 suffix products inside each
+// 64-token piece, times the product over the later pieces carried in double.  Step 1 may cut the sequences finer than step 3 (S1 = K S3
 // segments, so that it too fills the SMs); step 3 then starts its segment s
 // from step 2's start of segment K s.
 #pragma once
@@ -53,8 +53,8 @@ struct SegSmem {
     static constexpr uint32_t BETA = PARTS + 2 * 2 * TILE;         // [stages][64] floats
     static constexpr uint32_t GATE = BETA + kSegStages * 4 * kSegSub;
     static constexpr uint32_t W = GATE + kSegStages * 4 * kSegSub; // [2][64] weights
-    static constexpr uint32_t RED = W + 2 * 4 * kSegSub;           // [2][8] bound partials
-    static constexpr uint32_t BARS = RED + 64;    // load[stages] mma[2] wrdy[2] pdone[2] fin
+    static constexpr uint32_t RED = W + 2 * 4 * kSegSub;           // [2][prep warps] bound partials
+    static constexpr uint32_t BARS = RED + 8 * kSegPrepWarps;    // load[stages] mma[2] wrdy[2] pdone[2] fin
     static constexpr uint32_t TBASE = BARS + 8 * (kSegStages + 7);
     static constexpr uint32_t END = TBASE + 16;
     static constexpr size_t bytes = END + 1024;
@@ -156,7 +156,7 @@ k_seg_delta_tc(const __grid_constant__ StateMaps maps, const float *__restrict__
     const uint32_t tmem = *tbase;
 
     bool ok = true;
-    double suf = 0.0;   // control warp: summed log decay of the pieces after this one
+    double suf = 1.0;   // control warp: product of beta over the pieces after this one
     float binc_h = 0.f, binc_m = 0.f;   // prep threads: shares of the bound increments
     int last_load[kSegStages];   // control lane 0: piece last loaded into each stage
     for (int i = 0; i < kSegStages; ++i) last_load[i] = i < nsub && i < 2 ? i : -1;
@@ -170,28 +170,30 @@ k_seg_delta_tc(const __grid_constant__ StateMaps maps, const float *__restrict__
                 ok = false;
                 break;
             }
-            // weights(c) -> s_w[c & 1]: w_i = g_i exp(sum of the logs after token i in
-            // the segment); lane l holds tokens 2l, 2l + 1.  The buffer's last reader,
+            // weights(c) -> s_w[c & 1]: w_i = g_i prod_{m > i in the segment} beta_m,
+            // as fp32 suffix products inside the piece (as the one-pass kernel forms
+            // its chunk weights) times the product over the pieces after it, carried in
+            // double; lane l holds tokens 2l, 2l + 1.  The buffer's last reader,
             // parts(c - 2), finished before MMA(c - 2) was issued.
             const float *bt = s_beta + st * kSegSub;
-            const double l0 = fmax((double)logf(bt[2 * lane]), kLogBetaMin);
-            const double l1 = fmax((double)logf(bt[2 * lane + 1]), kLogBetaMin);
-            double tot = l0 + l1;   // -> sum over the tokens of this lane and the lanes above
+            const float b0 = bt[2 * lane], b1 = bt[2 * lane + 1];
+            float tot = b0 * b1;   // -> product over the tokens of this lane and the lanes above
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                const double y = __shfl_down_sync(0xffffffffu, tot, o);
-                if (lane + o < 32) tot += y;
+                const float y = __shfl_down_sync(0xffffffffu, tot, o);
+                if (lane + o < 32) tot *= y;
             }
-            double after = __shfl_down_sync(0xffffffffu, tot, 1);   // the lanes above
-            if (lane == 31) after = 0.0;
-            float w1 = decay_exp(suf + after), w0 = decay_exp(suf + after + l1);
+            float after = __shfl_down_sync(0xffffffffu, tot, 1);   // the lanes above
+            if (lane == 31) after = 1.f;
+            const float later = (float)suf;   // the pieces after this one
+            float w1 = later * after, w0 = later * (after * b1);
             if (gate) {
                 w0 *= s_gate[st * kSegSub + 2 * lane];
                 w1 *= s_gate[st * kSegSub + 2 * lane + 1];
             }
             s_w[(c & 1) * kSegSub + 2 * lane] = w0;
             s_w[(c & 1) * kSegSub + 2 * lane + 1] = w1;
-            suf += __shfl_sync(0xffffffffu, tot, 0);
+            suf *= (double)__shfl_sync(0xffffffffu, tot, 0);
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar_wrdy[c & 1]);
             // MMA(c - 1) once its parts are formed
@@ -284,7 +286,7 @@ k_seg_delta_tc(const __grid_constant__ StateMaps maps, const float *__restrict__
         binc_m = warp_sum(binc_m);
         if (lane == 0) {
             s_red[warp] = binc_h;
-            s_red[8 + warp] = binc_m;
+            s_red[kSegPrepWarps + warp] = binc_m;
         }
     }
     tc::fence_before_sync();
@@ -296,15 +298,16 @@ k_seg_delta_tc(const __grid_constant__ StateMaps maps, const float *__restrict__
                 float bh_ = 0.f, bm_ = 0.f;
                 for (int w = 0; w < kSegPrepWarps; ++w) {
                     bh_ += s_red[w];
-                    bm_ += s_red[8 + w];
+                    bm_ += s_red[kSegPrepWarps + w];
                 }
-                segdec[(size_t)bh * S + s] = decay_exp(suf);
+                segdec[(size_t)bh * S + s] = (float)suf;
                 seginc[((size_t)bh * S + s) * 2] = bh_;
                 seginc[((size_t)bh * S + s) * 2 + 1] = bm_;
             }
         } else {
             // rows of the two accumulators: warp w reads lane quarter w % 4, columns
-            // (w / 4) * 64 .. + 63 of H and of M
+            // (w / 4) * CW .. + CW - 1 of H and of M
+            constexpr int CW = 128 / (kSegPrepWarps / 4);
             const int quarter = warp & 3, half = warp >> 2;
             const int d = quarter * 32 + lane;
             const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
@@ -312,13 +315,13 @@ k_seg_delta_tc(const __grid_constant__ StateMaps maps, const float *__restrict__
 #pragma unroll 1
             for (int m = 0; m < 2; ++m)
 #pragma unroll
-                for (int cb = 0; cb < 64; cb += 16) {
+                for (int cb = 0; cb < CW; cb += 16) {
                     float v[16];
-                    tc::tmem_ld16(tl + m * 128 + half * 64 + cb, v);
+                    tc::tmem_ld16(tl + m * 128 + half * CW + cb, v);
                     tc::tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < 4; ++j)
-                        *reinterpret_cast<float4 *>(dst + (size_t)m * D * D + half * 64 + cb + 4 * j) =
+                        *reinterpret_cast<float4 *>(dst + (size_t)m * D * D + half * CW + cb + 4 * j) =
                             make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
                 }
         }
@@ -351,7 +354,9 @@ k_seg_scan(float *__restrict__ agg, const float *__restrict__ segdec,
     const int e = (blockIdx.x * 256 + threadIdx.x) * 4;
     float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
     float *base = agg + (size_t)bh * S * DD2 + e;
-#pragma unroll 1
+    // the loads of later segments do not depend on the carry: unrolled, several are
+    // in flight at once
+#pragma unroll 8
     for (int s = 0; s < S; ++s) {
         float4 *p = reinterpret_cast<float4 *>(base + (size_t)s * DD2);
         const float4 a = *p;
