@@ -38,21 +38,21 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # bench reports null.  The captures' commands sit beside their summaries.
 TRAFFIC = {
     # full-size forward workload (B8 H8 T2048 D128, chunk 64), one launch
-    "chunk_solve_tc": {"bytes": 237.182720e6 + 20.763136e6, "workload": "bf16_b8h8t2048d128",
+    "chunk_solve_tc": {"bytes": 237.150208e6 + 24.922368e6, "workload": "bf16_b8h8t2048d128",
                        "src": "test_ridge_regression_b200/csrc/solve_tc.cuh",
-                       "sha1": "45f1ba0509465c05e81305cbf9b066dcc0cd12f2"},
-    "state_pass_tc": {"bytes": 67.759872e6 + 80.081664e6, "workload": "bf16_b8h8t2048d128",
+                       "sha1": "286fdd815b3667d7662765cf1a59620fe4837263"},
+    "state_pass_tc": {"bytes": 67.709184e6 + 80.409600e6, "workload": "bf16_b8h8t2048d128",
                       "src": "test_ridge_regression_b200/csrc/state_tc.cuh",
-                      "sha1": "3bd3bff3a2f8e7bf8df221195dc42f9281487e71"},
+                      "sha1": "3eca50dc232392420fce4b8be90af9a2dbb55376"},
     # backward row products captured at B2 H8 T2048 (1024 chunks), scaled x4 to the
     # 4096 chunks of the full workload (per-chunk traffic does not depend on B)
     "bwd_rows_tc": {"bytes": 4 * (397.614848e6 + 72.314624e6), "workload": "bf16_b8h8t2048d128",
                     "src": "test_ridge_regression_b200/csrc/backward_tc.cuh",
                     "sha1": "bae7a862a52575dedb40425feeb40e75c13d8c07"},
     # decode captured on 64 x 32 heads (state above L2), scaled x4 to 256 x 32 heads
-    "decode_step": {"bytes": 4 * (270.059520e6 + 211.768320e6), "workload": "decode_bf16_b256h32d128",
+    "decode_step": {"bytes": 4 * (270.047744e6 + 209.314304e6), "workload": "decode_bf16_b256h32d128",
                     "src": "test_ridge_regression_b200/csrc/decode.cuh",
-                    "sha1": "584a95174601413ebccb32a81bd0bfb4d0217334"},
+                    "sha1": "d44e3d48e5d9db859d7f30a83bd2cb179807360a"},
 }
 
 def traffic_of(kernel, workload):

@@ -354,16 +354,27 @@ k_seg_scan(float *__restrict__ agg, const float *__restrict__ segdec,
     const int e = (blockIdx.x * 256 + threadIdx.x) * 4;
     float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
     float *base = agg + (size_t)bh * S * DD2 + e;
-    // the loads of later segments do not depend on the carry: unrolled, several are
-    // in flight at once
-#pragma unroll 8
-    for (int s = 0; s < S; ++s) {
-        float4 *p = reinterpret_cast<float4 *>(base + (size_t)s * DD2);
-        const float4 a = *p;
-        *p = run;
-        const float b = segdec[(size_t)bh * S + s];
-        run = make_float4(fmaf(b, run.x, a.x), fmaf(b, run.y, a.y), fmaf(b, run.z, a.z),
-                          fmaf(b, run.w, a.w));
+    // eight segments at a time: their loads go out before any store into the same
+    // array (which would otherwise order every load behind the previous store)
+    constexpr int kB = 8;
+#pragma unroll 1
+    for (int s0 = 0; s0 < S; s0 += kB) {
+        float4 av[kB];
+        float bv[kB];
+#pragma unroll
+        for (int j = 0; j < kB; ++j)
+            if (s0 + j < S) {
+                av[j] = *reinterpret_cast<const float4 *>(base + (size_t)(s0 + j) * DD2);
+                bv[j] = segdec[(size_t)bh * S + s0 + j];
+            }
+#pragma unroll
+        for (int j = 0; j < kB; ++j)
+            if (s0 + j < S) {
+                *reinterpret_cast<float4 *>(base + (size_t)(s0 + j) * DD2) = run;
+                const float bb = bv[j];
+                run = make_float4(fmaf(bb, run.x, av[j].x), fmaf(bb, run.y, av[j].y),
+                                  fmaf(bb, run.z, av[j].z), fmaf(bb, run.w, av[j].w));
+            }
     }
     if (blockIdx.x == 0 && threadIdx.x < 2) {
         float bd = 0.f;

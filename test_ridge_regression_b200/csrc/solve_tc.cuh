@@ -117,6 +117,12 @@ __device__ __forceinline__ float inv_pow2_above(float x) {
     return __int_as_float((rb < 1 ? 1 : rb) << 23);
 }
 
+// 2^e exactly, from the exponent field: e in [-126, 127] (float), [-1022, 1023] (double).
+__device__ __forceinline__ float pow2f(int e) { return __int_as_float((e + 127) << 23); }
+__device__ __forceinline__ double pow2d(int e) {
+    return __longlong_as_double((long long)(e + 1023) << 52);
+}
+
 // 16 consecutive fp32 values from shared memory (16-byte aligned), as 4 vector loads.
 __device__ __forceinline__ void ld_f32x16(const float *p, float *v) {
 #pragma unroll
@@ -467,7 +473,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
             upart[quarter * MG + wg * HALF + lane * (HALF / 32) + s2] = pv[s2];
     }
     __syncthreads();
-    const float inv_uscale = ldexpf(1.f, -eHexp) / (sK * sK);
+    const float inv_uscale = pow2f(-eHexp) / (sK * sK);   // state exponents lie in [-120, 120]
     if (tid < MG) s_u[tid] = (upart[tid] + upart[MG + tid] + upart[2 * MG + tid] +
                               upart[3 * MG + tid]) * inv_uscale;
     __syncthreads();
@@ -545,7 +551,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         // in double: after long runs of strong decay without writes b_j^2 ||H_s||^2
         // falls below the fp32 range while ||H_j|| itself (and, since the layer is
         // invariant to scaling H and M together, the output) is still well defined
-        const double hs2 = (double)hs2s * ldexp(1.0, -2 * eHexp);
+        const double hs2 = (double)hs2s * pow2d(-2 * eHexp);
         const float b = s_bt[j];
         const double bj = b;
         const double n2 = bj * bj * hs2 + 2.0 * bj * (double)(s_X[j] + s_X1[j]) + (double)s_R[j];
@@ -556,8 +562,8 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         const float invd = nj > 0.f ? 1.f / (P.half_1p2a * nj) : 0.f;
         const float *qpart = reinterpret_cast<const float *>(sm + L::QPART);
         const float qn = sqrtf(qpart[j] + qpart[TOK + j] + qpart[2 * TOK + j] + qpart[3 * TOK + j]);
-        const float eH = ldexpf(1.f, -eHexp);
-        const float eM = ldexpf(1.f, -eMexp);
+        const float eH = pow2f(-eHexp);
+        const float eM = pow2f(-eMexp);
         // The iterate of token j is kept as x~ = (sigma / invd_j) x with sigma a power of
         // two common to the CTA.  Every Chebyshev iterate obeys ||x|| <= ||q|| (1+2a) /
         // (a d), so ||x~|| <= sigma ||q|| (1+2a) / a for every token, and in the scaled
@@ -590,7 +596,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         c3max = fmaxf(c3max, red[4 + w]);
         c3min = fminf(c3min, s_mn[w]);
     }
-    const float sigma = ldexpf(inv_pow2_above(qmax * (2.f * P.half_1p2a / P.a)), 12);
+    const float sigma = inv_pow2_above(qmax * (2.f * P.half_1p2a / P.a)) * 4096.f;
     // The weighted products c3_j w S go to fp16 as s_j c3_j w S, and Z3's column j
     // carries s_j, which the update and the readout take out again (exactly: s_j is a
     // power of two).  Normally one s_j = sc3 serves the whole chunk, scaling its
