@@ -314,8 +314,10 @@ int gka_version(void);
 
 /* Launch profiler.  Kernels of the library, by index into gka_kernel_times. */
 enum {
-    GKA_KERNEL_CHUNK_DELTA = 0,   /* chunk-state increments (scan step 1a) */
-    GKA_KERNEL_STATE_SCAN = 1,    /* sequential state scan over chunks (step 1b) */
+    GKA_KERNEL_CHUNK_DELTA = 0,   /* chunk-state increments (scan step 1a); with few heads on the
+                                     tensor-core path, the segment aggregates */
+    GKA_KERNEL_STATE_SCAN = 1,    /* sequential state scan over chunks (step 1b); with few heads
+                                     on the tensor-core path, the scan of the segment starts */
     GKA_KERNEL_CHUNK_NORM = 2,    /* per-token ||H_t||_F */
     GKA_KERNEL_CHUNK_SOLVE = 3,   /* Chebyshev solve + readout */
     GKA_KERNEL_DECODE_STEP = 4,   /* recurrent decode step */
