@@ -50,9 +50,9 @@ TRAFFIC = {
                     "src": "test_ridge_regression_b200/csrc/backward_tc.cuh",
                     "sha1": "bae7a862a52575dedb40425feeb40e75c13d8c07"},
     # decode captured on 64 x 32 heads (state above L2), scaled x4 to 256 x 32 heads
-    "decode_step": {"bytes": 4 * (270.047744e6 + 209.314304e6), "workload": "decode_bf16_b256h32d128",
+    "decode_step": {"bytes": 4 * (270.045952e6 + 209.251584e6), "workload": "decode_bf16_b256h32d128",
                     "src": "test_ridge_regression_b200/csrc/decode.cuh",
-                    "sha1": "d44e3d48e5d9db859d7f30a83bd2cb179807360a"},
+                    "sha1": "7f7fb0601312f76476c7888b57b106839465129d"},
 }
 
 def traffic_of(kernel, workload):

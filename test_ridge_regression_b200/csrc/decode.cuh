@@ -302,16 +302,16 @@ k_decode_rows(const __grid_constant__ DecodeMaps maps, const Tin *__restrict__ q
     int cur = 0;
 #pragma unroll 1
     for (int it = 1; it < P.r; ++it) {
-        float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+        // packed f32x2 FMAs: half the issued instructions of scalar ones (the step runs
+        // close to the power cap, where fewer issued instructions leave more clock)
+        float2 y01 = make_float2(0.f, 0.f), y23 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int c = 0; c < D / 4; ++c) {
             const float4 xv = *reinterpret_cast<const float4 *>(&xbuf[cur][4 * c]);
-            y0 = fmaf(h[4 * c], xv.x, y0);
-            y1 = fmaf(h[4 * c + 1], xv.y, y1);
-            y2 = fmaf(h[4 * c + 2], xv.z, y2);
-            y3 = fmaf(h[4 * c + 3], xv.w, y3);
+            y01 = __ffma2_rn(make_float2(h[4 * c], h[4 * c + 1]), make_float2(xv.x, xv.y), y01);
+            y23 = __ffma2_rn(make_float2(h[4 * c + 2], h[4 * c + 3]), make_float2(xv.z, xv.w), y23);
         }
-        const float y = fmaf(lam, xcur, (y0 + y1) + (y2 + y3));
+        const float y = fmaf(lam, xcur, (y01.x + y01.y) + (y23.x + y23.y));
         const float xn = fmaf(P.omega[it], fmaf(qt - y, invd, xcur - xprev), xprev);
         xprev = xcur;
         xcur = xn;
@@ -326,24 +326,23 @@ k_decode_rows(const __grid_constant__ DecodeMaps maps, const Tin *__restrict__ q
     const float bm = beta[head];   // reloaded (cached) rather than held through the products
     // (h stays live through this loop for the store below: a partial unroll and two
     // accumulators keep the loop's temporaries within the register budget, no spill)
-    float o0 = 0.f, o1 = 0.f;
+    float2 o01 = make_float2(0.f, 0.f);
+    const float2 bm2 = make_float2(bm, bm), vt2 = make_float2(vt, vt);
 #pragma unroll 4
     for (int c = 0; c < D / 4; ++c) {
         float4 *p = reinterpret_cast<float4 *>(buf + dec_tile_off(t, c));
-        float4 mv = *p;
+        const float4 mv = *p;
         const float4 kv = *reinterpret_cast<const float4 *>(&ks[4 * c]);
         const float4 xv = *reinterpret_cast<const float4 *>(&xbuf[cur][4 * c]);
-        mv.x = fmaf(bm, mv.x, vt * kv.x);
-        mv.y = fmaf(bm, mv.y, vt * kv.y);
-        mv.z = fmaf(bm, mv.z, vt * kv.z);
-        mv.w = fmaf(bm, mv.w, vt * kv.w);
-        o0 = fmaf(mv.x, xv.x, o0);
-        o1 = fmaf(mv.y, xv.y, o1);
-        o0 = fmaf(mv.z, xv.z, o0);
-        o1 = fmaf(mv.w, xv.w, o1);
-        *p = mv;
+        const float2 m01 = __ffma2_rn(bm2, make_float2(mv.x, mv.y),
+                                      __fmul2_rn(vt2, make_float2(kv.x, kv.y)));
+        const float2 m23 = __ffma2_rn(bm2, make_float2(mv.z, mv.w),
+                                      __fmul2_rn(vt2, make_float2(kv.z, kv.w)));
+        o01 = __ffma2_rn(m01, make_float2(xv.x, xv.y), o01);
+        o01 = __ffma2_rn(m23, make_float2(xv.z, xv.w), o01);
+        *p = make_float4(m01.x, m01.y, m23.x, m23.y);
     }
-    store_f(o + (size_t)head * D + t, invd > 0.f ? o0 + o1 : 0.f);
+    store_f(o + (size_t)head * D + t, invd > 0.f ? o01.x + o01.y : 0.f);
     fence_proxy_async_smem();
     ok = __syncthreads_and(ok);
     if (t == 0 && ok) {
