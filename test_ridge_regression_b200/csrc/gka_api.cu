@@ -428,43 +428,45 @@ static int backward_simt(const Tin *q, const Tin *k, const Tin *v, const float *
 
     // forward recompute: chunk states, norms and the iterates x_t (bf16, D = 128: the
     // iterates and norms from the tensor-core forward, the fp32 chunk states here)
-    bool delta_tc = false;
+    bool states_done = false;
     if constexpr (std::is_same<Tin, __nv_bfloat16>::value && D == 128) {
         if (L.tc_recompute && C == 32) {
-            // the increments as fp16 MMAs (hi + lo weighted keys, fp32 accuracy)
+            // the chunk states in one sequential pass per (head, matrix) on tcgen05, written
+            // out in fp32 (no increments through memory), and the chunk decays
             int *flag = nullptr;
             if (int rc = timeout_flag_ptr(&flag)) return rc;
-            DeltaMaps dm;
-            if (int rc = rows128_map(&dm.k, k, (uint64_t)BH * T, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+            StateMaps sm32;
+            if (int rc = rows128_map(&sm32.k, k, (uint64_t)BH * T, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                                      64, 32))
                 return rc;
-            if (int rc = rows128_map(&dm.v, v, (uint64_t)BH * T, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+            if (int rc = rows128_map(&sm32.v, v, (uint64_t)BH * T, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                                      64, 32))
                 return rc;
-            if (int rc = rows128_map(&dm.out, states, (uint64_t)BH * (N + 1) * 2 * D,
+            if (int rc = rows128_map(&sm32.out, states, (uint64_t)BH * (N + 1) * 2 * D,
                                      CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 32, 128))
                 return rc;
-            if ((e = set_smem(k_chunk_delta_tc<32>, DeltaSmem<32>::bytes)) != cudaSuccess)
+            if ((e = set_smem(k_state_pass_tc<32>, StateSmem<32>::bytes)) != cudaSuccess)
                 return cuda_fail(e);
-            { ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
-            k_chunk_delta_tc<32><<<dim3(N, BH), kTcThreads, DeltaSmem<32>::bytes, s>>>(
-                dm, beta, gate, states, decay, nullptr, nullptr, 0, T, N, flag); }
+            { ProfScope ps(GKA_KERNEL_STATE_PASS_TC, s);
+            k_state_pass_tc<32><<<dim3(2, BH), kStateThreads, StateSmem<32>::bytes, s>>>(
+                sm32, beta, gate, nullptr, decay, nullptr, 0, nullptr, T, N, 1, 1, nullptr, nullptr,
+                flag); }
             if (int rc = check_launch()) return rc;
-            delta_tc = true;
+            states_done = true;
         }
     }
-    if (!delta_tc) {
+    if (!states_done) {
         const size_t sm_delta = sizeof(float) * 3 * (size_t)C * D;
         if ((e = set_smem(k_chunk_delta<Tin, D>, sm_delta)) != cudaSuccess) return cuda_fail(e);
         { ProfScope ps(GKA_KERNEL_CHUNK_DELTA, s);
         k_chunk_delta<Tin, D><<<dim3(N, BH), kSimtThreads, sm_delta, s>>>(
             k, v, beta, gate, states, decay, nullptr, T, N, C); }
         if (int rc = check_launch()) return rc;
+        { ProfScope ps(GKA_KERNEL_STATE_SCAN, s);
+        k_state_scan<<<dim3((DD2 + 1023) / 1024, BH), 256, 0, s>>>(states, decay, nullptr, nullptr,
+                                                                 nullptr, nullptr, N, DD2, true); }
+        if (int rc = check_launch()) return rc;
     }
-    { ProfScope ps(GKA_KERNEL_STATE_SCAN, s);
-    k_state_scan<<<dim3((DD2 + 1023) / 1024, BH), 256, 0, s>>>(states, decay, nullptr, nullptr,
-                                                             nullptr, nullptr, N, DD2, true); }
-    if (int rc = check_launch()) return rc;
     const size_t sm_solve = SolveSmem<D>::bytes(C);
     bool tc_done = false;
     if constexpr (std::is_same<Tin, __nv_bfloat16>::value && D == 128) {
