@@ -635,10 +635,10 @@ def bench_backward(args, w, dev, qd, kd, vd, bd, flush, rank, world, barrier, pe
     tc_rows = w.dtype == torch.bfloat16 and w.D == 128 and BWD_CHUNK == 32 and w.T % 64 == 0
     if dom == "bwd_rows" and tc_rows:
         # the row products run as fp16 MMAs; what they must move bounds them: per chunk the
-        # four fp32 D x D matrices, the k, v, g (bf16) and x, y (fp32) rows in, R1..R4 and
-        # the per-token scalars out
+        # fp16 copies of H_s and M_s and the two fp32 adjoints, the k, v, g (bf16) and x, y
+        # (fp32) rows in, R1..R4 and the per-token scalars out
         D, C = w.D, BWD_CHUNK
-        per_tok = 4 * D * D * 4 / C + 3 * D * 2 + 2 * D * 4 + 4 * D * 4 + 4 * 4
+        per_tok = (2 * D * D * 2 + 2 * D * D * 4) / C + 3 * D * 2 + 2 * D * 4 + 4 * D * 4 + 4 * 4
         byts = per_tok * head_tok
         ach = byts / (per_kernel[dom] / 1e3) / 1e9
         roof = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": peaks["hbm_gbs"],

@@ -1,20 +1,21 @@
 // Tensor-core row products of the backward pass (bf16 inputs, D = 128, chunks
 // of 32 tokens): the work of k_bwd_rows (backward_simt.cuh) as fp16 MMAs.
 //
-// Per chunk, with its fp32 matrices H_s, M_s (chunk-start states) and E^H, E^M
-// (adjoint states arriving from later chunks), and its rows k_t, v_t, g_t, x_t:
+// Per chunk, with its chunk-start states H_s, M_s (the recompute's state pass writes
+// them as fp16 copies scaled by 2^e, which arrive here by TMA) and its fp32 adjoint
+// states E^H, E^M (arriving from later chunks), and its rows k_t, v_t, g_t, x_t:
 //   R1 = H_s K^T,  Hx = H_s X^T,  Mg = M_s^T G^T,
 //   R2 = (E^H + E^H^T) K^T,  R3 = E^M^T V^T,  R4 = E^M K^T
 // as 128 x 32 tiles (row c = TMEM lane, column t = token), then
 //   R1, R2, R3, R4 to global (rows [B*H*T][128]), and per token
 //   uk = k . R1,  yhx = y . Hx,  gmx = x . Mg,  qe = k . R2 / 2 + v . R4,
 //   and per chunk hs2 = ||H_s||_F^2, eh = <E^H, H_s> + <E^M, M_s>.
-// Every matrix is converted in shared memory to fp16 with a power-of-two scale
-// that puts its largest entry below 1 (relative rounding 2^-11, as the forward's
-// fp16 state copies); k, v, g tiles likewise, x per token.  The accumulators are
-// fp32.  Two phases reuse the matrix tiles: (H_s, M_s) then (E^H, E^M); eh takes
-// H_s and M_s from the fp16 copies that E^H and E^M overwrite (E in fp32), so each
-// matrix is read from memory once.
+// E^H, E^M are converted in shared memory to fp16 with a power-of-two scale that
+// puts their largest entry below 1 (relative rounding 2^-11, as the fp16 state
+// copies); k, v, g tiles likewise, x per token.  The accumulators are fp32.  Two
+// phases reuse the matrix tiles: (H_s, M_s) then (E^H, E^M); eh takes H_s and M_s
+// from the fp16 copies that E^H and E^M overwrite (E in fp32), and hs2 from the fp16
+// copy of H_s, so each matrix is read from memory once.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -39,11 +40,39 @@ struct BwdRowsTcSmem {
     static constexpr uint32_t XS = RX + 8192;      // float[32] x scales
     static constexpr uint32_t RED = XS + 128;      // float[32][4] per-token partial sums
     static constexpr uint32_t MRED = RED + 512;    // float[16] block reductions
-    static constexpr uint32_t BARS = MRED + 64;    // 3 mbarriers: phase A, phase B, drain
+    static constexpr uint32_t BARS = MRED + 64;    // 4 mbarriers: phase A, phase B, drain, states
     static constexpr uint32_t TBASE = BARS + 32;
     static constexpr uint32_t END = TBASE + 16;
     static constexpr size_t bytes = END + 1024;    // + alignment slack
 };
+
+// One 128 x 128 fp16 chunk-start state copy (the state pass's output, scaled by
+// 2^e) from `map` (rows [B*H*N*2*128][128], boxes 64 x 64, 128B swizzle) into a
+// [2 column halves][128 rows][64] swizzled tile: four TMA loads completing on bar.
+__device__ __forceinline__ void load_state_tile(const CUtensorMap *map, int row0, uint8_t *tile,
+                                                uint64_t *bar) {
+    for (int h = 0; h < 2; ++h)
+        for (int rb = 0; rb < 2; ++rb)
+            tc::tma_load_2d(tile + h * 16384 + rb * 8192, map, h * 64, row0 + rb * 64, bar);
+}
+
+// Sum of squares of the fp16 values of a [2][128][64] tile (all 256 threads; this
+// thread's row r = tid / 2, column half tid % 2; the swizzle does not matter to a sum).
+__device__ __forceinline__ float tile_f16_sumsq(uint32_t tile) {
+    const int tid = threadIdx.x, r = tid >> 1, h = tid & 1;
+    float s2 = 0.f;
+#pragma unroll
+    for (int c8 = 0; c8 < 8; ++c8) {
+        const uint4 o = ld_shared_u4(tile + (uint32_t)h * 16384u + (uint32_t)r * 128u + c8 * 16u);
+        const uint32_t w4[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w4[i]));
+            s2 = fmaf(f.x, f.x, fmaf(f.y, f.y, s2));
+        }
+    }
+    return s2;
+}
 
 // Largest value over the block (256 threads); red: 8 floats.
 __device__ __forceinline__ float block_max256(float v, float *red) {
@@ -132,10 +161,12 @@ __device__ __forceinline__ float rows_to_f16_tile(const Src *__restrict__ src, u
     return per_token ? 1.f : sc;
 }
 
-// grid (N, B*H), block 256.  T = N * 32.
+// grid (N, B*H), block 256.  T = N * 32.  H_s, M_s: the fp16 chunk-start state copies
+// of the recompute's state pass (state_map, exponents sexp [B*H][N][2]).
 __global__ void __launch_bounds__(kSimtThreads, 2)
-k_bwd_rows_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
-              const __nv_bfloat16 *__restrict__ dout, const float *__restrict__ states,
+k_bwd_rows_tc(const __grid_constant__ CUtensorMap state_map, const int *__restrict__ sexp,
+              const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
+              const __nv_bfloat16 *__restrict__ dout,
               const float *__restrict__ adj, const float *__restrict__ xs,
               const float *__restrict__ ys, float *__restrict__ R, float *__restrict__ tokq,
               float *__restrict__ chq, int T, int N, int *__restrict__ timeout_flag) {
@@ -155,18 +186,19 @@ k_bwd_rows_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restri
     const int n = blockIdx.x, bh = blockIdx.y;
     const size_t tok0 = (size_t)bh * T + (size_t)n * C;
     const size_t plane = (size_t)gridDim.y * T, RD = plane * D;
-    const float *Hs = states + ((size_t)bh * (N + 1) + n) * 2 * D * D, *Ms = Hs + D * D;
     const float *EH = adj + ((size_t)bh * (N + 1) + n) * 2 * D * D, *EM = EH + D * D;
+    const int srow = (int)(((size_t)bh * N + n) * 2 * D);   // H_s row in the state map
 
     if (tid == 0) {
-        mbar_init(&bars[0], 1);
-        mbar_init(&bars[1], 1);
-        mbar_init(&bars[2], 1);
+        for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
+        // H_s and M_s as fp16 tiles (the state pass's copies), read while the rows convert
+        mbar_arrive_expect_tx(&bars[3], 2 * 32768);
+        load_state_tile(&state_map, srow, sm + L::MA, &bars[3]);
+        load_state_tile(&state_map, srow + D, sm + L::MB, &bars[3]);
     }
     if (tid == 32) {
-        // everything read after the rows: the four matrices and the fp32 y rows
-        bulk_prefetch_l2(Hs, 2 * D * D * 4);
+        // everything read after the rows: the two adjoints and the fp32 y rows
         bulk_prefetch_l2(EH, 2 * D * D * 4);
         bulk_prefetch_l2(ys + tok0 * D, C * D * 4);
     }
@@ -179,9 +211,12 @@ k_bwd_rows_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restri
     const float sV = rows_to_f16_tile(v + tok0 * D, sb + L::RV, mred, false, nullptr);
     const float sG = rows_to_f16_tile(dout + tok0 * D, sb + L::RG, mred, false, nullptr);
     rows_to_f16_tile(xs + tok0 * D, sb + L::RX, mred, true, xsc);
-    float hs2 = 0.f, eh = 0.f;
-    const float sH = mat_to_f16_tile(Hs, sb + L::MA, mred, 0.f, nullptr, &hs2);
-    const float sM = mat_to_f16_tile(Ms, sb + L::MB, mred, 0.f, nullptr, nullptr);
+    float eh = 0.f;
+    // the copies hold 2^e H_s and 2^e' M_s (exponents in [-120, 120])
+    const int eH = sexp[((size_t)bh * N + n) * 2], eM = sexp[((size_t)bh * N + n) * 2 + 1];
+    const float sH = pow2f(eH), sM = pow2f(eM);
+    bool ok = mbar_wait_bounded(&bars[3], 0, kTcWaitProbes);
+    float hs2 = tile_f16_sumsq(sb + L::MA) * (pow2f(-eH) * pow2f(-eH));
     fence_proxy_async_smem();
     tc::fence_before_sync();
     __syncthreads();
@@ -193,15 +228,17 @@ k_bwd_rows_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restri
     auto adesc_t = [&](uint32_t a, int kk) { return tc::sdesc(a + kk * 2048, 16384, 1024); };
     auto bdesc = [&](uint32_t b, int kk) { return tc::sdesc(b + (kk >> 2) * (C * 128) + (kk & 3) * 32, 16, 1024); };
     if (tid == 0) {
+        if (ok) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            tc::mma_f16(tmem + 0, adesc_k(sb + L::MA, kk), bdesc(sb + L::RK, kk), ID_K, kk > 0);
-            tc::mma_f16(tmem + 32, adesc_k(sb + L::MA, kk), bdesc(sb + L::RX, kk), ID_K, kk > 0);
-            tc::mma_f16(tmem + 64, adesc_t(sb + L::MB, kk), bdesc(sb + L::RG, kk), ID_T, kk > 0);
+            for (int kk = 0; kk < 8; ++kk) {
+                tc::mma_f16(tmem + 0, adesc_k(sb + L::MA, kk), bdesc(sb + L::RK, kk), ID_K, kk > 0);
+                tc::mma_f16(tmem + 32, adesc_k(sb + L::MA, kk), bdesc(sb + L::RX, kk), ID_K, kk > 0);
+                tc::mma_f16(tmem + 64, adesc_t(sb + L::MB, kk), bdesc(sb + L::RG, kk), ID_T, kk > 0);
+            }
         }
         tc::commit(&bars[0]);
     }
-    bool ok = mbar_wait_bounded(&bars[0], 0, kTcWaitProbes);
+    if (!mbar_wait_bounded(&bars[0], 0, kTcWaitProbes)) ok = false;
     tc::fence_after_sync();
 
     // per-token sums over the 128 rows: this thread's 16 partials -> red[t][quarter]
@@ -325,6 +362,7 @@ k_bwd_rows_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restri
         atomicExch(timeout_flag, 1);
         tc::commit(&bars[2]);
         mbar_wait_bounded(&bars[2], 0, kTcWaitProbes);
+        mbar_wait_bounded(&bars[3], 0, kTcWaitProbes);   // the state tiles' loads
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -357,16 +395,17 @@ struct BwdUTcSmem {
     static constexpr uint32_t PM = VH + 32 * KP * 4;   // float[32][33] P
     static constexpr uint32_t GR = PM + 32 * 33 * 4;   // bf16 [32][128] g
     static constexpr uint32_t MRED = GR + 8192;    // float[16]
-    static constexpr uint32_t BARS = MRED + 64;    // 2 mbarriers: product, drain
-    static constexpr uint32_t TBASE = BARS + 16;
+    static constexpr uint32_t BARS = MRED + 64;    // 3 mbarriers: product, drain, M_s
+    static constexpr uint32_t TBASE = BARS + 32;
     static constexpr uint32_t END = TBASE + 16;
     static constexpr size_t bytes = END + 1024;    // + alignment slack
 };
 
 __global__ void __launch_bounds__(kSimtThreads, 2)
-k_bwd_u_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
+k_bwd_u_tc(const __grid_constant__ CUtensorMap state_map, const int *__restrict__ sexp,
+           const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
            const float *__restrict__ beta, const float *__restrict__ gate,
-           const __nv_bfloat16 *__restrict__ dout, const float *__restrict__ states,
+           const __nv_bfloat16 *__restrict__ dout,
            __nv_bfloat16 *__restrict__ u_out, int T, int N, int *__restrict__ timeout_flag) {
     using L = BwdUTcSmem;
     constexpr int D = 128, C = kBrC, KP = L::KP, CP = C + 1;
@@ -385,12 +424,16 @@ k_bwd_u_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict_
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n = blockIdx.x, bh = blockIdx.y;
     const size_t tok0 = (size_t)bh * T + (size_t)n * C;
-    const float *Ms = states + ((size_t)bh * (N + 1) + n) * 2 * D * D + D * D;
+    const int srow = (int)(((size_t)bh * N + n) * 2 * D);   // H_s row in the state map; M_s follows
 
     if (tid == 0) {
         mbar_init(&bars[0], 1);
         mbar_init(&bars[1], 1);
+        mbar_init(&bars[2], 1);
         fence_mbar_init();
+        // M_s as an fp16 tile (the state pass's copy, 2^e M_s), read while the rows convert
+        mbar_arrive_expect_tx(&bars[2], 32768);
+        load_state_tile(&state_map, srow + D, sm + L::MB, &bars[2]);
     }
     if (warp == 0) {
         tc::tmem_alloc(tbase, 32);
@@ -407,7 +450,8 @@ k_bwd_u_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict_
         Gr[e] = dout[g];
     }
     const float sG = rows_to_f16_tile(dout + tok0 * D, sb + L::RG, mred, false, nullptr);
-    const float sM = mat_to_f16_tile(Ms, sb + L::MB, mred, 0.f, nullptr, nullptr);
+    const float sM = pow2f(sexp[((size_t)bh * N + n) * 2 + 1]);
+    bool ok = mbar_wait_bounded(&bars[2], 0, kTcWaitProbes);
     fence_proxy_async_smem();
     tc::fence_before_sync();
     __syncthreads();
@@ -415,11 +459,13 @@ k_bwd_u_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict_
     const uint32_t tmem = *tbase;
     if (tid == 0) {
         constexpr uint32_t ID_T = tc::idesc_f16(128, C, true, false);   // A = M_s^T (MN-major)
+        if (ok) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-            tc::mma_f16(tmem, tc::sdesc(sb + L::MB + kk * 2048, 16384, 1024),
-                        tc::sdesc(sb + L::RG + (kk >> 2) * (C * 128) + (kk & 3) * 32, 16, 1024),
-                        ID_T, kk > 0);
+            for (int kk = 0; kk < 8; ++kk)
+                tc::mma_f16(tmem, tc::sdesc(sb + L::MB + kk * 2048, 16384, 1024),
+                            tc::sdesc(sb + L::RG + (kk >> 2) * (C * 128) + (kk & 3) * 32, 16, 1024),
+                            ID_T, kk > 0);
+        }
         tc::commit(&bars[0]);
     }
     // P[t][i] = w_ti (v~_i . g_t), i <= t, while the product runs
@@ -439,7 +485,7 @@ k_bwd_u_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict_
         Pm[t * CP + i] = acc;
     }
     __syncthreads();
-    bool ok = mbar_wait_bounded(&bars[0], 0, kTcWaitProbes);
+    if (!mbar_wait_bounded(&bars[0], 0, kTcWaitProbes)) ok = false;
     tc::fence_after_sync();
     // thread (row c = TMEM lane, tokens 16 wg .. 16 wg + 15)
     const int quarter = warp & 3, wg = warp >> 2, c = quarter * 32 + lane;
@@ -458,6 +504,7 @@ k_bwd_u_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict_
         atomicExch(timeout_flag, 1);
         tc::commit(&bars[1]);
         mbar_wait_bounded(&bars[1], 0, kTcWaitProbes);
+        mbar_wait_bounded(&bars[2], 0, kTcWaitProbes);   // the M_s tile's loads
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -526,11 +573,14 @@ __device__ __forceinline__ void rows_store_f16(const Src *__restrict__ src, cons
 __global__ void __launch_bounds__(kSimtThreads, 2)
 k_bwd_delta_tc(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ beta,
                const float *__restrict__ gate, const __nv_bfloat16 *__restrict__ dout,
-               const float *__restrict__ states, const float *__restrict__ xs,
+               const __half *__restrict__ slp, const int *__restrict__ sexp,
+               const float *__restrict__ xs,
                const float *__restrict__ ys, const float *__restrict__ cvec,
                const __grid_constant__ CUtensorMap adj_map, int T, int N,
                int *__restrict__ timeout_flag) {
-    // adj_map: the adjoint states [B*H*(N+1)*2*128][128] fp32, box 32 x 128, 128B swizzle
+    // adj_map: the adjoint states [B*H*(N+1)*2*128][128] fp32, box 32 x 128, 128B swizzle;
+    // slp, sexp: the recompute's fp16 chunk-start state copies [B*H][N][2][128][128]
+    // (scaled by 2^e) and their exponents [B*H][N][2]
     using L = BwdDeltaTcSmem;
     constexpr int D = 128, C = kBrC;
     extern __shared__ uint8_t smraw[];
@@ -616,7 +666,9 @@ k_bwd_delta_tc(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ be
     // of dE^H (m = 0, with the H_start term) or dE^M (m = 1)
     const int quarter = warp & 3, wg = warp >> 2, p = quarter * 32 + lane;
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
-    const float *Hst = states + ((size_t)bh * (N + 1) + n) * 2 * D * D + (size_t)p * D;
+    // row p of H_start from its fp16 copy (2^e H_start), the scale undone below
+    const __half *Hst = slp + ((size_t)bh * N + n) * 2 * D * D + (size_t)p * D;
+    const float hsc = pow2f(-sexp[((size_t)bh * N + n) * 2]);
     const int orow = (int)(((size_t)bh * (N + 1) + n) * 2 * D);
     const float uH = 1.f / S, uM = 1.f / (sG * sX);
 #pragma unroll 1
@@ -631,7 +683,15 @@ k_bwd_delta_tc(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ be
         float4 h[8];
         if (m == 0) {
 #pragma unroll
-            for (int c = 0; c < 8; ++c) h[c] = *reinterpret_cast<const float4 *>(Hst + col + 4 * c);
+            for (int c = 0; c < 4; ++c) {
+                const uint4 u = *reinterpret_cast<const uint4 *>(Hst + col + 8 * c);
+                const float2 f0 = __half22float2(*reinterpret_cast<const __half2 *>(&u.x));
+                const float2 f1 = __half22float2(*reinterpret_cast<const __half2 *>(&u.y));
+                const float2 f2 = __half22float2(*reinterpret_cast<const __half2 *>(&u.z));
+                const float2 f3 = __half22float2(*reinterpret_cast<const __half2 *>(&u.w));
+                h[2 * c] = make_float4(f0.x * hsc, f0.y * hsc, f1.x * hsc, f1.y * hsc);
+                h[2 * c + 1] = make_float4(f2.x * hsc, f2.y * hsc, f3.x * hsc, f3.y * hsc);
+            }
         }
         tc::tmem_wait_ld();
 #pragma unroll

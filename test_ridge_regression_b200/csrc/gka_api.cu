@@ -428,11 +428,18 @@ static int backward_simt(const Tin *q, const Tin *k, const Tin *v, const float *
 
     // forward recompute: chunk states, norms and the iterates x_t (bf16, D = 128: the
     // iterates and norms from the tensor-core forward, the fp32 chunk states here)
+    // bf16, D = 128, C = 32: the chunk states as fp16 copies (scaled by 2^e, the tensor
+    // cores' operands) with their exponents, in the fp32 state region (twice their size),
+    // which this path leaves unused otherwise
+    __half *slp32 = reinterpret_cast<__half *>(states);
+    int *sexp32 = reinterpret_cast<int *>(reinterpret_cast<char *>(states) +
+                                          round256(sizeof(__half) * BH * (size_t)N * 2 * D * D));
+    CUtensorMap state_map;   // the fp16 copies, boxes 64 x 64, for the consumers' TMA loads
     bool states_done = false;
     if constexpr (std::is_same<Tin, __nv_bfloat16>::value && D == 128) {
         if (L.tc_recompute && C == 32) {
-            // the chunk states in one sequential pass per (head, matrix) on tcgen05, written
-            // out in fp32 (no increments through memory), and the chunk decays
+            // the chunk states in one sequential pass per (head, matrix) on tcgen05 (no
+            // increments through memory), and the chunk decays
             int *flag = nullptr;
             if (int rc = timeout_flag_ptr(&flag)) return rc;
             StateMaps sm32;
@@ -442,14 +449,17 @@ static int backward_simt(const Tin *q, const Tin *k, const Tin *v, const float *
             if (int rc = rows128_map(&sm32.v, v, (uint64_t)BH * T, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                                      64, 32))
                 return rc;
-            if (int rc = rows128_map(&sm32.out, states, (uint64_t)BH * (N + 1) * 2 * D,
-                                     CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 32, 128))
+            if (int rc = rows128_map(&sm32.out, slp32, (uint64_t)BH * N * 2 * D,
+                                     CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 64, 128))
+                return rc;
+            if (int rc = rows128_map(&state_map, slp32, (uint64_t)BH * N * 2 * D,
+                                     CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
                 return rc;
             if ((e = set_smem(k_state_pass_tc<32>, StateSmem<32>::bytes)) != cudaSuccess)
                 return cuda_fail(e);
             { ProfScope ps(GKA_KERNEL_STATE_PASS_TC, s);
             k_state_pass_tc<32><<<dim3(2, BH), kStateThreads, StateSmem<32>::bytes, s>>>(
-                sm32, beta, gate, nullptr, decay, nullptr, 0, nullptr, T, N, 1, 1, nullptr, nullptr,
+                sm32, beta, gate, sexp32, decay, nullptr, 0, nullptr, T, N, 1, 1, nullptr, nullptr,
                 flag); }
             if (int rc = check_launch()) return rc;
             states_done = true;
@@ -505,7 +515,7 @@ static int backward_simt(const Tin *q, const Tin *k, const Tin *v, const float *
             if ((e = set_smem(k_bwd_u_tc, BwdUTcSmem::bytes)) != cudaSuccess) return cuda_fail(e);
             { ProfScope ps(GKA_KERNEL_BWD_SOLVE, s);
             k_bwd_u_tc<<<dim3(N, BH), kSimtThreads, BwdUTcSmem::bytes, s>>>(
-                k, v, beta, gate, dout, states, u16, T, N, flag); }
+                state_map, sexp32, k, v, beta, gate, dout, u16, T, N, flag); }
             u_done = true;
         }
     }
@@ -543,7 +553,7 @@ static int backward_simt(const Tin *q, const Tin *k, const Tin *v, const float *
                 return cuda_fail(e);
             { ProfScope ps(GKA_KERNEL_BWD_DELTA, s);
             k_bwd_delta_tc<<<dim3(N, BH), kSimtThreads, BwdDeltaTcSmem::bytes, s>>>(
-                k, beta, gate, dout, states, xs, ys, cvec, adj_map, T, N, flag); }
+                k, beta, gate, dout, slp32, sexp32, xs, ys, cvec, adj_map, T, N, flag); }
             if (int rc = check_launch()) return rc;
             delta_done = true;
         }
@@ -570,7 +580,7 @@ static int backward_simt(const Tin *q, const Tin *k, const Tin *v, const float *
                 return cuda_fail(e);
             { ProfScope ps(GKA_KERNEL_BWD_ROWS, s);
             k_bwd_rows_tc<<<dim3(N, BH), kSimtThreads, BwdRowsTcSmem::bytes, s>>>(
-                k, v, dout, states, adj, xs, ys, rows, tokq, chq, T, N, flag); }
+                state_map, sexp32, k, v, dout, adj, xs, ys, rows, tokq, chq, T, N, flag); }
             if (int rc = check_launch()) return rc;
             rows_done = true;
         }

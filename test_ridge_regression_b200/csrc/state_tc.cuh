@@ -37,10 +37,8 @@
 //     every copied value <= 2^14.
 // The state after the last chunk goes to final_state (nullable).
 //
-// C = 32 (the backward's recompute): the chunk-start states go out in fp32
-// ([B*H][N+1][2][128][128], slot n = S_n, through the `out` map with 32 x 128 boxes)
-// instead of as scaled fp16 copies; no exponents, no per-token decays (tokdec
-// NULL), the chunk decays as always.
+// C = 32 serves the backward's recompute (32-row TMA boxes; tokdec may be NULL:
+// then no per-token decays, the chunk decays as always).
 //
 // With S > 1 the sequence of every head is cut into S segments of whole chunks
 // (seg_tc.cuh): CTA (m, bh * S + s) runs segment s from its start state
@@ -78,12 +76,11 @@ struct StateSmem {
     static constexpr uint32_t KS = 0;                       // 2 stages of keys
     static constexpr uint32_t VS = KS + 2 * TILE;           // 2 stages of values (M CTA)
     static constexpr uint32_t PARTS = VS + 2 * TILE;        // NPB x NP tiles of (w k) parts
-    // staging of one state copy for its TMA store, 128B-swizzled: fp16 [2 column
-    // halves][128 rows][64] in own space for 64-token chunks; fp32 [4 column
-    // quarters][128 rows][32] for 32-token chunks (fp32 output); with 128-token chunks
-    // the H CTA stages in its (unused) value stages and the M CTA in the key stage of
-    // the chunk it has just prepared (free until that stage is loaded again)
-    static constexpr uint32_t OUTB = C == 64 ? 32768 : (C == 32 ? 65536 : 0);
+    // fp16 staging of one state copy, [2 column halves][128 rows][64], 128B-swizzled:
+    // own space for chunks of up to 64 tokens; with 128-token chunks the H CTA stages
+    // in its (unused) value stages and the M CTA in the key stage of the chunk it has
+    // just prepared (free until that stage is loaded again)
+    static constexpr uint32_t OUTB = C <= 64 ? 32768 : 0;
     static constexpr uint32_t OUT = PARTS + NPB * NP * TILE;
     static constexpr uint32_t BETA = OUT + OUTB;            // [2][C]
     static constexpr uint32_t GATE = BETA + 2 * 4 * C;      // [2][C] write gates
@@ -122,7 +119,6 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
                 float *__restrict__ tokdec, size_t plane, float *__restrict__ final_state,
                 int T, int N, int S, int K, const float *__restrict__ seg_start,
                 const float *__restrict__ seg_bound, int *__restrict__ timeout_flag) {
-    constexpr bool kF32Out = C == 32;       // fp32 chunk states out, no fp16 copies
     constexpr int BOXR = C < 64 ? C : 64;   // rows per TMA box of k and v
     using L = StateSmem<C>;
     constexpr int D = 128, NP = L::NP, PER = C / 32;
@@ -409,16 +405,9 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
                 if (n + 1 < NL) issue_mma(tmem, n + 1);
                 if (!mbar_wait_bounded(bar_out, n & 1, kStateWaitProbes)) fail = true;
                 if (!fail) {
-                    if constexpr (kF32Out) {
-                        // fp32 S_n into slot n of [B*H][N+1][2][128][128]: four 32-column boxes
-                        const int row = (int)(((size_t)bh * (N + 1) + n0 + n) * 2 + m) * D;
-                        for (int cb = 0; cb < 4; ++cb)
-                            tc::tma_store_2d(&maps.out, cb * 32, row, sm + out_stage(n) + cb * 16384);
-                    } else {
-                        const int row = (int)(((size_t)bh * N + n0 + n) * 2 + m) * D;
-                        tc::tma_store_2d(&maps.out, 0, row, sm + out_stage(n));
-                        tc::tma_store_2d(&maps.out, 64, row, sm + out_stage(n) + 16384);
-                    }
+                    const int row = (int)(((size_t)bh * N + n0 + n) * 2 + m) * D;
+                    tc::tma_store_2d(&maps.out, 0, row, sm + out_stage(n));
+                    tc::tma_store_2d(&maps.out, 64, row, sm + out_stage(n) + 16384);
                     tc::bulk_commit();
                 }
             }
@@ -447,17 +436,7 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
         tc::fence_before_sync();
         ok = named_barrier_and(2, kStateBarThreads, ok && !fail);
         if (!ok) break;
-        if constexpr (kF32Out) {
-            // the chunk-start state S_n in fp32, staged in the TMA box layout: [column
-            // quarter cg][row][32], 16-byte chunk j of row d at j ^ (d % 8)
-            uint8_t *row = sm + out_stage(n) + cg * 16384 + d * 128;
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-                *reinterpret_cast<float4 *>(row + ((j ^ d) & 7) * 16) =
-                    make_float4(st[4 * j], st[4 * j + 1], st[4 * j + 2], st[4 * j + 3]);
-            fence_proxy_async_smem();
-            mbar_arrive(bar_out);
-        } else {
+        {
             // fp16 copy of the chunk-start state S_n, scaled by 2^e_n, staged in the TMA
             // box layout: [column half][row][64], 16-byte chunk j of row d at j ^ (d % 8)
             const int ex = lp_exponent_tc(bound);
