@@ -1,21 +1,22 @@
 // Tensor-core row products of the backward pass (bf16 inputs, D = 128, chunks
-// of 32 tokens): the work of k_bwd_rows (backward_simt.cuh) as fp16 MMAs.
+// of 32 tokens): the work of k_bwd_rows (backward_simt.cuh) as fp16 MMAs, and the
+// right-hand side of the adjoint solve.
 //
 // Per chunk, with its chunk-start states H_s, M_s (the recompute's state pass writes
-// them as fp16 copies scaled by 2^e, which arrive here by TMA) and its fp32 adjoint
-// states E^H, E^M (arriving from later chunks), and its rows k_t, v_t, g_t, x_t:
+// them as fp16 copies scaled by 2^e, which arrive here by TMA), its adjoint states
+// E^H, E^M arriving from later chunks (fp16 copies scaled by 2^e from the adjoint pass,
+// adjoint_tc.cuh, also by TMA) and its rows k_t, v_t, g_t, x_t:
 //   R1 = H_s K^T,  Hx = H_s X^T,  Mg = M_s^T G^T,
 //   R2 = (E^H + E^H^T) K^T,  R3 = E^M^T V^T,  R4 = E^M K^T
 // as 128 x 32 tiles (row c = TMEM lane, column t = token), then
 //   R1, R2, R3, R4 to global (rows [B*H*T][128]), and per token
 //   uk = k . R1,  yhx = y . Hx,  gmx = x . Mg,  qe = k . R2 / 2 + v . R4,
-//   and per chunk hs2 = ||H_s||_F^2, eh = <E^H, H_s> + <E^M, M_s>.
-// E^H, E^M are converted in shared memory to fp16 with a power-of-two scale that
-// puts their largest entry below 1 (relative rounding 2^-11, as the fp16 state
-// copies); k, v, g tiles likewise, x per token.  The accumulators are fp32.  Two
-// phases reuse the matrix tiles: (H_s, M_s) then (E^H, E^M); eh takes H_s and M_s
-// from the fp16 copies that E^H and E^M overwrite (E in fp32), and hs2 from the fp16
-// copy of H_s, so each matrix is read from memory once.
+//   and per chunk hs2 = ||H_s||_F^2 (from the fp16 copy) and eh = <E^H, H_s> +
+//   <E^M, M_s> (the adjoint pass forms both terms from its fp32 adjoints).
+// Every copy's largest entry lies below 2^14 (states) or 1 (adjoints); k, v, g tiles
+// are converted in shared memory with one power-of-two scale each, x with one per
+// token.  The accumulators are fp32.  Two phases share the matrix tiles: (H_s, M_s),
+// then (E^H, E^M), loaded once the first phase's products have read the states.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -40,8 +41,9 @@ struct BwdRowsTcSmem {
     static constexpr uint32_t XS = RX + 8192;      // float[32] x scales
     static constexpr uint32_t RED = XS + 128;      // float[32][4] per-token partial sums
     static constexpr uint32_t MRED = RED + 512;    // float[16] block reductions
-    static constexpr uint32_t BARS = MRED + 64;    // 4 mbarriers: phase A, phase B, drain, states
-    static constexpr uint32_t TBASE = BARS + 32;
+    static constexpr uint32_t BARS = MRED + 64;    // 5 mbarriers: phase A, phase B, drain,
+                                                   // states, adjoints
+    static constexpr uint32_t TBASE = BARS + 48;
     static constexpr uint32_t END = TBASE + 16;
     static constexpr size_t bytes = END + 1024;    // + alignment slack
 };
@@ -87,50 +89,6 @@ __device__ __forceinline__ float block_max256(float v, float *red) {
     return m;
 }
 
-// fp32 row-major 128 x 128 matrix -> fp16 [2][128][64] swizzled tile, scaled by a
-// power of two below 1/max.  Thread (row r = tid / 2, column half h = tid % 2) holds
-// its 64 elements in registers between the max and the conversion.
-// prev_scale > 0: the tile holds another matrix W as fp16 scaled by prev_scale; each
-// thread reads the entries it overwrites and accumulates sum A * W into *dot (W at
-// fp16 precision, A in fp32).  sq2 (nullable): accumulates sum A^2.  Returns the scale.
-__device__ __forceinline__ float mat_to_f16_tile(const float *__restrict__ A, uint32_t tile,
-                                                 float *red, float prev_scale, float *dot,
-                                                 float *sq2) {
-    const int tid = threadIdx.x, r = tid >> 1, h = tid & 1;
-    const float4 *src = reinterpret_cast<const float4 *>(A + r * 128 + h * 64);
-    float mx = 0.f, dp = 0.f, s2 = 0.f;
-    // all 16 loads of a pass are issued before their values are used
-    float4 x[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) x[i] = __ldg(src + i);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        mx = fmaxf(mx, fmaxf(fmaxf(fabsf(x[i].x), fabsf(x[i].y)), fmaxf(fabsf(x[i].z), fabsf(x[i].w))));
-        s2 = fmaf(x[i].x, x[i].x, fmaf(x[i].y, x[i].y, fmaf(x[i].z, x[i].z, fmaf(x[i].w, x[i].w, s2))));
-    }
-    if (sq2) *sq2 += s2;
-    const float sc = inv_pow2_above(block_max256(mx, red));
-    const uint32_t base = tile + (uint32_t)h * 16384u;
-#pragma unroll
-    for (int c8 = 0; c8 < 8; ++c8) {
-        const float4 a = x[2 * c8], b = x[2 * c8 + 1];
-        if (prev_scale > 0.f) {
-            const uint4 o = ld_shared_u4(base + (uint32_t)r * 128u + (((uint32_t)c8 ^ (uint32_t)r) & 7u) * 16u);
-            const float2 w0 = __half22float2(*reinterpret_cast<const __half2 *>(&o.x));
-            const float2 w1 = __half22float2(*reinterpret_cast<const __half2 *>(&o.y));
-            const float2 w2 = __half22float2(*reinterpret_cast<const __half2 *>(&o.z));
-            const float2 w3 = __half22float2(*reinterpret_cast<const __half2 *>(&o.w));
-            dp = fmaf(a.x, w0.x, fmaf(a.y, w0.y, fmaf(a.z, w1.x, fmaf(a.w, w1.y, dp))));
-            dp = fmaf(b.x, w2.x, fmaf(b.y, w2.y, fmaf(b.z, w3.x, fmaf(b.w, w3.y, dp))));
-        }
-        const float v[8] = {a.x * sc, a.y * sc, a.z * sc, a.w * sc,
-                            b.x * sc, b.y * sc, b.z * sc, b.w * sc};
-        st_row8(base, (uint32_t)r, (uint32_t)(c8 * 8), v);
-    }
-    if (prev_scale > 0.f) *dot += dp / prev_scale;
-    return sc;
-}
-
 // bf16 rows [32][128] (global) -> fp16 [2][32][64] swizzled tile with one power-of-two
 // scale (per_token: one scale per token row, written to xs).  Thread (token t = tid / 8,
 // 16 columns (tid % 8) * 16).  Returns the tile scale (1 with per_token).
@@ -162,12 +120,15 @@ __device__ __forceinline__ float rows_to_f16_tile(const Src *__restrict__ src, u
 }
 
 // grid (N, B*H), block 256.  T = N * 32.  H_s, M_s: the fp16 chunk-start state copies
-// of the recompute's state pass (state_map, exponents sexp [B*H][N][2]).
+// of the recompute's state pass (state_map, exponents sexp [B*H][N][2]); E^H, E^M: the
+// fp16 adjoint copies of the adjoint pass (adj_map over adj_lp, same layout, exponents
+// aexp) and its inner products eh_part [B*H][N][2] (<E^H, H_s>, <E^M, M_s>).
 __global__ void __launch_bounds__(kSimtThreads, 2)
 k_bwd_rows_tc(const __grid_constant__ CUtensorMap state_map, const int *__restrict__ sexp,
+              const __grid_constant__ CUtensorMap adj_map, const __half *__restrict__ adj_lp,
+              const int *__restrict__ aexp, const float *__restrict__ eh_part,
               const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
-              const __nv_bfloat16 *__restrict__ dout,
-              const float *__restrict__ adj, const float *__restrict__ xs,
+              const __nv_bfloat16 *__restrict__ dout, const float *__restrict__ xs,
               const float *__restrict__ ys, float *__restrict__ R, float *__restrict__ tokq,
               float *__restrict__ chq, int T, int N, int *__restrict__ timeout_flag) {
     using L = BwdRowsTcSmem;
@@ -186,11 +147,10 @@ k_bwd_rows_tc(const __grid_constant__ CUtensorMap state_map, const int *__restri
     const int n = blockIdx.x, bh = blockIdx.y;
     const size_t tok0 = (size_t)bh * T + (size_t)n * C;
     const size_t plane = (size_t)gridDim.y * T, RD = plane * D;
-    const float *EH = adj + ((size_t)bh * (N + 1) + n) * 2 * D * D, *EM = EH + D * D;
-    const int srow = (int)(((size_t)bh * N + n) * 2 * D);   // H_s row in the state map
+    const int srow = (int)(((size_t)bh * N + n) * 2 * D);   // H_s (E^H) row in the maps
 
     if (tid == 0) {
-        for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 5; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
         // H_s and M_s as fp16 tiles (the state pass's copies), read while the rows convert
         mbar_arrive_expect_tx(&bars[3], 2 * 32768);
@@ -198,8 +158,8 @@ k_bwd_rows_tc(const __grid_constant__ CUtensorMap state_map, const int *__restri
         load_state_tile(&state_map, srow + D, sm + L::MB, &bars[3]);
     }
     if (tid == 32) {
-        // everything read after the rows: the two adjoints and the fp32 y rows
-        bulk_prefetch_l2(EH, 2 * D * D * 4);
+        // everything read after the rows: the two adjoint copies and the fp32 y rows
+        bulk_prefetch_l2(adj_lp + (size_t)srow * D, 2 * D * D * 2);
         bulk_prefetch_l2(ys + tok0 * D, C * D * 4);
     }
     if (warp == 0) {
@@ -211,7 +171,6 @@ k_bwd_rows_tc(const __grid_constant__ CUtensorMap state_map, const int *__restri
     const float sV = rows_to_f16_tile(v + tok0 * D, sb + L::RV, mred, false, nullptr);
     const float sG = rows_to_f16_tile(dout + tok0 * D, sb + L::RG, mred, false, nullptr);
     rows_to_f16_tile(xs + tok0 * D, sb + L::RX, mred, true, xsc);
-    float eh = 0.f;
     // the copies hold 2^e H_s and 2^e' M_s (exponents in [-120, 120])
     const int eH = sexp[((size_t)bh * N + n) * 2], eM = sexp[((size_t)bh * N + n) * 2 + 1];
     const float sH = pow2f(eH), sM = pow2f(eM);
@@ -240,6 +199,15 @@ k_bwd_rows_tc(const __grid_constant__ CUtensorMap state_map, const int *__restri
     }
     if (!mbar_wait_bounded(&bars[0], 0, kTcWaitProbes)) ok = false;
     tc::fence_after_sync();
+    bool e_loaded = false;
+    if (tid == 0 && ok) {
+        // phase A's products have read H_s and M_s: E^H and E^M into their tiles, landing
+        // while the phase-A results leave
+        mbar_arrive_expect_tx(&bars[4], 2 * 32768);
+        load_state_tile(&adj_map, srow, sm + L::MA, &bars[4]);
+        load_state_tile(&adj_map, srow + D, sm + L::MB, &bars[4]);
+        e_loaded = true;
+    }
 
     // per-token sums over the 128 rows: this thread's 16 partials -> red[t][quarter]
     auto token_sum = [&](float *part, float *dst, float scale, bool add) {
@@ -289,13 +257,12 @@ k_bwd_rows_tc(const __grid_constant__ CUtensorMap state_map, const int *__restri
         }
         token_sum(part, tokq + 2 * plane, 1.f, false);
     }
-    // phase B: the adjoints into the same tiles (the phase-A products are complete)
-    // <E^H, H_s> + <E^M, M_s> against the fp16 copies of H_s, M_s that these overwrite
-    const float sEH = mat_to_f16_tile(EH, sb + L::MA, mred, sH, &eh, nullptr);
-    const float sEM = mat_to_f16_tile(EM, sb + L::MB, mred, sM, &eh, nullptr);
-    fence_proxy_async_smem();
+    // phase B: the adjoint copies (2^e E) in the same tiles
+    const float sEH = pow2f(aexp[((size_t)bh * N + n) * 2]);
+    const float sEM = pow2f(aexp[((size_t)bh * N + n) * 2 + 1]);
+    if (!mbar_wait_bounded(&bars[4], 0, kTcWaitProbes)) ok = false;
     tc::fence_before_sync();
-    __syncthreads();
+    ok = __syncthreads_and(ok);
     tc::fence_after_sync();
     if (tid == 0 && ok) {
 #pragma unroll
@@ -341,19 +308,17 @@ k_bwd_rows_tc(const __grid_constant__ CUtensorMap state_map, const int *__restri
         }
         token_sum(part, tokq + 3 * plane, 1.f, false);
     }
-    // chunk scalars
+    // chunk scalars: hs2, and eh from the adjoint pass's two inner products
     {
         hs2 = warp_sum(hs2);
-        eh = warp_sum(eh);
-        if (lane == 0) {
-            mred[warp] = hs2;
-            mred[8 + warp] = eh;
-        }
+        if (lane == 0) mred[warp] = hs2;
         __syncthreads();
-        if (tid < 2 && ok) {
+        if (tid == 0 && ok) {
             float s = 0.f;
-            for (int w = 0; w < 8; ++w) s += mred[tid * 8 + w];
-            chq[((size_t)bh * N + n) * 2 + tid] = s;
+            for (int w = 0; w < 8; ++w) s += mred[w];
+            const size_t e = ((size_t)bh * N + n) * 2;
+            chq[e] = s;
+            chq[e + 1] = eh_part[e] + eh_part[e + 1];
         }
     }
     if (!ok && tid == 0) {
@@ -363,6 +328,7 @@ k_bwd_rows_tc(const __grid_constant__ CUtensorMap state_map, const int *__restri
         tc::commit(&bars[2]);
         mbar_wait_bounded(&bars[2], 0, kTcWaitProbes);
         mbar_wait_bounded(&bars[3], 0, kTcWaitProbes);   // the state tiles' loads
+        if (e_loaded) mbar_wait_bounded(&bars[4], 0, kTcWaitProbes);
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -511,228 +477,6 @@ k_bwd_u_tc(const __grid_constant__ CUtensorMap state_map, const int *__restrict_
     if (warp == 0) {
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, 32);
-    }
-}
-
-// ---------------------------------------------------------------------------
-// k_bwd_delta_tc: the adjoint increments of one 32-token chunk on tcgen05
-// (the work of k_bwd_delta):
-//   dE^H = -(b o Y)^T X - (e o K~)^T K~ - (sum_s b_s^2 c_s) H_start,
-//   dE^M = (b o G)^T X,      e_i = sum_{s>=i} b_s c_s w_si,
-// two 128 x 128 x 32 accumulations (operands MN-major from token-row tiles, fp16
-// with power-of-two scales; the two products of dE^H scaled alike so that they
-// share one accumulator), the H_start term added in fp32 on the way out.  The
-// increments leave through shared memory: 32 columns of every row per round in a
-// [128][32] fp32 box (128B swizzle), written by TMA stores while the next round
-// fills the other of two buffers.
-// grid (N, B*H), block 256.
-// ---------------------------------------------------------------------------
-struct BwdDeltaTcSmem {
-    static constexpr uint32_t TY = 0;            // [2][32][64] fp16: -(b o y) rows
-    static constexpr uint32_t TX = TY + 8192;    // x rows
-    static constexpr uint32_t TE = TX + 8192;    // -(e o k~) rows
-    static constexpr uint32_t TK = TE + 8192;    // k~ rows
-    static constexpr uint32_t TG = TK + 8192;    // (b o g) rows
-    static constexpr uint32_t STG0 = TY;         // output staging: 2 x [128][32] fp32 over the
-    static constexpr uint32_t STG1 = TG + 8192;  // row tiles (free after the products), and its own
-    static constexpr uint32_t ELL = STG1 + 32768;   // double[32] + double[8]
-    static constexpr uint32_t SC = ELL + 320;    // float[32] b, float[32] e, float[32] sqrt(w)
-    static constexpr uint32_t MRED = SC + 384;   // float[16]
-    static constexpr uint32_t BARS = MRED + 64;  // 2 mbarriers: products, drain
-    static constexpr uint32_t TBASE = BARS + 16;
-    static constexpr uint32_t END = TBASE + 16;
-    static constexpr size_t bytes = END + 1024;
-};
-
-// rows [32][128] of src (fp32 or bf16) times a per-row weight -> fp16 swizzled
-// [2][32][64] tile, scaled by `sc` (a power of two); the caller picks the scale from
-// the maximum that rows_absmax returns.
-template <typename Src>
-__device__ __forceinline__ float rows_absmax(const Src *__restrict__ src, const float *wrow,
-                                             float *red) {
-    const int tid = threadIdx.x, t = tid >> 3, c0 = (tid & 7) * 16;
-    const float w = wrow ? wrow[t] : 1.f;
-    float mx = 0.f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) mx = fmaxf(mx, fabsf(to_f(src[t * 128 + c0 + i]) * w));
-    return block_max256(mx, red);
-}
-template <typename Src>
-__device__ __forceinline__ void rows_store_f16(const Src *__restrict__ src, const float *wrow,
-                                               float sc, uint32_t tile) {
-    const int tid = threadIdx.x, t = tid >> 3, c0 = (tid & 7) * 16;
-    const float w = (wrow ? wrow[t] : 1.f) * sc;
-    float v[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = to_f(src[t * 128 + c0 + i]) * w;
-    const uint32_t base = tile + (uint32_t)(c0 >> 6) * (kBrC * 128u);
-    st_row8(base, (uint32_t)t, (uint32_t)(c0 & 63), v);
-    st_row8(base, (uint32_t)t, (uint32_t)((c0 & 63) + 8), v + 8);
-}
-
-__global__ void __launch_bounds__(kSimtThreads, 2)
-k_bwd_delta_tc(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ beta,
-               const float *__restrict__ gate, const __nv_bfloat16 *__restrict__ dout,
-               const __half *__restrict__ slp, const int *__restrict__ sexp,
-               const float *__restrict__ xs,
-               const float *__restrict__ ys, const float *__restrict__ cvec,
-               const __grid_constant__ CUtensorMap adj_map, int T, int N,
-               int *__restrict__ timeout_flag) {
-    // adj_map: the adjoint states [B*H*(N+1)*2*128][128] fp32, box 32 x 128, 128B swizzle;
-    // slp, sexp: the recompute's fp16 chunk-start state copies [B*H][N][2][128][128]
-    // (scaled by 2^e) and their exponents [B*H][N][2]
-    using L = BwdDeltaTcSmem;
-    constexpr int D = 128, C = kBrC;
-    extern __shared__ uint8_t smraw[];
-    uint8_t *sm = smem_align1024(smraw);
-    const uint32_t sb = smem_u32(sm);
-    double *ell = reinterpret_cast<double *>(sm + L::ELL);
-    double *wtot = ell + C;
-    float *s_b = reinterpret_cast<float *>(sm + L::SC), *s_e = s_b + C, *s_sg = s_e + C;
-    float *mred = reinterpret_cast<float *>(sm + L::MRED);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BARS);
-    uint32_t *tbase = reinterpret_cast<uint32_t *>(sm + L::TBASE);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int n = blockIdx.x, bh = blockIdx.y;
-    const size_t tok0 = (size_t)bh * T + (size_t)n * C;
-    if (tid == 0) {
-        mbar_init(&bars[0], 1);
-        mbar_init(&bars[1], 1);
-        fence_mbar_init();
-    }
-    if (warp == 0) {
-        tc::tmem_alloc(tbase, 256);
-        tc::tmem_relinquish();
-    }
-    chunk_log_prefix(beta + tok0, C, ell, wtot);
-    if (tid < C) s_sg[tid] = gate ? sqrtf(gate[tok0 + tid]) : 1.f;
-    if (tid == 0) {
-        float e = 0.f, c1 = 0.f;
-        for (int i = C - 1; i >= 0; --i) {
-            const float b = decay_exp(ell[i]);
-            const float bc = b * cvec[tok0 + i];
-            const float nxt = i + 1 < C ? decay_exp(ell[i + 1] - ell[i]) : 0.f;
-            e = fmaf(nxt, e, bc);
-            s_e[i] = e;
-            s_b[i] = b;
-            c1 = fmaf(b, bc, c1);
-        }
-        mred[15] = c1;
-    }
-    __syncthreads();
-    const float c1 = mred[15];
-    // scales: x and k~ by their maxima; y and (e k~) so that both products of dE^H
-    // carry the same overall scale S = min(sY sX, sE sK)
-    const float *xrow = xs + tok0 * D, *yrow = ys + tok0 * D;
-    const __nv_bfloat16 *krow = k + tok0 * D, *grow = dout + tok0 * D;
-    // k~ = sqrt(w) k: weight s_sg; e o k~: weight s_e * s_sg (formed below)
-    __shared__ float s_ek[kBrC];
-    if (tid < C) s_ek[tid] = s_e[tid] * s_sg[tid];
-    __syncthreads();
-    const float mX = rows_absmax(xrow, nullptr, mred);
-    const float mK = rows_absmax(krow, s_sg, mred);
-    const float mY = rows_absmax(yrow, s_b, mred);
-    const float mE = rows_absmax(krow, s_ek, mred);
-    const float mG = rows_absmax(grow, s_b, mred);
-    const float sX = inv_pow2_above(mX), sK = inv_pow2_above(mK);
-    const float sY0 = inv_pow2_above(mY), sE0 = inv_pow2_above(mE), sG = inv_pow2_above(mG);
-    const float S = fminf(sY0 * sX, sE0 * sK);
-    const float sY = S / sX, sE = S / sK;    // both <= their own limits (powers of two)
-    rows_store_f16(xrow, nullptr, sX, sb + L::TX);
-    rows_store_f16(krow, s_sg, sK, sb + L::TK);
-    rows_store_f16(yrow, s_b, -sY, sb + L::TY);
-    rows_store_f16(krow, s_ek, -sE, sb + L::TE);
-    rows_store_f16(grow, s_b, sG, sb + L::TG);
-    fence_proxy_async_smem();
-    tc::fence_before_sync();
-    __syncthreads();
-    tc::fence_after_sync();
-    const uint32_t tmem = *tbase;
-    constexpr uint32_t ID = tc::idesc_f16(128, 128, true, true);
-    auto desc = [&](uint32_t t, int kk) { return tc::sdesc(t + kk * 2048, C * 128, 1024); };
-    if (tid == 0) {
-#pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk) {
-            tc::mma_f16(tmem + 0, desc(sb + L::TY, kk), desc(sb + L::TX, kk), ID, kk > 0);
-            tc::mma_f16(tmem + 0, desc(sb + L::TE, kk), desc(sb + L::TK, kk), ID, true);
-            tc::mma_f16(tmem + 128, desc(sb + L::TG, kk), desc(sb + L::TX, kk), ID, kk > 0);
-        }
-        tc::commit(&bars[0]);
-    }
-    bool ok = mbar_wait_bounded(&bars[0], 0, kTcWaitProbes);
-    tc::fence_after_sync();
-    ok = __syncthreads_and(ok);
-    // row p = TMEM lane of this thread; round (m, j) covers columns 64 wg + 32 j .. + 31
-    // of dE^H (m = 0, with the H_start term) or dE^M (m = 1)
-    const int quarter = warp & 3, wg = warp >> 2, p = quarter * 32 + lane;
-    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
-    // row p of H_start from its fp16 copy (2^e H_start), the scale undone below
-    const __half *Hst = slp + ((size_t)bh * N + n) * 2 * D * D + (size_t)p * D;
-    const float hsc = pow2f(-sexp[((size_t)bh * N + n) * 2]);
-    const int orow = (int)(((size_t)bh * (N + 1) + n) * 2 * D);
-    const float uH = 1.f / S, uM = 1.f / (sG * sX);
-#pragma unroll 1
-    for (int round = 0; round < 4 && ok; ++round) {
-        const int m = round >> 1, col = wg * 64 + (round & 1) * 32;
-        // buffer round % 2; the stores that last read it (round - 2) were waited for
-        // before the previous round's barrier
-        const uint32_t rowb = sb + ((round & 1) ? L::STG1 : L::STG0) + wg * 16384 + p * 128;
-        float a[32];
-        tc::tmem_ld16(tl + m * 128 + col, a);
-        tc::tmem_ld16(tl + m * 128 + col + 16, a + 16);
-        float4 h[8];
-        if (m == 0) {
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const uint4 u = *reinterpret_cast<const uint4 *>(Hst + col + 8 * c);
-                const float2 f0 = __half22float2(*reinterpret_cast<const __half2 *>(&u.x));
-                const float2 f1 = __half22float2(*reinterpret_cast<const __half2 *>(&u.y));
-                const float2 f2 = __half22float2(*reinterpret_cast<const __half2 *>(&u.z));
-                const float2 f3 = __half22float2(*reinterpret_cast<const __half2 *>(&u.w));
-                h[2 * c] = make_float4(f0.x * hsc, f0.y * hsc, f1.x * hsc, f1.y * hsc);
-                h[2 * c + 1] = make_float4(f2.x * hsc, f2.y * hsc, f3.x * hsc, f3.y * hsc);
-            }
-        }
-        tc::tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            float o0, o1, o2, o3;
-            if (m == 0) {
-                o0 = fmaf(-c1, h[c].x, a[4 * c] * uH);
-                o1 = fmaf(-c1, h[c].y, a[4 * c + 1] * uH);
-                o2 = fmaf(-c1, h[c].z, a[4 * c + 2] * uH);
-                o3 = fmaf(-c1, h[c].w, a[4 * c + 3] * uH);
-            } else {
-                o0 = a[4 * c] * uM;
-                o1 = a[4 * c + 1] * uM;
-                o2 = a[4 * c + 2] * uM;
-                o3 = a[4 * c + 3] * uM;
-            }
-            st_shared_v4(rowb + ((c ^ p) & 7) * 16, __float_as_uint(o0), __float_as_uint(o1),
-                         __float_as_uint(o2), __float_as_uint(o3));
-        }
-        fence_proxy_async_smem();
-        if (tid == 0) tc::bulk_wait_read0();   // the previous round's stores have read their buffer
-        __syncthreads();
-        if (tid == 0) {
-            const uint32_t buf = (round & 1) ? L::STG1 : L::STG0;
-            const int x = (round & 1) * 32;
-            tc::tma_store_2d(&adj_map, x, orow + m * D, sm + buf);
-            tc::tma_store_2d(&adj_map, 64 + x, orow + m * D, sm + buf + 16384);
-            tc::bulk_commit();
-        }
-    }
-    if (tid == 0) tc::bulk_wait0();
-    if (!ok && tid == 0) {
-        atomicExch(timeout_flag, 1);
-        tc::commit(&bars[1]);
-        mbar_wait_bounded(&bars[1], 0, kTcWaitProbes);
-    }
-    tc::fence_before_sync();
-    __syncthreads();
-    if (warp == 0) {
-        tc::fence_after_sync();
-        tc::tmem_dealloc(tmem, 256);
     }
 }
 

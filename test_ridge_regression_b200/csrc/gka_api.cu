@@ -15,6 +15,7 @@
 #include <cudaTypedefs.h>
 
 #include "backward_simt.cuh"
+#include "adjoint_tc.cuh"
 #include "backward_tc.cuh"
 #include "chunk_simt.cuh"
 #include "common.cuh"
@@ -538,52 +539,59 @@ static int backward_simt(const Tin *q, const Tin *k, const Tin *v, const float *
             if (int rc = check_launch()) return rc;
         }
     }
-    // adjoint chunk increments and their reverse scan
-    bool delta_done = false;
+    // the adjoint states: bf16, D = 128, C = 32: the increments and the reverse scan in
+    // one tensor-core pass per (head, matrix), written as fp16 copies (scaled by 2^e)
+    // with their exponents and inner products, in the adjoint region (half its size
+    // holds the copies); otherwise per-chunk increments and a reverse scan in fp32
+    __half *alp = reinterpret_cast<__half *>(adj);
+    int *aexp = reinterpret_cast<int *>(reinterpret_cast<char *>(adj) +
+                                        round256(sizeof(__half) * BH * (size_t)N * 2 * D * D));
+    float *ehp = reinterpret_cast<float *>(reinterpret_cast<char *>(aexp) +
+                                           round256(sizeof(int) * BH * (size_t)N * 2));
+    bool rows_done = false;
     if constexpr (std::is_same<Tin, __nv_bfloat16>::value && D == 128) {
         if (tc_done && C == kBrC) {
-            // bf16, D = 128: the adjoint increments as fp16 MMAs
             int *flag = nullptr;
             if (int rc = timeout_flag_ptr(&flag)) return rc;
-            CUtensorMap adj_map;
-            if (int rc = rows128_map(&adj_map, adj, (uint64_t)BH * (N + 1) * 2 * D,
-                                     CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 32, 128))
+            AdjMaps am;
+            const uint64_t ntok = (uint64_t)BH * T;
+            if (int rc = rows128_map(&am.y, ys, ntok, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 32, 32)) return rc;
+            if (int rc = rows128_map(&am.x, xs, ntok, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 32, 32)) return rc;
+            if (int rc = rows128_map(&am.k, k, ntok, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 64, 32)) return rc;
+            if (int rc = rows128_map(&am.g, dout, ntok, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 64, 32))
                 return rc;
-            if ((e = set_smem(k_bwd_delta_tc, BwdDeltaTcSmem::bytes)) != cudaSuccess)
-                return cuda_fail(e);
-            { ProfScope ps(GKA_KERNEL_BWD_DELTA, s);
-            k_bwd_delta_tc<<<dim3(N, BH), kSimtThreads, BwdDeltaTcSmem::bytes, s>>>(
-                k, beta, gate, dout, slp32, sexp32, xs, ys, cvec, adj_map, T, N, flag); }
+            am.state = state_map;
+            const uint64_t crows = (uint64_t)BH * N * 2 * D;
+            if (int rc = rows128_map(&am.out, alp, crows, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 64, 128))
+                return rc;
+            CUtensorMap adj_map;   // the copies, boxes 64 x 64, for the row kernel's loads
+            if (int rc = rows128_map(&adj_map, alp, crows, CU_TENSOR_MAP_DATA_TYPE_FLOAT16)) return rc;
+            if ((e = set_smem(k_adjoint_pass_tc, AdjSmem::bytes)) != cudaSuccess) return cuda_fail(e);
+            { ProfScope ps(GKA_KERNEL_ADJOINT_SCAN, s);
+            k_adjoint_pass_tc<<<dim3(2, BH), kAdjThreads, AdjSmem::bytes, s>>>(
+                am, beta, gate, cvec, sexp32, aexp, ehp, T, N, flag); }
             if (int rc = check_launch()) return rc;
-            delta_done = true;
+            // the chunk rows against H_s, M_s and the adjoints, as fp16 MMAs
+            if ((e = set_smem(k_bwd_rows_tc, BwdRowsTcSmem::bytes)) != cudaSuccess)
+                return cuda_fail(e);
+            { ProfScope ps(GKA_KERNEL_BWD_ROWS, s);
+            k_bwd_rows_tc<<<dim3(N, BH), kSimtThreads, BwdRowsTcSmem::bytes, s>>>(
+                state_map, sexp32, adj_map, alp, aexp, ehp, k, v, dout, xs, ys, rows, tokq, chq,
+                T, N, flag); }
+            if (int rc = check_launch()) return rc;
+            rows_done = true;
         }
     }
-    if (!delta_done) {
+    if (!rows_done) {
         const size_t sm_bd = sizeof(float) * 5 * (size_t)C * D;
         if ((e = set_smem(k_bwd_delta<Tin, D>, sm_bd)) != cudaSuccess) return cuda_fail(e);
         { ProfScope ps(GKA_KERNEL_BWD_DELTA, s);
         k_bwd_delta<Tin, D><<<dim3(N, BH), kSimtThreads, sm_bd, s>>>(k, beta, gate, dout, states,
                                                                     xs, ys, cvec, adj, T, N, C); }
         if (int rc = check_launch()) return rc;
-    }
-    { ProfScope ps(GKA_KERNEL_ADJOINT_SCAN, s);
-    k_adjoint_scan<<<dim3((DD2 / 4 + 255) / 256, BH), 256, 0, s>>>(adj, decay, N, DD2); }
-    if (int rc = check_launch()) return rc;
-    // the chunk rows against H_s, M_s and the adjoints
-    bool rows_done = false;
-    if constexpr (std::is_same<Tin, __nv_bfloat16>::value && D == 128) {
-        if (tc_done && C == kBrC) {
-            // bf16, D = 128: the row products as fp16 MMAs
-            int *flag = nullptr;
-            if (int rc = timeout_flag_ptr(&flag)) return rc;
-            if ((e = set_smem(k_bwd_rows_tc, BwdRowsTcSmem::bytes)) != cudaSuccess)
-                return cuda_fail(e);
-            { ProfScope ps(GKA_KERNEL_BWD_ROWS, s);
-            k_bwd_rows_tc<<<dim3(N, BH), kSimtThreads, BwdRowsTcSmem::bytes, s>>>(
-                state_map, sexp32, k, v, dout, adj, xs, ys, rows, tokq, chq, T, N, flag); }
-            if (int rc = check_launch()) return rc;
-            rows_done = true;
-        }
+        { ProfScope ps(GKA_KERNEL_ADJOINT_SCAN, s);
+        k_adjoint_scan<<<dim3((DD2 / 4 + 255) / 256, BH), 256, 0, s>>>(adj, decay, N, DD2); }
+        if (int rc = check_launch()) return rc;
     }
     if (rows_done) {
         // the tensor-core row products ran
