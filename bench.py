@@ -632,19 +632,29 @@ def bench_backward(args, w, dev, qd, kd, vd, bd, flush, rank, world, barrier, pe
     dom = max(own or per_kernel, key=(own or per_kernel).get)
     peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
     total_fl = sum(fl[n] for n in per_kernel if n in fl) * head_tok
-    tc_rows = w.dtype == torch.bfloat16 and w.D == 128 and BWD_CHUNK == 32 and w.T % 64 == 0
-    if dom == "bwd_rows" and tc_rows:
-        # the row products run as fp16 MMAs; what they must move bounds them: per chunk the
-        # fp16 copies of H_s and M_s and the two fp32 adjoints, the k, v, g (bf16) and x, y
-        # (fp32) rows in, R1..R4 and the per-token scalars out
+    tc_path = w.dtype == torch.bfloat16 and w.D == 128 and BWD_CHUNK == 32 and w.T % 64 == 0
+    # the tensor-core kernels of the backward are bound by what they must move
+    hbm = {}
+    if tc_path:
         D, C = w.D, BWD_CHUNK
-        per_tok = (2 * D * D * 2 + 2 * D * D * 4) / C + 3 * D * 2 + 2 * D * 4 + 4 * D * 4 + 4 * 4
-        byts = per_tok * head_tok
-        ach = byts / (per_kernel[dom] / 1e3) / 1e9
-        roof = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": ach / peaks["hbm_gbs"],
-                "traffic": traffic_of("bwd_rows_tc", w.name),
-                "peak_source": "measured copy bandwidth", "algorithmic_per_step": byts}
+        # row products: per chunk the fp16 copies of H_s, M_s, E^H, E^M; the k, v, g
+        # (bf16) and x, y (fp32) rows in, R1..R4 and the per-token scalars out
+        rows_tok = 4 * D * D * 2 / C + 3 * D * 2 + 2 * D * 4 + 4 * D * 4 + 4 * 4
+        # adjoint pass: per chunk the two state copies in and the two adjoint copies out
+        # (fp16); the y, x (fp32) and k, g (bf16) rows, beta and c in
+        adj_tok = 4 * D * D * 2 / C + 2 * D * 4 + 2 * D * 2 + 2 * 4
+        for name, per_tok, key in (("bwd_rows", rows_tok, "bwd_rows_tc"),
+                                   ("adjoint_scan", adj_tok, "adjoint_pass_tc")):
+            if name not in per_kernel:
+                continue
+            byts = per_tok * head_tok
+            ach = byts / (per_kernel[name] / 1e3) / 1e9
+            hbm[name] = {"bound": "hbm", "kernel": name, "achieved": ach,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"],
+                         "traffic": traffic_of(key, w.name),
+                         "peak_source": "measured copy bandwidth", "algorithmic_per_step": byts}
+    if dom in hbm:
+        roof = hbm[dom]
     else:
         achieved = fl.get(dom, 0) * head_tok / (per_kernel[dom] / 1e3) / 1e12
         roof = {"bound": "alu", "kernel": dom, "achieved": achieved, "peak": peak,
@@ -656,6 +666,7 @@ def bench_backward(args, w, dev, qd, kd, vd, bd, flush, rank, world, barrier, pe
             "kernels_ms_per_step": per_kernel,
             "gpu_launches": sum(n for _, n in kt.values()),
             "roofline": roof,
+            "hbm_rooflines": hbm,
             "step_frac_of_fp32_peak": total_fl / (total_ms / steps / 1e3) / 1e12 / peak}
 
 
