@@ -25,6 +25,7 @@
 #include "common.cuh"
 #include "ptx.cuh"
 #include "solve_tc.cuh"
+#include "state_tc.cuh"
 #include "tcgen05.cuh"
 
 namespace gka {
@@ -346,22 +347,28 @@ namespace gka {
 // k_bwd_u_tc: the right-hand side of the adjoint solve for one 32-token chunk
 // (bf16 inputs, D = 128; the tensor-core solve then solves for y on it):
 //   u_t = M_t^T g_t = b_t M_s^T g_t + sum_{i<=t} w_ti k~_i (v~_i . g_t),
-// M_s^T G^T as eight 128 x 32 x 16 fp16 MMAs (M_s and the g rows converted with
-// power-of-two scales, as in k_bwd_rows_tc) while the CUDA cores form the
-// intra-chunk matrix P[t][i] = w_ti (v~_i . g_t); thread (row c, 16 tokens) adds
-// the two parts and writes u in bf16 (the precision the tensor-core solve reads).
+// k~ = sqrt(w) k, v~ = sqrt(w) v the written keys and values.  Three fp16 MMA groups
+// (operands with power-of-two scales, fp32 accumulators), row c = TMEM lane:
+//   Q = G V~^T           (A = the 128-row operand region [G; V~; K~; -], only its
+//                         first 32 lanes are used; B = the V~ rows),
+//   A1 = M_s^T G^T       (the state pass's fp16 copy of M_s, MN-major),
+//   A2 = K~^T P^T        after one warp forms P[t][i] = w_ti Q[t][i] (i <= t) in fp16,
+// then u[t][c] = b_t A1[c][t] + A2[c][t], written in bf16 (the precision the
+// tensor-core solve reads).  The rows arrive by bulk copies, M_s by TMA.
 // grid (N, B*H), block 256.
 // ---------------------------------------------------------------------------
 struct BwdUTcSmem {
-    static constexpr int KP = 132;                 // fp32 row pitch of k~, v~
     static constexpr uint32_t MB = 0;              // [2][128][64] fp16 M_s
-    static constexpr uint32_t RG = MB + 32768;     // [2][32][64] fp16 g rows
-    static constexpr uint32_t KH = RG + 8192;      // float[32][KP] k~
-    static constexpr uint32_t VH = KH + 32 * KP * 4;   // float[32][KP] v~
-    static constexpr uint32_t PM = VH + 32 * KP * 4;   // float[32][33] P
-    static constexpr uint32_t GR = PM + 32 * 33 * 4;   // bf16 [32][128] g
-    static constexpr uint32_t MRED = GR + 8192;    // float[16]
-    static constexpr uint32_t BARS = MRED + 64;    // 3 mbarriers: product, drain, M_s
+    static constexpr uint32_t AT = MB + 32768;     // [2][128][64] fp16: G, V~, K~ rows (32 each)
+    static constexpr uint32_t PT = AT + 32768;     // [32][64] fp16 P (K-major, 32 columns used)
+    static constexpr uint32_t RK = PT + 4096;      // bf16 [32][128] k rows
+    static constexpr uint32_t RV = RK + 8192;      // v rows
+    static constexpr uint32_t RG = RV + 8192;      // g rows
+    static constexpr uint32_t SC = RG + 8192;      // float[32] beta, float[32] gate
+    static constexpr uint32_t ELL = SC + 256;      // double[32] + double[8]
+    static constexpr uint32_t SB = ELL + 320;      // float[32] b, float[32] sqrt(gate)
+    static constexpr uint32_t MRED = SB + 256;     // float[8][4] maxima, float scale of P
+    static constexpr uint32_t BARS = MRED + 144;   // 4 mbarriers: loads, Q and A1, A2, drain
     static constexpr uint32_t TBASE = BARS + 32;
     static constexpr uint32_t END = TBASE + 16;
     static constexpr size_t bytes = END + 1024;    // + alignment slack
@@ -374,109 +381,205 @@ k_bwd_u_tc(const __grid_constant__ CUtensorMap state_map, const int *__restrict_
            const __nv_bfloat16 *__restrict__ dout,
            __nv_bfloat16 *__restrict__ u_out, int T, int N, int *__restrict__ timeout_flag) {
     using L = BwdUTcSmem;
-    constexpr int D = 128, C = kBrC, KP = L::KP, CP = C + 1;
+    constexpr int D = 128, C = kBrC;
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = smem_align1024(smraw);
     const uint32_t sb = smem_u32(sm);
-    float *Kh = reinterpret_cast<float *>(sm + L::KH);
-    float *Vh = reinterpret_cast<float *>(sm + L::VH);
-    float *Pm = reinterpret_cast<float *>(sm + L::PM);
-    __nv_bfloat16 *Gr = reinterpret_cast<__nv_bfloat16 *>(sm + L::GR);
+    float *s_beta = reinterpret_cast<float *>(sm + L::SC), *s_gate = s_beta + 32;
+    double *ell = reinterpret_cast<double *>(sm + L::ELL), *wtot = ell + C;
+    float *s_b = reinterpret_cast<float *>(sm + L::SB), *s_sg = s_b + 32;
     float *mred = reinterpret_cast<float *>(sm + L::MRED);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BARS);
     uint32_t *tbase = reinterpret_cast<uint32_t *>(sm + L::TBASE);
-    __shared__ double ell[C], wtot[kSimtThreads / 32];
-    __shared__ float s_b[C];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n = blockIdx.x, bh = blockIdx.y;
     const size_t tok0 = (size_t)bh * T + (size_t)n * C;
     const int srow = (int)(((size_t)bh * N + n) * 2 * D);   // H_s row in the state map; M_s follows
 
     if (tid == 0) {
-        mbar_init(&bars[0], 1);
-        mbar_init(&bars[1], 1);
-        mbar_init(&bars[2], 1);
+        for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
-        // M_s as an fp16 tile (the state pass's copy, 2^e M_s), read while the rows convert
-        mbar_arrive_expect_tx(&bars[2], 32768);
-        load_state_tile(&state_map, srow + D, sm + L::MB, &bars[2]);
+        mbar_arrive_expect_tx(&bars[0], 32768 + 3 * 8192 + 128 + (gate ? 128 : 0));
+        load_state_tile(&state_map, srow + D, sm + L::MB, &bars[0]);
+        bulk_g2s(sm + L::RK, k + tok0 * D, 8192, &bars[0]);
+        bulk_g2s(sm + L::RV, v + tok0 * D, 8192, &bars[0]);
+        bulk_g2s(sm + L::RG, dout + tok0 * D, 8192, &bars[0]);
+        bulk_g2s(s_beta, beta + tok0, 128, &bars[0]);
+        if (gate) bulk_g2s(s_gate, gate + tok0, 128, &bars[0]);
     }
     if (warp == 0) {
-        tc::tmem_alloc(tbase, 32);
+        tc::tmem_alloc(tbase, 128);
         tc::tmem_relinquish();
     }
-    chunk_log_prefix(beta + tok0, C, ell, wtot);
-    if (tid < C) s_b[tid] = decay_exp(ell[tid]);
-    for (int e = tid; e < C * D; e += kSimtThreads) {
-        const int t = e / D, d = e % D;
-        const size_t g = tok0 * D + e;
-        const float sg = gate ? sqrtf(gate[tok0 + t]) : 1.f;
-        Kh[t * KP + d] = __bfloat162float(k[g]) * sg;
-        Vh[t * KP + d] = __bfloat162float(v[g]) * sg;
-        Gr[e] = dout[g];
+    __syncthreads();
+    bool ok = mbar_wait_bounded(&bars[0], 0, kTcWaitProbes);
+    chunk_log_prefix(s_beta, C, ell, wtot);
+    if (tid < C) {
+        s_b[tid] = decay_exp(ell[tid]);
+        s_sg[tid] = gate ? sqrtf(s_gate[tid]) : 1.f;
     }
-    const float sG = rows_to_f16_tile(dout + tok0 * D, sb + L::RG, mred, false, nullptr);
+    __syncthreads();
+    // the operand rows: item (token t, 8 columns 8j..) of each of G, V~, K~
+    float gv[2][8], vv[2][8], kv[2][8];
+    float mg = 0.f, mv = 0.f, mk = 0.f;
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const int item = tid + r * kSimtThreads, t = item >> 4, j = item & 15;
+        const uint32_t off = (uint32_t)(t * 256 + j * 16);
+        const uint4 ug = *reinterpret_cast<const uint4 *>(sm + L::RG + off);
+        const uint4 uv = *reinterpret_cast<const uint4 *>(sm + L::RV + off);
+        const uint4 uk = *reinterpret_cast<const uint4 *>(sm + L::RK + off);
+        const uint32_t wg4[4] = {ug.x, ug.y, ug.z, ug.w}, wv4[4] = {uv.x, uv.y, uv.z, uv.w},
+                       wk4[4] = {uk.x, uk.y, uk.z, uk.w};
+        const float sg = s_sg[t];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            gv[r][2 * q] = bf16_lo(wg4[q]);
+            gv[r][2 * q + 1] = bf16_hi(wg4[q]);
+            vv[r][2 * q] = bf16_lo(wv4[q]) * sg;
+            vv[r][2 * q + 1] = bf16_hi(wv4[q]) * sg;
+            kv[r][2 * q] = bf16_lo(wk4[q]) * sg;
+            kv[r][2 * q + 1] = bf16_hi(wk4[q]) * sg;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            mg = fmaxf(mg, fabsf(gv[r][e]));
+            mv = fmaxf(mv, fabsf(vv[r][e]));
+            mk = fmaxf(mk, fabsf(kv[r][e]));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        mg = fmaxf(mg, __shfl_xor_sync(0xffffffffu, mg, o));
+        mv = fmaxf(mv, __shfl_xor_sync(0xffffffffu, mv, o));
+        mk = fmaxf(mk, __shfl_xor_sync(0xffffffffu, mk, o));
+    }
+    if (lane == 0) {
+        mred[warp * 4] = mg;
+        mred[warp * 4 + 1] = mv;
+        mred[warp * 4 + 2] = mk;
+    }
+    __syncthreads();
+    mg = mv = mk = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+        mg = fmaxf(mg, mred[w * 4]);
+        mv = fmaxf(mv, mred[w * 4 + 1]);
+        mk = fmaxf(mk, mred[w * 4 + 2]);
+    }
+    const float sG = inv_pow2_above(mg), sV = inv_pow2_above(mv), sK = inv_pow2_above(mk);
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const int item = tid + r * kSimtThreads, t = item >> 4, j = item & 15;
+        // row t of the 32-row block at `row0` of the 128-row region, columns 8j..8j+7
+        auto put = [&](int row0, const float *x, float sc) {
+            const uint32_t row = (uint32_t)(row0 + t);
+            st_shared_v4(sb + L::AT + (uint32_t)(j >> 3) * 16384u + row * 128u +
+                             (((uint32_t)j ^ row) & 7u) * 16u,
+                         pack_f16(x[0] * sc, x[1] * sc), pack_f16(x[2] * sc, x[3] * sc),
+                         pack_f16(x[4] * sc, x[5] * sc), pack_f16(x[6] * sc, x[7] * sc));
+        };
+        put(0, gv[r], sG);
+        put(32, vv[r], sV);
+        put(64, kv[r], sK);
+    }
     const float sM = pow2f(sexp[((size_t)bh * N + n) * 2 + 1]);
-    bool ok = mbar_wait_bounded(&bars[2], 0, kTcWaitProbes);
     fence_proxy_async_smem();
     tc::fence_before_sync();
-    __syncthreads();
+    ok = __syncthreads_and(ok);
     tc::fence_after_sync();
     const uint32_t tmem = *tbase;
+    // K-major operand rows at `row0` of the region (K = d in two 64-column halves)
+    auto kdesc = [&](int row0, int kk) {
+        return tc::sdesc(sb + L::AT + (uint32_t)row0 * 128u + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+    };
     if (tid == 0) {
-        constexpr uint32_t ID_T = tc::idesc_f16(128, C, true, false);   // A = M_s^T (MN-major)
         if (ok) {
+            constexpr uint32_t ID_KK = tc::idesc_f16(128, C, false, false);
+            constexpr uint32_t ID_TK = tc::idesc_f16(128, C, true, false);   // A = M_s^T (MN-major)
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-                tc::mma_f16(tmem, tc::sdesc(sb + L::MB + kk * 2048, 16384, 1024),
-                            tc::sdesc(sb + L::RG + (kk >> 2) * (C * 128) + (kk & 3) * 32, 16, 1024),
-                            ID_T, kk > 0);
-        }
-        tc::commit(&bars[0]);
-    }
-    // P[t][i] = w_ti (v~_i . g_t), i <= t, while the product runs
-    for (int e = tid; e < C * C; e += kSimtThreads) {
-        const int t = e / C, i = e % C;
-        float acc = 0.f;
-        if (i <= t) {
-            for (int d = 0; d < D; d += 4) {
-                const float4 vv = *reinterpret_cast<const float4 *>(Vh + i * KP + d);
-                const __nv_bfloat162 g01 = *reinterpret_cast<const __nv_bfloat162 *>(Gr + t * D + d);
-                const __nv_bfloat162 g23 = *reinterpret_cast<const __nv_bfloat162 *>(Gr + t * D + d + 2);
-                acc = fmaf(vv.x, __low2float(g01), fmaf(vv.y, __high2float(g01),
-                      fmaf(vv.z, __low2float(g23), fmaf(vv.w, __high2float(g23), acc))));
+            for (int kk = 0; kk < 8; ++kk) {
+                tc::mma_f16(tmem, kdesc(0, kk), kdesc(32, kk), ID_KK, kk > 0);
+                tc::mma_f16(tmem + 32, tc::sdesc(sb + L::MB + kk * 2048, 16384, 1024), kdesc(0, kk),
+                            ID_TK, kk > 0);
             }
-            acc *= decay_exp(ell[t] - ell[i]);
         }
-        Pm[t * CP + i] = acc;
+        tc::commit(&bars[1]);
     }
-    __syncthreads();
-    if (!mbar_wait_bounded(&bars[0], 0, kTcWaitProbes)) ok = false;
+    if (warp == 0) {
+        // P[t][i] = w_ti Q[t][i] for i <= t (t = lane), in fp16 with one power-of-two scale
+        if (!mbar_wait_bounded(&bars[1], 0, kTcWaitProbes)) ok = false;
+        tc::fence_after_sync();
+        float q[32];
+        tc::tmem_ld16(tmem, q);
+        tc::tmem_ld16(tmem + 16, q + 16);
+        tc::tmem_wait_ld();
+        const int t = lane;
+        const float uq = 1.f / (sG * sV);
+        const double lt = ell[t];
+        float mp = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            q[i] = i <= t ? q[i] * uq * decay_exp(lt - ell[i]) : 0.f;
+            mp = fmaxf(mp, fabsf(q[i]));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mp = fmaxf(mp, __shfl_xor_sync(0xffffffffu, mp, o));
+        const float sP = inv_pow2_above(mp);
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            st_shared_v4(sb + L::PT + (uint32_t)t * 128u + (uint32_t)((c ^ t) & 7) * 16u,
+                         pack_f16(q[8 * c] * sP, q[8 * c + 1] * sP),
+                         pack_f16(q[8 * c + 2] * sP, q[8 * c + 3] * sP),
+                         pack_f16(q[8 * c + 4] * sP, q[8 * c + 5] * sP),
+                         pack_f16(q[8 * c + 6] * sP, q[8 * c + 7] * sP));
+        if (lane == 0) mred[32] = sP;
+        fence_proxy_async_smem();
+        tc::fence_before_sync();
+        ok = __all_sync(0xffffffffu, ok);
+        __syncwarp();
+        if (lane == 0) {
+            tc::fence_after_sync();
+            if (ok) {
+                // A2 = K~^T P^T: A MN-major (rows i of K~, the two column halves 16384 apart)
+                constexpr uint32_t ID_TK = tc::idesc_f16(128, C, true, false);
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
+                    tc::mma_f16(tmem + 64, tc::sdesc(sb + L::AT + 64 * 128 + kk * 2048, 16384, 1024),
+                                tc::sdesc(sb + L::PT + kk * 32, 16, 1024), ID_TK, kk > 0);
+            }
+            tc::commit(&bars[2]);
+        }
+        __syncwarp();
+    }
+    ok = __syncthreads_and(ok);
+    if (!mbar_wait_bounded(&bars[2], 0, kTcWaitProbes)) ok = false;
     tc::fence_after_sync();
     // thread (row c = TMEM lane, tokens 16 wg .. 16 wg + 15)
     const int quarter = warp & 3, wg = warp >> 2, c = quarter * 32 + lane;
-    float acc[16];
-    tc::tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(wg * 16), acc);
+    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(wg * 16);
+    float a1[16], a2[16];
+    tc::tmem_ld16(tl + 32, a1);
+    tc::tmem_ld16(tl + 64, a2);
     tc::tmem_wait_ld();
-    const float um = 1.f / (sM * sG);
+    const float u1 = 1.f / (sM * sG), u2 = 1.f / (sK * mred[32]);
 #pragma unroll
     for (int u = 0; u < 16; ++u) {
         const int t = wg * 16 + u;
-        float x = acc[u] * um * s_b[t];
-        for (int i = 0; i <= t; ++i) x = fmaf(Pm[t * CP + i], Kh[i * KP + c], x);
+        const float x = fmaf(a1[u] * u1, s_b[t], a2[u] * u2);
         if (ok) u_out[(tok0 + t) * D + c] = __float2bfloat16_rn(x);
     }
     if (!ok && tid == 0) {
         atomicExch(timeout_flag, 1);
-        tc::commit(&bars[1]);
-        mbar_wait_bounded(&bars[1], 0, kTcWaitProbes);
-        mbar_wait_bounded(&bars[2], 0, kTcWaitProbes);   // the M_s tile's loads
+        tc::commit(&bars[3]);
+        mbar_wait_bounded(&bars[3], 0, kTcWaitProbes);
+        mbar_wait_bounded(&bars[0], 0, kTcWaitProbes);   // the loads
     }
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 0) {
         tc::fence_after_sync();
-        tc::tmem_dealloc(tmem, 32);
+        tc::tmem_dealloc(tmem, 128);
     }
 }
 
