@@ -17,6 +17,7 @@
 #include "backward_simt.cuh"
 #include "adjoint_tc.cuh"
 #include "backward_tc.cuh"
+#include "grads_tc.cuh"
 #include "chunk_simt.cuh"
 #include "common.cuh"
 #include "decode.cuh"
@@ -610,6 +611,20 @@ static int backward_simt(const Tin *q, const Tin *k, const Tin *v, const float *
     }
     if (int rc = check_launch()) return rc;
     // gradients
+    if constexpr (std::is_same<Tin, __nv_bfloat16>::value && D == 128) {
+        if (rows_done) {
+            // bf16, D = 128, C = 32: the dot matrices and the row outputs as fp16 MMAs
+            int *flag = nullptr;
+            if (int rc = timeout_flag_ptr(&flag)) return rc;
+            if ((e = set_smem(k_bwd_grads_tc, BwdGradTcSmem::bytes)) != cudaSuccess)
+                return cuda_fail(e);
+            { ProfScope ps(GKA_KERNEL_BWD_GRADS, s);
+            k_bwd_grads_tc<<<dim3(N, BH), kSimtThreads, BwdGradTcSmem::bytes, s>>>(
+                k, v, beta, gate, dout, xs, ys, cvec, rows, tokq, chq, dk, dv, dbeta, dgate, T, N,
+                flag); }
+            return check_launch();
+        }
+    }
     if (C == 16) {
         constexpr size_t sm_gr = BwdGradSmem<D, 16>::bytes;
         if ((e = set_smem(k_bwd_grads<Tin, D, 16>, sm_gr)) != cudaSuccess) return cuda_fail(e);
