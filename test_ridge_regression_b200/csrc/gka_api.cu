@@ -334,20 +334,37 @@ static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
         if (int rc = check_launch()) return rc;
     }
 
+    // The solve after the state pass is launched as its programmatic dependent: its
+    // input loads, barriers and TMEM allocation overlap the pass, and it waits for the
+    // pass (griddepcontrol.wait) before reading the state copies and decays.  With
+    // solve_only the kernel before it may have written q, which the solve reads before
+    // that wait, so it is launched in plain stream order.
+    auto launch_solve = [&](auto kern, size_t smem) -> cudaError_t {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(N, BH);
+        cfg.blockDim = dim3(kSolveThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = solve_only ? 0 : 1;
+        return cudaLaunchKernelEx(&cfg, kern, maps, q, gate, (const float *)tokdec, plane, norms,
+                                  (const int *)sexp, o, x_out, T, N, C, P, flag);
+    };
     if (C == 64) {
         // one CTA per 64-token chunk
         auto kern = x_out ? k_chunk_solve_tc<64, 64, true> : k_chunk_solve_tc<64, 64, false>;
         if ((e = set_smem(kern, TcSmem<64, 64>::bytes)) != cudaSuccess) return cuda_fail(e);
         ProfScope ps(GKA_KERNEL_CHUNK_SOLVE_TC, s);
-        kern<<<dim3(N, BH), kSolveThreads, TcSmem<64, 64>::bytes, s>>>(
-            maps, q, gate, tokdec, plane, norms, sexp, o, x_out, T, N, C, P, flag);
+        if ((e = launch_solve(kern, TcSmem<64, 64>::bytes)) != cudaSuccess) return cuda_fail(e);
     } else {
         // one CTA per 128-token chunk (N = 128 MMAs)
         auto kern = x_out ? k_chunk_solve_tc<128, 128, true> : k_chunk_solve_tc<128, 128, false>;
         if ((e = set_smem(kern, TcSmem<128, 128>::bytes)) != cudaSuccess) return cuda_fail(e);
         ProfScope ps(GKA_KERNEL_CHUNK_SOLVE_TC, s);
-        kern<<<dim3(N, BH), kSolveThreads, TcSmem<128, 128>::bytes, s>>>(
-            maps, q, gate, tokdec, plane, norms, sexp, o, x_out, T, N, C, P, flag);
+        if ((e = launch_solve(kern, TcSmem<128, 128>::bytes)) != cudaSuccess) return cuda_fail(e);
     }
     if (int rc = check_launch()) return rc;
     return GKA_OK;

@@ -119,6 +119,18 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
         : "memory");
 }
 
+// Programmatic dependent launch.  griddep_launch_dependents: this CTA lets the grid
+// launched after it on the stream (with programmatic stream serialization) begin;
+// griddep_wait: waits until the grids this one depends on have completed and their
+// writes are visible (returns at once when the grid was launched without that
+// dependency).
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // Asks L2 to fetch `bytes` from global memory at src (16-byte aligned, a multiple
 // of 16 bytes) without waiting for it and without touching shared memory.
 __device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {

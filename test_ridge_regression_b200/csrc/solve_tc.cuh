@@ -326,18 +326,14 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     }
     __syncthreads();
     if (tid == 0) {
+        // the inputs first; the state pass's outputs (state copy, decays) after the wait
+        // for it (with programmatic dependent launch this set-up overlaps that pass)
         mbar_arrive_expect_tx(bar_load, 32768 + MG * 256 + TOK * kTcD * 2 + 16 * MG);
-        for (int h = 0; h < 2; ++h) {
-            for (int rb = 0; rb < 2; ++rb)
-                tc::tma_load_2d(sm + L::HM + h * 16384 + rb * 8192, &maps.state, h * 64,
-                                srow + rb * 64, bar_load);
+        for (int h = 0; h < 2; ++h)
             for (int rb = 0; rb < MG / 64; ++rb)
                 tc::tma_load_2d(sm + L::KT + h * MG * 128 + rb * 8192, &maps.k, h * 64,
                                 (int)tok0 + rb * 64, bar_load);
-        }
         bulk_g2s(sm + L::QS, q + tok0 * kTcD, TOK * kTcD * 2, bar_load);
-        for (int pl = 0; pl < 4; ++pl)
-            bulk_g2s(sm + L::DEC + pl * 4 * MG, tokdec + pl * plane + tok0, 4 * MG, bar_load);
         mbar_arrive_expect_tx(bar_v, MG * 256);
         for (int h = 0; h < 2; ++h)
             for (int rb = 0; rb < MG / 64; ++rb)
@@ -347,6 +343,15 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     if (warp == 0) {
         tc::tmem_alloc(tbase, TMEM_COLS);
         tc::tmem_relinquish();
+    }
+    griddep_wait();
+    if (tid == 0) {
+        for (int h = 0; h < 2; ++h)
+            for (int rb = 0; rb < 2; ++rb)
+                tc::tma_load_2d(sm + L::HM + h * 16384 + rb * 8192, &maps.state, h * 64,
+                                srow + rb * 64, bar_load);
+        for (int pl = 0; pl < 4; ++pl)
+            bulk_g2s(sm + L::DEC + pl * 4 * MG, tokdec + pl * plane + tok0, 4 * MG, bar_load);
     }
     // decays of every position (from the state pass): l2_t = l_t log2(e) with l_t
     // the chunk-relative cumulative log (w_ti = exp2(l2_t - l2_i)), b_t = exp(l_t),

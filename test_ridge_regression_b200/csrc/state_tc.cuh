@@ -123,6 +123,9 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
     using L = StateSmem<C>;
     constexpr int D = 128, NP = L::NP, PER = C / 32;
     constexpr uint32_t TILE = L::TILE;
+    // the solve launched after this kernel may start its state-independent set-up on
+    // the SMs this grid leaves free (it waits for this grid before reading its output)
+    griddep_launch_dependents();
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = smem_align1024(smraw);
     const uint32_t sb = smem_u32(sm);
