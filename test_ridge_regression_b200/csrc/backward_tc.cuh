@@ -32,6 +32,14 @@ namespace gka {
 
 constexpr int kBrC = 32;   // tokens per chunk of this kernel
 
+// Element (row t, column c) of a [2][32][64] fp16 row tile (128B swizzle).
+__device__ __forceinline__ float f16_tile_at(const uint8_t *tile, int t, int c) {
+    const int cc = c & 63;
+    const uint8_t *p = tile + (c >> 6) * (kBrC * 128) + t * 128 + ((((cc >> 3) ^ t) & 7) << 4) +
+                       (cc & 7) * 2;
+    return __half2float(*reinterpret_cast<const __half *>(p));
+}
+
 struct BwdRowsTcSmem {
     static constexpr uint32_t MA = 0;              // [2][128][64] fp16: H_s, then E^H
     static constexpr uint32_t MB = MA + 32768;     // [2][128][64] fp16: M_s, then E^M
@@ -40,8 +48,8 @@ struct BwdRowsTcSmem {
     static constexpr uint32_t RG = RV + 8192;      // g
     static constexpr uint32_t RX = RG + 8192;      // x (per-token scales)
     static constexpr uint32_t XS = RX + 8192;      // float[32] x scales
-    static constexpr uint32_t RED = XS + 128;      // float[32][4] per-token partial sums
-    static constexpr uint32_t MRED = RED + 512;    // float[16] block reductions
+    static constexpr uint32_t RED = XS + 128;      // float[3][32][4] per-token partial sums
+    static constexpr uint32_t MRED = RED + 1536;   // float[16] block reductions
     static constexpr uint32_t BARS = MRED + 64;    // 5 mbarriers: phase A, phase B, drain,
                                                    // states, adjoints
     static constexpr uint32_t TBASE = BARS + 48;
@@ -75,49 +83,6 @@ __device__ __forceinline__ float tile_f16_sumsq(uint32_t tile) {
         }
     }
     return s2;
-}
-
-// Largest value over the block (256 threads); red: 8 floats.
-__device__ __forceinline__ float block_max256(float v, float *red) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    __syncthreads();
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-    __syncthreads();
-    float m = 0.f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) m = fmaxf(m, red[w]);
-    return m;
-}
-
-// bf16 rows [32][128] (global) -> fp16 [2][32][64] swizzled tile with one power-of-two
-// scale (per_token: one scale per token row, written to xs).  Thread (token t = tid / 8,
-// 16 columns (tid % 8) * 16).  Returns the tile scale (1 with per_token).
-template <typename Src>
-__device__ __forceinline__ float rows_to_f16_tile(const Src *__restrict__ src, uint32_t tile,
-                                                  float *red, bool per_token, float *xs) {
-    const int tid = threadIdx.x, t = tid >> 3, c0 = (tid & 7) * 16;
-    float v[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = to_f(src[t * 128 + c0 + i]);
-    float mx = 0.f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) mx = fmaxf(mx, fabsf(v[i]));
-    float sc;
-    if (per_token) {
-#pragma unroll
-        for (int o = 1; o < 8; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        sc = inv_pow2_above(mx);
-        if ((tid & 7) == 0) xs[t] = sc;
-    } else {
-        sc = inv_pow2_above(block_max256(mx, red));
-    }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] *= sc;
-    const uint32_t base = tile + (uint32_t)(c0 >> 6) * (kBrC * 128u);
-    st_row8(base, (uint32_t)t, (uint32_t)(c0 & 63), v);
-    st_row8(base, (uint32_t)t, (uint32_t)((c0 & 63) + 8), v + 8);
-    return per_token ? 1.f : sc;
 }
 
 // grid (N, B*H), block 256.  T = N * 32.  H_s, M_s: the fp16 chunk-start state copies
@@ -167,11 +132,86 @@ k_bwd_rows_tc(const __grid_constant__ CUtensorMap state_map, const int *__restri
         tc::tmem_alloc(tbase, 256);
         tc::tmem_relinquish();
     }
-    // rows and phase-A matrices
-    const float sK = rows_to_f16_tile(k + tok0 * D, sb + L::RK, mred, false, nullptr);
-    const float sV = rows_to_f16_tile(v + tok0 * D, sb + L::RV, mred, false, nullptr);
-    const float sG = rows_to_f16_tile(dout + tok0 * D, sb + L::RG, mred, false, nullptr);
-    rows_to_f16_tile(xs + tok0 * D, sb + L::RX, mred, true, xsc);
+    // the k, v, g (bf16) and x (fp32) rows: every load issued before any is used; thread
+    // (token t = tid / 8, columns c0 .. c0 + 15); k, v, g with one power-of-two scale per
+    // tile (one block reduction for the three), x with one per token
+    float sK, sV, sG;
+    {
+        const int t = tid >> 3, c0 = (tid & 7) * 16;
+        const size_t g0 = (tok0 + t) * D + c0;
+        uint4 ur[3][2];
+        float4 xr[4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            ur[0][h] = *reinterpret_cast<const uint4 *>(k + g0 + 8 * h);
+            ur[1][h] = *reinterpret_cast<const uint4 *>(v + g0 + 8 * h);
+            ur[2][h] = *reinterpret_cast<const uint4 *>(dout + g0 + 8 * h);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) xr[i] = *reinterpret_cast<const float4 *>(xs + g0 + 4 * i);
+        float f[3][16], mx[3] = {0.f, 0.f, 0.f};
+#pragma unroll
+        for (int m = 0; m < 3; ++m)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t w4[4] = {ur[m][h].x, ur[m][h].y, ur[m][h].z, ur[m][h].w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    f[m][8 * h + 2 * q] = bf16_lo(w4[q]);
+                    f[m][8 * h + 2 * q + 1] = bf16_hi(w4[q]);
+                }
+            }
+#pragma unroll
+        for (int m = 0; m < 3; ++m) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) mx[m] = fmaxf(mx[m], fabsf(f[m][i]));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx[m] = fmaxf(mx[m], __shfl_xor_sync(0xffffffffu, mx[m], o));
+        }
+        if (lane == 0) {
+            mred[warp] = mx[0];
+            mred[8 + warp] = mx[1];
+            red[warp] = mx[2];
+        }
+        // x: one scale per token (its 8 threads)
+        float xv[16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            xv[4 * i] = xr[i].x; xv[4 * i + 1] = xr[i].y; xv[4 * i + 2] = xr[i].z; xv[4 * i + 3] = xr[i].w;
+        }
+        float mxx = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) mxx = fmaxf(mxx, fabsf(xv[i]));
+#pragma unroll
+        for (int o = 1; o < 8; o <<= 1) mxx = fmaxf(mxx, __shfl_xor_sync(0xffffffffu, mxx, o));
+        const float sx = inv_pow2_above(mxx);
+        if ((tid & 7) == 0) xsc[t] = sx;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) xv[i] *= sx;
+        const uint32_t half = (uint32_t)(c0 >> 6) * (kBrC * 128u), cc = (uint32_t)(c0 & 63);
+        st_row8(sb + L::RX + half, (uint32_t)t, cc, xv);
+        st_row8(sb + L::RX + half, (uint32_t)t, cc + 8, xv + 8);
+        __syncthreads();
+        float m3[3] = {0.f, 0.f, 0.f};
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            m3[0] = fmaxf(m3[0], mred[w]);
+            m3[1] = fmaxf(m3[1], mred[8 + w]);
+            m3[2] = fmaxf(m3[2], red[w]);
+        }
+        sK = inv_pow2_above(m3[0]);
+        sV = inv_pow2_above(m3[1]);
+        sG = inv_pow2_above(m3[2]);
+        const float scl[3] = {sK, sV, sG};
+        const uint32_t tiles[3] = {sb + L::RK, sb + L::RV, sb + L::RG};
+#pragma unroll
+        for (int m = 0; m < 3; ++m) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) f[m][i] *= scl[m];
+            st_row8(tiles[m] + half, (uint32_t)t, cc, f[m]);
+            st_row8(tiles[m] + half, (uint32_t)t, cc + 8, f[m] + 8);
+        }
+    }
     // the copies hold 2^e H_s and 2^e' M_s (exponents in [-120, 120])
     const int eH = sexp[((size_t)bh * N + n) * 2], eM = sexp[((size_t)bh * N + n) * 2 + 1];
     const float sH = pow2f(eH), sM = pow2f(eM);
@@ -225,38 +265,58 @@ k_bwd_rows_tc(const __grid_constant__ CUtensorMap state_map, const int *__restri
         __syncthreads();
     };
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(wg * 16);
+    // k, v, x of (token t, column c) from their fp16 tiles (k, v exact; x as the
+    // products saw it), y from memory
+    const float iK = 1.f / sK, iV = 1.f / sV;
+    auto k_at = [&](int t) { return f16_tile_at(sm + L::RK, t, c) * iK; };
+    auto v_at = [&](int t) { return f16_tile_at(sm + L::RV, t, c) * iV; };
     {
-        // one product at a time (register budget: two CTAs per SM)
-        float acc[16], part[16];
+        // the three products one at a time (register budget: two CTAs per SM), their
+        // per-token sums in one reduction
+        float acc[16], p1[16], p2[16], p3[16];
         tc::tmem_ld16(tl + 0, acc);
         tc::tmem_wait_ld();
         const float u1 = 1.f / (sH * sK);
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
-            const size_t g = (tok0 + wg * 16 + u) * D + c;
+            const int t = wg * 16 + u;
+            const size_t g = (tok0 + t) * D + c;
             const float a1 = acc[u] * u1;
             if (ok) R[g] = a1;
-            part[u] = a1 * __bfloat162float(k[g]);
+            p1[u] = a1 * k_at(t);
         }
-        token_sum(part, tokq, 1.f, false);
         tc::tmem_ld16(tl + 32, acc);
         tc::tmem_wait_ld();
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
             const int t = wg * 16 + u;
             const size_t g = (tok0 + t) * D + c;
-            part[u] = acc[u] / (sH * xsc[t]) * ys[g];
+            p2[u] = acc[u] / (sH * xsc[t]) * ys[g];
         }
-        token_sum(part, tokq + plane, 1.f, false);
         tc::tmem_ld16(tl + 64, acc);
         tc::tmem_wait_ld();
         const float u3 = 1.f / (sM * sG);
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
-            const size_t g = (tok0 + wg * 16 + u) * D + c;
-            part[u] = acc[u] * u3 * xs[g];
+            const int t = wg * 16 + u;
+            p3[u] = acc[u] * u3 * (f16_tile_at(sm + L::RX, t, c) / xsc[t]);
         }
-        token_sum(part, tokq + 2 * plane, 1.f, false);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const float a = warp_sum(p1[u]), b = warp_sum(p2[u]), d3 = warp_sum(p3[u]);
+            if (lane == 0) {
+                const int e = (wg * 16 + u) * 4 + quarter;
+                red[e] = a;
+                red[128 + e] = b;
+                red[256 + e] = d3;
+            }
+        }
+        __syncthreads();
+        if (tid < 3 * C && ok) {
+            const int m = tid >> 5, t = tid & 31;
+            const float *r4 = red + m * 128 + t * 4;
+            tokq[m * plane + tok0 + t] = r4[0] + r4[1] + r4[2] + r4[3];
+        }
     }
     // phase B: the adjoint copies (2^e E) in the same tiles
     const float sEH = pow2f(aexp[((size_t)bh * N + n) * 2]);
@@ -289,7 +349,7 @@ k_bwd_rows_tc(const __grid_constant__ CUtensorMap state_map, const int *__restri
             const size_t g = (tok0 + wg * 16 + u) * D + c;
             const float a2 = acc[u] * u2;
             if (ok) R[RD + g] = a2;
-            part[u] = 0.5f * a2 * __bfloat162float(k[g]);
+            part[u] = 0.5f * a2 * k_at(wg * 16 + u);
         }
         tc::tmem_ld16(tl + 128, acc);
         tc::tmem_wait_ld();
@@ -305,7 +365,7 @@ k_bwd_rows_tc(const __grid_constant__ CUtensorMap state_map, const int *__restri
             const size_t g = (tok0 + wg * 16 + u) * D + c;
             const float a4 = acc[u] * u4;
             if (ok) R[3 * RD + g] = a4;
-            part[u] = fmaf(a4, __bfloat162float(v[g]), part[u]);
+            part[u] = fmaf(a4, v_at(wg * 16 + u), part[u]);
         }
         token_sum(part, tokq + 3 * plane, 1.f, false);
     }

@@ -43,8 +43,8 @@ struct BwdGradTcSmem {
     static constexpr uint32_t HALF = 20480;                 // one 64-column half: 160 rows
     static constexpr uint32_t RGN = 0;                      // [2][160][64] fp16 rows X Y K G V
     static constexpr uint32_t PT = RGN + 2 * HALF;          // 4 x [32][64] fp16: Py Px Pk Pg
-    static constexpr uint32_t MAT = PT + 4 * 4096;          // 6 x float[32][33]: KX KY VG GK Q PHI
-    static constexpr uint32_t SIG = MAT + 6 * 32 * 33 * 4;  // float[5][32] row scales x y k g v
+    static constexpr uint32_t MAT = PT + 4 * 4096;          // 7 x float[32][33]: KX KY VG GK Q PHI W
+    static constexpr uint32_t SIG = MAT + 7 * 32 * 33 * 4;  // float[5][32] inverse row scales x y k g v
     static constexpr uint32_t SCAL = SIG + 5 * 128;         // float[13][32] per-token scalars
     static constexpr uint32_t RED = SCAL + 13 * 128;        // float[32][4] token sums
     static constexpr uint32_t MRED = RED + 512;             // float[8][2] maxima, 2 scales
@@ -69,8 +69,8 @@ k_bwd_grads_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restr
     uint8_t *sm = smem_align1024(smraw);
     const uint32_t sb = smem_u32(sm);
     float *KX = reinterpret_cast<float *>(sm + L::MAT), *KY = KX + C * CP, *VG = KY + C * CP,
-          *GK = VG + C * CP, *Qm = GK + C * CP, *PH = Qm + C * CP;
-    float *sig = reinterpret_cast<float *>(sm + L::SIG);    // x y k g v
+          *GK = VG + C * CP, *Qm = GK + C * CP, *PH = Qm + C * CP, *Wt = PH + C * CP;
+    float *isig = reinterpret_cast<float *>(sm + L::SIG);   // 1 / row scale: x y k g v
     float *sc = reinterpret_cast<float *>(sm + L::SCAL);
     float *s_b = sc, *s_step = sc + 32, *s_wend = sc + 64, *s_w = sc + 96, *s_c = sc + 128,
           *s_uk = sc + 160, *s_yhx = sc + 192, *s_gmx = sc + 224, *s_qe = sc + 256,
@@ -127,6 +127,11 @@ k_bwd_grads_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restr
         s_qe[tid] = tokq[3 * plane + tok0 + tid];
         s_bm1[tid] = tid == 0 ? 1.f : decay_exp(ell[tid - 1]);
     }
+    // W[l][s] = w_sl for s >= l, else 0
+    for (int e = tid; e < C * C; e += kSimtThreads) {
+        const int l = e >> 5, s2 = e & 31;
+        Wt[l * CP + s2] = s2 >= l ? decay_exp(ell[s2] - ell[l]) : 0.f;
+    }
     // the row tiles, one power-of-two scale per row (16 threads share a row)
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
@@ -138,7 +143,7 @@ k_bwd_grads_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restr
 #pragma unroll
             for (int o = 1; o < 16; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
             const float s = inv_pow2_above(mx);
-            if (j == 0) sig[tensor * 32 + t] = s;
+            if (j == 0) isig[tensor * 32 + t] = 1.f / s;   // a power of two: exact
             const uint32_t row = (uint32_t)(tensor * 32 + t);
             st_shared_v4(sb + L::RGN + (uint32_t)(j >> 3) * L::HALF + row * 128u +
                              (((uint32_t)j ^ row) & 7u) * 16u,
@@ -209,20 +214,20 @@ k_bwd_grads_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restr
         const int l = lane;
         const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         float d32[32];
-        auto row = [&](int col0, float *dst, const float *sig_b, float sa) {
+        auto row = [&](int col0, float *dst, const float *isig_b, float ia) {
             tc::tmem_ld16(tl + col0, d32);
             tc::tmem_ld16(tl + col0 + 16, d32 + 16);
             tc::tmem_wait_ld();
 #pragma unroll
-            for (int s2 = 0; s2 < 32; ++s2) dst[l * CP + s2] = d32[s2] / (sa * sig_b[s2]);
+            for (int s2 = 0; s2 < 32; ++s2) dst[l * CP + s2] = d32[s2] * ia * isig_b[s2];
         };
         if (warp == 0) {
-            row(0, KX, sig, sig[64 + l]);
-            row(32, KY, sig + 32, sig[64 + l]);
+            row(0, KX, isig, isig[64 + l]);
+            row(32, KY, isig + 32, isig[64 + l]);
         } else if (warp == 4) {
-            row(64, GK, sig + 64, sig[64 + l]);
+            row(64, GK, isig + 64, isig[64 + l]);
         } else {
-            row(96, VG, sig + 96, sig[128 + l]);
+            row(96, VG, isig + 96, isig[128 + l]);
         }
     }
     tc::fence_before_sync();
@@ -234,6 +239,7 @@ k_bwd_grads_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restr
         {
             const int i = lane;   // Q[i][s] = sum_{l<=s} w_sl w_l w_i (k_l . k_i)^2
             float qv = 0.f;
+#pragma unroll 8
             for (int s2 = 0; s2 < C; ++s2) {
                 const float g2 = GK[s2 * CP + i];
                 qv = fmaf(s2 == 0 ? 0.f : s_step[s2], qv, s_w[s2] * s_w[i] * g2 * g2);
@@ -242,9 +248,12 @@ k_bwd_grads_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restr
         }
         __syncwarp();
         {
+            // a fixed trip count (entries j > s are formed and dropped) so that the
+            // loads of several steps are issued together
             const int s2 = lane;
             float t1 = 0.f, t2 = 0.f, t3 = 0.f, u1 = 0.f;
-            for (int jj = 0; jj <= s2; ++jj) {
+#pragma unroll 8
+            for (int jj = 0; jj < C; ++jj) {
                 if (jj > 0) {
                     const int i = jj - 1;
                     const float st = s_step[i];
@@ -257,17 +266,21 @@ k_bwd_grads_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restr
                 const float phi = -(bm * s_yhx[s2] + t1)
                                   - s_c[s2] * (s_b[s2] * bm * hs2 + s_b[s2] * u1 + bm * s_X1[s2] + t2)
                                   + (bm * s_gmx[s2] + t3);
-                PH[jj * CP + s2] = decay_exp(ell[s2] - ell[jj]) * phi;   // w_sj Phi[j][s]
+                if (jj <= s2) PH[jj * CP + s2] = Wt[jj * CP + s2] * phi;   // w_sj Phi[j][s]
             }
         }
         __syncwarp();
         {
             const int jj = lane;
             float acc = 0.f;
-            for (int s2 = jj; s2 < C; ++s2) acc += PH[jj * CP + s2];
+#pragma unroll 8
+            for (int s2 = 0; s2 < C; ++s2)
+                if (s2 >= jj) acc += PH[jj * CP + s2];
             // the adjoint from later chunks: w_{C-1,j} (b_{j-1} eh + sum_{i<j} w_{j-1,i} w_i qe_i)
             float qe = 0.f;
-            for (int i = 0; i < jj; ++i) qe = fmaf(s_step[i], qe, s_w[i] * s_qe[i]);
+#pragma unroll 8
+            for (int i = 0; i < C; ++i)
+                if (i < jj) qe = fmaf(s_step[i], qe, s_w[i] * s_qe[i]);
             acc = fmaf(s_wend[jj], fmaf(s_bm1[jj], eh, qe), acc);
             if (ok) dbeta[tok0 + jj] = acc;
         }
@@ -277,14 +290,14 @@ k_bwd_grads_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restr
         constexpr int NT = kSimtThreads - 32;
         const int me = tid < 32 ? tid : tid - 32;
         auto coef = [&](int l, int s2, float *p4) {
-            const float w = s2 >= l ? decay_exp(ell[s2] - ell[l]) : 0.f;
+            const float w = Wt[l * CP + s2];
             const float kx = KX[l * CP + s2];
-            p4[0] = -w * kx / sig[32 + s2];                          // Py / sigma_y
-            p4[1] = w * (VG[l * CP + s2] - KY[l * CP + s2]) / sig[s2];   // Px / sigma_x
+            p4[0] = -w * kx * isig[32 + s2];                             // Py / sigma_y
+            p4[1] = w * (VG[l * CP + s2] - KY[l * CP + s2]) * isig[s2];  // Px / sigma_x
             const int m = l > s2 ? l : s2;
-            p4[2] = -2.f * s_R[m] * decay_exp(ell[m] - ell[l]) * decay_exp(ell[m] - ell[s2]) *
-                    s_w[s2] * GK[l * CP + s2] / sig[64 + s2];         // Pk / sigma_k
-            p4[3] = w * kx / sig[96 + s2];                           // Pg / sigma_g
+            p4[2] = -2.f * s_R[m] * Wt[l * CP + m] * Wt[s2 * CP + m] * s_w[s2] * GK[l * CP + s2] *
+                    isig[64 + s2];                                       // Pk / sigma_k
+            p4[3] = w * kx * isig[96 + s2];                              // Pg / sigma_g
         };
         float ma = 0.f, mg = 0.f;
         for (int e = me; e < C * C / 2; e += NT) {
@@ -378,8 +391,16 @@ k_bwd_grads_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restr
                 dk[g] = __float2bfloat16_rn(s_w[l] * a);
                 dv[g] = __float2bfloat16_rn(s_w[l] * bb);
             }
-            // write-gate gradient: (k . A + v . B) / 2 over the row
-            const float dgp = warp_sum(fmaf(__bfloat162float(k[g]), a, __bfloat162float(v[g]) * bb));
+            // write-gate gradient: (k . A + v . B) / 2 over the row (k, v from their
+            // row tiles, exact for bf16 inputs)
+            auto at = [&](int row) {
+                const int cc = c & 63;
+                const uint8_t *p = sm + L::RGN + (c >> 6) * L::HALF + row * 128 +
+                                   ((((cc >> 3) ^ row) & 7) << 4) + (cc & 7) * 2;
+                return __half2float(*reinterpret_cast<const __half *>(p));
+            };
+            const float kc = at(64 + l) * isig[64 + l], vc = at(128 + l) * isig[128 + l];
+            const float dgp = warp_sum(fmaf(kc, a, vc * bb));
             if (lane == 0) red[l * 4 + quarter] = dgp;
         }
     }
