@@ -21,7 +21,6 @@
 #include "chunk_simt.cuh"
 #include "common.cuh"
 #include "decode.cuh"
-#include "delta_tc.cuh"
 #include "seg_tc.cuh"
 #include "solve_tc.cuh"
 #include "state_tc.cuh"
