@@ -246,13 +246,33 @@ static int rows128_map(CUtensorMap *m, const void *base, uint64_t rows, CUtensor
 
 static int timeout_flag_ptr(int **ptr);
 
+// The tensor-core forward workspace's per-token decay planes (4 x B*H*T floats: l2, b,
+// beta, beta^2) for chunk C.
+static float *tc_tokdec(char *ws, const gka_workspace_layout &L, int BH, int T, int C) {
+    constexpr int D = 128;
+    const size_t BHN2 = (size_t)BH * (T / C) * 2;
+    return reinterpret_cast<float *>(ws + L.states_lp_offset + round256(2 * BHN2 * (size_t)D * D) +
+                                     round256(sizeof(float) * BHN2) + round256(sizeof(int) * BHN2));
+}
+
+// States written elsewhere for the solve: fp16 chunk-start copies and their exponents, one
+// every `sstride` entries (copies at chunks sstride times shorter), with the per-token decays
+// already in the workspace; `pdl`: the kernel before the solve writes none of its inputs.
+struct TcExternalStates {
+    const __half *slp;
+    const int *sexp;
+    int sstride;
+    bool pdl;
+};
+
 static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
                       const float *beta, const float *gate, __nv_bfloat16 *o, int B, int H, int T, int C,
                       const ChebParams &P, float *final_state, char *ws,
                       const gka_workspace_layout &L, cudaStream_t s, float *x_out = nullptr,
-                      bool solve_only = false) {
+                      bool solve_only = false, const TcExternalStates *ext = nullptr) {
     // x_out: write the iterates instead of o; solve_only: the chunk states in the
-    // workspace are current (an earlier call on the same keys, values and decays)
+    // workspace are current (an earlier call on the same keys, values and decays);
+    // ext (with solve_only): the states come from ext instead
     constexpr int D = 128;
     const int BH = B * H, N = T / C;
     float *states = reinterpret_cast<float *>(ws + L.states_offset);
@@ -273,9 +293,11 @@ static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
     TcMaps maps;
     if (int rc = rows128_map(&maps.k, k, (uint64_t)BH * T, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)) return rc;
     if (int rc = rows128_map(&maps.v, v, (uint64_t)BH * T, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)) return rc;
-    if (int rc = rows128_map(&maps.state, slp, (uint64_t)BH * N * 2 * D,
+    const int sstride = ext ? ext->sstride : 1;
+    if (int rc = rows128_map(&maps.state, ext ? ext->slp : slp, (uint64_t)BH * N * sstride * 2 * D,
                              CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
         return rc;
+    const int *sexp_solve = ext ? ext->sexp : sexp;
     cudaError_t e;
 
     if (solve_only) {
@@ -321,14 +343,14 @@ static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
             ProfScope ps(GKA_KERNEL_STATE_PASS_TC, s);
             k_state_pass_tc<64><<<dim3(2, BH * S), kStateThreads, StateSmem<64>::bytes, s>>>(
                 smaps, beta, gate, sexp, decay, tokdec, plane, final_state, T, N, S, K, seg_start,
-                seg_bound, flag);
+                seg_bound, flag, 1);
         } else {
             if ((e = set_smem(k_state_pass_tc<128>, StateSmem<128>::bytes)) != cudaSuccess)
                 return cuda_fail(e);
             ProfScope ps(GKA_KERNEL_STATE_PASS_TC, s);
             k_state_pass_tc<128><<<dim3(2, BH * S), kStateThreads, StateSmem<128>::bytes, s>>>(
                 smaps, beta, gate, sexp, decay, tokdec, plane, final_state, T, N, S, K, seg_start,
-                seg_bound, flag);
+                seg_bound, flag, 1);
         }
         if (int rc = check_launch()) return rc;
     }
@@ -337,7 +359,7 @@ static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
     // input loads, barriers and TMEM allocation overlap the pass, and it waits for the
     // pass (griddepcontrol.wait) before reading the state copies and decays.  With
     // solve_only the kernel before it may have written q, which the solve reads before
-    // that wait, so it is launched in plain stream order.
+    // that wait, so it is launched in plain stream order unless ext says otherwise.
     auto launch_solve = [&](auto kern, size_t smem) -> cudaError_t {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(N, BH);
@@ -348,9 +370,9 @@ static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
-        cfg.numAttrs = solve_only ? 0 : 1;
+        cfg.numAttrs = (!solve_only || (ext && ext->pdl)) ? 1 : 0;
         return cudaLaunchKernelEx(&cfg, kern, maps, q, gate, (const float *)tokdec, plane, norms,
-                                  (const int *)sexp, o, x_out, T, N, C, P, flag);
+                                  sexp_solve, o, x_out, T, N, C, P, flag, sstride);
     };
     if (C == 64) {
         // one CTA per 64-token chunk
@@ -457,7 +479,9 @@ static int backward_simt(const Tin *q, const Tin *k, const Tin *v, const float *
     if constexpr (std::is_same<Tin, __nv_bfloat16>::value && D == 128) {
         if (L.tc_recompute && C == 32) {
             // the chunk states in one sequential pass per (head, matrix) on tcgen05 (no
-            // increments through memory), and the chunk decays
+            // increments through memory), the chunk decays, and the per-token decays of
+            // 64-token groups in the tensor-core forward's workspace: the solves below read
+            // these copies at every second chunk instead of a pass of their own
             int *flag = nullptr;
             if (int rc = timeout_flag_ptr(&flag)) return rc;
             StateMaps sm32;
@@ -477,8 +501,8 @@ static int backward_simt(const Tin *q, const Tin *k, const Tin *v, const float *
                 return cuda_fail(e);
             { ProfScope ps(GKA_KERNEL_STATE_PASS_TC, s);
             k_state_pass_tc<32><<<dim3(2, BH), kStateThreads, StateSmem<32>::bytes, s>>>(
-                sm32, beta, gate, sexp32, decay, nullptr, 0, nullptr, T, N, 1, 1, nullptr, nullptr,
-                flag); }
+                sm32, beta, gate, sexp32, decay, tc_tokdec(ws + L.tc, L.tcl, BH, T, 64),
+                (size_t)BH * T, nullptr, T, N, 1, 1, nullptr, nullptr, flag, 2); }
             if (int rc = check_launch()) return rc;
             states_done = true;
         }
@@ -500,8 +524,11 @@ static int backward_simt(const Tin *q, const Tin *k, const Tin *v, const float *
     if constexpr (std::is_same<Tin, __nv_bfloat16>::value && D == 128) {
         if (L.tc_recompute) {
             char *tws = ws + L.tc;
+            // the iterates; with the 32-token copies (the state pass just before writes none
+            // of the solve's inputs: a programmatic dependent launch)
+            const TcExternalStates ext{slp32, sexp32, 2, true};
             if (int rc = forward_tc(q, k, v, beta, gate, nullptr, B, H, T, 64, P, nullptr, tws,
-                                    L.tcl, s, xs))
+                                    L.tcl, s, xs, states_done, states_done ? &ext : nullptr))
                 return rc;
             norms = reinterpret_cast<float *>(tws + L.tcl.norms_offset);
             tc_done = true;
@@ -547,8 +574,10 @@ static int backward_simt(const Tin *q, const Tin *k, const Tin *v, const float *
     if (int rc = check_launch()) return rc;
     if constexpr (std::is_same<Tin, __nv_bfloat16>::value && D == 128) {
         if (tc_done) {
+            // y on u (u was written by the kernel just before: plain stream order)
+            const TcExternalStates ext{slp32, sexp32, 2, false};
             if (int rc = forward_tc(u16, k, v, beta, gate, nullptr, B, H, T, 64, P, nullptr,
-                                    ws + L.tc, L.tcl, s, ys, true))
+                                    ws + L.tc, L.tcl, s, ys, true, states_done ? &ext : nullptr))
                 return rc;
             { ProfScope ps(GKA_KERNEL_BWD_SOLVE, s);
             k_bwd_yfinish<Tin, D><<<(unsigned)(((size_t)BH * T + 7) / 8), kSimtThreads, 0, s>>>(

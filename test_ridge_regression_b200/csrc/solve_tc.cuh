@@ -288,7 +288,9 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
                  const float *__restrict__ gate, const float *__restrict__ tokdec, size_t plane, float *__restrict__ norms,
                  const int *__restrict__ state_exp, __nv_bfloat16 *__restrict__ o,
                  float *__restrict__ x_out, int T, int N, int C, const ChebParams P,
-                 int *__restrict__ timeout_flag) {
+                 int *__restrict__ timeout_flag, int sstride) {
+    // sstride: chunk stride of the state copies and exponents (1: one copy per chunk of
+    // this kernel; 2: copies at half-size chunks, this chunk's start at every second)
     using L = TcSmem<MG, TOK>;
     constexpr int HALF = MG / 2;       // keys per warpgroup in the norm reductions
     constexpr int TPT = TOK / 2;       // tokens per thread
@@ -318,7 +320,8 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     const int tcol = wg * TPT;                // first token (TMEM column) of this thread
     const int n = blockIdx.x, bh = blockIdx.y;
     const size_t tok0 = (size_t)bh * T + (size_t)n * C;    // first token of the chunk
-    const int srow = (int)(((size_t)bh * N + n) * 2 * kTcD);   // H_s row in the state map
+    const size_t scopy = ((size_t)bh * N + n) * sstride;        // this chunk's state copy
+    const int srow = (int)(scopy * 2 * kTcD);                   // H_s row in the state map
 
     if (tid == 0) {
         for (int i = 0; i < 8; ++i) mbar_init(&bars[i], i == 5 ? 2 : 1);   // bar_fin: 2
@@ -359,8 +362,8 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
     // products of beta: w_{t,i-1} = w_ti beta_i and w_{t+1,i} = w_ti beta_{t+1}.
     float *s_l2 = reinterpret_cast<float *>(sm + L::DEC);
     float *s_bt = s_l2 + MG, *s_bet = s_bt + MG, *s_beta2 = s_bet + MG;
-    const int eHexp = state_exp[((size_t)bh * N + n) * 2];
-    const int eMexp = state_exp[((size_t)bh * N + n) * 2 + 1];
+    const int eHexp = state_exp[scopy * 2];
+    const int eMexp = state_exp[scopy * 2 + 1];
     bool ok = mbar_wait_sleep(bar_load, 0, kTcSleepProbes, kTcSleepNs);
     // keys: bf16 -> fp16 in place, scaled below 1 (the values follow while the norm
     // products run); with the write gate, key and value rows of token i are taken

@@ -118,7 +118,9 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
                 const float *__restrict__ gate, int *__restrict__ state_exp, float *__restrict__ decay,
                 float *__restrict__ tokdec, size_t plane, float *__restrict__ final_state,
                 int T, int N, int S, int K, const float *__restrict__ seg_start,
-                const float *__restrict__ seg_bound, int *__restrict__ timeout_flag) {
+                const float *__restrict__ seg_bound, int *__restrict__ timeout_flag, int tdc) {
+    // tdc: the per-token decays are relative to groups of tdc chunks (1: to this kernel's
+    // chunks; 2 with S == 1: to chunks twice as long, for a solve at that size)
     constexpr int BOXR = C < 64 ? C : 64;   // rows per TMA box of k and v
     using L = StateSmem<C>;
     constexpr int D = 128, NP = L::NP, PER = C / 32;
@@ -243,7 +245,9 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
 
     // Decay warp of the H CTA: chunk c's per-token decays for the solve
     // (l_t log2 e, exp(l_t), beta_t, beta_t^2; l from fp32 logs summed in
-    // double) and the chunk decay.
+    // double, relative to the start of the chunk's group of tdc chunks) and the
+    // chunk decay.
+    double goff = 0.0;   // summed log of the group's earlier chunks
     auto token_decays = [&](int c) {
         const float *bt = s_beta + (c & 1) * C;
         double x[PER];
@@ -259,9 +263,9 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
             const double y = __shfl_up_sync(0xffffffffu, t2, o);
             if (lane >= o) t2 += y;
         }
-        const double excl = t2 - acc;
-        double prev = __shfl_up_sync(0xffffffffu, t2, 1);
-        if (lane == 0) prev = 0.0;
+        const double excl = t2 - acc + goff;
+        double prev = __shfl_up_sync(0xffffffffu, t2, 1) + goff;
+        if (lane == 0) prev = goff;
 #pragma unroll
         for (int p = 0; p < PER; ++p) {
             const double l = x[p] + excl;
@@ -277,6 +281,7 @@ k_state_pass_tc(const __grid_constant__ StateMaps maps, const float *__restrict_
         }
         const double lend = __shfl_sync(0xffffffffu, t2, 31);
         if (lane == 0) decay[(size_t)bh * N + n0 + c] = decay_exp(lend);
+        goff = (n0 + c + 1) % tdc == 0 ? 0.0 : goff + lend;
         __syncwarp();
     };
 
