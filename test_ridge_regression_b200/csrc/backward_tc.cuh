@@ -41,18 +41,17 @@ __device__ __forceinline__ float f16_tile_at(const uint8_t *tile, int t, int c) 
 }
 
 struct BwdRowsTcSmem {
-    static constexpr uint32_t MA = 0;              // [2][128][64] fp16: H_s, then E^H
-    static constexpr uint32_t MB = MA + 32768;     // [2][128][64] fp16: M_s, then E^M
-    static constexpr uint32_t RK = MB + 32768;     // [2][32][64] fp16 rows of k
-    static constexpr uint32_t RV = RK + 8192;      // v
-    static constexpr uint32_t RG = RV + 8192;      // g
+    static constexpr uint32_t MA = 0;              // [2][128][64] fp16: H_s or M_s, then E^H or E^M
+    static constexpr uint32_t RK = MA + 32768;     // [2][32][64] fp16 rows of k
+    static constexpr uint32_t RV = RK + 8192;      // v (M role)
+    static constexpr uint32_t RG = RV + 8192;      // g (M role)
     static constexpr uint32_t RX = RG + 8192;      // x (per-token scales)
     static constexpr uint32_t XS = RX + 8192;      // float[32] x scales
-    static constexpr uint32_t RED = XS + 128;      // float[3][32][4] per-token partial sums
-    static constexpr uint32_t MRED = RED + 1536;   // float[16] block reductions
-    static constexpr uint32_t BARS = MRED + 64;    // 5 mbarriers: phase A, phase B, drain,
-                                                   // states, adjoints
-    static constexpr uint32_t TBASE = BARS + 48;
+    static constexpr uint32_t RED = XS + 128;      // float[2][32][4] per-token partial sums
+    static constexpr uint32_t MRED = RED + 1024;   // float[24] block reductions
+    static constexpr uint32_t BARS = MRED + 96;    // 5 mbarriers: products A, B; matrix;
+                                                   // adjoint; drain
+    static constexpr uint32_t TBASE = BARS + 40;
     static constexpr uint32_t END = TBASE + 16;
     static constexpr size_t bytes = END + 1024;    // + alignment slack
 };
@@ -85,11 +84,13 @@ __device__ __forceinline__ float tile_f16_sumsq(uint32_t tile) {
     return s2;
 }
 
-// grid (N, B*H), block 256.  T = N * 32.  H_s, M_s: the fp16 chunk-start state copies
-// of the recompute's state pass (state_map, exponents sexp [B*H][N][2]); E^H, E^M: the
-// fp16 adjoint copies of the adjoint pass (adj_map over adj_lp, same layout, exponents
-// aexp) and its inner products eh_part [B*H][N][2] (<E^H, H_s>, <E^M, M_s>).
-__global__ void __launch_bounds__(kSimtThreads, 2)
+// grid (N, B*H, 2), block 256, three CTAs per SM.  T = N * 32.  blockIdx.z = 0 (H role):
+// H_s, then E^H: R1, uk, yhx, R2, the H part of qe (tokq plane 3), hs2 and eh; 1 (M role):
+// M_s, then E^M: gmx, R3, R4, the M part of qe (tokq plane 4).  H_s, M_s: the fp16
+// chunk-start state copies of the recompute's state pass (state_map, exponents sexp
+// [B*H][N][2]); E^H, E^M: the fp16 adjoint copies of the adjoint pass (adj_map over adj_lp,
+// same layout, exponents aexp) and its inner products eh_part [B*H][N][2].
+__global__ void __launch_bounds__(kSimtThreads, 3)
 k_bwd_rows_tc(const __grid_constant__ CUtensorMap state_map, const int *__restrict__ sexp,
               const __grid_constant__ CUtensorMap adj_map, const __half *__restrict__ adj_lp,
               const int *__restrict__ aexp, const float *__restrict__ eh_part,
@@ -103,137 +104,151 @@ k_bwd_rows_tc(const __grid_constant__ CUtensorMap state_map, const int *__restri
     uint8_t *sm = smem_align1024(smraw);
     const uint32_t sb = smem_u32(sm);
     float *xsc = reinterpret_cast<float *>(sm + L::XS);
-    float *red = reinterpret_cast<float *>(sm + L::RED);    // [32 tokens][4 quarters]
+    float *red = reinterpret_cast<float *>(sm + L::RED);    // [2][32 tokens][4 quarters]
     float *mred = reinterpret_cast<float *>(sm + L::MRED);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BARS);
     uint32_t *tbase = reinterpret_cast<uint32_t *>(sm + L::TBASE);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3, wg = warp >> 2;
     const int c = quarter * 32 + lane;       // matrix row = TMEM lane of this thread
-    const int n = blockIdx.x, bh = blockIdx.y;
+    const int n = blockIdx.x, bh = blockIdx.y, m = blockIdx.z;   // m = 0: H role, 1: M role
+    const bool mrole = m == 1;
     const size_t tok0 = (size_t)bh * T + (size_t)n * C;
     const size_t plane = (size_t)gridDim.y * T, RD = plane * D;
-    const int srow = (int)(((size_t)bh * N + n) * 2 * D);   // H_s (E^H) row in the maps
+    const size_t e2 = ((size_t)bh * N + n) * 2;               // (chunk, matrix 0) entry
+    const int mrow = (int)((e2 + m) * D);                       // this role's matrix in the maps
 
     if (tid == 0) {
         for (int i = 0; i < 5; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
-        // H_s and M_s as fp16 tiles (the state pass's copies), read while the rows convert
-        mbar_arrive_expect_tx(&bars[3], 2 * 32768);
-        load_state_tile(&state_map, srow, sm + L::MA, &bars[3]);
-        load_state_tile(&state_map, srow + D, sm + L::MB, &bars[3]);
+        // this role's chunk-start state (fp16 copy), read while the rows convert
+        mbar_arrive_expect_tx(&bars[2], 32768);
+        load_state_tile(&state_map, mrow, sm + L::MA, &bars[2]);
     }
     if (tid == 32) {
-        // everything read after the rows: the two adjoint copies and the fp32 y rows
-        bulk_prefetch_l2(adj_lp + (size_t)srow * D, 2 * D * D * 2);
-        bulk_prefetch_l2(ys + tok0 * D, C * D * 4);
+        // read after the rows: this role's adjoint copy (and the fp32 y rows in the H role)
+        bulk_prefetch_l2(adj_lp + (size_t)mrow * D, D * D * 2);
+        if (!mrole) bulk_prefetch_l2(ys + tok0 * D, C * D * 4);
     }
     if (warp == 0) {
-        tc::tmem_alloc(tbase, 256);
+        tc::tmem_alloc(tbase, 128);
         tc::tmem_relinquish();
     }
-    // the k, v, g (bf16) and x (fp32) rows: every load issued before any is used; thread
-    // (token t = tid / 8, columns c0 .. c0 + 15); k, v, g with one power-of-two scale per
-    // tile (one block reduction for the three), x with one per token
-    float sK, sV, sG;
+    // rows, thread (token t = tid / 8, columns c0 .. c0 + 15): k (and in the M role v, g)
+    // in bf16 with one power-of-two scale per tile (one block reduction), x with one per
+    // token; every load issued before any is used
+    const int t8 = tid >> 3, c0 = (tid & 7) * 16;
+    const uint32_t rhalf = (uint32_t)(c0 >> 6) * (kBrC * 128u), rcc = (uint32_t)(c0 & 63);
+    float sK, sV = 1.f, sG = 1.f;
     {
-        const int t = tid >> 3, c0 = (tid & 7) * 16;
-        const size_t g0 = (tok0 + t) * D + c0;
+        const size_t g0 = (tok0 + t8) * D + c0;
         uint4 ur[3][2];
         float4 xr[4];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             ur[0][h] = *reinterpret_cast<const uint4 *>(k + g0 + 8 * h);
-            ur[1][h] = *reinterpret_cast<const uint4 *>(v + g0 + 8 * h);
-            ur[2][h] = *reinterpret_cast<const uint4 *>(dout + g0 + 8 * h);
+            if (mrole) {
+                ur[1][h] = *reinterpret_cast<const uint4 *>(v + g0 + 8 * h);
+                ur[2][h] = *reinterpret_cast<const uint4 *>(dout + g0 + 8 * h);
+            } else {
+                ur[1][h] = ur[2][h] = make_uint4(0u, 0u, 0u, 0u);
+            }
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i) xr[i] = *reinterpret_cast<const float4 *>(xs + g0 + 4 * i);
-        float f[3][16], mx[3] = {0.f, 0.f, 0.f};
+        // x: one scale per token (its 8 threads)
+        {
+            float xv[16];
 #pragma unroll
-        for (int m = 0; m < 3; ++m)
+            for (int i = 0; i < 4; ++i) {
+                xv[4 * i] = xr[i].x; xv[4 * i + 1] = xr[i].y; xv[4 * i + 2] = xr[i].z; xv[4 * i + 3] = xr[i].w;
+            }
+            float mxx = 0.f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) mxx = fmaxf(mxx, fabsf(xv[i]));
+#pragma unroll
+            for (int o = 1; o < 8; o <<= 1) mxx = fmaxf(mxx, __shfl_xor_sync(0xffffffffu, mxx, o));
+            const float sx = inv_pow2_above(mxx);
+            if ((tid & 7) == 0) xsc[t8] = sx;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) xv[i] *= sx;
+            st_row8(sb + L::RX + rhalf, (uint32_t)t8, rcc, xv);
+            st_row8(sb + L::RX + rhalf, (uint32_t)t8, rcc + 8, xv + 8);
+        }
+        float mx[3] = {0.f, 0.f, 0.f};
+#pragma unroll
+        for (int q = 0; q < 3; ++q) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                const uint32_t w4[4] = {ur[m][h].x, ur[m][h].y, ur[m][h].z, ur[m][h].w};
+                const uint32_t w4[4] = {ur[q][h].x, ur[q][h].y, ur[q][h].z, ur[q][h].w};
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    f[m][8 * h + 2 * q] = bf16_lo(w4[q]);
-                    f[m][8 * h + 2 * q + 1] = bf16_hi(w4[q]);
-                }
+                for (int i = 0; i < 4; ++i)
+                    mx[q] = fmaxf(mx[q], fmaxf(fabsf(bf16_lo(w4[i])), fabsf(bf16_hi(w4[i]))));
             }
 #pragma unroll
-        for (int m = 0; m < 3; ++m) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) mx[m] = fmaxf(mx[m], fabsf(f[m][i]));
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) mx[m] = fmaxf(mx[m], __shfl_xor_sync(0xffffffffu, mx[m], o));
+            for (int o = 16; o > 0; o >>= 1) mx[q] = fmaxf(mx[q], __shfl_xor_sync(0xffffffffu, mx[q], o));
         }
         if (lane == 0) {
             mred[warp] = mx[0];
             mred[8 + warp] = mx[1];
-            red[warp] = mx[2];
+            mred[16 + warp] = mx[2];
         }
-        // x: one scale per token (its 8 threads)
-        float xv[16];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            xv[4 * i] = xr[i].x; xv[4 * i + 1] = xr[i].y; xv[4 * i + 2] = xr[i].z; xv[4 * i + 3] = xr[i].w;
-        }
-        float mxx = 0.f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) mxx = fmaxf(mxx, fabsf(xv[i]));
-#pragma unroll
-        for (int o = 1; o < 8; o <<= 1) mxx = fmaxf(mxx, __shfl_xor_sync(0xffffffffu, mxx, o));
-        const float sx = inv_pow2_above(mxx);
-        if ((tid & 7) == 0) xsc[t] = sx;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) xv[i] *= sx;
-        const uint32_t half = (uint32_t)(c0 >> 6) * (kBrC * 128u), cc = (uint32_t)(c0 & 63);
-        st_row8(sb + L::RX + half, (uint32_t)t, cc, xv);
-        st_row8(sb + L::RX + half, (uint32_t)t, cc + 8, xv + 8);
         __syncthreads();
         float m3[3] = {0.f, 0.f, 0.f};
 #pragma unroll
         for (int w = 0; w < 8; ++w) {
             m3[0] = fmaxf(m3[0], mred[w]);
             m3[1] = fmaxf(m3[1], mred[8 + w]);
-            m3[2] = fmaxf(m3[2], red[w]);
+            m3[2] = fmaxf(m3[2], mred[16 + w]);
         }
         sK = inv_pow2_above(m3[0]);
-        sV = inv_pow2_above(m3[1]);
-        sG = inv_pow2_above(m3[2]);
+        if (mrole) {
+            sV = inv_pow2_above(m3[1]);
+            sG = inv_pow2_above(m3[2]);
+        }
         const float scl[3] = {sK, sV, sG};
         const uint32_t tiles[3] = {sb + L::RK, sb + L::RV, sb + L::RG};
 #pragma unroll
-        for (int m = 0; m < 3; ++m) {
+        for (int q = 0; q < 3; ++q) {
+            if (q > 0 && !mrole) break;
+            float f[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) f[m][i] *= scl[m];
-            st_row8(tiles[m] + half, (uint32_t)t, cc, f[m]);
-            st_row8(tiles[m] + half, (uint32_t)t, cc + 8, f[m] + 8);
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t w4[4] = {ur[q][h].x, ur[q][h].y, ur[q][h].z, ur[q][h].w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    f[8 * h + 2 * i] = bf16_lo(w4[i]) * scl[q];
+                    f[8 * h + 2 * i + 1] = bf16_hi(w4[i]) * scl[q];
+                }
+            }
+            st_row8(tiles[q] + rhalf, (uint32_t)t8, rcc, f);
+            st_row8(tiles[q] + rhalf, (uint32_t)t8, rcc + 8, f + 8);
         }
     }
-    // the copies hold 2^e H_s and 2^e' M_s (exponents in [-120, 120])
-    const int eH = sexp[((size_t)bh * N + n) * 2], eM = sexp[((size_t)bh * N + n) * 2 + 1];
-    const float sH = pow2f(eH), sM = pow2f(eM);
-    bool ok = mbar_wait_bounded(&bars[3], 0, kTcWaitProbes);
-    float hs2 = tile_f16_sumsq(sb + L::MA) * (pow2f(-eH) * pow2f(-eH));
+    // the copy holds 2^e S (exponents in [-120, 120])
+    const float sS = pow2f(sexp[e2 + m]);
+    bool ok = mbar_wait_bounded(&bars[2], 0, kTcWaitProbes);
+    float hs2 = mrole ? 0.f : tile_f16_sumsq(sb + L::MA) * (pow2f(-sexp[e2]) * pow2f(-sexp[e2]));
     fence_proxy_async_smem();
     tc::fence_before_sync();
-    __syncthreads();
+    ok = __syncthreads_and(ok);
     tc::fence_after_sync();
     const uint32_t tmem = *tbase;
     constexpr uint32_t ID_K = tc::idesc_f16(128, C, false, false);   // A K-major
     constexpr uint32_t ID_T = tc::idesc_f16(128, C, true, false);    // A MN-major (transposed)
-    auto adesc_k = [&](uint32_t a, int kk) { return tc::sdesc(a + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024); };
-    auto adesc_t = [&](uint32_t a, int kk) { return tc::sdesc(a + kk * 2048, 16384, 1024); };
+    auto adesc_k = [&](int kk) { return tc::sdesc(sb + L::MA + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024); };
+    auto adesc_t = [&](int kk) { return tc::sdesc(sb + L::MA + kk * 2048, 16384, 1024); };
     auto bdesc = [&](uint32_t b, int kk) { return tc::sdesc(b + (kk >> 2) * (C * 128) + (kk & 3) * 32, 16, 1024); };
     if (tid == 0) {
         if (ok) {
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-                tc::mma_f16(tmem + 0, adesc_k(sb + L::MA, kk), bdesc(sb + L::RK, kk), ID_K, kk > 0);
-                tc::mma_f16(tmem + 32, adesc_k(sb + L::MA, kk), bdesc(sb + L::RX, kk), ID_K, kk > 0);
-                tc::mma_f16(tmem + 64, adesc_t(sb + L::MB, kk), bdesc(sb + L::RG, kk), ID_T, kk > 0);
+                if (!mrole) {
+                    tc::mma_f16(tmem + 0, adesc_k(kk), bdesc(sb + L::RK, kk), ID_K, kk > 0);    // R1
+                    tc::mma_f16(tmem + 32, adesc_k(kk), bdesc(sb + L::RX, kk), ID_K, kk > 0);   // Hx
+                } else {
+                    tc::mma_f16(tmem + 0, adesc_t(kk), bdesc(sb + L::RG, kk), ID_T, kk > 0);    // Mg
+                }
             }
         }
         tc::commit(&bars[0]);
@@ -242,160 +257,164 @@ k_bwd_rows_tc(const __grid_constant__ CUtensorMap state_map, const int *__restri
     tc::fence_after_sync();
     bool e_loaded = false;
     if (tid == 0 && ok) {
-        // phase A's products have read H_s and M_s: E^H and E^M into their tiles, landing
-        // while the phase-A results leave
-        mbar_arrive_expect_tx(&bars[4], 2 * 32768);
-        load_state_tile(&adj_map, srow, sm + L::MA, &bars[4]);
-        load_state_tile(&adj_map, srow + D, sm + L::MB, &bars[4]);
+        // the products have read the state: this role's adjoint copy into the same tile,
+        // landing while the first results leave
+        mbar_arrive_expect_tx(&bars[3], 32768);
+        load_state_tile(&adj_map, mrow, sm + L::MA, &bars[3]);
         e_loaded = true;
     }
-
-    // per-token sums over the 128 rows: this thread's 16 partials -> red[t][quarter]
-    auto token_sum = [&](float *part, float *dst, float scale, bool add) {
+    // per-token sums over the 128 rows of `np` partial vectors: red[j][t][quarter], then
+    // tokq planes p0 (+ 1)
+    auto token_sums = [&](const float *pa, const float *pb, int np, int p0) {
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
-            const float s = warp_sum(part[u]);
-            if (lane == 0) red[(wg * 16 + u) * 4 + quarter] = s;
+            const float a = warp_sum(pa[u]);
+            const float b = np > 1 ? warp_sum(pb[u]) : 0.f;
+            if (lane == 0) {
+                const int e = (wg * 16 + u) * 4 + quarter;
+                red[e] = a;
+                if (np > 1) red[128 + e] = b;
+            }
         }
         __syncthreads();
-        if (tid < C) {
-            const float s = (red[tid * 4] + red[tid * 4 + 1] + red[tid * 4 + 2] + red[tid * 4 + 3]) * scale;
-            if (ok) dst[tok0 + tid] = add ? dst[tok0 + tid] + s : s;
+        if (tid < np * C && ok) {
+            const int j = tid >> 5, tt = tid & 31;
+            const float *r4 = red + j * 128 + tt * 4;
+            tokq[(p0 + j) * plane + tok0 + tt] = r4[0] + r4[1] + r4[2] + r4[3];
         }
         __syncthreads();
     };
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(wg * 16);
-    // k, v, x of (token t, column c) from their fp16 tiles (k, v exact; x as the
-    // products saw it), y from memory
-    const float iK = 1.f / sK, iV = 1.f / sV;
-    auto k_at = [&](int t) { return f16_tile_at(sm + L::RK, t, c) * iK; };
-    auto v_at = [&](int t) { return f16_tile_at(sm + L::RV, t, c) * iV; };
+    const float iK = 1.f / sK;
+    auto k_at = [&](int tt) { return f16_tile_at(sm + L::RK, tt, c) * iK; };
     {
-        // the three products one at a time (register budget: two CTAs per SM), their
-        // per-token sums in one reduction
-        float acc[16], p1[16], p2[16], p3[16];
-        tc::tmem_ld16(tl + 0, acc);
-        tc::tmem_wait_ld();
-        const float u1 = 1.f / (sH * sK);
+        float acc[16], p1[16], p2[16];
+        if (!mrole) {
+            // R1 = H_s k -> R plane 0, uk = k . R1;  yhx = y . (H_s x)
+            tc::tmem_ld16(tl + 0, acc);
+            tc::tmem_wait_ld();
+            const float u1 = 1.f / (sS * sK);
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-            const int t = wg * 16 + u;
-            const size_t g = (tok0 + t) * D + c;
-            const float a1 = acc[u] * u1;
-            if (ok) R[g] = a1;
-            p1[u] = a1 * k_at(t);
-        }
-        tc::tmem_ld16(tl + 32, acc);
-        tc::tmem_wait_ld();
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-            const int t = wg * 16 + u;
-            const size_t g = (tok0 + t) * D + c;
-            p2[u] = acc[u] / (sH * xsc[t]) * ys[g];
-        }
-        tc::tmem_ld16(tl + 64, acc);
-        tc::tmem_wait_ld();
-        const float u3 = 1.f / (sM * sG);
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-            const int t = wg * 16 + u;
-            p3[u] = acc[u] * u3 * (f16_tile_at(sm + L::RX, t, c) / xsc[t]);
-        }
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-            const float a = warp_sum(p1[u]), b = warp_sum(p2[u]), d3 = warp_sum(p3[u]);
-            if (lane == 0) {
-                const int e = (wg * 16 + u) * 4 + quarter;
-                red[e] = a;
-                red[128 + e] = b;
-                red[256 + e] = d3;
+            for (int u = 0; u < 16; ++u) {
+                const int tt = wg * 16 + u;
+                const float a1 = acc[u] * u1;
+                if (ok) R[(tok0 + tt) * D + c] = a1;
+                p1[u] = a1 * k_at(tt);
             }
-        }
-        __syncthreads();
-        if (tid < 3 * C && ok) {
-            const int m = tid >> 5, t = tid & 31;
-            const float *r4 = red + m * 128 + t * 4;
-            tokq[m * plane + tok0 + t] = r4[0] + r4[1] + r4[2] + r4[3];
+            tc::tmem_ld16(tl + 32, acc);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int tt = wg * 16 + u;
+                p2[u] = acc[u] / (sS * xsc[tt]) * ys[(tok0 + tt) * D + c];
+            }
+            token_sums(p1, p2, 2, 0);
+        } else {
+            // gmx = x . (M_s^T g), x as the products saw it
+            tc::tmem_ld16(tl + 0, acc);
+            tc::tmem_wait_ld();
+            const float u3 = 1.f / (sS * sG);
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int tt = wg * 16 + u;
+                p1[u] = acc[u] * u3 * (f16_tile_at(sm + L::RX, tt, c) / xsc[tt]);
+            }
+            token_sums(p1, p1, 1, 2);
         }
     }
-    // phase B: the adjoint copies (2^e E) in the same tiles
-    const float sEH = pow2f(aexp[((size_t)bh * N + n) * 2]);
-    const float sEM = pow2f(aexp[((size_t)bh * N + n) * 2 + 1]);
-    if (!mbar_wait_bounded(&bars[4], 0, kTcWaitProbes)) ok = false;
+    // phase B: the adjoint copy (2^e E) in the same tile
+    const float sE = pow2f(aexp[e2 + m]);
+    if (!mbar_wait_bounded(&bars[3], 0, kTcWaitProbes)) ok = false;
     tc::fence_before_sync();
     ok = __syncthreads_and(ok);
     tc::fence_after_sync();
-    if (tid == 0 && ok) {
+    if (tid == 0) {
+        if (ok) {
+            if (!mrole) {
+                // R2 = (E^H + E^H^T) k
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            tc::mma_f16(tmem + 96, adesc_k(sb + L::MA, kk), bdesc(sb + L::RK, kk), ID_K, kk > 0);
-            tc::mma_f16(tmem + 128, adesc_t(sb + L::MB, kk), bdesc(sb + L::RV, kk), ID_T, kk > 0);
-            tc::mma_f16(tmem + 160, adesc_k(sb + L::MB, kk), bdesc(sb + L::RK, kk), ID_K, kk > 0);
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_f16(tmem + 64, adesc_k(kk), bdesc(sb + L::RK, kk), ID_K, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_f16(tmem + 64, adesc_t(kk), bdesc(sb + L::RK, kk), ID_T, true);
+            } else {
+                // R3 = E^M^T v, R4 = E^M k
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    tc::mma_f16(tmem + 32, adesc_t(kk), bdesc(sb + L::RV, kk), ID_T, kk > 0);
+                    tc::mma_f16(tmem + 64, adesc_k(kk), bdesc(sb + L::RK, kk), ID_K, kk > 0);
+                }
+            }
         }
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-            tc::mma_f16(tmem + 96, adesc_t(sb + L::MA, kk), bdesc(sb + L::RK, kk), ID_T, true);
+        tc::commit(&bars[1]);
     }
-    if (tid == 0) tc::commit(&bars[1]);
     if (!mbar_wait_bounded(&bars[1], 0, kTcWaitProbes)) ok = false;
     tc::fence_after_sync();
     {
         float acc[16], part[16];
-        tc::tmem_ld16(tl + 96, acc);
-        tc::tmem_wait_ld();
-        const float u2 = 1.f / (sEH * sK), u3 = 1.f / (sEM * sV), u4 = 1.f / (sEM * sK);
+        if (!mrole) {
+            // R2 -> plane 1, qe's H part = k . R2 / 2 -> tokq plane 3
+            tc::tmem_ld16(tl + 64, acc);
+            tc::tmem_wait_ld();
+            const float u2 = 1.f / (sE * sK);
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-            const size_t g = (tok0 + wg * 16 + u) * D + c;
-            const float a2 = acc[u] * u2;
-            if (ok) R[RD + g] = a2;
-            part[u] = 0.5f * a2 * k_at(wg * 16 + u);
-        }
-        tc::tmem_ld16(tl + 128, acc);
-        tc::tmem_wait_ld();
+            for (int u = 0; u < 16; ++u) {
+                const int tt = wg * 16 + u;
+                const float a2 = acc[u] * u2;
+                if (ok) R[RD + (tok0 + tt) * D + c] = a2;
+                part[u] = 0.5f * a2 * k_at(tt);
+            }
+            token_sums(part, part, 1, 3);
+        } else {
+            // R3 -> plane 2, R4 -> plane 3, qe's M part = v . R4 -> tokq plane 4
+            const float iV = 1.f / sV;
+            tc::tmem_ld16(tl + 32, acc);
+            tc::tmem_wait_ld();
+            const float u3 = 1.f / (sE * sV), u4 = 1.f / (sE * sK);
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-            const size_t g = (tok0 + wg * 16 + u) * D + c;
-            if (ok) R[2 * RD + g] = acc[u] * u3;
-        }
-        tc::tmem_ld16(tl + 160, acc);
-        tc::tmem_wait_ld();
+            for (int u = 0; u < 16; ++u) {
+                const int tt = wg * 16 + u;
+                if (ok) R[2 * RD + (tok0 + tt) * D + c] = acc[u] * u3;
+            }
+            tc::tmem_ld16(tl + 64, acc);
+            tc::tmem_wait_ld();
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-            const size_t g = (tok0 + wg * 16 + u) * D + c;
-            const float a4 = acc[u] * u4;
-            if (ok) R[3 * RD + g] = a4;
-            part[u] = fmaf(a4, v_at(wg * 16 + u), part[u]);
+            for (int u = 0; u < 16; ++u) {
+                const int tt = wg * 16 + u;
+                const float a4 = acc[u] * u4;
+                if (ok) R[3 * RD + (tok0 + tt) * D + c] = a4;
+                part[u] = a4 * (f16_tile_at(sm + L::RV, tt, c) * iV);
+            }
+            token_sums(part, part, 1, 4);
         }
-        token_sum(part, tokq + 3 * plane, 1.f, false);
     }
-    // chunk scalars: hs2, and eh from the adjoint pass's two inner products
-    {
+    if (!mrole) {
+        // chunk scalars: hs2, and eh from the adjoint pass's two inner products
         hs2 = warp_sum(hs2);
         if (lane == 0) mred[warp] = hs2;
         __syncthreads();
         if (tid == 0 && ok) {
-            float s = 0.f;
-            for (int w = 0; w < 8; ++w) s += mred[w];
-            const size_t e = ((size_t)bh * N + n) * 2;
-            chq[e] = s;
-            chq[e + 1] = eh_part[e] + eh_part[e + 1];
+            float s2 = 0.f;
+            for (int w = 0; w < 8; ++w) s2 += mred[w];
+            chq[e2] = s2;
+            chq[e2 + 1] = eh_part[e2] + eh_part[e2 + 1];
         }
     }
     if (!ok && tid == 0) {
         // a wait gave up: flag it, and let every MMA this CTA issued finish before TMEM
         // is released (a commit after them, waited for with a bound)
         atomicExch(timeout_flag, 1);
-        tc::commit(&bars[2]);
-        mbar_wait_bounded(&bars[2], 0, kTcWaitProbes);
-        mbar_wait_bounded(&bars[3], 0, kTcWaitProbes);   // the state tiles' loads
-        if (e_loaded) mbar_wait_bounded(&bars[4], 0, kTcWaitProbes);
+        tc::commit(&bars[4]);
+        mbar_wait_bounded(&bars[4], 0, kTcWaitProbes);
+        mbar_wait_bounded(&bars[2], 0, kTcWaitProbes);   // the state tile's loads
+        if (e_loaded) mbar_wait_bounded(&bars[3], 0, kTcWaitProbes);
     }
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 0) {
         tc::fence_after_sync();
-        tc::tmem_dealloc(tmem, 256);
+        tc::tmem_dealloc(tmem, 128);
     }
 }
 

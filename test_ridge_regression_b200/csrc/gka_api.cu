@@ -436,7 +436,9 @@ static int bwd_layout(int B, int H, int T, int D, int C, gka_dtype dt, BwdLayout
     L->cvec = off; off = round256(off + sizeof(float) * BH * T);
     L->adj = off;  off = round256(off + sizeof(float) * BH * (N + 1) * 2 * D * D);
     L->rows = off; off = round256(off + 4 * sizeof(float) * TD);
-    L->tokq = off; off = round256(off + 4 * sizeof(float) * BH * T);
+    // per-token scalars uk, yhx, gmx, qe (the tensor-core row kernel writes qe's H and M
+    // parts as planes 3 and 4)
+    L->tokq = off; off = round256(off + 5 * sizeof(float) * BH * T);
     L->chq = off;  off = round256(off + 2 * sizeof(float) * BH * N);
     L->tc_recompute = tensor_core_path(D, 64, dt) && T % 64 == 0;
     L->tc = off;
@@ -621,7 +623,7 @@ static int backward_simt(const Tin *q, const Tin *k, const Tin *v, const float *
             if ((e = set_smem(k_bwd_rows_tc, BwdRowsTcSmem::bytes)) != cudaSuccess)
                 return cuda_fail(e);
             { ProfScope ps(GKA_KERNEL_BWD_ROWS, s);
-            k_bwd_rows_tc<<<dim3(N, BH), kSimtThreads, BwdRowsTcSmem::bytes, s>>>(
+            k_bwd_rows_tc<<<dim3(N, BH, 2), kSimtThreads, BwdRowsTcSmem::bytes, s>>>(
                 state_map, sexp32, adj_map, alp, aexp, ehp, k, v, dout, xs, ys, rows, tokq, chq,
                 T, N, flag); }
             if (int rc = check_launch()) return rc;

@@ -124,7 +124,7 @@ k_bwd_grads_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restr
         s_uk[tid] = tokq[tok0 + tid];
         s_yhx[tid] = tokq[plane + tok0 + tid];
         s_gmx[tid] = tokq[2 * plane + tok0 + tid];
-        s_qe[tid] = tokq[3 * plane + tok0 + tid];
+        s_qe[tid] = tokq[3 * plane + tok0 + tid] + tokq[4 * plane + tok0 + tid];   // H, M parts
         s_bm1[tid] = tid == 0 ? 1.f : decay_exp(ell[tid - 1]);
     }
     // W[l][s] = w_sl for s >= l, else 0
