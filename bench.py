@@ -38,17 +38,20 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # bench reports null.  The captures' commands sit beside their summaries.
 TRAFFIC = {
     # full-size forward workload (B8 H8 T2048 D128, chunk 64), one launch
-    "chunk_solve_tc": {"bytes": 237.150208e6 + 24.922368e6, "workload": "bf16_b8h8t2048d128",
+    "chunk_solve_tc": {"bytes": 237.094912e6 + 23.748096e6, "workload": "bf16_b8h8t2048d128",
                        "src": "test_ridge_regression_b200/csrc/solve_tc.cuh",
-                       "sha1": "286fdd815b3667d7662765cf1a59620fe4837263"},
-    "state_pass_tc": {"bytes": 67.709184e6 + 80.409600e6, "workload": "bf16_b8h8t2048d128",
+                       "sha1": "1da5f1a4b43087afd2a12ecc7601e5093ecbd7b9"},
+    "state_pass_tc": {"bytes": 67.716864e6 + 79.924480e6, "workload": "bf16_b8h8t2048d128",
                       "src": "test_ridge_regression_b200/csrc/state_tc.cuh",
-                      "sha1": "3eca50dc232392420fce4b8be90af9a2dbb55376"},
-    # backward row products captured at B2 H8 T2048 (1024 chunks), scaled x4 to the
-    # 4096 chunks of the full workload (per-chunk traffic does not depend on B)
-    "bwd_rows_tc": {"bytes": 4 * (397.614848e6 + 72.314624e6), "workload": "bf16_b8h8t2048d128",
+                      "sha1": "557968b9a4b4f6da6d895bc493988a8c16af285f"},
+    # backward kernels captured at B2 H8 T2048 (1024 chunks, 16 heads), scaled x4 to the
+    # full workload (the row kernel's traffic is per chunk, the adjoint pass's per head)
+    "bwd_rows_tc": {"bytes": 4 * (217.920256e6 + 43.090176e6), "workload": "bf16_b8h8t2048d128",
                     "src": "test_ridge_regression_b200/csrc/backward_tc.cuh",
-                    "sha1": "bae7a862a52575dedb40425feeb40e75c13d8c07"},
+                    "sha1": "50f080436884c190a86638f2c0973e7abbb3e2a1"},
+    "adjoint_pass_tc": {"bytes": 4 * (117.779968e6 + 37.594880e6), "workload": "bf16_b8h8t2048d128",
+                        "src": "test_ridge_regression_b200/csrc/adjoint_tc.cuh",
+                        "sha1": "4db525379c92ee230b2b00e0fe772ab42443cecc"},
     # decode captured on 64 x 32 heads (state above L2), scaled x4 to 256 x 32 heads
     "decode_step": {"bytes": 4 * (270.045952e6 + 209.251584e6), "workload": "decode_bf16_b256h32d128",
                     "src": "test_ridge_regression_b200/csrc/decode.cuh",
