@@ -75,6 +75,12 @@ struct AdjSmem {
     static constexpr size_t bytes = END + 1024;             // + alignment slack
 };
 
+// Largest of a non-negative float over the warp: the bit patterns of non-negative
+// floats order like unsigned integers, so one integer reduction does it.
+__device__ __forceinline__ float warp_max_nonneg(float x) {
+    return __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(x)));
+}
+
 // Exponent e of the power of two inv_pow2_above returns (x * 2^e lies in [1/2, 1)).
 __device__ __forceinline__ int inv_pow2_exponent(float x) {
     return ((__float_as_int(inv_pow2_above(x)) >> 23) & 0xff) - 127;
@@ -312,10 +318,7 @@ k_adjoint_pass_tc(const __grid_constant__ AdjMaps maps, const float *__restrict_
             }
         }
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1)
-                mx4[q] = fmaxf(mx4[q], __shfl_xor_sync(0xffffffffu, mx4[q], o));
+        for (int q = 0; q < 4; ++q) mx4[q] = warp_max_nonneg(mx4[q]);
         if (lane == 0)
             *reinterpret_cast<float4 *>(s_mx + warp * 4) = make_float4(mx4[0], mx4[1], mx4[2], mx4[3]);
         named_barrier_sync(1, kAdjEpiThreads);
@@ -325,15 +328,15 @@ k_adjoint_pass_tc(const __grid_constant__ AdjMaps maps, const float *__restrict_
             for (int q = 0; q < 16; ++q) s += s_eh[q];
             eh_part[((size_t)bh * N + n + 1) * 2 + m] = s;
         }
-        float MX = 0.f, MY = 0.f, MK = 0.f, ME = 0.f, EM = 0.f;
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-            const float4 v = *reinterpret_cast<const float4 *>(s_mx + q * 4);
-            MX = fmaxf(MX, v.x);
-            MY = fmaxf(MY, v.y);
-            MK = fmaxf(MK, v.z);
-            ME = fmaxf(ME, v.w);
-            EM = fmaxf(EM, s_emx[q]);
+        // the 16 warps' maxima: lane l reads warp l % 16's, one reduction each
+        float MX, MY, MK, ME, EM;
+        {
+            const float4 v = *reinterpret_cast<const float4 *>(s_mx + (lane & 15) * 4);
+            MX = warp_max_nonneg(v.x);
+            MY = warp_max_nonneg(v.y);
+            MK = warp_max_nonneg(v.z);
+            ME = warp_max_nonneg(v.w);
+            EM = warp_max_nonneg(s_emx[lane & 15]);
         }
         // pass 2: the fp16 operand tiles (single-buffered: the previous chunk's products
         // were waited for before its update)
@@ -430,8 +433,7 @@ k_adjoint_pass_tc(const __grid_constant__ AdjMaps maps, const float *__restrict_
                 E[e] = fmaf(dl[e], unscale, E[e]);
                 mx = fmaxf(mx, fabsf(E[e]));
             }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            mx = warp_max_nonneg(mx);
             if (lane == 0) s_emx[warp] = mx;
         }
         tc::fence_before_sync();
