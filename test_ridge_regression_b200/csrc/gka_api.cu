@@ -370,7 +370,9 @@ static int forward_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
-        cfg.numAttrs = (!solve_only || (ext && ext->pdl)) ? 1 : 0;
+        // 128-token chunks: one CTA per SM, and the early CTAs gained nothing (A/B on one
+        // box: 3.5577 against 3.5466 ms median on B1 H8 T131072), so plain order there
+        cfg.numAttrs = (C == 64 && (!solve_only || (ext && ext->pdl))) ? 1 : 0;
         return cudaLaunchKernelEx(&cfg, kern, maps, q, gate, (const float *)tokdec, plane, norms,
                                   sexp_solve, o, x_out, T, N, C, P, flag, sstride);
     };
