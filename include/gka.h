@@ -237,11 +237,12 @@ int gka_decode_step_gated(float *state, const void *q, const void *k, const void
  * carried back through the decayed, write-gated recurrence to dk, dv, dbeta
  * and dgate.  It recomputes the forward quantities it needs (chunk states,
  * norms, iterates) itself.  With bf16 inputs, D = 128, chunk 32 and T a
- * multiple of 64 the recompute, both Chebyshev solves, the chunk and adjoint
- * increments, u = M_t^T g_t and the row products run on the tensor cores
- * (fp16 operands with power-of-two scales, fp32 accumulation) and the scans
- * and final gradients in fp32 on CUDA cores; otherwise every step runs on
- * CUDA cores in fp32.
+ * multiple of 64 every product runs on the tensor cores (fp16 operands with
+ * power-of-two scales, fp32 accumulation, fp32 sums and recurrences): one
+ * chunk-state pass, both Chebyshev solves, u = M_t^T g_t, the adjoint states
+ * (increments and reverse scan in one pass per head), the row products and
+ * the gradients' intra-chunk products; otherwise every step runs on CUDA
+ * cores in fp32.
  *   q, k, v, beta, gate  the forward's inputs (gate nullable)
  *   dout        [B, H, T, D] in `dt`: dL/do
  *   dq, dk, dv  [B, H, T, D] in `dt` (written)
@@ -323,9 +324,13 @@ enum {
     GKA_KERNEL_DECODE_STEP = 4,   /* recurrent decode step */
     GKA_KERNEL_CHUNK_SOLVE_TC = 5,/* Chebyshev solve + readout on tensor cores (tcgen05) */
     GKA_KERNEL_STATE_PASS_TC = 6, /* chunk-state increments and scan in one pass (tcgen05) */
-    GKA_KERNEL_BWD_SOLVE = 7,     /* backward: u = M^T dL/do and the Chebyshev solve for dq */
-    GKA_KERNEL_BWD_DELTA = 8,     /* backward: per-chunk increments of the adjoint state */
-    GKA_KERNEL_ADJOINT_SCAN = 9,  /* backward: adjoint states, last chunk first */
+    GKA_KERNEL_BWD_SOLVE = 7,     /* backward: u = M^T dL/do and the Chebyshev solve for dq
+                                     (tensor-core path: u and dq's finish; the solve itself
+                                     counts as GKA_KERNEL_CHUNK_SOLVE_TC) */
+    GKA_KERNEL_BWD_DELTA = 8,     /* backward, CUDA-core path: per-chunk increments of the
+                                     adjoint state */
+    GKA_KERNEL_ADJOINT_SCAN = 9,  /* backward: adjoint states, last chunk first (tensor-core
+                                     path: increments and scan in one pass per head) */
     GKA_KERNEL_BWD_ROWS = 10,     /* backward: chunk rows against H_s, M_s and the adjoints */
     GKA_KERNEL_BWD_GRADS = 11,    /* backward: dk, dv, dbeta, dgate of each chunk */
     GKA_KERNEL_SOLVER_STUDY = 12, /* solver study: residual histories */
