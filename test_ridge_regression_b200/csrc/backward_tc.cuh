@@ -492,7 +492,7 @@ k_bwd_u_tc(const __grid_constant__ CUtensorMap state_map, const int *__restrict_
     }
     __syncthreads();
     bool ok = mbar_wait_bounded(&bars[0], 0, kTcWaitProbes);
-    chunk_log_prefix(s_beta, C, ell, wtot);
+    chunk_log_prefix_f32log(s_beta, C, ell, wtot);
     if (tid < C) {
         s_b[tid] = decay_exp(ell[tid]);
         s_sg[tid] = gate ? sqrtf(s_gate[tid]) : 1.f;

@@ -59,6 +59,28 @@ __device__ __forceinline__ void chunk_log_prefix(const float *beta, int C, doubl
     __syncthreads();
 }
 
+// chunk_log_prefix with log(beta) in fp32 (the cumulative sum still in double), as the
+// tensor-core state pass forms its decays; beta may be in shared or global memory.
+__device__ __forceinline__ void chunk_log_prefix_f32log(const float *beta, int C, double *ell,
+                                                        double *wtot) {
+    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+    double x = 0.0;
+    if (t < C) x = fmax((double)logf(beta[t]), kLogBetaMin);
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        double y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) wtot[w] = x;
+    __syncthreads();
+    if (t < C) {
+        double add = 0.0;
+        for (int i = 0; i < w; ++i) add += wtot[i];
+        ell[t] = x + add;
+    }
+    __syncthreads();
+}
+
 // exp of a (non-positive) difference of cumulative logs, evaluated in fp32.
 __device__ __forceinline__ float decay_exp(double d) { return expf((float)d); }
 

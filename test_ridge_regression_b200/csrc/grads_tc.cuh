@@ -22,8 +22,8 @@
 //   - the row outputs are M = 128 (column c), N = 32 (token l), K = 32 (token s) MMAs
 //     with the same row tiles read MN-major and the coefficient tiles (fp16, K-major,
 //     the row scales folded in) as B; A0's three products share one power-of-two scale.
-// Warp 1 runs the dbeta recurrences while the other warps form the coefficient tiles;
-// thread 0 issues every MMA.
+// Warps 1 and 3 form dbeta (its prefix sums over the chunk as 32 x 32 matrix products)
+// while the other warps form the coefficient tiles; thread 0 issues every MMA.
 // grid (N, B*H), block 256.
 #pragma once
 
@@ -112,7 +112,7 @@ k_bwd_grads_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restr
         ya[r] = *reinterpret_cast<const float4 *>(ys + g);
         yb[r] = *reinterpret_cast<const float4 *>(ys + g + 4);
     }
-    chunk_log_prefix(beta + tok0, C, ell, wtot);
+    chunk_log_prefix_f32log(beta + tok0, C, ell, wtot);
     const float hs2 = chq[((size_t)bh * N + n) * 2], eh = chq[((size_t)bh * N + n) * 2 + 1];
     if (tid < C) {
         const ChunkDecays dc = chunk_decays(ell, C, tid);
@@ -232,63 +232,114 @@ k_bwd_grads_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restr
     }
     tc::fence_before_sync();
     ok = __syncthreads_and(ok);
-    if (warp == 1) {
+    if (warp == 1 || warp == 3) {
         // dbeta_j = sum_{s>=j} w_sj Phi[j][s] + (adjoint from later chunks), with
-        //   Phi[j][s] = -y_s^T H_{j-1} x_s - c_s <H_s, H_{j-1}> + g_s^T M_{j-1} x_s,
-        // by prefix recurrences over j <= s (lane s), then sums over s (lane j).
+        //   Phi[j][s] = -y_s^T H_{j-1} x_s - c_s <H_s, H_{j-1}> + g_s^T M_{j-1} x_s
+        // (H_s the state at token s, H_{j-1} the one before token j, H_{-1} = H_start),
+        // through the prefix sums over i < j of its terms, as matrix products over the
+        // chunk (warps 1 and 3, thread dt: rows 8r + dt / 8, columns 8q + dt % 8):
+        //   Q  = (w o GK^2 o w)^T W,         Q[i][s] = sum_{l<=s} w_sl w_l w_i (k_l . k_i)^2,
+        //   T1 = L (w o KY o KX),  T2 = L Q,  T3 = L (w o VG o KX),  L[j][i] = w_{j-1,i} (i < j),
+        //   u1 = L (w o uk),  qe = L (w o qe),
+        //   Phi[j][s] = -(b_{j-1} yhx_s + T1) - c_s (b_s b_{j-1} hs2 + b_s u1_j + b_{j-1} X1_s + T2)
+        //               + (b_{j-1} gmx_s + T3)
+        const int dt = (warp == 1 ? 0 : 32) + lane, r0 = dt >> 3, q0 = dt & 7;
         {
-            const int i = lane;   // Q[i][s] = sum_{l<=s} w_sl w_l w_i (k_l . k_i)^2
-            float qv = 0.f;
-#pragma unroll 8
-            for (int s2 = 0; s2 < C; ++s2) {
-                const float g2 = GK[s2 * CP + i];
-                qv = fmaf(s2 == 0 ? 0.f : s_step[s2], qv, s_w[s2] * s_w[i] * g2 * g2);
-                Qm[i * CP + s2] = qv;
-            }
-        }
-        __syncwarp();
-        {
-            // a fixed trip count (entries j > s are formed and dropped) so that the
-            // loads of several steps are issued together
-            const int s2 = lane;
-            float t1 = 0.f, t2 = 0.f, t3 = 0.f, u1 = 0.f;
-#pragma unroll 8
-            for (int jj = 0; jj < C; ++jj) {
-                if (jj > 0) {
-                    const int i = jj - 1;
-                    const float st = s_step[i];
-                    t1 = fmaf(st, t1, s_w[i] * KY[i * CP + s2] * KX[i * CP + s2]);
-                    t3 = fmaf(st, t3, s_w[i] * VG[i * CP + s2] * KX[i * CP + s2]);
-                    t2 = fmaf(st, t2, Qm[i * CP + s2]);
-                    u1 = fmaf(st, u1, s_w[i] * s_uk[i]);
+            float acc[4][4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) acc[r][q] = 0.f;
+#pragma unroll 4
+            for (int l = 0; l < C; ++l) {
+                const float wl = s_w[l];
+                float g2[4], wt[4];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const float g = GK[l * CP + r0 + 8 * r];
+                    g2[r] = wl * g * g;
                 }
-                const float bm = s_bm1[jj];
-                const float phi = -(bm * s_yhx[s2] + t1)
-                                  - s_c[s2] * (s_b[s2] * bm * hs2 + s_b[s2] * u1 + bm * s_X1[s2] + t2)
-                                  + (bm * s_gmx[s2] + t3);
-                if (jj <= s2) PH[jj * CP + s2] = Wt[jj * CP + s2] * phi;   // w_sj Phi[j][s]
+#pragma unroll
+                for (int q = 0; q < 4; ++q) wt[q] = Wt[l * CP + q0 + 8 * q];
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) acc[r][q] = fmaf(g2[r], wt[q], acc[r][q]);
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int i = r0 + 8 * r;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) Qm[i * CP + q0 + 8 * q] = s_w[i] * acc[r][q];
             }
         }
-        __syncwarp();
+        named_barrier_sync(3, 64);
         {
-            const int jj = lane;
-            float acc = 0.f;
-#pragma unroll 8
-            for (int s2 = 0; s2 < C; ++s2)
-                if (s2 >= jj) acc += PH[jj * CP + s2];
-            // the adjoint from later chunks: w_{C-1,j} (b_{j-1} eh + sum_{i<j} w_{j-1,i} w_i qe_i)
-            float qe = 0.f;
-#pragma unroll 8
-            for (int i = 0; i < C; ++i)
-                if (i < jj) qe = fmaf(s_step[i], qe, s_w[i] * s_qe[i]);
-            acc = fmaf(s_wend[jj], fmaf(s_bm1[jj], eh, qe), acc);
-            if (ok) dbeta[tok0 + jj] = acc;
+            float t1[4][4], t2[4][4], t3[4][4], u1[4], qe[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                u1[r] = qe[r] = 0.f;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) t1[r][q] = t2[r][q] = t3[r][q] = 0.f;
+            }
+#pragma unroll 2
+            for (int i = 0; i < C; ++i) {
+                const float wi = s_w[i];
+                float lm[4], a1[4], a3[4], qm[4];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const int j = r0 + 8 * r;
+                    lm[r] = j >= 1 ? Wt[i * CP + j - 1] : 0.f;   // 0 unless i <= j - 1
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int s2 = q0 + 8 * q;
+                    const float kx = KX[i * CP + s2];
+                    a1[q] = wi * KY[i * CP + s2] * kx;
+                    a3[q] = wi * VG[i * CP + s2] * kx;
+                    qm[q] = Qm[i * CP + s2];
+                }
+                const float wuk = wi * s_uk[i], wqe = wi * s_qe[i];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    u1[r] = fmaf(lm[r], wuk, u1[r]);
+                    qe[r] = fmaf(lm[r], wqe, qe[r]);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        t1[r][q] = fmaf(lm[r], a1[q], t1[r][q]);
+                        t2[r][q] = fmaf(lm[r], qm[q], t2[r][q]);
+                        t3[r][q] = fmaf(lm[r], a3[q], t3[r][q]);
+                    }
+                }
+            }
+            // w_sj Phi[j][s] over this thread's columns, summed along the row, then over
+            // the 8 threads of the row (consecutive lanes)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int j = r0 + 8 * r;
+                const float bm = s_bm1[j];
+                float rs = 0.f;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int s2 = q0 + 8 * q;
+                    const float phi = -(bm * s_yhx[s2] + t1[r][q])
+                                      - s_c[s2] * (s_b[s2] * bm * hs2 + s_b[s2] * u1[r] +
+                                                   bm * s_X1[s2] + t2[r][q])
+                                      + (bm * s_gmx[s2] + t3[r][q]);
+                    rs += Wt[j * CP + s2] * phi;   // 0 for s < j
+                }
+                rs += __shfl_xor_sync(0xffffffffu, rs, 1);
+                rs += __shfl_xor_sync(0xffffffffu, rs, 2);
+                rs += __shfl_xor_sync(0xffffffffu, rs, 4);
+                // the adjoint from later chunks: w_{C-1,j} (b_{j-1} eh + sum_{i<j} w_{j-1,i} w_i qe_i)
+                if (q0 == 0 && ok) dbeta[tok0 + j] = fmaf(s_wend[j], fmaf(bm, eh, qe[r]), rs);
+            }
         }
     } else {
-        // warps 0, 2..7: the coefficient tiles, two adjacent s per item, with the row
+        // warps 0, 2, 4..7: the coefficient tiles, two adjacent s per item, with the row
         // scales of the A operand folded in (B[l][s] = P[l][s] pi / sigma_s)
-        constexpr int NT = kSimtThreads - 32;
-        const int me = tid < 32 ? tid : tid - 32;
+        constexpr int NT = kSimtThreads - 64;
+        const int me = warp == 0 ? lane : (warp == 2 ? 32 + lane : tid - 64);
         auto coef = [&](int l, int s2, float *p4) {
             const float w = Wt[l * CP + s2];
             const float kx = KX[l * CP + s2];
@@ -322,7 +373,7 @@ k_bwd_grads_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restr
         ma = mg = 0.f;
 #pragma unroll
         for (int w = 0; w < 8; ++w) {
-            if (w == 1) continue;
+            if (w == 1 || w == 3) continue;
             ma = fmaxf(ma, mred[w * 2]);
             mg = fmaxf(mg, mred[w * 2 + 1]);
         }
@@ -369,11 +420,23 @@ k_bwd_grads_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restr
         }
     }
     ok = __syncthreads_and(ok);
+    // epilogue: thread (column c = TMEM lane, tokens 16 wg .. 16 wg + 15); the row
+    // products R1..R4 of 8 tokens at a time are loaded before they are used (the first 8
+    // while the row outputs finish)
+    const int quarter = warp & 3, wg = warp >> 2, c = quarter * 32 + lane;
+    float rr[4][8];
+    auto load_r = [&](int u0) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const size_t g = (tok0 + wg * 16 + u0 + u) * D + c;
+#pragma unroll
+            for (int p = 0; p < 4; ++p) rr[p][u] = R[p * RD + g];
+        }
+    };
+    load_r(0);
     if (!mbar_wait_bounded(&bars[1], 0, kTcWaitProbes)) ok = false;
     tc::fence_after_sync();
-    // epilogue: thread (column c = TMEM lane, tokens 16 wg .. 16 wg + 15)
     {
-        const int quarter = warp & 3, wg = warp >> 2, c = quarter * 32 + lane;
         const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(wg * 16);
         float a0[16], b0[16];
         tc::tmem_ld16(tl + 128, a0);
@@ -382,11 +445,13 @@ k_bwd_grads_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restr
         const float ua = 1.f / mred[16], ug = 1.f / mred[17];
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
+            if (u == 8) load_r(8);
             const int l = wg * 16 + u;
             const size_t g = (tok0 + l) * D + c;
-            float a = fmaf(-2.f * s_f[l], R[g], a0[u] * ua);
-            a = fmaf(s_wend[l], R[RD + g] + R[2 * RD + g], a);
-            const float bb = fmaf(s_wend[l], R[3 * RD + g], b0[u] * ug);
+            const int ur = u & 7;
+            float a = fmaf(-2.f * s_f[l], rr[0][ur], a0[u] * ua);
+            a = fmaf(s_wend[l], rr[1][ur] + rr[2][ur], a);
+            const float bb = fmaf(s_wend[l], rr[3][ur], b0[u] * ug);
             if (ok) {
                 dk[g] = __float2bfloat16_rn(s_w[l] * a);
                 dv[g] = __float2bfloat16_rn(s_w[l] * bb);
