@@ -15,8 +15,9 @@
 //   <E^M, M_s> (the adjoint pass forms both terms from its fp32 adjoints).
 // Every copy's largest entry lies below 2^14 (states) or 1 (adjoints); k, v, g tiles
 // are converted in shared memory with one power-of-two scale each, x with one per
-// token.  The accumulators are fp32.  Two phases share the matrix tiles: (H_s, M_s),
-// then (E^H, E^M), loaded once the first phase's products have read the states.
+// token.  The accumulators are fp32.  Two CTAs serve a chunk, one per matrix (H: R1,
+// Hx, R2; M: Mg, R3, R4), each with one matrix tile: the state copy, then the adjoint
+// copy loaded into it once the first products have read the state.
 #pragma once
 
 #include <cuda_fp16.h>
