@@ -43,8 +43,8 @@ struct BwdGradTcSmem {
     static constexpr uint32_t HALF = 20480;                 // one 64-column half: 160 rows
     static constexpr uint32_t RGN = 0;                      // [2][160][64] fp16 rows X Y K G V
     static constexpr uint32_t PT = RGN + 2 * HALF;          // 4 x [32][64] fp16: Py Px Pk Pg
-    static constexpr uint32_t MAT = PT + 4 * 4096;          // 7 x float[32][33]: KX KY VG GK Q PHI W
-    static constexpr uint32_t SIG = MAT + 7 * 32 * 33 * 4;  // float[5][32] inverse row scales x y k g v
+    static constexpr uint32_t MAT = PT + 4 * 4096;          // 6 x float[32][33]: KX KY VG GK Q W
+    static constexpr uint32_t SIG = MAT + 6 * 32 * 33 * 4;  // float[5][32] inverse row scales x y k g v
     static constexpr uint32_t SCAL = SIG + 5 * 128;         // float[13][32] per-token scalars
     static constexpr uint32_t RED = SCAL + 13 * 128;        // float[32][4] token sums
     static constexpr uint32_t MRED = RED + 512;             // float[8][2] maxima, 2 scales
@@ -69,7 +69,7 @@ k_bwd_grads_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restr
     uint8_t *sm = smem_align1024(smraw);
     const uint32_t sb = smem_u32(sm);
     float *KX = reinterpret_cast<float *>(sm + L::MAT), *KY = KX + C * CP, *VG = KY + C * CP,
-          *GK = VG + C * CP, *Qm = GK + C * CP, *PH = Qm + C * CP, *Wt = PH + C * CP;
+          *GK = VG + C * CP, *Qm = GK + C * CP, *Wt = Qm + C * CP;
     float *isig = reinterpret_cast<float *>(sm + L::SIG);   // 1 / row scale: x y k g v
     float *sc = reinterpret_cast<float *>(sm + L::SCAL);
     float *s_b = sc, *s_step = sc + 32, *s_wend = sc + 64, *s_w = sc + 96, *s_c = sc + 128,
