@@ -46,9 +46,9 @@ TRAFFIC = {
                       "sha1": "557968b9a4b4f6da6d895bc493988a8c16af285f"},
     # backward kernels captured at B2 H8 T2048 (1024 chunks, 16 heads), scaled x4 to the
     # full workload (the row kernel's traffic is per chunk, the adjoint pass's per head)
-    "bwd_rows_tc": {"bytes": 4 * (217.920256e6 + 43.090176e6), "workload": "bf16_b8h8t2048d128",
+    "bwd_rows_tc": {"bytes": 4 * (217.924608e6 + 43.453184e6), "workload": "bf16_b8h8t2048d128",
                     "src": "test_ridge_regression_b200/csrc/backward_tc.cuh",
-                    "sha1": "50f080436884c190a86638f2c0973e7abbb3e2a1"},
+                    "sha1": "3766bfe51b74e452ca5370b9372efe91b296beec"},
     "adjoint_pass_tc": {"bytes": 4 * (117.882624e6 + 38.258432e6), "workload": "bf16_b8h8t2048d128",
                         "src": "test_ridge_regression_b200/csrc/adjoint_tc.cuh",
                         "sha1": "bcd3ef1e1b540648f212e8dd8eb7ac785171869a"},
