@@ -2,11 +2,11 @@
 ABI) against the float64 oracle's backward on the same seeded inputs.
 
 Metric: max over (batch, head) of the relative Frobenius error over the head's
-slab, for dq, dk, dv ([T, D]) and dbeta, dgate ([T]).  The backward computes in
-fp32 on CUDA cores; with bf16 inputs, D = 128 and T a multiple of 64 it takes the
-forward iterates and norms from the tensor-core forward (fp16 operands), so its
-gradients carry that forward's bf16-level error.  Bars: 1e-4 with fp32 inputs,
-2e-2 with bf16 inputs (dq, dk, dv are also rounded to bf16).
+slab, for dq, dk, dv ([T, D]) and dbeta, dgate ([T]).  With bf16 inputs, D = 128,
+chunk 32 and T a multiple of 64 every product of the backward runs on the tensor
+cores (fp16 operands with power-of-two scales, fp32 accumulation); otherwise it
+computes in fp32 on CUDA cores.  Bars: 1e-4 with fp32 inputs, 2e-2 with bf16 inputs
+(dq, dk, dv are also rounded to bf16).
 """
 import numpy as np
 import pytest
@@ -30,8 +30,9 @@ def _dout(shape, dtype, seed):
     return torch.randn(*shape, generator=g).to(dtype)
 
 
-def check_backward(q, k, v, beta, a, r, C, gate=None, seed=0):
-    dout = _dout(q.shape, q.dtype, 9000 + seed)
+def check_backward(q, k, v, beta, a, r, C, gate=None, seed=0, dout=None):
+    if dout is None:
+        dout = _dout(q.shape, q.dtype, 9000 + seed)
     dev = cuda(q, k, v, beta, dout)
     gd = gate.cuda() if gate is not None else None
     got = gka.gka_backward(dev[0], dev[1], dev[2], dev[3], dev[4], a, r, C, gate=gd)
@@ -74,6 +75,28 @@ def test_backward_bf16_state_pass_gate_resets():
     gate[0, 3, 10:20] = 0.0
     beta[0, 5, 64] = 0.0
     check_backward(q, k, v, beta, 0.5, 20, 32, gate=gate, seed=8)
+
+
+def test_backward_bf16_zero_upstream_gradient():
+    # dL/do = 0: u, y, every adjoint (and its fp16 copy) and every intra-chunk product
+    # vanish, so every gradient is exactly zero (all-zero tiles take the scale 1)
+    q, k, v, beta = make_inputs(1, 4, 128, 128, torch.bfloat16, 3.0, 1.0, seed=823)
+    gate = make_gate((1, 4, 128), 823)
+    dev = cuda(q, k, v, beta)
+    dout = torch.zeros_like(dev[0])
+    got = gka.gka_backward(dev[0], dev[1], dev[2], dev[3], dout, 0.5, 20, 32, gate=gate.cuda())
+    assert gka.device_status() == 0
+    for name, t in got.items():
+        assert torch.count_nonzero(t) == 0, name
+
+
+def test_backward_bf16_gradient_in_last_chunk_only():
+    # dL/do only on the last 32 tokens: the adjoints of every earlier chunk are what reaches
+    # them from the last one, their own increments zero
+    q, k, v, beta = make_inputs(1, 2, 256, 128, torch.bfloat16, 3.0, 1.0, seed=824)
+    dout = _dout(q.shape, q.dtype, 9100)
+    dout[:, :, :-32] = 0
+    check_backward(q, k, v, beta, 0.5, 20, 32, dout=dout)
 
 
 @pytest.mark.parametrize("D,C", [(64, 32), (128, 16), (32, 16)])
