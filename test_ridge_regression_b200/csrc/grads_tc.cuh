@@ -97,6 +97,20 @@ k_bwd_grads_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restr
         tc::tmem_alloc(tbase, 256);
         tc::tmem_relinquish();
     }
+    // per-token scalars (threads tid < 32) and the chunk's two scalars, loaded first so that
+    // their latency runs under the row loads and the log prefix
+    float p_beta = 1.f, p_w = 1.f, p_c = 0.f, p_tq[4] = {0.f, 0.f, 0.f, 0.f};
+    if (tid < C) {
+        const size_t tt = tok0 + tid;
+        p_beta = beta[tt];
+        p_w = gate ? gate[tt] : 1.f;
+        p_c = cvec[tt];
+        p_tq[0] = tokq[tt];
+        p_tq[1] = tokq[plane + tt];
+        p_tq[2] = tokq[2 * plane + tt];
+        p_tq[3] = tokq[3 * plane + tt] + tokq[4 * plane + tt];   // qe: the H and M parts
+    }
+    const float hs2 = chq[((size_t)bh * N + n) * 2], eh = chq[((size_t)bh * N + n) * 2 + 1];
     // this thread's items: token t = tid / 16 + 16 r, columns 8j .. 8j + 7
     const int j = tid & 15;
     uint4 ku[2], vu[2], gu[2];
@@ -112,19 +126,20 @@ k_bwd_grads_tc(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restr
         ya[r] = *reinterpret_cast<const float4 *>(ys + g);
         yb[r] = *reinterpret_cast<const float4 *>(ys + g + 4);
     }
-    chunk_log_prefix_f32log(beta + tok0, C, ell, wtot);
-    const float hs2 = chq[((size_t)bh * N + n) * 2], eh = chq[((size_t)bh * N + n) * 2 + 1];
+    // the log prefix reads beta from shared memory (thread t wrote entry t itself)
+    if (tid < C) s_b[tid] = p_beta;
+    chunk_log_prefix_f32log(s_b, C, ell, wtot);
     if (tid < C) {
         const ChunkDecays dc = chunk_decays(ell, C, tid);
         s_b[tid] = dc.b;
         s_step[tid] = dc.step;
         s_wend[tid] = dc.wend;
-        s_w[tid] = gate ? gate[tok0 + tid] : 1.f;
-        s_c[tid] = cvec[tok0 + tid];
-        s_uk[tid] = tokq[tok0 + tid];
-        s_yhx[tid] = tokq[plane + tok0 + tid];
-        s_gmx[tid] = tokq[2 * plane + tok0 + tid];
-        s_qe[tid] = tokq[3 * plane + tok0 + tid] + tokq[4 * plane + tok0 + tid];   // H, M parts
+        s_w[tid] = p_w;
+        s_c[tid] = p_c;
+        s_uk[tid] = p_tq[0];
+        s_yhx[tid] = p_tq[1];
+        s_gmx[tid] = p_tq[2];
+        s_qe[tid] = p_tq[3];
         s_bm1[tid] = tid == 0 ? 1.f : decay_exp(ell[tid - 1]);
     }
     // W[l][s] = w_sl for s >= l, else 0
