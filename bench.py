@@ -46,9 +46,9 @@ TRAFFIC = {
                       "sha1": "557968b9a4b4f6da6d895bc493988a8c16af285f"},
     # backward kernels captured at B2 H8 T2048 (1024 chunks, 16 heads), scaled x4 to the
     # full workload (the row kernel's traffic is per chunk, the adjoint pass's per head)
-    "bwd_rows_tc": {"bytes": 4 * (217.924608e6 + 43.453184e6), "workload": "bf16_b8h8t2048d128",
+    "bwd_rows_tc": {"bytes": 4 * (217.798144e6 + 43.793664e6), "workload": "bf16_b8h8t2048d128",
                     "src": "test_ridge_regression_b200/csrc/backward_tc.cuh",
-                    "sha1": "3766bfe51b74e452ca5370b9372efe91b296beec"},
+                    "sha1": "ac9c66bdb4db03eca297e2dd0a96931353d9febb"},
     "adjoint_pass_tc": {"bytes": 4 * (117.882624e6 + 38.258432e6), "workload": "bf16_b8h8t2048d128",
                         "src": "test_ridge_regression_b200/csrc/adjoint_tc.cuh",
                         "sha1": "bcd3ef1e1b540648f212e8dd8eb7ac785171869a"},

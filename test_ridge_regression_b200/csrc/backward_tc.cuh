@@ -479,25 +479,30 @@ k_bwd_u_tc(const __grid_constant__ CUtensorMap state_map, const int *__restrict_
     if (tid == 0) {
         for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
-        mbar_arrive_expect_tx(&bars[0], 32768 + 3 * 8192 + 128 + (gate ? 128 : 0));
+        mbar_arrive_expect_tx(&bars[0], 32768 + 3 * 8192);
         load_state_tile(&state_map, srow + D, sm + L::MB, &bars[0]);
         bulk_g2s(sm + L::RK, k + tok0 * D, 8192, &bars[0]);
         bulk_g2s(sm + L::RV, v + tok0 * D, 8192, &bars[0]);
         bulk_g2s(sm + L::RG, dout + tok0 * D, 8192, &bars[0]);
-        bulk_g2s(s_beta, beta + tok0, 128, &bars[0]);
-        if (gate) bulk_g2s(s_gate, gate + tok0, 128, &bars[0]);
+    }
+    // beta and the gate by the first 32 threads, so that the decays are formed while the
+    // tiles land
+    float p_gate = 1.f;
+    if (tid < C) {
+        s_beta[tid] = beta[tok0 + tid];
+        if (gate) p_gate = gate[tok0 + tid];
     }
     if (warp == 0) {
         tc::tmem_alloc(tbase, 128);
         tc::tmem_relinquish();
     }
     __syncthreads();
-    bool ok = mbar_wait_bounded(&bars[0], 0, kTcWaitProbes);
     chunk_log_prefix_f32log(s_beta, C, ell, wtot);
     if (tid < C) {
         s_b[tid] = decay_exp(ell[tid]);
-        s_sg[tid] = gate ? sqrtf(s_gate[tid]) : 1.f;
+        s_sg[tid] = gate ? sqrtf(p_gate) : 1.f;
     }
+    bool ok = mbar_wait_bounded(&bars[0], 0, kTcWaitProbes);
     __syncthreads();
     // the operand rows: item (token t, 8 columns 8j..) of each of G, V~, K~
     float gv[2][8], vv[2][8], kv[2][8];
