@@ -38,9 +38,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # bench reports null.  The captures' commands sit beside their summaries.
 TRAFFIC = {
     # full-size forward workload (B8 H8 T2048 D128, chunk 64), one launch
-    "chunk_solve_tc": {"bytes": 237.094912e6 + 23.748096e6, "workload": "bf16_b8h8t2048d128",
+    "chunk_solve_tc": {"bytes": 237.094400e6 + 23.277824e6, "workload": "bf16_b8h8t2048d128",
                        "src": "test_ridge_regression_b200/csrc/solve_tc.cuh",
-                       "sha1": "1da5f1a4b43087afd2a12ecc7601e5093ecbd7b9"},
+                       "sha1": "bf2266c98c0e6146d6f61891d28cc9b931a90aef"},
     "state_pass_tc": {"bytes": 67.716864e6 + 79.924480e6, "workload": "bf16_b8h8t2048d128",
                       "src": "test_ridge_regression_b200/csrc/state_tc.cuh",
                       "sha1": "557968b9a4b4f6da6d895bc493988a8c16af285f"},

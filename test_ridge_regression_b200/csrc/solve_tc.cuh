@@ -337,11 +337,14 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
                 tc::tma_load_2d(sm + L::KT + h * MG * 128 + rb * 8192, &maps.k, h * 64,
                                 (int)tok0 + rb * 64, bar_load);
         bulk_g2s(sm + L::QS, q + tok0 * kTcD, TOK * kTcD * 2, bar_load);
-        mbar_arrive_expect_tx(bar_v, MG * 256);
-        for (int h = 0; h < 2; ++h)
-            for (int rb = 0; rb < MG / 64; ++rb)
-                tc::tma_load_2d(sm + L::VT + h * MG * 128 + rb * 8192, &maps.v, h * 64,
-                                (int)tok0 + rb * 64, bar_v);
+        if constexpr (!XOUT) {
+            // the values, read by the readout only
+            mbar_arrive_expect_tx(bar_v, MG * 256);
+            for (int h = 0; h < 2; ++h)
+                for (int rb = 0; rb < MG / 64; ++rb)
+                    tc::tma_load_2d(sm + L::VT + h * MG * 128 + rb * 8192, &maps.v, h * 64,
+                                    (int)tok0 + rb * 64, bar_v);
+        }
     }
     if (warp == 0) {
         tc::tmem_alloc(tbase, TMEM_COLS);
@@ -415,10 +418,13 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
         }
         tc::commit(bar_n);
     }
-    // values: bf16 -> fp16 in place, scaled below 1 (first read by the readout)
-    ok = mbar_wait_sleep(bar_v, 0, kTcSleepProbes, kTcSleepNs) && ok;
-    const float sV = tile_bf16_to_f16_rows_scaled<MG * 256, kSolveThreads, MG>(sm + L::VT, red,
-                                                                               gate_rows);
+    // values: bf16 -> fp16 in place, scaled below 1 (first read by the readout; with
+    // XOUT there is no readout, and the value tile is neither loaded nor converted)
+    float sV = 1.f;
+    if constexpr (!XOUT) {
+        ok = mbar_wait_sleep(bar_v, 0, kTcSleepProbes, kTcSleepNs) && ok;
+        sV = tile_bf16_to_f16_rows_scaled<MG * 256, kSolveThreads, MG>(sm + L::VT, red, gate_rows);
+    }
     float *s_u = reinterpret_cast<float *>(sm + L::NRM);
     float *s_E = s_u + MG, *s_X = s_E + MG, *s_G = s_X + MG;   // [MG] each; E and X: wg 0 part
     float *s_E1 = reinterpret_cast<float *>(sm + L::NRM2), *s_X1 = s_E1 + MG;   // wg 1 part
@@ -935,7 +941,7 @@ k_chunk_solve_tc(const __grid_constant__ TcMaps maps, const __nv_bfloat16 *__res
             tc::commit(bar_fin);
             mbar_wait_bounded(bar_fin, 0, kTcWaitProbes);
             mbar_wait_bounded(bar_load, 0, kTcWaitProbes);
-            mbar_wait_bounded(bar_v, 0, kTcWaitProbes);
+            if (!XOUT) mbar_wait_bounded(bar_v, 0, kTcWaitProbes);
             if (m_requested) mbar_wait_bounded(bar_m, 0, kTcWaitProbes);
         }
     }
